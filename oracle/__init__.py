@@ -1,0 +1,166 @@
+"""CPU oracle for the forward convolutions (TEST INFRASTRUCTURE).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import this package. The library's CUDA path never imports it, and the two share no code;
+both only consume the seeded inputs of the ``workloads`` module.
+
+The arithmetic lives in ``conv_oracle.c`` (plain C, OpenMP over independent outputs):
+
+* ``conv2d_nhwc`` -- the seven-loop definition of the dense NHWC convolution of the CMU
+  DLSys Lecture 14 notes ("The hidden copy behind convolution as matrix multiplication",
+  section 1), accumulated in float64, with the per-output absolute sum sum|x||f| that the
+  dense tolerance is scaled by.
+* ``depthwise`` -- the per-output loop of the OneModel "Depthwise convolution" page
+  (section "What each output is"), in IEEE float32 in the page's order, exact or fast mode.
+
+Parity status: every function here is pinned by tests that do not call it to compute
+their expectation (worked examples printed on the pages, library routines for special
+cases, closed forms and invariants); see tests/test_oracle.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "conv_oracle.c")
+_LIB = os.path.join(_HERE, "_liboracle.so")
+
+DW_EXACT = 0
+DW_FAST = 1
+
+CFLAGS = ["-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+          "-fno-unsafe-math-optimizations", "-frounding-math", "-fsignaling-nans"]
+
+
+def build(force: bool = False) -> str:
+    """Compile conv_oracle.c into _liboracle.so with gcc (no CUDA)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        L = ctypes.c_int64
+        lib.oracle_conv2d_nhwc.argtypes = [P, P, P, P] + [I] * 6
+        lib.oracle_conv2d_nhwc.restype = None
+        lib.oracle_conv2d_nhwc_points.argtypes = [P, P, P, L, P, P] + [I] * 6
+        lib.oracle_conv2d_nhwc_points.restype = None
+        lib.oracle_depthwise.argtypes = [P, P, P, P] + [I] * 11
+        lib.oracle_depthwise.restype = I
+        lib.oracle_depthwise_points.argtypes = [P, P, P, P, L, P] + [I] * 11
+        lib.oracle_depthwise_points.restype = I
+        lib.oracle_depthwise_absbound.argtypes = [P, P, P, P] + [I] * 10
+        lib.oracle_depthwise_absbound.restype = I
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = I
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def conv2d_nhwc(X, F):
+    """Dense NHWC forward convolution in float64.
+
+    X: [N, H, W, Cin], F: [K, K, Cin, Cout] (float32 values; bfloat16 data is widened by the
+    caller). Returns (Y, abssum), both float64 [N, Ho, Wo, Cout].
+    """
+    X, F = _f32(X), _f32(F)
+    N, H, W, Cin = X.shape
+    K, K2, Cin2, Cout = F.shape
+    if K != K2 or Cin != Cin2 or K > min(H, W) or min(N, H, W, Cin, K, Cout) <= 0:
+        raise ValueError("incompatible input and square filter")
+    Ho, Wo = H - K + 1, W - K + 1
+    Y = np.empty((N, Ho, Wo, Cout), dtype=np.float64)
+    A = np.empty_like(Y)
+    _load().oracle_conv2d_nhwc(_ptr(X), _ptr(F), _ptr(Y), _ptr(A), N, H, W, Cin, Cout, K)
+    return Y, A
+
+
+def conv2d_nhwc_points(X, F, flat_idx):
+    """Selected outputs of conv2d_nhwc, by flat index into [N, Ho, Wo, Cout]."""
+    X, F = _f32(X), _f32(F)
+    N, H, W, Cin = X.shape
+    K, _, _, Cout = F.shape
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    y = np.empty(idx.size, dtype=np.float64)
+    a = np.empty(idx.size, dtype=np.float64)
+    _load().oracle_conv2d_nhwc_points(_ptr(X), _ptr(F), _ptr(idx), idx.size, _ptr(y), _ptr(a),
+                                      N, H, W, Cin, Cout, K)
+    return y, a
+
+
+def _dw_shape(x, w, mult, stride, pad, dil):
+    N, Cin, H, W = x.shape
+    Cout, KH, KW = w.shape
+    if Cout != Cin * mult:
+        raise ValueError("w must have Cin*mult planes")
+    Ho = (H + 2 * pad - (dil * (KH - 1) + 1)) // stride + 1
+    Wo = (W + 2 * pad - (dil * (KW - 1) + 1)) // stride + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    return N, Cin, H, W, Cout, KH, KW, Ho, Wo
+
+
+def depthwise(x, w, bias, mult=1, stride=1, pad=0, dil=1, mode=DW_EXACT):
+    """Depthwise forward convolution in float32, the page's order.
+
+    x: [N, Cin, H, W]; w: [Cin*mult, KH, KW]; bias: [Cin*mult] or None.
+    Returns y: float32 [N, Cin*mult, Ho, Wo].
+    """
+    x, w = _f32(x), _f32(w)
+    b = None if bias is None else _f32(bias)
+    N, Cin, H, W, Cout, KH, KW, Ho, Wo = _dw_shape(x, w, mult, stride, pad, dil)
+    y = np.empty((N, Cout, Ho, Wo), dtype=np.float32)
+    rc = _load().oracle_depthwise(_ptr(x), _ptr(w), _ptr(b), _ptr(y), N, Cin, mult, H, W, KH, KW,
+                                  stride, pad, dil, mode)
+    if rc != 0:
+        raise ValueError("empty output")
+    return y
+
+
+def depthwise_points(x, w, bias, flat_idx, mult=1, stride=1, pad=0, dil=1, mode=DW_EXACT):
+    """Selected outputs of depthwise, by flat index into [N, Cin*mult, Ho, Wo]."""
+    x, w = _f32(x), _f32(w)
+    b = None if bias is None else _f32(bias)
+    N, Cin, H, W, Cout, KH, KW, Ho, Wo = _dw_shape(x, w, mult, stride, pad, dil)
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    out = np.empty(idx.size, dtype=np.float32)
+    _load().oracle_depthwise_points(_ptr(x), _ptr(w), _ptr(b), _ptr(idx), idx.size, _ptr(out),
+                                    N, Cin, mult, H, W, KH, KW, stride, pad, dil, mode)
+    return out
+
+
+def depthwise_absbound(x, w, bias, mult=1, stride=1, pad=0, dil=1):
+    """sum over taps of |w*x| plus |bias| per output, float64 [N, Cin*mult, Ho, Wo]."""
+    x, w = _f32(x), _f32(w)
+    b = None if bias is None else _f32(bias)
+    N, Cin, H, W, Cout, KH, KW, Ho, Wo = _dw_shape(x, w, mult, stride, pad, dil)
+    out = np.empty((N, Cout, Ho, Wo), dtype=np.float64)
+    _load().oracle_depthwise_absbound(_ptr(x), _ptr(w), _ptr(b), _ptr(out), N, Cin, mult, H, W, KH,
+                                      KW, stride, pad, dil)
+    return out

@@ -1,0 +1,234 @@
+/*
+ * Oracle for the forward convolutions: plain, slow and written to be read against the
+ * pages it follows. This is TEST INFRASTRUCTURE. Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load it; the library's CUDA path never calls it and
+ * shares no code with it.
+ *
+ * Dense NHWC convolution -- CMU DLSys Lecture 14 notes, "The hidden copy behind convolution
+ * as matrix multiplication", section 1 "Fix the index contract before optimizing it":
+ *   X is N x H x W x Cin, F is K x K x Cin x Cout (KKIO), Ho = H-K+1, Wo = W-K+1, and
+ *   Y[n,y,x,o] = sum_{i<K} sum_{j<K} sum_{c<Cin} X[n,y+i,x+j,c] * F[i,j,c,o]
+ *   with the filter not reversed (cross-correlation). The same section calls the direct
+ *   seven-loop form the small correctness oracle; that is what oracle_conv2d_nhwc is.
+ *   Arithmetic is float64. For bfloat16 or small-integer float32 operands every product
+ *   is exact in float64, so the result is the exact sum up to float64 summation error.
+ *
+ * Depthwise convolution -- OneModel docs, "Depthwise convolution", section "What each
+ * output is": output channel oc reads input channel oc / mult; acc starts at +0; taps go
+ * ky outer, kx inner; padding is a real zero that is multiplied; exact mode rounds the
+ * product and then the sum (no fused operation) and rewrites a NaN result as 0x7FC00000;
+ * fast mode uses one fused multiply-add per tap; a bias is a separate pass of one rounded
+ * addition per output. Output size per axis follows "Convolution Is Wx+b Moving Across a
+ * Signal", section "Build an image-gradient map, one number at a time":
+ *   out = floor((in + 2*pad - (dil*(k-1)+1)) / stride) + 1.
+ * Padding is read as symmetric (pad zeros before and after each axis). The file must be
+ * built with -ffp-contract=off and without fast-math so that every float operation below
+ * is one IEEE binary32 operation, rounded to nearest even, with denormals kept.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define DW_EXACT 0
+#define DW_FAST 1
+
+/* ---------------------------------------------------------------------------------- */
+/* Dense                                                                               */
+/* ---------------------------------------------------------------------------------- */
+
+/* One output Y[n,y,x,o] and its absolute sum sum|X||F| over the same terms. */
+static void dense_one(const float *X, const float *F, int H, int W, int Cin, int Cout, int K,
+                      long n, long y, long x, long o, double *out, double *abs_out)
+{
+    double s = 0.0, a = 0.0;
+    for (int i = 0; i < K; ++i)
+        for (int j = 0; j < K; ++j)
+            for (int c = 0; c < Cin; ++c) {
+                double xv = X[((n * H + (y + i)) * W + (x + j)) * Cin + c];
+                double fv = F[(((long)i * K + j) * Cin + c) * Cout + o];
+                s += xv * fv;
+                a += fabs(xv) * fabs(fv);
+            }
+    *out = s;
+    *abs_out = a;
+}
+
+/* Full output. Loops n, y, x | i, j, c | o: the output channel o is the innermost loop so
+ * that the F row is read contiguously; every output is still summed in (i, j, c) order,
+ * exactly as dense_one does. abssum may be NULL. */
+void oracle_conv2d_nhwc(const float *X, const float *F, double *Y, double *abssum,
+                        int N, int H, int W, int Cin, int Cout, int K)
+{
+    const int Ho = H - K + 1, Wo = W - K + 1;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int n = 0; n < N; ++n)
+        for (int y = 0; y < Ho; ++y) {
+            double acc[Cout], aacc[Cout];
+            for (int x = 0; x < Wo; ++x) {
+                for (int o = 0; o < Cout; ++o) { acc[o] = 0.0; aacc[o] = 0.0; }
+                for (int i = 0; i < K; ++i)
+                    for (int j = 0; j < K; ++j)
+                        for (int c = 0; c < Cin; ++c) {
+                            double xv = X[(((long)n * H + (y + i)) * W + (x + j)) * Cin + c];
+                            const float *frow = F + (((long)i * K + j) * Cin + c) * Cout;
+                            for (int o = 0; o < Cout; ++o) {
+                                acc[o] += xv * (double)frow[o];
+                                aacc[o] += fabs(xv) * fabs((double)frow[o]);
+                            }
+                        }
+                long base = (((long)n * Ho + y) * Wo + x) * Cout;
+                for (int o = 0; o < Cout; ++o) {
+                    Y[base + o] = acc[o];
+                    if (abssum) abssum[base + o] = aacc[o];
+                }
+            }
+        }
+}
+
+/* Selected outputs, given as flat indices into Y[N][Ho][Wo][Cout]. */
+void oracle_conv2d_nhwc_points(const float *X, const float *F, const int64_t *idx, int64_t npts,
+                               double *y, double *abssum,
+                               int N, int H, int W, int Cin, int Cout, int K)
+{
+    const long Ho = H - K + 1, Wo = W - K + 1;
+    (void)N;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t p = 0; p < npts; ++p) {
+        long t = idx[p];
+        long o = t % Cout; t /= Cout;
+        long x = t % Wo; t /= Wo;
+        long yy = t % Ho; t /= Ho;
+        long n = t;
+        dense_one(X, F, H, W, Cin, Cout, K, n, yy, x, o, &y[p], &abssum[p]);
+    }
+}
+
+/* ---------------------------------------------------------------------------------- */
+/* Depthwise                                                                           */
+/* ---------------------------------------------------------------------------------- */
+
+static float canonical_nan(void)
+{
+    uint32_t bits = 0x7FC00000u;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return f;
+}
+
+static long dw_out_size(long in, int k, int stride, int pad, int dil)
+{
+    long eff = (long)dil * (k - 1) + 1;
+    return (in + 2L * pad - eff) / stride + 1;
+}
+
+/* One output plane position, in the page's order. */
+static float dw_one(const float *x, const float *w, const float *bias,
+                    int Cin, int mult, int H, int W, int KH, int KW,
+                    int stride, int pad, int dil, int mode,
+                    long n, long oc, long oy, long ox)
+{
+    const long ic = oc / mult;
+    const float *plane = x + ((n * Cin) + ic) * (long)H * W;
+    const float *wp = w + oc * (long)KH * KW;
+    float acc = +0.0f;
+    for (int ky = 0; ky < KH; ++ky)
+        for (int kx = 0; kx < KW; ++kx) {
+            long r = oy * stride + (long)ky * dil - pad;
+            long q = ox * stride + (long)kx * dil - pad;
+            float xv = (r >= 0 && r < H && q >= 0 && q < W) ? plane[r * W + q] : 0.0f;
+            float wv = wp[ky * KW + kx];
+            if (mode == DW_EXACT) {
+                float p = wv * xv;   /* rounded product */
+                acc = acc + p;       /* rounded sum */
+            } else {
+                acc = fmaf(wv, xv, acc);
+            }
+        }
+    if (mode == DW_EXACT && isnan(acc)) acc = canonical_nan();
+    if (bias) {
+        acc = acc + bias[oc];
+        if (mode == DW_EXACT && isnan(acc)) acc = canonical_nan();
+    }
+    return acc;
+}
+
+/* Full output y[N][Cin*mult][Ho][Wo]. Returns 0, or -1 when the output would be empty. */
+int oracle_depthwise(const float *x, const float *w, const float *bias, float *y,
+                     int N, int Cin, int mult, int H, int W, int KH, int KW,
+                     int stride, int pad, int dil, int mode)
+{
+    const long Ho = dw_out_size(H, KH, stride, pad, dil);
+    const long Wo = dw_out_size(W, KW, stride, pad, dil);
+    const long Cout = (long)Cin * mult;
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (long n = 0; n < N; ++n)
+        for (long oc = 0; oc < Cout; ++oc)
+            for (long oy = 0; oy < Ho; ++oy)
+                for (long ox = 0; ox < Wo; ++ox)
+                    y[((n * Cout + oc) * Ho + oy) * Wo + ox] =
+                        dw_one(x, w, bias, Cin, mult, H, W, KH, KW, stride, pad, dil, mode,
+                               n, oc, oy, ox);
+    return 0;
+}
+
+/* Selected outputs, given as flat indices into y[N][Cin*mult][Ho][Wo]. */
+int oracle_depthwise_points(const float *x, const float *w, const float *bias,
+                            const int64_t *idx, int64_t npts, float *out,
+                            int N, int Cin, int mult, int H, int W, int KH, int KW,
+                            int stride, int pad, int dil, int mode)
+{
+    const long Ho = dw_out_size(H, KH, stride, pad, dil);
+    const long Wo = dw_out_size(W, KW, stride, pad, dil);
+    const long Cout = (long)Cin * mult;
+    (void)N;
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for schedule(dynamic, 256)
+    for (int64_t p = 0; p < npts; ++p) {
+        long t = idx[p];
+        long ox = t % Wo; t /= Wo;
+        long oy = t % Ho; t /= Ho;
+        long oc = t % Cout; t /= Cout;
+        out[p] = dw_one(x, w, bias, Cin, mult, H, W, KH, KW, stride, pad, dil, mode, t, oc, oy, ox);
+    }
+    return 0;
+}
+
+/* Magnitude scale of each output for tolerance checks: sum over taps of |w * x| plus |bias|,
+ * in float64, same indexing as dw_one. */
+int oracle_depthwise_absbound(const float *x, const float *w, const float *bias, double *out,
+                              int N, int Cin, int mult, int H, int W, int KH, int KW,
+                              int stride, int pad, int dil)
+{
+    const long Ho = dw_out_size(H, KH, stride, pad, dil);
+    const long Wo = dw_out_size(W, KW, stride, pad, dil);
+    const long Cout = (long)Cin * mult;
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (long n = 0; n < N; ++n)
+        for (long oc = 0; oc < Cout; ++oc) {
+            const float *plane = x + ((n * Cin) + oc / mult) * (long)H * W;
+            const float *wp = w + oc * (long)KH * KW;
+            for (long oy = 0; oy < Ho; ++oy)
+                for (long ox = 0; ox < Wo; ++ox) {
+                    double s = bias ? fabs((double)bias[oc]) : 0.0;
+                    for (int ky = 0; ky < KH; ++ky)
+                        for (int kx = 0; kx < KW; ++kx) {
+                            long r = oy * stride + (long)ky * dil - pad;
+                            long q = ox * stride + (long)kx * dil - pad;
+                            double xv = (r >= 0 && r < H && q >= 0 && q < W) ? plane[r * W + q] : 0.0;
+                            s += fabs((double)wp[ky * KW + kx] * xv);
+                        }
+                    out[((n * Cout + oc) * Ho + oy) * Wo + ox] = s;
+                }
+        }
+    return 0;
+}
+
+/* Threads the OpenMP runtime will use (for reporting the CPU baseline's core count). */
+#ifdef _OPENMP
+#include <omp.h>
+int oracle_num_threads(void) { return omp_get_max_threads(); }
+#else
+int oracle_num_threads(void) { return 1; }
+#endif

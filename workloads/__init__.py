@@ -1,0 +1,228 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests and benchmark and by the oracle.
+
+This module holds no convolution arithmetic. It only draws numbers and stores them in
+the layouts the two sides consume, so that both read identical bits:
+
+* SplitMix64 (Steele, Lea, Flood, "Fast splittable pseudorandom number generators",
+  OOPSLA 2014) as a counter-based stream: value i of a stream with seed s is
+  mix(s + (i + 1) * GAMMA).
+* Uniform doubles in [0, 1) from the top 53 bits of each 64-bit value.
+* Normals by the Box-Muller transform (Box and Muller, 1958), one pair per two uniforms.
+* Round-to-nearest-even narrowing of float32 to bfloat16 bit patterns.
+
+The workload table below describes the shapes and value distributions of the
+configurations the library is tested and measured on. The dense shapes follow the
+NHWC / KKIO contract of the CMU DLSys Lecture 14 notes ("The hidden copy behind
+convolution as matrix multiplication", section 1); the depthwise sweep is the set of
+MobileNetV3-large depthwise layers measured in the OneModel "Depthwise convolution"
+page (section "Measured"), with batch 64 standing in for the unspecified batch.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+_CHUNK = 1 << 22
+
+
+def _mix(z: np.ndarray) -> np.ndarray:
+    z = (z ^ (z >> np.uint64(30))) * _M1
+    z = (z ^ (z >> np.uint64(27))) * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def splitmix64(seed: int, n: int, offset: int = 0) -> np.ndarray:
+    """Values offset .. offset+n-1 of the SplitMix64 stream with the given seed (uint64)."""
+    with np.errstate(over="ignore"):
+        i = np.arange(offset + 1, offset + n + 1, dtype=np.uint64)
+        return _mix(np.uint64(seed & 0xFFFFFFFFFFFFFFFF) + i * GAMMA)
+
+
+def stream_seed(seed: int, tensor_id: int) -> int:
+    """Seed of the independent stream used for one tensor of one workload."""
+    with np.errstate(over="ignore"):
+        z = _mix(np.array([(seed * 0x100000001B3 + tensor_id + 1) & 0xFFFFFFFFFFFFFFFF],
+                          dtype=np.uint64))
+    return int(z[0])
+
+
+def uniform01(seed: int, n: int) -> np.ndarray:
+    """n doubles in [0, 1): (value >> 11) * 2**-53."""
+    out = np.empty(n, dtype=np.float64)
+    for s in range(0, n, _CHUNK):
+        m = min(_CHUNK, n - s)
+        out[s:s + m] = (splitmix64(seed, m, s) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+    return out
+
+
+def uniform(seed: int, n: int, lo: float, hi: float) -> np.ndarray:
+    """float32 samples of U(lo, hi)."""
+    u = uniform01(seed, n)
+    return (lo + (hi - lo) * u).astype(np.float32)
+
+
+def normal(seed: int, n: int, std: float) -> np.ndarray:
+    """float32 samples of N(0, std**2) by Box-Muller on consecutive uniform pairs."""
+    out = np.empty(n, dtype=np.float32)
+    pairs = (n + 1) // 2
+    for s in range(0, pairs, _CHUNK):
+        m = min(_CHUNK, pairs - s)
+        u = (splitmix64(seed, 2 * m, 2 * s) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+        u1, u2 = u[0::2], u[1::2]
+        r = np.sqrt(-2.0 * np.log1p(-u1))
+        t = 2.0 * math.pi * u2
+        z = np.empty(2 * m, dtype=np.float64)
+        z[0::2] = r * np.cos(t)
+        z[1::2] = r * np.sin(t)
+        lo = 2 * s
+        hi = min(n, lo + 2 * m)
+        out[lo:hi] = (std * z[: hi - lo]).astype(np.float32)
+    return out
+
+
+def int_uniform(seed: int, n: int, lo: int, hi: int) -> np.ndarray:
+    """float32 holding integers drawn uniformly from lo..hi inclusive."""
+    u = uniform01(seed, n)
+    k = np.floor(u * (hi - lo + 1)).astype(np.int64) + lo
+    return k.astype(np.float32)
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16, nearest-even; returns the uint16 bit patterns (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_to_f32(b: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bit patterns to float32 (exact)."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# ----------------------------------------------------------------------------------------
+# Workload table
+# ----------------------------------------------------------------------------------------
+
+
+@dataclasses.dataclass(frozen=True)
+class DenseCase:
+    """Dense NHWC forward convolution: X[N,H,W,Cin], F[K,K,Cin,Cout] (KKIO), Y[N,Ho,Wo,Cout]."""
+    name: str
+    N: int
+    H: int
+    W: int
+    Cin: int
+    Cout: int
+    K: int
+    dtype: str          # "bf16" or "f32": storage type of X, F and Y
+    dist: str           # "normal" (X~N(0,1), F~N(0,1/(K*K*Cin))) or "int3" (integers in [-3,3])
+    seed: int = 0
+
+    @property
+    def Ho(self) -> int:
+        return self.H - self.K + 1
+
+    @property
+    def Wo(self) -> int:
+        return self.W - self.K + 1
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.N * self.Ho * self.Wo * self.Cout * self.K * self.K * self.Cin
+
+    @property
+    def bytes(self) -> int:
+        e = 2 if self.dtype == "bf16" else 4
+        return e * (self.N * self.H * self.W * self.Cin + self.K * self.K * self.Cin * self.Cout
+                    + self.N * self.Ho * self.Wo * self.Cout)
+
+
+@dataclasses.dataclass(frozen=True)
+class DepthwiseCase:
+    """Depthwise forward convolution on NCHW float32 planes, Cout = Cin * mult."""
+    name: str
+    N: int
+    C: int
+    mult: int
+    H: int
+    W: int
+    KH: int
+    KW: int
+    stride: int
+    pad: int
+    dil: int
+    bias: bool = True
+    seed: int = 0
+
+    @property
+    def Ho(self) -> int:
+        return (self.H + 2 * self.pad - (self.dil * (self.KH - 1) + 1)) // self.stride + 1
+
+    @property
+    def Wo(self) -> int:
+        return (self.W + 2 * self.pad - (self.dil * (self.KW - 1) + 1)) // self.stride + 1
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.KH * self.KW * self.N * self.C * self.mult * self.Ho * self.Wo
+
+    @property
+    def bytes(self) -> int:
+        co = self.C * self.mult
+        return 4 * (self.N * self.C * self.H * self.W + co * self.KH * self.KW
+                    + (co if self.bias else 0) + self.N * co * self.Ho * self.Wo)
+
+
+DENSE_TINY = DenseCase("tiny dense fp32 N2 H8 W8 Cin4 Cout8 K3", 2, 8, 8, 4, 8, 3, "f32", "int3", 0)
+DENSE_3X3 = DenseCase("dense bf16 N32 H56 W56 Cin64 Cout64 K3", 32, 56, 56, 64, 64, 3, "bf16", "normal", 0)
+DENSE_1X1 = DenseCase("pointwise bf16 N32 H28 W28 Cin256 Cout512 K1", 32, 28, 28, 256, 512, 1, "bf16",
+                      "normal", 0)
+DENSE_LARGE = DenseCase("large dense bf16 N64 H112 W112 Cin128 Cout128 K5", 64, 112, 112, 128, 128, 5,
+                        "bf16", "normal", 0)
+
+# MobileNetV3-large depthwise layers (C, K, stride, input H=W), batch 64, multiplier 1,
+# pad (K-1)/2, dilation 1.
+DW_LAYERS = [(16, 3, 1, 112), (64, 3, 2, 112), (72, 5, 2, 56), (120, 5, 1, 28), (672, 3, 1, 14),
+             (960, 5, 1, 7)]
+DW_SWEEP = [DepthwiseCase(f"depthwise C{c} K{k} s{s} H{h}", 64, c, 1, h, h, k, k, s, (k - 1) // 2, 1,
+                          True, 0) for (c, k, s, h) in DW_LAYERS]
+
+
+def dense_inputs(case: DenseCase):
+    """Seeded X (NHWC) and F (KKIO).
+
+    Returns (X, F) as uint16 bf16 bit patterns for bf16 cases, float32 arrays otherwise.
+    """
+    nx = case.N * case.H * case.W * case.Cin
+    nf = case.K * case.K * case.Cin * case.Cout
+    sx, sf = stream_seed(case.seed, 0), stream_seed(case.seed, 1)
+    if case.dist == "int3":
+        X = int_uniform(sx, nx, -3, 3)
+        F = int_uniform(sf, nf, -3, 3)
+    elif case.dist == "normal":
+        X = normal(sx, nx, 1.0)
+        F = normal(sf, nf, 1.0 / math.sqrt(case.K * case.K * case.Cin))
+    else:
+        raise ValueError(case.dist)
+    X = X.reshape(case.N, case.H, case.W, case.Cin)
+    F = F.reshape(case.K, case.K, case.Cin, case.Cout)
+    if case.dtype == "bf16":
+        return bf16_bits(X), bf16_bits(F)
+    return X, F
+
+
+def depthwise_inputs(case: DepthwiseCase):
+    """Seeded x (NCHW), w ([C*mult][KH][KW]) and bias ([C*mult] or None), float32.
+
+    x ~ U(-1, 1), w ~ N(0, 1/(KH*KW)), bias ~ N(0, 0.1) with 0.1 read as the variance.
+    """
+    co = case.C * case.mult
+    x = uniform(stream_seed(case.seed, 0), case.N * case.C * case.H * case.W, -1.0, 1.0)
+    w = normal(stream_seed(case.seed, 1), co * case.KH * case.KW, 1.0 / math.sqrt(case.KH * case.KW))
+    b = normal(stream_seed(case.seed, 2), co, math.sqrt(0.1)) if case.bias else None
+    return (x.reshape(case.N, case.C, case.H, case.W), w.reshape(co, case.KH, case.KW), b)
