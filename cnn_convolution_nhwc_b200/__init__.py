@@ -1,0 +1,148 @@
+"""Forward 2-D convolution on B200 (sm_100a): thin Python binding of the C ABI.
+
+The functions here only marshal arguments -- shape and dtype checks, output allocation
+through PyTorch, the current CUDA stream -- and call the C entry points of
+libconv_b200.so with the same names (declared in include/conv_b200.h). Every step of the
+computation runs in the library's CUDA kernels; there is no CPU or PyTorch fallback, and
+importing this package fails if the library cannot be loaded.
+
+    conv2d_nhwc_fwd(X, F)        dense NHWC conv, bf16 [N,H,W,Cin] x [K,K,Cin,Cout] -> bf16
+    conv2d_nhwc_fwd_f32(X, F)    the same with float32 tensors
+    depthwise_fwd(x, w, bias)    depthwise conv, float32 NCHW, exact or fast mode
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import build as _build
+
+CONV_OK = 0
+CONV_ERR_INVALID_ARG = -1
+CONV_ERR_UNSUPPORTED = -2
+CONV_ERR_MISALIGNED = -3
+CONV_ERR_CUDA = -4
+CONV_ERR_DEVICE_TIMEOUT = -5
+DW_EXACT = 0
+DW_FAST = 1
+
+LIB_PATH = _build.build()
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+lib.conv2d_nhwc_fwd.argtypes = [_P, _P, _P] + [_I] * 6 + [_P]
+lib.conv2d_nhwc_fwd.restype = _I
+lib.conv2d_nhwc_fwd_f32.argtypes = [_P, _P, _P] + [_I] * 6 + [_P]
+lib.conv2d_nhwc_fwd_f32.restype = _I
+lib.depthwise_fwd.argtypes = [_P, _P, _P, _P] + [_I] * 11 + [_P]
+lib.depthwise_fwd.restype = _I
+lib.conv_status_string.argtypes = [_I]
+lib.conv_status_string.restype = ctypes.c_char_p
+lib.conv_device_status.argtypes = [_P, _I]
+lib.conv_device_status.restype = _I
+
+EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "depthwise_fwd", "conv_status_string",
+           "conv_device_status")
+
+
+class ConvError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {conv_status_string(code)} ({code})")
+        self.code = code
+
+
+def conv_status_string(code: int) -> str:
+    return lib.conv_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str) -> None:
+    if code != CONV_OK:
+        raise ConvError(code, what)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _tensor(t, dtype, ndim, name):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {t.dim()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (the C ABI takes dense row-major tensors); "
+                         "call .contiguous() first")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dense(X, F, Y, stream, dtype, fn, what):
+    import torch
+    px = _tensor(X, dtype, 4, "X")
+    pf = _tensor(F, dtype, 4, "F")
+    N, H, W, Cin = X.shape
+    K, K2, Cin2, Cout = F.shape
+    if K != K2 or Cin2 != Cin:
+        raise ValueError("F must be [K, K, Cin, Cout] matching X")
+    if K > min(H, W):
+        raise ValueError("K must not exceed min(H, W)")
+    if Y is None:
+        Y = torch.empty((N, H - K + 1, W - K + 1, Cout), dtype=dtype, device=X.device)
+    elif tuple(Y.shape) != (N, H - K + 1, W - K + 1, Cout):
+        raise ValueError("Y has the wrong shape")
+    py = _tensor(Y, dtype, 4, "Y")
+    _check(fn(px, pf, py, N, H, W, Cin, Cout, K, _stream(stream)), what)
+    return Y
+
+
+def conv2d_nhwc_fwd(X, F, Y=None, stream=None):
+    """Dense NHWC convolution, bfloat16: X [N,H,W,Cin], F [K,K,Cin,Cout] -> Y [N,Ho,Wo,Cout]."""
+    import torch
+    return _dense(X, F, Y, stream, torch.bfloat16, lib.conv2d_nhwc_fwd, "conv2d_nhwc_fwd")
+
+
+def conv2d_nhwc_fwd_f32(X, F, Y=None, stream=None):
+    """Dense NHWC convolution, float32 tensors."""
+    import torch
+    return _dense(X, F, Y, stream, torch.float32, lib.conv2d_nhwc_fwd_f32, "conv2d_nhwc_fwd_f32")
+
+
+def depthwise_fwd(x, w, bias=None, y=None, stride=1, pad=0, dil=1, mode=DW_EXACT, stream=None):
+    """Depthwise convolution, float32: x [N,Cin,H,W], w [Cin*mult,KH,KW], bias [Cin*mult] or None."""
+    import torch
+    px = _tensor(x, torch.float32, 4, "x")
+    pw = _tensor(w, torch.float32, 3, "w")
+    N, Cin, H, W = x.shape
+    Cout, KH, KW = w.shape
+    if Cout % Cin != 0:
+        raise ValueError("w must have Cin * mult planes")
+    mult = Cout // Cin
+    pb = ctypes.c_void_p(None)
+    if bias is not None:
+        pb = _tensor(bias, torch.float32, 1, "bias")
+        if bias.shape[0] != Cout:
+            raise ValueError("bias must have Cin * mult entries")
+    Ho = (H + 2 * pad - (dil * (KH - 1) + 1)) // stride + 1
+    Wo = (W + 2 * pad - (dil * (KW - 1) + 1)) // stride + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    if y is None:
+        y = torch.empty((N, Cout, Ho, Wo), dtype=torch.float32, device=x.device)
+    elif tuple(y.shape) != (N, Cout, Ho, Wo):
+        raise ValueError("y has the wrong shape")
+    py = _tensor(y, torch.float32, 4, "y")
+    _check(lib.depthwise_fwd(px, pw, pb, py, N, Cin, mult, H, W, KH, KW, stride, pad, dil, int(mode),
+                             _stream(stream)), "depthwise_fwd")
+    return y
+
+
+def conv_device_status(stream=None, reset=False) -> int:
+    """Synchronises the stream and returns the device status word as a conv_status code."""
+    return lib.conv_device_status(_stream(stream), 1 if reset else 0)

@@ -1,0 +1,386 @@
+// C ABI of the library: argument checks, path choice, TMA tensor maps, launches.
+//
+// Every entry point validates its arguments before touching CUDA, so a rejected call has
+// no device-side effect. Validation mirrors the teaching implementation of the CMU DLSys
+// Lecture 14 notes, section 5 (positive dimensions, square filter no larger than the
+// image, matching shapes) and the output-size rule of "Convolution Is Wx+b Moving Across a
+// Signal" (section "Build an image-gradient map, one number at a time") for depthwise.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/conv_b200.h"
+#include "dense_direct.cuh"
+#include "dense_tc.cuh"
+#include "depthwise.cuh"
+#include "ptx.cuh"
+
+namespace convb200 {
+
+// One status word per device; kernels set bits in it with atomicOr.
+__device__ unsigned int g_conv_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr long long kInt32Max = 2147483647LL;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+using EncodeIm2colFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                    const cuuint64_t *, const cuuint64_t *, const int *, const int *,
+                                    cuuint32_t, cuuint32_t, const cuuint32_t *, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned int *status = nullptr;   // device address of g_conv_status on this device
+    unsigned attr_done = 0;           // bit per kernel whose shared-memory limit is raised
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode_tiled = nullptr;
+EncodeIm2colFn g_encode_im2col = nullptr;
+
+// Per-device set-up, done once with that device current.
+int device_state(DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return CONV_ERR_CUDA;
+        void *addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_conv_status) != cudaSuccess) return CONV_ERR_CUDA;
+        d.status = static_cast<unsigned int *>(addr);
+        d.ready = true;
+    }
+    if (!g_encode_tiled || !g_encode_im2col) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+            return CONV_ERR_CUDA;
+        g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
+        fn = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeIm2col", &fn, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+            return CONV_ERR_CUDA;
+        g_encode_im2col = reinterpret_cast<EncodeIm2colFn>(fn);
+    }
+    *out = &d;
+    return CONV_OK;
+}
+
+template <typename Kern>
+int ensure_smem_attr(DeviceState *d, unsigned bit, Kern kern, int bytes) {
+    if (d->attr_done & (1u << bit)) return CONV_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return CONV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    d->attr_done |= 1u << bit;
+    return CONV_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool overlaps(const void *a, long long abytes, const void *b, long long bbytes) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
+}
+
+const char *env(const char *name) {
+    const char *v = std::getenv(name);
+    return (v && *v) ? v : nullptr;
+}
+
+// ---------------------------------------------------------------------------------------
+// Dense
+// ---------------------------------------------------------------------------------------
+int check_dense(const void *X, const void *F, const void *Y, int N, int H, int W, int Cin, int Cout,
+                int K, int elem) {
+    if (!X || !F || !Y) return CONV_ERR_INVALID_ARG;
+    if (N < 1 || H < 1 || W < 1 || Cin < 1 || Cout < 1 || K < 1) return CONV_ERR_INVALID_ARG;
+    if (K > H || K > W) return CONV_ERR_INVALID_ARG;
+    const long long Ho = H - K + 1, Wo = W - K + 1;
+    const long long nx = 1LL * N * H * W * Cin, nf = 1LL * K * K * Cin * Cout, ny = 1LL * N * Ho * Wo * Cout;
+    if (nx > kInt32Max || nf > kInt32Max || ny > kInt32Max || 1LL * N * Ho * Wo > kInt32Max)
+        return CONV_ERR_UNSUPPORTED;
+    if (!aligned(X, elem) || !aligned(F, elem) || !aligned(Y, elem)) return CONV_ERR_MISALIGNED;
+    if (overlaps(Y, ny * elem, X, nx * elem) || overlaps(Y, ny * elem, F, nf * elem))
+        return CONV_ERR_INVALID_ARG;
+    return CONV_OK;
+}
+
+template <typename T>
+int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int Cin, int Cout, int K,
+                        cudaStream_t stream, DeviceState *d) {
+    DenseDirectParams p;
+    p.H = H; p.W = W; p.Cin = Cin; p.Cout = Cout; p.K = K;
+    p.Ho = H - K + 1; p.Wo = W - K + 1;
+    p.total = 1LL * N * p.Ho * p.Wo * Cout;
+    long long blocks = (p.total + 255) / 256;
+    const long long cap = 1LL * d->num_sms * 16;
+    if (blocks > cap) blocks = cap;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, dense_direct_kernel<T>, X, F, Y, p) == cudaSuccess ? CONV_OK
+                                                                                      : CONV_ERR_CUDA;
+}
+
+template <class Cfg>
+int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
+                    cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
+    const int Ho = H - K + 1, Wo = W - K + 1;
+    alignas(64) CUtensorMap tmX, tmF, tmY;
+    {   // X: 4-D {Cin, W, H, N} im2col; the bounding box of valid filter origins is
+        // [0, W-K] x [0, H-K] (upper corner -(K-1)), i.e. exactly the output pixels.
+        const cuuint64_t dims[4] = {(cuuint64_t)Cin, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)N};
+        const cuuint64_t strides[3] = {(cuuint64_t)Cin * 2, (cuuint64_t)W * Cin * 2, (cuuint64_t)H * W * Cin * 2};
+        const int lower[2] = {0, 0};
+        const int upper[2] = {-(K - 1), -(K - 1)};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (g_encode_im2col(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(X), dims, strides,
+                            lower, upper, 64, Cfg::BM, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    {   // F: 3-D {Cout, Cin, K*K}; a box is 64 reduction rows (channels) x 64 output channels
+        const cuuint64_t dims[3] = {(cuuint64_t)Cout, (cuuint64_t)Cin, (cuuint64_t)K * K};
+        const cuuint64_t strides[2] = {(cuuint64_t)Cout * 2, (cuuint64_t)Cin * Cout * 2};
+        const cuuint32_t box[3] = {64, 64, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(F), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    const long long M = 1LL * N * Ho * Wo;
+    {   // Y: 2-D {Cout, M}; a box is 32 rows x 64 channels
+        const cuuint64_t dims[2] = {(cuuint64_t)Cout, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)Cout * 2};
+        const cuuint32_t box[2] = {64, 32};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode_tiled(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    DenseTcParams p;
+    p.M = static_cast<int>(M);
+    p.Wo = Wo;
+    p.HoWo = Ho * Wo;
+    p.K = K;
+    p.Cout = Cout;
+    p.num_cblk = (Cin + 63) / 64;
+    p.num_kblk = K * K * p.num_cblk;
+    p.num_ntiles = (Cout + Cfg::BN - 1) / Cfg::BN;
+    const long long tiles = ((M + Cfg::BM - 1) / Cfg::BM) * p.num_ntiles;
+    if (tiles > kInt32Max) return CONV_ERR_UNSUPPORTED;
+    p.num_tiles = static_cast<int>(tiles);
+    auto kern = dense_tc_kernel<Cfg>;
+    if (int rc = ensure_smem_attr(d, attr_bit, kern, Cfg::SMEM_BYTES)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.num_tiles < d->num_sms ? p.num_tiles : d->num_sms));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kern, tmX, tmF, tmY, p, d->status) == cudaSuccess ? CONV_OK
+                                                                                      : CONV_ERR_CUDA;
+}
+
+using CfgBN64 = DenseTcCfg<64, 6>;
+using CfgBN128 = DenseTcCfg<128, 5>;
+using CfgBN256 = DenseTcCfg<256, 3>;
+
+// ---------------------------------------------------------------------------------------
+// Depthwise
+// ---------------------------------------------------------------------------------------
+constexpr int kDwSmemLimit = 48 * 1024;
+
+long long dw_out(long long in, int k, int s, int pad, int dil) {
+    return (in + 2LL * pad - (1LL * dil * (k - 1) + 1)) / s + 1;
+}
+
+int dw_smem_bytes(const DwParams &p) {
+    return 4 * p.P * (p.w_stride + p.rows_in * p.cols_in);
+}
+
+void dw_set_window(DwParams &p) {
+    p.rows_in = (p.R - 1) * p.stride + (p.KH - 1) * p.dil + 1;
+    p.cols_in = (p.CW - 1) * p.stride + (p.KW - 1) * p.dil + 1;
+}
+
+// Job shape: about 2048 outputs per CTA, whole planes grouped when they are small, and a
+// staged window that fits in kDwSmemLimit.
+void dw_choose_tiles(DwParams &p) {
+    constexpr int kTarget = 2048;
+    p.CW = p.Wo < 128 ? p.Wo : 128;
+    p.R = kTarget / p.CW;
+    if (p.R < 1) p.R = 1;
+    if (p.R > p.Ho) p.R = p.Ho;
+    p.P = 1;
+    if (p.R == p.Ho && p.CW == p.Wo) {
+        long long per = 1LL * p.Ho * p.Wo;
+        long long P = kTarget / per;
+        if (P < 1) P = 1;
+        if (P > 64) P = 64;
+        if (P > p.num_planes) P = p.num_planes;
+        p.P = static_cast<int>(P);
+    }
+    dw_set_window(p);
+    while (dw_smem_bytes(p) > kDwSmemLimit) {
+        if (p.P > 1) p.P = (p.P + 1) / 2;
+        else if (p.R > 1) p.R = (p.R + 1) / 2;
+        else if (p.CW > 1) p.CW = (p.CW + 1) / 2;
+        else break;
+        dw_set_window(p);
+    }
+}
+
+template <int MODE, bool HB>
+int launch_dw(const float *x, const float *w, const float *bias, float *y, const DwParams &p,
+              long long jobs, cudaStream_t stream, DeviceState *d, unsigned bit) {
+    auto kern = depthwise_kernel<MODE, HB>;
+    const int smem = dw_smem_bytes(p);
+    if (smem > 48 * 1024)
+        if (int rc = ensure_smem_attr(d, bit, kern, 227 * 1024)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(jobs));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p) == cudaSuccess ? CONV_OK : CONV_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace convb200
+
+using namespace convb200;
+
+extern "C" {
+
+int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
+                    cudaStream_t stream) {
+    if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 2)) return rc;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    const char *force = env("CONV_B200_DENSE");
+    const bool tc_ok = (Cin % 8 == 0) && (Cout % 8 == 0) && K <= 128 && aligned(X, 16) && aligned(F, 16) &&
+                       aligned(Y, 16) && 2LL * N * H * W * Cin >= 128 * 1024;
+    if (force && std::strcmp(force, "direct") == 0)
+        return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
+                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d);
+    if (!tc_ok) {
+        if (force && std::strncmp(force, "bn", 2) == 0) return CONV_ERR_UNSUPPORTED;
+        return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
+                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d);
+    }
+    int bn = Cout <= 64 ? 64 : 128;
+    if (force && std::strcmp(force, "bn64") == 0) bn = 64;
+    if (force && std::strcmp(force, "bn128") == 0) bn = 128;
+    if (force && std::strcmp(force, "bn256") == 0) bn = 256;
+    if (bn == 64) return launch_dense_tc<CfgBN64>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 0);
+    if (bn == 128) return launch_dense_tc<CfgBN128>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 1);
+    return launch_dense_tc<CfgBN256>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 2);
+}
+
+int conv2d_nhwc_fwd_f32(const float *X, const float *F, float *Y, int N, int H, int W, int Cin, int Cout,
+                        int K, cudaStream_t stream) {
+    if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 4)) return rc;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    return launch_dense_direct(X, F, Y, N, H, W, Cin, Cout, K, stream, d);
+}
+
+int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, int N, int Cin, int mult, int H,
+                  int W, int KH, int KW, int stride, int pad, int dil, int mode, cudaStream_t stream) {
+    if (!x || !w || !y) return CONV_ERR_INVALID_ARG;
+    if (N < 1 || Cin < 1 || mult < 1 || H < 1 || W < 1 || KH < 1 || KW < 1 || stride < 1 || dil < 1 || pad < 0)
+        return CONV_ERR_INVALID_ARG;
+    if (mode != DW_EXACT && mode != DW_FAST) return CONV_ERR_INVALID_ARG;
+    const long long Ho = dw_out(H, KH, stride, pad, dil), Wo = dw_out(W, KW, stride, pad, dil);
+    if (1LL * H + 2LL * pad < 1LL * dil * (KH - 1) + 1 || 1LL * W + 2LL * pad < 1LL * dil * (KW - 1) + 1 ||
+        Ho < 1 || Wo < 1)
+        return CONV_ERR_INVALID_ARG;
+    const long long Cout = 1LL * Cin * mult;
+    const long long nx = 1LL * N * Cin * H * W, nw = Cout * KH * KW, ny = 1LL * N * Cout * Ho * Wo;
+    if (Cout > kInt32Max || nx > kInt32Max || nw > kInt32Max || ny > kInt32Max || 1LL * KH * KW > 4096 ||
+        1LL * H + 2LL * pad > kInt32Max / 2 || 1LL * W + 2LL * pad > kInt32Max / 2)
+        return CONV_ERR_UNSUPPORTED;
+    if (!aligned(x, 4) || !aligned(w, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4)))
+        return CONV_ERR_MISALIGNED;
+    if (overlaps(y, ny * 4, x, nx * 4) || overlaps(y, ny * 4, w, nw * 4) || (bias && overlaps(y, ny * 4, bias, Cout * 4)))
+        return CONV_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+
+    DwParams p;
+    p.Cin = Cin; p.mult = mult; p.Cout = static_cast<int>(Cout); p.H = H; p.W = W; p.KH = KH; p.KW = KW;
+    p.stride = stride; p.pad = pad; p.dil = dil; p.Ho = static_cast<int>(Ho); p.Wo = static_cast<int>(Wo);
+    p.num_planes = 1LL * N * Cout;
+    p.w_stride = (KH * KW + 3) & ~3;
+    dw_choose_tiles(p);
+    if (const char *t = env("CONV_B200_DW_TILE")) {   // "P,R,CW": a forced job shape (tests)
+        int P = 0, R = 0, CW = 0;
+        if (std::sscanf(t, "%d,%d,%d", &P, &R, &CW) == 3 && P >= 1 && R >= 1 && CW >= 1) {
+            p.R = R < p.Ho ? R : p.Ho;
+            p.CW = CW < p.Wo ? CW : p.Wo;
+            p.P = (p.R == p.Ho && p.CW == p.Wo) ? static_cast<int>(P < p.num_planes ? P : p.num_planes) : 1;
+            dw_set_window(p);
+        }
+    }
+    if (dw_smem_bytes(p) > 227 * 1024) return CONV_ERR_UNSUPPORTED;
+    p.n_rbands = (p.Ho + p.R - 1) / p.R;
+    p.n_cbands = (p.Wo + p.CW - 1) / p.CW;
+    const long long groups = (p.num_planes + p.P - 1) / p.P;
+    const long long jobs = groups * p.n_rbands * p.n_cbands;
+    if (jobs > kInt32Max) return CONV_ERR_UNSUPPORTED;
+    const bool hb = bias != nullptr;
+    if (mode == DW_EXACT)
+        return hb ? launch_dw<0, true>(x, w, bias, y, p, jobs, stream, d, 8)
+                  : launch_dw<0, false>(x, w, bias, y, p, jobs, stream, d, 9);
+    return hb ? launch_dw<1, true>(x, w, bias, y, p, jobs, stream, d, 10)
+              : launch_dw<1, false>(x, w, bias, y, p, jobs, stream, d, 11);
+}
+
+const char *conv_status_string(int status) {
+    switch (status) {
+        case CONV_OK: return "ok";
+        case CONV_ERR_INVALID_ARG: return "invalid argument";
+        case CONV_ERR_UNSUPPORTED: return "unsupported shape or size";
+        case CONV_ERR_MISALIGNED: return "misaligned pointer";
+        case CONV_ERR_CUDA: return "CUDA call failed";
+        case CONV_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int conv_device_status(cudaStream_t stream, int reset) {
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return CONV_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpy(&v, d->status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return CONV_ERR_CUDA;
+    if (reset) {
+        const unsigned int zero = 0;
+        if (cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return CONV_ERR_CUDA;
+    }
+    return (v & kStatusTimeout) ? CONV_ERR_DEVICE_TIMEOUT : CONV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Dense NHWC forward convolution on the CUDA cores, one output per thread.
+//
+// This is the path for shapes the tensor-core kernel cannot address with TMA (Cin or Cout
+// not a multiple of 8, tensors below 128 KiB, K > 128) and for the float32 entry point. It
+// evaluates the index contract of the CMU DLSys Lecture 14 notes, section 1, directly:
+// Y[n,y,x,o] = sum over (i, j, c) of X[n,y+i,x+j,c] * F[i,j,c,o], as float32 fused
+// multiply-adds in (i, j, c) order, rounded once to the output type. Consecutive threads
+// take consecutive output channels o, so the F row reads are coalesced and the X reads are
+// warp-uniform broadcasts.
+#pragma once
+#include <cuda_bf16.h>
+
+namespace convb200 {
+
+struct DenseDirectParams {
+    int H, W, Cin, Cout, K, Ho, Wo;
+    long long total;   // N * Ho * Wo * Cout
+};
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
+__device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+dense_direct_kernel(const T *__restrict__ X, const T *__restrict__ F, T *__restrict__ Y,
+                    const DenseDirectParams p) {
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < p.total;
+         idx += stride) {
+        long long t = idx;
+        const int o = static_cast<int>(t % p.Cout);
+        t /= p.Cout;
+        const int x = static_cast<int>(t % p.Wo);
+        t /= p.Wo;
+        const int y = static_cast<int>(t % p.Ho);
+        const long long n = t / p.Ho;
+        float acc = 0.0f;
+        for (int i = 0; i < p.K; ++i) {
+            for (int j = 0; j < p.K; ++j) {
+                const T *xr = X + ((n * p.H + (y + i)) * p.W + (x + j)) * p.Cin;
+                const T *fr = F + ((static_cast<long long>(i) * p.K + j) * p.Cin) * p.Cout + o;
+                for (int c = 0; c < p.Cin; ++c)
+                    acc = __fmaf_rn(to_f32(xr[c]), to_f32(fr[static_cast<long long>(c) * p.Cout]), acc);
+            }
+        }
+        store_out(Y + idx, acc);
+    }
+}
+
+}  // namespace convb200

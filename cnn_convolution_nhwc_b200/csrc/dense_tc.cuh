@@ -1,0 +1,276 @@
+// Dense NHWC forward convolution as an implicit GEMM on the sm_100a tensor cores.
+//
+// Matrix form (CMU DLSys Lecture 14 notes, section 5 "Generalize the patch matrix to
+// channels and batches"): A_col[(n,y,x), (i,j,c)] = X[n, y+i, x+j, c] is the
+// (N*Ho*Wo) x (K*K*Cin) patch matrix, F_mat is F viewed as (K*K*Cin) x Cout, and
+// Y_mat = A_col * F_mat is Y viewed as (N*Ho*Wo) x Cout. The notes' closing remark in
+// section 6 -- generate patch fragments as needed instead of materialising the matrix --
+// is what this kernel does: A_col never exists in memory. Each 128-row x 64-column block of
+// it is gathered straight from X by one TMA im2col load (the hardware form of the
+// overlapping-window view of section 4), for filter tap (i, j) and channel block c0, and
+// consumed from shared memory by tcgen05 MMAs. The reduction runs tap by tap, which is the
+// sum of K*K shifted-slice channel matmuls of section 2.
+//
+// Roles inside one persistent CTA of 6 warps:
+//   warp 0      one thread issues TMA loads into a STAGES-deep ring of (A, B) slots;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) into one
+//               of two TMEM accumulators, and tcgen05.commit to free ring slots;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads TMEM lanes
+//               32*(w%4) .. +31), round to bf16, 128-byte-swizzled staging in shared
+//               memory, TMA store to Y. The two accumulators let tile t+1's MMAs run
+//               while tile t is stored.
+// Shared-memory operand layouts (both 128-byte swizzled, as TMA writes them):
+//   A slot: 128 pixel rows x 64 channels (128 B per row) -- K-major.
+//   B slot: BN/64 boxes, each 64 reduction rows x 64 output channels (128 B per row) --
+//           MN-major, read in place from the KKIO filter, no repacking.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace convb200 {
+
+struct DenseTcParams {
+    int M;          // N * Ho * Wo (GEMM rows)
+    int Wo;
+    int HoWo;
+    int K;
+    int Cout;
+    int num_cblk;   // ceil(Cin / 64)
+    int num_kblk;   // K * K * num_cblk
+    int num_ntiles; // ceil(Cout / BN)
+    int num_tiles;  // ceil(M / 128) * num_ntiles
+};
+
+template <int BN_, int STAGES_>
+struct DenseTcCfg {
+    static constexpr int BN = BN_;
+    static constexpr int STAGES = STAGES_;
+    static constexpr int BM = 128;
+    static constexpr int BK = 64;
+    static constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+    static constexpr int B_BOX_BYTES = BK * 64 * 2;    // 8 KB: 64 k-rows x 64 channels
+    static constexpr int B_BYTES = BK * BN * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int EPI_WARP_BYTES = 32 * BN * 2; // 32 rows x BN channels
+    static constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+    static constexpr int TMEM_COLS = 2 * BN;           // two accumulators
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
+    static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ true);
+    static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
+    static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM columns");
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(192, 1)
+dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
+                const __grid_constant__ CUtensorMap tmY, const DenseTcParams p,
+                unsigned int *status) {
+    constexpr int BN = Cfg::BN;
+    constexpr int STAGES = Cfg::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;   // 1024-B alignment for the swizzle
+    uint8_t *smem = smem_raw + (base - raw_base);
+
+    const uint32_t sA = base;
+    const uint32_t sB = base + STAGES * Cfg::A_BYTES;
+    uint8_t *sEpi = smem + STAGES * Cfg::STAGE_BYTES;
+    const uint32_t bars = base + STAGES * Cfg::STAGE_BYTES + Cfg::EPI_BYTES;
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
+    auto accf_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
+    auto acce_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t done_bar = bars + 8u * (2 * STAGES + 4);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + STAGES * Cfg::STAGE_BYTES +
+                                                         Cfg::EPI_BYTES + Cfg::NUM_BARS * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf_bar(b), 1);
+            mbar_init(acce_bar(b), 128);
+        }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmF);
+        prefetch_tensormap(&tmY);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    auto fail = [&]() {
+        atomicOr(status, kStatusTimeout);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------- TMA producer -------------------------------
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
+                const int mt = tile / p.num_ntiles;
+                const int nt = tile - mt * p.num_ntiles;
+                const int m0 = mt * Cfg::BM;
+                const int n0 = nt * BN;
+                const int img = m0 / p.HoWo;
+                const int rem = m0 - img * p.HoWo;
+                const int oy = rem / p.Wo;
+                const int ox = rem - oy * p.Wo;
+                bool ok = true;
+                for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
+                    const int tap = kb / p.num_cblk;
+                    const int cb = kb - tap * p.num_cblk;
+                    const int ky = tap / p.K;
+                    const int kx = tap - ky * p.K;
+                    const uint32_t s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u)) { fail(); ok = false; break; }
+                    mbar_arrive_expect_tx(full_bar(s), Cfg::STAGE_BYTES);
+                    tma_load_im2col_4d(sA + s * Cfg::A_BYTES, &tmX, full_bar(s), cb * 64, ox, oy, img,
+                                       static_cast<uint16_t>(kx), static_cast<uint16_t>(ky));
+#pragma unroll
+                    for (int h = 0; h < BN / 64; ++h)
+                        tma_load_3d(sB + s * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, &tmF, full_bar(s),
+                                    n0 + h * 64, cb * 64, tap);
+                }
+                if (!ok) break;
+            }
+            // Drain: every load issued has landed before the CTA may exit.
+            const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+            for (uint32_t j = first; j < it; ++j)
+                if (!mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1u)) { fail(); break; }
+        }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer ---------------------------------
+        if (lane == 0) {
+            uint32_t it = 0, local = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x, ++local) {
+                const uint32_t b = local & 1u;
+                const uint32_t aph = (local >> 1) & 1u;
+                if (!mbar_wait(acce_bar(b), aph ^ 1u)) { fail(); break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * BN;
+                bool ok = true;
+                for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
+                    const uint32_t s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(full_bar(s), ph)) { fail(); ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = sA + s * Cfg::A_BYTES;
+                    const uint32_t b0 = sB + s * Cfg::B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
+                        // A: K-major, advance 16 channels = 32 B inside the swizzle atom;
+                        //    8-row groups are 1024 B apart.
+                        const uint64_t ad = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+                        // B: MN-major, advance 16 reduction rows = 2048 B; 8-row groups
+                        //    1024 B apart (SBO), 64-channel boxes 8 KB apart (LBO).
+                        const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, Cfg::B_BOX_BYTES, 1024);
+                        umma_f16_ss(d_tmem, ad, bd, Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(empty_bar(s));
+                }
+                if (!ok) break;
+                umma_commit(accf_bar(b));
+            }
+            // All MMAs issued by this thread complete before TMEM is released.
+            umma_commit(done_bar);
+            if (!mbar_wait(done_bar, 0)) fail();
+        }
+    } else {
+        // ------------------------------- Epilogue -----------------------------------
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        uint8_t *stage = sEpi + q * Cfg::EPI_WARP_BYTES;
+        const uint32_t stage_s = smem_u32(stage);
+        uint32_t local = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            const uint32_t b = local & 1u;
+            const uint32_t aph = (local >> 1) & 1u;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(accf_bar(b), aph));
+            if (!ok) { if (lane == 0) fail(); break; }
+            tc_fence_after();
+            const int mt = tile / p.num_ntiles;
+            const int nt = tile - mt * p.num_ntiles;
+            const int m0 = mt * Cfg::BM;
+            const int n0 = nt * BN;
+            // the staging buffer is free once the previous tile's stores have read it
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+#pragma unroll 1
+            for (int h = 0; h < BN / 64; ++h) {
+                uint32_t r[4][16];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + h * 64 + g * 16, r[g]);
+                tmem_wait_ld();
+                const uint32_t row_addr = stage_s + h * 4096 + lane * 128;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const uint32_t c = g * 2 + cc;   // 16-byte chunk = 8 channels
+                        const uint32_t* v = &r[g][cc * 8];
+                        st_shared_v4(row_addr + ((c ^ (lane & 7)) << 4),
+                                     pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                                     pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                                     pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                                     pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                    }
+                }
+            }
+            // accumulator b may now be overwritten by the MMA warp
+            tc_fence_before();
+            mbar_arrive(acce_bar(b));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int row0 = m0 + q * 32;
+                if (row0 < p.M) {
+#pragma unroll
+                    for (int h = 0; h < BN / 64; ++h)
+                        if (n0 + h * 64 < p.Cout) tma_store_2d(&tmY, stage_s + h * 4096, n0 + h * 64, row0);
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+}  // namespace convb200

@@ -1,0 +1,112 @@
+/*
+ * conv_b200 -- forward 2-D convolution for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * Two operations, both in the neural-network cross-correlation convention (the filter is
+ * not reversed):
+ *
+ *  1. Dense NHWC convolution with a square K x K filter, unit stride, no padding, no
+ *     dilation, no groups and no bias. Defined in the CMU DLSys Lecture 14 notes, "The hidden
+ *     copy behind convolution as matrix multiplication", section 1 "Fix the index contract
+ *     before optimizing it":
+ *         Ho = H - K + 1,  Wo = W - K + 1,
+ *         Y[n,y,x,o] = sum_{i<K} sum_{j<K} sum_{c<Cin} X[n,y+i,x+j,c] * F[i,j,c,o].
+ *     Section 5 of the same notes gives the matrix form the kernel evaluates without ever
+ *     storing the patch matrix: rows are the N*Ho*Wo output pixels, the reduction runs over
+ *     (i, j, c) and the columns are the Cout filters.
+ *
+ *  2. Depthwise convolution (groups == Cin, Cout = Cin * mult) on NCHW planes with stride,
+ *     zero padding, dilation and an optional bias. Defined in the OneModel docs, "Depthwise
+ *     convolution", section "What each output is": output channel oc reads input channel
+ *     oc / mult; acc starts at +0; taps run ky outer, kx inner; padding is a real zero that
+ *     is multiplied (so an infinite or NaN weight meeting padding gives NaN); the bias is a
+ *     separate pass of one rounded addition. Output size per axis from "Convolution Is Wx+b
+ *     Moving Across a Signal", section "Build an image-gradient map, one number at a time":
+ *         out = floor((in + 2*pad - (dil*(k-1) + 1)) / stride) + 1.
+ *
+ * Common rules for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller (for example allocated by
+ *    PyTorch). Tensors are dense and contiguous in the stated layout. The library keeps no
+ *    reference to them after the call returns and allocates no device memory per call.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream) and never synchronise.
+ *    Outputs are fully overwritten. Inputs are read only. Outputs must not overlap inputs.
+ *  - The return value is a conv_status; no exception or abort crosses the ABI. Argument
+ *    checks happen before any CUDA call, so a rejected call has no effect on the device.
+ *  - A device-side wait that exceeds its time limit (about one second) makes the kernel
+ *    stop, record CONV_ERR_DEVICE_TIMEOUT in a per-process device status word and return;
+ *    read it with conv_device_status().
+ */
+#ifndef CONV_B200_H
+#define CONV_B200_H
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CONV_OK = 0,
+    CONV_ERR_INVALID_ARG = -1,    /* null tensor pointer, non-positive size, K > min(H, W), ... */
+    CONV_ERR_UNSUPPORTED = -2,    /* valid arguments outside what this library implements */
+    CONV_ERR_MISALIGNED = -3,     /* a pointer not aligned to its element size */
+    CONV_ERR_CUDA = -4,           /* a CUDA runtime or driver call failed (launch, tensor map) */
+    CONV_ERR_DEVICE_TIMEOUT = -5  /* a bounded device-side wait ran out (see conv_device_status) */
+} conv_status;
+
+typedef enum {
+    DW_EXACT = 0, /* product rounded, then sum rounded; NaN results become 0x7FC00000 */
+    DW_FAST = 1   /* one fused multiply-add per tap */
+} dw_mode;
+
+/*
+ * Dense NHWC forward convolution, bfloat16 in and out, float32 accumulation.
+ *   X : bfloat16 [N][H][W][Cin]          (NHWC, channels contiguous)
+ *   F : bfloat16 [K][K][Cin][Cout]       (KKIO: row (i, j, c) of the K*K*Cin x Cout matrix)
+ *   Y : bfloat16 [N][H-K+1][W-K+1][Cout] (NHWC), each output rounded to nearest even once
+ * Requirements: N, H, W, Cin, Cout, K >= 1; K <= min(H, W); all pointers non-null and
+ * 2-byte aligned; N*H*W*Cin, N*Ho*Wo*Cout and K*K*Cin*Cout below 2^31.
+ * The tensor-core path needs Cin and Cout multiples of 8, 16-byte aligned pointers and
+ * K <= 128; other valid shapes take a CUDA-core path with the same contract.
+ */
+int conv2d_nhwc_fwd(const void *X, const void *F, void *Y,
+                    int N, int H, int W, int Cin, int Cout, int K, cudaStream_t stream);
+
+/*
+ * The same operation with float32 tensors (same layouts and requirements; 4-byte aligned
+ * pointers). Products and sums are float32 fused multiply-adds in (i, j, c) order, so any
+ * input whose partial sums are integers below 2^24 in magnitude gives the exact result.
+ */
+int conv2d_nhwc_fwd_f32(const float *X, const float *F, float *Y,
+                        int N, int H, int W, int Cin, int Cout, int K, cudaStream_t stream);
+
+/*
+ * Depthwise forward convolution, float32.
+ *   x    : [N][Cin][H][W]
+ *   w    : [Cin*mult][KH][KW]   (plane oc belongs to input channel oc / mult)
+ *   bias : [Cin*mult] or NULL
+ *   y    : [N][Cin*mult][Ho][Wo]
+ * stride, pad and dil apply to both axes; padding is symmetric. mode is DW_EXACT or DW_FAST.
+ * Requirements: N, Cin, mult, H, W, KH, KW, stride, dil >= 1; pad >= 0; Ho, Wo >= 1;
+ * pointers non-null (bias may be NULL) and 4-byte aligned; element counts below 2^31.
+ * Exact mode is bit-for-bit the page's definition; fast mode uses a correctly rounded
+ * fused multiply-add per tap in the same order.
+ */
+int depthwise_fwd(const float *x, const float *w, const float *bias, float *y,
+                  int N, int Cin, int mult, int H, int W, int KH, int KW,
+                  int stride, int pad, int dil, int mode, cudaStream_t stream);
+
+/* Static English text for a conv_status value (never NULL). */
+const char *conv_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads the device status word of the current device:
+ * CONV_OK, CONV_ERR_DEVICE_TIMEOUT, or CONV_ERR_CUDA if the synchronisation itself failed.
+ * With reset != 0 the word is cleared afterwards.
+ */
+int conv_device_status(cudaStream_t stream, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONV_B200_H */

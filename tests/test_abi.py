@@ -1,0 +1,100 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header declares, and
+rejects bad arguments with the documented status codes before it makes any CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import cnn_convolution_nhwc_b200 as cb
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "conv_b200.h")
+V = ctypes.c_void_p
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", src, flags=re.M))
+
+
+def test_header_declares_the_entry_points():
+    assert _declared() == set(cb.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", cb.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared():
+        assert name in syms, name
+        assert getattr(cb.lib, name) is not None
+
+
+def test_status_strings():
+    for code in (cb.CONV_OK, cb.CONV_ERR_INVALID_ARG, cb.CONV_ERR_UNSUPPORTED, cb.CONV_ERR_MISALIGNED,
+                 cb.CONV_ERR_CUDA, cb.CONV_ERR_DEVICE_TIMEOUT):
+        s = cb.conv_status_string(code)
+        assert s and s != "unknown status"
+    assert cb.conv_status_string(12345) == "unknown status"
+
+
+# Fake device addresses: validation only looks at their values, never dereferences them.
+X, F, Y = V(1 << 20), V(1 << 24), V(1 << 28)
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, F, Y, 1, 5, 5, 8, 8, 3), cb.CONV_ERR_INVALID_ARG),
+    ((X, None, Y, 1, 5, 5, 8, 8, 3), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, None, 1, 5, 5, 8, 8, 3), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, Y, 0, 5, 5, 8, 8, 3), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, Y, 1, 5, 5, 0, 8, 3), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, Y, 1, 5, 5, 8, -2, 3), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, Y, 1, 5, 5, 8, 8, 0), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, Y, 1, 5, 2, 8, 8, 3), cb.CONV_ERR_INVALID_ARG),        # K > W
+    ((X, F, Y, 1, 2, 5, 8, 8, 3), cb.CONV_ERR_INVALID_ARG),        # K > H
+    ((V((1 << 20) + 1), F, Y, 1, 5, 5, 8, 8, 3), cb.CONV_ERR_MISALIGNED),
+    ((X, F, V(1 << 20), 1, 5, 5, 8, 8, 3), cb.CONV_ERR_INVALID_ARG),  # Y aliases X
+    ((X, F, Y, 4096, 4096, 4096, 64, 8, 3), cb.CONV_ERR_UNSUPPORTED),
+])
+def test_dense_rejects(args, code):
+    assert cb.lib.conv2d_nhwc_fwd(*args, None) == code
+    if code != cb.CONV_ERR_MISALIGNED:
+        assert cb.lib.conv2d_nhwc_fwd_f32(*args, None) == code
+
+
+def test_dense_f32_needs_4_byte_alignment():
+    assert cb.lib.conv2d_nhwc_fwd_f32(V((1 << 20) + 2), F, Y, 1, 5, 5, 8, 8, 3, None) == cb.CONV_ERR_MISALIGNED
+
+
+B = V(1 << 30)
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, F, B, Y, 1, 2, 1, 5, 5, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_INVALID_ARG),
+    ((X, None, B, Y, 1, 2, 1, 5, 5, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, B, None, 1, 2, 1, 5, 5, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, B, Y, 1, 2, 0, 5, 5, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_INVALID_ARG),   # mult 0
+    ((X, F, B, Y, 1, 2, 1, 5, 5, 3, 3, 0, 1, 1, 0), cb.CONV_ERR_INVALID_ARG),   # stride 0
+    ((X, F, B, Y, 1, 2, 1, 5, 5, 3, 3, 1, -1, 1, 0), cb.CONV_ERR_INVALID_ARG),  # pad < 0
+    ((X, F, B, Y, 1, 2, 1, 5, 5, 3, 3, 1, 1, 0, 0), cb.CONV_ERR_INVALID_ARG),   # dil 0
+    ((X, F, B, Y, 1, 2, 1, 5, 5, 3, 3, 1, 1, 1, 2), cb.CONV_ERR_INVALID_ARG),   # bad mode
+    ((X, F, B, Y, 1, 2, 1, 2, 2, 5, 5, 1, 0, 1, 0), cb.CONV_ERR_INVALID_ARG),   # empty output
+    ((X, F, B, Y, 1, 2, 1, 5, 5, 3, 3, 1, 0, 3, 0), cb.CONV_ERR_INVALID_ARG),   # dilated kernel too big
+    ((V((1 << 20) + 2), F, B, Y, 1, 2, 1, 5, 5, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_MISALIGNED),
+    ((X, F, V((1 << 30) + 1), Y, 1, 2, 1, 5, 5, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_MISALIGNED),
+    ((X, F, B, V((1 << 20) + 64), 1, 2, 1, 5, 5, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_INVALID_ARG),  # y overlaps x
+    ((X, F, B, Y, 65536, 65536, 1, 8, 8, 3, 3, 1, 1, 1, 0), cb.CONV_ERR_UNSUPPORTED),
+])
+def test_depthwise_rejects(args, code):
+    assert cb.lib.depthwise_fwd(*args, None) == code
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        cb.conv2d_nhwc_fwd(torch.zeros(1, 5, 5, 8, dtype=torch.bfloat16), torch.zeros(3, 3, 8, 8, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        cb.depthwise_fwd(torch.zeros(1, 2, 5, 5), torch.zeros(2, 3, 3))

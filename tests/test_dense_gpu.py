@@ -1,0 +1,241 @@
+"""Dense NHWC convolution on the GPU against the CPU oracle, through the C ABI.
+
+Tolerance for bfloat16 output: |y - y_ref| <= 4e-3 * sum|x||w| per output, where y_ref is the
+oracle's float64 sum of the same bfloat16 operands. The budget is one round-to-nearest of the
+output to bfloat16 (at most 2**-9 relative, below 1.96e-3 of the magnitude sum) plus float32
+accumulation error (below 2**-24 * (terms + 1) of the magnitude sum, well inside the rest).
+The float32 entry point on small-integer inputs must be exact.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.conftest import GOLDEN
+
+pytestmark = pytest.mark.gpu
+
+TOL = 4e-3
+
+
+@pytest.fixture(scope="module")
+def cb(cuda):
+    import cnn_convolution_nhwc_b200 as cb
+    return cb
+
+
+def _dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _host_bf16(t):
+    return workloads.bf16_to_f32(t.view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def _run_bf16(cb, Xb, Fb, env=None):
+    old = os.environ.get("CONV_B200_DENSE")
+    if env is not None:
+        os.environ["CONV_B200_DENSE"] = env
+    try:
+        Y = cb.conv2d_nhwc_fwd(_dev_bf16(Xb), _dev_bf16(Fb))
+        torch.cuda.synchronize()
+    finally:
+        if env is not None:
+            if old is None:
+                del os.environ["CONV_B200_DENSE"]
+            else:
+                os.environ["CONV_B200_DENSE"] = old
+    assert cb.conv_device_status() == cb.CONV_OK
+    return _host_bf16(Y)
+
+
+def _check_bf16(y, Xb, Fb):
+    ref, absum = oracle.conv2d_nhwc(workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb))
+    assert y.shape == ref.shape
+    assert np.all(np.isfinite(y))
+    err = np.abs(y.astype(np.float64) - ref)
+    bad = err > TOL * absum
+    assert not bad.any(), f"{bad.sum()} outputs out of tolerance; worst {np.max(err / np.maximum(absum, 1e-30))}"
+    return ref
+
+
+def _case_inputs(N, H, W, Cin, Cout, K, seed):
+    c = workloads.DenseCase("t", N, H, W, Cin, Cout, K, "bf16", "normal", seed)
+    return workloads.dense_inputs(c)
+
+
+# ------------------------------------------------------------------------------------------
+# Worked examples from the pages, through both paths
+# ------------------------------------------------------------------------------------------
+
+
+def test_pins_direct_path(cb):
+    g = json.load(open(os.path.join(GOLDEN, "dlsys14_patch_example.json")))
+    X = np.arange(36, dtype=np.float32).reshape(1, 6, 6, 1)
+    F = np.arange(9, dtype=np.float32).reshape(3, 3, 1, 1)
+    Y = cb.conv2d_nhwc_fwd_f32(torch.from_numpy(X).cuda(), torch.from_numpy(F).cuda()).cpu().numpy()
+    assert np.array_equal(Y[0, :, :, 0], np.array(g["output"], np.float32))
+    # bfloat16 entry: inputs are exact, outputs above 256 round (1122 -> 1120)
+    y = _run_bf16(cb, workloads.bf16_bits(X), workloads.bf16_bits(F))
+    assert np.array_equal(y[0, :, :, 0], workloads.bf16_to_f32(workloads.bf16_bits(np.array(g["output"], np.float32))))
+    s = json.load(open(os.path.join(GOLDEN, "wxb_2d_examples.json")))
+    t = s["tiny_2d"]
+    Y = cb.conv2d_nhwc_fwd_f32(torch.tensor(t["image"], dtype=torch.float32).reshape(1, 3, 3, 1).cuda(),
+                               torch.tensor(t["filter"], dtype=torch.float32).reshape(2, 2, 1, 1).cuda())
+    assert Y[0, :, :, 0].cpu().tolist() == t["output"]
+    so = s["sobel"]
+    Fs = torch.stack([torch.tensor(so["gx"]), torch.tensor(so["gy"])], -1).float().reshape(3, 3, 1, 2)
+    Y = cb.conv2d_nhwc_fwd_f32(torch.tensor(so["image"], dtype=torch.float32).reshape(1, 6, 6, 1).cuda(), Fs.cuda())
+    assert Y[0, :, :, 0].cpu().tolist() == so["gx_output"] and Y[0, :, :, 1].cpu().tolist() == so["gy_output"]
+
+
+def test_pins_tensor_core_path(cb):
+    # The 6x6 example and the Sobel pair, replicated over 256 images and placed in channel 0
+    # of 8 input channels and output channels 0 and 1 of 8, so the tensor-core path takes it.
+    g = json.load(open(os.path.join(GOLDEN, "dlsys14_patch_example.json")))
+    so = json.load(open(os.path.join(GOLDEN, "wxb_2d_examples.json")))["sobel"]
+    N = 256
+    X = np.zeros((N, 6, 6, 8), np.float32)
+    X[:, :, :, 0] = np.arange(36, dtype=np.float32).reshape(6, 6)
+    X[:, :, :, 3] = np.array(so["image"], np.float32)
+    F = np.zeros((3, 3, 8, 8), np.float32)
+    F[:, :, 0, 0] = np.arange(9, dtype=np.float32).reshape(3, 3)
+    F[:, :, 3, 1] = np.array(so["gx"], np.float32)
+    F[:, :, 3, 2] = np.array(so["gy"], np.float32)
+    y = _run_bf16(cb, workloads.bf16_bits(X), workloads.bf16_bits(F), env="bn64")
+    exp0 = workloads.bf16_to_f32(workloads.bf16_bits(np.array(g["output"], np.float32)))
+    for n in (0, 1, 100, N - 1):
+        assert np.array_equal(y[n, :, :, 0], exp0)
+        assert np.array_equal(y[n, :, :, 1], np.array(so["gx_output"], np.float32))
+        assert np.array_equal(y[n, :, :, 2], np.array(so["gy_output"], np.float32))
+        assert not y[n, :, :, 3:].any()
+
+
+# ------------------------------------------------------------------------------------------
+# The workloads
+# ------------------------------------------------------------------------------------------
+
+
+def test_tiny_fp32_config_exact(cb):
+    c = workloads.DENSE_TINY
+    X, F = workloads.dense_inputs(c)
+    Y = cb.conv2d_nhwc_fwd_f32(torch.from_numpy(X).cuda(), torch.from_numpy(F).cuda()).cpu().numpy()
+    ref, _ = oracle.conv2d_nhwc(X, F)
+    assert np.array_equal(Y.astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("case", [workloads.DENSE_3X3, workloads.DENSE_1X1], ids=lambda c: c.name)
+def test_workload_full_output(cb, case):
+    Xb, Fb = workloads.dense_inputs(case)
+    y = _run_bf16(cb, Xb, Fb)
+    _check_bf16(y, Xb, Fb)
+
+
+def test_pointwise_is_matmul(cb):
+    # K = 1: Y = X @ F[0,0] (DLSys notes section 2), checked against a float64 matmul
+    case = workloads.DENSE_1X1
+    Xb, Fb = workloads.dense_inputs(case)
+    y = _run_bf16(cb, Xb, Fb)
+    Xf = workloads.bf16_to_f32(Xb).reshape(-1, case.Cin).astype(np.float64)
+    Ff = workloads.bf16_to_f32(Fb)[0, 0].astype(np.float64)
+    ref = Xf @ Ff
+    bound = np.abs(Xf) @ np.abs(Ff)
+    assert np.all(np.abs(y.reshape(ref.shape) - ref) <= TOL * bound)
+
+
+def test_large_workload_sampled(cb):
+    # N=64, 112x112, 128->128, K=5: compare 20000 sampled outputs (including the first and
+    # last pixels of every image corner region and the last M tile) with the oracle.
+    case = workloads.DENSE_LARGE
+    Xb, Fb = workloads.dense_inputs(case)
+    y = _run_bf16(cb, Xb, Fb)
+    Ho, Wo, Co = case.Ho, case.Wo, case.Cout
+    total = case.N * Ho * Wo * Co
+    r = workloads.splitmix64(77, 20000)
+    idx = (r % np.uint64(total)).astype(np.int64)
+    corners = []
+    for n in (0, case.N // 2, case.N - 1):
+        for (yy, xx) in ((0, 0), (0, Wo - 1), (Ho - 1, 0), (Ho - 1, Wo - 1)):
+            for o in (0, Co - 1):
+                corners.append(((n * Ho + yy) * Wo + xx) * Co + o)
+    idx = np.concatenate([idx, np.array(corners, np.int64), np.arange(total - 128 * Co, total, 97)])
+    ref, absum = oracle.conv2d_nhwc_points(workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb), idx)
+    got = y.reshape(-1)[idx].astype(np.float64)
+    assert np.all(np.abs(got - ref) <= TOL * absum)
+    assert np.all(np.isfinite(y))
+
+
+# ------------------------------------------------------------------------------------------
+# Edge shapes: ragged M and N tiles, partial channel blocks, small / odd channel counts,
+# full-image filters, K = 7, non-square images
+# ------------------------------------------------------------------------------------------
+
+EDGE = [
+    (3, 20, 23, 72, 24, 3),     # ragged M tile, Cin = 64 + 8, Cout < 64
+    (64, 16, 16, 8, 16, 3),     # Cin = 8
+    (8, 30, 17, 24, 40, 2),     # Cin = 24, even K, non-square
+    (32, 8, 8, 64, 64, 8),      # K = H = W: Ho = Wo = 1, each output a dot product
+    (4, 19, 27, 64, 136, 7),    # K = 7, Cout = 128 + 8
+    (2, 40, 40, 128, 256, 1),   # pointwise with two 128-wide N tiles
+    (5, 33, 9, 40, 200, 4),     # Cout = 200
+]
+
+
+@pytest.mark.parametrize("shape", EDGE, ids=lambda s: "x".join(map(str, s)))
+def test_edge_shapes(cb, shape):
+    N, H, W, Cin, Cout, K = shape
+    Xb, Fb = _case_inputs(N, H, W, Cin, Cout, K, seed=sum(shape))
+    y = _run_bf16(cb, Xb, Fb)
+    _check_bf16(y, Xb, Fb)
+
+
+@pytest.mark.parametrize("shape", [(2, 7, 9, 3, 5, 3), (1, 5, 5, 1, 1, 5), (3, 6, 11, 12, 10, 2)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_unaligned_channels_direct_path(cb, shape):
+    N, H, W, Cin, Cout, K = shape
+    Xb, Fb = _case_inputs(N, H, W, Cin, Cout, K, seed=sum(shape) + 1)
+    y = _run_bf16(cb, Xb, Fb)
+    _check_bf16(y, Xb, Fb)
+
+
+def test_tile_width_choices_agree(cb):
+    # every tile width computes each output with the same MMA sequence over the reduction
+    Xb, Fb = _case_inputs(4, 24, 24, 64, 256, 3, seed=5)
+    ys = {bn: _run_bf16(cb, Xb, Fb, env=bn) for bn in ("bn64", "bn128", "bn256")}
+    _check_bf16(ys["bn64"], Xb, Fb)
+    for bn in ("bn128", "bn256"):
+        assert np.array_equal(ys[bn], ys["bn64"]), bn
+    yd = _run_bf16(cb, Xb, Fb, env="direct")
+    _check_bf16(yd, Xb, Fb)
+
+
+def test_repeatable(cb):
+    Xb, Fb = workloads.dense_inputs(workloads.DENSE_3X3)
+    a = _run_bf16(cb, Xb, Fb)
+    b = _run_bf16(cb, Xb, Fb)
+    assert np.array_equal(a, b)
+
+
+def test_translation_equivariance(cb):
+    # shifting the input one column right shifts the output one column (stride 1, interior)
+    Xb, Fb = _case_inputs(8, 20, 30, 64, 64, 3, seed=9)
+    Xs = np.zeros_like(Xb)
+    Xs[:, :, 1:, :] = Xb[:, :, :-1, :]
+    y = _run_bf16(cb, Xb, Fb)
+    ys = _run_bf16(cb, Xs, Fb)
+    assert np.array_equal(ys[:, :, 1:, :], y[:, :, :-1, :])
+
+
+def test_noncontiguous_rejected_and_contiguous_copy_works(cb):
+    Xb, Fb = _case_inputs(4, 16, 16, 64, 64, 3, seed=3)
+    X = _dev_bf16(Xb)
+    Xt = X.permute(0, 2, 1, 3)   # a transposed view: not contiguous
+    with pytest.raises(ValueError):
+        cb.conv2d_nhwc_fwd(Xt, _dev_bf16(Fb))
+    y = _host_bf16(cb.conv2d_nhwc_fwd(Xt.contiguous(), _dev_bf16(Fb)))
+    torch.cuda.synchronize()
+    _check_bf16(y, np.ascontiguousarray(Xb.transpose(0, 2, 1, 3)), Fb)

@@ -1,0 +1,196 @@
+"""Depthwise convolution on the GPU against the CPU oracle, through the C ABI.
+
+Exact mode must be bit-identical to the oracle. Fast mode must satisfy
+|y - y_ref| <= 1e-6 * (sum over taps |w*x| + |bias|) per output (the relative bound, scaled
+by the magnitude of the terms so outputs near zero are not judged by a meaningless ratio);
+both sides use a correctly rounded fused multiply-add in the same order, so the tests also
+expect bit identity there. NaN outputs compare as NaN on both sides in fast mode.
+"""
+import json
+import os
+import struct
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.conftest import GOLDEN
+
+pytestmark = pytest.mark.gpu
+
+MODES = [oracle.DW_EXACT, oracle.DW_FAST]
+
+
+@pytest.fixture(scope="module")
+def cb(cuda):
+    import cnn_convolution_nhwc_b200 as cb
+    return cb
+
+
+def _bits(a):
+    return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+
+
+def _gpu(cb, x, w, b, stride=1, pad=0, dil=1, mode=0, tile=None):
+    old = os.environ.get("CONV_B200_DW_TILE")
+    if tile is not None:
+        os.environ["CONV_B200_DW_TILE"] = tile
+    try:
+        y = cb.depthwise_fwd(torch.from_numpy(np.ascontiguousarray(x, np.float32)).cuda(),
+                             torch.from_numpy(np.ascontiguousarray(w, np.float32)).cuda(),
+                             None if b is None else torch.from_numpy(np.ascontiguousarray(b, np.float32)).cuda(),
+                             stride=stride, pad=pad, dil=dil, mode=mode)
+        out = y.cpu().numpy()
+    finally:
+        if tile is not None:
+            if old is None:
+                del os.environ["CONV_B200_DW_TILE"]
+            else:
+                os.environ["CONV_B200_DW_TILE"] = old
+    assert cb.conv_device_status() == cb.CONV_OK
+    return out
+
+
+def _compare(y, x, w, b, mult, stride, pad, dil, mode):
+    ref = oracle.depthwise(x, w, b, mult=mult, stride=stride, pad=pad, dil=dil, mode=mode)
+    assert y.shape == ref.shape
+    if mode == oracle.DW_EXACT:
+        same = _bits(y) == _bits(ref)
+        assert same.all(), f"{(~same).sum()} of {y.size} outputs differ in exact mode"
+    else:
+        bound = oracle.depthwise_absbound(x, w, b, mult=mult, stride=stride, pad=pad, dil=dil)
+        both_nan = np.isnan(y) & np.isnan(ref)
+        ok = both_nan | (np.abs(y.astype(np.float64) - ref) <= 1e-6 * bound)
+        assert ok.all(), f"{(~ok).sum()} fast-mode outputs out of tolerance"
+        same = (_bits(y) == _bits(ref)) | both_nan
+        assert same.all(), f"fast mode: {(~same).sum()} outputs not bit-identical"
+
+
+@pytest.mark.parametrize("mode", MODES, ids=["exact", "fast"])
+@pytest.mark.parametrize("case", workloads.DW_SWEEP, ids=lambda c: c.name)
+def test_sweep_full_output(cb, case, mode):
+    x, w, b = workloads.depthwise_inputs(case)
+    y = _gpu(cb, x, w, b, case.stride, case.pad, case.dil, mode)
+    _compare(y, x, w, b, case.mult, case.stride, case.pad, case.dil, mode)
+
+
+@pytest.mark.parametrize("mode", MODES, ids=["exact", "fast"])
+def test_page_examples(cb, mode):
+    g = json.load(open(os.path.join(GOLDEN, "wxb_1d_examples.json")))
+    e = g["weighted_sum_with_bias"]
+    y = _gpu(cb, np.array(e["x"]).reshape(1, 1, 1, -1), np.array(e["k"]).reshape(1, 1, -1), [e["bias"]], mode=mode)
+    assert y.ravel().tolist() == e["output"]
+    third = np.float32(1) / np.float32(3)
+    y = _gpu(cb, np.array(g["spike_average"]["x"]).reshape(1, 1, 1, -1), np.full((1, 1, 3), third), None, mode=mode)
+    assert y.ravel().tolist() == g["spike_average"]["output"]
+    for name in ("step_difference", "motif"):
+        e = g[name]
+        y = _gpu(cb, np.array(e["x"]).reshape(1, 1, 1, -1), np.array(e["k"]).reshape(1, 1, -1), None, mode=mode)
+        assert y.ravel().tolist() == e["output"], name
+    e = g["two_filters_with_bias"]
+    y = _gpu(cb, np.array(e["x"]).reshape(1, 1, 1, -1), np.array(e["filters"]).reshape(2, 1, 3), e["bias"], mode=mode)
+    assert y[0, :, 0, :].tolist() == e["output_per_filter"]
+    s = json.load(open(os.path.join(GOLDEN, "wxb_2d_examples.json")))
+    t = s["tiny_2d"]
+    y = _gpu(cb, np.array(t["image"]).reshape(1, 1, 3, 3), np.array(t["filter"]).reshape(1, 2, 2), None, mode=mode)
+    assert y[0, 0].tolist() == t["output"]
+    so = s["sobel"]
+    y = _gpu(cb, np.array(so["image"]).reshape(1, 1, 6, 6), np.stack([so["gx"], so["gy"]]), None, mode=mode)
+    assert y[0, 0].tolist() == so["gx_output"] and y[0, 1].tolist() == so["gy_output"]
+
+
+def test_ieee_closed_forms(cb):
+    # row-major tap order: products 1e8, -1e8, 1, 0 give 1 (column-major would give 0)
+    x = np.array([[1e8, -1e8], [1.0, 0.0]], np.float32).reshape(1, 1, 2, 2)
+    for mode in MODES:
+        assert _gpu(cb, x, np.ones((1, 2, 2)), None, mode=mode).ravel().tolist() == [1.0]
+    # exact rounds the product (tie to even) and cancels to +0; fast keeps 2**-24
+    a = np.float32(1 + 2.0 ** -12)
+    x = np.array([1 + 2.0 ** -11, a], np.float32).reshape(1, 1, 1, 2)
+    w = np.array([-1.0, a], np.float32).reshape(1, 1, 2)
+    assert _bits(_gpu(cb, x, w, None, mode=0)).ravel().tolist() == [0]
+    assert _gpu(cb, x, w, None, mode=1).ravel().tolist() == [2.0 ** -24]
+    # accumulator starts at +0: all products -0 give +0
+    for mode in MODES:
+        y = _gpu(cb, np.zeros((1, 1, 4, 4)), -np.ones((1, 3, 3)), None, pad=1, mode=mode)
+        assert np.all(_bits(y) == 0)
+    # denormal products are kept
+    for mode in MODES:
+        y = _gpu(cb, np.full((1, 1, 1, 1), 2.0 ** -70), np.full((1, 1, 1), 2.0 ** -70), None, mode=mode)
+        assert y.ravel()[0] == np.float32(2.0 ** -140)
+
+
+def test_padding_nan_rule(cb):
+    H = W = 5
+    x = np.full((1, 1, H, W), 2.0, np.float32)
+    w = np.ones((1, 3, 3), np.float32)
+    w[0, 0, 0] = np.inf
+    for bias in (None, np.array([0.5], np.float32)):
+        y = _gpu(cb, x, w, bias, pad=1, mode=0)[0, 0]
+        b = _bits(y)
+        for oy in range(H):
+            for ox in range(W):
+                if oy == 0 or ox == 0:
+                    assert b[oy, ox] == 0x7FC00000
+                else:
+                    assert y[oy, ox] == np.inf
+        yf = _gpu(cb, x, w, bias, pad=1, mode=1)[0, 0]
+        assert np.isnan(yf[0, 0]) and np.isnan(yf[3, 0]) and yf[2, 2] == np.inf
+    nan = struct.unpack("<f", struct.pack("<I", 0xFFC00001))[0]
+    x = np.ones((2, 3, 6, 7), np.float32)
+    x[1, 2, 3, 4] = nan
+    w = workloads.normal(5, 3 * 9, 1.0).reshape(3, 3, 3)
+    for mode in MODES:
+        y = _gpu(cb, x, w, np.zeros(3, np.float32), pad=1, mode=mode)
+        _compare(y, x, w, np.zeros(3, np.float32), 1, 1, 1, 1, mode)
+
+
+def _tiny(count, seed):
+    v = workloads.splitmix64(seed, count * 9)
+    out = []
+    for t in range(count):
+        z = [int(q) for q in v[9 * t: 9 * t + 9]]
+        N, C, m = 1 + z[0] % 3, 1 + z[1] % 5, 1 + z[2] % 3
+        KH, KW = 1 + z[3] % 5, 1 + (z[3] >> 8) % 5
+        s, p, d = 1 + z[4] % 3, z[5] % 3, 1 + z[6] % 2
+        H, W = 1 + z[7] % 23, 1 + (z[7] >> 8) % 23
+        if H + 2 * p < d * (KH - 1) + 1 or W + 2 * p < d * (KW - 1) + 1:
+            continue
+        out.append((N, C, m, H, W, KH, KW, s, p, d, z[8]))
+    return out
+
+
+@pytest.mark.parametrize("case", _tiny(40, 7), ids=lambda c: "_".join(map(str, c[:10])))
+def test_random_small_shapes(cb, case):
+    N, C, m, H, W, KH, KW, s, p, d, seed = case
+    x = workloads.uniform(seed, N * C * H * W, -1, 1).reshape(N, C, H, W)
+    w = workloads.normal(seed + 1, C * m * KH * KW, 1.0).reshape(C * m, KH, KW)
+    b = workloads.normal(seed + 2, C * m, 0.3) if seed % 2 else None
+    for mode in MODES:
+        _compare(_gpu(cb, x, w, b, s, p, d, mode), x, w, b, m, s, p, d, mode)
+
+
+@pytest.mark.parametrize("K,s,d,m", [(9, 1, 1, 1), (3, 9, 1, 2), (11, 2, 1, 1), (3, 3, 2, 3), (5, 1, 3, 2)])
+def test_many_taps_wide_stride_dilation(cb, K, s, d, m):
+    N, C, H, W = 2, 6, 37, 45
+    x = workloads.uniform(K * 100 + s, N * C * H * W, -1, 1).reshape(N, C, H, W)
+    w = workloads.normal(K + s, C * m * K * K, 1.0 / K).reshape(C * m, K, K)
+    b = workloads.normal(K, C * m, 0.3)
+    pad = (d * (K - 1)) // 2
+    for mode in MODES:
+        _compare(_gpu(cb, x, w, b, s, pad, d, mode), x, w, b, m, s, pad, d, mode)
+
+
+@pytest.mark.parametrize("tile", ["1,1,1", "1,3,7", "3,100,100", "64,1000,1000", "2,5,1000", "7,2,16"])
+def test_results_independent_of_tiling(cb, tile):
+    # the page's determinism property: each output has one order, so any job shape gives
+    # the same bits
+    case = workloads.DepthwiseCase("t", 3, 5, 2, 19, 23, 3, 5, 2, 2, 1, True, 3)
+    x, w, b = workloads.depthwise_inputs(case)
+    for mode in MODES:
+        base = _gpu(cb, x, w, b, case.stride, case.pad, case.dil, mode)
+        y = _gpu(cb, x, w, b, case.stride, case.pad, case.dil, mode, tile=tile)
+        assert np.array_equal(_bits(y), _bits(base))
+        _compare(y, x, w, b, case.mult, case.stride, case.pad, case.dil, mode)
