@@ -1,6 +1,7 @@
 """Benchmark: dense NHWC convolution (bf16, N=32, 56x56, 64->64, K=3) on B200, one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extras]
+                    [--workload NAME]
 
 A step is one forward dense convolution over one batch of 32 images (the hot path: tensor
 maps, TMA im2col gather, tcgen05 mainloop, epilogue) with inputs resident in HBM. Inputs and
@@ -17,6 +18,8 @@ workload (rank 0, N=1); and, unless --no-extras, the other configurations (point
 dense, the depthwise sweep in both modes) as secondary measurements.
 
 --impl reference times the CPU oracle itself on the same workload (rank 0 only).
+--workload selects another single configuration (for timing or profiling one kernel alone):
+"pointwise", "dense-large" or "dw-C<C>-K<K>-s<stride>-H<H>-exact|fast" from the depthwise sweep.
 """
 from __future__ import annotations
 
@@ -40,6 +43,20 @@ import workloads  # noqa: E402
 METRIC = "dense conv TFLOP/s (% bf16 TC peak); depthwise GB/s (% HBM) on 1 B200"
 L2_BYTES = 126 * 1024 * 1024
 CASE = workloads.DENSE_3X3
+
+
+def workload_table():
+    """Name -> (kind, case, mode). The default headline is the dense 3x3 configuration; the
+    others exist so any single kernel can be timed or profiled alone."""
+    t = {"dense3x3": ("dense", workloads.DENSE_3X3, None),
+         "pointwise": ("dense", workloads.DENSE_1X1, None),
+         "dense-large": ("dense", workloads.DENSE_LARGE, None)}
+    for c in workloads.DW_SWEEP:
+        for mode, name in ((0, "exact"), (1, "fast")):
+            t[f"dw-C{c.C}-K{c.KH}-s{c.stride}-H{c.H}-{name}"] = ("depthwise", c, mode)
+    return t
+
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -52,24 +69,28 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash() -> str:
+KERNEL_SOURCES = {"dense_tc_kernel": ("dense_tc.cuh", "ptx.cuh"), "depthwise_kernel": ("depthwise.cuh",)}
+
+
+def source_hash(kernel: str) -> str:
+    """Hash of the source files that define a kernel (its DRAM counters go stale with them)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "cnn_convolution_nhwc_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on these sources."""
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     rec = d.get(kernel, {}).get(workload)
-    if not rec or rec.get("source_hash") != source_hash():
+    if not rec or rec.get("source_hash") != source_hash(kernel):
         return None
     return rec.get("bytes_per_launch")
 
@@ -241,56 +262,71 @@ def time_graph_steps(singles, cycle, steps: int, warmup: int, dist=None, sampler
 # ------------------------------------------------------------------------------------------
 # Our arm
 # ------------------------------------------------------------------------------------------
-def dense_bench(cb, torch, case, X0, F0, steps, warmup, dist=None, sampler=None):
-    set_bytes = case.bytes
-    R = rotating_sets(set_bytes)
-    Xs = [X0.clone() for _ in range(R)]
-    Fs = [F0.clone() for _ in range(R)]
-    Ys = [torch.empty((case.N, case.Ho, case.Wo, case.Cout), dtype=X0.dtype, device=X0.device) for _ in range(R)]
-    fns = [(lambda i=i: cb.conv2d_nhwc_fwd(Xs[i], Fs[i], Ys[i])) for i in range(R)]
-    singles, cycle = capture(fns)
-    ms = time_graph_steps(singles, cycle, steps, warmup, dist, sampler)
-    del singles, cycle
-    return ms, R
-
-
-def depthwise_bench(cb, torch, case, mode, steps):
-    g = torch.Generator(device="cuda").manual_seed(case.seed)
-    co = case.C * case.mult
-    x0 = torch.rand((case.N, case.C, case.H, case.W), device="cuda", generator=g) * 2 - 1
-    w0 = torch.randn((co, case.KH, case.KW), device="cuda", generator=g) / math.sqrt(case.KH * case.KW)
-    b0 = torch.randn((co,), device="cuda", generator=g) * math.sqrt(0.1)
-    R = rotating_sets(case.bytes)
-    xs = [x0.clone() for _ in range(R)]
-    ys = [torch.empty((case.N, co, case.Ho, case.Wo), device="cuda") for _ in range(R)]
-    fns = [(lambda i=i: cb.depthwise_fwd(xs[i], w0, b0, ys[i], case.stride, case.pad, case.dil, mode))
-           for i in range(R)]
-    singles, cycle = capture(fns)
-    ms = time_graph_steps(singles, cycle, steps, max(3, steps // 10))
-    return ms / steps, R
-
-
-def dense_extra(cb, torch, case, steps):
-    g = torch.Generator(device="cuda").manual_seed(case.seed)
+def dense_device_inputs(torch, case, seed):
+    """Seeded bf16 X, F generated on the device (for the secondary measurements)."""
+    g = torch.Generator(device="cuda").manual_seed(seed)
     X = torch.randn((case.N, case.H, case.W, case.Cin), device="cuda", generator=g).to(torch.bfloat16)
     F = (torch.randn((case.K, case.K, case.Cin, case.Cout), device="cuda", generator=g)
          / math.sqrt(case.K * case.K * case.Cin)).to(torch.bfloat16)
-    ms, R = dense_bench(cb, torch, case, X, F, steps, max(3, steps // 10))
-    return ms / steps, R
+    return X, F
 
 
-def e2e_bench(cb, torch, case, Xh, Fh, steps, warmup):
+def dw_device_inputs(torch, case, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    co = case.C * case.mult
+    x = torch.rand((case.N, case.C, case.H, case.W), device="cuda", generator=g) * 2 - 1
+    w = torch.randn((co, case.KH, case.KW), device="cuda", generator=g) / math.sqrt(case.KH * case.KW)
+    b = torch.randn((co,), device="cuda", generator=g) * math.sqrt(0.1)
+    return x, w, b
+
+
+def steps_fns(cb, torch, kind, case, mode, inputs):
+    """R rotating buffer sets (total at least twice the L2) and one C-ABI call per set."""
+    R = rotating_sets(case.bytes)
+    if kind == "dense":
+        X0, F0 = inputs
+        Xs = [X0.clone() for _ in range(R)]
+        Fs = [F0.clone() for _ in range(R)]
+        Ys = [torch.empty((case.N, case.Ho, case.Wo, case.Cout), dtype=X0.dtype, device=X0.device)
+              for _ in range(R)]
+        fns = [(lambda i=i: cb.conv2d_nhwc_fwd(Xs[i], Fs[i], Ys[i])) for i in range(R)]
+        keep = (Xs, Fs, Ys)
+    else:
+        x0, w0, b0 = inputs
+        xs = [x0.clone() for _ in range(R)]
+        ys = [torch.empty((case.N, case.C * case.mult, case.Ho, case.Wo), device=x0.device) for _ in range(R)]
+        fns = [(lambda i=i: cb.depthwise_fwd(xs[i], w0, b0, ys[i], case.stride, case.pad, case.dil, mode))
+               for i in range(R)]
+        keep = (xs, ys)
+    return fns, R, keep
+
+
+def time_case(cb, torch, kind, case, mode, inputs, steps, warmup, dist=None, sampler=None):
+    fns, R, keep = steps_fns(cb, torch, kind, case, mode, inputs)
+    singles, cycle = capture(fns)
+    ms = time_graph_steps(singles, cycle, steps, warmup, dist, sampler)
+    del singles, cycle, keep
+    return ms, R
+
+
+def e2e_bench(cb, torch, kind, case, mode, host, steps, warmup):
     """Public API end to end: pinned host inputs -> device, convolution, output -> pinned host."""
-    X = torch.empty(Xh.shape, dtype=Xh.dtype, device="cuda")
-    F = torch.empty(Fh.shape, dtype=Fh.dtype, device="cuda")
-    Y = torch.empty((case.N, case.Ho, case.Wo, case.Cout), dtype=Xh.dtype, device="cuda")
-    Yh = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
+    dev = [torch.empty(h.shape, dtype=h.dtype, device="cuda") if h is not None else None for h in host]
+    if kind == "dense":
+        out = torch.empty((case.N, case.Ho, case.Wo, case.Cout), dtype=host[0].dtype, device="cuda")
+    else:
+        out = torch.empty((case.N, case.C * case.mult, case.Ho, case.Wo), device="cuda")
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
 
     def step():
-        X.copy_(Xh, non_blocking=True)
-        F.copy_(Fh, non_blocking=True)
-        cb.conv2d_nhwc_fwd(X, F, Y)
-        Yh.copy_(Y, non_blocking=True)
+        for d, h in zip(dev, host):
+            if h is not None:
+                d.copy_(h, non_blocking=True)
+        if kind == "dense":
+            cb.conv2d_nhwc_fwd(dev[0], dev[1], out)
+        else:
+            cb.depthwise_fwd(dev[0], dev[1], dev[2], out, case.stride, case.pad, case.dil, mode)
+        out_h.copy_(out, non_blocking=True)
 
     for _ in range(warmup):
         step()
@@ -303,143 +339,190 @@ def e2e_bench(cb, torch, case, Xh, Fh, steps, warmup):
     end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end) / steps
-    h2d = Xh.numel() * Xh.element_size() + Fh.numel() * Fh.element_size()
-    d2h = Yh.numel() * Yh.element_size()
+    h2d = sum(h.numel() * h.element_size() for h in host if h is not None)
+    d2h = out_h.numel() * out_h.element_size()
     return ms, h2d, d2h
 
 
-def cpu_baseline_dense(case, Xb, Fb, budget_s=12.0):
+def cpu_baseline(kind, case, mode, host_np, budget_s=12.0):
     """The oracle as it stands on this host: whole images until about budget_s of work."""
     import oracle
-    X = workloads.bf16_to_f32(Xb)
-    F = workloads.bf16_to_f32(Fb)
-    per_image = case.flops / case.N
-    done = 0
-    t0 = time.perf_counter()
+    done = 0.0
     n = 0
+    t0 = time.perf_counter()
     while n < case.N and (time.perf_counter() - t0) < budget_s:
-        oracle.conv2d_nhwc(X[n:n + 1], F)
-        done += per_image
+        if kind == "dense":
+            X, F = host_np
+            oracle.conv2d_nhwc(X[n:n + 1], F)
+            done += case.flops / case.N
+        else:
+            x, w, b = host_np
+            oracle.depthwise(x[n:n + 1], w, b, mult=case.mult, stride=case.stride, pad=case.pad, dil=case.dil,
+                             mode=mode)
+            done += case.bytes / case.N
         n += 1
     dt = time.perf_counter() - t0
-    return {"value": done / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{n} of {case.N} images of the workload, float64 seven-loop oracle, {dt:.1f} s"}
+    unit = "TFLOP/s" if kind == "dense" else "GB/s"
+    scale = 1e12 if kind == "dense" else 1e9
+    what = "float64 seven-loop oracle" if kind == "dense" else f"float32 per-output oracle, {'exact' if mode == 0 else 'fast'} mode"
+    return {"value": done / dt / scale, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} of {case.N} images of the workload, {what}, {dt:.1f} s"}
+
+
+def host_inputs(torch, kind, case, seed):
+    """Seeded host inputs from the workloads generators, as numpy (oracle view) and pinned torch."""
+    if kind == "dense":
+        c = workloads.DenseCase(case.name, case.N, case.H, case.W, case.Cin, case.Cout, case.K, "bf16", "normal", seed)
+        Xb, Fb = workloads.dense_inputs(c)
+        host = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (Xb, Fb)]
+        return (workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb)), host
+    c = workloads.DepthwiseCase(case.name, case.N, case.C, case.mult, case.H, case.W, case.KH, case.KW, case.stride,
+                                case.pad, case.dil, case.bias, seed)
+    x, w, b = workloads.depthwise_inputs(c)
+    host = [torch.from_numpy(a).pin_memory() for a in (x, w, b)]
+    return (x, w, b), host
 
 
 def run_ours(args, dist):
     import torch
     import cnn_convolution_nhwc_b200 as cb
 
+    kind, case, mode = workload_table()[args.workload]
     torch.cuda.set_device(dist.local_rank)
-    dev = torch.device("cuda", dist.local_rank)
     peaks, peaks_src = load_peaks()
-    case = workloads.DenseCase(CASE.name, CASE.N, CASE.H, CASE.W, CASE.Cin, CASE.Cout, CASE.K, "bf16",
-                               "normal", seed=dist.rank)
-    Xb, Fb = workloads.dense_inputs(case)
-    Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
-    Fh = torch.from_numpy(Fb.view(np.int16)).view(torch.bfloat16).pin_memory()
-    X0 = Xh.to(dev)
-    F0 = Fh.to(dev)
+    host_np, host = host_inputs(torch, kind, case, seed=dist.rank)
+    dev_inputs = tuple(h.to("cuda") for h in host)
 
     sampler = ClockSampler(dist.local_rank)
-    ms, R = dense_bench(cb, torch, case, X0, F0, args.steps, args.warmup, dist, sampler)
+    ms, R = time_case(cb, torch, kind, case, mode, dev_inputs, args.steps, args.warmup, dist, sampler)
     ms_step = ms / args.steps
-    value = dist.world * case.flops * args.steps / (ms * 1e-3) / 1e12
-    achieved = case.flops / (ms_step * 1e-3) / 1e12
     e2e_steps = max(10, min(200, args.steps // 10))
-    e2e_ms, h2d, d2h = e2e_bench(cb, torch, case, Xh, Fh, e2e_steps, 3)
+    e2e_ms, h2d, d2h = e2e_bench(cb, torch, kind, case, mode, host, e2e_steps, 3)
     e2e_ms = dist.max(e2e_ms)
-    e2e_value = dist.world * case.flops / (e2e_ms * 1e-3) / 1e12
     status = cb.conv_device_status()
 
+    if kind == "dense":
+        unit, work, scale = "TFLOP/s", case.flops, 1e12
+        kernel = "dense_tc_kernel"
+        achieved = case.flops / (ms_step * 1e-3) / 1e12
+        roof = {"kernel": kernel, "bound": "tensor", "achieved": round(achieved, 3), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": traffic_for(kernel, case.name), "algorithmic_bytes": case.bytes,
+                "algorithmic_flops": case.flops,
+                "hbm_frac": round(case.bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peaks_src}: bf16 burst (kernel timed alone); HBM copy {peaks['hbm_gbs']} GB/s"}
+        dtype = "bf16"
+        data = "synthetic (seeded SplitMix64 / Box-Muller: X~N(0,1), F~N(0,1/(K*K*Cin)), rounded to bf16)"
+        cfg = {"workload": case.name, "N_per_gpu": case.N, "H": case.H, "W": case.W, "Cin": case.Cin,
+               "Cout": case.Cout, "K": case.K, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
+    else:
+        unit, work, scale = "GB/s", case.bytes, 1e9
+        kernel = "depthwise_kernel"
+        achieved = case.bytes / (ms_step * 1e-3) / 1e9
+        roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic_for(kernel, args.workload), "algorithmic_bytes": case.bytes,
+                "GFLOP/s": round(case.flops / (ms_step * 1e-3) / 1e9, 1),
+                "peak_source": f"{peaks_src}: HBM copy"}
+        dtype = "f32"
+        data = "synthetic (seeded SplitMix64 / Box-Muller: x~U(-1,1), w~N(0,1/K^2), bias~N(0,0.1))"
+        cfg = {"workload": case.name + (" exact" if mode == 0 else " fast"), "N_per_gpu": case.N, "C": case.C,
+               "mult": case.mult, "H": case.H, "W": case.W, "K": case.KH, "stride": case.stride, "pad": case.pad,
+               "dil": case.dil, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
+    cfg.update({"l2": f"inputs larger than L2: {R} rotating buffer sets of {case.bytes / 1e6:.2f} MB",
+                "launch": "CUDA graph replay of the C-ABI call", "parallelism": f"replicas x{dist.world}"})
+    value = dist.world * work * args.steps / (ms * 1e-3) / scale
+    e2e_value = dist.world * work / (e2e_ms * 1e-3) / scale
     line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": dist.world,
+        "metric": METRIC, "value": round(value, 4), "unit": unit, "n_gpus": dist.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded SplitMix64 / Box-Muller: X~N(0,1), F~N(0,1/(K*K*Cin)), rounded to bf16)",
-        "config": {"workload": CASE.name, "N_per_gpu": case.N, "H": case.H, "W": case.W, "Cin": case.Cin,
-                   "Cout": case.Cout, "K": case.K, "flop_per_step": case.flops, "bytes_per_step": case.bytes,
-                   "l2": f"inputs larger than L2: {R} rotating X/F/Y sets of {case.bytes / 1e6:.2f} MB",
-                   "launch": "CUDA graph replay of the C-ABI call", "parallelism": f"replicas x{dist.world}"},
-        "roofline": {"kernel": "dense_tc_kernel (BN=64)", "bound": "tensor", "achieved": round(achieved, 3),
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                     "traffic": traffic_for("dense_tc_kernel", CASE.name),
-                     "algorithmic_bytes": case.bytes,
-                     "hbm_frac": round(case.bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                     "peak_source": f"{peaks_src} (bf16 burst; HBM copy {peaks['hbm_gbs']} GB/s)"},
-        "e2e": {"value": round(e2e_value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms, 4), "path": "python binding -> C ABI, pinned host copies in the timed region"},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": data,
+        "config": cfg, "roofline": roof,
+        "e2e": {"value": round(e2e_value, 4), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4),
+                "path": "python binding -> C ABI, pinned host copies in the timed region"},
         "gpu_launches": args.steps,
         "clocks": sampler.summary(),
         "device_status": cb.conv_status_string(status),
     }
     if dist.world == 1 and not args.no_extras:
-        line["extras"] = extras(cb, torch, peaks)
+        line["extras"] = extras(cb, torch, peaks, skip=args.workload)
     if dist.rank == 0 and dist.world == 1:
-        line["cpu_baseline"] = cpu_baseline_dense(case, Xb, Fb)
+        line["cpu_baseline"] = cpu_baseline(kind, case, mode, host_np)
     return line
 
 
-def extras(cb, torch, peaks):
+def extras(cb, torch, peaks, skip):
     out = {"dense": [], "depthwise": []}
-    for case in (workloads.DENSE_1X1, workloads.DENSE_LARGE):
-        steps = 200 if case.flops < 1e11 else 40
-        ms, R = dense_extra(cb, torch, case, steps)
-        tf = case.flops / (ms * 1e-3) / 1e12
-        out["dense"].append({"workload": case.name, "ms": round(ms, 5), "TFLOP/s": round(tf, 2),
-                             "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
-                             "GB/s": round(case.bytes / (ms * 1e-3) / 1e9, 1),
-                             "frac_hbm": round(case.bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                             "rotating_sets": R})
-    for case in workloads.DW_SWEEP:
-        for mode, name in ((0, "exact"), (1, "fast")):
-            ms, R = depthwise_bench(cb, torch, case, mode, 200)
+    for name, (kind, case, mode) in workload_table().items():
+        if name == skip:
+            continue
+        if kind == "dense":
+            steps = 200 if case.flops < 1e11 else 40
+            ms, R = time_case(cb, torch, kind, case, mode, dense_device_inputs(torch, case, 0), steps, 5)
+            ms /= steps
+            tf = case.flops / (ms * 1e-3) / 1e12
+            out["dense"].append({"workload": name, "ms": round(ms, 5), "TFLOP/s": round(tf, 2),
+                                 "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+                                 "GB/s": round(case.bytes / (ms * 1e-3) / 1e9, 1),
+                                 "frac_hbm": round(case.bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                 "rotating_sets": R})
+        else:
+            ms, R = time_case(cb, torch, kind, case, mode, dw_device_inputs(torch, case, 0), 200, 20)
+            ms /= 200
             gbs = case.bytes / (ms * 1e-3) / 1e9
-            out["depthwise"].append({"workload": case.name, "mode": name, "ms": round(ms, 5),
-                                     "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            out["depthwise"].append({"workload": name, "ms": round(ms, 5), "GB/s": round(gbs, 1),
+                                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
                                      "GFLOP/s": round(case.flops / (ms * 1e-3) / 1e9, 1), "rotating_sets": R})
     return out
 
 
 # ------------------------------------------------------------------------------------------
-# Reference arm: the CPU oracle
+# Reference arm: the CPU oracle, as it stands, on the host cores
 # ------------------------------------------------------------------------------------------
 def run_reference(args, dist):
     import oracle
-    case = CASE
-    Xb, Fb = workloads.dense_inputs(case)
-    X = workloads.bf16_to_f32(Xb)
-    F = workloads.bf16_to_f32(Fb)
-    total = case.N * case.Ho * case.Wo * case.Cout
-    flop_per_out = 2 * case.K * case.K * case.Cin
-    # calibrate: points per second of the oracle's per-output routine
+    kind, case, mode = workload_table()[args.workload]
+    if kind == "dense":
+        Xb, Fb = workloads.dense_inputs(case)
+        X, F = workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb)
+        total = case.N * case.Ho * case.Wo * case.Cout
+        work_per_out, unit, scale = 2 * case.K * case.K * case.Cin, "TFLOP/s", 1e12
+
+        def run(idx):
+            oracle.conv2d_nhwc_points(X, F, idx)
+    else:
+        x, w, b = workloads.depthwise_inputs(case)
+        total = case.N * case.C * case.mult * case.Ho * case.Wo
+        work_per_out, unit, scale = case.bytes / total, "GB/s", 1e9
+
+        def run(idx):
+            oracle.depthwise_points(x, w, b, idx, mult=case.mult, stride=case.stride, pad=case.pad, dil=case.dil,
+                                    mode=mode)
     idx = (workloads.splitmix64(1, 4096) % np.uint64(total)).astype(np.int64)
     t0 = time.perf_counter()
-    oracle.conv2d_nhwc_points(X, F, idx)
+    run(idx)
     rate = 4096 / max(1e-6, time.perf_counter() - t0)
     per_step = int(min(total, max(64, rate * 90.0 / max(1, args.steps + args.warmup))))
-    samples = [(workloads.splitmix64(100 + s, per_step) % np.uint64(total)).astype(np.int64)
-               for s in range(min(8, args.steps + args.warmup))]
+    samples = [(workloads.splitmix64(100 + s, per_step) % np.uint64(total)).astype(np.int64) for s in range(8)]
     for s in range(args.warmup):
-        oracle.conv2d_nhwc_points(X, F, samples[s % len(samples)])
+        run(samples[s % 8])
     t0 = time.perf_counter()
     for s in range(args.steps):
-        oracle.conv2d_nhwc_points(X, F, samples[s % len(samples)])
+        run(samples[s % 8])
     dt = time.perf_counter() - t0
-    ms = dt * 1e3 / args.steps
-    value = per_step * flop_per_out / (dt / args.steps) / 1e12
-    cores = oracle.num_threads()
-    sample = (f"{per_step} sampled outputs of the workload per step (of {total}), float64 oracle, "
-              f"OpenMP over outputs")
+    value = per_step * work_per_out / (dt / args.steps) / scale
+    sample = f"{per_step} sampled outputs of the workload per step (of {total}), oracle per-output routine"
     return {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": dist.world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the GPU arm)",
-        "config": {"workload": case.name, "N_per_gpu": case.N, "H": case.H, "W": case.W, "Cin": case.Cin,
-                   "Cout": case.Cout, "K": case.K},
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64" if kind == "dense" else "f32",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": case.name if kind == "dense" else args.workload},
         "impl": "reference",
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
@@ -449,6 +532,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50000)
     ap.add_argument("--warmup", type=int, default=500)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dense3x3", choices=sorted(workload_table()))
     ap.add_argument("--no-extras", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -216,47 +216,72 @@ long long dw_out(long long in, int k, int s, int pad, int dil) {
     return (in + 2LL * pad - (1LL * dil * (k - 1) + 1)) / s + 1;
 }
 
-int dw_smem_bytes(const DwParams &p) {
-    return 4 * p.P * (p.w_stride + p.rows_in * p.cols_in);
+// Compile-time specialisations: (KW, stride) with unit dilation, 4 outputs per thread.
+enum DwSpec { kDwGeneric = 0, kDwK3S1, kDwK3S2, kDwK5S1, kDwK5S2 };
+
+DwSpec dw_spec(const DwParams &p) {
+    if (p.dil != 1) return kDwGeneric;
+    if (p.KW == 3 && p.stride == 1) return kDwK3S1;
+    if (p.KW == 3 && p.stride == 2) return kDwK3S2;
+    if (p.KW == 5 && p.stride == 1) return kDwK5S1;
+    if (p.KW == 5 && p.stride == 2) return kDwK5S2;
+    return kDwGeneric;
 }
 
-void dw_set_window(DwParams &p) {
+int dw_vx(DwSpec s) { return s == kDwGeneric ? 1 : 4; }
+
+long long dw_smem_bytes(const DwParams &p) {
+    return 4LL * p.P * (p.w_stride + 1LL * p.rows_in * p.pitch);
+}
+
+// Staged window and shared-memory pitch for the current job shape. The pitch also covers
+// the 128-bit window reads of the last strip of a row in the specialised kernels.
+void dw_set_window(DwParams &p, DwSpec s) {
     p.rows_in = (p.R - 1) * p.stride + (p.KH - 1) * p.dil + 1;
     p.cols_in = (p.CW - 1) * p.stride + (p.KW - 1) * p.dil + 1;
+    int need = p.cols_in;
+    if (s != kDwGeneric) {
+        const int vx = dw_vx(s);
+        const int strips = (p.CW + vx - 1) / vx;
+        const int win = (vx - 1) * p.stride + p.KW;
+        const int reach = (strips - 1) * vx * p.stride + ((win + 3) / 4) * 4;
+        if (reach > need) need = reach;
+    }
+    p.pitch = (need + 3) & ~3;
 }
 
-// Job shape: about 2048 outputs per CTA, whole planes grouped when they are small, and a
-// staged window that fits in kDwSmemLimit.
-void dw_choose_tiles(DwParams &p) {
+// Job shape: about 2048 outputs per CTA, whole small planes grouped, column bands a
+// multiple of the strip width, and a staged window within kDwSmemLimit.
+void dw_choose_tiles(DwParams &p, DwSpec s) {
     constexpr int kTarget = 2048;
-    p.CW = p.Wo < 128 ? p.Wo : 128;
+    const int vx = dw_vx(s);
+    p.CW = p.Wo <= 128 ? p.Wo : 128;
     p.R = kTarget / p.CW;
     if (p.R < 1) p.R = 1;
     if (p.R > p.Ho) p.R = p.Ho;
     p.P = 1;
     if (p.R == p.Ho && p.CW == p.Wo) {
-        long long per = 1LL * p.Ho * p.Wo;
-        long long P = kTarget / per;
+        long long P = kTarget / (1LL * p.Ho * p.Wo);
         if (P < 1) P = 1;
         if (P > 64) P = 64;
         if (P > p.num_planes) P = p.num_planes;
         p.P = static_cast<int>(P);
     }
-    dw_set_window(p);
+    dw_set_window(p, s);
     while (dw_smem_bytes(p) > kDwSmemLimit) {
         if (p.P > 1) p.P = (p.P + 1) / 2;
         else if (p.R > 1) p.R = (p.R + 1) / 2;
-        else if (p.CW > 1) p.CW = (p.CW + 1) / 2;
+        else if (p.CW > vx) p.CW = ((p.CW / 2 + vx - 1) / vx) * vx;
         else break;
-        dw_set_window(p);
+        dw_set_window(p, s);
     }
 }
 
-template <int MODE, bool HB>
-int launch_dw(const float *x, const float *w, const float *bias, float *y, const DwParams &p,
-              long long jobs, cudaStream_t stream, DeviceState *d, unsigned bit) {
-    auto kern = depthwise_kernel<MODE, HB>;
-    const int smem = dw_smem_bytes(p);
+template <int MODE, bool HB, int KW, int S, int VX>
+int launch_dw_one(const float *x, const float *w, const float *bias, float *y, const DwParams &p, long long jobs,
+                  cudaStream_t stream, DeviceState *d, unsigned bit) {
+    auto kern = depthwise_kernel<MODE, HB, KW, S, VX>;
+    const int smem = static_cast<int>(dw_smem_bytes(p));
     if (smem > 48 * 1024)
         if (int rc = ensure_smem_attr(d, bit, kern, 227 * 1024)) return rc;
     cudaLaunchConfig_t cfg = {};
@@ -265,6 +290,20 @@ int launch_dw(const float *x, const float *w, const float *bias, float *y, const
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     return cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p) == cudaSuccess ? CONV_OK : CONV_ERR_CUDA;
+}
+
+template <int MODE, bool HB>
+int launch_dw(const float *x, const float *w, const float *bias, float *y, const DwParams &p, DwSpec s,
+              long long jobs, cudaStream_t stream, DeviceState *d) {
+    // attribute bits 8..27: one per instantiation
+    const unsigned base = 8u + 5u * (2u * MODE + (HB ? 1u : 0u));
+    switch (s) {
+        case kDwK3S1: return launch_dw_one<MODE, HB, 3, 1, 4>(x, w, bias, y, p, jobs, stream, d, base + 1);
+        case kDwK3S2: return launch_dw_one<MODE, HB, 3, 2, 4>(x, w, bias, y, p, jobs, stream, d, base + 2);
+        case kDwK5S1: return launch_dw_one<MODE, HB, 5, 1, 4>(x, w, bias, y, p, jobs, stream, d, base + 3);
+        case kDwK5S2: return launch_dw_one<MODE, HB, 5, 2, 4>(x, w, bias, y, p, jobs, stream, d, base + 4);
+        default: return launch_dw_one<MODE, HB, 0, 0, 1>(x, w, bias, y, p, jobs, stream, d, base);
+    }
 }
 
 }  // namespace
@@ -332,16 +371,21 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
     DwParams p;
     p.Cin = Cin; p.mult = mult; p.Cout = static_cast<int>(Cout); p.H = H; p.W = W; p.KH = KH; p.KW = KW;
     p.stride = stride; p.pad = pad; p.dil = dil; p.Ho = static_cast<int>(Ho); p.Wo = static_cast<int>(Wo);
-    p.num_planes = 1LL * N * Cout;
+    p.num_planes = static_cast<int>(1LL * N * Cout);
     p.w_stride = (KH * KW + 3) & ~3;
-    dw_choose_tiles(p);
+    DwSpec spec = dw_spec(p);
+    if (const char *g = env("CONV_B200_DW_GENERIC"))   // force the runtime-shape kernel (tests)
+        if (g[0] == '1') spec = kDwGeneric;
+    dw_choose_tiles(p, spec);
     if (const char *t = env("CONV_B200_DW_TILE")) {   // "P,R,CW": a forced job shape (tests)
         int P = 0, R = 0, CW = 0;
         if (std::sscanf(t, "%d,%d,%d", &P, &R, &CW) == 3 && P >= 1 && R >= 1 && CW >= 1) {
+            const int vx = dw_vx(spec);
             p.R = R < p.Ho ? R : p.Ho;
-            p.CW = CW < p.Wo ? CW : p.Wo;
-            p.P = (p.R == p.Ho && p.CW == p.Wo) ? static_cast<int>(P < p.num_planes ? P : p.num_planes) : 1;
-            dw_set_window(p);
+            p.CW = CW < p.Wo ? ((CW + vx - 1) / vx) * vx : p.Wo;
+            if (p.CW > p.Wo) p.CW = p.Wo;
+            p.P = (p.R == p.Ho && p.CW == p.Wo) ? (P < p.num_planes ? P : p.num_planes) : 1;
+            dw_set_window(p, spec);
         }
     }
     if (dw_smem_bytes(p) > 227 * 1024) return CONV_ERR_UNSUPPORTED;
@@ -352,10 +396,10 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
     if (jobs > kInt32Max) return CONV_ERR_UNSUPPORTED;
     const bool hb = bias != nullptr;
     if (mode == DW_EXACT)
-        return hb ? launch_dw<0, true>(x, w, bias, y, p, jobs, stream, d, 8)
-                  : launch_dw<0, false>(x, w, bias, y, p, jobs, stream, d, 9);
-    return hb ? launch_dw<1, true>(x, w, bias, y, p, jobs, stream, d, 10)
-              : launch_dw<1, false>(x, w, bias, y, p, jobs, stream, d, 11);
+        return hb ? launch_dw<0, true>(x, w, bias, y, p, spec, jobs, stream, d)
+                  : launch_dw<0, false>(x, w, bias, y, p, spec, jobs, stream, d);
+    return hb ? launch_dw<1, true>(x, w, bias, y, p, spec, jobs, stream, d)
+              : launch_dw<1, false>(x, w, bias, y, p, spec, jobs, stream, d);
 }
 
 const char *conv_status_string(int status) {
