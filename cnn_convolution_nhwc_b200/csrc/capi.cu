@@ -17,6 +17,7 @@
 #include "../../include/conv_b200.h"
 #include "dense_direct.cuh"
 #include "dense_tc.cuh"
+#include "dense_halo.cuh"
 #include "depthwise.cuh"
 #include "ptx.cuh"
 
@@ -203,6 +204,139 @@ int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, 
                                                                                       : CONV_ERR_CUDA;
 }
 
+// ---- halo kernel ------------------------------------------------------------------------
+constexpr int kSmemLimit = 232448;   // 227 KB of dynamic shared memory per CTA
+
+struct HaloPlan {
+    bool ok = false;
+    int bn = 0;
+    bool bres = false;
+    DenseHaloParams p{};
+    int smem = 0;
+    int grid = 0;
+};
+
+template <int BN, bool BRES>
+int halo_fixed_bytes() { return DenseHaloCfg<BN, BRES>::FIXED_BYTES; }
+
+// Picks tile width, filter residency and ring depths so that everything fits in shared
+// memory; returns !ok when even one halo slot does not fit (the im2col kernel then runs).
+HaloPlan plan_halo(int N, int H, int W, int Cin, int Cout, int K, int num_sms, int force_bn) {
+    HaloPlan pl;
+    const long long rows = 1LL * N * H * W;
+    if (rows + 1024 > kInt32Max) return pl;
+    const int need = 128 + (K - 1) * W + (K - 1);
+    if (need > 4096) return pl;
+    const int n_boxes = (need + 255) / 256;
+    const int box_rows = (((need + n_boxes - 1) / n_boxes) + 7) & ~7;
+    const int halo_rows = n_boxes * box_rows;
+    const int halo_bytes = halo_rows * 128;
+    const int num_cblk = (Cin + 63) / 64;
+    const int num_kblk = K * K * num_cblk;
+    int bn = Cout <= 64 ? 64 : (Cout <= 128 ? 128 : 256);
+    if (force_bn) bn = force_bn;
+    const int b_bytes = 64 * bn * 2;
+    const int fixed = bn == 64 ? halo_fixed_bytes<64, true>() : (bn == 128 ? halo_fixed_bytes<128, true>()
+                                                                            : halo_fixed_bytes<256, true>());
+    const int num_mtiles = static_cast<int>((rows + 127) / 128);
+    const int num_ntiles = (Cout + bn - 1) / bn;
+    DenseHaloParams &p = pl.p;
+    // resident filter: the CTA's whole N-tile slice, loaded once
+    const long long b_res = 1LL * num_kblk * b_bytes;
+    if (b_res <= 128 * 1024 && num_ntiles <= num_sms && fixed + b_res + 2LL * halo_bytes <= kSmemLimit) {
+        pl.bres = true;
+        p.b_region = static_cast<int>(b_res);
+        p.HS = static_cast<int>((kSmemLimit - fixed - b_res) / halo_bytes);
+        p.BS = 1;
+    } else {
+        pl.bres = false;
+        for (int bs : {4, 3, 2}) {
+            const long long avail = kSmemLimit - fixed - 1LL * bs * b_bytes;
+            if (avail >= 2LL * halo_bytes || (bs == 2 && avail >= halo_bytes)) {
+                p.BS = bs;
+                p.b_region = bs * b_bytes;
+                p.HS = static_cast<int>(avail / halo_bytes);
+                break;
+            }
+        }
+        if (p.BS == 0) return pl;
+    }
+    if (p.HS > DenseHaloCfg<64, true>::MAX_RING) p.HS = DenseHaloCfg<64, true>::MAX_RING;
+    if (p.HS < 1) return pl;
+    p.rows = static_cast<int>(rows);
+    p.H = H; p.W = W; p.Ho = H - K + 1; p.Wo = W - K + 1;
+    p.K = K; p.KK = K * K; p.Cout = Cout;
+    p.num_cblk = num_cblk;
+    p.num_kblk = num_kblk;
+    p.halo_rows = halo_rows;
+    p.box_rows = box_rows;
+    p.n_boxes = n_boxes;
+    p.halo_bytes = halo_bytes;
+    p.num_mtiles = num_mtiles;
+    p.num_ntiles = num_ntiles;
+    p.num_tiles = num_mtiles * num_ntiles;
+    if (pl.bres && num_ntiles > 1) {
+        p.n_fixed = 1;
+        int per_n = num_sms / num_ntiles;
+        if (per_n > num_mtiles) per_n = num_mtiles;
+        pl.grid = per_n * num_ntiles;
+    } else {
+        p.n_fixed = 0;
+        pl.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    }
+    pl.smem = fixed + p.b_region + p.HS * halo_bytes;
+    pl.bn = bn;
+    pl.ok = pl.smem <= kSmemLimit && pl.grid >= 1;
+    return pl;
+}
+
+template <class Cfg>
+int launch_dense_halo(const void *X, const void *F, void *Y, int Cin, int Cout, int K, const HaloPlan &pl,
+                      cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
+    alignas(64) CUtensorMap tmX, tmF;
+    {   // X as a 2-D matrix: rows = flattened (n, y, x), Cin channels per row
+        const cuuint64_t dims[2] = {(cuuint64_t)Cin, (cuuint64_t)pl.p.rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)Cin * 2};
+        const cuuint32_t box[2] = {64, (cuuint32_t)pl.p.box_rows};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode_tiled(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    {   // F: 3-D {Cout, Cin, K*K}; a box is 64 reduction rows (channels) x 64 output channels
+        const cuuint64_t dims[3] = {(cuuint64_t)Cout, (cuuint64_t)Cin, (cuuint64_t)K * K};
+        const cuuint64_t strides[2] = {(cuuint64_t)Cout * 2, (cuuint64_t)Cin * Cout * 2};
+        const cuuint32_t box[3] = {64, 64, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(F), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    auto kern = dense_halo_kernel<Cfg>;
+    if (int rc = ensure_smem_attr(d, attr_bit, kern, kSmemLimit)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status) == cudaSuccess
+               ? CONV_OK
+               : CONV_ERR_CUDA;
+}
+
+int dispatch_halo(const void *X, const void *F, void *Y, int Cin, int Cout, int K, const HaloPlan &pl,
+                  cudaStream_t stream, DeviceState *d) {
+    // shared-memory attribute bits 3..8
+    if (pl.bn == 64) return pl.bres ? launch_dense_halo<DenseHaloCfg<64, true>>(X, F, Y, Cin, Cout, K, pl, stream, d, 3)
+                                    : launch_dense_halo<DenseHaloCfg<64, false>>(X, F, Y, Cin, Cout, K, pl, stream, d, 4);
+    if (pl.bn == 128) return pl.bres ? launch_dense_halo<DenseHaloCfg<128, true>>(X, F, Y, Cin, Cout, K, pl, stream, d, 5)
+                                     : launch_dense_halo<DenseHaloCfg<128, false>>(X, F, Y, Cin, Cout, K, pl, stream, d, 6);
+    return pl.bres ? launch_dense_halo<DenseHaloCfg<256, true>>(X, F, Y, Cin, Cout, K, pl, stream, d, 7)
+                   : launch_dense_halo<DenseHaloCfg<256, false>>(X, F, Y, Cin, Cout, K, pl, stream, d, 28);
+}
+
 using CfgBN64 = DenseTcCfg<64, 6>;
 using CfgBN128 = DenseTcCfg<128, 5>;
 using CfgBN256 = DenseTcCfg<256, 3>;
@@ -231,7 +365,7 @@ DwSpec dw_spec(const DwParams &p) {
 int dw_vx(DwSpec s) { return s == kDwGeneric ? 1 : 4; }
 
 long long dw_smem_bytes(const DwParams &p) {
-    return 4LL * p.P * (p.w_stride + 1LL * p.rows_in * p.pitch);
+    return 4LL * (dw_smem_head_floats(p.P, p.w_stride) + 1LL * p.P * p.rows_in * p.pitch);
 }
 
 // Staged window and shared-memory pitch for the current job shape. The pitch also covers
@@ -248,6 +382,9 @@ void dw_set_window(DwParams &p, DwSpec s) {
         if (reach > need) need = reach;
     }
     p.pitch = (need + 3) & ~3;
+    int lg = 0;
+    while ((1 << lg) < p.cols_in && lg < 8) ++lg;
+    p.tc_log2 = lg;
 }
 
 // Job shape: about 2048 outputs per CTA, whole small planes grouped, column bands a
@@ -319,20 +456,36 @@ int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, 
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
     const char *force = env("CONV_B200_DENSE");
-    const bool tc_ok = (Cin % 8 == 0) && (Cout % 8 == 0) && K <= 128 && aligned(X, 16) && aligned(F, 16) &&
-                       aligned(Y, 16) && 2LL * N * H * W * Cin >= 128 * 1024;
-    if (force && std::strcmp(force, "direct") == 0)
+    // Tensor-core paths need 16-byte rows (Cin, Cout multiples of 8) and 16-byte aligned
+    // tensors. The im2col tensor map is used only for inputs of at least 128 KiB.
+    const bool tc_shape = (Cin % 8 == 0) && (Cout % 8 == 0) && aligned(X, 16) && aligned(F, 16) && aligned(Y, 16);
+    const bool im2col_ok = tc_shape && K <= 128 && 2LL * N * H * W * Cin >= 128 * 1024;
+    if ((force && std::strcmp(force, "direct") == 0) || !tc_shape)
         return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
                                    static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d);
-    if (!tc_ok) {
-        if (force && std::strncmp(force, "bn", 2) == 0) return CONV_ERR_UNSUPPORTED;
+    // Default: the halo kernel; the im2col kernel when a halo does not fit in shared memory
+    // (very wide images) or when forced. CONV_B200_DENSE (tests): "direct", "halo",
+    // "halo64/128/256" (halo kernel with that tile width), "bn64/128/256" (im2col kernel).
+    int force_bn = 0;
+    bool force_im2col = false, force_halo = false;
+    if (force) {
+        if (std::strncmp(force, "halo", 4) == 0) { force_halo = true; force_bn = std::atoi(force + 4); }
+        if (std::strncmp(force, "bn", 2) == 0) { force_im2col = true; force_bn = std::atoi(force + 2); }
+    }
+    if (force_bn != 0 && force_bn != 64 && force_bn != 128 && force_bn != 256) return CONV_ERR_INVALID_ARG;
+    if (!force_im2col) {
+        // By default the halo kernel runs when the filter stays resident in shared memory;
+        // with a streamed filter the im2col kernel measured faster (deeper operand ring).
+        const HaloPlan pl = plan_halo(N, H, W, Cin, Cout, K, d->num_sms, force_bn);
+        if (pl.ok && (pl.bres || force_halo || !im2col_ok)) return dispatch_halo(X, F, Y, Cin, Cout, K, pl, stream, d);
+        if (force_halo) return CONV_ERR_UNSUPPORTED;
+    }
+    if (!im2col_ok) {
+        if (force_im2col) return CONV_ERR_UNSUPPORTED;
         return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
                                    static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d);
     }
-    int bn = Cout <= 64 ? 64 : 128;
-    if (force && std::strcmp(force, "bn64") == 0) bn = 64;
-    if (force && std::strcmp(force, "bn128") == 0) bn = 128;
-    if (force && std::strcmp(force, "bn256") == 0) bn = 256;
+    int bn = force_bn ? force_bn : (Cout <= 64 ? 64 : 128);
     if (bn == 64) return launch_dense_tc<CfgBN64>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 0);
     if (bn == 128) return launch_dense_tc<CfgBN128>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 1);
     return launch_dense_tc<CfgBN256>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 2);
@@ -394,6 +547,12 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
     const long long groups = (p.num_planes + p.P - 1) / p.P;
     const long long jobs = groups * p.n_rbands * p.n_cbands;
     if (jobs > kInt32Max) return CONV_ERR_UNSUPPORTED;
+    p.vec_store = (p.Wo % 4 == 0 && aligned(y, 16)) ? 1 : 0;
+    p.div_cout = make_fastdiv(static_cast<uint32_t>(p.Cout));
+    p.div_mult = make_fastdiv(static_cast<uint32_t>(p.mult));
+    p.div_taps = make_fastdiv(static_cast<uint32_t>(KH * KW));
+    p.div_cbands = make_fastdiv(static_cast<uint32_t>(p.n_cbands));
+    p.div_rbands = make_fastdiv(static_cast<uint32_t>(p.n_rbands));
     const bool hb = bias != nullptr;
     if (mode == DW_EXACT)
         return hb ? launch_dw<0, true>(x, w, bias, y, p, spec, jobs, stream, d)

@@ -11,10 +11,11 @@
 // consumed from shared memory by tcgen05 MMAs. The reduction runs tap by tap, which is the
 // sum of K*K shifted-slice channel matmuls of section 2.
 //
-// Roles inside one persistent CTA of 6 warps:
-//   warp 0      one thread issues TMA loads into a STAGES-deep ring of (A, B) slots;
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) into one
-//               of two TMEM accumulators, and tcgen05.commit to free ring slots;
+// Roles inside one persistent CTA of 6 warps (each role loop is walked by whole, converged
+// warps; a single lane issues the asynchronous instructions):
+//   warp 0      TMA loads into a STAGES-deep ring of (A, B) slots;
+//   warp 1      allocates TMEM; issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM
+//               accumulators, and tcgen05.commit to free ring slots;
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads TMEM lanes
 //               32*(w%4) .. +31), round to bf16, 128-byte-swizzled staging in shared
 //               memory, TMA store to Y. The two accumulators let tile t+1's MMAs run
@@ -134,26 +135,28 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 
     if (warp == 0) {
         // ------------------------------- TMA producer -------------------------------
-        if (lane == 0) {
-            uint32_t it = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
-                const int mt = tile / p.num_ntiles;
-                const int nt = tile - mt * p.num_ntiles;
-                const int m0 = mt * Cfg::BM;
-                const int n0 = nt * BN;
-                const int img = m0 / p.HoWo;
-                const int rem = m0 - img * p.HoWo;
-                const int oy = rem / p.Wo;
-                const int ox = rem - oy * p.Wo;
-                bool ok = true;
-                for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
-                    const int tap = kb / p.num_cblk;
-                    const int cb = kb - tap * p.num_cblk;
-                    const int ky = tap / p.K;
-                    const int kx = tap - ky * p.K;
-                    const uint32_t s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1u;
-                    if (!mbar_wait(empty_bar(s), ph ^ 1u)) { fail(); ok = false; break; }
+        // The whole warp walks the loop (it stays converged); lane 0 issues.
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
+            const int mt = tile / p.num_ntiles;
+            const int nt = tile - mt * p.num_ntiles;
+            const int m0 = mt * Cfg::BM;
+            const int n0 = nt * BN;
+            const int img = m0 / p.HoWo;
+            const int rem = m0 - img * p.HoWo;
+            const int oy = rem / p.Wo;
+            const int ox = rem - oy * p.Wo;
+            bool ok = true;
+            int tap = 0, cb = 0, ky = 0, kx = 0;
+            for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
+                const uint32_t s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1u;
+                if (!mbar_wait_warp(empty_bar(s), ph ^ 1u)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
                     mbar_arrive_expect_tx(full_bar(s), Cfg::STAGE_BYTES);
                     tma_load_im2col_4d(sA + s * Cfg::A_BYTES, &tmX, full_bar(s), cb * 64, ox, oy, img,
                                        static_cast<uint16_t>(kx), static_cast<uint16_t>(ky));
@@ -162,29 +165,47 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         tma_load_3d(sB + s * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, &tmF, full_bar(s),
                                     n0 + h * 64, cb * 64, tap);
                 }
-                if (!ok) break;
+                __syncwarp();
+                // next (tap, channel block) in (i, j, c) order
+                if (++cb == p.num_cblk) {
+                    cb = 0;
+                    ++tap;
+                    if (++kx == p.K) { kx = 0; ++ky; }
+                }
             }
-            // Drain: every load issued has landed before the CTA may exit.
-            const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
-            for (uint32_t j = first; j < it; ++j)
-                if (!mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1u)) { fail(); break; }
+            if (!ok) break;
         }
+        // Drain: every load issued has landed before the CTA may exit.
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+        for (uint32_t j = first; j < it; ++j)
+            if (!mbar_wait_warp(full_bar(j % STAGES), (j / STAGES) & 1u)) {
+                if (lane == 0) fail();
+                break;
+            }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
-        if (lane == 0) {
-            uint32_t it = 0, local = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x, ++local) {
-                const uint32_t b = local & 1u;
-                const uint32_t aph = (local >> 1) & 1u;
-                if (!mbar_wait(acce_bar(b), aph ^ 1u)) { fail(); break; }
+        // The whole warp walks the loop; lane 0 issues the MMAs and commits.
+        uint32_t it = 0, local = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x, ++local) {
+            const uint32_t b = local & 1u;
+            const uint32_t aph = (local >> 1) & 1u;
+            if (!mbar_wait_warp(acce_bar(b), aph ^ 1u)) {
+                if (lane == 0) fail();
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + b * BN;
+            bool ok = true;
+            for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
+                const uint32_t s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1u;
+                if (!mbar_wait_warp(full_bar(s), ph)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + b * BN;
-                bool ok = true;
-                for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
-                    const uint32_t s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1u;
-                    if (!mbar_wait(full_bar(s), ph)) { fail(); ok = false; break; }
-                    tc_fence_after();
+                if (lane == 0) {
                     const uint32_t a0 = sA + s * Cfg::A_BYTES;
                     const uint32_t b0 = sB + s * Cfg::B_BYTES;
 #pragma unroll
@@ -199,13 +220,18 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     }
                     umma_commit(empty_bar(s));
                 }
-                if (!ok) break;
-                umma_commit(accf_bar(b));
+                __syncwarp();
             }
-            // All MMAs issued by this thread complete before TMEM is released.
+            if (!ok) break;
+            if (lane == 0) umma_commit(accf_bar(b));
+            __syncwarp();
+        }
+        // All MMAs issued by this warp complete before TMEM is released.
+        if (lane == 0) {
             umma_commit(done_bar);
             if (!mbar_wait(done_bar, 0)) fail();
         }
+        __syncwarp();
     } else {
         // ------------------------------- Epilogue -----------------------------------
         const int q = warp & 3;   // TMEM lane quarter this warp may access
@@ -216,7 +242,7 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const uint32_t b = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(accf_bar(b), aph));
+            const bool ok = mbar_wait_warp(accf_bar(b), aph);
             if (!ok) { if (lane == 0) fail(); break; }
             tc_fence_after();
             const int mt = tile / p.num_ntiles;

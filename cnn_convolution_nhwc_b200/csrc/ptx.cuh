@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use: mbarriers, TMA
-// (tiled and im2col loads, tiled stores), tcgen05 (TMEM allocation, MMA, commit, loads) and
-// the global timer that bounds every wait.
+// (tiled and im2col loads, tiled stores) and tcgen05 (TMEM allocation, MMA, commit, loads);
+// every mbarrier wait is bounded by the SM cycle counter.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -10,17 +10,13 @@ namespace convb200 {
 // Device status word bits (one per failure kind). Written with atomicOr, read by the host.
 enum : unsigned { kStatusTimeout = 1u };
 
-// Every spin on an mbarrier gives up after this many nanoseconds.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+// Every spin on an mbarrier gives up after this many SM clock cycles (about one second at
+// the B200's 1.9-2.0 GHz; longer at lower clocks). The SM-local cycle counter is cheap to read,
+// unlike %globaltimer, so the check costs nothing on the fast path.
+constexpr long long kWaitLimitCycles = 2000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long global_timer_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -43,6 +39,8 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One poll of the phase with the given parity (no suspend-time hint: measured on B200, a
+// hinted wait resumes late and slows the pipelines several-fold).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -56,16 +54,46 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Returns false if the wait ran
-// past kWaitLimitNs; the caller then records the timeout and stops.
+// past kWaitLimitCycles; the caller then records the timeout and stops.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_timer_ns();
+    const long long t0 = clock64();
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if (clock64() - t0 > kWaitLimitCycles) return false;
     }
+}
+
+// Wait for a role that is not on the critical path (producer, epilogue): between polls the
+// warp sleeps for about sleep_ns, so it does not compete with the MMA warp and the tensor
+// cores for issue slots and the shared-memory pipe.
+__device__ __forceinline__ bool mbar_wait_backoff(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(sleep_ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+    }
+}
+
+__device__ __forceinline__ bool mbar_wait_warp_backoff(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+    uint32_t ready = 0;
+    if ((threadIdx.x & 31) == 0) ready = mbar_try_wait(bar, parity) ? 1u : 0u;
+    if (__shfl_sync(0xffffffffu, ready, 0)) return true;
+    return __all_sync(0xffffffffu, mbar_wait_backoff(bar, parity, sleep_ns));
+}
+
+// Whole-warp wait. Fast path: one poll by lane 0 (32 lanes polling one barrier serialise,
+// about 15 cycles each). Slow path: every lane polls (measured faster on B200 than one polling
+// lane with the others parked). True only if every lane saw the phase complete.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity) {
+    uint32_t ready = 0;
+    if ((threadIdx.x & 31) == 0) ready = mbar_try_wait(bar, parity) ? 1u : 0u;
+    if (__shfl_sync(0xffffffffu, ready, 0)) return true;
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
 // ---------------------------------------------------------------------------------------

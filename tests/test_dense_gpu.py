@@ -63,6 +63,15 @@ def _check_bf16(y, Xb, Fb):
     return ref
 
 
+_LARGE = {}
+
+
+def _large_inputs():
+    if not _LARGE:
+        _LARGE["v"] = workloads.dense_inputs(workloads.DENSE_LARGE)
+    return _LARGE["v"]
+
+
 def _case_inputs(N, H, W, Cin, Cout, K, seed):
     c = workloads.DenseCase("t", N, H, W, Cin, Cout, K, "bf16", "normal", seed)
     return workloads.dense_inputs(c)
@@ -106,13 +115,14 @@ def test_pins_tensor_core_path(cb):
     F[:, :, 0, 0] = np.arange(9, dtype=np.float32).reshape(3, 3)
     F[:, :, 3, 1] = np.array(so["gx"], np.float32)
     F[:, :, 3, 2] = np.array(so["gy"], np.float32)
-    y = _run_bf16(cb, workloads.bf16_bits(X), workloads.bf16_bits(F), env="bn64")
     exp0 = workloads.bf16_to_f32(workloads.bf16_bits(np.array(g["output"], np.float32)))
-    for n in (0, 1, 100, N - 1):
-        assert np.array_equal(y[n, :, :, 0], exp0)
-        assert np.array_equal(y[n, :, :, 1], np.array(so["gx_output"], np.float32))
-        assert np.array_equal(y[n, :, :, 2], np.array(so["gy_output"], np.float32))
-        assert not y[n, :, :, 3:].any()
+    for path in ("halo64", "bn64"):   # the halo kernel and the im2col kernel
+        y = _run_bf16(cb, workloads.bf16_bits(X), workloads.bf16_bits(F), env=path)
+        for n in (0, 1, 100, N - 1):
+            assert np.array_equal(y[n, :, :, 0], exp0), path
+            assert np.array_equal(y[n, :, :, 1], np.array(so["gx_output"], np.float32)), path
+            assert np.array_equal(y[n, :, :, 2], np.array(so["gy_output"], np.float32)), path
+            assert not y[n, :, :, 3:].any(), path
 
 
 # ------------------------------------------------------------------------------------------
@@ -147,12 +157,14 @@ def test_pointwise_is_matmul(cb):
     assert np.all(np.abs(y.reshape(ref.shape) - ref) <= TOL * bound)
 
 
-def test_large_workload_sampled(cb):
+@pytest.mark.parametrize("path", [None, "halo"], ids=["default", "halo"])
+def test_large_workload_sampled(cb, path):
     # N=64, 112x112, 128->128, K=5: compare 20000 sampled outputs (including the first and
-    # last pixels of every image corner region and the last M tile) with the oracle.
+    # last pixels of every image corner region and the last M tile) with the oracle; the
+    # default path and the halo kernel with its streamed filter.
     case = workloads.DENSE_LARGE
-    Xb, Fb = workloads.dense_inputs(case)
-    y = _run_bf16(cb, Xb, Fb)
+    Xb, Fb = _large_inputs()
+    y = _run_bf16(cb, Xb, Fb, env=path)
     Ho, Wo, Co = case.Ho, case.Wo, case.Cout
     total = case.N * Ho * Wo * Co
     r = workloads.splitmix64(77, 20000)
@@ -185,12 +197,37 @@ EDGE = [
 ]
 
 
+@pytest.mark.parametrize("path", [None, "bn64"], ids=["halo", "im2col"])
 @pytest.mark.parametrize("shape", EDGE, ids=lambda s: "x".join(map(str, s)))
-def test_edge_shapes(cb, shape):
+def test_edge_shapes(cb, shape, path):
     N, H, W, Cin, Cout, K = shape
     Xb, Fb = _case_inputs(N, H, W, Cin, Cout, K, seed=sum(shape))
-    y = _run_bf16(cb, Xb, Fb)
+    if path == "bn64" and Xb.nbytes < 128 * 1024:
+        # the im2col kernel serves inputs of at least 128 KiB; forcing it below is refused
+        os.environ["CONV_B200_DENSE"] = path
+        try:
+            with pytest.raises(cb.ConvError) as e:
+                cb.conv2d_nhwc_fwd(_dev_bf16(Xb), _dev_bf16(Fb))
+            assert e.value.code == cb.CONV_ERR_UNSUPPORTED
+        finally:
+            del os.environ["CONV_B200_DENSE"]
+        return
+    y = _run_bf16(cb, Xb, Fb, env=path)
     _check_bf16(y, Xb, Fb)
+
+
+def test_wide_image_falls_back_to_im2col(cb):
+    # a 2100-pixel-wide image: the halo (128 + 2*2100 rows) does not fit in shared memory,
+    # so the im2col kernel runs; forcing the halo kernel is reported as unsupported
+    Xb, Fb = _case_inputs(2, 3, 2100, 64, 64, 3, seed=21)
+    _check_bf16(_run_bf16(cb, Xb, Fb), Xb, Fb)
+    os.environ["CONV_B200_DENSE"] = "halo"
+    try:
+        with pytest.raises(cb.ConvError) as e:
+            cb.conv2d_nhwc_fwd(_dev_bf16(Xb), _dev_bf16(Fb))
+        assert e.value.code == cb.CONV_ERR_UNSUPPORTED
+    finally:
+        del os.environ["CONV_B200_DENSE"]
 
 
 @pytest.mark.parametrize("shape", [(2, 7, 9, 3, 5, 3), (1, 5, 5, 1, 1, 5), (3, 6, 11, 12, 10, 2)],
@@ -202,15 +239,25 @@ def test_unaligned_channels_direct_path(cb, shape):
     _check_bf16(y, Xb, Fb)
 
 
-def test_tile_width_choices_agree(cb):
-    # every tile width computes each output with the same MMA sequence over the reduction
+def test_kernel_and_tile_width_choices_agree(cb):
+    # Cin = 64 is one channel block, so every kernel and tile width issues the same MMA
+    # sequence per output (taps in (i, j) order, 16 channels per step): identical bits
     Xb, Fb = _case_inputs(4, 24, 24, 64, 256, 3, seed=5)
-    ys = {bn: _run_bf16(cb, Xb, Fb, env=bn) for bn in ("bn64", "bn128", "bn256")}
-    _check_bf16(ys["bn64"], Xb, Fb)
-    for bn in ("bn128", "bn256"):
-        assert np.array_equal(ys[bn], ys["bn64"]), bn
+    ys = {v: _run_bf16(cb, Xb, Fb, env=v) for v in ("halo64", "halo128", "halo256", "bn64", "bn128", "bn256")}
+    _check_bf16(ys["halo64"], Xb, Fb)
+    for v, y in ys.items():
+        assert np.array_equal(y, ys["halo64"]), v
     yd = _run_bf16(cb, Xb, Fb, env="direct")
     _check_bf16(yd, Xb, Fb)
+
+
+def test_streamed_filter_multi_block(cb):
+    # Cin = 192 (three channel blocks) and a filter too large to keep resident: the halo
+    # kernel streams the filter per tap; the im2col kernel agrees within tolerance
+    Xb, Fb = _case_inputs(2, 30, 26, 192, 320, 5, seed=8)
+    _check_bf16(_run_bf16(cb, Xb, Fb, env="halo"), Xb, Fb)
+    _check_bf16(_run_bf16(cb, Xb, Fb), Xb, Fb)
+    _check_bf16(_run_bf16(cb, Xb, Fb, env="bn128"), Xb, Fb)
 
 
 def test_repeatable(cb):
