@@ -19,6 +19,7 @@
 #include "dense_tc.cuh"
 #include "dense_halo.cuh"
 #include "depthwise.cuh"
+#include "depthwise_reg.cuh"
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -429,6 +430,61 @@ int launch_dw_one(const float *x, const float *w, const float *bias, float *y, c
     return cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p) == cudaSuccess ? CONV_OK : CONV_ERR_CUDA;
 }
 
+// ---- register-window kernel ---------------------------------------------------------------
+template <int MODE, bool HB, int K, int S>
+int launch_dw_reg_one(const float *x, const float *w, const float *bias, float *y, const DwRegParams &rp,
+                      cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((rp.num_jobs + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, depthwise_reg_kernel<MODE, HB, K, S, (K - 1) / 2>, x, w, bias, y, rp) == cudaSuccess
+               ? CONV_OK
+               : CONV_ERR_CUDA;
+}
+
+template <int MODE, bool HB>
+int launch_dw_reg(const float *x, const float *w, const float *bias, float *y, const DwRegParams &rp, int K, int S,
+                  cudaStream_t stream) {
+    if (K == 3 && S == 1) return launch_dw_reg_one<MODE, HB, 3, 1>(x, w, bias, y, rp, stream);
+    if (K == 3 && S == 2) return launch_dw_reg_one<MODE, HB, 3, 2>(x, w, bias, y, rp, stream);
+    if (K == 5 && S == 1) return launch_dw_reg_one<MODE, HB, 5, 1>(x, w, bias, y, rp, stream);
+    return launch_dw_reg_one<MODE, HB, 5, 2>(x, w, bias, y, rp, stream);
+}
+
+// The register kernel serves square 3x3 / 5x5 filters, stride 1 or 2, "same" padding
+// (K-1)/2, no dilation, and output rows of at most 128 columns (one warp per row).
+bool dw_reg_eligible(int KH, int KW, int stride, int pad, int dil, long long Wo) {
+    return KH == KW && (KH == 3 || KH == 5) && (stride == 1 || stride == 2) && pad == (KH - 1) / 2 && dil == 1 &&
+           Wo <= 128;
+}
+
+DwRegParams dw_reg_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, int num_sms, const float *x,
+                        const float *y) {
+    DwRegParams rp{};
+    rp.Cin = Cin; rp.mult = mult; rp.Cout = Cin * mult; rp.H = H; rp.W = W; rp.Ho = Ho; rp.Wo = Wo;
+    rp.lpp = (Wo + 3) / 4;
+    rp.ppw = 32 / rp.lpp;
+    rp.num_planes = N * rp.Cout;
+    const long long groups = (rp.num_planes + rp.ppw - 1) / rp.ppw;
+    // bands of output rows: enough warps to fill the machine about twice (64 resident warps
+    // per SM), but no band shorter than 8 rows unless the plane is
+    const long long want = 2LL * num_sms * 64;
+    int nb = static_cast<int>((want + groups - 1) / groups);
+    if (nb > (Ho + 7) / 8) nb = (Ho + 7) / 8;
+    if (nb < 1) nb = 1;
+    rp.band = (Ho + nb - 1) / nb;
+    rp.nbands = (Ho + rp.band - 1) / rp.band;
+    rp.num_jobs = static_cast<int>(groups * rp.nbands);
+    rp.vec_in = (W % 4 == 0 && aligned(x, 16)) ? 1 : 0;
+    rp.vec_out = (Wo % 4 == 0 && aligned(y, 16)) ? 1 : 0;
+    rp.div_cout = make_fastdiv(static_cast<uint32_t>(rp.Cout));
+    rp.div_mult = make_fastdiv(static_cast<uint32_t>(mult));
+    rp.div_nbands = make_fastdiv(static_cast<uint32_t>(rp.nbands));
+    rp.div_lpp = make_fastdiv(static_cast<uint32_t>(rp.lpp));
+    return rp;
+}
+
 template <int MODE, bool HB>
 int launch_dw(const float *x, const float *w, const float *bias, float *y, const DwParams &p, DwSpec s,
               long long jobs, cudaStream_t stream, DeviceState *d) {
@@ -520,6 +576,23 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
         return CONV_ERR_INVALID_ARG;
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
+
+    // Register-window kernel for the common shapes (CONV_B200_DW_KERNEL=smem forces the
+    // shared-memory kernel, =reg requires the register kernel; tests).
+    const char *kforce = env("CONV_B200_DW_KERNEL");
+    const bool force_smem = kforce && std::strcmp(kforce, "smem") == 0;
+    const bool force_reg = kforce && std::strcmp(kforce, "reg") == 0;
+    const bool reg_ok = dw_reg_eligible(KH, KW, stride, pad, dil, Wo) && 1LL * N * Cout <= kInt32Max;
+    if (force_reg && !reg_ok) return CONV_ERR_UNSUPPORTED;
+    if (reg_ok && !force_smem && !env("CONV_B200_DW_TILE")) {
+        const DwRegParams rp = dw_reg_plan(N, Cin, mult, H, W, static_cast<int>(Ho), static_cast<int>(Wo), d->num_sms, x, y);
+        const bool hb = bias != nullptr;
+        if (mode == DW_EXACT)
+            return hb ? launch_dw_reg<0, true>(x, w, bias, y, rp, KH, stride, stream)
+                      : launch_dw_reg<0, false>(x, w, bias, y, rp, KH, stride, stream);
+        return hb ? launch_dw_reg<1, true>(x, w, bias, y, rp, KH, stride, stream)
+                  : launch_dw_reg<1, false>(x, w, bias, y, rp, KH, stride, stream);
+    }
 
     DwParams p;
     p.Cin = Cin; p.mult = mult; p.Cout = static_cast<int>(Cout); p.H = H; p.W = W; p.KH = KH; p.KW = KW;

@@ -194,3 +194,39 @@ def test_results_independent_of_tiling(cb, tile):
         y = _gpu(cb, x, w, b, case.stride, case.pad, case.dil, mode, tile=tile)
         assert np.array_equal(_bits(y), _bits(base))
         _compare(y, x, w, b, case.mult, case.stride, case.pad, case.dil, mode)
+
+
+def _with_env(name, value, fn):
+    old = os.environ.get(name)
+    os.environ[name] = value
+    try:
+        return fn()
+    finally:
+        if old is None:
+            del os.environ[name]
+        else:
+            os.environ[name] = old
+
+
+@pytest.mark.parametrize("case", workloads.DW_SWEEP, ids=lambda c: c.name)
+def test_register_and_shared_kernels_identical(cb, case):
+    # the register-window kernel (the default for these shapes) and the shared-memory kernel
+    # compute every output in the same order: identical bits, both equal to the oracle
+    small = workloads.DepthwiseCase(case.name, 2, case.C, 2 if case.C <= 72 else 1, case.H, case.W, case.KH,
+                                    case.KW, case.stride, case.pad, case.dil, True, 11)
+    x, w, b = workloads.depthwise_inputs(small)
+    for mode in MODES:
+        yr = _with_env("CONV_B200_DW_KERNEL", "reg",
+                       lambda: _gpu(cb, x, w, b, small.stride, small.pad, small.dil, mode))
+        ys = _with_env("CONV_B200_DW_KERNEL", "smem",
+                       lambda: _gpu(cb, x, w, b, small.stride, small.pad, small.dil, mode))
+        assert np.array_equal(_bits(yr), _bits(ys))
+        _compare(yr, x, w, b, small.mult, small.stride, small.pad, small.dil, mode)
+
+
+def test_register_kernel_refuses_other_shapes(cb):
+    x = np.ones((1, 2, 9, 9), np.float32)
+    w = np.ones((2, 3, 3), np.float32)
+    with pytest.raises(cb.ConvError) as e:
+        _with_env("CONV_B200_DW_KERNEL", "reg", lambda: _gpu(cb, x, w, None, 1, 0, 1, 0))   # pad 0
+    assert e.value.code == cb.CONV_ERR_UNSUPPORTED
