@@ -40,9 +40,13 @@ lib.conv_status_string.argtypes = [_I]
 lib.conv_status_string.restype = ctypes.c_char_p
 lib.conv_device_status.argtypes = [_P, _I]
 lib.conv_device_status.restype = _I
+lib.conv_last_kernel.argtypes = []
+lib.conv_last_kernel.restype = ctypes.c_char_p
+lib.conv_selftest_wait_timeout.argtypes = [_P]
+lib.conv_selftest_wait_timeout.restype = _I
 
 EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "depthwise_fwd", "conv_status_string",
-           "conv_device_status")
+           "conv_device_status", "conv_last_kernel", "conv_selftest_wait_timeout")
 
 
 class ConvError(RuntimeError):
@@ -141,6 +145,16 @@ def depthwise_fwd(x, w, bias=None, y=None, stride=1, pad=0, dil=1, mode=DW_EXACT
     _check(lib.depthwise_fwd(px, pw, pb, py, N, Cin, mult, H, W, KH, KW, stride, pad, dil, int(mode),
                              _stream(stream)), "depthwise_fwd")
     return y
+
+
+def conv_last_kernel() -> str:
+    """Kernel family the last successful call on this thread launched (the dispatcher's choice)."""
+    return lib.conv_last_kernel().decode()
+
+
+def conv_selftest_wait_timeout(stream=None) -> int:
+    """Runs the bounded-wait diagnostic (about one second); returns the launch status."""
+    return lib.conv_selftest_wait_timeout(_stream(stream))
 
 
 def conv_device_status(stream=None, reset=False) -> int:

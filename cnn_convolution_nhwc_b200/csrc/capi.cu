@@ -18,8 +18,10 @@
 #include "dense_direct.cuh"
 #include "dense_tc.cuh"
 #include "dense_halo.cuh"
+#include "dense_fold.cuh"
 #include "depthwise.cuh"
 #include "depthwise_reg.cuh"
+#include "depthwise_tma.cuh"
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -27,7 +29,28 @@ namespace convb200 {
 // One status word per device; kernels set bits in it with atomicOr.
 __device__ unsigned int g_conv_status;
 
+// One CTA waiting on a barrier that nothing completes: exercises the bounded wait.
+__global__ void selftest_wait_kernel(unsigned int *status) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(b, 0)) atomicOr(status, kStatusTimeout);
+}
+
 namespace {
+
+// family name of the kernel the last successful launch on this host thread used
+thread_local const char *t_last_kernel = "";
+
+int launched(cudaError_t e, const char *name) {
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    t_last_kernel = name;
+    return CONV_OK;
+}
 
 constexpr int kMaxDevices = 64;
 constexpr long long kInt32Max = 2147483647LL;
@@ -46,7 +69,7 @@ struct DeviceState {
     bool ready = false;
     int num_sms = 0;
     unsigned int *status = nullptr;   // device address of g_conv_status on this device
-    unsigned attr_done = 0;           // bit per kernel whose shared-memory limit is raised
+    unsigned long long attr_done = 0; // bit per kernel whose shared-memory limit is raised
 };
 
 std::mutex g_mu;
@@ -87,11 +110,11 @@ int device_state(DeviceState **out) {
 
 template <typename Kern>
 int ensure_smem_attr(DeviceState *d, unsigned bit, Kern kern, int bytes) {
-    if (d->attr_done & (1u << bit)) return CONV_OK;
+    if (d->attr_done & (1ull << bit)) return CONV_OK;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return CONV_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    d->attr_done |= 1u << bit;
+    d->attr_done |= 1ull << bit;
     return CONV_OK;
 }
 
@@ -139,8 +162,7 @@ int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int C
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, dense_direct_kernel<T>, X, F, Y, p) == cudaSuccess ? CONV_OK
-                                                                                      : CONV_ERR_CUDA;
+    return launched(cudaLaunchKernelEx(&cfg, dense_direct_kernel<T>, X, F, Y, p), "dense_direct_kernel");
 }
 
 template <class Cfg>
@@ -201,8 +223,7 @@ int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, 
     cfg.blockDim = dim3(192);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, kern, tmX, tmF, tmY, p, d->status) == cudaSuccess ? CONV_OK
-                                                                                      : CONV_ERR_CUDA;
+    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, tmY, p, d->status), "dense_tc_kernel");
 }
 
 // ---- halo kernel ------------------------------------------------------------------------
@@ -322,9 +343,8 @@ int launch_dense_halo(const void *X, const void *F, void *Y, int Cin, int Cout, 
     cfg.blockDim = dim3(192);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status) == cudaSuccess
-               ? CONV_OK
-               : CONV_ERR_CUDA;
+    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
+                    "dense_halo_kernel");
 }
 
 int dispatch_halo(const void *X, const void *F, void *Y, int Cin, int Cout, int K, const HaloPlan &pl,
@@ -336,6 +356,99 @@ int dispatch_halo(const void *X, const void *F, void *Y, int Cin, int Cout, int 
                                      : launch_dense_halo<DenseHaloCfg<128, false>>(X, F, Y, Cin, Cout, K, pl, stream, d, 6);
     return pl.bres ? launch_dense_halo<DenseHaloCfg<256, true>>(X, F, Y, Cin, Cout, K, pl, stream, d, 7)
                    : launch_dense_halo<DenseHaloCfg<256, false>>(X, F, Y, Cin, Cout, K, pl, stream, d, 28);
+}
+
+// ---- folded-tap kernel (Cout <= 64, K = 2..4) ---------------------------------------------
+struct FoldPlan {
+    bool ok = false;
+    DenseFoldParams p{};
+    int smem = 0;
+    int grid = 0;
+};
+
+template <int KF>
+int fold_fixed_bytes() { return DenseFoldCfg<KF>::FIXED_BYTES; }
+
+FoldPlan plan_fold(int N, int H, int W, int Cin, int Cout, int K, int num_sms) {
+    FoldPlan pl;
+    if (Cout > 64 || K < 2 || K > 4) return pl;
+    const long long rows = 1LL * N * H * W;
+    if (rows + 1024 > kInt32Max) return pl;
+    const int need = 128 + (K - 1) * W;
+    if (need > 4096) return pl;
+    const int n_boxes = (need + 255) / 256;
+    const int box_rows = (((need + n_boxes - 1) / n_boxes) + 7) & ~7;
+    const int halo_rows = n_boxes * box_rows;
+    const int halo_bytes = halo_rows * 128;
+    const int num_cblk = (Cin + 63) / 64;
+    const int num_kblk = K * K * num_cblk;
+    const int fixed = K == 2 ? fold_fixed_bytes<2>() : (K == 3 ? fold_fixed_bytes<3>() : fold_fixed_bytes<4>());
+    const long long b_res = 1LL * num_kblk * DenseFoldCfg<2>::SLOT_BYTES;
+    if (fixed + b_res + 2LL * halo_bytes > kSmemLimit) return pl;
+    DenseFoldParams &p = pl.p;
+    p.HS = static_cast<int>((kSmemLimit - fixed - b_res) / halo_bytes);
+    if (p.HS > DenseFoldCfg<2>::MAX_RING) p.HS = DenseFoldCfg<2>::MAX_RING;
+    const int TM = 128 - (K - 1);
+    p.rows = static_cast<int>(rows);
+    p.H = H; p.W = W; p.Ho = H - K + 1; p.Wo = W - K + 1;
+    p.K = K; p.KK = K * K; p.Cout = Cout;
+    p.num_cblk = num_cblk;
+    p.num_kblk = num_kblk;
+    p.halo_rows = halo_rows;
+    p.box_rows = box_rows;
+    p.n_boxes = n_boxes;
+    p.halo_bytes = halo_bytes;
+    p.b_region = static_cast<int>(b_res);
+    p.num_tiles = static_cast<int>((rows + TM - 1) / TM);
+    pl.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    pl.smem = fixed + p.b_region + p.HS * halo_bytes;
+    // more than half of the shared memory keeps a second CTA (and its TMEM allocation) off the SM
+    if (pl.smem < 116 * 1024) pl.smem = 116 * 1024;
+    pl.ok = pl.smem <= kSmemLimit;
+    return pl;
+}
+
+template <int KF>
+int launch_dense_fold(const void *X, const void *F, void *Y, int Cin, int Cout, const FoldPlan &pl,
+                      cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
+    alignas(64) CUtensorMap tmX, tmF;
+    {   // X as a 2-D matrix: rows = flattened (n, y, x), Cin channels per row
+        const cuuint64_t dims[2] = {(cuuint64_t)Cin, (cuuint64_t)pl.p.rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)Cin * 2};
+        const cuuint32_t box[2] = {64, (cuuint32_t)pl.p.box_rows};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode_tiled(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    {   // F: 3-D {Cout, Cin, K*K}; a box is 64 channels x 64 output channels of one tap
+        const cuuint64_t dims[3] = {(cuuint64_t)Cout, (cuuint64_t)Cin, (cuuint64_t)KF * KF};
+        const cuuint64_t strides[2] = {(cuuint64_t)Cout * 2, (cuuint64_t)Cin * Cout * 2};
+        const cuuint32_t box[3] = {64, 64, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(F), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    auto kern = dense_fold_kernel<DenseFoldCfg<KF>>;
+    if (int rc = ensure_smem_attr(d, attr_bit, kern, kSmemLimit)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
+                    "dense_fold_kernel");
+}
+
+int dispatch_fold(const void *X, const void *F, void *Y, int Cin, int Cout, int K, const FoldPlan &pl,
+                  cudaStream_t stream, DeviceState *d) {
+    // shared-memory attribute bits 29..31
+    if (K == 2) return launch_dense_fold<2>(X, F, Y, Cin, Cout, pl, stream, d, 29);
+    if (K == 3) return launch_dense_fold<3>(X, F, Y, Cin, Cout, pl, stream, d, 30);
+    return launch_dense_fold<4>(X, F, Y, Cin, Cout, pl, stream, d, 31);
 }
 
 using CfgBN64 = DenseTcCfg<64, 6>;
@@ -427,7 +540,7 @@ int launch_dw_one(const float *x, const float *w, const float *bias, float *y, c
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p) == cudaSuccess ? CONV_OK : CONV_ERR_CUDA;
+    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p), "depthwise_kernel");
 }
 
 // ---- register-window kernel ---------------------------------------------------------------
@@ -438,9 +551,8 @@ int launch_dw_reg_one(const float *x, const float *w, const float *bias, float *
     cfg.gridDim = dim3(static_cast<unsigned>((rp.num_jobs + 7) / 8));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, depthwise_reg_kernel<MODE, HB, K, S, (K - 1) / 2>, x, w, bias, y, rp) == cudaSuccess
-               ? CONV_OK
-               : CONV_ERR_CUDA;
+    return launched(cudaLaunchKernelEx(&cfg, depthwise_reg_kernel<MODE, HB, K, S, (K - 1) / 2>, x, w, bias, y, rp),
+                    "depthwise_reg_kernel");
 }
 
 template <int MODE, bool HB>
@@ -485,6 +597,106 @@ DwRegParams dw_reg_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, 
     return rp;
 }
 
+// ---- TMA-staged kernel ----------------------------------------------------------------------
+constexpr int kDwTmaMaxSmem = 160 * 1024;   // per CTA: 4 warps x 2 buffers
+
+struct DwTmaPlan {
+    bool ok = false;
+    DwTmaParams p{};
+    int grid = 0;
+    int smem = 0;
+};
+
+DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, int K, int S, int num_sms,
+                      const float *x, const float *y) {
+    DwTmaPlan pl;
+    if (mult != 1) return pl;
+    DwTmaParams &p = pl.p;
+    p.H = H; p.W = W; p.Ho = Ho; p.Wo = Wo; p.C = Cin;
+    p.lpp = (Wo + 3) / 4;
+    p.ppw = 32 / p.lpp;
+    if (p.ppw < 1) return pl;
+    p.num_planes = N * Cin;
+    p.Wp = p.lpp * 4 * S + 8;                       // 4 zeros, the lanes' columns, the right reach
+    p.use_tma = (W % 4 == 0 && aligned(x, 16)) ? 1 : 0;
+    // staged bytes per job buffer: whole planes when they fit, else bands of rows
+    const long long row_bytes = 4LL * p.Wp * p.ppw;
+    // about 9 KB per buffer keeps 12 warps (3 CTAs) per SM with both buffers resident
+    const long long kBufBytes = 9 * 1024;
+    const int whole_rows = (Ho - 1) * S + K;
+    if (whole_rows * row_bytes <= kBufBytes || !p.use_tma) {
+        p.Rw = Ho;
+        if (!p.use_tma && whole_rows * row_bytes > 2 * kBufBytes) return pl;   // cp.async jobs are whole planes
+    } else {
+        int Rw = static_cast<int>((kBufBytes / row_bytes - K) / S + 1);
+        if (Rw < 4) Rw = 4;
+        p.Rw = Rw;
+    }
+    p.rows_in = (p.Rw - 1) * S + K;
+    if (p.use_tma && (p.Wp > 256 || p.rows_in > 256)) return pl;
+    p.box_floats = p.ppw * p.rows_in * p.Wp;
+    p.buf_floats = (p.box_floats + 31) & ~31;
+    p.nbands = (Ho + p.Rw - 1) / p.Rw;
+    const long long groups = (p.num_planes + p.ppw - 1) / p.ppw;
+    if (groups * p.nbands > kInt32Max) return pl;
+    p.num_jobs = static_cast<int>(groups * p.nbands);
+    p.vec_out = (Wo % 4 == 0 && aligned(y, 16)) ? 1 : 0;
+    p.div_nbands = make_fastdiv(static_cast<uint32_t>(p.nbands));
+    p.div_lpp = make_fastdiv(static_cast<uint32_t>(p.lpp));
+    p.div_c = make_fastdiv(static_cast<uint32_t>(p.C));
+    p.div_w = make_fastdiv(static_cast<uint32_t>(W));
+    pl.smem = kDwWarpsPerCta * 2 * 4 * p.buf_floats + 128;   // + alignment slack
+    if (pl.smem > kDwTmaMaxSmem) return pl;
+    int per_sm = (227 * 1024) / (pl.smem + 1024);
+    if (per_sm > 16) per_sm = 16;
+    if (per_sm < 1) return pl;
+    const long long warps_needed = p.num_jobs;
+    long long g = 1LL * num_sms * per_sm;
+    const long long g_jobs = (warps_needed + kDwWarpsPerCta - 1) / kDwWarpsPerCta;
+    if (g > g_jobs) g = g_jobs;
+    pl.grid = static_cast<int>(g);
+    pl.ok = true;
+    return pl;
+}
+
+template <int MODE, bool HB, int K, int S>
+int launch_dw_tma_one(const float *x, const float *w, const float *bias, float *y, const DwTmaPlan &pl, int Cin, int N,
+                      cudaStream_t stream, DeviceState *d, unsigned bit) {
+    const DwTmaParams &p = pl.p;
+    alignas(64) CUtensorMap tm;
+    std::memset(&tm, 0, sizeof tm);
+    if (p.use_tma) {
+        const cuuint64_t dims[3] = {(cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)N * Cin};
+        const cuuint64_t strides[2] = {(cuuint64_t)p.W * 4, (cuuint64_t)p.H * p.W * 4};
+        const cuuint32_t box[3] = {(cuuint32_t)p.Wp, (cuuint32_t)p.rows_in, (cuuint32_t)p.ppw};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode_tiled(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(x), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    auto kern = depthwise_tma_kernel<MODE, HB, K, S>;
+    if (pl.smem > 48 * 1024)
+        if (int rc = ensure_smem_attr(d, bit, kern, kDwTmaMaxSmem)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(32 * kDwWarpsPerCta);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    return launched(cudaLaunchKernelEx(&cfg, kern, tm, x, w, bias, y, p, d->status), "depthwise_tma_kernel");
+}
+
+template <int MODE, bool HB>
+int launch_dw_tma(const float *x, const float *w, const float *bias, float *y, const DwTmaPlan &pl, int K, int S,
+                  int Cin, int N, cudaStream_t stream, DeviceState *d) {
+    // shared-memory attribute bits 32..47
+    const unsigned base = 32u + 4u * (2u * MODE + (HB ? 1u : 0u));
+    if (K == 3 && S == 1) return launch_dw_tma_one<MODE, HB, 3, 1>(x, w, bias, y, pl, Cin, N, stream, d, base + 0);
+    if (K == 3 && S == 2) return launch_dw_tma_one<MODE, HB, 3, 2>(x, w, bias, y, pl, Cin, N, stream, d, base + 1);
+    if (K == 5 && S == 1) return launch_dw_tma_one<MODE, HB, 5, 1>(x, w, bias, y, pl, Cin, N, stream, d, base + 2);
+    return launch_dw_tma_one<MODE, HB, 5, 2>(x, w, bias, y, pl, Cin, N, stream, d, base + 3);
+}
+
 template <int MODE, bool HB>
 int launch_dw(const float *x, const float *w, const float *bias, float *y, const DwParams &p, DwSpec s,
               long long jobs, cudaStream_t stream, DeviceState *d) {
@@ -524,11 +736,19 @@ int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, 
     // "halo64/128/256" (halo kernel with that tile width), "bn64/128/256" (im2col kernel).
     int force_bn = 0;
     bool force_im2col = false, force_halo = false;
+    const bool force_fold = force && std::strcmp(force, "fold") == 0;
     if (force) {
         if (std::strncmp(force, "halo", 4) == 0) { force_halo = true; force_bn = std::atoi(force + 4); }
         if (std::strncmp(force, "bn", 2) == 0) { force_im2col = true; force_bn = std::atoi(force + 2); }
     }
     if (force_bn != 0 && force_bn != 64 && force_bn != 128 && force_bn != 256) return CONV_ERR_INVALID_ARG;
+    // Narrow layers (Cout <= 64, K = 2..4) with a resident filter: the folded-tap kernel
+    // ("fold" forces it).
+    if (force_fold || (!force_im2col && !force_halo)) {
+        const FoldPlan fp = plan_fold(N, H, W, Cin, Cout, K, d->num_sms);
+        if (fp.ok) return dispatch_fold(X, F, Y, Cin, Cout, K, fp, stream, d);
+        if (force_fold) return CONV_ERR_UNSUPPORTED;
+    }
     if (!force_im2col) {
         // By default the halo kernel runs when the filter stays resident in shared memory;
         // with a streamed filter the im2col kernel measured faster (deeper operand ring).
@@ -584,6 +804,20 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
     const bool force_reg = kforce && std::strcmp(kforce, "reg") == 0;
     const bool reg_ok = dw_reg_eligible(KH, KW, stride, pad, dil, Wo) && 1LL * N * Cout <= kInt32Max;
     if (force_reg && !reg_ok) return CONV_ERR_UNSUPPORTED;
+    const bool force_tma = kforce && std::strcmp(kforce, "tma") == 0;
+    if (reg_ok && !force_smem && !force_reg && !env("CONV_B200_DW_TILE")) {
+        const DwTmaPlan tp = dw_tma_plan(N, Cin, mult, H, W, static_cast<int>(Ho), static_cast<int>(Wo), KH, stride,
+                                         d->num_sms, x, y);
+        if (tp.ok) {
+            const bool hb = bias != nullptr;
+            if (mode == DW_EXACT)
+                return hb ? launch_dw_tma<0, true>(x, w, bias, y, tp, KH, stride, Cin, N, stream, d)
+                          : launch_dw_tma<0, false>(x, w, bias, y, tp, KH, stride, Cin, N, stream, d);
+            return hb ? launch_dw_tma<1, true>(x, w, bias, y, tp, KH, stride, Cin, N, stream, d)
+                      : launch_dw_tma<1, false>(x, w, bias, y, tp, KH, stride, Cin, N, stream, d);
+        }
+    }
+    if (force_tma) return CONV_ERR_UNSUPPORTED;
     if (reg_ok && !force_smem && !env("CONV_B200_DW_TILE")) {
         const DwRegParams rp = dw_reg_plan(N, Cin, mult, H, W, static_cast<int>(Ho), static_cast<int>(Wo), d->num_sms, x, y);
         const bool hb = bias != nullptr;
@@ -644,6 +878,18 @@ const char *conv_status_string(int status) {
         case CONV_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
         default: return "unknown status";
     }
+}
+
+const char *conv_last_kernel(void) { return t_last_kernel; }
+
+int conv_selftest_wait_timeout(cudaStream_t stream) {
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(32);
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, selftest_wait_kernel, d->status) == cudaSuccess ? CONV_OK : CONV_ERR_CUDA;
 }
 
 int conv_device_status(cudaStream_t stream, int reset) {

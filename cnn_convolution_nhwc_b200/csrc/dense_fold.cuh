@@ -1,0 +1,330 @@
+// Dense NHWC forward convolution for narrow layers (Cout <= 64, 2 <= K <= 4): the halo
+// implicit GEMM with the filter's column taps folded into the MMA's N dimension.
+//
+// Same operation and flattened-row addressing as dense_halo.cuh (CMU DLSys Lecture 14 notes,
+// section 1 "Fix the index contract before optimizing it" for the definition, section 2 "Move
+// the channel contraction into matrix multiplication" for the per-tap matrix products). With
+// Cout = 64 every tap of the halo kernel is an M=128, N=64 tcgen05.mma, which sm_100a issues at
+// about half the tensor rate of N >= 128. Here the K column taps j of one filter row i share
+// one MMA of N = 64*K instead:
+//
+//     D_j[m, o] = sum_i sum_c X[m + i*W, c] * F[i, j, c, o]      (one MMA per (i, 16 channels))
+//     Y[m, o]   = D_0[m, o] + D_1[m + 1, o] + ... + D_{K-1}[m + K-1, o]
+//
+// B of that MMA is the K filter slots (i, 0..K-1) side by side, which the resident filter
+// already holds contiguously (one 64-column MN-major box per slot), so the descriptor's
+// leading-byte offset steps from one tap to the next. The row shift m + j moves from the A
+// operand to the epilogue: a TMEM lane holds one row, so lane r adds group j of row r + j,
+// taken from the lane j below by a warp shuffle, or -- for the last K-1 lanes of a warp --
+// from the next warp's first lanes through a small shared-memory exchange. A tile computes 128
+// rows of D and keeps the first 128 - (K-1) rows of Y; consecutive tiles overlap by K-1 rows.
+//
+// Summation order per output: fp32 tensor-core sums over (i, c) inside each group j, then the
+// groups added in j order in fp32, one rounding to bf16 -- a different order from the other
+// kernels, within the same error bound.
+//
+// Roles as in the halo kernel (warp 0 TMA, warp 1 TMEM + MMA, warps 2..5 epilogue); the
+// filter is always resident here.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "dense_halo.cuh"
+#include "dense_tc.cuh"
+#include "ptx.cuh"
+
+namespace convb200 {
+
+struct DenseFoldParams {
+    int rows;          // N * H * W: flattened input positions
+    int H, W, Ho, Wo;
+    int K, KK, Cout;
+    int num_cblk;      // ceil(Cin / 64)
+    int num_kblk;      // KK * num_cblk filter slots, channel block outer, tap (i, j) inner
+    int halo_rows, box_rows, n_boxes, halo_bytes;
+    int num_tiles;     // ceil(rows / (128 - (K-1)))
+    int HS;            // halo ring slots
+    int b_region;      // bytes of the resident filter
+};
+
+template <int KF>
+struct DenseFoldCfg {
+    static constexpr int K = KF;
+    static constexpr int NF = 64 * KF;                 // MMA N: K groups of 64 columns
+    static constexpr int BM = 128;
+    static constexpr int TM = BM - (KF - 1);           // output rows kept per tile
+    static constexpr int SLOT_BYTES = 64 * 64 * 2;     // one (tap, channel block) filter slot
+    static constexpr int EPI_BYTES = 4 * 32 * 128;     // per-warp 32 rows x 64 channels staging
+    static constexpr int MAX_RING = 8;
+    // exchange: lanes 0..j-1 of group j (j >= 1), 64 floats each, per warp and tile parity
+    static constexpr int XCH_FLOATS = KF * (KF - 1) / 2 * 64;
+    static constexpr int XCH_BYTES = 2 * 4 * XCH_FLOATS * 4;
+    static constexpr int NUM_BARS = 2 * MAX_RING /*halo*/ + 1 /*filter*/ + 4 /*acc*/ + 2 /*xch*/ + 1;
+    static constexpr int TMEM_COLS = 2 * NF <= 256 ? 256 : 512;
+    static constexpr uint32_t IDESC = idesc_bf16_f32(BM, NF, /*B MN-major*/ true);
+    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + XCH_BYTES + NUM_BARS * 8 + 4 * 32 * 8 + 16;
+    static_assert(KF >= 2 && KF <= 4, "N = 64*K must stay within 256");
+};
+
+template <class Cfg>
+__global__ void __launch_bounds__(192, 1)
+dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
+                  __nv_bfloat16 *__restrict__ Y, const DenseFoldParams p, unsigned int *status) {
+    constexpr int K = Cfg::K;
+    constexpr int NF = Cfg::NF;
+    constexpr int TM = Cfg::TM;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;   // 1024-B alignment for the swizzle
+    uint8_t *smem = smem_raw + (base - raw_base);
+
+    const uint32_t sB = base;                                 // resident filter
+    const uint32_t sH = base + p.b_region;                    // halo ring
+    const uint32_t epi_off = p.b_region + p.HS * p.halo_bytes;
+    const uint32_t sEpi = base + epi_off;
+    float *xch = reinterpret_cast<float *>(smem + epi_off + Cfg::EPI_BYTES);
+    const uint32_t bars = sEpi + Cfg::EPI_BYTES + Cfg::XCH_BYTES;
+    constexpr int R = Cfg::MAX_RING;
+    auto hfull = [&](int s) { return bars + 8u * s; };
+    auto hempty = [&](int s) { return bars + 8u * (R + s); };
+    const uint32_t bfull = bars + 8u * (2 * R);
+    auto accf = [&](int b) { return bars + 8u * (2 * R + 1 + b); };
+    auto acce = [&](int b) { return bars + 8u * (2 * R + 3 + b); };
+    auto xbar = [&](int b) { return bars + 8u * (2 * R + 5 + b); };
+    const uint32_t done_bar = bars + 8u * (2 * R + 7);
+    long long *rowoff_all =
+        reinterpret_cast<long long *>(smem + epi_off + Cfg::EPI_BYTES + Cfg::XCH_BYTES + Cfg::NUM_BARS * 8);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rowoff_all + 4 * 32);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < R; ++s) {
+            mbar_init(hfull(s), 1);
+            mbar_init(hempty(s), 1);
+        }
+        mbar_init(bfull, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf(b), 1);
+            mbar_init(acce(b), 128);
+            mbar_init(xbar(b), 128);
+        }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmF);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    auto fail = [&]() {
+        atomicOr(status, kStatusTimeout);
+        *abort_flag = 1;
+    };
+    const int first = static_cast<int>(blockIdx.x);
+    const int step = static_cast<int>(gridDim.x);
+
+    if (warp == 0) {
+        // ------------------------------- TMA producer -------------------------------
+        uint32_t hit = 0;
+        bool ok = true, filter_issued = false;
+        auto load_filter = [&]() {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bfull, p.num_kblk * Cfg::SLOT_BYTES);
+                for (int kb = 0; kb < p.num_kblk; ++kb) {
+                    const int cb = kb / p.KK, tap = kb - cb * p.KK;
+                    tma_load_3d(sB + kb * Cfg::SLOT_BYTES, &tmF, bfull, 0, cb * 64, tap);
+                }
+            }
+            __syncwarp();
+        };
+        for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step) {
+            const int P0 = t * TM;
+            for (int cb = 0; cb < p.num_cblk; ++cb) {
+                const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
+                if (!mbar_wait_warp_backoff(hempty(hs), hph ^ 1u, 64)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(hfull(hs), p.halo_bytes);
+                    for (int bx = 0; bx < p.n_boxes; ++bx)
+                        tma_load_2d(sH + hs * p.halo_bytes + bx * p.box_rows * 128, &tmX, hfull(hs), cb * 64,
+                                    P0 + bx * p.box_rows);
+                }
+                __syncwarp();
+                ++hit;
+                if (!filter_issued) {   // after the first halo, so the first tile's operands arrive together
+                    load_filter();
+                    filter_issued = true;
+                }
+            }
+        }
+        if (!filter_issued) load_filter();
+        if (!ok && lane == 0) fail();
+        // Drain: every load issued has landed before the CTA may exit.
+        if (!mbar_wait_warp(bfull, 0) && lane == 0) fail();
+        for (uint32_t j = hit > (uint32_t)p.HS ? hit - p.HS : 0u; j < hit; ++j)
+            if (!mbar_wait_warp(hfull(j % p.HS), (j / p.HS) & 1u)) { if (lane == 0) fail(); break; }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer ---------------------------------
+        uint32_t hit = 0, local = 0;
+        bool ok = mbar_wait_warp(bfull, 0);
+        for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step, ++local) {
+            const uint32_t b = local & 1u;
+            if (!mbar_wait_warp(acce(b), ((local >> 1) & 1u) ^ 1u)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + b * NF;
+            for (int cb = 0; cb < p.num_cblk; ++cb) {
+                const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
+                if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
+                tc_fence_after();
+                if (lane == 0) {
+                    // filter row i reads the halo from row i*W on (start field in 16-byte
+                    // units: +8 per 128-byte row, +2 per 16 channels); B spans the K slots
+                    // (i, 0..K-1), 8 KB apart (the leading-byte offset), +128 per 16 channels
+                    const uint64_t a0 = smem_desc_sw128(sH + hs * p.halo_bytes, 16, 1024);
+#pragma unroll
+                    for (int i = 0; i < K; ++i) {
+                        const uint64_t ad = a0 + static_cast<uint64_t>(i * p.W * 8);
+                        const uint64_t bd = smem_desc_sw128(sB + (cb * p.KK + i * K) * Cfg::SLOT_BYTES,
+                                                            Cfg::SLOT_BYTES, 1024);
+                        umma_f16_ss(d_tmem, ad, bd, Cfg::IDESC, (cb | i) != 0 ? 1u : 0u);
+                        umma_f16_ss(d_tmem, ad + 2, bd + 128, Cfg::IDESC, 1u);
+                        umma_f16_ss(d_tmem, ad + 4, bd + 256, Cfg::IDESC, 1u);
+                        umma_f16_ss(d_tmem, ad + 6, bd + 384, Cfg::IDESC, 1u);
+                    }
+                    umma_commit(hempty(hs));
+                }
+                __syncwarp();
+                ++hit;
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(accf(b));
+            __syncwarp();
+        }
+        if (!ok && lane == 0) fail();
+        if (lane == 0) {
+            umma_commit(done_bar);
+            if (!mbar_wait(done_bar, 0)) fail();
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------- Epilogue -----------------------------------
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const uint32_t stage = sEpi + q * 4096;
+        long long *rowoff = rowoff_all + q * 32;
+        uint32_t local = 0;
+        for (int t = first; t < p.num_tiles; t += step, ++local) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            const uint32_t b = local & 1u, par = local & 1u;
+            if (!mbar_wait_warp_backoff(accf(b), (local >> 1) & 1u, 128)) { if (lane == 0) fail(); break; }
+            tc_fence_after();
+            // this lane's row r of the tile: an output if r < TM and (y, x) is a valid origin
+            {
+                const int r = q * 32 + lane;
+                const int P = t * TM + r;
+                long long off = -1;
+                if (r < TM && P < p.rows) {
+                    const int row = P / p.W;
+                    const int x = P - row * p.W;
+                    const int n = row / p.H;
+                    const int y = row - n * p.H;
+                    if (x < p.Wo && y < p.Ho)
+                        off = ((static_cast<long long>(n) * p.Ho + y) * p.Wo + x) * p.Cout;
+                }
+                rowoff[lane] = off;
+            }
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * NF;
+            // publish lanes 0..j-1 of groups j >= 1 for the warp above (rows 32q - K + 1 ..)
+            float *my_x = xch + (par * 4 + q) * Cfg::XCH_FLOATS;
+            if (q > 0) {
+#pragma unroll
+                for (int j = 1; j < K; ++j) {
+                    uint32_t v[4][16];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + j * 64 + g * 16, v[g]);
+                    tmem_wait_ld();
+                    if (lane < j) {
+                        float4 *dst = reinterpret_cast<float4 *>(my_x + (j * (j - 1) / 2 + lane) * 64);
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                dst[g * 4 + c] = make_float4(__uint_as_float(v[g][4 * c]), __uint_as_float(v[g][4 * c + 1]),
+                                                             __uint_as_float(v[g][4 * c + 2]), __uint_as_float(v[g][4 * c + 3]));
+                    }
+                }
+            }
+            mbar_arrive(xbar(par));
+            const float *next_x = xch + (par * 4 + (q < 3 ? q + 1 : q)) * Cfg::XCH_FLOATS;
+            bool xok = true;
+            const uint32_t row_addr = stage + lane * 128;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint32_t d[K][16];
+#pragma unroll
+                for (int j = 0; j < K; ++j) tmem_ld_32x32b_x16(t_row + j * 64 + g * 16, d[j]);
+                tmem_wait_ld();
+                if (g == 3) {   // accumulator fully read: the MMA warp may reuse it
+                    tc_fence_before();
+                    mbar_arrive(acce(b));
+                }
+                if (g == 0) xok = mbar_wait_warp(xbar(par), (local >> 1) & 1u);
+                float y[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) y[c] = __uint_as_float(d[0][c]);
+#pragma unroll
+                for (int j = 1; j < K; ++j) {
+                    const bool from_next = lane + j >= 32;
+                    const float *src = next_x + (j * (j - 1) / 2 + (lane + j - 32 < 0 ? 0 : lane + j - 32)) * 64 + g * 16;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        float v = __shfl_down_sync(0xffffffffu, __uint_as_float(d[j][c]), j);
+                        if (from_next) v = (q < 3 && xok) ? src[c] : 0.0f;
+                        y[c] = __fadd_rn(y[c], v);
+                    }
+                }
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t c = g * 2 + cc;
+                    const float *v = &y[cc * 8];
+                    st_shared_v4(row_addr + ((c ^ (lane & 7)) << 4), halo_pack_bf16x2(v[0], v[1]),
+                                 halo_pack_bf16x2(v[2], v[3]), halo_pack_bf16x2(v[4], v[5]),
+                                 halo_pack_bf16x2(v[6], v[7]));
+                }
+            }
+            if (!xok) { if (lane == 0) fail(); break; }
+            __syncwarp();
+            // coalesced stores: 8 lanes per row, 4 rows per instruction
+            const int col = (lane & 7) * 8;
+            if (col < p.Cout) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = i * 4 + (lane >> 3);
+                    const long long off = rowoff[rr];
+                    if (off >= 0) {
+                        uint32_t a, bb, c, dd;
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(a), "=r"(bb), "=r"(c), "=r"(dd)
+                                     : "r"(stage + rr * 128 + ((((lane & 7) ^ (rr & 7))) << 4)));
+                        *reinterpret_cast<uint4 *>(Y + off + col) = make_uint4(a, bb, c, dd);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+}  // namespace convb200

@@ -113,6 +113,18 @@ depthwise_reg_kernel(const float *__restrict__ x, const float *__restrict__ w,
             assemble(own, rows[ky]);
         }
     }
+    // L2 prefetch of the input rows AHEAD output rows ahead: more bytes in flight per warp
+    // without holding them in registers (one prefetch per lane per row; lanes of a 128-byte
+    // line repeat it, which is cheaper than computing a leader)
+    constexpr int AHEAD = S == 1 ? 4 : 2;
+    auto prefetch_row = [&](int r) {
+        if (lane_has_cols && r >= 0 && r < p.H)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(xp + static_cast<long long>(r) * p.W + c0));
+    };
+#pragma unroll
+    for (int a = 1; a <= AHEAD; ++a)
+#pragma unroll
+        for (int s = 0; s < S; ++s) prefetch_row((oy0 + 1 + a) * S - PAD + (K - S) + s);
     float nxt[S][OWN];
 #pragma unroll
     for (int s = 0; s < S; ++s) load_own((oy0 + 1) * S - PAD + (K - S) + s, nxt[s]);
@@ -150,6 +162,10 @@ depthwise_reg_kernel(const float *__restrict__ x, const float *__restrict__ w,
         if (i + 1 < nrows) {
 #pragma unroll
             for (int s = 0; s < S; ++s) load_own((oy + 2) * S - PAD + (K - S) + s, nxt[s]);
+            if (i + 2 + AHEAD <= nrows) {
+#pragma unroll
+                for (int s = 0; s < S; ++s) prefetch_row((oy + 2 + AHEAD) * S - PAD + (K - S) + s);
+            }
         }
     }
 }

@@ -1,0 +1,224 @@
+// Depthwise forward convolution on NCHW float32 planes: per-warp asynchronous staging into a
+// zero-padded shared-memory window, computed from a register window that never moves.
+//
+// Same contract as depthwise.cuh (the OneModel "Depthwise convolution" page, section "What
+// each output is": acc = +0; ky outer, kx inner; padding a real zero that is multiplied; exact
+// mode __fmul_rn then __fadd_rn with NaN rewritten as 0x7FC00000; fast mode one __fmaf_rn per
+// tap; the bias one rounded addition afterwards), for compile-time K x K, stride S, padding
+// PAD = (K-1)/2, dilation 1, multiplier 1.
+//
+// Work layout. Every warp runs its own pipeline over a list of jobs; a job is ppw planes x Rw
+// output rows. The warp stages a job's input window into one of its two shared-memory buffers
+// while it computes from the other. The buffer holds, per plane and staged input row, 4 zeros,
+// the row, and zeros up to the pitch Wp, so the compute loop has no bounds tests and no
+// shuffles. Rows that are 16-byte multiples arrive as one 3-D TMA box {Wp, rows, planes} whose
+// x starts at -4: the copy engine writes every zero of the padding itself (left, right, above,
+// below). Other widths are staged only as whole planes: 4-byte cp.async copies of the image
+// into buffers whose padding was zeroed once at start (it never changes, since every job
+// places its planes identically).
+//
+// Lane g of a plane owns output columns 4g .. 4g+3 and reads its input window -- input columns
+// 4gS - PAD .. 4gS - PAD + 3S + K - 1 -- straight from the buffer with the widest aligned
+// shared loads the offset allows. Input rows live in a ring of K register rows indexed by
+// (staged row mod K); the row loop is unrolled by K, so every ring index is a compile-time
+// constant and advancing the window costs only the S new rows' loads. No CTA-wide barrier:
+// warps never wait on each other. Every output is computed independently in the one tap order,
+// so results are bit-identical to the other depthwise kernels.
+#pragma once
+#include <cstdint>
+
+#include "depthwise.cuh"
+#include "ptx.cuh"
+
+namespace convb200 {
+
+struct DwTmaParams {
+    int H, W, Ho, Wo, C;   // C = Cin = Cout (multiplier 1)
+    int lpp, ppw;          // lanes per plane, planes per warp
+    int Rw;                // output rows per job (Ho when jobs are whole planes)
+    int rows_in;           // staged input rows per plane: (Rw - 1) * S + K
+    int Wp;                // buffer row pitch in floats (multiple of 4)
+    int nbands;            // row bands per plane group
+    int num_planes, num_jobs;
+    int box_floats;        // ppw * rows_in * Wp: one staged job
+    int buf_floats;        // buffer stride: box_floats rounded up to 128 bytes (TMA destinations
+                           // in shared memory must be 128-byte aligned)
+    int use_tma;           // 1: TMA box (W % 4 == 0); 0: cp.async copies of whole planes
+    int vec_out;           // 1: 128-bit output stores
+    FastDiv div_nbands, div_lpp, div_c, div_w;
+};
+
+constexpr int kDwWarpsPerCta = 4;
+
+// N consecutive floats from shared memory starting at base + A (base 16-byte aligned), with
+// the widest loads the compile-time offset allows
+template <int A, int N>
+__device__ __forceinline__ void dw_ld_span(const float *base, float *out) {
+    if constexpr (N > 0) {
+        if constexpr (A % 4 == 0 && N >= 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(base + A);
+            out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+            dw_ld_span<A + 4, N - 4>(base, out + 4);
+        } else if constexpr (A % 2 == 0 && N >= 2) {
+            const float2 v = *reinterpret_cast<const float2 *>(base + A);
+            out[0] = v.x; out[1] = v.y;
+            dw_ld_span<A + 2, N - 2>(base, out + 2);
+        } else {
+            out[0] = base[A];
+            dw_ld_span<A + 1, N - 1>(base, out + 1);
+        }
+    }
+}
+
+template <int MODE, bool HAS_BIAS, int K, int S>
+__global__ void __launch_bounds__(32 * kDwWarpsPerCta)
+depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__restrict__ x,
+                     const float *__restrict__ w, const float *__restrict__ bias, float *__restrict__ y,
+                     const DwTmaParams p, unsigned int *status) {
+    constexpr int PAD = (K - 1) / 2;
+    constexpr int VX = 4;
+    constexpr int OWN = VX * S;
+    constexpr int WIN = (VX - 1) * S + K;
+    extern __shared__ __align__(128) float sraw[];
+    __shared__ __align__(8) uint64_t full_all[kDwWarpsPerCta][2];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the dynamic region is only guaranteed 16-byte alignment: align the buffers to 128 bytes
+    const uint32_t raw_s = static_cast<uint32_t>(__cvta_generic_to_shared(sraw));
+    float *sbuf = sraw + (((raw_s + 127u) & ~127u) - raw_s) / 4u;
+    float *my_buf = sbuf + static_cast<size_t>(warp) * 2 * p.buf_floats;
+    const uint32_t buf_s = static_cast<uint32_t>(__cvta_generic_to_shared(my_buf));
+    const uint32_t full0 = static_cast<uint32_t>(__cvta_generic_to_shared(&full_all[warp][0]));
+    auto full = [&](int b) { return full0 + 8u * b; };
+
+    const int gw = blockIdx.x * kDwWarpsPerCta + warp;
+    const int GW = gridDim.x * kDwWarpsPerCta;
+
+    // stage job `job` into buffer `b`
+    auto issue = [&](int job, int b) {
+        const int pg = fdiv(job, p.div_nbands);
+        const int band = job - pg * p.nbands;
+        const int plane0 = pg * p.ppw;
+        const uint32_t dst = buf_s + 4u * b * p.buf_floats;
+        if (p.use_tma) {
+            if (lane == 0) {
+                // the box always has ppw planes; planes past the tensor arrive as zeros
+                const int iy0 = band * p.Rw * S - PAD;
+                mbar_arrive_expect_tx(full(b), 4u * p.box_floats);
+                asm volatile(
+                    "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                    " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+                    "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(full(b)), "r"(-4), "r"(iy0), "r"(plane0)
+                    : "memory");
+            }
+        } else {
+            // whole planes: image element e of plane slot s goes to staged row PAD + e / W,
+            // buffer column 4 + e % W; the padding around it is already zero
+            const int HW = p.H * p.W;
+            for (int s = 0; s < p.ppw; ++s) {
+                const int plane = plane0 + s;
+                if (plane >= p.num_planes) break;
+                const float *src = x + static_cast<long long>(plane) * HW;
+                const uint32_t dplane = dst + 4u * (s * p.rows_in + PAD) * p.Wp + 16u;
+                for (int e = lane; e < HW; e += 32) {
+                    const int r = fdiv(e, p.div_w);
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dplane + 4u * (r * p.Wp + e - r * p.W)),
+                                 "l"(src + e)
+                                 : "memory");
+                }
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared.b64 [%0];" ::"r"(full(b)) : "memory");
+        }
+    };
+
+    if (lane == 0) {
+        mbar_init(full(0), p.use_tma ? 1 : 32);
+        mbar_init(full(1), p.use_tma ? 1 : 32);
+        fence_barrier_init();
+        if (p.use_tma) prefetch_tensormap(&tmx);
+    }
+    if (!p.use_tma) {   // zero both buffers once: the padding of whole-plane jobs never changes
+        float4 *z = reinterpret_cast<float4 *>(my_buf);
+        for (int i = lane; i < p.buf_floats / 2; i += 32) z[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+    __syncwarp();
+    if (gw < p.num_jobs) issue(gw, 0);
+    if (gw + GW < p.num_jobs) issue(gw + GW, 1);
+
+    // lane geometry (fixed for the kernel's life)
+    const int ps = fdiv(lane, p.div_lpp);
+    const int cg = lane - ps * p.lpp;
+    const bool lane_ok = ps < p.ppw;
+    const int ox = cg * VX;
+    const int c0 = cg * OWN;   // first input column this lane owns: buffer column c0 + 4
+
+    int k = 0;
+    bool ok = true;
+    for (int job = gw; job < p.num_jobs; job += GW, ++k) {
+        const int b = k & 1;
+        if (!mbar_wait_warp(full(b), (k >> 1) & 1)) { ok = false; break; }
+        const int pg = fdiv(job, p.div_nbands);
+        const int band = job - pg * p.nbands;
+        const int oy0 = band * p.Rw;
+        const int nrows = min(p.Rw, p.Ho - oy0);
+        const int plane = pg * p.ppw + (lane_ok ? ps : 0);
+        const bool active = lane_ok && plane < p.num_planes;
+        const int c = active ? plane - fdiv(plane, p.div_c) * p.C : 0;
+        float wr[K * K];
+#pragma unroll
+        for (int t = 0; t < K * K; ++t) wr[t] = __ldg(w + c * (K * K) + t);
+        const float bv = HAS_BIAS ? __ldg(bias + c) : 0.0f;
+        // staged row r of this lane's plane; buffer column c0 + 4 - PAD is input column c0 - PAD
+        const float *pb = my_buf + b * p.buf_floats + (lane_ok ? ps : 0) * (p.rows_in * p.Wp) + c0;
+        float *yp = y + (static_cast<long long>(active ? plane : 0) * p.Ho + oy0) * p.Wo + ox;
+
+        float ring[K][WIN];
+#pragma unroll
+        for (int r = 0; r < K - S; ++r) dw_ld_span<4 - PAD, WIN>(pb + r * p.Wp, ring[r]);
+
+        for (int base = 0; base < nrows; base += K) {
+#pragma unroll
+            for (int u = 0; u < K; ++u) {
+                const int i = base + u;
+                if (i < nrows) {
+                    // staged rows i*S + K - S .. i*S + K - 1 complete the window of output row i
+                    // (base is a multiple of K, so row r sits in ring slot (u*S + r - i*S) % K)
+#pragma unroll
+                    for (int s = 0; s < S; ++s)
+                        dw_ld_span<4 - PAD, WIN>(pb + (i * S + K - S + s) * p.Wp, ring[(u * S + K - S + s) % K]);
+                    float acc[VX];
+#pragma unroll
+                    for (int v = 0; v < VX; ++v) {
+                        float a = 0.0f;
+#pragma unroll
+                        for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                            for (int kx = 0; kx < K; ++kx)
+                                a = dw_tap<MODE>(a, wr[ky * K + kx], ring[(u * S + ky) % K][v * S + kx]);
+                        acc[v] = dw_finish<MODE, HAS_BIAS>(a, bv);
+                    }
+                    if (active) {
+                        float *dst = yp + static_cast<long long>(i) * p.Wo;
+                        if (p.vec_out && ox + VX <= p.Wo) {
+                            *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < VX; ++v)
+                                if (ox + v < p.Wo) dst[v] = acc[v];
+                        }
+                    }
+                }
+            }
+        }
+        // every lane is done with buffer b; refill it two jobs ahead
+        __syncwarp();
+        if (job + 2 * GW < p.num_jobs) issue(job + 2 * GW, b);
+    }
+    if (!ok) {
+        if (lane == 0) atomicOr(status, kStatusTimeout);
+        // drain: copies still in flight land before the warp exits (bounded waits)
+        for (int kk = k; kk < k + 2; ++kk)
+            if (gw + kk * GW < p.num_jobs) mbar_wait_warp(full(kk & 1), (kk >> 1) & 1);
+    }
+}
+
+}  // namespace convb200

@@ -105,6 +105,24 @@ const char *conv_status_string(int status);
  */
 int conv_device_status(cudaStream_t stream, int reset);
 
+/*
+ * Name of the kernel family the last successful conv2d_nhwc_fwd, conv2d_nhwc_fwd_f32 or
+ * depthwise_fwd call on the calling host thread launched ("dense_halo_kernel",
+ * "dense_tc_kernel", "dense_direct_kernel", "depthwise_tma_kernel", "depthwise_reg_kernel",
+ * "depthwise_kernel"); "" before the first one. Static storage, never NULL. Host only: it
+ * reports the dispatcher's choice, it does not wait for the kernel.
+ */
+const char *conv_last_kernel(void);
+
+/*
+ * Diagnostic for the bounded device waits: launches one CTA that waits, with the same bounded
+ * wait every kernel of the library uses, on a shared-memory barrier that nothing completes.
+ * After about one second of SM clock cycles the wait gives up, the kernel records
+ * CONV_ERR_DEVICE_TIMEOUT in the device status word and returns normally; the CUDA context
+ * stays usable. Returns the launch status; read the outcome with conv_device_status().
+ */
+int conv_selftest_wait_timeout(cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

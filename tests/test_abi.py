@@ -98,3 +98,9 @@ def test_python_binding_rejects_cpu_tensors():
         cb.conv2d_nhwc_fwd(torch.zeros(1, 5, 5, 8, dtype=torch.bfloat16), torch.zeros(3, 3, 8, 8, dtype=torch.bfloat16))
     with pytest.raises(ValueError):
         cb.depthwise_fwd(torch.zeros(1, 2, 5, 5), torch.zeros(2, 3, 3))
+
+
+def test_last_kernel_is_empty_before_any_launch():
+    # rejected calls launch nothing, so the dispatcher's record stays empty on a CPU-only host
+    assert cb.lib.conv2d_nhwc_fwd(None, F, Y, 1, 5, 5, 8, 8, 3, None) == cb.CONV_ERR_INVALID_ARG
+    assert cb.conv_last_kernel() == ""

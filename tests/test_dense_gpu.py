@@ -116,7 +116,7 @@ def test_pins_tensor_core_path(cb):
     F[:, :, 3, 1] = np.array(so["gx"], np.float32)
     F[:, :, 3, 2] = np.array(so["gy"], np.float32)
     exp0 = workloads.bf16_to_f32(workloads.bf16_bits(np.array(g["output"], np.float32)))
-    for path in ("halo64", "bn64"):   # the halo kernel and the im2col kernel
+    for path in ("fold", "halo64", "bn64"):   # folded-tap, halo and im2col kernels
         y = _run_bf16(cb, workloads.bf16_bits(X), workloads.bf16_bits(F), env=path)
         for n in (0, 1, 100, N - 1):
             assert np.array_equal(y[n, :, :, 0], exp0), path
@@ -286,3 +286,47 @@ def test_noncontiguous_rejected_and_contiguous_copy_works(cb):
     y = _host_bf16(cb.conv2d_nhwc_fwd(Xt.contiguous(), _dev_bf16(Fb)))
     torch.cuda.synchronize()
     _check_bf16(y, np.ascontiguousarray(Xb.transpose(0, 2, 1, 3)), Fb)
+
+
+def test_dispatcher_choices(cb):
+    # Cout <= 64 with K = 3 -> folded-tap kernel; wider Cout with a resident filter -> halo
+    # kernel; channels not multiples of 8 -> CUDA-core kernel; a forced im2col tile width ->
+    # im2col kernel
+    Xb, Fb = _case_inputs(2, 20, 20, 64, 64, 3, seed=21)
+    _run_bf16(cb, Xb, Fb)
+    assert cb.conv_last_kernel() == "dense_fold_kernel"
+    Xb, Fb = _case_inputs(2, 20, 20, 64, 128, 3, seed=24)
+    _run_bf16(cb, Xb, Fb)
+    assert cb.conv_last_kernel() == "dense_halo_kernel"
+    Xb2, Fb2 = _case_inputs(1, 7, 9, 3, 5, 3, seed=22)
+    _run_bf16(cb, Xb2, Fb2)
+    assert cb.conv_last_kernel() == "dense_direct_kernel"
+    Xb3, Fb3 = _case_inputs(4, 40, 40, 64, 128, 3, seed=23)     # input above 128 KiB
+    _run_bf16(cb, Xb3, Fb3, env="bn128")
+    assert cb.conv_last_kernel() == "dense_tc_kernel"
+
+
+# (N, H, W, Cin, Cout, K): the folded-tap kernel (Cout <= 64, K = 2..4, resident filter):
+# ragged last tile, Cout below one 64-column group, several channel blocks, a halo spanning
+# several TMA boxes (128 + (K-1)*W > 256 rows), one image smaller than a tile
+FOLD_SHAPES = [(2, 20, 20, 64, 64, 3), (3, 9, 13, 16, 8, 2), (2, 17, 11, 128, 40, 2), (1, 30, 70, 32, 64, 3),
+               (2, 12, 12, 8, 64, 4), (1, 4, 4, 64, 24, 4), (4, 40, 40, 64, 64, 3)]
+
+
+@pytest.mark.parametrize("shape", FOLD_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_folded_taps(cb, shape):
+    N, H, W, Cin, Cout, K = shape
+    Xb, Fb = _case_inputs(N, H, W, Cin, Cout, K, seed=sum(shape) + 7)
+    y = _run_bf16(cb, Xb, Fb, env="fold")
+    assert cb.conv_last_kernel() == "dense_fold_kernel"
+    _check_bf16(y, Xb, Fb)
+
+
+@pytest.mark.parametrize("shape", [(1, 9, 9, 64, 64, 1), (1, 9, 9, 64, 64, 5), (1, 9, 9, 64, 72, 3)],
+                         ids=["K1", "K5", "Cout72"])
+def test_folded_taps_refuses_other_shapes(cb, shape):
+    N, H, W, Cin, Cout, K = shape
+    Xb, Fb = _case_inputs(N, H, W, Cin, Cout, K, seed=3)
+    with pytest.raises(cb.ConvError) as e:
+        _run_bf16(cb, Xb, Fb, env="fold")
+    assert e.value.code == cb.CONV_ERR_UNSUPPORTED

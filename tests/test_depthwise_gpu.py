@@ -230,3 +230,63 @@ def test_register_kernel_refuses_other_shapes(cb):
     with pytest.raises(cb.ConvError) as e:
         _with_env("CONV_B200_DW_KERNEL", "reg", lambda: _gpu(cb, x, w, None, 1, 0, 1, 0))   # pad 0
     assert e.value.code == cb.CONV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("case", workloads.DW_SWEEP, ids=lambda c: c.name)
+def test_tma_staged_and_shared_kernels_identical(cb, case):
+    # the TMA-staged kernel (the default for multiplier 1) against the shared-memory kernel:
+    # identical bits, both equal to the oracle; batch 3 leaves a ragged last job
+    small = workloads.DepthwiseCase(case.name, 3, case.C, 1, case.H, case.W, case.KH, case.KW, case.stride,
+                                    case.pad, case.dil, True, 12)
+    x, w, b = workloads.depthwise_inputs(small)
+    for mode in MODES:
+        yt = _with_env("CONV_B200_DW_KERNEL", "tma",
+                       lambda: _gpu(cb, x, w, b, small.stride, small.pad, small.dil, mode))
+        ys = _with_env("CONV_B200_DW_KERNEL", "smem",
+                       lambda: _gpu(cb, x, w, b, small.stride, small.pad, small.dil, mode))
+        assert np.array_equal(_bits(yt), _bits(ys))
+        _compare(yt, x, w, b, 1, small.stride, small.pad, small.dil, mode)
+
+
+# (N, C, H, W, K, S): TMA bands with a ragged last band; TMA bands with fewer planes than a
+# warp's group (the box's missing planes arrive as zeros); a small plane split in two bands;
+# whole planes through cp.async (rows not 16-byte multiples), with a partial last group
+TMA_SHAPES = [(2, 5, 36, 20, 3, 1), (1, 7, 13, 12, 5, 2), (3, 10, 8, 8, 3, 1), (2, 6, 10, 10, 3, 2),
+              (1, 3, 7, 7, 5, 1), (2, 3, 14, 14, 3, 1), (1, 2, 40, 24, 5, 2)]
+
+
+@pytest.mark.parametrize("shape", TMA_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_tma_staged_job_modes(cb, shape):
+    N, C, H, W, K, S = shape
+    case = workloads.DepthwiseCase("tma", N, C, 1, H, W, K, K, S, (K - 1) // 2, 1, True, 13)
+    x, w, b = workloads.depthwise_inputs(case)
+    for mode in MODES:
+        yt = _with_env("CONV_B200_DW_KERNEL", "tma", lambda: _gpu(cb, x, w, b, S, case.pad, 1, mode))
+        assert cb.conv_last_kernel() == "depthwise_tma_kernel"
+        ys = _with_env("CONV_B200_DW_KERNEL", "smem", lambda: _gpu(cb, x, w, b, S, case.pad, 1, mode))
+        assert cb.conv_last_kernel() == "depthwise_kernel"
+        assert np.array_equal(_bits(yt), _bits(ys))
+        _compare(yt, x, w, b, 1, S, case.pad, 1, mode)
+
+
+def test_dispatcher_choices(cb):
+    x, w, b = workloads.depthwise_inputs(
+        workloads.DepthwiseCase("d", 1, 8, 1, 16, 16, 3, 3, 1, 1, 1, True, 14))
+    _gpu(cb, x, w, b, 1, 1, 1, 0)
+    assert cb.conv_last_kernel() == "depthwise_tma_kernel"     # multiplier 1, K 3, 'same' padding
+    x2, w2, b2 = workloads.depthwise_inputs(
+        workloads.DepthwiseCase("d", 1, 8, 2, 16, 16, 3, 3, 1, 1, 1, True, 14))
+    _gpu(cb, x2, w2, b2, 1, 1, 1, 0)
+    assert cb.conv_last_kernel() == "depthwise_reg_kernel"     # multiplier 2
+    _gpu(cb, x, w, b, 1, 0, 1, 0)
+    assert cb.conv_last_kernel() == "depthwise_kernel"         # no padding
+
+
+def test_forced_tma_refuses_unaligned_planes(cb):
+    # rows of 66 floats are not 16-byte multiples, and a 64 x 66 plane is too large to stage
+    # whole, so the staged kernel is not eligible
+    x = np.ones((1, 2, 64, 66), np.float32)
+    w = np.ones((2, 3, 3), np.float32)
+    with pytest.raises(cb.ConvError) as e:
+        _with_env("CONV_B200_DW_KERNEL", "tma", lambda: _gpu(cb, x, w, None, 1, 1, 1, 0))
+    assert e.value.code == cb.CONV_ERR_UNSUPPORTED
