@@ -10,6 +10,9 @@ The arithmetic lives in ``conv_oracle.c`` (plain C, OpenMP over independent outp
   DLSys Lecture 14 notes ("The hidden copy behind convolution as matrix multiplication",
   section 1), accumulated in float64, with the per-output absolute sum sum|x||f| that the
   dense tolerance is scaled by.
+* ``conv2d_nhwc_ex`` -- the same sum with the stride, zero-padding, dilation and bias variants
+  of "Convolution Is Wx+b Moving Across a Signal" (output-size rule of section "Build an
+  image-gradient map, one number at a time"), float64.
 * ``depthwise`` -- the per-output loop of the OneModel "Depthwise convolution" page
   (section "What each output is"), in IEEE float32 in the page's order, exact or fast mode.
 
@@ -59,6 +62,10 @@ def _load():
         lib.oracle_conv2d_nhwc.restype = None
         lib.oracle_conv2d_nhwc_points.argtypes = [P, P, P, L, P, P] + [I] * 6
         lib.oracle_conv2d_nhwc_points.restype = None
+        lib.oracle_conv2d_nhwc_ex.argtypes = [P, P, P, P, P] + [I] * 9
+        lib.oracle_conv2d_nhwc_ex.restype = I
+        lib.oracle_conv2d_nhwc_ex_points.argtypes = [P, P, P, P, L, P, P] + [I] * 9
+        lib.oracle_conv2d_nhwc_ex_points.restype = I
         lib.oracle_depthwise.argtypes = [P, P, P, P] + [I] * 11
         lib.oracle_depthwise.restype = I
         lib.oracle_depthwise_points.argtypes = [P, P, P, P, L, P] + [I] * 11
@@ -111,6 +118,52 @@ def conv2d_nhwc_points(X, F, flat_idx):
     a = np.empty(idx.size, dtype=np.float64)
     _load().oracle_conv2d_nhwc_points(_ptr(X), _ptr(F), _ptr(idx), idx.size, _ptr(y), _ptr(a),
                                       N, H, W, Cin, Cout, K)
+    return y, a
+
+
+def _dense_ex_shape(X, F, bias, stride, pad, dil):
+    N, H, W, Cin = X.shape
+    K, K2, Cin2, Cout = F.shape
+    if K != K2 or Cin != Cin2 or min(N, H, W, Cin, K, Cout, stride, dil) <= 0 or pad < 0:
+        raise ValueError("incompatible input and square filter")
+    if bias is not None and bias.shape != (Cout,):
+        raise ValueError("bias must have Cout entries")
+    Ho = (H + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    Wo = (W + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    return N, H, W, Cin, Cout, K, Ho, Wo
+
+
+def conv2d_nhwc_ex(X, F, bias=None, stride=1, pad=0, dil=1):
+    """Dense NHWC forward convolution with stride, symmetric zero padding, dilation and a
+    per-output-channel bias, in float64 (the variants of "Convolution Is Wx+b Moving Across a
+    Signal": output size per axis floor((in + 2*pad - (dil*(K-1)+1)) / stride) + 1, window of
+    output (y, x) starting at (y*stride - pad, x*stride - pad), tap (i, j) dil*i rows and dil*j
+    columns on, zeros outside the image, bias added to the sum).
+
+    Returns (Y, abssum), float64 [N, Ho, Wo, Cout]; abssum = sum|x||f| + |b|.
+    """
+    X, F = _f32(X), _f32(F)
+    b = None if bias is None else _f32(bias)
+    N, H, W, Cin, Cout, K, Ho, Wo = _dense_ex_shape(X, F, b, stride, pad, dil)
+    Y = np.empty((N, Ho, Wo, Cout), dtype=np.float64)
+    A = np.empty_like(Y)
+    _load().oracle_conv2d_nhwc_ex(_ptr(X), _ptr(F), _ptr(b), _ptr(Y), _ptr(A), N, H, W, Cin, Cout, K,
+                                  stride, pad, dil)
+    return Y, A
+
+
+def conv2d_nhwc_ex_points(X, F, flat_idx, bias=None, stride=1, pad=0, dil=1):
+    """Selected outputs of conv2d_nhwc_ex, by flat index into [N, Ho, Wo, Cout]."""
+    X, F = _f32(X), _f32(F)
+    b = None if bias is None else _f32(bias)
+    N, H, W, Cin, Cout, K, Ho, Wo = _dense_ex_shape(X, F, b, stride, pad, dil)
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    y = np.empty(idx.size, dtype=np.float64)
+    a = np.empty(idx.size, dtype=np.float64)
+    _load().oracle_conv2d_nhwc_ex_points(_ptr(X), _ptr(F), _ptr(b), _ptr(idx), idx.size, _ptr(y), _ptr(a),
+                                         N, H, W, Cin, Cout, K, stride, pad, dil)
     return y, a
 
 

@@ -104,6 +104,88 @@ void oracle_conv2d_nhwc_points(const float *X, const float *F, const int64_t *id
 }
 
 /* ---------------------------------------------------------------------------------- */
+/* Dense with stride, zero padding, dilation and bias                                  */
+/* ---------------------------------------------------------------------------------- */
+/*
+ * The same sum with the variants of "Convolution Is Wx+b Moving Across a Signal": output size
+ * per axis from section "Build an image-gradient map, one number at a time",
+ *   Ho = floor((H + 2*pad - (dil*(K-1) + 1)) / stride) + 1   (Wo likewise),
+ * the window of output (y, x) starting at input row y*stride - pad and column x*stride - pad,
+ * filter tap (i, j) reading dil*i rows and dil*j columns further on (the pseudocode of section
+ * "Find the same sum in CKE's C kernels" indexes out*stride + tap - padding), positions outside
+ * the image reading zero, and a per-output-channel bias added to the sum. Float64; abssum is
+ * sum|x||f| + |b| over the same terms.
+ */
+static long dense_out_size(long in, int k, int stride, int pad, int dil)
+{
+    long eff = (long)dil * (k - 1) + 1;
+    return (in + 2L * pad - eff) / stride + 1;
+}
+
+static void dense_ex_one(const float *X, const float *F, const float *bias, int H, int W, int Cin,
+                         int Cout, int K, int stride, int pad, int dil, long n, long y, long x, long o,
+                         double *out, double *abs_out)
+{
+    double s = 0.0, a = 0.0;
+    for (int i = 0; i < K; ++i)
+        for (int j = 0; j < K; ++j) {
+            long r = y * stride + (long)i * dil - pad;
+            long q = x * stride + (long)j * dil - pad;
+            if (r < 0 || r >= H || q < 0 || q >= W) continue;   /* zero padding */
+            for (int c = 0; c < Cin; ++c) {
+                double xv = X[((n * H + r) * W + q) * Cin + c];
+                double fv = F[(((long)i * K + j) * Cin + c) * Cout + o];
+                s += xv * fv;
+                a += fabs(xv) * fabs(fv);
+            }
+        }
+    if (bias) {
+        s += (double)bias[o];
+        a += fabs((double)bias[o]);
+    }
+    *out = s;
+    *abs_out = a;
+}
+
+/* Full output Y[N][Ho][Wo][Cout]. Returns 0, or -1 when the output would be empty. */
+int oracle_conv2d_nhwc_ex(const float *X, const float *F, const float *bias, double *Y, double *abssum,
+                          int N, int H, int W, int Cin, int Cout, int K, int stride, int pad, int dil)
+{
+    const long Ho = dense_out_size(H, K, stride, pad, dil), Wo = dense_out_size(W, K, stride, pad, dil);
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (long n = 0; n < N; ++n)
+        for (long y = 0; y < Ho; ++y)
+            for (long x = 0; x < Wo; ++x)
+                for (long o = 0; o < Cout; ++o) {
+                    long t = ((n * Ho + y) * Wo + x) * Cout + o;
+                    double a;
+                    dense_ex_one(X, F, bias, H, W, Cin, Cout, K, stride, pad, dil, n, y, x, o, &Y[t], &a);
+                    if (abssum) abssum[t] = a;
+                }
+    return 0;
+}
+
+/* Selected outputs, given as flat indices into Y[N][Ho][Wo][Cout]. */
+int oracle_conv2d_nhwc_ex_points(const float *X, const float *F, const float *bias, const int64_t *idx,
+                                 int64_t npts, double *y, double *abssum, int N, int H, int W, int Cin,
+                                 int Cout, int K, int stride, int pad, int dil)
+{
+    const long Ho = dense_out_size(H, K, stride, pad, dil), Wo = dense_out_size(W, K, stride, pad, dil);
+    (void)N;
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t p = 0; p < npts; ++p) {
+        long t = idx[p];
+        long o = t % Cout; t /= Cout;
+        long x = t % Wo; t /= Wo;
+        long yy = t % Ho; t /= Ho;
+        dense_ex_one(X, F, bias, H, W, Cin, Cout, K, stride, pad, dil, t, yy, x, o, &y[p], &abssum[p]);
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------- */
 /* Depthwise                                                                           */
 /* ---------------------------------------------------------------------------------- */
 

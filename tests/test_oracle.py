@@ -211,6 +211,144 @@ def test_dense_points_match_full():
     assert np.array_equal(y, Y.ravel()[idx]) and np.array_equal(a, A.ravel()[idx])
 
 
+# ------------------------------------------------------------------------------------------
+# Dense with stride, zero padding, dilation and bias ("Convolution Is Wx+b Moving Across a
+# Signal"): each variant pinned to the plain definition composed with a numpy reshaping that
+# has its own textbook meaning (zero-padded input, subsampled output, zero-inserted filter)
+# ------------------------------------------------------------------------------------------
+
+
+def _dilate_filter(F, d):
+    K = F.shape[0]
+    Kd = d * (K - 1) + 1
+    out = np.zeros((Kd, Kd) + F.shape[2:], dtype=F.dtype)
+    out[::d, ::d] = F
+    return out
+
+
+def test_dense_ex_defaults_are_the_plain_definition():
+    X = _ints(61, (2, 7, 9, 3))
+    F = _ints(62, (3, 3, 3, 4))
+    Y, A = oracle.conv2d_nhwc_ex(X, F)
+    Y0, A0 = oracle.conv2d_nhwc(X, F)
+    assert np.array_equal(Y, Y0) and np.array_equal(A, A0)
+
+
+@pytest.mark.parametrize("pad", [1, 2, 4])
+def test_dense_ex_padding_is_a_zero_padded_input(pad):
+    X = _ints(63, (2, 6, 5, 3))
+    F = _ints(64, (3, 3, 3, 2))
+    Y, _ = oracle.conv2d_nhwc_ex(X, F, pad=pad)
+    Xp = np.pad(X, ((0, 0), (pad, pad), (pad, pad), (0, 0)))
+    ref, _ = oracle.conv2d_nhwc(Xp, F)
+    assert np.array_equal(Y, ref)
+
+
+@pytest.mark.parametrize("stride", [2, 3])
+def test_dense_ex_stride_subsamples_the_output(stride):
+    X = _ints(65, (2, 11, 10, 3))
+    F = _ints(66, (3, 3, 3, 2))
+    Y, _ = oracle.conv2d_nhwc_ex(X, F, stride=stride)
+    ref, _ = oracle.conv2d_nhwc(X, F)
+    assert np.array_equal(Y, ref[:, ::stride, ::stride, :])
+
+
+@pytest.mark.parametrize("dil", [2, 3])
+def test_dense_ex_dilation_is_a_zero_inserted_filter(dil):
+    X = _ints(67, (1, 12, 13, 2))
+    F = _ints(68, (3, 3, 2, 3))
+    Y, _ = oracle.conv2d_nhwc_ex(X, F, dil=dil)
+    ref, _ = oracle.conv2d_nhwc(X, _dilate_filter(F, dil))
+    assert np.array_equal(Y, ref)
+
+
+def test_dense_ex_bias_is_added_per_output_channel():
+    X = _ints(69, (2, 6, 6, 3))
+    F = _ints(70, (3, 3, 3, 4))
+    b = np.array([1.0, -2.0, 0.5, 3.0], dtype=np.float32)
+    Y, A = oracle.conv2d_nhwc_ex(X, F, bias=b)
+    Y0, A0 = oracle.conv2d_nhwc(X, F)
+    assert np.array_equal(Y, Y0 + b) and np.array_equal(A, A0 + np.abs(b))
+
+
+@pytest.mark.parametrize("stride,pad,dil", [(2, 1, 1), (2, 2, 2), (3, 1, 2), (1, 3, 3)])
+def test_dense_ex_all_variants_compose(stride, pad, dil):
+    X = _ints(71, (2, 13, 11, 3))
+    F = _ints(72, (3, 3, 3, 2))
+    b = np.array([0.25, -1.0], dtype=np.float32)
+    Y, _ = oracle.conv2d_nhwc_ex(X, F, bias=b, stride=stride, pad=pad, dil=dil)
+    Xp = np.pad(X, ((0, 0), (pad, pad), (pad, pad), (0, 0)))
+    ref, _ = oracle.conv2d_nhwc(Xp, _dilate_filter(F, dil))
+    ref = ref[:, ::stride, ::stride, :] + b
+    assert np.array_equal(Y, ref)
+
+
+def test_dense_ex_matches_torch_conv2d_f64():
+    X = workloads.normal(73, 2 * 15 * 14 * 5, 1.0).reshape(2, 15, 14, 5)
+    F = workloads.normal(74, 3 * 3 * 5 * 6, 0.3).reshape(3, 3, 5, 6)
+    b = workloads.normal(75, 6, 0.5)
+    Y, A = oracle.conv2d_nhwc_ex(X, F, bias=b, stride=2, pad=1, dil=2)
+    x = torch.from_numpy(np.asarray(X, dtype=np.float64)).permute(0, 3, 1, 2)
+    f = torch.from_numpy(np.asarray(F, dtype=np.float64)).permute(3, 2, 0, 1)
+    ref = torch.nn.functional.conv2d(x, f, torch.from_numpy(np.asarray(b, dtype=np.float64)), stride=2, padding=1,
+                                     dilation=2).permute(0, 2, 3, 1).numpy()
+    assert Y.shape == ref.shape
+    assert np.all(np.abs(Y - ref) <= 1e-13 * A)
+
+
+def test_dense_ex_output_size_rule():
+    # "Build an image-gradient map, one number at a time": five inputs, a width-three filter,
+    # no padding, stride and dilation one give 5 - 3 + 1 = 3 positions; the general rule is
+    # floor((in + 2*pad - (dil*(k-1) + 1)) / stride) + 1 per axis
+    X = np.zeros((1, 3, 5, 1), np.float32)
+    F = np.zeros((3, 3, 1, 1), np.float32)
+    assert oracle.conv2d_nhwc_ex(X, F)[0].shape == (1, 1, 3, 1)
+    X = np.zeros((1, 17, 23, 1), np.float32)
+    for stride in (1, 2, 3):
+        for pad in (0, 1, 2):
+            for dil in (1, 2):
+                Y, _ = oracle.conv2d_nhwc_ex(X, F, stride=stride, pad=pad, dil=dil)
+                eff = dil * 2 + 1
+                assert Y.shape[1:3] == ((17 + 2 * pad - eff) // stride + 1, (23 + 2 * pad - eff) // stride + 1)
+
+
+def test_dense_ex_weighted_sum_with_bias_example():
+    # the page's first window with bias: x = 1..5, k = (2, 0, -1), b = 1 -> (0, 1, 2)
+    e = _golden("wxb_1d_examples.json")["weighted_sum_with_bias"]
+    X, F = _embed_1d(e["x"], [e["k"]])
+    Y, _ = oracle.conv2d_nhwc_ex(X, F, bias=np.array([e["bias"]], np.float32))
+    assert np.array_equal(Y[0, 0, :, 0], np.array(e["output"], dtype=np.float64))
+    e = _golden("wxb_1d_examples.json")["two_filters_with_bias"]
+    X, F = _embed_1d(e["x"], e["filters"])
+    Y, _ = oracle.conv2d_nhwc_ex(X, F, bias=np.array(e["bias"], np.float32))
+    for o in range(2):
+        assert np.array_equal(Y[0, 0, :, o], np.array(e["output_per_filter"][o], dtype=np.float64))
+
+
+def test_dense_ex_patch_projection_is_flattened_patches_times_weights():
+    # "Why variants matter": kernel = stride = P turns each non-overlapping P x P patch into one
+    # output; with corresponding weights and bias it equals flattened patches times a
+    # [P*P*Cin, D] matrix plus the bias
+    N, P, G, C, D = 2, 4, 3, 3, 5
+    X = _ints(76, (N, G * P, G * P, C)).astype(np.float64)
+    F = _ints(77, (P, P, C, D)).astype(np.float64)
+    b = np.array([1.0, 2.0, -1.0, 0.5, 0.0])
+    Y, _ = oracle.conv2d_nhwc_ex(X, F, bias=b, stride=P)
+    patches = X.reshape(N, G, P, G, P, C).transpose(0, 1, 3, 2, 4, 5).reshape(N * G * G, P * P * C)
+    ref = (patches @ F.reshape(P * P * C, D) + b).reshape(N, G, G, D)
+    assert np.array_equal(Y, ref)
+
+
+def test_dense_ex_points_match_full():
+    X = _ints(78, (2, 9, 8, 3))
+    F = _ints(79, (3, 3, 3, 4))
+    b = np.array([1, 2, 3, 4], np.float32)
+    Y, A = oracle.conv2d_nhwc_ex(X, F, bias=b, stride=2, pad=1, dil=2)
+    idx = np.arange(Y.size, dtype=np.int64)[::7]
+    y, a = oracle.conv2d_nhwc_ex_points(X, F, idx, bias=b, stride=2, pad=1, dil=2)
+    assert np.array_equal(y, Y.reshape(-1)[idx]) and np.array_equal(a, A.reshape(-1)[idx])
+
+
 def test_dense_rejects_incompatible_shapes():
     with pytest.raises(ValueError):
         oracle.conv2d_nhwc(np.zeros((1, 3, 3, 2), np.float32), np.zeros((4, 4, 2, 1), np.float32))
