@@ -24,6 +24,7 @@ dense, the depthwise sweep in both modes) as secondary measurements.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -50,7 +51,8 @@ def workload_table():
     others exist so any single kernel can be timed or profiled alone."""
     t = {"dense3x3": ("dense", workloads.DENSE_3X3, None),
          "pointwise": ("dense", workloads.DENSE_1X1, None),
-         "dense-large": ("dense", workloads.DENSE_LARGE, None)}
+         "dense-large": ("dense", workloads.DENSE_LARGE, None),
+         "dense-s2": ("dense", workloads.DENSE_S2, None)}
     for c in workloads.DW_SWEEP:
         for mode, name in ((0, "exact"), (1, "fast")):
             t[f"dw-C{c.C}-K{c.KH}-s{c.stride}-H{c.H}-{name}"] = ("depthwise", c, mode)
@@ -272,12 +274,26 @@ def time_graph_steps(singles, cycle, steps: int, warmup: int, dist=None, sampler
 # Our arm
 # ------------------------------------------------------------------------------------------
 def dense_device_inputs(torch, case, seed):
-    """Seeded bf16 X, F generated on the device (for the secondary measurements)."""
+    """Seeded bf16 X, F (and the float32 bias, if the case has one) generated on the device
+    (for the secondary measurements)."""
     g = torch.Generator(device="cuda").manual_seed(seed)
     X = torch.randn((case.N, case.H, case.W, case.Cin), device="cuda", generator=g).to(torch.bfloat16)
     F = (torch.randn((case.K, case.K, case.Cin, case.Cout), device="cuda", generator=g)
          / math.sqrt(case.K * case.K * case.Cin)).to(torch.bfloat16)
-    return X, F
+    b = torch.randn((case.Cout,), device="cuda", generator=g) * math.sqrt(0.1) if case.bias else None
+    return X, F, b
+
+
+def dense_plain(case):
+    return case.stride == 1 and case.pad == 0 and case.dil == 1 and not case.bias
+
+
+def dense_call(cb, case, X, F, b, Y):
+    """The public entry a user calls for this case: the plain one, or the one with stride,
+    padding, dilation and bias."""
+    if dense_plain(case):
+        return cb.conv2d_nhwc_fwd(X, F, Y)
+    return cb.conv2d_nhwc_fwd_ex(X, F, b, Y, case.stride, case.pad, case.dil)
 
 
 def dw_device_inputs(torch, case, seed):
@@ -293,13 +309,13 @@ def steps_fns(cb, torch, kind, case, mode, inputs):
     """R rotating buffer sets (total at least twice the L2) and one C-ABI call per set."""
     R = rotating_sets(case.bytes)
     if kind == "dense":
-        X0, F0 = inputs
+        X0, F0, b0 = inputs
         Xs = [X0.clone() for _ in range(R)]
         Fs = [F0.clone() for _ in range(R)]
         Ys = [torch.empty((case.N, case.Ho, case.Wo, case.Cout), dtype=X0.dtype, device=X0.device)
               for _ in range(R)]
-        fns = [(lambda i=i: cb.conv2d_nhwc_fwd(Xs[i], Fs[i], Ys[i])) for i in range(R)]
-        keep = (Xs, Fs, Ys)
+        fns = [(lambda i=i: dense_call(cb, case, Xs[i], Fs[i], b0, Ys[i])) for i in range(R)]
+        keep = (Xs, Fs, Ys, b0)
     else:
         x0, w0, b0 = inputs
         xs = [x0.clone() for _ in range(R)]
@@ -333,7 +349,7 @@ def e2e_bench(cb, torch, kind, case, mode, host, steps, warmup):
             if h is not None:
                 d.copy_(h, non_blocking=True)
         if kind == "dense":
-            cb.conv2d_nhwc_fwd(dev[0], dev[1], out)
+            dense_call(cb, case, dev[0], dev[1], dev[2], out)
         else:
             cb.depthwise_fwd(dev[0], dev[1], dev[2], out, case.stride, case.pad, case.dil, mode)
         out_h.copy_(out, non_blocking=True)
@@ -364,8 +380,11 @@ def cpu_baseline(kind, case, mode, host_np, budget_s=10.0):
     while (time.perf_counter() - t0) < budget_s:
         i = n % case.N
         if kind == "dense":
-            X, F = host_np
-            oracle.conv2d_nhwc(X[i:i + 1], F)
+            X, F, b = host_np
+            if dense_plain(case):
+                oracle.conv2d_nhwc(X[i:i + 1], F)
+            else:
+                oracle.conv2d_nhwc_ex(X[i:i + 1], F, b, case.stride, case.pad, case.dil)
             done += case.flops / case.N
         else:
             x, w, b = host_np
@@ -384,10 +403,12 @@ def cpu_baseline(kind, case, mode, host_np, budget_s=10.0):
 def host_inputs(torch, kind, case, seed):
     """Seeded host inputs from the workloads generators, as numpy (oracle view) and pinned torch."""
     if kind == "dense":
-        c = workloads.DenseCase(case.name, case.N, case.H, case.W, case.Cin, case.Cout, case.K, "bf16", "normal", seed)
+        c = dataclasses.replace(case, seed=seed)
         Xb, Fb = workloads.dense_inputs(c)
+        b = workloads.dense_bias(c)
         host = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (Xb, Fb)]
-        return (workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb)), host
+        host.append(None if b is None else torch.from_numpy(b).pin_memory())
+        return (workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb), b), host
     c = workloads.DepthwiseCase(case.name, case.N, case.C, case.mult, case.H, case.W, case.KH, case.KW, case.stride,
                                 case.pad, case.dil, case.bias, seed)
     x, w, b = workloads.depthwise_inputs(c)
@@ -403,7 +424,7 @@ def run_ours(args, dist):
     torch.cuda.set_device(dist.local_rank)
     peaks, peaks_src = load_peaks()
     host_np, host = host_inputs(torch, kind, case, seed=dist.rank)
-    dev_inputs = tuple(h.to("cuda") for h in host)
+    dev_inputs = tuple(None if h is None else h.to("cuda") for h in host)
 
     sampler = ClockSampler(dist.local_rank)
     ms, R, kernel = time_case(cb, torch, kind, case, mode, dev_inputs, args.steps, args.warmup, dist, sampler)
@@ -425,7 +446,8 @@ def run_ours(args, dist):
         dtype = "bf16"
         data = "synthetic (seeded SplitMix64 / Box-Muller: X~N(0,1), F~N(0,1/(K*K*Cin)), rounded to bf16)"
         cfg = {"workload": case.name, "N_per_gpu": case.N, "H": case.H, "W": case.W, "Cin": case.Cin,
-               "Cout": case.Cout, "K": case.K, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
+               "Cout": case.Cout, "K": case.K, "stride": case.stride, "pad": case.pad, "dil": case.dil,
+               "bias": case.bias, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
     else:
         unit, work, scale = "GB/s", case.bytes, 1e9
         achieved = case.bytes / (ms_step * 1e-3) / 1e9
@@ -496,11 +518,15 @@ def run_reference(args, dist):
     if kind == "dense":
         Xb, Fb = workloads.dense_inputs(case)
         X, F = workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb)
+        b = workloads.dense_bias(case)
         total = case.N * case.Ho * case.Wo * case.Cout
         work_per_out, unit, scale = 2 * case.K * case.K * case.Cin, "TFLOP/s", 1e12
 
         def run(idx):
-            oracle.conv2d_nhwc_points(X, F, idx)
+            if dense_plain(case):
+                oracle.conv2d_nhwc_points(X, F, idx)
+            else:
+                oracle.conv2d_nhwc_ex_points(X, F, idx, b, case.stride, case.pad, case.dil)
     else:
         x, w, b = workloads.depthwise_inputs(case)
         total = case.N * case.C * case.mult * case.Ho * case.Wo

@@ -8,6 +8,7 @@ importing this package fails if the library cannot be loaded.
 
     conv2d_nhwc_fwd(X, F)        dense NHWC conv, bf16 [N,H,W,Cin] x [K,K,Cin,Cout] -> bf16
     conv2d_nhwc_fwd_f32(X, F)    the same with float32 tensors
+    conv2d_nhwc_fwd_ex(X, F, b)  bf16 with stride, zero padding, dilation and a float32 bias
     depthwise_fwd(x, w, bias)    depthwise conv, float32 NCHW, exact or fast mode
 """
 from __future__ import annotations
@@ -34,6 +35,8 @@ lib.conv2d_nhwc_fwd.argtypes = [_P, _P, _P] + [_I] * 6 + [_P]
 lib.conv2d_nhwc_fwd.restype = _I
 lib.conv2d_nhwc_fwd_f32.argtypes = [_P, _P, _P] + [_I] * 6 + [_P]
 lib.conv2d_nhwc_fwd_f32.restype = _I
+lib.conv2d_nhwc_fwd_ex.argtypes = [_P, _P, _P, _P] + [_I] * 9 + [_P]
+lib.conv2d_nhwc_fwd_ex.restype = _I
 lib.depthwise_fwd.argtypes = [_P, _P, _P, _P] + [_I] * 11 + [_P]
 lib.depthwise_fwd.restype = _I
 lib.conv_status_string.argtypes = [_I]
@@ -45,7 +48,7 @@ lib.conv_last_kernel.restype = ctypes.c_char_p
 lib.conv_selftest_wait_timeout.argtypes = [_P]
 lib.conv_selftest_wait_timeout.restype = _I
 
-EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "depthwise_fwd", "conv_status_string",
+EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "depthwise_fwd", "conv_status_string",
            "conv_device_status", "conv_last_kernel", "conv_selftest_wait_timeout")
 
 
@@ -116,6 +119,35 @@ def conv2d_nhwc_fwd_f32(X, F, Y=None, stream=None):
     """Dense NHWC convolution, float32 tensors."""
     import torch
     return _dense(X, F, Y, stream, torch.float32, lib.conv2d_nhwc_fwd_f32, "conv2d_nhwc_fwd_f32")
+
+
+def conv2d_nhwc_fwd_ex(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, stream=None):
+    """Dense NHWC convolution, bfloat16, with stride, zero padding, dilation and an optional
+    float32 bias [Cout]: X [N,H,W,Cin], F [K,K,Cin,Cout] -> Y [N,Ho,Wo,Cout]."""
+    import torch
+    px = _tensor(X, torch.bfloat16, 4, "X")
+    pf = _tensor(F, torch.bfloat16, 4, "F")
+    N, H, W, Cin = X.shape
+    K, K2, Cin2, Cout = F.shape
+    if K != K2 or Cin2 != Cin:
+        raise ValueError("F must be [K, K, Cin, Cout] matching X")
+    pb = ctypes.c_void_p(None)
+    if bias is not None:
+        pb = _tensor(bias, torch.float32, 1, "bias")
+        if bias.shape[0] != Cout:
+            raise ValueError("bias must have Cout entries")
+    Ho = (H + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    Wo = (W + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    if Y is None:
+        Y = torch.empty((N, Ho, Wo, Cout), dtype=torch.bfloat16, device=X.device)
+    elif tuple(Y.shape) != (N, Ho, Wo, Cout):
+        raise ValueError("Y has the wrong shape")
+    py = _tensor(Y, torch.bfloat16, 4, "Y")
+    _check(lib.conv2d_nhwc_fwd_ex(px, pf, pb, py, N, H, W, Cin, Cout, K, stride, pad, dil, _stream(stream)),
+           "conv2d_nhwc_fwd_ex")
+    return Y
 
 
 def depthwise_fwd(x, w, bias=None, y=None, stride=1, pad=0, dil=1, mode=DW_EXACT, stream=None):

@@ -148,12 +148,22 @@ int check_dense(const void *X, const void *F, const void *Y, int N, int H, int W
     return CONV_OK;
 }
 
+// Stride, zero padding, dilation and bias of a dense convolution (the plain operation is
+// {1, 0, 1, null}).
+struct DenseGeom {
+    int stride = 1, pad = 0, dil = 1;
+    const float *bias = nullptr;
+    long long ho(int H, int K) const { return (1LL * H + 2LL * pad - (1LL * dil * (K - 1) + 1)) / stride + 1; }
+    bool plain() const { return stride == 1 && pad == 0 && dil == 1 && bias == nullptr; }
+};
+
 template <typename T>
 int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int Cin, int Cout, int K,
-                        cudaStream_t stream, DeviceState *d) {
+                        cudaStream_t stream, DeviceState *d, const DenseGeom &g = DenseGeom()) {
     DenseDirectParams p;
     p.H = H; p.W = W; p.Cin = Cin; p.Cout = Cout; p.K = K;
-    p.Ho = H - K + 1; p.Wo = W - K + 1;
+    p.Ho = static_cast<int>(g.ho(H, K)); p.Wo = static_cast<int>(g.ho(W, K));
+    p.stride = g.stride; p.pad = g.pad; p.dil = g.dil; p.bias = g.bias;
     p.total = 1LL * N * p.Ho * p.Wo * Cout;
     long long blocks = (p.total + 255) / 256;
     const long long cap = 1LL * d->num_sms * 16;
@@ -167,16 +177,18 @@ int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int C
 
 template <class Cfg>
 int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
-                    cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
-    const int Ho = H - K + 1, Wo = W - K + 1;
+                    cudaStream_t stream, DeviceState *d, unsigned attr_bit, const DenseGeom &g = DenseGeom()) {
+    const int Ho = static_cast<int>(g.ho(H, K)), Wo = static_cast<int>(g.ho(W, K));
     alignas(64) CUtensorMap tmX, tmF, tmY;
-    {   // X: 4-D {Cin, W, H, N} im2col; the bounding box of valid filter origins is
-        // [0, W-K] x [0, H-K] (upper corner -(K-1)), i.e. exactly the output pixels.
+    {   // X: 4-D {Cin, W, H, N} im2col. The bounding box of window origins runs from -pad to
+        // (size - 1) + pad - dil*(K-1) on each spatial axis, walked with the convolution stride
+        // as element stride, so its pixels are exactly the output positions; origins and taps
+        // outside the image read zeros.
         const cuuint64_t dims[4] = {(cuuint64_t)Cin, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)N};
         const cuuint64_t strides[3] = {(cuuint64_t)Cin * 2, (cuuint64_t)W * Cin * 2, (cuuint64_t)H * W * Cin * 2};
-        const int lower[2] = {0, 0};
-        const int upper[2] = {-(K - 1), -(K - 1)};
-        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        const int lower[2] = {-g.pad, -g.pad};
+        const int upper[2] = {g.pad - g.dil * (K - 1), g.pad - g.dil * (K - 1)};
+        const cuuint32_t estr[4] = {1, (cuuint32_t)g.stride, (cuuint32_t)g.stride, 1};
         if (g_encode_im2col(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(X), dims, strides,
                             lower, upper, 64, Cfg::BM, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -213,6 +225,7 @@ int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, 
     p.num_cblk = (Cin + 63) / 64;
     p.num_kblk = K * K * p.num_cblk;
     p.num_ntiles = (Cout + Cfg::BN - 1) / Cfg::BN;
+    p.stride = g.stride; p.pad = g.pad; p.dil = g.dil; p.bias = g.bias;
     const long long tiles = ((M + Cfg::BM - 1) / Cfg::BM) * p.num_ntiles;
     if (tiles > kInt32Max) return CONV_ERR_UNSUPPORTED;
     p.num_tiles = static_cast<int>(tiles);
@@ -400,6 +413,8 @@ FoldPlan plan_fold(int N, int H, int W, int Cin, int Cout, int K, int num_sms) {
     p.halo_bytes = halo_bytes;
     p.b_region = static_cast<int>(b_res);
     p.num_tiles = static_cast<int>((rows + TM - 1) / TM);
+    p.div_w = make_fastdiv(static_cast<uint32_t>(W));
+    p.div_h = make_fastdiv(static_cast<uint32_t>(H));
     pl.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
     pl.smem = fixed + p.b_region + p.HS * halo_bytes;
     // more than half of the shared memory keeps a second CTA (and its TMEM allocation) off the SM
@@ -436,7 +451,7 @@ int launch_dense_fold(const void *X, const void *F, void *Y, int Cin, int Cout, 
     if (int rc = ensure_smem_attr(d, attr_bit, kern, kSmemLimit)) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(DenseFoldCfg<KF>::THREADS);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
     return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
@@ -620,8 +635,8 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
     p.Wp = p.lpp * 4 * S + 8;                       // 4 zeros, the lanes' columns, the right reach
     p.use_tma = (W % 4 == 0 && aligned(x, 16)) ? 1 : 0;
     // staged bytes per job buffer: whole planes when they fit, else bands of rows
+    // (about 9 KB per buffer keeps 12 warps, 3 CTAs, per SM with both buffers resident)
     const long long row_bytes = 4LL * p.Wp * p.ppw;
-    // about 9 KB per buffer keeps 12 warps (3 CTAs) per SM with both buffers resident
     const long long kBufBytes = 9 * 1024;
     const int whole_rows = (Ho - 1) * S + K;
     if (whole_rows * row_bytes <= kBufBytes || !p.use_tma) {
@@ -633,6 +648,40 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
         p.Rw = Rw;
     }
     p.rows_in = (p.Rw - 1) * S + K;
+    // With several planes per warp, a plane stride rows_in * Wp = 4 * lpp * S (mod 32 floats)
+    // makes the next plane's lanes continue this plane's shared-memory bank pattern, so the
+    // 128-bit loads of a warp do not collide. Reach it with the cheapest of a slightly shorter
+    // band, a wider pitch, or extra staged rows (zeros or input rows nobody reads); keep the
+    // plain layout if nothing is within 25 % more staged bytes per output row or the larger
+    // buffers would fit fewer CTAs per SM.
+    if (p.ppw > 1) {
+        const int target = (4 * p.lpp * S) % 32;
+        const bool whole = p.Rw == Ho;
+        double best = 1e30;
+        int bRw = p.Rw, bRows = p.rows_in, bWp = p.Wp;
+        for (int dr = 0; dr < 8; ++dr) {
+            const int Rw = whole ? p.Rw : p.Rw - dr;
+            if (Rw < 1) break;
+            const int rows0 = (Rw - 1) * S + K;
+            for (int extra = 0; extra < 8; ++extra) {
+                if (!whole && extra > 0) break;
+                for (int t = 0; t < 8; ++t) {
+                    const int rows = rows0 + extra, wp = p.Wp + 4 * t;
+                    if ((rows * wp) % 32 != target) continue;
+                    const double cost = static_cast<double>(rows) * wp / Rw;
+                    if (cost < best) { best = cost; bRw = Rw; bRows = rows; bWp = wp; }
+                }
+            }
+        }
+        const double plain = static_cast<double>(p.rows_in) * p.Wp / p.Rw;
+        auto ctas = [&](int rows, int wp) {   // CTAs per SM the buffers allow
+            const long long buf = ((1LL * p.ppw * rows * wp + 31) & ~31LL) * 4;
+            return (227 * 1024) / (kDwWarpsPerCta * 2 * buf + 128 + 1024);
+        };
+        if (best <= 1.25 * plain && ctas(bRows, bWp) >= ctas(p.rows_in, p.Wp)) {
+            p.Rw = bRw; p.rows_in = bRows; p.Wp = bWp;
+        }
+    }
     if (p.use_tma && (p.Wp > 256 || p.rows_in > 256)) return pl;
     p.box_floats = p.ppw * p.rows_in * p.Wp;
     p.buf_floats = (p.box_floats + 31) & ~31;
@@ -645,7 +694,24 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
     p.div_lpp = make_fastdiv(static_cast<uint32_t>(p.lpp));
     p.div_c = make_fastdiv(static_cast<uint32_t>(p.C));
     p.div_w = make_fastdiv(static_cast<uint32_t>(W));
-    pl.smem = kDwWarpsPerCta * 2 * 4 * p.buf_floats + 128;   // + alignment slack
+    // whole-plane jobs whose rows cannot be stored 16 bytes at a time collect the outputs in
+    // shared memory and store the job's contiguous range coalesced, when that costs no CTA per SM
+    p.stage_out = 0;
+    p.out_floats = 0;
+    p.vec_out_staged = aligned(y, 16) ? 1 : 0;
+    p.warp_floats = 2 * p.buf_floats;
+    if (p.Rw == Ho && !p.vec_out) {
+        const int out_floats = (p.ppw * Ho * Wo + 31) & ~31;
+        const int smem_plain = kDwWarpsPerCta * 4 * p.warp_floats + 128;
+        const int smem_staged = kDwWarpsPerCta * 4 * (p.warp_floats + out_floats) + 128;
+        if (smem_staged <= kDwTmaMaxSmem &&
+            (227 * 1024) / (smem_staged + 1024) >= (227 * 1024) / (smem_plain + 1024)) {
+            p.stage_out = 1;
+            p.out_floats = out_floats;
+            p.warp_floats += out_floats;
+        }
+    }
+    pl.smem = kDwWarpsPerCta * 4 * p.warp_floats + 128;   // + alignment slack
     if (pl.smem > kDwTmaMaxSmem) return pl;
     int per_sm = (227 * 1024) / (pl.smem + 1024);
     if (per_sm > 16) per_sm = 16;
@@ -773,6 +839,49 @@ int conv2d_nhwc_fwd_f32(const float *X, const float *F, float *Y, int N, int H, 
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
     return launch_dense_direct(X, F, Y, N, H, W, Cin, Cout, K, stream, d);
+}
+
+int conv2d_nhwc_fwd_ex(const void *X, const void *F, const float *bias, void *Y, int N, int H, int W, int Cin,
+                       int Cout, int K, int stride, int pad, int dil, cudaStream_t stream) {
+    if (!X || !F || !Y) return CONV_ERR_INVALID_ARG;
+    if (N < 1 || H < 1 || W < 1 || Cin < 1 || Cout < 1 || K < 1 || stride < 1 || dil < 1 || pad < 0)
+        return CONV_ERR_INVALID_ARG;
+    DenseGeom g;
+    g.stride = stride; g.pad = pad; g.dil = dil; g.bias = bias;
+    if (1LL * H + 2LL * pad > kInt32Max / 2 || 1LL * W + 2LL * pad > kInt32Max / 2 ||
+        1LL * dil * (K - 1) > kInt32Max / 2)
+        return CONV_ERR_UNSUPPORTED;
+    const long long Ho = g.ho(H, K), Wo = g.ho(W, K);
+    if (1LL * H + 2LL * pad < 1LL * dil * (K - 1) + 1 || 1LL * W + 2LL * pad < 1LL * dil * (K - 1) + 1 || Ho < 1 ||
+        Wo < 1)
+        return CONV_ERR_INVALID_ARG;
+    if (g.plain()) return conv2d_nhwc_fwd(X, F, Y, N, H, W, Cin, Cout, K, stream);
+    const long long nx = 1LL * N * H * W * Cin, nf = 1LL * K * K * Cin * Cout, ny = 1LL * N * Ho * Wo * Cout;
+    if (nx > kInt32Max || nf > kInt32Max || ny > kInt32Max || 1LL * N * Ho * Wo > kInt32Max)
+        return CONV_ERR_UNSUPPORTED;
+    if (!aligned(X, 2) || !aligned(F, 2) || !aligned(Y, 2) || (bias && !aligned(bias, 4))) return CONV_ERR_MISALIGNED;
+    if (overlaps(Y, ny * 2, X, nx * 2) || overlaps(Y, ny * 2, F, nf * 2) || (bias && overlaps(Y, ny * 2, bias, 4LL * Cout)))
+        return CONV_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    const char *force = env("CONV_B200_DENSE");
+    // Tensor cores through the TMA im2col unit: 16-byte channel rows and tensors, and window
+    // corners and tap offsets inside the 4-D im2col ranges (|corner| <= 127, offset <= 127).
+    const bool tc_shape = (Cin % 8 == 0) && (Cout % 8 == 0) && aligned(X, 16) && aligned(F, 16) && aligned(Y, 16);
+    const long long reach = 1LL * dil * (K - 1);
+    const bool im2col_ok = tc_shape && pad <= 127 && reach <= 127 && pad - reach >= -127 && pad - reach <= 127 &&
+                           2LL * N * H * W * Cin >= 128 * 1024;
+    if ((force && std::strcmp(force, "direct") == 0) || !im2col_ok) {
+        if (force && std::strncmp(force, "bn", 2) == 0) return CONV_ERR_UNSUPPORTED;
+        return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
+                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d, g);
+    }
+    int bn = Cout <= 64 ? 64 : 128;
+    if (force && std::strncmp(force, "bn", 2) == 0) bn = std::atoi(force + 2);
+    if (bn == 64) return launch_dense_tc<CfgBN64>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 0, g);
+    if (bn == 128) return launch_dense_tc<CfgBN128>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 1, g);
+    if (bn == 256) return launch_dense_tc<CfgBN256>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 2, g);
+    return CONV_ERR_INVALID_ARG;
 }
 
 int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, int N, int Cin, int mult, int H,

@@ -4,7 +4,10 @@
 // not a multiple of 8, tensors below 128 KiB, K > 128) and for the float32 entry point. It
 // evaluates the index contract of the CMU DLSys Lecture 14 notes, section 1, directly:
 // Y[n,y,x,o] = sum over (i, j, c) of X[n,y+i,x+j,c] * F[i,j,c,o], as float32 fused
-// multiply-adds in (i, j, c) order, rounded once to the output type. Consecutive threads
+// multiply-adds in (i, j, c) order, rounded once to the output type -- and the stride, zero
+// padding, dilation and bias variants of "Convolution Is Wx+b Moving Across a Signal" (window
+// of output (y, x) at (y*stride - pad, x*stride - pad), taps dil apart, positions outside the
+// image skipped as zeros, the bias one fp32 addition before the rounding). Consecutive threads
 // take consecutive output channels o, so the F row reads are coalesced and the X reads are
 // warp-uniform broadcasts.
 #pragma once
@@ -14,7 +17,9 @@ namespace convb200 {
 
 struct DenseDirectParams {
     int H, W, Cin, Cout, K, Ho, Wo;
-    long long total;   // N * Ho * Wo * Cout
+    int stride, pad, dil;   // "Convolution Is Wx+b Moving Across a Signal" variants
+    const float *bias;      // per output channel or null; added in fp32 before the rounding
+    long long total;        // N * Ho * Wo * Cout
 };
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
@@ -38,13 +43,18 @@ dense_direct_kernel(const T *__restrict__ X, const T *__restrict__ F, T *__restr
         const long long n = t / p.Ho;
         float acc = 0.0f;
         for (int i = 0; i < p.K; ++i) {
+            const int r = y * p.stride + i * p.dil - p.pad;
+            if (r < 0 || r >= p.H) continue;   // zero padding contributes nothing
             for (int j = 0; j < p.K; ++j) {
-                const T *xr = X + ((n * p.H + (y + i)) * p.W + (x + j)) * p.Cin;
+                const int q = x * p.stride + j * p.dil - p.pad;
+                if (q < 0 || q >= p.W) continue;
+                const T *xr = X + ((n * p.H + r) * p.W + q) * p.Cin;
                 const T *fr = F + ((static_cast<long long>(i) * p.K + j) * p.Cin) * p.Cout + o;
                 for (int c = 0; c < p.Cin; ++c)
                     acc = __fmaf_rn(to_f32(xr[c]), to_f32(fr[static_cast<long long>(c) * p.Cout]), acc);
             }
         }
+        if (p.bias) acc = __fadd_rn(acc, __ldg(p.bias + o));
         store_out(Y + idx, acc);
     }
 }

@@ -23,13 +23,15 @@
 // groups added in j order in fp32, one rounding to bf16 -- a different order from the other
 // kernels, within the same error bound.
 //
-// Roles as in the halo kernel (warp 0 TMA, warp 1 TMEM + MMA, warps 2..5 epilogue); the
-// filter is always resident here.
+// Roles: warp 0 TMA, warp 1 TMEM + MMA, warps 2..9 epilogue (two warps per TMEM lane quarter,
+// 32 output channels each, so two epilogue warps share each SM sub-partition and hide each
+// other's TMEM-load and shuffle latencies); the filter is always resident here.
 #pragma once
 #include <cuda_bf16.h>
 
 #include "dense_halo.cuh"
 #include "dense_tc.cuh"
+#include "depthwise.cuh"   // FastDiv
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -44,6 +46,7 @@ struct DenseFoldParams {
     int num_tiles;     // ceil(rows / (128 - (K-1)))
     int HS;            // halo ring slots
     int b_region;      // bytes of the resident filter
+    FastDiv div_w, div_h;
 };
 
 template <int KF>
@@ -53,20 +56,36 @@ struct DenseFoldCfg {
     static constexpr int BM = 128;
     static constexpr int TM = BM - (KF - 1);           // output rows kept per tile
     static constexpr int SLOT_BYTES = 64 * 64 * 2;     // one (tap, channel block) filter slot
-    static constexpr int EPI_BYTES = 4 * 32 * 128;     // per-warp 32 rows x 64 channels staging
+    static constexpr int NUM_EPI = 8;                  // epilogue warps: 4 lane quarters x 2 column halves
+    static constexpr int THREADS = 64 + 32 * NUM_EPI;
+    static constexpr int EPI_BYTES = NUM_EPI * 32 * 64;   // per-warp 32 rows x 32 channels staging
     static constexpr int MAX_RING = 8;
-    // exchange: lanes 0..j-1 of group j (j >= 1), 64 floats each, per warp and tile parity
-    static constexpr int XCH_FLOATS = KF * (KF - 1) / 2 * 64;
-    static constexpr int XCH_BYTES = 2 * 4 * XCH_FLOATS * 4;
+    // exchange: lanes 0..j-1 of group j (j >= 1), 32 floats each, per warp and tile parity
+    static constexpr int XCH_FLOATS = KF * (KF - 1) / 2 * 32;
+    static constexpr int XCH_BYTES = 2 * NUM_EPI * XCH_FLOATS * 4;
     static constexpr int NUM_BARS = 2 * MAX_RING /*halo*/ + 1 /*filter*/ + 4 /*acc*/ + 2 /*xch*/ + 1;
     static constexpr int TMEM_COLS = 2 * NF <= 256 ? 256 : 512;
     static constexpr uint32_t IDESC = idesc_bf16_f32(BM, NF, /*B MN-major*/ true);
-    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + XCH_BYTES + NUM_BARS * 8 + 4 * 32 * 8 + 16;
+    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + XCH_BYTES + NUM_BARS * 8 + NUM_EPI * 32 * 8 + 16;
     static_assert(KF >= 2 && KF <= 4, "N = 64*K must stay within 256");
 };
 
+// st.shared.v4 executed only where pred != 0 (predicated, no branch)
+__device__ __forceinline__ void st_shared_v4_if(uint32_t pred, uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                                uint32_t d) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %0, 0; @p st.shared.v4.b32 [%1], {%2, %3, %4, %5}; }" ::"r"(pred),
+                 "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
 template <class Cfg>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
 dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
                   __nv_bfloat16 *__restrict__ Y, const DenseFoldParams p, unsigned int *status) {
     constexpr int K = Cfg::K;
@@ -81,7 +100,7 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const uint32_t sH = base + p.b_region;                    // halo ring
     const uint32_t epi_off = p.b_region + p.HS * p.halo_bytes;
     const uint32_t sEpi = base + epi_off;
-    float *xch = reinterpret_cast<float *>(smem + epi_off + Cfg::EPI_BYTES);
+    const uint32_t sX = sEpi + Cfg::EPI_BYTES;                 // row-shift exchange
     const uint32_t bars = sEpi + Cfg::EPI_BYTES + Cfg::XCH_BYTES;
     constexpr int R = Cfg::MAX_RING;
     auto hfull = [&](int s) { return bars + 8u * s; };
@@ -91,9 +110,10 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     auto acce = [&](int b) { return bars + 8u * (2 * R + 3 + b); };
     auto xbar = [&](int b) { return bars + 8u * (2 * R + 5 + b); };
     const uint32_t done_bar = bars + 8u * (2 * R + 7);
-    long long *rowoff_all =
-        reinterpret_cast<long long *>(smem + epi_off + Cfg::EPI_BYTES + Cfg::XCH_BYTES + Cfg::NUM_BARS * 8);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rowoff_all + 4 * 32);
+    const uint32_t rowoff_all = sEpi + Cfg::EPI_BYTES + Cfg::XCH_BYTES + Cfg::NUM_BARS * 8;   // s64 per row
+    uint32_t *tmem_holder =
+        reinterpret_cast<uint32_t *>(smem + epi_off + Cfg::EPI_BYTES + Cfg::XCH_BYTES + Cfg::NUM_BARS * 8 +
+                                     Cfg::NUM_EPI * 32 * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -107,8 +127,8 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         mbar_init(bfull, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf(b), 1);
-            mbar_init(acce(b), 128);
-            mbar_init(xbar(b), 128);
+            mbar_init(acce(b), Cfg::NUM_EPI);   // one arrival per epilogue warp
+            mbar_init(xbar(b), Cfg::NUM_EPI);
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -177,7 +197,8 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         bool ok = mbar_wait_warp(bfull, 0);
         for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step, ++local) {
             const uint32_t b = local & 1u;
-            if (!mbar_wait_warp(acce(b), ((local >> 1) & 1u) ^ 1u)) { ok = false; break; }
+            // the epilogue is the slower role: sleep between polls instead of taking its issue slots
+            if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + b * NF;
             for (int cb = 0; cb < p.num_cblk; ++cb) {
@@ -216,9 +237,13 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         __syncwarp();
     } else {
         // ------------------------------- Epilogue -----------------------------------
-        const int q = warp & 3;   // TMEM lane quarter this warp may access
-        const uint32_t stage = sEpi + q * 4096;
-        long long *rowoff = rowoff_all + q * 32;
+        // warp e = warp - 2: TMEM lane quarter q = warp % 4 (the quarter a warp may access),
+        // output channels 32h .. 32h + 31 with h = e / 4
+        const int e = warp - 2;
+        const int q = warp & 3;
+        const int h = e >> 2;
+        const uint32_t stage = sEpi + e * 2048;
+        const uint32_t rowoff = rowoff_all + e * 32 * 8;
         uint32_t local = 0;
         for (int t = first; t < p.num_tiles; t += step, ++local) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
@@ -231,88 +256,98 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const int P = t * TM + r;
                 long long off = -1;
                 if (r < TM && P < p.rows) {
-                    const int row = P / p.W;
+                    const int row = fdiv(P, p.div_w);
                     const int x = P - row * p.W;
-                    const int n = row / p.H;
+                    const int n = fdiv(row, p.div_h);
                     const int y = row - n * p.H;
                     if (x < p.Wo && y < p.Ho)
                         off = ((static_cast<long long>(n) * p.Ho + y) * p.Wo + x) * p.Cout;
                 }
-                rowoff[lane] = off;
+                asm volatile("st.shared.s64 [%0], %1;" ::"r"(rowoff + 8u * lane), "l"(off) : "memory");
             }
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * NF;
-            // publish lanes 0..j-1 of groups j >= 1 for the warp above (rows 32q - K + 1 ..)
-            float *my_x = xch + (par * 4 + q) * Cfg::XCH_FLOATS;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * NF + h * 32;
+            // one round trip to TMEM: all K groups of this warp's 32 columns
+            uint32_t d[K][2][16];
+#pragma unroll
+            for (int j = 0; j < K; ++j)
+#pragma unroll
+                for (int g = 0; g < 2; ++g) tmem_ld_32x32b_x16(t_row + j * 64 + g * 16, d[j][g]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce(b));   // accumulator read: the MMA warp may reuse it
+            // publish lanes 0..j-1 of groups j >= 1 for the warp of the quarter above
             if (q > 0) {
+                const uint32_t my_x = sX + 4u * ((par * 4 + q) * 2 + h) * Cfg::XCH_FLOATS;
 #pragma unroll
                 for (int j = 1; j < K; ++j) {
-                    uint32_t v[4][16];
+                    const uint32_t pub = lane < j ? 1u : 0u;   // predicated stores: no divergent branch
+                    const uint32_t dst = my_x + 4u * (j * (j - 1) / 2 + (lane < j ? lane : 0)) * 32;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + j * 64 + g * 16, v[g]);
-                    tmem_wait_ld();
-                    if (lane < j) {
-                        float4 *dst = reinterpret_cast<float4 *>(my_x + (j * (j - 1) / 2 + lane) * 64);
+                    for (int g = 0; g < 2; ++g)
 #pragma unroll
-                        for (int g = 0; g < 4; ++g)
-#pragma unroll
-                            for (int c = 0; c < 4; ++c)
-                                dst[g * 4 + c] = make_float4(__uint_as_float(v[g][4 * c]), __uint_as_float(v[g][4 * c + 1]),
-                                                             __uint_as_float(v[g][4 * c + 2]), __uint_as_float(v[g][4 * c + 3]));
-                    }
+                        for (int c = 0; c < 4; ++c)
+                            st_shared_v4_if(pub, dst + 16u * (g * 4 + c), d[j][g][4 * c], d[j][g][4 * c + 1],
+                                            d[j][g][4 * c + 2], d[j][g][4 * c + 3]);
                 }
             }
-            mbar_arrive(xbar(par));
-            const float *next_x = xch + (par * 4 + (q < 3 ? q + 1 : q)) * Cfg::XCH_FLOATS;
-            bool xok = true;
-            const uint32_t row_addr = stage + lane * 128;
+            __syncwarp();   // the lanes' exchange stores are ordered before lane 0's release
+            if (lane == 0) mbar_arrive(xbar(par));
+            const uint32_t next_x = sX + 4u * ((par * 4 + (q < 3 ? q + 1 : q)) * 2 + h) * Cfg::XCH_FLOATS;
+            const bool xok = mbar_wait_warp_backoff(xbar(par), (local >> 1) & 1u, 32);
+            const uint32_t row_addr = stage + lane * 64;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                uint32_t d[K][16];
-#pragma unroll
-                for (int j = 0; j < K; ++j) tmem_ld_32x32b_x16(t_row + j * 64 + g * 16, d[j]);
-                tmem_wait_ld();
-                if (g == 3) {   // accumulator fully read: the MMA warp may reuse it
-                    tc_fence_before();
-                    mbar_arrive(acce(b));
-                }
-                if (g == 0) xok = mbar_wait_warp(xbar(par), (local >> 1) & 1u);
+            for (int g = 0; g < 2; ++g) {
                 float y[16];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) y[c] = __uint_as_float(d[0][c]);
+                for (int c = 0; c < 16; ++c) y[c] = __uint_as_float(d[0][g][c]);
 #pragma unroll
                 for (int j = 1; j < K; ++j) {
+                    // lanes 32-j .. 31 take row r + j from the next quarter's exchange; every lane
+                    // loads (a valid address, mostly a broadcast) and selects, so nothing diverges
                     const bool from_next = lane + j >= 32;
-                    const float *src = next_x + (j * (j - 1) / 2 + (lane + j - 32 < 0 ? 0 : lane + j - 32)) * 64 + g * 16;
+                    const bool from_smem = from_next && q < 3 && xok;
+                    const uint32_t src = next_x + 4u * ((j * (j - 1) / 2 + (from_next ? lane + j - 32 : 0)) * 32 + g * 16);
+                    float xv[16];
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const float4 t4 = ld_shared_f4(src + 16u * c4);
+                        xv[4 * c4] = t4.x; xv[4 * c4 + 1] = t4.y; xv[4 * c4 + 2] = t4.z; xv[4 * c4 + 3] = t4.w;
+                    }
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        float v = __shfl_down_sync(0xffffffffu, __uint_as_float(d[j][c]), j);
-                        if (from_next) v = (q < 3 && xok) ? src[c] : 0.0f;
+                        const float sv = __shfl_down_sync(0xffffffffu, __uint_as_float(d[j][g][c]), j);
+                        const float v = from_next ? (from_smem ? xv[c] : 0.0f) : sv;
                         y[c] = __fadd_rn(y[c], v);
                     }
                 }
+                // 64-byte staging rows, 16-byte chunks swizzled by (row / 2) % 4: conflict-free
+                // writes (one row per lane) and reads (two rows per 8 lanes)
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const uint32_t c = g * 2 + cc;
                     const float *v = &y[cc * 8];
-                    st_shared_v4(row_addr + ((c ^ (lane & 7)) << 4), halo_pack_bf16x2(v[0], v[1]),
+                    st_shared_v4(row_addr + ((c ^ ((lane >> 1) & 3)) << 4), halo_pack_bf16x2(v[0], v[1]),
                                  halo_pack_bf16x2(v[2], v[3]), halo_pack_bf16x2(v[4], v[5]),
                                  halo_pack_bf16x2(v[6], v[7]));
                 }
             }
             if (!xok) { if (lane == 0) fail(); break; }
             __syncwarp();
-            // coalesced stores: 8 lanes per row, 4 rows per instruction
-            const int col = (lane & 7) * 8;
+            // coalesced stores: 4 lanes per 64-byte row, 8 rows per instruction
+            const int cc = lane & 3;
+            const int col = h * 32 + cc * 8;
             if (col < p.Cout) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int rr = i * 4 + (lane >> 3);
-                    const long long off = rowoff[rr];
+                for (int i = 0; i < 4; ++i) {
+                    const int rr = i * 8 + (lane >> 2);
+                    long long off;
+                    asm volatile("ld.shared.s64 %0, [%1];" : "=l"(off) : "r"(rowoff + 8u * rr));
                     if (off >= 0) {
                         uint32_t a, bb, c, dd;
                         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                      : "=r"(a), "=r"(bb), "=r"(c), "=r"(dd)
-                                     : "r"(stage + rr * 128 + ((((lane & 7) ^ (rr & 7))) << 4)));
+                                     : "r"(stage + rr * 64 + ((cc ^ ((rr >> 1) & 3)) << 4)));
                         *reinterpret_cast<uint4 *>(Y + off + col) = make_uint4(a, bb, c, dd);
                     }
                 }

@@ -122,7 +122,7 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf(b), 1);
-            mbar_init(acce(b), 128);
+            mbar_init(acce(b), 4);   // one arrival per epilogue warp
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -228,7 +228,9 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (BRES && !mbar_wait_warp(bfull(0), 0)) ok = false;
         for (int t = first; t < count && ok && !*abort_flag; t += step, ++local) {
             const uint32_t b = local & 1u;
-            if (!mbar_wait_warp(acce(b), ((local >> 1) & 1u) ^ 1u)) { ok = false; break; }
+            // waiting here means the epilogue is the slower role: sleep between polls instead
+            // of taking its issue slots
+            if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + b * BN;
             for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
@@ -363,7 +365,8 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 __syncwarp();
             }
             tc_fence_before();
-            mbar_arrive(acce(b));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce(b));
         }
     }
 

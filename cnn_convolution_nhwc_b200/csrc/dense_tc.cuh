@@ -1,7 +1,10 @@
 // Dense NHWC forward convolution as an implicit GEMM on the sm_100a tensor cores.
 //
 // Matrix form (CMU DLSys Lecture 14 notes, section 5 "Generalize the patch matrix to
-// channels and batches"): A_col[(n,y,x), (i,j,c)] = X[n, y+i, x+j, c] is the
+// channels and batches"; with the stride, zero-padding, dilation and bias variants of
+// "Convolution Is Wx+b Moving Across a Signal", which the TMA im2col unit expresses directly:
+// element strides for the stride, a bounding box that starts at -pad for the padding, with
+// out-of-range pixels read as zeros, and tap offsets scaled by the dilation): A_col[(n,y,x), (i,j,c)] = X[n, y+i, x+j, c] is the
 // (N*Ho*Wo) x (K*K*Cin) patch matrix, F_mat is F viewed as (K*K*Cin) x Cout, and
 // Y_mat = A_col * F_mat is Y viewed as (N*Ho*Wo) x Cout. The notes' closing remark in
 // section 6 -- generate patch fragments as needed instead of materialising the matrix --
@@ -41,6 +44,9 @@ struct DenseTcParams {
     int num_kblk;   // K * K * num_cblk
     int num_ntiles; // ceil(Cout / BN)
     int num_tiles;  // ceil(M / 128) * num_ntiles
+    int stride, pad, dil;   // window of output (y, x) starts at (y*stride - pad, x*stride - pad);
+                            // tap (i, j) is dil*i rows and dil*j columns further on
+    const float *bias;      // per output channel, added in fp32 before the bf16 rounding; or null
 };
 
 template <int BN_, int STAGES_>
@@ -110,7 +116,7 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf_bar(b), 1);
-            mbar_init(acce_bar(b), 128);
+            mbar_init(acce_bar(b), 4);   // one arrival per epilogue warp
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -158,8 +164,9 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(full_bar(s), Cfg::STAGE_BYTES);
-                    tma_load_im2col_4d(sA + s * Cfg::A_BYTES, &tmX, full_bar(s), cb * 64, ox, oy, img,
-                                       static_cast<uint16_t>(kx), static_cast<uint16_t>(ky));
+                    tma_load_im2col_4d(sA + s * Cfg::A_BYTES, &tmX, full_bar(s), cb * 64, ox * p.stride - p.pad,
+                                       oy * p.stride - p.pad, img, static_cast<uint16_t>(kx * p.dil),
+                                       static_cast<uint16_t>(ky * p.dil));
 #pragma unroll
                     for (int h = 0; h < BN / 64; ++h)
                         tma_load_3d(sB + s * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, &tmF, full_bar(s),
@@ -189,7 +196,9 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x, ++local) {
             const uint32_t b = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
-            if (!mbar_wait_warp(acce_bar(b), aph ^ 1u)) {
+            // waiting here means the epilogue is the slower role: sleep between polls instead
+            // of taking its issue slots
+            if (!mbar_wait_warp_backoff(acce_bar(b), aph ^ 1u, 64)) {
                 if (lane == 0) fail();
                 break;
             }
@@ -259,6 +268,17 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
                 for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + h * 64 + g * 16, r[g]);
                 tmem_wait_ld();
+                if (p.bias) {   // one fp32 addition per output, before the single rounding
+                    const int c0 = n0 + h * 64;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int col = c0 + g * 16 + c;
+                            const float bv = col < p.Cout ? __ldg(p.bias + col) : 0.0f;
+                            r[g][c] = __float_as_uint(__fadd_rn(__uint_as_float(r[g][c]), bv));
+                        }
+                }
                 const uint32_t row_addr = stage_s + h * 4096 + lane * 128;
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
@@ -276,7 +296,8 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             }
             // accumulator b may now be overwritten by the MMA warp
             tc_fence_before();
-            mbar_arrive(acce_bar(b));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce_bar(b));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {

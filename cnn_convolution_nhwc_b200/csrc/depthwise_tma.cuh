@@ -45,6 +45,11 @@ struct DwTmaParams {
                            // in shared memory must be 128-byte aligned)
     int use_tma;           // 1: TMA box (W % 4 == 0); 0: cp.async copies of whole planes
     int vec_out;           // 1: 128-bit output stores
+    int stage_out;         // 1: whole-plane jobs collect their outputs in shared memory and write
+                           //    the job's contiguous output range with coalesced stores
+    int out_floats;        // per-warp output staging (ppw * Ho * Wo rounded up to 128 bytes)
+    int warp_floats;       // per-warp shared memory: 2 * buf_floats + out_floats
+    int vec_out_staged;    // 1: y 16-byte aligned (staged copies may use 128-bit stores)
     FastDiv div_nbands, div_lpp, div_c, div_w;
 };
 
@@ -70,6 +75,38 @@ __device__ __forceinline__ void dw_ld_span(const float *base, float *out) {
     }
 }
 
+// Packed pairs of float32 (sm_100 f32x2 arithmetic): two neighbouring outputs of a lane advance
+// together; each half is an IEEE binary32 operation rounded to nearest, exactly as the scalar
+// __fmul_rn / __fmaf_rn, so results are bit-identical to the scalar kernels.
+__device__ __forceinline__ uint64_t dw_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void dw_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// Exact-mode tap for two outputs (lo, hi): one packed multiply and two scalar rounded additions
+// -- a packed multiply whose only use is a packed addition was measured to come out fused (one
+// rounding), so the additions stay scalar.
+__device__ __forceinline__ void dw_tap2_exact(float &lo, float &hi, uint64_t w2, uint64_t x2) {
+    uint64_t prod;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(prod) : "l"(w2), "l"(x2));
+    float p0, p1;
+    dw_unpack(prod, p0, p1);
+    lo = __fadd_rn(lo, p0);
+    hi = __fadd_rn(hi, p1);
+}
+
+// Fast-mode tap for two outputs: one packed fused multiply-add.
+__device__ __forceinline__ uint64_t dw_tap2_fast(uint64_t acc, uint64_t w2, uint64_t x2) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(w2), "l"(x2), "l"(acc));
+    return r;
+}
+
 template <int MODE, bool HAS_BIAS, int K, int S>
 __global__ void __launch_bounds__(32 * kDwWarpsPerCta)
 depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__restrict__ x,
@@ -85,7 +122,8 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
     // the dynamic region is only guaranteed 16-byte alignment: align the buffers to 128 bytes
     const uint32_t raw_s = static_cast<uint32_t>(__cvta_generic_to_shared(sraw));
     float *sbuf = sraw + (((raw_s + 127u) & ~127u) - raw_s) / 4u;
-    float *my_buf = sbuf + static_cast<size_t>(warp) * 2 * p.buf_floats;
+    float *my_buf = sbuf + static_cast<size_t>(warp) * p.warp_floats;
+    float *sout = my_buf + 2 * p.buf_floats;
     const uint32_t buf_s = static_cast<uint32_t>(__cvta_generic_to_shared(my_buf));
     const uint32_t full0 = static_cast<uint32_t>(__cvta_generic_to_shared(&full_all[warp][0]));
     auto full = [&](int b) { return full0 + 8u * b; };
@@ -171,45 +209,129 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
         const float *pb = my_buf + b * p.buf_floats + (lane_ok ? ps : 0) * (p.rows_in * p.Wp) + c0;
         float *yp = y + (static_cast<long long>(active ? plane : 0) * p.Ho + oy0) * p.Wo + ox;
 
-        float ring[K][WIN];
+        auto store_row = [&](int i, const float (&acc)[VX]) {
+            if (p.stage_out) {   // whole-plane job: row oy0 + i = i of plane slot ps
+                if (active) {
+                    float *dst = sout + (ps * p.Ho + i) * p.Wo + ox;
 #pragma unroll
-        for (int r = 0; r < K - S; ++r) dw_ld_span<4 - PAD, WIN>(pb + r * p.Wp, ring[r]);
+                    for (int v = 0; v < VX; ++v)
+                        if (ox + v < p.Wo) dst[v] = acc[v];
+                }
+            } else if (active) {
+                float *dst = yp + static_cast<long long>(i) * p.Wo;
+                if (p.vec_out && ox + VX <= p.Wo) {
+                    *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < VX; ++v)
+                        if (ox + v < p.Wo) dst[v] = acc[v];
+                }
+            }
+        };
 
-        for (int base = 0; base < nrows; base += K) {
+        if constexpr (S == 1) {
+            // ring of K rows held as the WIN - 1 overlapping pairs (x[t], x[t+1]): outputs
+            // (2q, 2q+1) at tap kx read pair 2q + kx, and the weight is a pair (w, w)
+            uint64_t w2[K * K];
 #pragma unroll
-            for (int u = 0; u < K; ++u) {
-                const int i = base + u;
-                if (i < nrows) {
-                    // staged rows i*S + K - S .. i*S + K - 1 complete the window of output row i
-                    // (base is a multiple of K, so row r sits in ring slot (u*S + r - i*S) % K)
+            for (int t = 0; t < K * K; ++t) w2[t] = dw_pack(wr[t], wr[t]);
+            uint64_t ring[K][WIN - 1];
+            auto load_pairs = [&](int r, uint64_t (&dst)[WIN - 1]) {
+                float f[WIN];
+                dw_ld_span<4 - PAD, WIN>(pb + r * p.Wp, f);
 #pragma unroll
-                    for (int s = 0; s < S; ++s)
-                        dw_ld_span<4 - PAD, WIN>(pb + (i * S + K - S + s) * p.Wp, ring[(u * S + K - S + s) % K]);
-                    float acc[VX];
+                for (int t = 0; t < WIN - 1; ++t) dst[t] = dw_pack(f[t], f[t + 1]);
+            };
 #pragma unroll
-                    for (int v = 0; v < VX; ++v) {
-                        float a = 0.0f;
+            for (int r = 0; r < K - 1; ++r) load_pairs(r, ring[r]);
+            for (int base = 0; base < nrows; base += K) {
 #pragma unroll
-                        for (int ky = 0; ky < K; ++ky)
+                for (int u = 0; u < K; ++u) {
+                    const int i = base + u;
+                    if (i < nrows) {
+                        // staged row i + K - 1 completes the window of output row i (ring slot
+                        // of staged row r: (u + r - i) % K, base being a multiple of K)
+                        load_pairs(i + K - 1, ring[(u + K - 1) % K]);
+                        float acc[VX];
+                        if constexpr (MODE == 0) {
 #pragma unroll
-                            for (int kx = 0; kx < K; ++kx)
-                                a = dw_tap<MODE>(a, wr[ky * K + kx], ring[(u * S + ky) % K][v * S + kx]);
-                        acc[v] = dw_finish<MODE, HAS_BIAS>(a, bv);
-                    }
-                    if (active) {
-                        float *dst = yp + static_cast<long long>(i) * p.Wo;
-                        if (p.vec_out && ox + VX <= p.Wo) {
-                            *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                            for (int v = 0; v < VX; ++v) acc[v] = 0.0f;
+#pragma unroll
+                            for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                                for (int kx = 0; kx < K; ++kx)
+#pragma unroll
+                                    for (int q = 0; q < VX / 2; ++q)
+                                        dw_tap2_exact(acc[2 * q], acc[2 * q + 1], w2[ky * K + kx],
+                                                      ring[(u + ky) % K][2 * q + kx]);
                         } else {
+                            uint64_t a2[VX / 2];
 #pragma unroll
-                            for (int v = 0; v < VX; ++v)
-                                if (ox + v < p.Wo) dst[v] = acc[v];
+                            for (int q = 0; q < VX / 2; ++q) a2[q] = dw_pack(0.0f, 0.0f);
+#pragma unroll
+                            for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                                for (int kx = 0; kx < K; ++kx)
+#pragma unroll
+                                    for (int q = 0; q < VX / 2; ++q)
+                                        a2[q] = dw_tap2_fast(a2[q], w2[ky * K + kx], ring[(u + ky) % K][2 * q + kx]);
+#pragma unroll
+                            for (int q = 0; q < VX / 2; ++q) dw_unpack(a2[q], acc[2 * q], acc[2 * q + 1]);
                         }
+#pragma unroll
+                        for (int v = 0; v < VX; ++v) acc[v] = dw_finish<MODE, HAS_BIAS>(acc[v], bv);
+                        store_row(i, acc);
+                    }
+                }
+            }
+        } else {
+            float ring[K][WIN];
+#pragma unroll
+            for (int r = 0; r < K - S; ++r) dw_ld_span<4 - PAD, WIN>(pb + r * p.Wp, ring[r]);
+            for (int base = 0; base < nrows; base += K) {
+#pragma unroll
+                for (int u = 0; u < K; ++u) {
+                    const int i = base + u;
+                    if (i < nrows) {
+                        // staged rows i*S + K - S .. i*S + K - 1 complete the window of output row
+                        // i (base is a multiple of K, so row r sits in ring slot (u*S + r - i*S) % K)
+#pragma unroll
+                        for (int s = 0; s < S; ++s)
+                            dw_ld_span<4 - PAD, WIN>(pb + (i * S + K - S + s) * p.Wp, ring[(u * S + K - S + s) % K]);
+                        float acc[VX];
+#pragma unroll
+                        for (int v = 0; v < VX; ++v) {
+                            float a = 0.0f;
+#pragma unroll
+                            for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                                for (int kx = 0; kx < K; ++kx)
+                                    a = dw_tap<MODE>(a, wr[ky * K + kx], ring[(u * S + ky) % K][v * S + kx]);
+                            acc[v] = dw_finish<MODE, HAS_BIAS>(a, bv);
+                        }
+                        store_row(i, acc);
                     }
                 }
             }
         }
-        // every lane is done with buffer b; refill it two jobs ahead
+        if (p.stage_out) {
+            // the job's planes are contiguous in y: copy them out with coalesced stores
+            __syncwarp();
+            const int plane0 = pg * p.ppw;
+            const int nplanes = min(p.ppw, p.num_planes - plane0);
+            const int plane_out = p.Ho * p.Wo;
+            const int total = nplanes * plane_out;
+            float *gdst = y + static_cast<long long>(plane0) * plane_out;
+            if (p.vec_out_staged && ((plane0 * plane_out) & 3) == 0) {
+                const int n4 = total >> 2;
+                for (int e = lane; e < n4; e += 32)
+                    reinterpret_cast<float4 *>(gdst)[e] = reinterpret_cast<const float4 *>(sout)[e];
+                for (int e = (n4 << 2) + lane; e < total; e += 32) gdst[e] = sout[e];
+            } else {
+                for (int e = lane; e < total; e += 32) gdst[e] = sout[e];
+            }
+        }
+        // every lane is done with buffer b (and the output staging); refill b two jobs ahead
         __syncwarp();
         if (job + 2 * GW < p.num_jobs) issue(job + 2 * GW, b);
     }

@@ -80,6 +80,28 @@ int conv2d_nhwc_fwd_f32(const float *X, const float *F, float *Y,
                         int N, int H, int W, int Cin, int Cout, int K, cudaStream_t stream);
 
 /*
+ * Dense NHWC forward convolution with stride, symmetric zero padding, dilation and an optional
+ * bias: the variants of "Convolution Is Wx+b Moving Across a Signal" (section "Build an
+ * image-gradient map, one number at a time" for the output size; section "Find the same sum in
+ * CKE's C kernels" for the window indexing out*stride + tap - padding):
+ *     Ho = floor((H + 2*pad - (dil*(K-1) + 1)) / stride) + 1   (Wo likewise),
+ *     Y[n,y,x,o] = bias[o] + sum_{i,j,c} X[n, y*stride + i*dil - pad, x*stride + j*dil - pad, c]
+ *                                         * F[i,j,c,o],
+ * with X read as zero outside the image.
+ *   X, F, Y : bfloat16, layouts as conv2d_nhwc_fwd (Y is [N][Ho][Wo][Cout])
+ *   bias    : float32 [Cout] or NULL; added in float32 to the float32 sum before the single
+ *             rounding to bfloat16
+ * Requirements: N, H, W, Cin, Cout, K, stride, dil >= 1; pad >= 0; Ho, Wo >= 1; X, F, Y non-null
+ * and 2-byte aligned, bias 4-byte aligned; element counts below 2^31. With stride 1, pad 0,
+ * dil 1 and no bias this is exactly conv2d_nhwc_fwd. Otherwise the tensor-core path needs Cin and
+ * Cout multiples of 8, 16-byte aligned tensors, pad <= 127, dil*(K-1) <= 127 and
+ * |pad - dil*(K-1)| <= 127; other valid shapes take a CUDA-core path with the same contract.
+ */
+int conv2d_nhwc_fwd_ex(const void *X, const void *F, const float *bias, void *Y,
+                       int N, int H, int W, int Cin, int Cout, int K,
+                       int stride, int pad, int dil, cudaStream_t stream);
+
+/*
  * Depthwise forward convolution, float32.
  *   x    : [N][Cin][H][W]
  *   w    : [Cin*mult][KH][KW]   (plane oc belongs to input channel oc / mult)

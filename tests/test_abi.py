@@ -92,6 +92,35 @@ def test_depthwise_rejects(args, code):
     assert cb.lib.depthwise_fwd(*args, None) == code
 
 
+@pytest.mark.parametrize("args,code", [
+    # X, F, bias, Y, N, H, W, Cin, Cout, K, stride, pad, dil
+    ((None, F, B, Y, 1, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_INVALID_ARG),
+    ((X, None, B, Y, 1, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, B, None, 1, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, B, Y, 0, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 0, 1, 1), cb.CONV_ERR_INVALID_ARG),      # stride 0
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 2, -1, 1), cb.CONV_ERR_INVALID_ARG),     # pad < 0
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 2, 1, 0), cb.CONV_ERR_INVALID_ARG),      # dil 0
+    ((X, F, B, Y, 1, 2, 2, 8, 8, 5, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),      # dilated window > padded image
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 1, 0, 5), cb.CONV_ERR_INVALID_ARG),      # dilation 5: reach 11 > 9
+    ((V((1 << 20) + 1), F, B, Y, 1, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_MISALIGNED),
+    ((X, F, V((1 << 30) + 2), Y, 1, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_MISALIGNED),   # bias not 4-byte aligned
+    ((X, F, B, V(1 << 20), 1, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_INVALID_ARG),       # Y aliases X
+    ((X, F, V((1 << 28) + 8), Y, 1, 9, 9, 8, 8, 3, 2, 1, 1), cb.CONV_ERR_INVALID_ARG),  # bias inside Y
+    ((X, F, B, Y, 4096, 4096, 4096, 64, 8, 3, 2, 1, 1), cb.CONV_ERR_UNSUPPORTED),
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 1, 2 ** 30, 1), cb.CONV_ERR_UNSUPPORTED),          # padding beyond int range
+])
+def test_dense_ex_rejects(args, code):
+    assert cb.lib.conv2d_nhwc_fwd_ex(*args, None) == code
+
+
+def test_dense_ex_plain_geometry_validates_like_the_plain_entry():
+    # stride 1, pad 0, dil 1, no bias is conv2d_nhwc_fwd: the same argument checks apply
+    assert cb.lib.conv2d_nhwc_fwd_ex(X, F, None, Y, 1, 5, 2, 8, 8, 3, 1, 0, 1, None) == cb.CONV_ERR_INVALID_ARG
+    assert cb.lib.conv2d_nhwc_fwd_ex(V((1 << 20) + 1), F, None, Y, 1, 5, 5, 8, 8, 3, 1, 0, 1, None) == \
+        cb.CONV_ERR_MISALIGNED
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

@@ -122,14 +122,18 @@ class DenseCase:
     dtype: str          # "bf16" or "f32": storage type of X, F and Y
     dist: str           # "normal" (X~N(0,1), F~N(0,1/(K*K*Cin))) or "int3" (integers in [-3,3])
     seed: int = 0
+    stride: int = 1
+    pad: int = 0
+    dil: int = 1
+    bias: bool = False  # a float32 bias[Cout] ~ N(0, 0.1)
 
     @property
     def Ho(self) -> int:
-        return self.H - self.K + 1
+        return (self.H + 2 * self.pad - (self.dil * (self.K - 1) + 1)) // self.stride + 1
 
     @property
     def Wo(self) -> int:
-        return self.W - self.K + 1
+        return (self.W + 2 * self.pad - (self.dil * (self.K - 1) + 1)) // self.stride + 1
 
     @property
     def flops(self) -> int:
@@ -139,7 +143,7 @@ class DenseCase:
     def bytes(self) -> int:
         e = 2 if self.dtype == "bf16" else 4
         return e * (self.N * self.H * self.W * self.Cin + self.K * self.K * self.Cin * self.Cout
-                    + self.N * self.Ho * self.Wo * self.Cout)
+                    + self.N * self.Ho * self.Wo * self.Cout) + (4 * self.Cout if self.bias else 0)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -185,12 +189,22 @@ DENSE_1X1 = DenseCase("pointwise bf16 N32 H28 W28 Cin256 Cout512 K1", 32, 28, 28
 DENSE_LARGE = DenseCase("large dense bf16 N64 H112 W112 Cin128 Cout128 K5", 64, 112, 112, 128, 128, 5,
                         "bf16", "normal", 0)
 
+# stride-2 3x3 layer with "same" padding and a bias (a ResNet stage transition, 56 -> 28)
+DENSE_S2 = DenseCase("dense bf16 N32 H56 W56 Cin64 Cout128 K3 s2 p1 bias", 32, 56, 56, 64, 128, 3, "bf16", "normal", 0,
+                     stride=2, pad=1, bias=True)
 # MobileNetV3-large depthwise layers (C, K, stride, input H=W), batch 64, multiplier 1,
 # pad (K-1)/2, dilation 1.
 DW_LAYERS = [(16, 3, 1, 112), (64, 3, 2, 112), (72, 5, 2, 56), (120, 5, 1, 28), (672, 3, 1, 14),
              (960, 5, 1, 7)]
 DW_SWEEP = [DepthwiseCase(f"depthwise C{c} K{k} s{s} H{h}", 64, c, 1, h, h, k, k, s, (k - 1) // 2, 1,
                           True, 0) for (c, k, s, h) in DW_LAYERS]
+
+
+def dense_bias(case: DenseCase):
+    """Seeded float32 bias[Cout] ~ N(0, 0.1) of a case with a bias (None otherwise)."""
+    if not case.bias:
+        return None
+    return normal(stream_seed(case.seed, 2), case.Cout, math.sqrt(0.1))
 
 
 def dense_inputs(case: DenseCase):
