@@ -23,9 +23,9 @@
 // groups added in j order in fp32, one rounding to bf16 -- a different order from the other
 // kernels, within the same error bound.
 //
-// Roles: warp 0 TMA, warp 1 TMEM + MMA, warps 2..9 epilogue (two warps per TMEM lane quarter,
-// 32 output channels each, so two epilogue warps share each SM sub-partition and hide each
-// other's TMEM-load and shuffle latencies); the filter is always resident here.
+// Roles: warp 0 TMA, warp 1 TMEM + MMA, then the epilogue warps: 64/CW per TMEM lane quarter,
+// CW output channels each (CW = 16: 16 warps, four per SM sub-partition, hiding each other's
+// TMEM-load, shuffle and store latencies); the filter is always resident here.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -49,25 +49,30 @@ struct DenseFoldParams {
     FastDiv div_w, div_h;
 };
 
-template <int KF>
+template <int KF, int CW_ = 16>
 struct DenseFoldCfg {
     static constexpr int K = KF;
     static constexpr int NF = 64 * KF;                 // MMA N: K groups of 64 columns
     static constexpr int BM = 128;
     static constexpr int TM = BM - (KF - 1);           // output rows kept per tile
     static constexpr int SLOT_BYTES = 64 * 64 * 2;     // one (tap, channel block) filter slot
-    static constexpr int NUM_EPI = 8;                  // epilogue warps: 4 lane quarters x 2 column halves
+    static constexpr int CW = CW_;                     // output channels per epilogue warp
+    static constexpr int G = CW / 16;                  // 16-column TMEM chunks per warp
+    static constexpr int CPR = CW / 8;                 // 16-byte chunks per staged row
+    static constexpr int RPL = 64 / CW;                // staged rows per 128 bytes
+    static constexpr int NUM_EPI = 4 * (64 / CW);      // epilogue warps: 4 lane quarters x 64/CW column slices
     static constexpr int THREADS = 64 + 32 * NUM_EPI;
-    static constexpr int EPI_BYTES = NUM_EPI * 32 * 64;   // per-warp 32 rows x 32 channels staging
+    static constexpr int EPI_BYTES = NUM_EPI * 32 * CW * 2;   // per-warp 32 rows x CW channels staging
     static constexpr int MAX_RING = 8;
-    // exchange: lanes 0..j-1 of group j (j >= 1), 32 floats each, per warp and tile parity
-    static constexpr int XCH_FLOATS = KF * (KF - 1) / 2 * 32;
+    // exchange: lanes 0..j-1 of group j (j >= 1), CW floats each, per warp and tile parity
+    static constexpr int XCH_FLOATS = KF * (KF - 1) / 2 * CW;
     static constexpr int XCH_BYTES = 2 * NUM_EPI * XCH_FLOATS * 4;
-    static constexpr int NUM_BARS = 2 * MAX_RING /*halo*/ + 1 /*filter*/ + 4 /*acc*/ + 2 /*xch*/ + 1;
+    static constexpr int NUM_BARS = 2 * MAX_RING /*halo*/ + 4 /*filter rows*/ + 4 /*acc*/ + 2 /*xch*/ + 1;
     static constexpr int TMEM_COLS = 2 * NF <= 256 ? 256 : 512;
     static constexpr uint32_t IDESC = idesc_bf16_f32(BM, NF, /*B MN-major*/ true);
     static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + XCH_BYTES + NUM_BARS * 8 + NUM_EPI * 32 * 8 + 16;
     static_assert(KF >= 2 && KF <= 4, "N = 64*K must stay within 256");
+    static_assert(CW == 16 || CW == 32, "CW");
 };
 
 // st.shared.v4 executed only where pred != 0 (predicated, no branch)
@@ -105,11 +110,11 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     constexpr int R = Cfg::MAX_RING;
     auto hfull = [&](int s) { return bars + 8u * s; };
     auto hempty = [&](int s) { return bars + 8u * (R + s); };
-    const uint32_t bfull = bars + 8u * (2 * R);
-    auto accf = [&](int b) { return bars + 8u * (2 * R + 1 + b); };
-    auto acce = [&](int b) { return bars + 8u * (2 * R + 3 + b); };
-    auto xbar = [&](int b) { return bars + 8u * (2 * R + 5 + b); };
-    const uint32_t done_bar = bars + 8u * (2 * R + 7);
+    auto bfull = [&](int i) { return bars + 8u * (2 * R + i); };   // filter row i resident
+    auto accf = [&](int b) { return bars + 8u * (2 * R + 4 + b); };
+    auto acce = [&](int b) { return bars + 8u * (2 * R + 6 + b); };
+    auto xbar = [&](int b) { return bars + 8u * (2 * R + 8 + b); };
+    const uint32_t done_bar = bars + 8u * (2 * R + 10);
     const uint32_t rowoff_all = sEpi + Cfg::EPI_BYTES + Cfg::XCH_BYTES + Cfg::NUM_BARS * 8;   // s64 per row
     uint32_t *tmem_holder =
         reinterpret_cast<uint32_t *>(smem + epi_off + Cfg::EPI_BYTES + Cfg::XCH_BYTES + Cfg::NUM_BARS * 8 +
@@ -124,7 +129,7 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             mbar_init(hfull(s), 1);
             mbar_init(hempty(s), 1);
         }
-        mbar_init(bfull, 1);
+        for (int i = 0; i < K; ++i) mbar_init(bfull(i), 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf(b), 1);
             mbar_init(acce(b), Cfg::NUM_EPI);   // one arrival per epilogue warp
@@ -156,12 +161,16 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         // ------------------------------- TMA producer -------------------------------
         uint32_t hit = 0;
         bool ok = true, filter_issued = false;
+        // the filter row by row, each with its own barrier, so the first tile's MMAs for
+        // row 0 start while rows 1.. are still in flight
         auto load_filter = [&]() {
             if (lane == 0) {
-                mbar_arrive_expect_tx(bfull, p.num_kblk * Cfg::SLOT_BYTES);
-                for (int kb = 0; kb < p.num_kblk; ++kb) {
-                    const int cb = kb / p.KK, tap = kb - cb * p.KK;
-                    tma_load_3d(sB + kb * Cfg::SLOT_BYTES, &tmF, bfull, 0, cb * 64, tap);
+                for (int i = 0; i < K; ++i) {
+                    mbar_arrive_expect_tx(bfull(i), p.num_cblk * K * Cfg::SLOT_BYTES);
+                    for (int cb = 0; cb < p.num_cblk; ++cb)
+                        for (int j = 0; j < K; ++j)
+                            tma_load_3d(sB + (cb * p.KK + i * K + j) * Cfg::SLOT_BYTES, &tmF, bfull(i), 0, cb * 64,
+                                        i * K + j);
                 }
             }
             __syncwarp();
@@ -188,13 +197,14 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (!filter_issued) load_filter();
         if (!ok && lane == 0) fail();
         // Drain: every load issued has landed before the CTA may exit.
-        if (!mbar_wait_warp(bfull, 0) && lane == 0) fail();
+        for (int i = 0; i < K; ++i)
+            if (!mbar_wait_warp(bfull(i), 0)) { if (lane == 0) fail(); break; }
         for (uint32_t j = hit > (uint32_t)p.HS ? hit - p.HS : 0u; j < hit; ++j)
             if (!mbar_wait_warp(hfull(j % p.HS), (j / p.HS) & 1u)) { if (lane == 0) fail(); break; }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
         uint32_t hit = 0, local = 0;
-        bool ok = mbar_wait_warp(bfull, 0);
+        bool ok = mbar_wait_warp(bfull(0), 0);
         for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step, ++local) {
             const uint32_t b = local & 1u;
             // the epilogue is the slower role: sleep between polls instead of taking its issue slots
@@ -205,6 +215,7 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
                 if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
                 tc_fence_after();
+                uint32_t filter_ok = 1;
                 if (lane == 0) {
                     // filter row i reads the halo from row i*W on (start field in 16-byte
                     // units: +8 per 128-byte row, +2 per 16 channels); B spans the K slots
@@ -212,6 +223,7 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const uint64_t a0 = smem_desc_sw128(sH + hs * p.halo_bytes, 16, 1024);
 #pragma unroll
                     for (int i = 0; i < K; ++i) {
+                        if (local == 0 && cb == 0 && i > 0 && !mbar_wait(bfull(i), 0)) { filter_ok = 0; break; }
                         const uint64_t ad = a0 + static_cast<uint64_t>(i * p.W * 8);
                         const uint64_t bd = smem_desc_sw128(sB + (cb * p.KK + i * K) * Cfg::SLOT_BYTES,
                                                             Cfg::SLOT_BYTES, 1024);
@@ -222,7 +234,7 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     }
                     umma_commit(hempty(hs));
                 }
-                __syncwarp();
+                if (!__shfl_sync(0xffffffffu, filter_ok, 0)) { ok = false; break; }
                 ++hit;
             }
             if (!ok) break;
@@ -238,11 +250,12 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     } else {
         // ------------------------------- Epilogue -----------------------------------
         // warp e = warp - 2: TMEM lane quarter q = warp % 4 (the quarter a warp may access),
-        // output channels 32h .. 32h + 31 with h = e / 4
+        // output channels CW*h .. CW*h + CW - 1 with h = e / 4
+        constexpr int CW = Cfg::CW, G = Cfg::G, CPR = Cfg::CPR, RPL = Cfg::RPL;
         const int e = warp - 2;
         const int q = warp & 3;
         const int h = e >> 2;
-        const uint32_t stage = sEpi + e * 2048;
+        const uint32_t stage = sEpi + e * (32 * CW * 2);
         const uint32_t rowoff = rowoff_all + e * 32 * 8;
         uint32_t local = 0;
         for (int t = first; t < p.num_tiles; t += step, ++local) {
@@ -265,26 +278,26 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
                 asm volatile("st.shared.s64 [%0], %1;" ::"r"(rowoff + 8u * lane), "l"(off) : "memory");
             }
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * NF + h * 32;
-            // one round trip to TMEM: all K groups of this warp's 32 columns
-            uint32_t d[K][2][16];
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * NF + h * CW;
+            // one round trip to TMEM: all K groups of this warp's CW columns
+            uint32_t d[K][G][16];
 #pragma unroll
             for (int j = 0; j < K; ++j)
 #pragma unroll
-                for (int g = 0; g < 2; ++g) tmem_ld_32x32b_x16(t_row + j * 64 + g * 16, d[j][g]);
+                for (int g = 0; g < G; ++g) tmem_ld_32x32b_x16(t_row + j * 64 + g * 16, d[j][g]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acce(b));   // accumulator read: the MMA warp may reuse it
             // publish lanes 0..j-1 of groups j >= 1 for the warp of the quarter above
             if (q > 0) {
-                const uint32_t my_x = sX + 4u * ((par * 4 + q) * 2 + h) * Cfg::XCH_FLOATS;
+                const uint32_t my_x = sX + 4u * ((par * 4 + q) * (64 / CW) + h) * Cfg::XCH_FLOATS;
 #pragma unroll
                 for (int j = 1; j < K; ++j) {
                     const uint32_t pub = lane < j ? 1u : 0u;   // predicated stores: no divergent branch
-                    const uint32_t dst = my_x + 4u * (j * (j - 1) / 2 + (lane < j ? lane : 0)) * 32;
+                    const uint32_t dst = my_x + 4u * (j * (j - 1) / 2 + (lane < j ? lane : 0)) * CW;
 #pragma unroll
-                    for (int g = 0; g < 2; ++g)
+                    for (int g = 0; g < G; ++g)
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
                             st_shared_v4_if(pub, dst + 16u * (g * 4 + c), d[j][g][4 * c], d[j][g][4 * c + 1],
@@ -293,11 +306,11 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
             __syncwarp();   // the lanes' exchange stores are ordered before lane 0's release
             if (lane == 0) mbar_arrive(xbar(par));
-            const uint32_t next_x = sX + 4u * ((par * 4 + (q < 3 ? q + 1 : q)) * 2 + h) * Cfg::XCH_FLOATS;
+            const uint32_t next_x = sX + 4u * ((par * 4 + (q < 3 ? q + 1 : q)) * (64 / CW) + h) * Cfg::XCH_FLOATS;
             const bool xok = mbar_wait_warp_backoff(xbar(par), (local >> 1) & 1u, 32);
-            const uint32_t row_addr = stage + lane * 64;
+            const uint32_t row_addr = stage + lane * (CW * 2);
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
+            for (int g = 0; g < G; ++g) {
                 float y[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c) y[c] = __uint_as_float(d[0][g][c]);
@@ -307,7 +320,7 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     // loads (a valid address, mostly a broadcast) and selects, so nothing diverges
                     const bool from_next = lane + j >= 32;
                     const bool from_smem = from_next && q < 3 && xok;
-                    const uint32_t src = next_x + 4u * ((j * (j - 1) / 2 + (from_next ? lane + j - 32 : 0)) * 32 + g * 16);
+                    const uint32_t src = next_x + 4u * ((j * (j - 1) / 2 + (from_next ? lane + j - 32 : 0)) * CW + g * 16);
                     float xv[16];
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -321,33 +334,33 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         y[c] = __fadd_rn(y[c], v);
                     }
                 }
-                // 64-byte staging rows, 16-byte chunks swizzled by (row / 2) % 4: conflict-free
-                // writes (one row per lane) and reads (two rows per 8 lanes)
+                // 2*CW-byte staging rows, 16-byte chunks swizzled by (row / RPL) % CPR:
+                // conflict-free writes (one row per lane) and reads (RPL rows per 8 lanes)
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const uint32_t c = g * 2 + cc;
                     const float *v = &y[cc * 8];
-                    st_shared_v4(row_addr + ((c ^ ((lane >> 1) & 3)) << 4), halo_pack_bf16x2(v[0], v[1]),
+                    st_shared_v4(row_addr + ((c ^ ((lane / RPL) % CPR)) << 4), halo_pack_bf16x2(v[0], v[1]),
                                  halo_pack_bf16x2(v[2], v[3]), halo_pack_bf16x2(v[4], v[5]),
                                  halo_pack_bf16x2(v[6], v[7]));
                 }
             }
             if (!xok) { if (lane == 0) fail(); break; }
             __syncwarp();
-            // coalesced stores: 4 lanes per 64-byte row, 8 rows per instruction
-            const int cc = lane & 3;
-            const int col = h * 32 + cc * 8;
+            // coalesced stores: CPR lanes per staged row, 32 / CPR rows per instruction
+            const int cc = lane % CPR;
+            const int col = h * CW + cc * 8;
             if (col < p.Cout) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int rr = i * 8 + (lane >> 2);
+                for (int i = 0; i < CPR; ++i) {
+                    const int rr = i * (32 / CPR) + lane / CPR;
                     long long off;
                     asm volatile("ld.shared.s64 %0, [%1];" : "=l"(off) : "r"(rowoff + 8u * rr));
                     if (off >= 0) {
                         uint32_t a, bb, c, dd;
                         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                      : "=r"(a), "=r"(bb), "=r"(c), "=r"(dd)
-                                     : "r"(stage + rr * 64 + ((cc ^ ((rr >> 1) & 3)) << 4)));
+                                     : "r"(stage + rr * (CW * 2) + ((cc ^ ((rr / RPL) % CPR)) << 4)));
                         *reinterpret_cast<uint4 *>(Y + off + col) = make_uint4(a, bb, c, dd);
                     }
                 }
