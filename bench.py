@@ -72,6 +72,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
+    "dense_fold_kernel": ("dense_fold.cuh", "dense_halo.cuh", "dense_tc.cuh", "depthwise.cuh", "ptx.cuh"),
     "dense_halo_kernel": ("dense_halo.cuh", "ptx.cuh"),
     "dense_tc_kernel": ("dense_tc.cuh", "ptx.cuh"),
     "dense_direct_kernel": ("dense_direct.cuh",),
