@@ -52,7 +52,9 @@ def workload_table():
     t = {"dense3x3": ("dense", workloads.DENSE_3X3, None),
          "pointwise": ("dense", workloads.DENSE_1X1, None),
          "dense-large": ("dense", workloads.DENSE_LARGE, None),
-         "dense-s2": ("dense", workloads.DENSE_S2, None)}
+         "dense-s2": ("dense", workloads.DENSE_S2, None),
+         # comparison path: explicit patch matrix + one cuBLAS GEMM, packing inside the timing
+         "dense3x3-explicit-im2col": ("dense", workloads.DENSE_3X3, "im2col")}
     for c in workloads.DW_SWEEP:
         for mode, name in ((0, "exact"), (1, "fast")):
             t[f"dw-C{c.C}-K{c.KH}-s{c.stride}-H{c.H}-{name}"] = ("depthwise", c, mode)
@@ -289,12 +291,21 @@ def dense_plain(case):
     return case.stride == 1 and case.pad == 0 and case.dil == 1 and not case.bias
 
 
-def dense_call(cb, case, X, F, b, Y):
-    """The public entry a user calls for this case: the plain one, or the one with stride,
-    padding, dilation and bias."""
+def dense_call(cb, case, X, F, b, Y, mode=None, ws=None):
+    """The public entry a user calls for this case: the plain one, the one with stride,
+    padding, dilation and bias, or (mode "im2col") the explicit-im2col comparison path."""
+    if mode == "im2col":
+        return cb.conv2d_nhwc_fwd_im2col(X, F, Y, workspace=ws)
     if dense_plain(case):
         return cb.conv2d_nhwc_fwd(X, F, Y)
     return cb.conv2d_nhwc_fwd_ex(X, F, b, Y, case.stride, case.pad, case.dil)
+
+
+def im2col_workspace(cb, torch, case, mode):
+    if mode != "im2col":
+        return None
+    return torch.empty(cb.lib.conv2d_nhwc_im2col_workspace(case.N, case.H, case.W, case.Cin, case.K),
+                       dtype=torch.uint8, device="cuda")
 
 
 def dw_device_inputs(torch, case, seed):
@@ -315,8 +326,9 @@ def steps_fns(cb, torch, kind, case, mode, inputs):
         Fs = [F0.clone() for _ in range(R)]
         Ys = [torch.empty((case.N, case.Ho, case.Wo, case.Cout), dtype=X0.dtype, device=X0.device)
               for _ in range(R)]
-        fns = [(lambda i=i: dense_call(cb, case, Xs[i], Fs[i], b0, Ys[i])) for i in range(R)]
-        keep = (Xs, Fs, Ys, b0)
+        ws = im2col_workspace(cb, torch, case, mode)
+        fns = [(lambda i=i: dense_call(cb, case, Xs[i], Fs[i], b0, Ys[i], mode, ws)) for i in range(R)]
+        keep = (Xs, Fs, Ys, b0, ws)
     else:
         x0, w0, b0 = inputs
         xs = [x0.clone() for _ in range(R)]
@@ -344,13 +356,14 @@ def e2e_bench(cb, torch, kind, case, mode, host, steps, warmup):
     else:
         out = torch.empty((case.N, case.C * case.mult, case.Ho, case.Wo), device="cuda")
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    ws = im2col_workspace(cb, torch, case, mode) if kind == "dense" else None
 
     def step():
         for d, h in zip(dev, host):
             if h is not None:
                 d.copy_(h, non_blocking=True)
         if kind == "dense":
-            dense_call(cb, case, dev[0], dev[1], dev[2], out)
+            dense_call(cb, case, dev[0], dev[1], dev[2], out, mode, ws)
         else:
             cb.depthwise_fwd(dev[0], dev[1], dev[2], out, case.stride, case.pad, case.dil, mode)
         out_h.copy_(out, non_blocking=True)
@@ -449,6 +462,8 @@ def run_ours(args, dist):
         cfg = {"workload": case.name, "N_per_gpu": case.N, "H": case.H, "W": case.W, "Cin": case.Cin,
                "Cout": case.Cout, "K": case.K, "stride": case.stride, "pad": case.pad, "dil": case.dil,
                "bias": case.bias, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
+        if mode == "im2col":
+            cfg["path"] = "explicit patch matrix in a workspace + one cuBLAS GEMM (comparison path)"
     else:
         unit, work, scale = "GB/s", case.bytes, 1e9
         achieved = case.bytes / (ms_step * 1e-3) / 1e9

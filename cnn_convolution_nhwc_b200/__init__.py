@@ -37,6 +37,10 @@ lib.conv2d_nhwc_fwd_f32.argtypes = [_P, _P, _P] + [_I] * 6 + [_P]
 lib.conv2d_nhwc_fwd_f32.restype = _I
 lib.conv2d_nhwc_fwd_ex.argtypes = [_P, _P, _P, _P] + [_I] * 9 + [_P]
 lib.conv2d_nhwc_fwd_ex.restype = _I
+lib.conv2d_nhwc_im2col_workspace.argtypes = [_I] * 5
+lib.conv2d_nhwc_im2col_workspace.restype = ctypes.c_size_t
+lib.conv2d_nhwc_fwd_im2col.argtypes = [_P, _P, _P, _P, ctypes.c_size_t] + [_I] * 6 + [_P]
+lib.conv2d_nhwc_fwd_im2col.restype = _I
 lib.depthwise_fwd.argtypes = [_P, _P, _P, _P] + [_I] * 11 + [_P]
 lib.depthwise_fwd.restype = _I
 lib.conv_status_string.argtypes = [_I]
@@ -48,7 +52,8 @@ lib.conv_last_kernel.restype = ctypes.c_char_p
 lib.conv_selftest_wait_timeout.argtypes = [_P]
 lib.conv_selftest_wait_timeout.restype = _I
 
-EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "depthwise_fwd", "conv_status_string",
+EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "conv2d_nhwc_im2col_workspace",
+           "conv2d_nhwc_fwd_im2col", "depthwise_fwd", "conv_status_string",
            "conv_device_status", "conv_last_kernel", "conv_selftest_wait_timeout")
 
 
@@ -147,6 +152,32 @@ def conv2d_nhwc_fwd_ex(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, stream=N
     py = _tensor(Y, torch.bfloat16, 4, "Y")
     _check(lib.conv2d_nhwc_fwd_ex(px, pf, pb, py, N, H, W, Cin, Cout, K, stride, pad, dil, _stream(stream)),
            "conv2d_nhwc_fwd_ex")
+    return Y
+
+
+def conv2d_nhwc_fwd_im2col(X, F, Y=None, workspace=None, stream=None):
+    """Comparison path: explicit patch matrix in `workspace` (allocated here if None, as a uint8
+    CUDA tensor of conv2d_nhwc_im2col_workspace bytes), then one cuBLAS GEMM."""
+    import torch
+    px = _tensor(X, torch.bfloat16, 4, "X")
+    pf = _tensor(F, torch.bfloat16, 4, "F")
+    N, H, W, Cin = X.shape
+    K, K2, Cin2, Cout = F.shape
+    if K != K2 or Cin2 != Cin:
+        raise ValueError("F must be [K, K, Cin, Cout] matching X")
+    need = lib.conv2d_nhwc_im2col_workspace(N, H, W, Cin, K)
+    if need == 0:
+        raise ValueError("invalid shape")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    if not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if Y is None:
+        Y = torch.empty((N, H - K + 1, W - K + 1, Cout), dtype=torch.bfloat16, device=X.device)
+    py = _tensor(Y, torch.bfloat16, 4, "Y")
+    _check(lib.conv2d_nhwc_fwd_im2col(px, pf, py, ctypes.c_void_p(workspace.data_ptr()),
+                                      workspace.numel() * workspace.element_size(), N, H, W, Cin, Cout, K,
+                                      _stream(stream)), "conv2d_nhwc_fwd_im2col")
     return Y
 
 

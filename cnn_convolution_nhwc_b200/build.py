@@ -52,7 +52,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         try:
             if force or stale():
                 tmp = LIB + f".tmp{os.getpid()}"
-                cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, MAIN]
+                cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, MAIN, "-lcublas"]
                 r = subprocess.run(cmd, capture_output=True, text=True)
                 if r.returncode != 0:
                     raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)

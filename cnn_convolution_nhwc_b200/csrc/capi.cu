@@ -5,6 +5,7 @@
 // Lecture 14 notes, section 5 (positive dimensions, square filter no larger than the
 // image, matching shapes) and the output-size rule of "Convolution Is Wx+b Moving Across a
 // Signal" (section "Build an image-gradient map, one number at a time") for depthwise.
+#include <cublas_v2.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -19,6 +20,7 @@
 #include "dense_tc.cuh"
 #include "dense_halo.cuh"
 #include "dense_fold.cuh"
+#include "im2col_gemm.cuh"
 #include "depthwise.cuh"
 #include "depthwise_reg.cuh"
 #include "depthwise_tma.cuh"
@@ -70,6 +72,7 @@ struct DeviceState {
     int num_sms = 0;
     unsigned int *status = nullptr;   // device address of g_conv_status on this device
     unsigned long long attr_done = 0; // bit per kernel whose shared-memory limit is raised
+    cublasHandle_t blas = nullptr;    // for the explicit-im2col comparison path, made on first use
 };
 
 std::mutex g_mu;
@@ -882,6 +885,57 @@ int conv2d_nhwc_fwd_ex(const void *X, const void *F, const float *bias, void *Y,
     if (bn == 128) return launch_dense_tc<CfgBN128>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 1, g);
     if (bn == 256) return launch_dense_tc<CfgBN256>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 2, g);
     return CONV_ERR_INVALID_ARG;
+}
+
+size_t conv2d_nhwc_im2col_workspace(int N, int H, int W, int Cin, int K) {
+    if (N < 1 || H < 1 || W < 1 || Cin < 1 || K < 1 || K > H || K > W) return 0;
+    return static_cast<size_t>(1ULL * N * (H - K + 1) * (W - K + 1) * K * K * Cin * 2);
+}
+
+int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspace, size_t workspace_bytes, int N,
+                           int H, int W, int Cin, int Cout, int K, cudaStream_t stream) {
+    if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 2)) return rc;
+    const size_t need = conv2d_nhwc_im2col_workspace(N, H, W, Cin, K);
+    if (!workspace || workspace_bytes < need) return CONV_ERR_INVALID_ARG;
+    const long long Ho = H - K + 1, Wo = W - K + 1, M = 1LL * N * Ho * Wo, kd = 1LL * K * K * Cin;
+    if (M * kd > kInt32Max * 4LL || M > kInt32Max || kd > kInt32Max) return CONV_ERR_UNSUPPORTED;
+    if (!aligned(workspace, 16)) return CONV_ERR_MISALIGNED;
+    const long long nx = 1LL * N * H * W * Cin, nf = kd * Cout, ny = M * Cout;
+    if (overlaps(workspace, static_cast<long long>(need), X, 2 * nx) ||
+        overlaps(workspace, static_cast<long long>(need), F, 2 * nf) ||
+        overlaps(workspace, static_cast<long long>(need), Y, 2 * ny))
+        return CONV_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!d->blas && cublasCreate(&d->blas) != CUBLAS_STATUS_SUCCESS) return CONV_ERR_CUDA;
+    }
+    Im2colParams p;
+    p.H = H; p.W = W; p.Cin = Cin; p.K = K; p.Ho = static_cast<int>(Ho); p.Wo = static_cast<int>(Wo);
+    p.kd = static_cast<int>(kd);
+    p.chunk = (Cin % 8 == 0 && aligned(X, 16)) ? 8 : 1;
+    p.chunks = M * kd / p.chunk;
+    long long blocks = (p.chunks + 255) / 256;
+    if (blocks > 1LL * d->num_sms * 8) blocks = 1LL * d->num_sms * 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    auto *A = static_cast<__nv_bfloat16 *>(workspace);
+    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p),
+                 "im2col_pack_kernel") != CONV_OK)
+        return CONV_ERR_CUDA;
+    // Y (M x Cout, row-major) = A (M x kd) * F (kd x Cout): in cuBLAS's column-major terms
+    // Y^T = F^T * A^T with leading dimensions Cout, Cout and kd
+    const float alpha = 1.0f, beta = 0.0f;
+    if (cublasSetStream(d->blas, stream) != CUBLAS_STATUS_SUCCESS) return CONV_ERR_CUDA;
+    if (cublasGemmEx(d->blas, CUBLAS_OP_N, CUBLAS_OP_N, Cout, static_cast<int>(M), static_cast<int>(kd), &alpha, F,
+                     CUDA_R_16BF, Cout, A, CUDA_R_16BF, static_cast<int>(kd), &beta, Y, CUDA_R_16BF, Cout,
+                     CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+        return CONV_ERR_CUDA;
+    t_last_kernel = "im2col_pack_kernel+cublas";
+    return CONV_OK;
 }
 
 int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, int N, int Cin, int mult, int H,

@@ -102,6 +102,22 @@ int conv2d_nhwc_fwd_ex(const void *X, const void *F, const float *bias, void *Y,
                        int stride, int pad, int dil, cudaStream_t stream);
 
 /*
+ * Comparison path: the same operation as conv2d_nhwc_fwd computed the way the CMU DLSys Lecture
+ * 14 notes build it in section 5 "Generalize the patch matrix to channels and batches" -- an
+ * explicit patch matrix A[(n,y,x), (i,j,c)] = X[n,y+i,x+j,c] of N*Ho*Wo rows by K*K*Cin columns,
+ * written to `workspace`, then one library GEMM Y = A * F (cuBLAS: bf16 operands, float32
+ * accumulation, bf16 output). It exists to measure the storage bill of section 6 against the
+ * implicit kernels; the pages have no separate definition for it.
+ *   workspace       : DEVICE memory owned by the caller, at least conv2d_nhwc_im2col_workspace()
+ *                     bytes, 16-byte aligned, not overlapping X, F or Y; overwritten
+ * Requirements as conv2d_nhwc_fwd. The first call on a device creates a cuBLAS handle (which
+ * allocates cuBLAS's own workspace); later calls allocate nothing.
+ */
+size_t conv2d_nhwc_im2col_workspace(int N, int H, int W, int Cin, int K);   /* 0 if invalid */
+int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspace, size_t workspace_bytes,
+                           int N, int H, int W, int Cin, int Cout, int K, cudaStream_t stream);
+
+/*
  * Depthwise forward convolution, float32.
  *   x    : [N][Cin][H][W]
  *   w    : [Cin*mult][KH][KW]   (plane oc belongs to input channel oc / mult)

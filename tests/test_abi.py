@@ -133,3 +133,24 @@ def test_last_kernel_is_empty_before_any_launch():
     # rejected calls launch nothing, so the dispatcher's record stays empty on a CPU-only host
     assert cb.lib.conv2d_nhwc_fwd(None, F, Y, 1, 5, 5, 8, 8, 3, None) == cb.CONV_ERR_INVALID_ARG
     assert cb.conv_last_kernel() == ""
+
+
+def test_im2col_workspace_size():
+    # N*Ho*Wo rows of K*K*Cin bf16 values (the DLSys notes' patch matrix)
+    assert cb.lib.conv2d_nhwc_im2col_workspace(32, 56, 56, 64, 3) == 32 * 54 * 54 * 9 * 64 * 2
+    assert cb.lib.conv2d_nhwc_im2col_workspace(1, 6, 6, 1, 3) == 16 * 9 * 2
+    assert cb.lib.conv2d_nhwc_im2col_workspace(1, 2, 6, 1, 3) == 0     # K > H
+    assert cb.lib.conv2d_nhwc_im2col_workspace(0, 6, 6, 1, 3) == 0
+
+
+WS = V(1 << 32)
+
+
+@pytest.mark.parametrize("ws,nbytes,code", [
+    (None, 1 << 20, cb.CONV_ERR_INVALID_ARG),
+    (WS, 100, cb.CONV_ERR_INVALID_ARG),                     # smaller than the patch matrix
+    (V((1 << 32) + 8), 1 << 20, cb.CONV_ERR_MISALIGNED),     # not 16-byte aligned
+    (V((1 << 20) - 64), 1 << 20, cb.CONV_ERR_INVALID_ARG),   # overlaps X
+])
+def test_im2col_path_rejects(ws, nbytes, code):
+    assert cb.lib.conv2d_nhwc_fwd_im2col(X, F, Y, ws, nbytes, 1, 5, 5, 8, 8, 3, None) == code
