@@ -24,6 +24,7 @@
 #include "depthwise.cuh"
 #include "depthwise_reg.cuh"
 #include "depthwise_tma.cuh"
+#include "depthwise_plane.cuh"
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -71,7 +72,7 @@ struct DeviceState {
     bool ready = false;
     int num_sms = 0;
     unsigned int *status = nullptr;   // device address of g_conv_status on this device
-    unsigned long long attr_done = 0; // bit per kernel whose shared-memory limit is raised
+    unsigned long long attr_done[2] = {0, 0};   // bit per kernel whose shared-memory limit is raised
     cublasHandle_t blas = nullptr;    // for the explicit-im2col comparison path, made on first use
 };
 
@@ -113,11 +114,11 @@ int device_state(DeviceState **out) {
 
 template <typename Kern>
 int ensure_smem_attr(DeviceState *d, unsigned bit, Kern kern, int bytes) {
-    if (d->attr_done & (1ull << bit)) return CONV_OK;
+    if (d->attr_done[bit >> 6] & (1ull << (bit & 63))) return CONV_OK;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return CONV_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    d->attr_done |= 1ull << bit;
+    d->attr_done[bit >> 6] |= 1ull << (bit & 63);
     return CONV_OK;
 }
 
@@ -766,6 +767,70 @@ int launch_dw_tma(const float *x, const float *w, const float *bias, float *y, c
     return launch_dw_tma_one<MODE, HB, 5, 2>(x, w, bias, y, pl, Cin, N, stream, d, base + 3);
 }
 
+// ---- lane-per-plane kernel (7x7 and 14x14 planes) --------------------------------------------
+struct DwPlanePlan {
+    bool ok = false;
+    DwPlaneParams p{};
+    int grid = 0;
+    int smem = 0;
+};
+
+DwPlanePlan dw_plane_plan(int N, int Cin, int mult, int H, int W, int K, int S, int num_sms, const float *x,
+                          const float *y) {
+    DwPlanePlan pl;
+    if (mult != 1 || H != W || (H != 7 && H != 14) || !aligned(x, 16)) return pl;
+    const int HW = H, PAD = (K - 1) / 2;
+    const int HO = (HW + 2 * PAD - K) / S + 1;
+    const int LPP = HW <= 8 ? 1 : 2, PPJ = 32 / LPP;
+    DwPlaneParams &p = pl.p;
+    p.C = Cin;
+    p.num_planes = N * Cin;
+    p.num_jobs = (p.num_planes + PPJ - 1) / PPJ;
+    p.in_floats = (PPJ * HW * HW + 31) & ~31;
+    p.out_floats = (PPJ * HO * HO + 31) & ~31;
+    p.vec_y = aligned(y, 16) ? 1 : 0;
+    p.div_c = make_fastdiv(static_cast<uint32_t>(Cin));
+    pl.smem = kDwPlaneWarps * (p.in_floats + p.out_floats) * 4;
+    if (pl.smem > 200 * 1024) return pl;
+    int per_sm = (227 * 1024) / (pl.smem + 1024);
+    if (per_sm > 8) per_sm = 8;
+    if (per_sm < 1) return pl;
+    const long long g_jobs = (p.num_jobs + kDwPlaneWarps - 1) / kDwPlaneWarps;
+    const long long g = 1LL * num_sms * per_sm;
+    pl.grid = static_cast<int>(g < g_jobs ? g : g_jobs);
+    pl.ok = true;
+    return pl;
+}
+
+template <int MODE, bool HB, int K, int S, int HW>
+int launch_dw_plane_one(const float *x, const float *w, const float *bias, float *y, const DwPlanePlan &pl,
+                        cudaStream_t stream, DeviceState *d, unsigned bit) {
+    auto kern = depthwise_plane_kernel<MODE, HB, K, S, HW>;
+    if (pl.smem > 48 * 1024)
+        if (int rc = ensure_smem_attr(d, bit, kern, 200 * 1024)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(32 * kDwPlaneWarps);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, pl.p, d->status), "depthwise_plane_kernel");
+}
+
+template <int MODE, bool HB>
+int launch_dw_plane(const float *x, const float *w, const float *bias, float *y, const DwPlanePlan &pl, int K, int S,
+                    int HW, cudaStream_t stream, DeviceState *d) {
+    // shared-memory attribute bits 64..95: (MODE, HB) x (K, S, HW)
+    const unsigned b = 64u + 8u * (2u * MODE + (HB ? 1u : 0u));
+    if (K == 3 && S == 1 && HW == 7) return launch_dw_plane_one<MODE, HB, 3, 1, 7>(x, w, bias, y, pl, stream, d, b + 0);
+    if (K == 3 && S == 2 && HW == 7) return launch_dw_plane_one<MODE, HB, 3, 2, 7>(x, w, bias, y, pl, stream, d, b + 1);
+    if (K == 5 && S == 1 && HW == 7) return launch_dw_plane_one<MODE, HB, 5, 1, 7>(x, w, bias, y, pl, stream, d, b + 2);
+    if (K == 5 && S == 2 && HW == 7) return launch_dw_plane_one<MODE, HB, 5, 2, 7>(x, w, bias, y, pl, stream, d, b + 3);
+    if (K == 3 && S == 1) return launch_dw_plane_one<MODE, HB, 3, 1, 14>(x, w, bias, y, pl, stream, d, b + 4);
+    if (K == 3 && S == 2) return launch_dw_plane_one<MODE, HB, 3, 2, 14>(x, w, bias, y, pl, stream, d, b + 5);
+    if (K == 5 && S == 1) return launch_dw_plane_one<MODE, HB, 5, 1, 14>(x, w, bias, y, pl, stream, d, b + 6);
+    return launch_dw_plane_one<MODE, HB, 5, 2, 14>(x, w, bias, y, pl, stream, d, b + 7);
+}
+
 template <int MODE, bool HB>
 int launch_dw(const float *x, const float *w, const float *bias, float *y, const DwParams &p, DwSpec s,
               long long jobs, cudaStream_t stream, DeviceState *d) {
@@ -968,6 +1033,20 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
     const bool reg_ok = dw_reg_eligible(KH, KW, stride, pad, dil, Wo) && 1LL * N * Cout <= kInt32Max;
     if (force_reg && !reg_ok) return CONV_ERR_UNSUPPORTED;
     const bool force_tma = kforce && std::strcmp(kforce, "tma") == 0;
+    const bool force_plane = kforce && std::strcmp(kforce, "plane") == 0;
+    // 7x7 and 14x14 planes: a lane per plane (CONV_B200_DW_KERNEL=plane forces it)
+    if (reg_ok && !force_smem && !force_reg && !force_tma && !env("CONV_B200_DW_TILE")) {
+        const DwPlanePlan pp = dw_plane_plan(N, Cin, mult, H, W, KH, stride, d->num_sms, x, y);
+        if (pp.ok) {
+            const bool hb = bias != nullptr;
+            if (mode == DW_EXACT)
+                return hb ? launch_dw_plane<0, true>(x, w, bias, y, pp, KH, stride, H, stream, d)
+                          : launch_dw_plane<0, false>(x, w, bias, y, pp, KH, stride, H, stream, d);
+            return hb ? launch_dw_plane<1, true>(x, w, bias, y, pp, KH, stride, H, stream, d)
+                      : launch_dw_plane<1, false>(x, w, bias, y, pp, KH, stride, H, stream, d);
+        }
+    }
+    if (force_plane) return CONV_ERR_UNSUPPORTED;
     if (reg_ok && !force_smem && !force_reg && !env("CONV_B200_DW_TILE")) {
         const DwTmaPlan tp = dw_tma_plan(N, Cin, mult, H, W, static_cast<int>(Ho), static_cast<int>(Wo), KH, stride,
                                          d->num_sms, x, y);

@@ -1,0 +1,163 @@
+// Depthwise forward convolution for small square planes (7x7, 14x14): a lane owns a plane.
+//
+// Same contract as depthwise.cuh (the OneModel "Depthwise convolution" page, section "What
+// each output is": acc = +0; ky outer, kx inner; padding a real zero that is multiplied; exact
+// mode __fmul_rn then __fadd_rn with NaN rewritten as 0x7FC00000; fast mode one __fmaf_rn per
+// tap; the bias one rounded addition afterwards), for compile-time plane size HW, K x K, stride
+// S, padding (K-1)/2, dilation 1, multiplier 1.
+//
+// Work layout. With planes this small, "lanes are neighbouring output columns" leaves most of a
+// warp idle or spread over many planes with tiny rows. Here one warp takes a job of 32 / LPP
+// consecutive planes -- one contiguous range of x -- and stages it into shared memory with a
+// single 1-D bulk copy. Each lane then computes a whole plane (LPP = 1) or half of its columns
+// (LPP = 2): every output row is WOL independent accumulations (no shuffles, no cross-lane
+// data), the rows are fully unrolled with a ring of K input rows in registers, and a plane
+// stride that is odd (7x7) keeps the lanes' shared loads in different banks. Outputs go to a
+// shared-memory staging area and leave as one contiguous, coalesced range of y. The next job's
+// bulk copy is issued as soon as the compute has read the input buffer.
+#pragma once
+#include <cstdint>
+
+#include "depthwise.cuh"
+#include "ptx.cuh"
+
+namespace convb200 {
+
+struct DwPlaneParams {
+    int C;               // channels (= planes per image, multiplier 1)
+    int num_planes;      // N * C
+    int num_jobs;        // ceil(num_planes / planes per job)
+    int in_floats;       // per-warp input buffer (planes per job * HW * HW, rounded to 4)
+    int out_floats;      // per-warp output staging (planes per job * HO * WO, rounded to 4)
+    int vec_y;           // 1: y 16-byte aligned
+    FastDiv div_c;
+};
+
+constexpr int kDwPlaneWarps = 4;
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+template <int MODE, bool HAS_BIAS, int K, int S, int HW>
+__global__ void __launch_bounds__(32 * kDwPlaneWarps)
+depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
+                       float *__restrict__ y, const DwPlaneParams p, unsigned int *status) {
+    constexpr int PAD = (K - 1) / 2;
+    constexpr int HO = (HW + 2 * PAD - K) / S + 1;
+    constexpr int WO = HO;
+    constexpr int LPP = HW <= 8 ? 1 : 2;            // lanes per plane
+    constexpr int PPJ = 32 / LPP;                   // planes per job
+    constexpr int WOL = (WO + LPP - 1) / LPP;       // output columns per lane
+    constexpr int WINC = (WOL - 1) * S + K;         // input columns a lane reads per row
+    extern __shared__ __align__(128) float sraw[];
+    __shared__ __align__(8) uint64_t full_all[kDwPlaneWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *sin = sraw + static_cast<size_t>(warp) * (p.in_floats + p.out_floats);
+    float *sout = sin + p.in_floats;
+    const uint32_t sin_s = static_cast<uint32_t>(__cvta_generic_to_shared(sin));
+    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&full_all[warp]));
+    const int gw = blockIdx.x * kDwPlaneWarps + warp;
+    const int GW = gridDim.x * kDwPlaneWarps;
+
+    // stage job `job`: its planes are one contiguous range of x; the 16-byte multiple goes by
+    // one bulk copy, the last 0..3 floats by lane 0
+    auto issue = [&](int job) {
+        const int plane0 = job * PPJ;
+        const int nplanes = min(PPJ, p.num_planes - plane0);
+        const uint32_t total = static_cast<uint32_t>(nplanes * HW * HW);
+        const uint32_t bulk = total & ~3u;
+        const float *src = x + static_cast<long long>(plane0) * (HW * HW);
+        if (lane == 0) {
+            for (uint32_t e = bulk; e < total; ++e) sin[e] = src[e];
+            mbar_arrive_expect_tx(bar, 4u * bulk);
+            if (bulk) bulk_g2s(sin_s, src, 4u * bulk, bar);
+        }
+    };
+
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (gw < p.num_jobs) issue(gw);
+
+    const int slot = lane / LPP;          // plane slot of this lane in the job
+    const int part = lane - slot * LPP;   // column part
+    const int ox0 = part * WOL;
+    const int ix0 = ox0 * S - PAD;        // first input column this lane reads
+    const float *pb = sin + slot * (HW * HW);
+
+    int k = 0;
+    bool ok = true;
+    for (int job = gw; job < p.num_jobs; job += GW, ++k) {
+        if (!mbar_wait_warp(bar, k & 1)) { ok = false; break; }
+        const int plane0 = job * PPJ;
+        const int plane = plane0 + slot;
+        const bool active = plane < p.num_planes;
+        const int c = active ? plane - fdiv(plane, p.div_c) * p.C : 0;
+        float wr[K * K];
+#pragma unroll
+        for (int t = 0; t < K * K; ++t) wr[t] = __ldg(w + c * (K * K) + t);
+        const float bv = HAS_BIAS ? __ldg(bias + c) : 0.0f;
+
+        // input row iy (compile-time) of this lane's columns; zeros outside the plane
+        auto load_row = [&](int iy, float (&row)[WINC]) {
+#pragma unroll
+            for (int t = 0; t < WINC; ++t) {
+                const int col = ix0 + t;
+                row[t] = (iy >= 0 && iy < HW && col >= 0 && col < HW) ? pb[iy * HW + col] : 0.0f;
+            }
+        };
+        float ring[K][WINC];
+#pragma unroll
+        for (int r = 0; r < K - S; ++r) load_row(r - PAD, ring[(r + K) % K]);
+#pragma unroll
+        for (int oy = 0; oy < HO; ++oy) {
+            // window rows oy*S - PAD + ky; ring slot of input row iy: (iy + PAD) % K
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                const int iy = oy * S - PAD + K - S + s;
+                load_row(iy, ring[(iy + PAD + K) % K]);
+            }
+            float acc[WOL];
+#pragma unroll
+            for (int v = 0; v < WOL; ++v) {
+                float a = 0.0f;
+#pragma unroll
+                for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                    for (int kx = 0; kx < K; ++kx)
+                        a = dw_tap<MODE>(a, wr[ky * K + kx], ring[(oy * S + ky) % K][v * S + kx]);
+                acc[v] = dw_finish<MODE, HAS_BIAS>(a, bv);
+            }
+#pragma unroll
+            for (int v = 0; v < WOL; ++v)
+                if (ox0 + v < WO) sout[slot * (HO * WO) + oy * WO + ox0 + v] = acc[v];
+        }
+        // the input buffer is free: stage the next job while this one's outputs leave
+        __syncwarp();
+        if (job + GW < p.num_jobs) issue(job + GW);
+        const int nplanes = min(PPJ, p.num_planes - plane0);
+        const int total = nplanes * (HO * WO);
+        float *gdst = y + static_cast<long long>(plane0) * (HO * WO);
+        if (p.vec_y && ((plane0 * (HO * WO)) & 3) == 0) {
+            const int n4 = total >> 2;
+            for (int e = lane; e < n4; e += 32)
+                reinterpret_cast<float4 *>(gdst)[e] = reinterpret_cast<const float4 *>(sout)[e];
+            for (int e = (n4 << 2) + lane; e < total; e += 32) gdst[e] = sout[e];
+        } else {
+            for (int e = lane; e < total; e += 32) gdst[e] = sout[e];
+        }
+        __syncwarp();
+    }
+    if (!ok) {
+        if (lane == 0) atomicOr(status, kStatusTimeout);
+        // the copy in flight lands before the warp exits (bounded wait)
+        mbar_wait_warp(bar, k & 1);
+    }
+}
+
+}  // namespace convb200

@@ -290,3 +290,24 @@ def test_forced_tma_refuses_unaligned_planes(cb):
     with pytest.raises(cb.ConvError) as e:
         _with_env("CONV_B200_DW_KERNEL", "tma", lambda: _gpu(cb, x, w, None, 1, 1, 1, 0))
     assert e.value.code == cb.CONV_ERR_UNSUPPORTED
+
+
+# (N, C, HW, K, S): 7x7 and 14x14 planes, a lane per plane; plane counts that leave a partial
+# last job, and (7x7, 33 planes) a last job whose size is not a 16-byte multiple
+PLANE_SHAPES = [(1, 33, 7, 5, 1), (2, 21, 7, 3, 1), (3, 5, 7, 3, 2), (1, 40, 7, 5, 2), (2, 9, 14, 3, 1),
+                (1, 17, 14, 5, 1), (2, 12, 14, 3, 2), (1, 7, 14, 5, 2)]
+
+
+@pytest.mark.parametrize("shape", PLANE_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_plane_kernel(cb, shape):
+    N, C, HW, K, S = shape
+    case = workloads.DepthwiseCase("plane", N, C, 1, HW, HW, K, K, S, (K - 1) // 2, 1, True, 17)
+    x, w, b = workloads.depthwise_inputs(case)
+    for mode in MODES:
+        yp = _gpu(cb, x, w, b, S, case.pad, 1, mode)
+        assert cb.conv_last_kernel() == "depthwise_plane_kernel"
+        ys = _with_env("CONV_B200_DW_KERNEL", "smem", lambda: _gpu(cb, x, w, b, S, case.pad, 1, mode))
+        assert np.array_equal(_bits(yp), _bits(ys))
+        _compare(yp, x, w, b, 1, S, case.pad, 1, mode)
+        yn = _gpu(cb, x, w, None, S, case.pad, 1, mode)          # no bias
+        _compare(yn, x, w, None, 1, S, case.pad, 1, mode)
