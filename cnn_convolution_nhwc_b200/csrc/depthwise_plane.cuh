@@ -19,6 +19,7 @@
 #include <cstdint>
 
 #include "depthwise.cuh"
+#include "depthwise_tma.cuh"   // packed-pair helpers
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -111,31 +112,101 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
                 row[t] = (iy >= 0 && iy < HW && col >= 0 && col < HW) ? pb[iy * HW + col] : 0.0f;
             }
         };
-        float ring[K][WINC];
-#pragma unroll
-        for (int r = 0; r < K - S; ++r) load_row(r - PAD, ring[(r + K) % K]);
-#pragma unroll
-        for (int oy = 0; oy < HO; ++oy) {
-            // window rows oy*S - PAD + ky; ring slot of input row iy: (iy + PAD) % K
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                const int iy = oy * S - PAD + K - S + s;
-                load_row(iy, ring[(iy + PAD + K) % K]);
-            }
-            float acc[WOL];
-#pragma unroll
-            for (int v = 0; v < WOL; ++v) {
-                float a = 0.0f;
-#pragma unroll
-                for (int ky = 0; ky < K; ++ky)
-#pragma unroll
-                    for (int kx = 0; kx < K; ++kx)
-                        a = dw_tap<MODE>(a, wr[ky * K + kx], ring[(oy * S + ky) % K][v * S + kx]);
-                acc[v] = dw_finish<MODE, HAS_BIAS>(a, bv);
-            }
+        auto store_row = [&](int oy, const float (&acc)[WOL]) {
 #pragma unroll
             for (int v = 0; v < WOL; ++v)
                 if (ox0 + v < WO) sout[slot * (HO * WO) + oy * WO + ox0 + v] = acc[v];
+        };
+        if constexpr (S == 1) {
+            // stride 1: the ring holds each row as its WINC - 1 overlapping pairs (x[t], x[t+1]);
+            // outputs (2q, 2q+1) at tap kx read pair 2q + kx (packed f32x2 arithmetic, the same
+            // roundings as the scalar path)
+            uint64_t w2[K * K];
+#pragma unroll
+            for (int t = 0; t < K * K; ++t) w2[t] = dw_pack(wr[t], wr[t]);
+            uint64_t ring[K][WINC - 1];
+            // element t of a row held as pairs: the low half of pair t, or for the last element
+            // the high half of the last pair
+            auto pair_elem = [&](const uint64_t (&row)[WINC - 1], int t) {
+                float lo, hi;
+                dw_unpack(row[t < WINC - 1 ? t : WINC - 2], lo, hi);
+                return t < WINC - 1 ? lo : hi;
+            };
+            auto load_pairs = [&](int iy, uint64_t (&dst)[WINC - 1]) {
+                float f[WINC];
+                load_row(iy, f);
+#pragma unroll
+                for (int t = 0; t < WINC - 1; ++t) dst[t] = dw_pack(f[t], f[t + 1]);
+            };
+#pragma unroll
+            for (int r = 0; r < K - 1; ++r) load_pairs(r - PAD, ring[r]);
+#pragma unroll
+            for (int oy = 0; oy < HO; ++oy) {
+                load_pairs(oy - PAD + K - 1, ring[(oy + K - 1) % K]);
+                float acc[WOL];
+                constexpr int NP = WOL / 2;
+                if constexpr (MODE == 0) {
+#pragma unroll
+                    for (int v = 0; v < WOL; ++v) acc[v] = 0.0f;
+#pragma unroll
+                    for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                        for (int kx = 0; kx < K; ++kx) {
+#pragma unroll
+                            for (int q = 0; q < NP; ++q)
+                                dw_tap2_exact(acc[2 * q], acc[2 * q + 1], w2[ky * K + kx], ring[(oy + ky) % K][2 * q + kx]);
+                            if constexpr (WOL % 2 == 1)
+                                acc[WOL - 1] = dw_tap<MODE>(acc[WOL - 1], wr[ky * K + kx],
+                                                            pair_elem(ring[(oy + ky) % K], WOL - 1 + kx));
+                        }
+                } else {
+                    uint64_t a2[NP > 0 ? NP : 1];
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) a2[q] = dw_pack(0.0f, 0.0f);
+                    float last = 0.0f;
+#pragma unroll
+                    for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                        for (int kx = 0; kx < K; ++kx) {
+#pragma unroll
+                            for (int q = 0; q < NP; ++q)
+                                a2[q] = dw_tap2_fast(a2[q], w2[ky * K + kx], ring[(oy + ky) % K][2 * q + kx]);
+                            if constexpr (WOL % 2 == 1)
+                                last = dw_tap<MODE>(last, wr[ky * K + kx], pair_elem(ring[(oy + ky) % K], WOL - 1 + kx));
+                        }
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) dw_unpack(a2[q], acc[2 * q], acc[2 * q + 1]);
+                    if constexpr (WOL % 2 == 1) acc[WOL - 1] = last;
+                }
+#pragma unroll
+                for (int v = 0; v < WOL; ++v) acc[v] = dw_finish<MODE, HAS_BIAS>(acc[v], bv);
+                store_row(oy, acc);
+            }
+        } else {
+            float ring[K][WINC];
+#pragma unroll
+            for (int r = 0; r < K - S; ++r) load_row(r - PAD, ring[(r + K) % K]);
+#pragma unroll
+            for (int oy = 0; oy < HO; ++oy) {
+                // window rows oy*S - PAD + ky; ring slot of input row iy: (iy + PAD) % K
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    const int iy = oy * S - PAD + K - S + s;
+                    load_row(iy, ring[(iy + PAD + K) % K]);
+                }
+                float acc[WOL];
+#pragma unroll
+                for (int v = 0; v < WOL; ++v) {
+                    float a = 0.0f;
+#pragma unroll
+                    for (int ky = 0; ky < K; ++ky)
+#pragma unroll
+                        for (int kx = 0; kx < K; ++kx)
+                            a = dw_tap<MODE>(a, wr[ky * K + kx], ring[(oy * S + ky) % K][v * S + kx]);
+                    acc[v] = dw_finish<MODE, HAS_BIAS>(a, bv);
+                }
+                store_row(oy, acc);
+            }
         }
         // the input buffer is free: stage the next job while this one's outputs leave
         __syncwarp();
