@@ -13,6 +13,9 @@ The arithmetic lives in ``conv_oracle.c`` (plain C, OpenMP over independent outp
 * ``conv2d_nhwc_ex`` -- the same sum with the stride, zero-padding, dilation and bias variants
   of "Convolution Is Wx+b Moving Across a Signal" (output-size rule of section "Build an
   image-gradient map, one number at a time"), float64.
+* ``conv2d_grouped`` -- the same sum split into channel groups, with per-axis geometry and a
+  KH x KW kernel (Conv1D is H = KH = 1), after the grouped Conv1D of the Wx+b page's CKE
+  section, float64.
 * ``depthwise`` -- the per-output loop of the OneModel "Depthwise convolution" page
   (section "What each output is"), in IEEE float32 in the page's order, exact or fast mode.
 
@@ -66,6 +69,8 @@ def _load():
         lib.oracle_conv2d_nhwc_ex.restype = I
         lib.oracle_conv2d_nhwc_ex_points.argtypes = [P, P, P, P, L, P, P] + [I] * 9
         lib.oracle_conv2d_nhwc_ex_points.restype = I
+        lib.oracle_conv2d_grouped.argtypes = [P, P, P, P, P] + [I] * 14
+        lib.oracle_conv2d_grouped.restype = I
         lib.oracle_depthwise.argtypes = [P, P, P, P] + [I] * 11
         lib.oracle_depthwise.restype = I
         lib.oracle_depthwise_points.argtypes = [P, P, P, P, L, P] + [I] * 11
@@ -165,6 +170,37 @@ def conv2d_nhwc_ex_points(X, F, flat_idx, bias=None, stride=1, pad=0, dil=1):
     _load().oracle_conv2d_nhwc_ex_points(_ptr(X), _ptr(F), _ptr(b), _ptr(idx), idx.size, _ptr(y), _ptr(a),
                                          N, H, W, Cin, Cout, K, stride, pad, dil)
     return y, a
+
+
+def _pair(v):
+    return (v, v) if isinstance(v, int) else (int(v[0]), int(v[1]))
+
+
+def conv2d_grouped(X, F, bias=None, stride=1, pad=0, dil=1, groups=1):
+    """Grouped NHWC convolution with per-axis stride / padding / dilation ((h, w) pairs or one
+    int for both) and a KH x KW kernel, float64. X: [N, H, W, Cin]; F: [KH, KW, Cin/groups, Cout]
+    (output channel o uses input channels of group o // (Cout/groups)); bias: [Cout] or None.
+    Conv1D is H = KH = 1. Returns (Y, abssum), float64 [N, Ho, Wo, Cout]."""
+    X, F = _f32(X), _f32(F)
+    b = None if bias is None else _f32(bias)
+    N, H, W, Cin = X.shape
+    KH, KW, Cg, Cout = F.shape
+    (sh, sw), (ph, pw), (dh, dw) = _pair(stride), _pair(pad), _pair(dil)
+    if groups < 1 or Cin % groups or Cout % groups or Cg * groups != Cin:
+        raise ValueError("channels must split into the groups")
+    if b is not None and b.shape != (Cout,):
+        raise ValueError("bias must have Cout entries")
+    Ho = (H + 2 * ph - (dh * (KH - 1) + 1)) // sh + 1
+    Wo = (W + 2 * pw - (dw * (KW - 1) + 1)) // sw + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    Y = np.empty((N, Ho, Wo, Cout), dtype=np.float64)
+    A = np.empty_like(Y)
+    rc = _load().oracle_conv2d_grouped(_ptr(X), _ptr(F), _ptr(b), _ptr(Y), _ptr(A), N, H, W, Cin, Cout, KH, KW,
+                                       sh, sw, ph, pw, dh, dw, groups)
+    if rc != 0:
+        raise ValueError("bad shape")
+    return Y, A
 
 
 def _dw_shape(x, w, mult, stride, pad, dil):

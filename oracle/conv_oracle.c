@@ -186,6 +186,66 @@ int oracle_conv2d_nhwc_ex_points(const float *X, const float *F, const float *bi
 }
 
 /* ---------------------------------------------------------------------------------- */
+/* Grouped, per-axis geometry, non-square kernels (Conv1D is H = KH = 1)                */
+/* ---------------------------------------------------------------------------------- */
+/*
+ * The same sum with the channels split into `groups` independent groups: output channel o
+ * belongs to group g = o / (Cout/groups) and reads only input channels g*Cg .. g*Cg + Cg - 1
+ * (Cg = Cin/groups) through filter F[i][j][c][o], c < Cg ("Convolution Is Wx+b Moving Across a
+ * Signal", section "Find the same sum in CKE's C kernels": grouped Conv1D with a bias). Window
+ * and output size per axis as in oracle_conv2d_nhwc_ex, with separate stride, padding and
+ * dilation for rows (h) and columns (w); a kernel of KH x KW taps. Float64; abssum as before.
+ */
+static void grouped_one(const float *X, const float *F, const float *bias, int H, int W, int Cin, int Cout,
+                        int KH, int KW, int sh, int sw, int ph, int pw, int dh, int dw, int groups,
+                        long n, long y, long x, long o, double *out, double *abs_out)
+{
+    const int Cg = Cin / groups, Og = Cout / groups;
+    const long g = o / Og;
+    double s = 0.0, a = 0.0;
+    for (int i = 0; i < KH; ++i)
+        for (int j = 0; j < KW; ++j) {
+            long r = y * sh + (long)i * dh - ph;
+            long q = x * sw + (long)j * dw - pw;
+            if (r < 0 || r >= H || q < 0 || q >= W) continue;   /* zero padding */
+            for (int c = 0; c < Cg; ++c) {
+                double xv = X[((n * H + r) * W + q) * Cin + g * Cg + c];
+                double fv = F[(((long)i * KW + j) * Cg + c) * Cout + o];
+                s += xv * fv;
+                a += fabs(xv) * fabs(fv);
+            }
+        }
+    if (bias) {
+        s += (double)bias[o];
+        a += fabs((double)bias[o]);
+    }
+    *out = s;
+    *abs_out = a;
+}
+
+/* Full output Y[N][Ho][Wo][Cout]. Returns 0, or -1 for an empty output or bad groups. */
+int oracle_conv2d_grouped(const float *X, const float *F, const float *bias, double *Y, double *abssum,
+                          int N, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int ph, int pw,
+                          int dh, int dw, int groups)
+{
+    if (groups < 1 || Cin % groups || Cout % groups) return -1;
+    const long Ho = dense_out_size(H, KH, sh, ph, dh), Wo = dense_out_size(W, KW, sw, pw, dw);
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (long n = 0; n < N; ++n)
+        for (long y = 0; y < Ho; ++y)
+            for (long x = 0; x < Wo; ++x)
+                for (long o = 0; o < Cout; ++o) {
+                    long t = ((n * Ho + y) * Wo + x) * Cout + o;
+                    double a;
+                    grouped_one(X, F, bias, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups, n, y, x, o,
+                                &Y[t], &a);
+                    if (abssum) abssum[t] = a;
+                }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------- */
 /* Depthwise                                                                           */
 /* ---------------------------------------------------------------------------------- */
 

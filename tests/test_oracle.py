@@ -349,6 +349,81 @@ def test_dense_ex_points_match_full():
     assert np.array_equal(y, Y.reshape(-1)[idx]) and np.array_equal(a, A.reshape(-1)[idx])
 
 
+# ------------------------------------------------------------------------------------------
+# Grouped convolution, per-axis geometry, KH x KW kernels, Conv1D (the Wx+b page's CKE
+# section: grouped Conv1D with a bias)
+# ------------------------------------------------------------------------------------------
+
+
+def test_grouped_one_group_square_is_the_ex_definition():
+    X = _ints(81, (2, 9, 8, 6))
+    F = _ints(82, (3, 3, 6, 4))
+    b = np.array([1, -1, 2, 0.5], np.float32)
+    Y, A = oracle.conv2d_grouped(X, F, bias=b, stride=2, pad=1, dil=2)
+    Y0, A0 = oracle.conv2d_nhwc_ex(X, F, bias=b, stride=2, pad=1, dil=2)
+    assert np.array_equal(Y, Y0) and np.array_equal(A, A0)
+
+
+@pytest.mark.parametrize("groups", [2, 3, 6])
+def test_grouped_is_independent_convolutions_of_the_channel_slices(groups):
+    Cin, Cout = 12, 6 * groups
+    Cg, Og = Cin // groups, Cout // groups
+    X = _ints(83, (2, 8, 7, Cin))
+    F = _ints(84, (3, 3, Cg, Cout))
+    b = _ints(85, (Cout,)).astype(np.float32)
+    Y, _ = oracle.conv2d_grouped(X, F, bias=b, stride=(2, 1), pad=(1, 2), groups=groups)
+    for g in range(groups):
+        ref, _ = oracle.conv2d_grouped(X[..., g * Cg:(g + 1) * Cg], F[..., g * Og:(g + 1) * Og], bias=b[g * Og:(g + 1) * Og],
+                                       stride=(2, 1), pad=(1, 2))
+        assert np.array_equal(Y[..., g * Og:(g + 1) * Og], ref)
+
+
+@pytest.mark.parametrize("case", [((2, 1), (1, 0), (1, 1), (3, 2)), ((1, 3), (0, 2), (2, 1), (2, 5)),
+                                  ((2, 2), (1, 1), (1, 2), (1, 3))])
+def test_grouped_per_axis_and_non_square_match_torch(case):
+    (sh, sw), (ph, pw), (dh, dw), (KH, KW) = case
+    groups = 2
+    X = workloads.normal(86, 2 * 13 * 11 * 8, 1.0).reshape(2, 13, 11, 8)
+    F = workloads.normal(87, KH * KW * 4 * 6, 0.3).reshape(KH, KW, 4, 6)
+    b = workloads.normal(88, 6, 0.5)
+    Y, A = oracle.conv2d_grouped(X, F, bias=b, stride=(sh, sw), pad=(ph, pw), dil=(dh, dw), groups=groups)
+    x = torch.from_numpy(np.asarray(X, dtype=np.float64)).permute(0, 3, 1, 2)
+    f = torch.from_numpy(np.asarray(F, dtype=np.float64)).permute(3, 2, 0, 1)
+    ref = torch.nn.functional.conv2d(x, f, torch.from_numpy(np.asarray(b, dtype=np.float64)), stride=(sh, sw),
+                                     padding=(ph, pw), dilation=(dh, dw), groups=groups).permute(0, 2, 3, 1).numpy()
+    assert Y.shape == ref.shape
+    assert np.all(np.abs(Y - ref) <= 1e-13 * A)
+
+
+def test_conv1d_is_the_one_dimensional_correlation():
+    # H = KH = 1: every output is numpy's valid 1-D correlation of one input channel with one
+    # filter row, summed over the group's channels
+    L, Cin, Cout, K = 20, 4, 6, 5
+    X = _ints(89, (3, 1, L, Cin))
+    F = _ints(90, (1, K, Cin, Cout))
+    Y, _ = oracle.conv2d_grouped(X, F)
+    for n in range(3):
+        for o in range(Cout):
+            ref = sum(np.correlate(X[n, 0, :, c].astype(np.float64), F[0, :, c, o].astype(np.float64), "valid")
+                      for c in range(Cin))
+            assert np.array_equal(Y[n, 0, :, o], ref)
+
+
+def test_conv1d_page_example_two_filters_with_bias():
+    # "The matrix connection": x = 1..5, filters (2, 0, -1) and (1, 1, 1), biases (1, 0)
+    e = _golden("wxb_1d_examples.json")["two_filters_with_bias"]
+    X = np.array(e["x"], np.float32).reshape(1, 1, 5, 1)
+    F = np.array(e["filters"], np.float32).T.reshape(1, 3, 1, 2)
+    Y, _ = oracle.conv2d_grouped(X, F, bias=np.array(e["bias"], np.float32))
+    for o in range(2):
+        assert np.array_equal(Y[0, 0, :, o], np.array(e["output_per_filter"][o], dtype=np.float64))
+
+
+def test_grouped_rejects_bad_groups():
+    with pytest.raises(ValueError):
+        oracle.conv2d_grouped(np.zeros((1, 5, 5, 6), np.float32), np.zeros((3, 3, 2, 4), np.float32), groups=4)
+
+
 def test_dense_rejects_incompatible_shapes():
     with pytest.raises(ValueError):
         oracle.conv2d_nhwc(np.zeros((1, 3, 3, 2), np.float32), np.zeros((4, 4, 2, 1), np.float32))
