@@ -71,6 +71,8 @@ def _load():
         lib.oracle_conv2d_nhwc_ex_points.restype = I
         lib.oracle_conv2d_grouped.argtypes = [P, P, P, P, P] + [I] * 14
         lib.oracle_conv2d_grouped.restype = I
+        lib.oracle_conv2d_grouped_points.argtypes = [P, P, P, P, L, P, P] + [I] * 13
+        lib.oracle_conv2d_grouped_points.restype = I
         lib.oracle_depthwise.argtypes = [P, P, P, P] + [I] * 11
         lib.oracle_depthwise.restype = I
         lib.oracle_depthwise_points.argtypes = [P, P, P, P, L, P] + [I] * 11
@@ -201,6 +203,27 @@ def conv2d_grouped(X, F, bias=None, stride=1, pad=0, dil=1, groups=1):
     if rc != 0:
         raise ValueError("bad shape")
     return Y, A
+
+
+def conv2d_grouped_points(X, F, flat_idx, bias=None, stride=1, pad=0, dil=1, groups=1):
+    """Selected outputs of conv2d_grouped, by flat index into [N, Ho, Wo, Cout]."""
+    X, F = _f32(X), _f32(F)
+    b = None if bias is None else _f32(bias)
+    N, H, W, Cin = X.shape
+    KH, KW, Cg, Cout = F.shape
+    (sh, sw), (ph, pw), (dh, dw) = _pair(stride), _pair(pad), _pair(dil)
+    if groups < 1 or Cin % groups or Cout % groups or Cg * groups != Cin:
+        raise ValueError("channels must split into the groups")
+    Ho = (H + 2 * ph - (dh * (KH - 1) + 1)) // sh + 1
+    Wo = (W + 2 * pw - (dw * (KW - 1) + 1)) // sw + 1
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    if Ho < 1 or Wo < 1 or (idx.size and (idx.min() < 0 or idx.max() >= N * Ho * Wo * Cout)):
+        raise ValueError("bad shape or index")
+    y = np.empty(idx.size, dtype=np.float64)
+    a = np.empty(idx.size, dtype=np.float64)
+    _load().oracle_conv2d_grouped_points(_ptr(X), _ptr(F), _ptr(b), _ptr(idx), idx.size, _ptr(y), _ptr(a), H, W,
+                                         Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups)
+    return y, a
 
 
 def _dw_shape(x, w, mult, stride, pad, dil):

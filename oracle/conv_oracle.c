@@ -245,6 +245,26 @@ int oracle_conv2d_grouped(const float *X, const float *F, const float *bias, dou
     return 0;
 }
 
+/* Selected outputs of oracle_conv2d_grouped, by flat index into [N][Ho][Wo][Cout]. */
+int oracle_conv2d_grouped_points(const float *X, const float *F, const float *bias, const int64_t *idx,
+                                 int64_t npts, double *y, double *abssum, int H, int W, int Cin, int Cout, int KH,
+                                 int KW, int sh, int sw, int ph, int pw, int dh, int dw, int groups)
+{
+    if (groups < 1 || Cin % groups || Cout % groups) return -1;
+    const long Ho = dense_out_size(H, KH, sh, ph, dh), Wo = dense_out_size(W, KW, sw, pw, dw);
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t p = 0; p < npts; ++p) {
+        long t = idx[p];
+        long o = t % Cout; t /= Cout;
+        long x = t % Wo; t /= Wo;
+        long yy = t % Ho; t /= Ho;
+        grouped_one(X, F, bias, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups, t, yy, x, o, &y[p],
+                    &abssum[p]);
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------------------------- */
 /* Depthwise                                                                           */
 /* ---------------------------------------------------------------------------------- */

@@ -419,6 +419,17 @@ def test_conv1d_page_example_two_filters_with_bias():
         assert np.array_equal(Y[0, 0, :, o], np.array(e["output_per_filter"][o], dtype=np.float64))
 
 
+def test_grouped_points_are_the_full_output():
+    X = workloads.normal(91, 2 * 9 * 10 * 12, 1.0).reshape(2, 9, 10, 12)
+    F = workloads.normal(92, 3 * 2 * 4 * 6, 0.3).reshape(3, 2, 4, 6)
+    b = workloads.normal(93, 6, 0.5)
+    kw = dict(stride=(2, 1), pad=(1, 0), dil=(1, 2), groups=3)
+    Y, A = oracle.conv2d_grouped(X, F, b, **kw)
+    idx = (workloads.splitmix64(94, 300) % np.uint64(Y.size)).astype(np.int64)
+    y, a = oracle.conv2d_grouped_points(X, F, idx, b, **kw)
+    assert np.array_equal(y, Y.reshape(-1)[idx]) and np.array_equal(a, A.reshape(-1)[idx])
+
+
 def test_grouped_rejects_bad_groups():
     with pytest.raises(ValueError):
         oracle.conv2d_grouped(np.zeros((1, 5, 5, 6), np.float32), np.zeros((3, 3, 2, 4), np.float32), groups=4)
