@@ -18,6 +18,9 @@ The arithmetic lives in ``conv_oracle.c`` (plain C, OpenMP over independent outp
   section, float64.
 * ``depthwise`` -- the per-output loop of the OneModel "Depthwise convolution" page
   (section "What each output is"), in IEEE float32 in the page's order, exact or fast mode.
+* ``dwpw`` -- a depthwise pass followed by a pointwise 1 x 1 pass (Wx+b page, section "Why
+  variants matter"): the depthwise output above, rounded to bfloat16 (nearest even), then the
+  channel-mixing sum with a bias in float64.
 
 Parity status: every function here is pinned by tests that do not call it to compute
 their expectation (worked examples printed on the pages, library routines for special
@@ -73,6 +76,10 @@ def _load():
         lib.oracle_conv2d_grouped.restype = I
         lib.oracle_conv2d_grouped_points.argtypes = [P, P, P, P, L, P, P] + [I] * 13
         lib.oracle_conv2d_grouped_points.restype = I
+        lib.oracle_dwpw.argtypes = [P] * 7 + [I] * 10
+        lib.oracle_dwpw.restype = I
+        lib.oracle_dwpw_points.argtypes = [P] * 6 + [L, P, P] + [I] * 9
+        lib.oracle_dwpw_points.restype = I
         lib.oracle_depthwise.argtypes = [P, P, P, P] + [I] * 11
         lib.oracle_depthwise.restype = I
         lib.oracle_depthwise_points.argtypes = [P, P, P, P, L, P] + [I] * 11
@@ -276,3 +283,55 @@ def depthwise_absbound(x, w, bias, mult=1, stride=1, pad=0, dil=1):
     _load().oracle_depthwise_absbound(_ptr(x), _ptr(w), _ptr(b), _ptr(out), N, Cin, mult, H, W, KH,
                                       KW, stride, pad, dil)
     return out
+
+
+def _dwpw_shape(x, w, F, b_dw, b_pw, stride, pad, dil):
+    N, C, H, W = x.shape
+    if w.ndim != 3 or w.shape[0] != C or w.shape[1] != w.shape[2]:
+        raise ValueError("w must be [C, K, K]")
+    K = w.shape[1]
+    if F.ndim != 2 or F.shape[0] != C:
+        raise ValueError("F must be [C, Cout]")
+    Cout = F.shape[1]
+    if b_dw is not None and b_dw.shape != (C,):
+        raise ValueError("depthwise bias must have C entries")
+    if b_pw is not None and b_pw.shape != (Cout,):
+        raise ValueError("pointwise bias must have Cout entries")
+    Ho = (H + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    Wo = (W + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    return N, C, H, W, K, Cout, Ho, Wo
+
+
+def dwpw(x, w, b_dw, F, b_pw, stride=1, pad=0, dil=1, mode=DW_EXACT):
+    """Depthwise (x [N,C,H,W] float32, w [C,K,K], b_dw [C] or None; the page's order and
+    mode) then pointwise (F [C,Cout], the float32 values of bf16 weights; b_pw [Cout] or
+    None) over the bfloat16-rounded intermediate. Returns (y, abssum), float64
+    [N, Cout, Ho, Wo]."""
+    x, w, F = _f32(x), _f32(w), _f32(F)
+    bd = None if b_dw is None else _f32(b_dw)
+    bp = None if b_pw is None else _f32(b_pw)
+    N, C, H, W, K, Cout, Ho, Wo = _dwpw_shape(x, w, F, bd, bp, stride, pad, dil)
+    y = np.empty((N, Cout, Ho, Wo), dtype=np.float64)
+    a = np.empty_like(y)
+    if _load().oracle_dwpw(_ptr(x), _ptr(w), _ptr(bd), _ptr(F), _ptr(bp), _ptr(y), _ptr(a), N, C, H, W, K, stride,
+                           pad, dil, mode, Cout) != 0:
+        raise ValueError("bad shape")
+    return y, a
+
+
+def dwpw_points(x, w, b_dw, F, b_pw, flat_idx, stride=1, pad=0, dil=1, mode=DW_EXACT):
+    """Selected outputs of dwpw, by flat index into [N, Cout, Ho, Wo]."""
+    x, w, F = _f32(x), _f32(w), _f32(F)
+    bd = None if b_dw is None else _f32(b_dw)
+    bp = None if b_pw is None else _f32(b_pw)
+    N, C, H, W, K, Cout, Ho, Wo = _dwpw_shape(x, w, F, bd, bp, stride, pad, dil)
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    if idx.size and (idx.min() < 0 or idx.max() >= N * Cout * Ho * Wo):
+        raise ValueError("index out of range")
+    y = np.empty(idx.size, dtype=np.float64)
+    a = np.empty(idx.size, dtype=np.float64)
+    _load().oracle_dwpw_points(_ptr(x), _ptr(w), _ptr(bd), _ptr(F), _ptr(bp), _ptr(idx), idx.size, _ptr(y), _ptr(a),
+                               C, H, W, K, stride, pad, dil, mode, Cout)
+    return y, a

@@ -27,6 +27,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define DW_EXACT 0
@@ -394,3 +395,107 @@ int oracle_num_threads(void) { return omp_get_max_threads(); }
 #else
 int oracle_num_threads(void) { return 1; }
 #endif
+
+/* ---------------------------------------------------------------------------------- */
+/* Depthwise followed by pointwise (one block)                                         */
+/* ---------------------------------------------------------------------------------- */
+/*
+ * "Convolution Is Wx+b Moving Across a Signal", section "Why variants matter": a depthwise
+ * K x K pass followed by a pointwise 1 x 1 channel-mixing pass. Stage 1 is the depthwise
+ * output above (OneModel page, multiplier 1, float32 in the page's order, exact or fast mode,
+ * with its own bias). Stage 2 feeds it to the tensor cores, so the intermediate is rounded
+ * to bfloat16 (nearest, ties to even; a NaN stays a NaN), and the pointwise sum over the
+ * channels, y[n][o][oy][ox] = bias_pw[o] + sum_c bf16(d[n][c][oy][ox]) * F[c][o], is taken in
+ * float64 with the same absolute sum as the dense oracle.
+ */
+static float round_bf16(float v)
+{
+    uint32_t u;
+    memcpy(&u, &v, sizeof u);
+    if (isnan(v)) {
+        u = (u | 0x00400000u) & 0xFFFF0000u;   /* quiet, upper half kept */
+    } else {
+        /* nearest, ties to even, on the 16 bits that are dropped */
+        uint32_t low = u & 0xFFFFu, keep = u & 0xFFFF0000u;
+        if (low > 0x8000u || (low == 0x8000u && (keep & 0x10000u))) keep += 0x10000u;
+        u = keep;
+    }
+    float r;
+    memcpy(&r, &u, sizeof r);
+    return r;
+}
+
+/* All Cout outputs of one output pixel; a[] is scratch of C floats. */
+static void dwpw_pixel(const float *x, const float *w, const float *bias_dw, const float *F, const float *bias_pw,
+                       int C, int H, int W, int K, int stride, int pad, int dil, int mode, int Cout, long n,
+                       long oy, long ox, float *a, double *out, double *abs_out, long out_stride)
+{
+    for (long c = 0; c < C; ++c)
+        a[c] = round_bf16(dw_one(x, w, bias_dw, C, 1, H, W, K, K, stride, pad, dil, mode, n, c, oy, ox));
+    for (long o = 0; o < Cout; ++o) {
+        double s = 0.0, t = 0.0;
+        for (long c = 0; c < C; ++c) {
+            double av = a[c], fv = F[c * Cout + o];
+            s += av * fv;
+            t += fabs(av) * fabs(fv);
+        }
+        if (bias_pw) {
+            s += (double)bias_pw[o];
+            t += fabs((double)bias_pw[o]);
+        }
+        out[o * out_stride] = s;
+        if (abs_out) abs_out[o * out_stride] = t;
+    }
+}
+
+/* Full output y[N][Cout][Ho][Wo] (float64) and its absolute sums. */
+int oracle_dwpw(const float *x, const float *w, const float *bias_dw, const float *F, const float *bias_pw, double *y,
+                double *abssum, int N, int C, int H, int W, int K, int stride, int pad, int dil, int mode, int Cout)
+{
+    const long Ho = dw_out_size(H, K, stride, pad, dil), Wo = dw_out_size(W, K, stride, pad, dil);
+    if (Ho < 1 || Wo < 1) return -1;
+    const long plane = Ho * Wo;
+#pragma omp parallel
+    {
+        float *a = (float *)malloc(sizeof(float) * (size_t)C);
+#pragma omp for collapse(2) schedule(dynamic)
+        for (long n = 0; n < N; ++n)
+            for (long oy = 0; oy < Ho; ++oy)
+                for (long ox = 0; ox < Wo; ++ox) {
+                    long t = n * Cout * plane + oy * Wo + ox;
+                    dwpw_pixel(x, w, bias_dw, F, bias_pw, C, H, W, K, stride, pad, dil, mode, Cout, n, oy, ox, a,
+                               &y[t], abssum ? &abssum[t] : NULL, plane);
+                }
+        free(a);
+    }
+    return 0;
+}
+
+/* Selected outputs, by flat index into [N][Cout][Ho][Wo]. */
+int oracle_dwpw_points(const float *x, const float *w, const float *bias_dw, const float *F, const float *bias_pw,
+                       const int64_t *idx, int64_t npts, double *y, double *abssum, int C, int H, int W, int K,
+                       int stride, int pad, int dil, int mode, int Cout)
+{
+    const long Ho = dw_out_size(H, K, stride, pad, dil), Wo = dw_out_size(W, K, stride, pad, dil);
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel
+    {
+        float *a = (float *)malloc(sizeof(float) * (size_t)C);
+        double *col = (double *)malloc(sizeof(double) * (size_t)Cout * 2);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t p = 0; p < npts; ++p) {
+            long t = idx[p];
+            long ox = t % Wo; t /= Wo;
+            long oy = t % Ho; t /= Ho;
+            long o = t % Cout;
+            long n = t / Cout;
+            dwpw_pixel(x, w, bias_dw, F, bias_pw, C, H, W, K, stride, pad, dil, mode, Cout, n, oy, ox, a, col,
+                       col + Cout, 1);
+            y[p] = col[o];
+            abssum[p] = col[Cout + o];
+        }
+        free(a);
+        free(col);
+    }
+    return 0;
+}

@@ -687,3 +687,79 @@ def test_storage_bill_table():
     assert math.isclose(rows * cols * 4 / 1e6, g["megabytes_f32"]["patches"])
     e = g["small_example"]
     assert ((e["H"] - e["K"] + 1) * (e["W"] - e["K"] + 1) * e["K"] ** 2) / (e["H"] * e["W"]) == e["ratio"]
+
+
+# ------------------------------------------------------------------------------------------
+# Depthwise followed by pointwise (the Wx+b page's section "Why variants matter")
+# ------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("geom", [(3, 1, 1, 1), (3, 2, 1, 1), (5, 1, 2, 1), (3, 1, 2, 2), (1, 1, 0, 1)])
+def test_dwpw_is_depthwise_then_channel_mixing_on_integers(geom):
+    # small integers keep every stage exact (|d| <= 25*3*2 fits bf16's 8-bit significand), so
+    # the block must equal torch's grouped depthwise conv followed by a 1x1 mixing, in float64
+    K, s, p, d = geom
+    N, C, H, W, Cout = 2, 6, 9, 8, 5
+    x = workloads.int_uniform(101, N * C * H * W, -3, 3).reshape(N, C, H, W)
+    w = workloads.int_uniform(102, C * K * K, -2, 2).reshape(C, K, K)
+    F = workloads.int_uniform(103, C * Cout, -3, 3).reshape(C, Cout)
+    bd = workloads.int_uniform(104, C, -4, 4)
+    bp = workloads.int_uniform(105, Cout, -4, 4)
+    for mode in (oracle.DW_EXACT, oracle.DW_FAST):
+        y, a = oracle.dwpw(x, w, bd, F, bp, s, p, d, mode)
+        t = torch.nn.functional.conv2d(torch.from_numpy(x.astype(np.float64)), torch.from_numpy(w.astype(np.float64))[:, None],
+                                       torch.from_numpy(bd.astype(np.float64)), stride=s, padding=p, dilation=d, groups=C)
+        ref = torch.einsum("nchw,co->nohw", t, torch.from_numpy(F.astype(np.float64))) + \
+            torch.from_numpy(bp.astype(np.float64))[None, :, None, None]
+        assert np.array_equal(y, ref.numpy())
+        refa = torch.einsum("nchw,co->nohw", t.abs(), torch.from_numpy(np.abs(F).astype(np.float64))) + \
+            torch.from_numpy(np.abs(bp).astype(np.float64))[None, :, None, None]
+        assert np.array_equal(a, refa.numpy())
+
+
+def test_dwpw_rounds_the_intermediate_to_bf16_nearest_even():
+    # K = 1, w = 1, F = 1: y is the bf16 rounding of x itself
+    vals = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -7 + 2 ** -9, -(1 + 2 ** -8), 65535.0, 2 ** -130],
+                    np.float32)
+    expect = [1.0, 1.015625, 1.0078125, -1.0, 65536.0, 2 ** -130]   # ties go to the even significand
+    x = vals.reshape(1, 1, 1, -1)
+    y, _ = oracle.dwpw(x, np.ones((1, 1, 1), np.float32), None, np.ones((1, 1), np.float32), None)
+    assert y.reshape(-1).tolist() == expect
+
+
+def test_dwpw_nan_intermediate_stays_nan():
+    x = np.array([np.nan, 1.0], np.float32).reshape(1, 1, 1, 2)
+    y, _ = oracle.dwpw(x, np.ones((1, 1, 1), np.float32), None, np.full((1, 2), 2.0, np.float32), None)
+    assert np.isnan(y[0, :, 0, 0]).all() and (y[0, :, 0, 1] == 2.0).all()
+
+
+@pytest.mark.parametrize("mode", [oracle.DW_EXACT, oracle.DW_FAST])
+def test_dwpw_identity_mixing_gives_the_rounded_depthwise_output(mode):
+    # F = I: the block returns the depthwise output of the page (its own, pinned oracle)
+    # rounded to bf16, here by the input module's independent rounding routine
+    N, C, H, W, K = 2, 4, 10, 9, 3
+    x = workloads.uniform(106, N * C * H * W, -1, 1).reshape(N, C, H, W)
+    w = workloads.normal(107, C * K * K, 1 / 3).reshape(C, K, K)
+    b = workloads.normal(108, C, 0.3)
+    y, _ = oracle.dwpw(x, w, b, np.eye(C, dtype=np.float32), None, 2, 1, 1, mode)
+    dref = oracle.depthwise(x, w, b, mult=1, stride=2, pad=1, dil=1, mode=mode)
+    assert np.array_equal(y, workloads.bf16_to_f32(workloads.bf16_bits(dref)).astype(np.float64))
+
+
+def test_dwpw_points_are_the_full_output():
+    N, C, H, W, K, Cout = 2, 5, 7, 6, 3, 7
+    x = workloads.uniform(109, N * C * H * W, -1, 1).reshape(N, C, H, W)
+    w = workloads.normal(110, C * K * K, 1 / 3).reshape(C, K, K)
+    F = workloads.normal(111, C * Cout, 0.4).reshape(C, Cout)
+    bp = workloads.normal(112, Cout, 0.3)
+    y, a = oracle.dwpw(x, w, None, F, bp, 1, 1, 1)
+    idx = (workloads.splitmix64(113, 200) % np.uint64(y.size)).astype(np.int64)
+    yp, ap = oracle.dwpw_points(x, w, None, F, bp, idx, 1, 1, 1)
+    assert np.array_equal(yp, y.reshape(-1)[idx]) and np.array_equal(ap, a.reshape(-1)[idx])
+
+
+def test_dwpw_weight_counts_of_the_page():
+    # "Why variants matter": 64 -> 64 channels, 3x3: dense 36,864 weights, depthwise plus
+    # pointwise 4,672, about 7.9x fewer
+    dense, factored = 64 * 64 * 3 * 3, 64 * 3 * 3 + 64 * 64
+    assert (dense, factored) == (36864, 4672) and round(dense / factored, 1) == 7.9
