@@ -53,6 +53,9 @@ def workload_table():
          "pointwise": ("dense", workloads.DENSE_1X1, None),
          "dense-large": ("dense", workloads.DENSE_LARGE, None),
          "dense-s2": ("dense", workloads.DENSE_S2, None),
+         "grouped": ("dense", workloads.DENSE_GROUPED, None),
+         "conv1d-stem1": ("dense", workloads.CONV1D_STEM1, None),
+         "conv1d-stem2": ("dense", workloads.CONV1D_STEM2, None),
          # comparison path: explicit patch matrix + one cuBLAS GEMM, packing inside the timing
          "dense3x3-explicit-im2col": ("dense", workloads.DENSE_3X3, "im2col")}
     for c in workloads.DW_SWEEP:
@@ -281,14 +284,14 @@ def dense_device_inputs(torch, case, seed):
     (for the secondary measurements)."""
     g = torch.Generator(device="cuda").manual_seed(seed)
     X = torch.randn((case.N, case.H, case.W, case.Cin), device="cuda", generator=g).to(torch.bfloat16)
-    F = (torch.randn((case.K, case.K, case.Cin, case.Cout), device="cuda", generator=g)
-         / math.sqrt(case.K * case.K * case.Cin)).to(torch.bfloat16)
+    F = (torch.randn(case.f_shape, device="cuda", generator=g)
+         / math.sqrt(case.kh * case.kw * case.cin_g)).to(torch.bfloat16)
     b = torch.randn((case.Cout,), device="cuda", generator=g) * math.sqrt(0.1) if case.bias else None
     return X, F, b
 
 
 def dense_plain(case):
-    return case.stride == 1 and case.pad == 0 and case.dil == 1 and not case.bias
+    return case.square and case.stride == 1 and case.pad == 0 and case.dil == 1 and not case.bias
 
 
 def dense_call(cb, case, X, F, b, Y, mode=None, ws=None):
@@ -298,7 +301,20 @@ def dense_call(cb, case, X, F, b, Y, mode=None, ws=None):
         return cb.conv2d_nhwc_fwd_im2col(X, F, Y, workspace=ws)
     if dense_plain(case):
         return cb.conv2d_nhwc_fwd(X, F, Y)
-    return cb.conv2d_nhwc_fwd_ex(X, F, b, Y, case.stride, case.pad, case.dil)
+    if case.square:
+        return cb.conv2d_nhwc_fwd_ex(X, F, b, Y, case.stride, case.pad, case.dil)
+    return cb.conv2d_nhwc_fwd_grouped(X, F, b, Y, (case.stride, case.sw), (case.pad, case.pw), (case.dil, case.dw),
+                                      case.groups)
+
+
+def oracle_dense(oracle, case, X, F, b):
+    """The oracle entry for a dense case (whole images of X)."""
+    if dense_plain(case):
+        return oracle.conv2d_nhwc(X, F)
+    if case.square:
+        return oracle.conv2d_nhwc_ex(X, F, b, case.stride, case.pad, case.dil)
+    return oracle.conv2d_grouped(X, F, b, (case.stride, case.sw), (case.pad, case.pw), (case.dil, case.dw),
+                                 case.groups)
 
 
 def im2col_workspace(cb, torch, case, mode):
@@ -395,10 +411,7 @@ def cpu_baseline(kind, case, mode, host_np, budget_s=10.0):
         i = n % case.N
         if kind == "dense":
             X, F, b = host_np
-            if dense_plain(case):
-                oracle.conv2d_nhwc(X[i:i + 1], F)
-            else:
-                oracle.conv2d_nhwc_ex(X[i:i + 1], F, b, case.stride, case.pad, case.dil)
+            oracle_dense(oracle, case, X[i:i + 1], F, b)
             done += case.flops / case.N
         else:
             x, w, b = host_np
@@ -462,6 +475,9 @@ def run_ours(args, dist):
         cfg = {"workload": case.name, "N_per_gpu": case.N, "H": case.H, "W": case.W, "Cin": case.Cin,
                "Cout": case.Cout, "K": case.K, "stride": case.stride, "pad": case.pad, "dil": case.dil,
                "bias": case.bias, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
+        if not case.square:
+            cfg.update({"KH": case.kh, "KW": case.kw, "stride_w": case.sw, "pad_w": case.pw, "dil_w": case.dw,
+                        "groups": case.groups})
         if mode == "im2col":
             cfg["path"] = "explicit patch matrix in a workspace + one cuBLAS GEMM (comparison path)"
     else:
@@ -536,13 +552,16 @@ def run_reference(args, dist):
         X, F = workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb)
         b = workloads.dense_bias(case)
         total = case.N * case.Ho * case.Wo * case.Cout
-        work_per_out, unit, scale = 2 * case.K * case.K * case.Cin, "TFLOP/s", 1e12
+        work_per_out, unit, scale = 2 * case.kh * case.kw * case.cin_g, "TFLOP/s", 1e12
 
         def run(idx):
             if dense_plain(case):
                 oracle.conv2d_nhwc_points(X, F, idx)
-            else:
+            elif case.square:
                 oracle.conv2d_nhwc_ex_points(X, F, idx, b, case.stride, case.pad, case.dil)
+            else:
+                oracle.conv2d_grouped_points(X, F, idx, b, (case.stride, case.sw), (case.pad, case.pw),
+                                             (case.dil, case.dw), case.groups)
     else:
         x, w, b = workloads.depthwise_inputs(case)
         total = case.N * case.C * case.mult * case.Ho * case.Wo

@@ -37,6 +37,8 @@ lib.conv2d_nhwc_fwd_f32.argtypes = [_P, _P, _P] + [_I] * 6 + [_P]
 lib.conv2d_nhwc_fwd_f32.restype = _I
 lib.conv2d_nhwc_fwd_ex.argtypes = [_P, _P, _P, _P] + [_I] * 9 + [_P]
 lib.conv2d_nhwc_fwd_ex.restype = _I
+lib.conv2d_nhwc_fwd_grouped.argtypes = [_P, _P, _P, _P] + [_I] * 14 + [_P]
+lib.conv2d_nhwc_fwd_grouped.restype = _I
 lib.conv2d_nhwc_im2col_workspace.argtypes = [_I] * 5
 lib.conv2d_nhwc_im2col_workspace.restype = ctypes.c_size_t
 lib.conv2d_nhwc_fwd_im2col.argtypes = [_P, _P, _P, _P, ctypes.c_size_t] + [_I] * 6 + [_P]
@@ -52,8 +54,8 @@ lib.conv_last_kernel.restype = ctypes.c_char_p
 lib.conv_selftest_wait_timeout.argtypes = [_P]
 lib.conv_selftest_wait_timeout.restype = _I
 
-EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "conv2d_nhwc_im2col_workspace",
-           "conv2d_nhwc_fwd_im2col", "depthwise_fwd", "conv_status_string",
+EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "conv2d_nhwc_fwd_grouped",
+           "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "depthwise_fwd", "conv_status_string",
            "conv_device_status", "conv_last_kernel", "conv_selftest_wait_timeout")
 
 
@@ -152,6 +154,46 @@ def conv2d_nhwc_fwd_ex(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, stream=N
     py = _tensor(Y, torch.bfloat16, 4, "Y")
     _check(lib.conv2d_nhwc_fwd_ex(px, pf, pb, py, N, H, W, Cin, Cout, K, stride, pad, dil, _stream(stream)),
            "conv2d_nhwc_fwd_ex")
+    return Y
+
+
+def _pair(v, name):
+    if isinstance(v, (tuple, list)):
+        if len(v) != 2:
+            raise ValueError(f"{name} must be an int or a pair")
+        return int(v[0]), int(v[1])
+    return int(v), int(v)
+
+
+def conv2d_nhwc_fwd_grouped(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, groups=1, stream=None):
+    """Grouped dense NHWC convolution, bfloat16, with a KH x KW filter and per-axis stride,
+    zero padding and dilation (ints or (h, w) pairs) and an optional float32 bias [Cout]:
+    X [N,H,W,Cin], F [KH,KW,Cin/groups,Cout] -> Y [N,Ho,Wo,Cout]. A Conv1D is H = KH = 1."""
+    import torch
+    px = _tensor(X, torch.bfloat16, 4, "X")
+    pf = _tensor(F, torch.bfloat16, 4, "F")
+    N, H, W, Cin = X.shape
+    KH, KW, Cg, Cout = F.shape
+    groups = int(groups)
+    if groups < 1 or Cin % groups or Cout % groups or Cg != Cin // groups:
+        raise ValueError("F must be [KH, KW, Cin/groups, Cout] with groups dividing Cin and Cout")
+    (sh, sw), (ph, pw), (dh, dw) = _pair(stride, "stride"), _pair(pad, "pad"), _pair(dil, "dil")
+    pb = ctypes.c_void_p(None)
+    if bias is not None:
+        pb = _tensor(bias, torch.float32, 1, "bias")
+        if bias.shape[0] != Cout:
+            raise ValueError("bias must have Cout entries")
+    Ho = (H + 2 * ph - (dh * (KH - 1) + 1)) // sh + 1
+    Wo = (W + 2 * pw - (dw * (KW - 1) + 1)) // sw + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    if Y is None:
+        Y = torch.empty((N, Ho, Wo, Cout), dtype=torch.bfloat16, device=X.device)
+    elif tuple(Y.shape) != (N, Ho, Wo, Cout):
+        raise ValueError("Y has the wrong shape")
+    py = _tensor(Y, torch.bfloat16, 4, "Y")
+    _check(lib.conv2d_nhwc_fwd_grouped(px, pf, pb, py, N, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups,
+                                       _stream(stream)), "conv2d_nhwc_fwd_grouped")
     return Y
 
 

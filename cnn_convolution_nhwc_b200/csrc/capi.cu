@@ -152,22 +152,40 @@ int check_dense(const void *X, const void *F, const void *Y, int N, int H, int W
     return CONV_OK;
 }
 
-// Stride, zero padding, dilation and bias of a dense convolution (the plain operation is
-// {1, 0, 1, null}).
+// Geometry of a dense convolution: a KH x KW filter, stride, zero padding and dilation per
+// axis, channel groups and an optional bias. The plain operation is a square K with stride 1,
+// no padding, dilation 1, one group and no bias.
 struct DenseGeom {
-    int stride = 1, pad = 0, dil = 1;
+    int KH = 1, KW = 1;
+    int sh = 1, sw = 1, ph = 0, pw = 0, dh = 1, dw = 1;
+    int groups = 1;
     const float *bias = nullptr;
-    long long ho(int H, int K) const { return (1LL * H + 2LL * pad - (1LL * dil * (K - 1) + 1)) / stride + 1; }
-    bool plain() const { return stride == 1 && pad == 0 && dil == 1 && bias == nullptr; }
+    static DenseGeom square(int K, int stride = 1, int pad = 0, int dil = 1, const float *bias = nullptr) {
+        DenseGeom g;
+        g.KH = g.KW = K;
+        g.sh = g.sw = stride;
+        g.ph = g.pw = pad;
+        g.dh = g.dw = dil;
+        g.bias = bias;
+        return g;
+    }
+    // output extents; the caller has checked that the dilated filter fits the padded input
+    long long ho(int H) const { return (1LL * H + 2LL * ph - (1LL * dh * (KH - 1) + 1)) / sh + 1; }
+    long long wo(int W) const { return (1LL * W + 2LL * pw - (1LL * dw * (KW - 1) + 1)) / sw + 1; }
+    bool plain() const {
+        return KH == KW && sh == 1 && sw == 1 && ph == 0 && pw == 0 && dh == 1 && dw == 1 && groups == 1 &&
+               bias == nullptr;
+    }
 };
 
 template <typename T>
-int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int Cin, int Cout, int K,
-                        cudaStream_t stream, DeviceState *d, const DenseGeom &g = DenseGeom()) {
+int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int Cin, int Cout, const DenseGeom &g,
+                        cudaStream_t stream, DeviceState *d) {
     DenseDirectParams p;
-    p.H = H; p.W = W; p.Cin = Cin; p.Cout = Cout; p.K = K;
-    p.Ho = static_cast<int>(g.ho(H, K)); p.Wo = static_cast<int>(g.ho(W, K));
-    p.stride = g.stride; p.pad = g.pad; p.dil = g.dil; p.bias = g.bias;
+    p.H = H; p.W = W; p.Cin = Cin; p.Cout = Cout; p.KH = g.KH; p.KW = g.KW;
+    p.Ho = static_cast<int>(g.ho(H)); p.Wo = static_cast<int>(g.wo(W));
+    p.Cin_g = Cin / g.groups; p.Cout_g = Cout / g.groups;
+    p.sh = g.sh; p.sw = g.sw; p.ph = g.ph; p.pw = g.pw; p.dh = g.dh; p.dw = g.dw; p.bias = g.bias;
     p.total = 1LL * N * p.Ho * p.Wo * Cout;
     long long blocks = (p.total + 255) / 256;
     const long long cap = 1LL * d->num_sms * 16;
@@ -179,68 +197,91 @@ int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int C
     return launched(cudaLaunchKernelEx(&cfg, dense_direct_kernel<T>, X, F, Y, p), "dense_direct_kernel");
 }
 
-template <class Cfg>
-int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
-                    cudaStream_t stream, DeviceState *d, unsigned attr_bit, const DenseGeom &g = DenseGeom()) {
-    const int Ho = static_cast<int>(g.ho(H, K)), Wo = static_cast<int>(g.ho(W, K));
-    alignas(64) CUtensorMap tmX, tmF, tmY;
-    {   // X: 4-D {Cin, W, H, N} im2col. The bounding box of window origins runs from -pad to
-        // (size - 1) + pad - dil*(K-1) on each spatial axis, walked with the convolution stride
-        // as element stride, so its pixels are exactly the output positions; origins and taps
-        // outside the image read zeros.
-        const cuuint64_t dims[4] = {(cuuint64_t)Cin, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)N};
-        const cuuint64_t strides[3] = {(cuuint64_t)Cin * 2, (cuuint64_t)W * Cin * 2, (cuuint64_t)H * W * Cin * 2};
-        const int lower[2] = {-g.pad, -g.pad};
-        const int upper[2] = {g.pad - g.dil * (K - 1), g.pad - g.dil * (K - 1)};
-        const cuuint32_t estr[4] = {1, (cuuint32_t)g.stride, (cuuint32_t)g.stride, 1};
-        if (g_encode_im2col(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(X), dims, strides,
-                            lower, upper, 64, Cfg::BM, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return CONV_ERR_CUDA;
-    }
-    {   // F: 3-D {Cout, Cin, K*K}; a box is 64 reduction rows (channels) x 64 output channels
-        const cuuint64_t dims[3] = {(cuuint64_t)Cout, (cuuint64_t)Cin, (cuuint64_t)K * K};
-        const cuuint64_t strides[2] = {(cuuint64_t)Cout * 2, (cuuint64_t)Cin * Cout * 2};
-        const cuuint32_t box[3] = {64, 64, 1};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(F), dims, strides, box,
-                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return CONV_ERR_CUDA;
-    }
+// The im2col tensor-core kernel over groups g0 .. g0 + NG - 1 per launch (one launch when
+// there is one group). Per group: X channels g*Cin_g .. +Cin_g, filter and Y columns
+// g*Cout_g .. +Cout_g; the caller guarantees Cin_g and Cout_g multiples of 8 (16-byte map
+// bases) and window corners and tap reaches inside the 4-D im2col ranges.
+template <class Cfg, int NG>
+int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout,
+                    const DenseGeom &g, cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
+    const int Ho = static_cast<int>(g.ho(H)), Wo = static_cast<int>(g.wo(W));
+    const int Cin_g = Cin / g.groups, Cout_g = Cout / g.groups;
     const long long M = 1LL * N * Ho * Wo;
-    {   // Y: 2-D {Cout, M}; a box is 32 rows x 64 channels
-        const cuuint64_t dims[2] = {(cuuint64_t)Cout, (cuuint64_t)M};
-        const cuuint64_t strides[1] = {(cuuint64_t)Cout * 2};
-        const cuuint32_t box[2] = {64, 32};
-        const cuuint32_t estr[2] = {1, 1};
-        if (g_encode_tiled(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return CONV_ERR_CUDA;
-    }
     DenseTcParams p;
     p.M = static_cast<int>(M);
     p.Wo = Wo;
     p.HoWo = Ho * Wo;
-    p.K = K;
-    p.Cout = Cout;
-    p.num_cblk = (Cin + 63) / 64;
-    p.num_kblk = K * K * p.num_cblk;
-    p.num_ntiles = (Cout + Cfg::BN - 1) / Cfg::BN;
-    p.stride = g.stride; p.pad = g.pad; p.dil = g.dil; p.bias = g.bias;
-    const long long tiles = ((M + Cfg::BM - 1) / Cfg::BM) * p.num_ntiles;
-    if (tiles > kInt32Max) return CONV_ERR_UNSUPPORTED;
-    p.num_tiles = static_cast<int>(tiles);
-    auto kern = dense_tc_kernel<Cfg>;
+    p.KW = g.KW;
+    p.ncols = Cout_g;
+    p.num_cblk = (Cin_g + 63) / 64;
+    p.num_kblk = g.KH * g.KW * p.num_cblk;
+    p.num_ntiles = (Cout_g + Cfg::BN - 1) / Cfg::BN;
+    p.sh = g.sh; p.sw = g.sw; p.ph = g.ph; p.pw = g.pw; p.dh = g.dh; p.dw = g.dw;
+    const long long per_group = ((M + Cfg::BM - 1) / Cfg::BM) * p.num_ntiles;
+    if (per_group * NG > kInt32Max) return CONV_ERR_UNSUPPORTED;
+    p.tiles_per_group = static_cast<int>(per_group);
+    auto kern = dense_tc_kernel<Cfg, NG>;
     if (int rc = ensure_smem_attr(d, attr_bit, kern, Cfg::SMEM_BYTES)) return rc;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(p.num_tiles < d->num_sms ? p.num_tiles : d->num_sms));
-    cfg.blockDim = dim3(192);
-    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
-    cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, tmY, p, d->status), "dense_tc_kernel");
+    const auto *xb = static_cast<const __nv_bfloat16 *>(X);
+    const auto *fb = static_cast<const __nv_bfloat16 *>(F);
+    auto *yb = static_cast<__nv_bfloat16 *>(Y);
+    for (int g0 = 0; g0 < g.groups; g0 += NG) {
+        const int ng = g.groups - g0 < NG ? g.groups - g0 : NG;
+        DenseTcMaps<NG> maps;
+        for (int gl = 0; gl < NG; ++gl) {
+            // unused slots repeat the first group's maps (never dereferenced)
+            const int gg = g0 + (gl < ng ? gl : 0);
+            {   // X: 4-D {Cin_g, W, H, N} im2col at channel gg*Cin_g. The bounding box of window
+                // origins runs from -pad to (size - 1) + pad - dil*(taps - 1) on each spatial
+                // axis, walked with that axis's stride as element stride, so its pixels are
+                // exactly the output positions; origins, taps and channels outside read zeros.
+                const cuuint64_t dims[4] = {(cuuint64_t)Cin_g, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)N};
+                const cuuint64_t strides[3] = {(cuuint64_t)Cin * 2, (cuuint64_t)W * Cin * 2,
+                                               (cuuint64_t)H * W * Cin * 2};
+                const int lower[2] = {-g.pw, -g.ph};
+                const int upper[2] = {g.pw - g.dw * (g.KW - 1), g.ph - g.dh * (g.KH - 1)};
+                const cuuint32_t estr[4] = {1, (cuuint32_t)g.sw, (cuuint32_t)g.sh, 1};
+                if (g_encode_im2col(&maps.x[gl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                                    const_cast<__nv_bfloat16 *>(xb + 1LL * gg * Cin_g), dims, strides, lower, upper,
+                                    64, Cfg::BM, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                    return CONV_ERR_CUDA;
+            }
+            {   // F: 3-D {Cout_g, Cin_g, KH*KW} at column gg*Cout_g; a box is 64 reduction rows
+                // (channels) x 64 output channels
+                const cuuint64_t dims[3] = {(cuuint64_t)Cout_g, (cuuint64_t)Cin_g, (cuuint64_t)g.KH * g.KW};
+                const cuuint64_t strides[2] = {(cuuint64_t)Cout * 2, (cuuint64_t)Cin_g * Cout * 2};
+                const cuuint32_t box[3] = {64, 64, 1};
+                const cuuint32_t estr[3] = {1, 1, 1};
+                if (g_encode_tiled(&maps.f[gl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                                   const_cast<__nv_bfloat16 *>(fb + 1LL * gg * Cout_g), dims, strides, box, estr,
+                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                    return CONV_ERR_CUDA;
+            }
+            {   // Y: 2-D {Cout_g, M} at column gg*Cout_g; a box is 32 rows x 64 channels
+                const cuuint64_t dims[2] = {(cuuint64_t)Cout_g, (cuuint64_t)M};
+                const cuuint64_t strides[1] = {(cuuint64_t)Cout * 2};
+                const cuuint32_t box[2] = {64, 32};
+                const cuuint32_t estr[2] = {1, 1};
+                if (g_encode_tiled(&maps.y[gl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, yb + 1LL * gg * Cout_g, dims,
+                                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                    return CONV_ERR_CUDA;
+            }
+        }
+        p.groups = ng;
+        p.num_tiles = ng * p.tiles_per_group;
+        p.bias = g.bias ? g.bias + 1LL * g0 * Cout_g : nullptr;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(p.num_tiles < d->num_sms ? p.num_tiles : d->num_sms));
+        cfg.blockDim = dim3(192);
+        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cfg.stream = stream;
+        if (int rc = launched(cudaLaunchKernelEx(&cfg, kern, maps, p, d->status), "dense_tc_kernel")) return rc;
+    }
+    return CONV_OK;
 }
 
 // ---- halo kernel ------------------------------------------------------------------------
@@ -862,9 +903,10 @@ int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, 
     // tensors. The im2col tensor map is used only for inputs of at least 128 KiB.
     const bool tc_shape = (Cin % 8 == 0) && (Cout % 8 == 0) && aligned(X, 16) && aligned(F, 16) && aligned(Y, 16);
     const bool im2col_ok = tc_shape && K <= 128 && 2LL * N * H * W * Cin >= 128 * 1024;
+    const DenseGeom sq = DenseGeom::square(K);
     if ((force && std::strcmp(force, "direct") == 0) || !tc_shape)
         return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
-                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d);
+                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, sq, stream, d);
     // Default: the halo kernel; the im2col kernel when a halo does not fit in shared memory
     // (very wide images) or when forced. CONV_B200_DENSE (tests): "direct", "halo",
     // "halo64/128/256" (halo kernel with that tile width), "bn64/128/256" (im2col kernel).
@@ -893,12 +935,12 @@ int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, 
     if (!im2col_ok) {
         if (force_im2col) return CONV_ERR_UNSUPPORTED;
         return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
-                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d);
+                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, sq, stream, d);
     }
     int bn = force_bn ? force_bn : (Cout <= 64 ? 64 : 128);
-    if (bn == 64) return launch_dense_tc<CfgBN64>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 0);
-    if (bn == 128) return launch_dense_tc<CfgBN128>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 1);
-    return launch_dense_tc<CfgBN256>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 2);
+    if (bn == 64) return launch_dense_tc<CfgBN64, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 0);
+    if (bn == 128) return launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 1);
+    return launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 2);
 }
 
 int conv2d_nhwc_fwd_f32(const float *X, const float *F, float *Y, int N, int H, int W, int Cin, int Cout,
@@ -906,50 +948,103 @@ int conv2d_nhwc_fwd_f32(const float *X, const float *F, float *Y, int N, int H, 
     if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 4)) return rc;
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
-    return launch_dense_direct(X, F, Y, N, H, W, Cin, Cout, K, stream, d);
+    return launch_dense_direct(X, F, Y, N, H, W, Cin, Cout, DenseGeom::square(K), stream, d);
 }
+
+}  // extern "C"
+
+namespace convb200 {
+namespace {
+
+// Validation, dispatch and launch of the general dense convolution (every geometry field of g
+// set; g.plain() operations already routed to the plain entry by the callers).
+int dense_general(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout,
+                  const DenseGeom &g, cudaStream_t stream) {
+    const long long Ho = g.ho(H), Wo = g.wo(W);
+    const long long nx = 1LL * N * H * W * Cin, nf = 1LL * g.KH * g.KW * (Cin / g.groups) * Cout,
+                    ny = 1LL * N * Ho * Wo * Cout;
+    if (nx > kInt32Max || nf > kInt32Max || ny > kInt32Max || 1LL * N * Ho * Wo > kInt32Max)
+        return CONV_ERR_UNSUPPORTED;
+    if (!aligned(X, 2) || !aligned(F, 2) || !aligned(Y, 2) || (g.bias && !aligned(g.bias, 4)))
+        return CONV_ERR_MISALIGNED;
+    if (overlaps(Y, ny * 2, X, nx * 2) || overlaps(Y, ny * 2, F, nf * 2) ||
+        (g.bias && overlaps(Y, ny * 2, g.bias, 4LL * Cout)))
+        return CONV_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    const char *force = env("CONV_B200_DENSE");
+    // Tensor cores through the TMA im2col unit: 16-byte channel rows per group (group bases
+    // 16-byte aligned), 16-byte aligned tensors, and window corners and tap offsets inside the
+    // 4-D im2col ranges (|corner| <= 127, offset <= 127).
+    const int Cin_g = Cin / g.groups, Cout_g = Cout / g.groups;
+    const bool tc_shape = (Cin_g % 8 == 0) && (Cout_g % 8 == 0) && aligned(X, 16) && aligned(F, 16) && aligned(Y, 16);
+    auto axis_ok = [](int pad, int dil, int taps) {
+        const long long reach = 1LL * dil * (taps - 1);
+        return pad <= 127 && reach <= 127 && pad - reach >= -127 && pad - reach <= 127;
+    };
+    const bool im2col_ok = tc_shape && axis_ok(g.ph, g.dh, g.KH) && axis_ok(g.pw, g.dw, g.KW) &&
+                           2LL * N * H * W * Cin >= 128 * 1024;
+    const bool force_bn = force && std::strncmp(force, "bn", 2) == 0;
+    if ((force && std::strcmp(force, "direct") == 0) || !im2col_ok) {
+        if (force_bn) return CONV_ERR_UNSUPPORTED;
+        return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
+                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, g, stream, d);
+    }
+    int bn = Cout_g <= 64 ? 64 : 128;
+    if (force_bn) bn = std::atoi(force + 2);
+    if (g.groups == 1) {
+        if (bn == 64) return launch_dense_tc<CfgBN64, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 0);
+        if (bn == 128) return launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 1);
+        if (bn == 256) return launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 2);
+        return CONV_ERR_INVALID_ARG;
+    }
+    // several groups: up to kTcGroups per launch (shared-memory attribute bits 48..50)
+    if (bn == 64) return launch_dense_tc<CfgBN64, kTcGroups>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 48);
+    if (bn == 128) return launch_dense_tc<CfgBN128, kTcGroups>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 49);
+    if (bn == 256) return launch_dense_tc<CfgBN256, kTcGroups>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 50);
+    return CONV_ERR_INVALID_ARG;
+}
+
+}  // namespace
+}  // namespace convb200
+
+extern "C" {
 
 int conv2d_nhwc_fwd_ex(const void *X, const void *F, const float *bias, void *Y, int N, int H, int W, int Cin,
                        int Cout, int K, int stride, int pad, int dil, cudaStream_t stream) {
     if (!X || !F || !Y) return CONV_ERR_INVALID_ARG;
     if (N < 1 || H < 1 || W < 1 || Cin < 1 || Cout < 1 || K < 1 || stride < 1 || dil < 1 || pad < 0)
         return CONV_ERR_INVALID_ARG;
-    DenseGeom g;
-    g.stride = stride; g.pad = pad; g.dil = dil; g.bias = bias;
+    const DenseGeom g = DenseGeom::square(K, stride, pad, dil, bias);
     if (1LL * H + 2LL * pad > kInt32Max / 2 || 1LL * W + 2LL * pad > kInt32Max / 2 ||
         1LL * dil * (K - 1) > kInt32Max / 2)
         return CONV_ERR_UNSUPPORTED;
-    const long long Ho = g.ho(H, K), Wo = g.ho(W, K);
-    if (1LL * H + 2LL * pad < 1LL * dil * (K - 1) + 1 || 1LL * W + 2LL * pad < 1LL * dil * (K - 1) + 1 || Ho < 1 ||
-        Wo < 1)
+    if (1LL * H + 2LL * pad < 1LL * dil * (K - 1) + 1 || 1LL * W + 2LL * pad < 1LL * dil * (K - 1) + 1)
         return CONV_ERR_INVALID_ARG;
     if (g.plain()) return conv2d_nhwc_fwd(X, F, Y, N, H, W, Cin, Cout, K, stream);
-    const long long nx = 1LL * N * H * W * Cin, nf = 1LL * K * K * Cin * Cout, ny = 1LL * N * Ho * Wo * Cout;
-    if (nx > kInt32Max || nf > kInt32Max || ny > kInt32Max || 1LL * N * Ho * Wo > kInt32Max)
-        return CONV_ERR_UNSUPPORTED;
-    if (!aligned(X, 2) || !aligned(F, 2) || !aligned(Y, 2) || (bias && !aligned(bias, 4))) return CONV_ERR_MISALIGNED;
-    if (overlaps(Y, ny * 2, X, nx * 2) || overlaps(Y, ny * 2, F, nf * 2) || (bias && overlaps(Y, ny * 2, bias, 4LL * Cout)))
+    return dense_general(X, F, Y, N, H, W, Cin, Cout, g, stream);
+}
+
+int conv2d_nhwc_fwd_grouped(const void *X, const void *F, const float *bias, void *Y, int N, int H, int W, int Cin,
+                            int Cout, int KH, int KW, int stride_h, int stride_w, int pad_h, int pad_w, int dil_h,
+                            int dil_w, int groups, cudaStream_t stream) {
+    if (!X || !F || !Y) return CONV_ERR_INVALID_ARG;
+    if (N < 1 || H < 1 || W < 1 || Cin < 1 || Cout < 1 || KH < 1 || KW < 1 || stride_h < 1 || stride_w < 1 ||
+        dil_h < 1 || dil_w < 1 || pad_h < 0 || pad_w < 0 || groups < 1 || Cin % groups != 0 || Cout % groups != 0)
         return CONV_ERR_INVALID_ARG;
-    DeviceState *d = nullptr;
-    if (int rc = device_state(&d)) return rc;
-    const char *force = env("CONV_B200_DENSE");
-    // Tensor cores through the TMA im2col unit: 16-byte channel rows and tensors, and window
-    // corners and tap offsets inside the 4-D im2col ranges (|corner| <= 127, offset <= 127).
-    const bool tc_shape = (Cin % 8 == 0) && (Cout % 8 == 0) && aligned(X, 16) && aligned(F, 16) && aligned(Y, 16);
-    const long long reach = 1LL * dil * (K - 1);
-    const bool im2col_ok = tc_shape && pad <= 127 && reach <= 127 && pad - reach >= -127 && pad - reach <= 127 &&
-                           2LL * N * H * W * Cin >= 128 * 1024;
-    if ((force && std::strcmp(force, "direct") == 0) || !im2col_ok) {
-        if (force && std::strncmp(force, "bn", 2) == 0) return CONV_ERR_UNSUPPORTED;
-        return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
-                                   static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, K, stream, d, g);
-    }
-    int bn = Cout <= 64 ? 64 : 128;
-    if (force && std::strncmp(force, "bn", 2) == 0) bn = std::atoi(force + 2);
-    if (bn == 64) return launch_dense_tc<CfgBN64>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 0, g);
-    if (bn == 128) return launch_dense_tc<CfgBN128>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 1, g);
-    if (bn == 256) return launch_dense_tc<CfgBN256>(X, F, Y, N, H, W, Cin, Cout, K, stream, d, 2, g);
-    return CONV_ERR_INVALID_ARG;
+    if (1LL * H + 2LL * pad_h > kInt32Max / 2 || 1LL * W + 2LL * pad_w > kInt32Max / 2 ||
+        1LL * dil_h * (KH - 1) > kInt32Max / 2 || 1LL * dil_w * (KW - 1) > kInt32Max / 2)
+        return CONV_ERR_UNSUPPORTED;
+    if (1LL * H + 2LL * pad_h < 1LL * dil_h * (KH - 1) + 1 || 1LL * W + 2LL * pad_w < 1LL * dil_w * (KW - 1) + 1)
+        return CONV_ERR_INVALID_ARG;
+    DenseGeom g;
+    g.KH = KH; g.KW = KW;
+    g.sh = stride_h; g.sw = stride_w; g.ph = pad_h; g.pw = pad_w; g.dh = dil_h; g.dw = dil_w;
+    g.groups = groups;
+    g.bias = bias;
+    if (KH == KW && stride_h == stride_w && pad_h == pad_w && dil_h == dil_w && groups == 1)
+        return conv2d_nhwc_fwd_ex(X, F, bias, Y, N, H, W, Cin, Cout, KH, stride_h, pad_h, dil_h, stream);
+    return dense_general(X, F, Y, N, H, W, Cin, Cout, g, stream);
 }
 
 size_t conv2d_nhwc_im2col_workspace(int N, int H, int W, int Cin, int K) {

@@ -7,17 +7,21 @@
 // multiply-adds in (i, j, c) order, rounded once to the output type -- and the stride, zero
 // padding, dilation and bias variants of "Convolution Is Wx+b Moving Across a Signal" (window
 // of output (y, x) at (y*stride - pad, x*stride - pad), taps dil apart, positions outside the
-// image skipped as zeros, the bias one fp32 addition before the rounding). Consecutive threads
-// take consecutive output channels o, so the F row reads are coalesced and the X reads are
-// warp-uniform broadcasts.
+// image skipped as zeros, the bias one fp32 addition before the rounding), with separate
+// height and width geometry, KH x KW filters and channel groups (output channel o of group
+// g = o / (Cout/groups) sums only input channels g*Cin_g .. +Cin_g, Cin_g = Cin/groups, with
+// filter F[i, j, c, o] for the group-local channel c; a Conv1D is the H = KH = 1 case).
+// Consecutive threads take consecutive output channels o, so the F row reads are coalesced and
+// the X reads are warp-uniform broadcasts (or few-address ones across a group boundary).
 #pragma once
 #include <cuda_bf16.h>
 
 namespace convb200 {
 
 struct DenseDirectParams {
-    int H, W, Cin, Cout, K, Ho, Wo;
-    int stride, pad, dil;   // "Convolution Is Wx+b Moving Across a Signal" variants
+    int H, W, Cin, Cout, KH, KW, Ho, Wo;
+    int Cin_g, Cout_g;      // channels of one group (Cin, Cout when there is one group)
+    int sh, sw, ph, pw, dh, dw;   // "Convolution Is Wx+b Moving Across a Signal" variants
     const float *bias;      // per output channel or null; added in fp32 before the rounding
     long long total;        // N * Ho * Wo * Cout
 };
@@ -41,16 +45,17 @@ dense_direct_kernel(const T *__restrict__ X, const T *__restrict__ F, T *__restr
         t /= p.Wo;
         const int y = static_cast<int>(t % p.Ho);
         const long long n = t / p.Ho;
+        const int cin0 = (o / p.Cout_g) * p.Cin_g;
         float acc = 0.0f;
-        for (int i = 0; i < p.K; ++i) {
-            const int r = y * p.stride + i * p.dil - p.pad;
+        for (int i = 0; i < p.KH; ++i) {
+            const int r = y * p.sh + i * p.dh - p.ph;
             if (r < 0 || r >= p.H) continue;   // zero padding contributes nothing
-            for (int j = 0; j < p.K; ++j) {
-                const int q = x * p.stride + j * p.dil - p.pad;
+            for (int j = 0; j < p.KW; ++j) {
+                const int q = x * p.sw + j * p.dw - p.pw;
                 if (q < 0 || q >= p.W) continue;
-                const T *xr = X + ((n * p.H + r) * p.W + q) * p.Cin;
-                const T *fr = F + ((static_cast<long long>(i) * p.K + j) * p.Cin) * p.Cout + o;
-                for (int c = 0; c < p.Cin; ++c)
+                const T *xr = X + ((n * p.H + r) * p.W + q) * p.Cin + cin0;
+                const T *fr = F + ((static_cast<long long>(i) * p.KW + j) * p.Cin_g) * p.Cout + o;
+                for (int c = 0; c < p.Cin_g; ++c)
                     acc = __fmaf_rn(to_f32(xr[c]), to_f32(fr[static_cast<long long>(c) * p.Cout]), acc);
             }
         }

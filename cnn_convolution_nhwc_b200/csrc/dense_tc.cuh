@@ -4,15 +4,22 @@
 // channels and batches"; with the stride, zero-padding, dilation and bias variants of
 // "Convolution Is Wx+b Moving Across a Signal", which the TMA im2col unit expresses directly:
 // element strides for the stride, a bounding box that starts at -pad for the padding, with
-// out-of-range pixels read as zeros, and tap offsets scaled by the dilation): A_col[(n,y,x), (i,j,c)] = X[n, y+i, x+j, c] is the
-// (N*Ho*Wo) x (K*K*Cin) patch matrix, F_mat is F viewed as (K*K*Cin) x Cout, and
-// Y_mat = A_col * F_mat is Y viewed as (N*Ho*Wo) x Cout. The notes' closing remark in
-// section 6 -- generate patch fragments as needed instead of materialising the matrix --
-// is what this kernel does: A_col never exists in memory. Each 128-row x 64-column block of
-// it is gathered straight from X by one TMA im2col load (the hardware form of the
-// overlapping-window view of section 4), for filter tap (i, j) and channel block c0, and
-// consumed from shared memory by tcgen05 MMAs. The reduction runs tap by tap, which is the
-// sum of K*K shifted-slice channel matmuls of section 2.
+// out-of-range pixels read as zeros, and tap offsets scaled by the dilation, each per axis):
+// A_col[(n,y,x), (i,j,c)] = X[n, y+i, x+j, c] is the (N*Ho*Wo) x (KH*KW*Cin) patch matrix,
+// F_mat is F viewed as (KH*KW*Cin) x Cout, and Y_mat = A_col * F_mat is Y viewed as
+// (N*Ho*Wo) x Cout. The notes' closing remark in section 6 -- generate patch fragments as
+// needed instead of materialising the matrix -- is what this kernel does: A_col never exists
+// in memory. Each 128-row x 64-column block of it is gathered straight from X by one TMA
+// im2col load (the hardware form of the overlapping-window view of section 4), for filter
+// tap (i, j) and channel block c0, and consumed from shared memory by tcgen05 MMAs. The
+// reduction runs tap by tap, which is the sum of KH*KW shifted-slice channel matmuls of
+// section 2.
+//
+// Channel groups (the grouped Conv1D of the Wx+b page's section "Find the same sum in CKE's
+// C kernels", on two axes) are independent GEMMs of the same shape: a group has its own three
+// tensor maps (X at channel g*Cin_g, F and Y at column g*Cout_g, each with the group's extent,
+// so boxes past a group's end read zeros and stores are clipped to it), and the persistent
+// tile loop runs over (group, row block, column block).
 //
 // Roles inside one persistent CTA of 6 warps (each role loop is walked by whole, converged
 // warps; a single lane issues the asynchronous instructions):
@@ -35,18 +42,34 @@
 namespace convb200 {
 
 struct DenseTcParams {
-    int M;          // N * Ho * Wo (GEMM rows)
+    int M;          // N * Ho * Wo (GEMM rows of every group)
     int Wo;
     int HoWo;
-    int K;
-    int Cout;
-    int num_cblk;   // ceil(Cin / 64)
-    int num_kblk;   // K * K * num_cblk
-    int num_ntiles; // ceil(Cout / BN)
-    int num_tiles;  // ceil(M / 128) * num_ntiles
-    int stride, pad, dil;   // window of output (y, x) starts at (y*stride - pad, x*stride - pad);
-                            // tap (i, j) is dil*i rows and dil*j columns further on
-    const float *bias;      // per output channel, added in fp32 before the bf16 rounding; or null
+    int KW;         // taps per filter row (the reduction walks ky outer, kx inner)
+    int ncols;      // output channels of one group (Cout / groups)
+    int num_cblk;   // ceil(Cin_g / 64), Cin_g = input channels of one group
+    int num_kblk;   // KH * KW * num_cblk
+    int num_ntiles; // ceil(ncols / BN)
+    int tiles_per_group;   // ceil(M / 128) * num_ntiles
+    int num_tiles;  // groups of this launch * tiles_per_group
+    int groups;     // groups of this launch (tensor maps in use)
+    int sh, sw, ph, pw, dh, dw;   // window of output (y, x) starts at (y*sh - ph, x*sw - pw);
+                                  // tap (i, j) is dh*i rows and dw*j columns further on
+    const float *bias;      // per output channel of this launch's first group (group g's at
+                            // bias + g*ncols), added in fp32 before the bf16 rounding; or null
+};
+
+// Tensor maps of the groups one launch covers: group g reads X channels g*Cin_g .. +Cin_g
+// (map x[g], channel extent Cin_g, so a 64-channel box past the group reads zeros), filter
+// columns g*ncols .. +ncols (f[g]) and writes Y columns g*ncols .. +ncols (y[g], stores
+// clipped to the group).
+constexpr int kTcGroups = 8;   // groups per launch of the grouped instantiation (24 maps, 3 KB)
+
+template <int NG>
+struct alignas(64) DenseTcMaps {
+    CUtensorMap x[NG];
+    CUtensorMap f[NG];
+    CUtensorMap y[NG];
 };
 
 template <int BN_, int STAGES_>
@@ -81,11 +104,9 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-template <class Cfg>
+template <class Cfg, int NG>
 __global__ void __launch_bounds__(192, 1)
-dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
-                const __grid_constant__ CUtensorMap tmY, const DenseTcParams p,
-                unsigned int *status) {
+dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParams p, unsigned int *status) {
     constexpr int BN = Cfg::BN;
     constexpr int STAGES = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -121,9 +142,11 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         mbar_init(done_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
-        prefetch_tensormap(&tmX);
-        prefetch_tensormap(&tmF);
-        prefetch_tensormap(&tmY);
+        for (int g = 0; g < p.groups; ++g) {
+            prefetch_tensormap(&maps.x[g]);
+            prefetch_tensormap(&maps.f[g]);
+            prefetch_tensormap(&maps.y[g]);
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
@@ -138,14 +161,23 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         atomicOr(status, kStatusTimeout);
         *abort_flag = 1;
     };
+    // tile -> (group of this launch, 128-row block, BN-column block)
+    auto split = [&](int tile, int &g, int &mt, int &nt) {
+        g = NG == 1 ? 0 : tile / p.tiles_per_group;
+        const int rem = tile - g * p.tiles_per_group;
+        mt = rem / p.num_ntiles;
+        nt = rem - mt * p.num_ntiles;
+    };
 
     if (warp == 0) {
         // ------------------------------- TMA producer -------------------------------
         // The whole warp walks the loop (it stays converged); lane 0 issues.
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
-            const int mt = tile / p.num_ntiles;
-            const int nt = tile - mt * p.num_ntiles;
+            int g, mt, nt;
+            split(tile, g, mt, nt);
+            const CUtensorMap *tmX = &maps.x[g];
+            const CUtensorMap *tmF = &maps.f[g];
             const int m0 = mt * Cfg::BM;
             const int n0 = nt * BN;
             const int img = m0 / p.HoWo;
@@ -164,12 +196,12 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(full_bar(s), Cfg::STAGE_BYTES);
-                    tma_load_im2col_4d(sA + s * Cfg::A_BYTES, &tmX, full_bar(s), cb * 64, ox * p.stride - p.pad,
-                                       oy * p.stride - p.pad, img, static_cast<uint16_t>(kx * p.dil),
-                                       static_cast<uint16_t>(ky * p.dil));
+                    tma_load_im2col_4d(sA + s * Cfg::A_BYTES, tmX, full_bar(s), cb * 64, ox * p.sw - p.pw,
+                                       oy * p.sh - p.ph, img, static_cast<uint16_t>(kx * p.dw),
+                                       static_cast<uint16_t>(ky * p.dh));
 #pragma unroll
                     for (int h = 0; h < BN / 64; ++h)
-                        tma_load_3d(sB + s * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, &tmF, full_bar(s),
+                        tma_load_3d(sB + s * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, tmF, full_bar(s),
                                     n0 + h * 64, cb * 64, tap);
                 }
                 __syncwarp();
@@ -177,7 +209,7 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 if (++cb == p.num_cblk) {
                     cb = 0;
                     ++tap;
-                    if (++kx == p.K) { kx = 0; ++ky; }
+                    if (++kx == p.KW) { kx = 0; ++ky; }
                 }
             }
             if (!ok) break;
@@ -254,8 +286,8 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             const bool ok = mbar_wait_warp(accf_bar(b), aph);
             if (!ok) { if (lane == 0) fail(); break; }
             tc_fence_after();
-            const int mt = tile / p.num_ntiles;
-            const int nt = tile - mt * p.num_ntiles;
+            int g, mt, nt;
+            split(tile, g, mt, nt);
             const int m0 = mt * Cfg::BM;
             const int n0 = nt * BN;
             // the staging buffer is free once the previous tile's stores have read it
@@ -270,13 +302,14 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 tmem_wait_ld();
                 if (p.bias) {   // one fp32 addition per output, before the single rounding
                     const int c0 = n0 + h * 64;
+                    const float *bg = p.bias + static_cast<long long>(g) * p.ncols;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
+                    for (int u = 0; u < 4; ++u)
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
-                            const int col = c0 + g * 16 + c;
-                            const float bv = col < p.Cout ? __ldg(p.bias + col) : 0.0f;
-                            r[g][c] = __float_as_uint(__fadd_rn(__uint_as_float(r[g][c]), bv));
+                            const int col = c0 + u * 16 + c;
+                            const float bv = col < p.ncols ? __ldg(bg + col) : 0.0f;
+                            r[u][c] = __float_as_uint(__fadd_rn(__uint_as_float(r[u][c]), bv));
                         }
                 }
                 const uint32_t row_addr = stage_s + h * 4096 + lane * 128;
@@ -305,7 +338,7 @@ dense_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 if (row0 < p.M) {
 #pragma unroll
                     for (int h = 0; h < BN / 64; ++h)
-                        if (n0 + h * 64 < p.Cout) tma_store_2d(&tmY, stage_s + h * 4096, n0 + h * 64, row0);
+                        if (n0 + h * 64 < p.ncols) tma_store_2d(&maps.y[g], stage_s + h * 4096, n0 + h * 64, row0);
                     bulk_commit_group();
                 }
             }

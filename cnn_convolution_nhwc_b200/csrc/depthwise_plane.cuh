@@ -94,15 +94,16 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
     int k = 0;
     bool ok = true;
     for (int job = gw; job < p.num_jobs; job += GW, ++k) {
-        if (!mbar_wait_warp(bar, k & 1)) { ok = false; break; }
         const int plane0 = job * PPJ;
         const int plane = plane0 + slot;
         const bool active = plane < p.num_planes;
         const int c = active ? plane - fdiv(plane, p.div_c) * p.C : 0;
+        // the plane's weights load while the bulk copy is in flight
         float wr[K * K];
 #pragma unroll
         for (int t = 0; t < K * K; ++t) wr[t] = __ldg(w + c * (K * K) + t);
         const float bv = HAS_BIAS ? __ldg(bias + c) : 0.0f;
+        if (!mbar_wait_warp(bar, k & 1)) { ok = false; break; }
 
         // input row iy (compile-time) of this lane's columns; zeros outside the plane
         auto load_row = [&](int iy, float (&row)[WINC]) {

@@ -102,6 +102,38 @@ int conv2d_nhwc_fwd_ex(const void *X, const void *F, const float *bias, void *Y,
                        int stride, int pad, int dil, cudaStream_t stream);
 
 /*
+ * Grouped dense NHWC forward convolution with a KH x KW filter and separate height and width
+ * geometry; a Conv1D over a sequence of W frames is the H = KH = 1 case. The grouping is the
+ * one "Convolution Is Wx+b Moving Across a Signal" describes in section "Find the same sum in
+ * CKE's C kernels" (an output channel sums only the input channels and taps of its own group,
+ * frame index out*stride + tap - padding, taps outside the input skipped), extended to two
+ * axes as that section's 2-D grouped kernel does:
+ *     Cin_g = Cin / groups, Cout_g = Cout / groups, g(o) = o / Cout_g,
+ *     Ho = floor((H + 2*pad_h - (dil_h*(KH-1) + 1)) / stride_h) + 1   (Wo likewise with _w),
+ *     Y[n,y,x,o] = bias[o] + sum_{i<KH, j<KW, c<Cin_g}
+ *                  X[n, y*stride_h + i*dil_h - pad_h, x*stride_w + j*dil_w - pad_w, g(o)*Cin_g + c]
+ *                  * F[i,j,c,o],
+ * with X read as zero outside the image.
+ *   X    : bfloat16 [N][H][W][Cin]
+ *   F    : bfloat16 [KH][KW][Cin_g][Cout] (row (i, j, c) of group g(o)'s filter matrix, column o)
+ *   bias : float32 [Cout] or NULL; added in float32 to the float32 sum before the single
+ *          rounding to bfloat16 (the order of the dense entries; the page's scalar Conv1D starts
+ *          its float32 accumulator at the bias instead, which only reorders the rounding)
+ *   Y    : bfloat16 [N][Ho][Wo][Cout]
+ * Requirements: N, H, W, Cin, Cout, KH, KW, strides, dilations, groups >= 1; pads >= 0; groups
+ * divides Cin and Cout; Ho, Wo >= 1; X, F, Y non-null and 2-byte aligned, bias 4-byte aligned;
+ * element counts below 2^31. With KH = KW, equal per-axis values and one group this is exactly
+ * conv2d_nhwc_fwd_ex. The tensor-core path needs Cin_g and Cout_g multiples of 8, 16-byte aligned
+ * tensors and, per axis, pad <= 127, dil*(taps-1) <= 127 and |pad - dil*(taps-1)| <= 127; other
+ * valid shapes take a CUDA-core path with the same contract. Several groups run as independent
+ * implicit GEMMs inside one persistent launch per 8 groups.
+ */
+int conv2d_nhwc_fwd_grouped(const void *X, const void *F, const float *bias, void *Y,
+                            int N, int H, int W, int Cin, int Cout, int KH, int KW,
+                            int stride_h, int stride_w, int pad_h, int pad_w, int dil_h, int dil_w,
+                            int groups, cudaStream_t stream);
+
+/*
  * Comparison path: the same operation as conv2d_nhwc_fwd computed the way the CMU DLSys Lecture
  * 14 notes build it in section 5 "Generalize the patch matrix to channels and batches" -- an
  * explicit patch matrix A[(n,y,x), (i,j,c)] = X[n,y+i,x+j,c] of N*Ho*Wo rows by K*K*Cin columns,

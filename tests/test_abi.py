@@ -121,6 +121,33 @@ def test_dense_ex_plain_geometry_validates_like_the_plain_entry():
         cb.CONV_ERR_MISALIGNED
 
 
+@pytest.mark.parametrize("args,code", [
+    # X, F, bias, Y, N, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups
+    ((None, F, B, Y, 1, 9, 9, 8, 8, 3, 3, 1, 1, 0, 0, 1, 1, 2), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 3, 1, 1, 0, 0, 1, 1, 0), cb.CONV_ERR_INVALID_ARG),     # no groups
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 3, 1, 1, 0, 0, 1, 1, 3), cb.CONV_ERR_INVALID_ARG),     # 3 does not divide 8
+    ((X, F, B, Y, 1, 9, 9, 12, 8, 3, 3, 1, 1, 0, 0, 1, 1, 3), cb.CONV_ERR_INVALID_ARG),    # ... nor Cout
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 0, 3, 1, 1, 0, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),     # KH 0
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 3, 1, 0, 0, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),     # stride_w 0
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 3, 1, 1, 0, -1, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),    # pad_w < 0
+    ((X, F, B, Y, 1, 9, 9, 8, 8, 3, 3, 1, 1, 0, 0, 0, 1, 1), cb.CONV_ERR_INVALID_ARG),     # dil_h 0
+    ((X, F, B, Y, 1, 1, 9, 8, 8, 3, 1, 1, 1, 0, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),     # KH 3 on one row
+    ((X, F, B, Y, 1, 9, 4, 8, 8, 1, 3, 1, 1, 0, 0, 1, 2, 1), cb.CONV_ERR_INVALID_ARG),     # dilated KW > W
+    ((V((1 << 20) + 1), F, B, Y, 1, 9, 9, 8, 8, 3, 1, 2, 1, 1, 0, 1, 1, 2), cb.CONV_ERR_MISALIGNED),
+    ((X, F, B, V(1 << 20), 1, 9, 9, 8, 8, 1, 3, 1, 2, 0, 1, 1, 1, 2), cb.CONV_ERR_INVALID_ARG),   # Y aliases X
+    ((X, F, B, Y, 4096, 4096, 4096, 64, 8, 3, 1, 1, 2, 1, 1, 1, 1, 8), cb.CONV_ERR_UNSUPPORTED),
+])
+def test_dense_grouped_rejects(args, code):
+    assert cb.lib.conv2d_nhwc_fwd_grouped(*args, None) == code
+
+
+def test_dense_grouped_square_one_group_validates_like_ex():
+    # KH = KW, equal axes and one group is conv2d_nhwc_fwd_ex: the same checks apply
+    args = (X, F, B, Y, 1, 2, 2, 8, 8, 5, 5, 1, 1, 1, 1, 1, 1, 1)
+    assert cb.lib.conv2d_nhwc_fwd_grouped(*args, None) == cb.CONV_ERR_INVALID_ARG
+    assert cb.lib.conv2d_nhwc_fwd_ex(X, F, B, Y, 1, 2, 2, 8, 8, 5, 1, 1, 1, None) == cb.CONV_ERR_INVALID_ARG
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

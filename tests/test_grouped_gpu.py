@@ -1,0 +1,180 @@
+"""GPU parity of conv2d_nhwc_fwd_grouped (channel groups, KH x KW filters, per-axis stride,
+padding and dilation, Conv1D as H = 1) against the float64 grouped oracle.
+
+Every case goes through the C ABI with seeded bf16 operands; the bar is the dense tolerance
+|y - y_ref| <= 4e-3 * (sum|x||w| + |b|) per output.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+TOL = 4e-3
+
+
+@pytest.fixture(scope="module")
+def cb(cuda):
+    import cnn_convolution_nhwc_b200 as cb
+    return cb
+
+
+def _case(N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, seed=0):
+    return workloads.DenseCase("t", N, H, W, Cin, Cout, KH, "bf16", "normal", seed, stride=s[0], pad=p[0], dil=d[0],
+                               bias=bias, groups=groups, KW=KW, stride_w=s[1], pad_w=p[1], dil_w=d[1])
+
+
+def _geom(c):
+    return (c.stride, c.sw), (c.pad, c.pw), (c.dil, c.dw)
+
+
+def _run(cb, c, Xb, Fb, b, env=None):
+    old = os.environ.get("CONV_B200_DENSE")
+    if env is not None:
+        os.environ["CONV_B200_DENSE"] = env
+    try:
+        X = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).cuda()
+        F = torch.from_numpy(Fb.view(np.int16)).view(torch.bfloat16).cuda()
+        bt = None if b is None else torch.from_numpy(np.ascontiguousarray(b, np.float32)).cuda()
+        s, p, d = _geom(c)
+        Y = cb.conv2d_nhwc_fwd_grouped(X, F, bt, stride=s, pad=p, dil=d, groups=c.groups)
+        kernel = cb.conv_last_kernel()
+        y = workloads.bf16_to_f32(Y.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
+    finally:
+        if env is not None:
+            if old is None:
+                del os.environ["CONV_B200_DENSE"]
+            else:
+                os.environ["CONV_B200_DENSE"] = old
+    assert cb.conv_device_status() == cb.CONV_OK
+    return y, kernel
+
+
+def _check(c, y, Xb, Fb, b):
+    s, p, d = _geom(c)
+    ref, absum = oracle.conv2d_grouped(workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb), b, s, p, d, c.groups)
+    assert y.shape == ref.shape
+    assert np.all(np.isfinite(y))
+    bad = np.abs(y - ref) > TOL * absum
+    assert not bad.any(), f"{bad.sum()} outputs out of tolerance"
+
+
+# (N, H, W, Cin, Cout, KH, KW, stride, pad, dil, groups, bias, kernel expected by default)
+CASES = [
+    (4, 28, 28, 128, 128, 3, 3, (1, 1), (1, 1), (1, 1), 2, True, "dense_tc_kernel"),       # two 64-wide groups
+    (2, 28, 28, 256, 256, 3, 3, (2, 2), (1, 1), (1, 1), 4, True, "dense_tc_kernel"),       # RegNet-style, stride 2
+    (2, 16, 16, 256, 256, 3, 3, (1, 1), (1, 1), (1, 1), 16, False, "dense_tc_kernel"),     # 16 groups: two launches
+    (1, 20, 20, 256, 256, 3, 3, (1, 1), (1, 1), (1, 1), 32, True, "dense_tc_kernel"),      # 8-channel groups
+    (2, 24, 20, 96, 192, 3, 3, (1, 1), (2, 2), (2, 1), 3, True, "dense_tc_kernel"),        # dilation per axis, ragged N tile
+    (4, 17, 17, 64, 64, 1, 7, (1, 1), (0, 3), (1, 1), 1, True, "dense_tc_kernel"),         # 1x7, one group
+    (4, 17, 17, 64, 96, 7, 1, (1, 1), (3, 0), (1, 1), 1, False, "dense_tc_kernel"),        # 7x1
+    (4, 30, 30, 64, 64, 3, 1, (2, 1), (1, 0), (1, 1), 1, True, "dense_tc_kernel"),         # stride per axis
+    (2, 1, 3000, 80, 512, 1, 3, (1, 1), (0, 1), (1, 1), 1, True, "dense_tc_kernel"),      # Conv1D, 80 channels
+    (2, 1, 3000, 256, 256, 1, 3, (1, 2), (0, 1), (1, 1), 1, True, "dense_tc_kernel"),     # Conv1D, stride 2
+    (2, 1, 1000, 128, 128, 1, 5, (1, 1), (0, 4), (1, 2), 4, True, "dense_tc_kernel"),     # grouped dilated Conv1D
+    (2, 9, 11, 12, 24, 3, 2, (1, 2), (1, 0), (1, 1), 3, True, "dense_direct_kernel"),     # 4-channel groups
+    (2, 1, 50, 8, 8, 1, 3, (1, 1), (0, 1), (1, 1), 2, False, "dense_direct_kernel"),      # tiny Conv1D
+]
+
+
+def _ids(c):
+    return "N{}H{}W{}C{}-{}k{}x{}s{}p{}d{}g{}".format(*c[:7], *["".join(map(str, t)) for t in c[7:10]], c[10]) + \
+        ("b" if c[11] else "")
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_grouped_geometry(cb, case):
+    N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, expected = case
+    c = _case(N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, seed=abs(hash(case[:11])) % 1000)
+    Xb, Fb = workloads.dense_inputs(c)
+    b = workloads.dense_bias(c)
+    y, kernel = _run(cb, c, Xb, Fb, b)
+    _check(c, y, Xb, Fb, b)
+    assert kernel == expected
+
+
+@pytest.mark.parametrize("case", [CASES[1], CASES[4], CASES[8]], ids=_ids)
+def test_tensor_core_and_direct_paths_agree(cb, case):
+    N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, _ = case
+    c = _case(N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, seed=5)
+    Xb, Fb = workloads.dense_inputs(c)
+    b = workloads.dense_bias(c)
+    y_tc, k_tc = _run(cb, c, Xb, Fb, b)
+    y_cc, k_cc = _run(cb, c, Xb, Fb, b, env="direct")
+    assert (k_tc, k_cc) == ("dense_tc_kernel", "dense_direct_kernel")
+    _check(c, y_tc, Xb, Fb, b)
+    _check(c, y_cc, Xb, Fb, b)
+
+
+@pytest.mark.parametrize("bn", ["bn64", "bn128", "bn256"])
+def test_grouped_tile_widths(cb, bn):
+    c = _case(2, 20, 20, 384, 384, 3, 3, (1, 1), (1, 1), (1, 1), 2, True, seed=8)   # 192-wide groups
+    Xb, Fb = workloads.dense_inputs(c)
+    b = workloads.dense_bias(c)
+    y, kernel = _run(cb, c, Xb, Fb, b, env=bn)
+    assert kernel == "dense_tc_kernel"
+    _check(c, y, Xb, Fb, b)
+
+
+def test_one_group_square_is_the_ex_entry(cb):
+    c = _case(4, 30, 30, 64, 64, 3, 3, (2, 2), (1, 1), (1, 1), 1, True, seed=3)
+    Xb, Fb = workloads.dense_inputs(c)
+    b = workloads.dense_bias(c)
+    y, _ = _run(cb, c, Xb, Fb, b)
+    X = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).cuda()
+    F = torch.from_numpy(Fb.view(np.int16)).view(torch.bfloat16).cuda()
+    y0 = cb.conv2d_nhwc_fwd_ex(X, F, torch.from_numpy(b).cuda(), stride=2, pad=1, dil=1)
+    y0 = workloads.bf16_to_f32(y0.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
+    assert np.array_equal(y, y0)
+
+
+def test_groups_do_not_mix(cb):
+    # a NaN planted in one group's input channels stays out of the other groups' outputs
+    c = _case(2, 20, 20, 128, 128, 3, 3, (1, 1), (1, 1), (1, 1), 2, False, seed=4)
+    Xb, Fb = workloads.dense_inputs(c)
+    Xb = Xb.copy()
+    Xb[..., 64:] = np.uint16(0x7FC0)   # bf16 quiet NaN
+    y, kernel = _run(cb, c, Xb, Fb, None)
+    assert kernel == "dense_tc_kernel"
+    assert np.all(np.isnan(y[..., 64:]))
+    ref, absum = oracle.conv2d_grouped(workloads.bf16_to_f32(Xb[..., :64]), workloads.bf16_to_f32(Fb[..., :64]), None,
+                                       1, 1, 1, 1)
+    assert np.all(np.abs(y[..., :64] - ref) <= TOL * absum)
+
+
+def test_page_two_filters_with_bias_as_conv1d(cb):
+    # "The matrix connection": x = 1..5, filters (2, 0, -1) and (1, 1, 1), biases 1 and 0 give
+    # (0, 1, 2) and (6, 9, 12); a one-row sequence of 8 channels (channel 0 carries the signal),
+    # 8 filters of which 0 and 1 are used
+    X = np.zeros((1, 1, 5, 8), np.float32)
+    X[0, 0, :, 0] = [1, 2, 3, 4, 5]
+    F = np.zeros((1, 3, 8, 8), np.float32)
+    F[0, :, 0, 0] = [2, 0, -1]
+    F[0, :, 0, 1] = [1, 1, 1]
+    b = np.zeros(8, np.float32)
+    b[0] = 1
+    c = _case(1, 1, 5, 8, 8, 1, 3, (1, 1), (0, 0), (1, 1), 1, True)
+    y, _ = _run(cb, c, workloads.bf16_bits(X), workloads.bf16_bits(F), b)
+    assert np.array_equal(y[0, 0, :, 0], [0, 1, 2]) and np.array_equal(y[0, 0, :, 1], [6, 9, 12])
+
+
+@pytest.mark.parametrize("case", [workloads.DENSE_GROUPED, workloads.CONV1D_STEM1, workloads.CONV1D_STEM2],
+                         ids=["grouped", "conv1d-stem1", "conv1d-stem2"])
+def test_full_size_workloads_sampled(cb, case):
+    # the benchmark's workloads at full size, checked on 20000 sampled outputs
+    Xb, Fb = workloads.dense_inputs(case)
+    b = workloads.dense_bias(case)
+    y, kernel = _run(cb, case, Xb, Fb, b)
+    assert kernel == "dense_tc_kernel"
+    idx = (workloads.splitmix64(6, 20000) % np.uint64(y.size)).astype(np.int64)
+    s, p, d = _geom(case)
+    ref, absum = oracle.conv2d_grouped_points(workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb), idx, b, s, p, d,
+                                              case.groups)
+    assert np.all(np.abs(y.reshape(-1)[idx] - ref) <= TOL * absum)
+    assert np.all(np.isfinite(y))
+

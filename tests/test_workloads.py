@@ -46,3 +46,13 @@ def test_workload_shapes():
     assert set(np.unique(X).tolist()) <= set(range(-3, 4))
     x, w, b = workloads.depthwise_inputs(workloads.DW_SWEEP[0])
     assert x.shape == (64, 16, 112, 112) and w.shape == (16, 3, 3) and b.shape == (16,)
+
+
+def test_grouped_and_conv1d_case_shapes():
+    c = workloads.DENSE_GROUPED
+    assert c.f_shape == (3, 3, 64, 256) and (c.Ho, c.Wo) == (28, 28) and not c.square
+    assert c.flops == 2 * 32 * 28 * 28 * 256 * 9 * 64
+    s1, s2 = workloads.CONV1D_STEM1, workloads.CONV1D_STEM2
+    assert s1.f_shape == (1, 3, 80, 512) and (s1.Ho, s1.Wo) == (1, 3000)
+    assert s2.f_shape == (1, 3, 512, 512) and (s2.Ho, s2.Wo) == (1, 1500)
+    assert workloads.DENSE_S2.square and workloads.DENSE_S2.f_shape == (3, 3, 64, 128)

@@ -126,23 +126,62 @@ class DenseCase:
     pad: int = 0
     dil: int = 1
     bias: bool = False  # a float32 bias[Cout] ~ N(0, 0.1)
+    groups: int = 1     # channel groups: F is [KH, KW, Cin/groups, Cout]
+    KW: int = 0         # filter width when it differs from K (K is then the height)
+    stride_w: int = 0   # width-axis stride, padding, dilation when they differ (0 / -1: as the
+    pad_w: int = -1     # height axis)
+    dil_w: int = 0
+
+    @property
+    def kh(self) -> int:
+        return self.K
+
+    @property
+    def kw(self) -> int:
+        return self.KW or self.K
+
+    @property
+    def sw(self) -> int:
+        return self.stride_w or self.stride
+
+    @property
+    def pw(self) -> int:
+        return self.pad if self.pad_w < 0 else self.pad_w
+
+    @property
+    def dw(self) -> int:
+        return self.dil_w or self.dil
+
+    @property
+    def cin_g(self) -> int:
+        return self.Cin // self.groups
+
+    @property
+    def square(self) -> bool:
+        """One K, one stride, padding and dilation for both axes, one group."""
+        return self.kw == self.K and self.sw == self.stride and self.pw == self.pad and self.dw == self.dil and \
+            self.groups == 1
+
+    @property
+    def f_shape(self):
+        return (self.kh, self.kw, self.cin_g, self.Cout)
 
     @property
     def Ho(self) -> int:
-        return (self.H + 2 * self.pad - (self.dil * (self.K - 1) + 1)) // self.stride + 1
+        return (self.H + 2 * self.pad - (self.dil * (self.kh - 1) + 1)) // self.stride + 1
 
     @property
     def Wo(self) -> int:
-        return (self.W + 2 * self.pad - (self.dil * (self.K - 1) + 1)) // self.stride + 1
+        return (self.W + 2 * self.pw - (self.dw * (self.kw - 1) + 1)) // self.sw + 1
 
     @property
     def flops(self) -> int:
-        return 2 * self.N * self.Ho * self.Wo * self.Cout * self.K * self.K * self.Cin
+        return 2 * self.N * self.Ho * self.Wo * self.Cout * self.kh * self.kw * self.cin_g
 
     @property
     def bytes(self) -> int:
         e = 2 if self.dtype == "bf16" else 4
-        return e * (self.N * self.H * self.W * self.Cin + self.K * self.K * self.Cin * self.Cout
+        return e * (self.N * self.H * self.W * self.Cin + self.kh * self.kw * self.cin_g * self.Cout
                     + self.N * self.Ho * self.Wo * self.Cout) + (4 * self.Cout if self.bias else 0)
 
 
@@ -192,6 +231,16 @@ DENSE_LARGE = DenseCase("large dense bf16 N64 H112 W112 Cin128 Cout128 K5", 64, 
 # stride-2 3x3 layer with "same" padding and a bias (a ResNet stage transition, 56 -> 28)
 DENSE_S2 = DenseCase("dense bf16 N32 H56 W56 Cin64 Cout128 K3 s2 p1 bias", 32, 56, 56, 64, 128, 3, "bf16", "normal", 0,
                      stride=2, pad=1, bias=True)
+# grouped 3x3 layer, 4 groups of 64 channels (a RegNet-style group width) with a bias
+DENSE_GROUPED = DenseCase("grouped bf16 N32 H28 W28 Cin256 Cout256 K3 p1 g4 bias", 32, 28, 28, 256, 256, 3, "bf16",
+                          "normal", 0, pad=1, bias=True, groups=4)
+# Conv1D audio stem over 3000 log-mel frames (30 s at 10 ms), batch 16, width 512: the first
+# layer mixes nearby frames (80 -> 512, K 3, pad 1), the second halves the frame rate
+# (512 -> 512, K 3, stride 2, pad 1); both with a bias. A sequence is one image row (H = 1).
+CONV1D_STEM1 = DenseCase("conv1d bf16 N16 L3000 Cin80 Cout512 K3 p1 bias", 16, 1, 3000, 80, 512, 1, "bf16", "normal",
+                         0, bias=True, KW=3, pad_w=1)
+CONV1D_STEM2 = DenseCase("conv1d bf16 N16 L3000 Cin512 Cout512 K3 s2 p1 bias", 16, 1, 3000, 512, 512, 1, "bf16",
+                         "normal", 0, bias=True, KW=3, stride_w=2, pad_w=1)
 # MobileNetV3-large depthwise layers (C, K, stride, input H=W), batch 64, multiplier 1,
 # pad (K-1)/2, dilation 1.
 DW_LAYERS = [(16, 3, 1, 112), (64, 3, 2, 112), (72, 5, 2, 56), (120, 5, 1, 28), (672, 3, 1, 14),
@@ -208,23 +257,23 @@ def dense_bias(case: DenseCase):
 
 
 def dense_inputs(case: DenseCase):
-    """Seeded X (NHWC) and F (KKIO).
+    """Seeded X (NHWC) and F (KKIO; [KH, KW, Cin/groups, Cout] for a grouped case).
 
     Returns (X, F) as uint16 bf16 bit patterns for bf16 cases, float32 arrays otherwise.
     """
     nx = case.N * case.H * case.W * case.Cin
-    nf = case.K * case.K * case.Cin * case.Cout
+    nf = case.kh * case.kw * case.cin_g * case.Cout
     sx, sf = stream_seed(case.seed, 0), stream_seed(case.seed, 1)
     if case.dist == "int3":
         X = int_uniform(sx, nx, -3, 3)
         F = int_uniform(sf, nf, -3, 3)
     elif case.dist == "normal":
         X = normal(sx, nx, 1.0)
-        F = normal(sf, nf, 1.0 / math.sqrt(case.K * case.K * case.Cin))
+        F = normal(sf, nf, 1.0 / math.sqrt(case.kh * case.kw * case.cin_g))
     else:
         raise ValueError(case.dist)
     X = X.reshape(case.N, case.H, case.W, case.Cin)
-    F = F.reshape(case.K, case.K, case.Cin, case.Cout)
+    F = F.reshape(case.f_shape)
     if case.dtype == "bf16":
         return bf16_bits(X), bf16_bits(F)
     return X, F
