@@ -58,6 +58,9 @@ def workload_table():
          "conv1d-stem2": ("dense", workloads.CONV1D_STEM2, None),
          # comparison path: explicit patch matrix + one cuBLAS GEMM, packing inside the timing
          "dense3x3-explicit-im2col": ("dense", workloads.DENSE_3X3, "im2col")}
+    for c in workloads.DWPW_BLOCKS:
+        for mode, name in ((0, "exact"), (1, "fast")):
+            t[f"dwpw-C{c.C}-K{c.K}-H{c.H}-Cout{c.Cout}-{name}"] = ("dwpw", c, mode)
     for c in workloads.DW_SWEEP:
         for mode, name in ((0, "exact"), (1, "fast")):
             t[f"dw-C{c.C}-K{c.KH}-s{c.stride}-H{c.H}-{name}"] = ("depthwise", c, mode)
@@ -84,6 +87,7 @@ KERNEL_SOURCES = {
     "depthwise_tma_kernel": ("depthwise_tma.cuh", "depthwise.cuh", "ptx.cuh"),
     "depthwise_reg_kernel": ("depthwise_reg.cuh", "depthwise.cuh"),
     "depthwise_kernel": ("depthwise.cuh",),
+    "dwpw_kernel": ("dwpw.cuh", "dense_tc.cuh", "depthwise.cuh", "ptx.cuh"),
 }
 
 
@@ -333,6 +337,36 @@ def dw_device_inputs(torch, case, seed):
     return x, w, b
 
 
+def dwpw_device_inputs(torch, case, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    x = torch.rand((case.N, case.C, case.H, case.W), device="cuda", generator=g) * 2 - 1
+    w = torch.randn((case.C, case.K, case.K), device="cuda", generator=g) / case.K
+    F = (torch.randn((case.C, case.Cout), device="cuda", generator=g) / math.sqrt(case.C)).to(torch.bfloat16)
+    bd = torch.randn((case.C,), device="cuda", generator=g) * math.sqrt(0.1) if case.bias else None
+    bp = torch.randn((case.Cout,), device="cuda", generator=g) * math.sqrt(0.1) if case.bias else None
+    return x, w, bd, F, bp
+
+
+def device_inputs(torch, kind, case, seed):
+    if kind == "dense":
+        return dense_device_inputs(torch, case, seed)
+    if kind == "dwpw":
+        return dwpw_device_inputs(torch, case, seed)
+    return dw_device_inputs(torch, case, seed)
+
+
+def out_shape(kind, case):
+    if kind == "dense":
+        return (case.N, case.Ho, case.Wo, case.Cout)
+    if kind == "dwpw":
+        return (case.N, case.Cout, case.Ho, case.Wo)
+    return (case.N, case.C * case.mult, case.Ho, case.Wo)
+
+
+def dwpw_call(cb, case, x, w, bd, F, bp, y, mode):
+    return cb.dwpw_fwd(x, w, bd, F, bp, y, case.stride, case.pad, case.dil, mode)
+
+
 def steps_fns(cb, torch, kind, case, mode, inputs):
     """R rotating buffer sets (total at least twice the L2) and one C-ABI call per set."""
     R = rotating_sets(case.bytes)
@@ -345,6 +379,12 @@ def steps_fns(cb, torch, kind, case, mode, inputs):
         ws = im2col_workspace(cb, torch, case, mode)
         fns = [(lambda i=i: dense_call(cb, case, Xs[i], Fs[i], b0, Ys[i], mode, ws)) for i in range(R)]
         keep = (Xs, Fs, Ys, b0, ws)
+    elif kind == "dwpw":
+        x0, w0, bd0, F0, bp0 = inputs
+        xs = [x0.clone() for _ in range(R)]
+        ys = [torch.empty(out_shape(kind, case), device=x0.device) for _ in range(R)]
+        fns = [(lambda i=i: dwpw_call(cb, case, xs[i], w0, bd0, F0, bp0, ys[i], mode)) for i in range(R)]
+        keep = (xs, ys)
     else:
         x0, w0, b0 = inputs
         xs = [x0.clone() for _ in range(R)]
@@ -368,9 +408,9 @@ def e2e_bench(cb, torch, kind, case, mode, host, steps, warmup):
     """Public API end to end: pinned host inputs -> device, convolution, output -> pinned host."""
     dev = [torch.empty(h.shape, dtype=h.dtype, device="cuda") if h is not None else None for h in host]
     if kind == "dense":
-        out = torch.empty((case.N, case.Ho, case.Wo, case.Cout), dtype=host[0].dtype, device="cuda")
+        out = torch.empty(out_shape(kind, case), dtype=host[0].dtype, device="cuda")
     else:
-        out = torch.empty((case.N, case.C * case.mult, case.Ho, case.Wo), device="cuda")
+        out = torch.empty(out_shape(kind, case), device="cuda")
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     ws = im2col_workspace(cb, torch, case, mode) if kind == "dense" else None
 
@@ -380,6 +420,8 @@ def e2e_bench(cb, torch, kind, case, mode, host, steps, warmup):
                 d.copy_(h, non_blocking=True)
         if kind == "dense":
             dense_call(cb, case, dev[0], dev[1], dev[2], out, mode, ws)
+        elif kind == "dwpw":
+            dwpw_call(cb, case, dev[0], dev[1], dev[2], dev[3], dev[4], out, mode)
         else:
             cb.depthwise_fwd(dev[0], dev[1], dev[2], out, case.stride, case.pad, case.dil, mode)
         out_h.copy_(out, non_blocking=True)
@@ -413,6 +455,10 @@ def cpu_baseline(kind, case, mode, host_np, budget_s=10.0):
             X, F, b = host_np
             oracle_dense(oracle, case, X[i:i + 1], F, b)
             done += case.flops / case.N
+        elif kind == "dwpw":
+            x, w, bd, F, bp = host_np
+            oracle.dwpw(x[i:i + 1], w, bd, F, bp, case.stride, case.pad, case.dil, mode)
+            done += case.bytes / case.N
         else:
             x, w, b = host_np
             oracle.depthwise(x[i:i + 1], w, b, mult=case.mult, stride=case.stride, pad=case.pad, dil=case.dil,
@@ -422,7 +468,12 @@ def cpu_baseline(kind, case, mode, host_np, budget_s=10.0):
     dt = time.perf_counter() - t0
     unit = "TFLOP/s" if kind == "dense" else "GB/s"
     scale = 1e12 if kind == "dense" else 1e9
-    what = "float64 seven-loop oracle" if kind == "dense" else f"float32 per-output oracle, {'exact' if mode == 0 else 'fast'} mode"
+    if kind == "dense":
+        what = "float64 seven-loop oracle"
+    elif kind == "dwpw":
+        what = f"float32 depthwise oracle ({'exact' if mode == 0 else 'fast'} mode) + float64 pointwise"
+    else:
+        what = f"float32 per-output oracle, {'exact' if mode == 0 else 'fast'} mode"
     return {"value": done / dt / scale, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{n} single-image calls cycling over the {case.N} images of the workload, {what}, {dt:.1f} s"}
 
@@ -436,6 +487,13 @@ def host_inputs(torch, kind, case, seed):
         host = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (Xb, Fb)]
         host.append(None if b is None else torch.from_numpy(b).pin_memory())
         return (workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb), b), host
+    if kind == "dwpw":
+        x, w, bd, F, bp = workloads.dwpw_inputs(dataclasses.replace(case, seed=seed))
+        host = [torch.from_numpy(x).pin_memory(), torch.from_numpy(w).pin_memory(),
+                None if bd is None else torch.from_numpy(bd).pin_memory(),
+                torch.from_numpy(F.view(np.int16)).view(torch.bfloat16).pin_memory(),
+                None if bp is None else torch.from_numpy(bp).pin_memory()]
+        return (x, w, bd, workloads.bf16_to_f32(F), bp), host
     c = workloads.DepthwiseCase(case.name, case.N, case.C, case.mult, case.H, case.W, case.KH, case.KW, case.stride,
                                 case.pad, case.dil, case.bias, seed)
     x, w, b = workloads.depthwise_inputs(c)
@@ -490,9 +548,17 @@ def run_ours(args, dist):
                 "peak_source": f"{peaks_src}: HBM copy"}
         dtype = "f32"
         data = "synthetic (seeded SplitMix64 / Box-Muller: x~U(-1,1), w~N(0,1/K^2), bias~N(0,0.1))"
-        cfg = {"workload": case.name + (" exact" if mode == 0 else " fast"), "N_per_gpu": case.N, "C": case.C,
-               "mult": case.mult, "H": case.H, "W": case.W, "K": case.KH, "stride": case.stride, "pad": case.pad,
-               "dil": case.dil, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
+        if kind == "dwpw":
+            data = ("synthetic (seeded SplitMix64 / Box-Muller: x~U(-1,1), w~N(0,1/K^2), F~N(0,1/C) rounded to bf16, "
+                    "biases~N(0,0.1))")
+            cfg = {"workload": case.name + (" exact" if mode == 0 else " fast"), "N_per_gpu": case.N, "C": case.C,
+                   "H": case.H, "W": case.W, "K": case.K, "stride": case.stride, "pad": case.pad, "dil": case.dil,
+                   "Cout": case.Cout, "flop_per_step": case.flops, "bytes_per_step": case.bytes,
+                   "intermediate": "depthwise output rounded to bf16 in shared memory, never in HBM"}
+        else:
+            cfg = {"workload": case.name + (" exact" if mode == 0 else " fast"), "N_per_gpu": case.N, "C": case.C,
+                   "mult": case.mult, "H": case.H, "W": case.W, "K": case.KH, "stride": case.stride,
+                   "pad": case.pad, "dil": case.dil, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
     cfg.update({"l2": f"inputs larger than L2: {R} rotating buffer sets of {case.bytes / 1e6:.2f} MB",
                 "launch": "CUDA graph replay of the C-ABI call", "parallelism": f"replicas x{dist.world}"})
     value = dist.world * work * args.steps / (ms * 1e-3) / scale
@@ -517,7 +583,7 @@ def run_ours(args, dist):
 
 
 def extras(cb, torch, peaks, skip):
-    out = {"dense": [], "depthwise": []}
+    out = {"dense": [], "depthwise": [], "dwpw": []}
     for name, (kind, case, mode) in workload_table().items():
         if name == skip:
             continue
@@ -532,10 +598,10 @@ def extras(cb, torch, peaks, skip):
                                  "frac_hbm": round(case.bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                                  "rotating_sets": R})
         else:
-            ms, R, kernel = time_case(cb, torch, kind, case, mode, dw_device_inputs(torch, case, 0), 200, 20)
+            ms, R, kernel = time_case(cb, torch, kind, case, mode, device_inputs(torch, kind, case, 0), 200, 20)
             ms /= 200
             gbs = case.bytes / (ms * 1e-3) / 1e9
-            out["depthwise"].append({"workload": name, "kernel": kernel, "ms": round(ms, 5), "GB/s": round(gbs, 1),
+            out["depthwise" if kind == "depthwise" else "dwpw"].append({"workload": name, "kernel": kernel, "ms": round(ms, 5), "GB/s": round(gbs, 1),
                                      "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
                                      "GFLOP/s": round(case.flops / (ms * 1e-3) / 1e9, 1), "rotating_sets": R})
     return out
@@ -562,6 +628,14 @@ def run_reference(args, dist):
             else:
                 oracle.conv2d_grouped_points(X, F, idx, b, (case.stride, case.sw), (case.pad, case.pw),
                                              (case.dil, case.dw), case.groups)
+    elif kind == "dwpw":
+        x, w, bd, Fb, bp = workloads.dwpw_inputs(case)
+        F = workloads.bf16_to_f32(Fb)
+        total = case.N * case.Cout * case.Ho * case.Wo
+        work_per_out, unit, scale = case.bytes / total, "GB/s", 1e9
+
+        def run(idx):
+            oracle.dwpw_points(x, w, bd, F, bp, idx, case.stride, case.pad, case.dil, mode)
     else:
         x, w, b = workloads.depthwise_inputs(case)
         total = case.N * case.C * case.mult * case.Ho * case.Wo

@@ -43,6 +43,8 @@ lib.conv2d_nhwc_im2col_workspace.argtypes = [_I] * 5
 lib.conv2d_nhwc_im2col_workspace.restype = ctypes.c_size_t
 lib.conv2d_nhwc_fwd_im2col.argtypes = [_P, _P, _P, _P, ctypes.c_size_t] + [_I] * 6 + [_P]
 lib.conv2d_nhwc_fwd_im2col.restype = _I
+lib.dwpw_fwd.argtypes = [_P] * 6 + [_I] * 10 + [_P]
+lib.dwpw_fwd.restype = _I
 lib.depthwise_fwd.argtypes = [_P, _P, _P, _P] + [_I] * 11 + [_P]
 lib.depthwise_fwd.restype = _I
 lib.conv_status_string.argtypes = [_I]
@@ -55,7 +57,7 @@ lib.conv_selftest_wait_timeout.argtypes = [_P]
 lib.conv_selftest_wait_timeout.restype = _I
 
 EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "conv2d_nhwc_fwd_grouped",
-           "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "depthwise_fwd", "conv_status_string",
+           "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "dwpw_fwd", "depthwise_fwd", "conv_status_string",
            "conv_device_status", "conv_last_kernel", "conv_selftest_wait_timeout")
 
 
@@ -249,6 +251,44 @@ def depthwise_fwd(x, w, bias=None, y=None, stride=1, pad=0, dil=1, mode=DW_EXACT
     py = _tensor(y, torch.float32, 4, "y")
     _check(lib.depthwise_fwd(px, pw, pb, py, N, Cin, mult, H, W, KH, KW, stride, pad, dil, int(mode),
                              _stream(stream)), "depthwise_fwd")
+    return y
+
+
+def dwpw_fwd(x, w_dw, b_dw, F, b_pw=None, y=None, stride=1, pad=0, dil=1, mode=DW_EXACT, stream=None):
+    """Depthwise then pointwise, fused: x float32 [N,C,H,W], w_dw float32 [C,K,K], b_dw float32
+    [C] or None, F bfloat16 [C,Cout], b_pw float32 [Cout] or None -> y float32 [N,Cout,Ho,Wo]."""
+    import torch
+    px = _tensor(x, torch.float32, 4, "x")
+    pw = _tensor(w_dw, torch.float32, 3, "w_dw")
+    pf = _tensor(F, torch.bfloat16, 2, "F")
+    N, C, H, W = x.shape
+    C2, K, K2 = w_dw.shape
+    if C2 != C or K != K2:
+        raise ValueError("w_dw must be [C, K, K]")
+    C3, Cout = F.shape
+    if C3 != C:
+        raise ValueError("F must be [C, Cout]")
+    pbd = ctypes.c_void_p(None)
+    if b_dw is not None:
+        pbd = _tensor(b_dw, torch.float32, 1, "b_dw")
+        if b_dw.shape[0] != C:
+            raise ValueError("b_dw must have C entries")
+    pbp = ctypes.c_void_p(None)
+    if b_pw is not None:
+        pbp = _tensor(b_pw, torch.float32, 1, "b_pw")
+        if b_pw.shape[0] != Cout:
+            raise ValueError("b_pw must have Cout entries")
+    Ho = (H + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    Wo = (W + 2 * pad - (dil * (K - 1) + 1)) // stride + 1
+    if Ho < 1 or Wo < 1:
+        raise ValueError("empty output")
+    if y is None:
+        y = torch.empty((N, Cout, Ho, Wo), dtype=torch.float32, device=x.device)
+    elif tuple(y.shape) != (N, Cout, Ho, Wo):
+        raise ValueError("y has the wrong shape")
+    py = _tensor(y, torch.float32, 4, "y")
+    _check(lib.dwpw_fwd(px, pw, pbd, pf, pbp, py, N, C, H, W, K, stride, pad, dil, Cout, int(mode), _stream(stream)),
+           "dwpw_fwd")
     return y
 
 

@@ -25,6 +25,7 @@
 #include "depthwise_reg.cuh"
 #include "depthwise_tma.cuh"
 #include "depthwise_plane.cuh"
+#include "dwpw.cuh"
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -886,6 +887,22 @@ int launch_dw(const float *x, const float *w, const float *bias, float *y, const
     }
 }
 
+// ---- fused depthwise -> pointwise -------------------------------------------------------
+// shared-memory attribute bits 51..56: MODE x (K 3, K 5, other K)
+template <int MODE, int KC>
+int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y, const DwPwParams &p,
+                cudaStream_t stream, DeviceState *d, unsigned bit) {
+    auto kern = dwpw_kernel<MODE, KC>;
+    if (int rc = ensure_smem_attr(d, bit, kern, kDwPwSmem)) return rc;
+    const int grid = p.num_tiles < 2 * d->num_sms ? p.num_tiles : 2 * d->num_sms;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kDwPwThreads);
+    cfg.dynamicSmemBytes = kDwPwSmem;
+    cfg.stream = stream;
+    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_kernel");
+}
+
 }  // namespace
 }  // namespace convb200
 
@@ -1240,6 +1257,70 @@ int conv_device_status(cudaStream_t stream, int reset) {
         if (cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return CONV_ERR_CUDA;
     }
     return (v & kStatusTimeout) ? CONV_ERR_DEVICE_TIMEOUT : CONV_OK;
+}
+
+int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F, const float *b_pw, float *y, int N,
+             int C, int H, int W, int K, int stride, int pad, int dil, int Cout, int mode, cudaStream_t stream) {
+    if (!x || !w_dw || !F || !y) return CONV_ERR_INVALID_ARG;
+    if (N < 1 || C < 1 || H < 1 || W < 1 || K < 1 || stride < 1 || dil < 1 || pad < 0 || Cout < 1)
+        return CONV_ERR_INVALID_ARG;
+    if (mode != DW_EXACT && mode != DW_FAST) return CONV_ERR_INVALID_ARG;
+    if (1LL * H + 2LL * pad > kInt32Max / 2 || 1LL * W + 2LL * pad > kInt32Max / 2 ||
+        1LL * dil * (K - 1) > kInt32Max / 2)
+        return CONV_ERR_UNSUPPORTED;
+    if (1LL * H + 2LL * pad < 1LL * dil * (K - 1) + 1 || 1LL * W + 2LL * pad < 1LL * dil * (K - 1) + 1)
+        return CONV_ERR_INVALID_ARG;
+    const long long Ho = dw_out(H, K, stride, pad, dil), Wo = dw_out(W, K, stride, pad, dil);
+    const long long nx = 1LL * N * C * H * W, nw = 1LL * C * K * K, nf = 1LL * C * Cout, ny = 1LL * N * Cout * Ho * Wo;
+    if (nx > kInt32Max || nw > kInt32Max || nf > kInt32Max || ny > kInt32Max || 1LL * N * Ho * Wo > kInt32Max - 128 ||
+        1LL * K * K > 4096)
+        return CONV_ERR_UNSUPPORTED;
+    // the pointwise stage runs on the tensor cores: whole 16-byte filter rows, one MMA width
+    if (Cout % 8 != 0 || Cout > 256) return CONV_ERR_UNSUPPORTED;
+    if (!aligned(F, 16) || !aligned(x, 4) || !aligned(w_dw, 4) || !aligned(y, 4) || (b_dw && !aligned(b_dw, 4)) ||
+        (b_pw && !aligned(b_pw, 4)))
+        return CONV_ERR_MISALIGNED;
+    if (overlaps(y, ny * 4, x, nx * 4) || overlaps(y, ny * 4, w_dw, nw * 4) || overlaps(y, ny * 4, F, nf * 2) ||
+        (b_dw && overlaps(y, ny * 4, b_dw, 4LL * C)) || (b_pw && overlaps(y, ny * 4, b_pw, 4LL * Cout)))
+        return CONV_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    alignas(64) CUtensorMap tmF;
+    {   // F: 3-D {Cout, C, 1}; a box is 64 channel rows x 64 outputs (rows past C and columns
+        // past Cout read zeros)
+        const cuuint64_t dims[3] = {(cuuint64_t)Cout, (cuuint64_t)C, 1};
+        const cuuint64_t strides[2] = {(cuuint64_t)Cout * 2, (cuuint64_t)C * Cout * 2};
+        const cuuint32_t box[3] = {64, 64, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(F), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    DwPwParams p;
+    p.C = C; p.H = H; p.W = W; p.Ho = static_cast<int>(Ho); p.Wo = static_cast<int>(Wo); p.HoWo = p.Ho * p.Wo;
+    p.K = K; p.stride = stride; p.pad = pad; p.dil = dil;
+    p.Cout = Cout;
+    p.n_mma = (Cout + 15) / 16 * 16;
+    p.n_boxes = (Cout + 63) / 64;
+    p.num_kblk = (C + 63) / 64;
+    p.M = static_cast<int>(1LL * N * Ho * Wo);
+    p.num_tiles = (p.M + 127) / 128;
+    p.idesc = idesc_bf16_f32(128, p.n_mma, /*B MN-major*/ true);
+    p.tmem_cols = 32;
+    while (p.tmem_cols < static_cast<uint32_t>(p.n_mma)) p.tmem_cols <<= 1;
+    p.b_dw = b_dw;
+    p.b_pw = b_pw;
+    p.div_howo = make_fastdiv(static_cast<uint32_t>(p.HoWo));
+    p.div_wo = make_fastdiv(static_cast<uint32_t>(p.Wo));
+    if (mode == DW_EXACT) {
+        if (K == 3) return launch_dwpw<0, 3>(x, w_dw, tmF, y, p, stream, d, 51);
+        if (K == 5) return launch_dwpw<0, 5>(x, w_dw, tmF, y, p, stream, d, 52);
+        return launch_dwpw<0, 0>(x, w_dw, tmF, y, p, stream, d, 53);
+    }
+    if (K == 3) return launch_dwpw<1, 3>(x, w_dw, tmF, y, p, stream, d, 54);
+    if (K == 5) return launch_dwpw<1, 5>(x, w_dw, tmF, y, p, stream, d, 55);
+    return launch_dwpw<1, 0>(x, w_dw, tmF, y, p, stream, d, 56);
 }
 
 }  // extern "C"

@@ -23,6 +23,11 @@
  *     Moving Across a Signal", section "Build an image-gradient map, one number at a time":
  *         out = floor((in + 2*pad - (dil*(k-1) + 1)) / stride) + 1.
  *
+ * Around them: the dense operation with stride, padding, dilation and bias (conv2d_nhwc_fwd_ex),
+ * with channel groups, KH x KW filters and per-axis geometry, Conv1D included
+ * (conv2d_nhwc_fwd_grouped), a depthwise pass fused with the pointwise pass after it (dwpw_fwd),
+ * and an explicit-im2col comparison path (conv2d_nhwc_fwd_im2col).
+ *
  * Common rules for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller (for example allocated by
  *    PyTorch). Tensors are dense and contiguous in the stated layout. The library keeps no
@@ -164,6 +169,26 @@ int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspac
 int depthwise_fwd(const float *x, const float *w, const float *bias, float *y,
                   int N, int Cin, int mult, int H, int W, int KH, int KW,
                   int stride, int pad, int dil, int mode, cudaStream_t stream);
+
+/*
+ * A depthwise K x K pass followed by a pointwise 1 x 1 pass, fused in one kernel: the block of
+ * "Convolution Is Wx+b Moving Across a Signal", section "Why variants matter" (a depthwise filter
+ * per channel, then a channel-mixing 1 x 1 layer). The intermediate never goes to memory.
+ *     d[n,c,oy,ox] = depthwise_fwd's output for multiplier 1 (same order, mode and bias rule),
+ *     y[n,o,oy,ox] = b_pw[o] + sum_c bf16(d[n,c,oy,ox]) * F[c,o],
+ * with bf16() rounding to nearest even (the tensor cores' operand type), the sum accumulated in
+ * float32 and b_pw added once in float32.
+ *   x    : float32 [N][C][H][W]
+ *   w_dw : float32 [C][K][K];  b_dw : float32 [C] or NULL
+ *   F    : bfloat16 [C][Cout], 16-byte aligned;  b_pw : float32 [Cout] or NULL
+ *   y    : float32 [N][Cout][Ho][Wo], Ho/Wo as depthwise_fwd (stride, pad, dil on both axes)
+ * Requirements: N, C, H, W, K, stride, dil, Cout >= 1; pad >= 0; Ho, Wo >= 1; mode DW_EXACT or
+ * DW_FAST; x, w_dw, y, biases 4-byte aligned; element counts below 2^31. Cout must be a multiple
+ * of 8 and at most 256 (one tensor-core tile width); other Cout return CONV_ERR_UNSUPPORTED.
+ */
+int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F, const float *b_pw, float *y,
+             int N, int C, int H, int W, int K, int stride, int pad, int dil, int Cout, int mode,
+             cudaStream_t stream);
 
 /* Static English text for a conv_status value (never NULL). */
 const char *conv_status_string(int status);

@@ -181,3 +181,21 @@ WS = V(1 << 32)
 ])
 def test_im2col_path_rejects(ws, nbytes, code):
     assert cb.lib.conv2d_nhwc_fwd_im2col(X, F, Y, ws, nbytes, 1, 5, 5, 8, 8, 3, None) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    # x, w_dw, b_dw, F, b_pw, y, N, C, H, W, K, stride, pad, dil, Cout, mode
+    ((None, B, None, F, None, Y, 1, 8, 9, 9, 3, 1, 1, 1, 16, 0), cb.CONV_ERR_INVALID_ARG),
+    ((X, B, None, None, None, Y, 1, 8, 9, 9, 3, 1, 1, 1, 16, 0), cb.CONV_ERR_INVALID_ARG),
+    ((X, B, None, F, None, Y, 1, 8, 9, 9, 3, 1, 1, 1, 16, 2), cb.CONV_ERR_INVALID_ARG),       # mode 2
+    ((X, B, None, F, None, Y, 1, 8, 9, 9, 3, 0, 1, 1, 16, 0), cb.CONV_ERR_INVALID_ARG),       # stride 0
+    ((X, B, None, F, None, Y, 1, 8, 2, 2, 5, 1, 1, 1, 16, 0), cb.CONV_ERR_INVALID_ARG),       # window > image
+    ((X, B, None, F, None, Y, 1, 8, 9, 9, 3, 1, 1, 1, 12, 0), cb.CONV_ERR_UNSUPPORTED),       # Cout % 8
+    ((X, B, None, F, None, Y, 1, 8, 9, 9, 3, 1, 1, 1, 264, 0), cb.CONV_ERR_UNSUPPORTED),      # Cout > 256
+    ((X, B, None, V((1 << 22) + 8), None, Y, 1, 8, 9, 9, 3, 1, 1, 1, 16, 0), cb.CONV_ERR_MISALIGNED),  # F
+    ((V((1 << 20) + 2), B, None, F, None, Y, 1, 8, 9, 9, 3, 1, 1, 1, 16, 0), cb.CONV_ERR_MISALIGNED),
+    ((X, B, None, F, None, V(1 << 20), 1, 8, 9, 9, 3, 1, 1, 1, 16, 0), cb.CONV_ERR_INVALID_ARG),       # y on x
+    ((X, B, None, F, None, Y, 4096, 64, 4096, 4096, 3, 1, 1, 1, 16, 0), cb.CONV_ERR_UNSUPPORTED),
+])
+def test_dwpw_rejects(args, code):
+    assert cb.lib.dwpw_fwd(*args, None) == code

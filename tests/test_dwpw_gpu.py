@@ -1,0 +1,108 @@
+"""GPU parity of dwpw_fwd (depthwise then pointwise, fused) against the oracle.
+
+The depthwise stage is the page's bit-exact contract, so both sides round the same float32
+intermediate to bf16 and differ only in how the pointwise sum is accumulated: every product
+a*F of two bf16 values is exact in float32, and a float32 sum of C + 1 terms in any order, with
+any rounding mode, is within (C + 2) * 2^-23 of the absolute sum. That is the bar per output.
+Where the mixing matrix is the identity, the block must reproduce the rounded depthwise output
+bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cb(cuda):
+    import cnn_convolution_nhwc_b200 as cb
+    return cb
+
+
+def _dev(a, bf16=False):
+    if a is None:
+        return None
+    if bf16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+def _run(cb, case, x, w, bd, F, bp, mode):
+    y = cb.dwpw_fwd(_dev(x), _dev(w), _dev(bd), _dev(F, bf16=True), _dev(bp), stride=case.stride, pad=case.pad,
+                    dil=case.dil, mode=mode)
+    kernel = cb.conv_last_kernel()
+    out = y.cpu().numpy().astype(np.float64)
+    assert cb.conv_device_status() == cb.CONV_OK
+    return out, kernel
+
+
+def _tol(C):
+    return (C + 2) * 2.0 ** -23
+
+
+# (N, C, H, K, stride, pad, dil, Cout, mode, biases)
+CASES = [
+    (2, 64, 14, 3, 1, 1, 1, 64, 0, True),       # one channel block
+    (4, 72, 28, 5, 2, 2, 1, 40, 0, True),       # ragged channel block, N = 48 MMA
+    (2, 120, 28, 5, 1, 2, 1, 40, 1, False),     # fast mode, no biases
+    (8, 672, 14, 3, 1, 1, 1, 112, 0, True),     # 10.5 channel blocks, tiles across images
+    (4, 960, 7, 5, 1, 2, 1, 160, 1, True),      # three filter boxes, 49-pixel images
+    (2, 16, 30, 3, 1, 1, 1, 16, 0, True),       # 16 channels into 16 outputs
+    (1, 8, 9, 7, 1, 3, 1, 256, 0, True),        # 7x7 (runtime filter size), 256 outputs
+    (3, 24, 11, 3, 2, 1, 2, 24, 1, True),       # stride 2 with dilation 2, N = 32 MMA
+    (2, 40, 12, 3, 1, 0, 1, 8, 0, True),        # no padding, 8 outputs
+]
+
+
+def _ids(c):
+    return "N{}C{}H{}K{}s{}p{}d{}-O{}-{}".format(*c[:8], "exact" if c[8] == 0 else "fast") + ("b" if c[9] else "")
+
+
+@pytest.mark.parametrize("c", CASES, ids=_ids)
+def test_block_matches_oracle(cb, c):
+    N, C, H, K, s, p, d, Cout, mode, bias = c
+    case = workloads.DwPwCase("t", N, C, H, H, K, s, p, d, Cout, bias, seed=C + K + Cout)
+    x, w, bd, F, bp = workloads.dwpw_inputs(case)
+    y, kernel = _run(cb, case, x, w, bd, F, bp, mode)
+    assert kernel == "dwpw_kernel"
+    ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, s, p, d, mode)
+    assert y.shape == ref.shape
+    assert np.all(np.isfinite(y))
+    bad = np.abs(y - ref) > _tol(C) * absum
+    assert not bad.any(), f"{bad.sum()} outputs out of tolerance"
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_identity_mixing_is_the_rounded_depthwise_output(cb, mode):
+    # F = I: every output is one exact product plus zeros, so the block must equal the
+    # depthwise output rounded to bf16, bit for bit
+    case = workloads.DwPwCase("t", 3, 64, 20, 20, 3, 2, 1, 1, 64, True, seed=3)
+    x, w, bd, _, _ = workloads.dwpw_inputs(case)
+    F = workloads.bf16_bits(np.eye(64, dtype=np.float32))
+    y, _ = _run(cb, case, x, w, bd, F, None, mode)
+    dref = oracle.depthwise(x, w, bd, mult=1, stride=2, pad=1, dil=1, mode=mode)
+    assert np.array_equal(y, workloads.bf16_to_f32(workloads.bf16_bits(dref)).astype(np.float64))
+
+
+def test_unsupported_output_width_is_refused(cb):
+    case = workloads.DwPwCase("t", 1, 8, 9, 9, 3, 1, 1, 1, 12, False)
+    x, w, _, F, _ = workloads.dwpw_inputs(case)
+    with pytest.raises(cb.ConvError) as e:
+        _run(cb, case, x, w, None, F, None, 0)
+    assert e.value.code == cb.CONV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("case", workloads.DWPW_BLOCKS, ids=lambda c: c.name.replace(" ", "-"))
+def test_full_size_blocks_sampled(cb, case):
+    x, w, bd, F, bp = workloads.dwpw_inputs(case)
+    for mode in (0, 1):
+        y, kernel = _run(cb, case, x, w, bd, F, bp, mode)
+        assert kernel == "dwpw_kernel" and np.all(np.isfinite(y))
+        idx = (workloads.splitmix64(7 + mode, 20000) % np.uint64(y.size)).astype(np.int64)
+        ref, absum = oracle.dwpw_points(x, w, bd, workloads.bf16_to_f32(F), bp, idx, case.stride, case.pad, case.dil,
+                                        mode)
+        assert np.all(np.abs(y.reshape(-1)[idx] - ref) <= _tol(case.C) * absum)

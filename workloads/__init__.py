@@ -221,6 +221,56 @@ class DepthwiseCase:
                     + (co if self.bias else 0) + self.N * co * self.Ho * self.Wo)
 
 
+@dataclasses.dataclass(frozen=True)
+class DwPwCase:
+    """Depthwise K x K (multiplier 1) on NCHW float32 planes, then pointwise C -> Cout with
+    bfloat16 weights F[C][Cout]; y float32 NCHW [N][Cout][Ho][Wo]."""
+    name: str
+    N: int
+    C: int
+    H: int
+    W: int
+    K: int
+    stride: int
+    pad: int
+    dil: int
+    Cout: int
+    bias: bool = True   # both biases present
+    seed: int = 0
+
+    @property
+    def Ho(self) -> int:
+        return (self.H + 2 * self.pad - (self.dil * (self.K - 1) + 1)) // self.stride + 1
+
+    @property
+    def Wo(self) -> int:
+        return (self.W + 2 * self.pad - (self.dil * (self.K - 1) + 1)) // self.stride + 1
+
+    @property
+    def flops(self) -> int:
+        pix = self.N * self.Ho * self.Wo
+        return 2 * pix * self.C * self.K * self.K + 2 * pix * self.C * self.Cout
+
+    @property
+    def bytes(self) -> int:
+        b = 4 * (self.N * self.C * self.H * self.W + self.C * self.K * self.K + self.N * self.Cout * self.Ho * self.Wo)
+        b += 2 * self.C * self.Cout
+        if self.bias:
+            b += 4 * (self.C + self.Cout)
+        return b
+
+
+def dwpw_inputs(case: DwPwCase):
+    """Seeded x ~ U(-1, 1), w ~ N(0, 1/K^2), F ~ N(0, 1/C) as bf16 bits, biases ~ N(0, 0.1)."""
+    s = [stream_seed(case.seed, i) for i in range(5)]
+    x = uniform(s[0], case.N * case.C * case.H * case.W, -1.0, 1.0).reshape(case.N, case.C, case.H, case.W)
+    w = normal(s[1], case.C * case.K * case.K, 1.0 / case.K).reshape(case.C, case.K, case.K)
+    F = bf16_bits(normal(s[2], case.C * case.Cout, 1.0 / math.sqrt(case.C)).reshape(case.C, case.Cout))
+    bd = normal(s[3], case.C, math.sqrt(0.1)) if case.bias else None
+    bp = normal(s[4], case.Cout, math.sqrt(0.1)) if case.bias else None
+    return x, w, bd, F, bp
+
+
 DENSE_TINY = DenseCase("tiny dense fp32 N2 H8 W8 Cin4 Cout8 K3", 2, 8, 8, 4, 8, 3, "f32", "int3", 0)
 DENSE_3X3 = DenseCase("dense bf16 N32 H56 W56 Cin64 Cout64 K3", 32, 56, 56, 64, 64, 3, "bf16", "normal", 0)
 DENSE_1X1 = DenseCase("pointwise bf16 N32 H28 W28 Cin256 Cout512 K1", 32, 28, 28, 256, 512, 1, "bf16",
@@ -241,6 +291,10 @@ CONV1D_STEM1 = DenseCase("conv1d bf16 N16 L3000 Cin80 Cout512 K3 p1 bias", 16, 1
                          0, bias=True, KW=3, pad_w=1)
 CONV1D_STEM2 = DenseCase("conv1d bf16 N16 L3000 Cin512 Cout512 K3 s2 p1 bias", 16, 1, 3000, 512, 512, 1, "bf16",
                          "normal", 0, bias=True, KW=3, stride_w=2, pad_w=1)
+# depthwise then pointwise blocks (MobileNetV3-large shapes): 672 channels at 14x14, 3x3, into
+# 112 outputs; 960 channels at 7x7, 5x5, into 160 outputs; batch 64, both biases
+DWPW_BLOCKS = [DwPwCase("dwpw C672 K3 s1 H14 Cout112", 64, 672, 14, 14, 3, 1, 1, 1, 112),
+               DwPwCase("dwpw C960 K5 s1 H7 Cout160", 64, 960, 7, 7, 5, 1, 2, 1, 160)]
 # MobileNetV3-large depthwise layers (C, K, stride, input H=W), batch 64, multiplier 1,
 # pad (K-1)/2, dilation 1.
 DW_LAYERS = [(16, 3, 1, 112), (64, 3, 2, 112), (72, 5, 2, 56), (120, 5, 1, 28), (672, 3, 1, 14),
