@@ -893,13 +893,29 @@ template <int MODE, int KC>
 int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y, const DwPwParams &p,
                 cudaStream_t stream, DeviceState *d, unsigned bit) {
     auto kern = dwpw_kernel<MODE, KC>;
-    if (int rc = ensure_smem_attr(d, bit, kern, kDwPwSmem)) return rc;
-    const int grid = p.num_tiles < 2 * d->num_sms ? p.num_tiles : 2 * d->num_sms;
+    if (int rc = ensure_smem_attr(d, bit, kern, kDwPwMaxSmem)) return rc;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cudaLaunchAttribute attr[1];
     cfg.blockDim = dim3(kDwPwThreads);
-    cfg.dynamicSmemBytes = kDwPwSmem;
+    cfg.dynamicSmemBytes = kDwPwFixed + 4 * p.w_floats;
     cfg.stream = stream;
+    int clusters = p.num_tiles < d->num_sms ? p.num_tiles : d->num_sms;
+    if (p.S > 1) {
+        // clusters of S CTAs split a tile's channel blocks; as many clusters as fit at once
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(static_cast<unsigned>(p.S));
+        int active = 0;
+        if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active < 1) return CONV_ERR_CUDA;
+        if (clusters > active) clusters = active;
+        cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S));
+    } else {
+        cfg.gridDim = dim3(static_cast<unsigned>(clusters));
+    }
     return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_kernel");
 }
 
@@ -1313,13 +1329,43 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
     p.b_pw = b_pw;
     p.div_howo = make_fastdiv(static_cast<uint32_t>(p.HoWo));
     p.div_wo = make_fastdiv(static_cast<uint32_t>(p.Wo));
+    // Too few pixel tiles to fill the GPU: a cluster of S CTAs splits each tile's channel blocks
+    // and reduces the partial sums in a fixed rank order through distributed shared memory
+    // (S * owned chunks of 8 KB must fit the 96 KB stage area they reuse).
+    {
+        const int nch = p.n_mma / 16;
+        p.S = 1;
+        p.owned = nch;
+        if (2 * p.num_tiles <= d->num_sms) {
+            int S = d->num_sms / p.num_tiles;
+            if (S > 4) S = 4;
+            if (S > p.num_kblk) S = p.num_kblk;
+            while (S > 1 && S * ((nch + S - 1) / S) * kDwPwChunkBytes > kDwPwStages) --S;
+            if (S > 1) {
+                p.S = S;
+                p.owned = (nch + S - 1) / S;
+            }
+        }
+        const char *force = env("CONV_B200_DWPW_SPLIT");   // tests: force a split (1..4)
+        if (force) {
+            const int S = std::atoi(force);
+            if (S < 1 || S > 4 || S > p.num_kblk || S * ((nch + S - 1) / S) * kDwPwChunkBytes > kDwPwStages)
+                return CONV_ERR_UNSUPPORTED;
+            p.S = S;
+            p.owned = (nch + S - 1) / S;
+        }
+    }
+    // K = 3 and K = 5 stage the depthwise weights in shared memory when they fit; other filter
+    // sizes (or very many channels) read them from global memory
+    const bool staged = (K == 3 || K == 5) && 4LL * C * dwpw_kkp(K) <= kDwPwMaxSmem - kDwPwFixed;
+    p.w_floats = staged ? C * dwpw_kkp(K) : 0;
     if (mode == DW_EXACT) {
-        if (K == 3) return launch_dwpw<0, 3>(x, w_dw, tmF, y, p, stream, d, 51);
-        if (K == 5) return launch_dwpw<0, 5>(x, w_dw, tmF, y, p, stream, d, 52);
+        if (staged && K == 3) return launch_dwpw<0, 3>(x, w_dw, tmF, y, p, stream, d, 51);
+        if (staged && K == 5) return launch_dwpw<0, 5>(x, w_dw, tmF, y, p, stream, d, 52);
         return launch_dwpw<0, 0>(x, w_dw, tmF, y, p, stream, d, 53);
     }
-    if (K == 3) return launch_dwpw<1, 3>(x, w_dw, tmF, y, p, stream, d, 54);
-    if (K == 5) return launch_dwpw<1, 5>(x, w_dw, tmF, y, p, stream, d, 55);
+    if (staged && K == 3) return launch_dwpw<1, 3>(x, w_dw, tmF, y, p, stream, d, 54);
+    if (staged && K == 5) return launch_dwpw<1, 5>(x, w_dw, tmF, y, p, stream, d, 55);
     return launch_dwpw<1, 0>(x, w_dw, tmF, y, p, stream, d, 56);
 }
 

@@ -10,23 +10,36 @@
 // with the depthwise output rounded to bfloat16 (nearest even) as the A operand, F bfloat16
 // [C][Cout] as the B operand, float32 accumulation in TMEM, and y written as float32 NCHW.
 //
-// Work layout. A persistent CTA of 8 warps owns 128 consecutive output pixels of the flattened
+// Work layout. A persistent CTA of 16 warps owns 128 consecutive output pixels of the flattened
 // (n, oy, ox) space (a tile may span images) and walks the channels in blocks of 64:
-//   * every thread computes 32 depthwise outputs of one pixel (thread t: pixel t % 128, channels
-//     (t / 128) * 32 .. +31 of the block; a warp's 32 pixels are consecutive, so each tap's x
-//     loads are one coalesced row segment and the weights are warp-uniform) and writes them, as
-//     bf16 pairs, into a 128 x 64 A tile laid out exactly as a 128-byte-swizzled K-major TMA
-//     tile would be;
+//   * every thread computes 16 depthwise outputs of one pixel (thread t: pixel t % 128, channels
+//     (t / 128) * 16 .. +15 of the block; a warp's 32 pixels are consecutive, so each tap's x
+//     loads are one coalesced row segment). The pixel's in-image taps are worked out once per
+//     tile (3x3: predicated loads; 5x5: unpredicated loads from clamped offsets, masked to +0),
+//     the weights sit in shared memory (read as float4, one address for the whole warp), and the
+//     loads of 4 channels (3x3) or of one channel's 25 taps (5x5) are issued before their
+//     arithmetic. The outputs go, as bf16 values or quads, into a 128 x 64 A tile laid out
+//     exactly as a 128-byte-swizzled K-major TMA tile would be;
 //   * thread 0 loads the block's 64 x Cout filter rows by TMA (MN-major, 64-column boxes) and,
 //     after the CTA barrier that publishes the A tile, issues the four K = 16 MMAs of the block
 //     into one TMEM accumulator of N = Cout (rounded up to 16) columns, then commits to the
 //     stage's barrier, which frees that A/B stage two blocks later;
-//   * after the last block, all 8 warps read the accumulator (warp w: TMEM lanes 32*(w%4), one
-//     half of the 16-column chunks), add the pointwise bias and store y: for each output channel
+//   * after the last block, all 16 warps read the accumulator (warp w: TMEM lanes 32*(w%4), one
+//     quarter of the 16-column chunks), add the pointwise bias and store y: for each output channel
 //     a warp writes 32 consecutive pixels of one NCHW plane.
 // Two A/B stages let the tensor cores and the TMA run under the next block's depthwise work.
+//
+// Few pixel tiles (small images: 64 images of 7x7 make only 25 tiles) would leave most SMs idle,
+// so a cluster of S CTAs (S <= 4) can share one tile: rank k takes channel blocks k, k + S, ...
+// into its own accumulator, and the partial sums meet in distributed shared memory. Chunk cb of
+// 16 output columns belongs to rank cb % S; every rank writes its partial of the chunk into slot
+// k of the owner's (then idle) stage area, and the owner adds the slots in rank order -- a fixed
+// order, so a given split always gives the same bits.
+//
 // Every wait is bounded; the CTA decides to stop with a barrier-wide OR, so all threads leave
-// together, and all MMAs complete before TMEM is freed.
+// the channel loop together; a CTA whose wait ran out still takes every cluster barrier of the
+// remaining tiles (its peers never wait for it forever), and all MMAs complete before TMEM is
+// freed.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -47,6 +60,9 @@ struct DwPwParams {
     int num_kblk;              // ceil(C / 64)
     int M;                     // N * Ho * Wo
     int num_tiles;             // ceil(M / 128)
+    int w_floats;              // depthwise weights staged in shared memory: C * KKP (K = 3, 5), else 0
+    int S;                     // CTAs of a cluster that split the channel blocks of one tile (1: none)
+    int owned;                 // 16-column chunks of the accumulator each cluster rank reduces
     uint32_t idesc;
     uint32_t tmem_cols;        // power of two >= max(32, n_mma)
     const float *b_dw;         // [C] or null
@@ -54,31 +70,68 @@ struct DwPwParams {
     FastDiv div_howo, div_wo;
 };
 
-constexpr int kDwPwThreads = 256;
+constexpr int kDwPwThreads = 512;
 constexpr int kDwPwA = 128 * 128;      // A stage: 128 pixel rows x 64 channels, bf16 (16 KB)
 constexpr int kDwPwBox = 64 * 128;     // one filter box: 64 channel rows x 64 outputs, bf16 (8 KB)
 constexpr int kDwPwB = 4 * kDwPwBox;   // B stage: up to 256 outputs
-constexpr int kDwPwSmem = 1024 + 2 * kDwPwA + 2 * kDwPwB + 64;
+constexpr int kDwPwStages = 2 * kDwPwA + 2 * kDwPwB;              // 96 KB, reused by the reduction
+constexpr int kDwPwFixed = 1024 + kDwPwStages + 64;               // plus the staged weights
+constexpr int kDwPwMaxSmem = 227 * 1024;
+constexpr int kDwPwChunkBytes = 128 * 16 * 4;                     // 128 rows x 16 fp32 columns
+
+// taps per channel rounded up to a float4 (the staged weight row)
+__host__ __device__ constexpr int dwpw_kkp(int K) { return (K * K + 3) & ~3; }
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// shared::cta address -> the same offset in cluster rank `rank`'s shared memory
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
 
 template <int MODE, int KC>
-__global__ void __launch_bounds__(kDwPwThreads, 2)
+__global__ void __launch_bounds__(kDwPwThreads, 1)
 dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
             float *__restrict__ y, const DwPwParams p, unsigned int *status) {
     const int K = KC ? KC : p.K;
+    constexpr int KK = KC * KC;
+    constexpr int KKP = (KK + 3) & ~3;
+    constexpr int CG = KC <= 3 ? 4 : 1;   // channels whose loads are in flight together
+    constexpr int GU = KC <= 3 ? 4 : 1;   // channel groups unrolled
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;   // swizzle atoms need 1024-byte alignment
     uint8_t *smem = smem_raw + (base - raw);
     const uint32_t sA = base;
     const uint32_t sB = base + 2 * kDwPwA;
-    const uint32_t bars = sB + 2 * kDwPwB;
+    const uint32_t bars = base + kDwPwStages;
     auto bfull = [&](uint32_t s) { return bars + 8u * s; };
     auto afree = [&](uint32_t s) { return bars + 16u + 8u * s; };
     const uint32_t accf = bars + 32u;
     const uint32_t done = bars + 40u;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + (bars - base) + 48);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + (bars - base) + 52);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + kDwPwStages + 48);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kDwPwStages + 52);
+    float *sW = reinterpret_cast<float *>(smem + kDwPwStages + 64);   // [C][KKP]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int S = p.S;
+    const uint32_t rank = S > 1 ? cluster_rank() : 0u;
+    const int cluster = S > 1 ? static_cast<int>(blockIdx.x) / S : static_cast<int>(blockIdx.x);
+    const int num_clusters = S > 1 ? static_cast<int>(gridDim.x) / S : static_cast<int>(gridDim.x);
 
     if (tid == 0) {
         mbar_init(bfull(0), 1);
@@ -91,6 +144,12 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
         fence_barrier_init();
         prefetch_tensormap(&tmF);
     }
+    if (KC > 0) {   // the depthwise weights, once per CTA, as rows of KKP floats
+        for (int i = tid; i < p.C * KK; i += kDwPwThreads) {
+            const int c = i / KK;
+            sW[c * KKP + (i - c * KK)] = __ldg(w + i);
+        }
+    }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_holder), p.tmem_cols);
         tmem_relinquish();
@@ -101,10 +160,11 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
     const uint32_t tmem = *tmem_holder;
 
     const int r = tid & 127;       // pixel row of the tile for the depthwise stage
-    const int half = tid >> 7;     // channels half*32 .. +31 of each block
+    const int quarter = tid >> 7;  // channels quarter*16 .. +15 of each block
     const long long plane = static_cast<long long>(p.H) * p.W;
     uint32_t it = 0, ntile = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ntile) {
+    bool dead = false;             // a bounded wait ran out: skip the work, keep the cluster in step
+    for (int tile = cluster; tile < p.num_tiles; tile += num_clusters, ++ntile) {
         const int m = tile * 128 + r;
         const bool valid = m < p.M;
         int n = 0, oy = 0, ox = 0;
@@ -116,44 +176,109 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
         }
         const int iy0 = oy * p.stride - p.pad, ix0 = ox * p.stride - p.pad;
         const float *xn = x + static_cast<long long>(n) * p.C * plane;
-        bool stop = false;
-        for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
+        // this pixel's taps, once per tile: which lie inside the image (bit t of inmask, tap
+        // t = ky*K + kx) and, for 5x5, an offset inside the plane (a harmless in-plane one for
+        // taps outside the image) with a mask that turns those taps into +0
+        constexpr bool kMasked = KC >= 5;   // 5x5: unpredicated loads; 3x3: predicated loads
+        constexpr int NOFF = kMasked ? KK : 1;
+        int off[NOFF];
+        uint32_t msk[NOFF];
+        uint32_t inmask = 0;
+        const int boff = iy0 * p.W + ix0, rstep = p.dil * p.W;
+        if (KC) {
+#pragma unroll
+            for (int ky = 0; ky < KC; ++ky)
+#pragma unroll
+                for (int kx = 0; kx < KC; ++kx) {
+                    const int iy = iy0 + ky * p.dil, ix = ix0 + kx * p.dil;
+                    const bool in = valid && static_cast<unsigned>(iy) < static_cast<unsigned>(p.H) &&
+                                    static_cast<unsigned>(ix) < static_cast<unsigned>(p.W);
+                    inmask |= (in ? 1u : 0u) << (ky * KC + kx);
+                    if constexpr (kMasked) {
+                        off[ky * KC + kx] = in ? iy * p.W + ix : 0;
+                        msk[ky * KC + kx] = in ? 0xFFFFFFFFu : 0u;
+                    }
+                }
+        }
+        // this rank's channel blocks: rank, rank + S, ...
+        int kcount = 0;
+        for (int kb = static_cast<int>(rank); kb < p.num_kblk && !dead; kb += S, ++it, ++kcount) {
             const uint32_t s = it & 1u, use = it >> 1;
             // stage s is free once the MMAs of two blocks ago have read it
             const bool w_ok = it < 2 || mbar_wait(afree(s), (use - 1u) & 1u);
-            if (__syncthreads_or(!w_ok || *abort_flag)) { stop = true; break; }
+            if (__syncthreads_or(!w_ok || *abort_flag)) { dead = true; break; }
             if (tid == 0) {
                 mbar_arrive_expect_tx(bfull(s), static_cast<uint32_t>(p.n_boxes * kDwPwBox));
                 for (int h = 0; h < p.n_boxes; ++h)
                     tma_load_3d(sB + s * kDwPwB + h * kDwPwBox, &tmF, bfull(s), h * 64, kb * 64, 0);
             }
-            // depthwise outputs of 32 channels at this pixel -> bf16 pairs in row r of A[s]
-            uint8_t *arow = smem + s * kDwPwA + r * 128;
-#pragma unroll 1
-            for (int j = 0; j < 32; j += 2) {
-                const int cl = half * 32 + j;
-                float v[2];
+            // depthwise outputs of 16 channels at this pixel -> row r of A[s] as bf16
+            const int c0 = kb * 64 + quarter * 16;
+            const uint32_t arow = sA + s * kDwPwA + r * 128;
+            // local channel cl -> byte address of its bf16 in the swizzled row
+            auto a_addr = [&](int cl) {
+                return arow + ((static_cast<uint32_t>(cl >> 3) ^ static_cast<uint32_t>(r & 7)) << 4) + (cl & 7) * 2;
+            };
+            if constexpr (KC > 0) {   // weights staged in shared memory (the host guarantees it)
+#pragma unroll GU
+                for (int g = 0; g < 16; g += CG) {
+                    float xv[CG][KK > 0 ? KK : 1];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int c = kb * 64 + cl + u;
-                    float acc = 0.0f;
-                    if (valid && c < p.C) {
-                        const float *xp = xn + c * plane;
-                        const float *wp = w + c * K * K;
-                        if (KC) {   // compile-time filter size: fully unrolled taps
+                    for (int u = 0; u < CG; ++u) {
+                        const int c = c0 + g + u;
+                        const float *xp = xn + (c < p.C ? c : 0) * plane;
 #pragma unroll
-                            for (int ky = 0; ky < KC; ++ky) {
-                                const int iy = iy0 + ky * p.dil;
-                                const bool rok = static_cast<unsigned>(iy) < static_cast<unsigned>(p.H);
+                        for (int t = 0; t < KK; ++t) {
+                            if constexpr (kMasked)
+                                xv[u][t] = __uint_as_float(__float_as_uint(__ldg(xp + off[t])) & msk[t]);
+                            else
+                                xv[u][t] = (c < p.C && ((inmask >> t) & 1u))
+                                               ? __ldg(xp + (boff + (t / KC) * rstep + (t % KC) * p.dil)) : 0.0f;
+                        }
+                    }
+                    float v[CG];
 #pragma unroll
-                                for (int kx = 0; kx < KC; ++kx) {
-                                    const int ix = ix0 + kx * p.dil;
-                                    const bool in = rok && static_cast<unsigned>(ix) < static_cast<unsigned>(p.W);
-                                    const float xv = in ? __ldg(xp + iy * p.W + ix) : 0.0f;
-                                    acc = dw_tap<MODE>(acc, __ldg(wp + ky * KC + kx), xv);
-                                }
+                    for (int u = 0; u < CG; ++u) {
+                        const int c = c0 + g + u;
+                        float acc = 0.0f;
+                        if (valid && c < p.C) {
+                            const float4 *w4 = reinterpret_cast<const float4 *>(sW + c * KKP);
+#pragma unroll
+                            for (int t4 = 0; t4 < KKP / 4; ++t4) {
+                                const float4 wv = w4[t4];
+                                const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    if (4 * t4 + e < KK) acc = dw_tap<MODE>(acc, ws[e], xv[u][4 * t4 + e]);
                             }
-                        } else {
+                            acc = p.b_dw ? dw_finish<MODE, true>(acc, __ldg(p.b_dw + c))
+                                         : dw_finish<MODE, false>(acc, 0.0f);
+                        }
+                        v[u] = acc;
+                    }
+                    const uint32_t addr = a_addr(quarter * 16 + g);
+                    if constexpr (CG == 4) {
+                        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(pack_bf16x2(v[0], v[1])),
+                                     "r"(pack_bf16x2(v[2], v[3]))
+                                     : "memory");
+                    } else {
+                        const __nv_bfloat16 hb = __float2bfloat16_rn(v[0]);
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<const uint16_t *>(&hb))
+                                     : "memory");
+                    }
+                }
+            } else {
+                // any filter size: weights and inputs straight from global memory
+#pragma unroll 1
+                for (int j = 0; j < 16; j += 2) {
+                    float v[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int c = c0 + j + u;
+                        float acc = 0.0f;
+                        if (valid && c < p.C) {
+                            const float *xp = xn + c * plane;
+                            const float *wp = w + c * K * K;
                             for (int ky = 0; ky < K; ++ky) {
                                 const int iy = iy0 + ky * p.dil;
                                 const bool rok = static_cast<unsigned>(iy) < static_cast<unsigned>(p.H);
@@ -164,13 +289,14 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
                                     acc = dw_tap<MODE>(acc, __ldg(wp + ky * K + kx), xv);
                                 }
                             }
+                            acc = p.b_dw ? dw_finish<MODE, true>(acc, __ldg(p.b_dw + c))
+                                         : dw_finish<MODE, false>(acc, 0.0f);
                         }
-                        acc = p.b_dw ? dw_finish<MODE, true>(acc, __ldg(p.b_dw + c)) : dw_finish<MODE, false>(acc, 0.0f);
+                        v[u] = acc;
                     }
-                    v[u] = acc;
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(a_addr(quarter * 16 + j)), "r"(pack_bf16x2(v[0], v[1]))
+                                 : "memory");
                 }
-                const uint32_t chunk = static_cast<uint32_t>(cl >> 3) ^ static_cast<uint32_t>(r & 7);
-                *reinterpret_cast<uint32_t *>(arow + (chunk << 4) + (cl & 7) * 2) = pack_bf16x2(v[0], v[1]);
             }
             fence_proxy_async_smem();   // the A tile is read by the tensor cores (async proxy)
             __syncthreads();
@@ -185,7 +311,7 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
                         // 8 KB apart.
                         const uint64_t ad = smem_desc_sw128(a0 + kk * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, kDwPwBox, 1024);
-                        umma_f16_ss(tmem, ad, bd, p.idesc, (kb | kk) != 0 ? 1u : 0u);
+                        umma_f16_ss(tmem, ad, bd, p.idesc, (kcount | kk) != 0 ? 1u : 0u);
                     }
                     umma_commit(afree(s));
                 } else {
@@ -194,40 +320,97 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
                 }
             }
         }
-        if (stop) break;
-        if (tid == 0) umma_commit(accf);
-        const bool a_ok = mbar_wait(accf, ntile & 1u);
-        if (__syncthreads_or(!a_ok || *abort_flag)) break;
+        if (!dead) {
+            if (tid == 0) umma_commit(accf);
+            const bool a_ok = mbar_wait(accf, ntile & 1u);
+            if (__syncthreads_or(!a_ok || *abort_flag)) dead = true;
+        }
         tc_fence_after();
-        // epilogue: accumulator rows -> y (NCHW float32), plus the pointwise bias
-        {
-            const int q = warp & 3;                 // TMEM lane quarter of this warp
-            const int row = q * 32 + lane;
-            const int me = tile * 128 + row;
-            const bool ve = me < p.M;
-            int ne = 0, pix = 0;
-            if (ve) {
-                ne = fdiv(me, p.div_howo);
-                pix = me - ne * p.HoWo;
-            }
-            float *yrow = y + static_cast<long long>(ne) * p.Cout * p.HoWo + pix;
-            const int nch = p.n_mma >> 4;
-            for (int cb = warp >> 2; cb < nch; cb += 2) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + cb * 16, v);
-                tmem_wait_ld();
+        const bool have = !dead && kcount > 0;   // this CTA's accumulator holds a partial sum
+        const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int row = q * 32 + lane;
+        const int me = tile * 128 + row;
+        const int nch = p.n_mma >> 4;
+        if (S == 1) {
+            // accumulator rows -> y (NCHW float32), plus the pointwise bias
+            if (have) {
+                const bool ve = me < p.M;
+                int ne = 0, pix = 0;
                 if (ve) {
+                    ne = fdiv(me, p.div_howo);
+                    pix = me - ne * p.HoWo;
+                }
+                float *yrow = y + static_cast<long long>(ne) * p.Cout * p.HoWo + pix;
+                for (int cb = warp >> 2; cb < nch; cb += kDwPwThreads / 128) {
+                    uint32_t t[16];
+                    tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + cb * 16, t);
+                    tmem_wait_ld();
+                    if (ve) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int o = cb * 16 + j;
-                        if (o < p.Cout) {
-                            float val = __uint_as_float(v[j]);
-                            if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
-                            yrow[static_cast<long long>(o) * p.HoWo] = val;
+                        for (int j = 0; j < 16; ++j) {
+                            const int o = cb * 16 + j;
+                            if (o < p.Cout) {
+                                float val = __uint_as_float(t[j]);
+                                if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
+                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                            }
                         }
                     }
                 }
             }
+        } else {
+            // Channel-split reduction across the cluster. Chunk cb (16 columns) belongs to rank
+            // cb % S, which receives every rank's partial of it in slot `rank` of its stage area
+            // ([slot][owned chunk][128 rows][16 floats]) and adds the slots in rank order.
+            cluster_sync_all();   // every rank is done with its stage area (MMAs complete)
+            for (int cb = warp >> 2; cb < nch; cb += kDwPwThreads / 128) {
+                uint32_t t[16];
+                if (have) {
+                    tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + cb * 16, t);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) t[j] = 0u;
+                }
+                const uint32_t owner = static_cast<uint32_t>(cb % S);
+                const uint32_t slot_off = ((rank * p.owned + static_cast<uint32_t>(cb / S)) * 128u + row) * 64u;
+                const uint32_t dst = map_rank(sA + slot_off, owner);
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) st_cluster_v4(dst + j * 4, t[j], t[j + 1], t[j + 2], t[j + 3]);
+            }
+            cluster_sync_all();   // every partial has landed
+            if (!dead) {
+                // this rank's chunks: 128 rows x 16 columns each; thread -> (row, 4 columns)
+                const int rr = tid & 127, cq = tid >> 7;
+                const int mr = tile * 128 + rr;
+                if (mr < p.M) {
+                    const int ne = fdiv(mr, p.div_howo);
+                    const int pix = mr - ne * p.HoWo;
+                    float *yrow = y + static_cast<long long>(ne) * p.Cout * p.HoWo + pix;
+                    for (int lc = 0; lc * S + static_cast<int>(rank) < nch; ++lc) {
+                        const int cb = lc * S + static_cast<int>(rank);
+                        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                        for (int sl = 0; sl < S; ++sl) {
+                            const float4 v = *reinterpret_cast<const float4 *>(
+                                smem + ((sl * p.owned + lc) * 128 + rr) * 64 + cq * 16);
+                            acc[0] = __fadd_rn(acc[0], v.x);
+                            acc[1] = __fadd_rn(acc[1], v.y);
+                            acc[2] = __fadd_rn(acc[2], v.z);
+                            acc[3] = __fadd_rn(acc[3], v.w);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int o = cb * 16 + cq * 4 + j;
+                            if (o < p.Cout) {
+                                float val = acc[j];
+                                if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
+                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                            }
+                        }
+                    }
+                }
+            }
+            __syncthreads();   // the stage area is read before the next tile's loads overwrite it
         }
         tc_fence_before();
         __syncthreads();   // the accumulator is free for the next tile's MMAs

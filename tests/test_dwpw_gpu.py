@@ -106,3 +106,28 @@ def test_full_size_blocks_sampled(cb, case):
         ref, absum = oracle.dwpw_points(x, w, bd, workloads.bf16_to_f32(F), bp, idx, case.stride, case.pad, case.dil,
                                         mode)
         assert np.all(np.abs(y.reshape(-1)[idx] - ref) <= _tol(case.C) * absum)
+
+
+@pytest.mark.parametrize("split", ["1", "2", "3", "4"])
+def test_channel_split_across_a_cluster(cb, split, monkeypatch):
+    # 13 pixel tiles and 11 channel blocks: by default a 4-CTA cluster splits the channels; every
+    # split must meet the same bar, and a given split must repeat its bits exactly
+    monkeypatch.setenv("CONV_B200_DWPW_SPLIT", split)
+    case = workloads.DwPwCase("t", 8, 672, 14, 14, 3, 1, 1, 1, 112, True, seed=11)
+    x, w, bd, F, bp = workloads.dwpw_inputs(case)
+    y, kernel = _run(cb, case, x, w, bd, F, bp, 0)
+    y2, _ = _run(cb, case, x, w, bd, F, bp, 0)
+    assert kernel == "dwpw_kernel" and np.array_equal(y, y2)
+    ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, 1, 1, 1, 0)
+    assert np.all(np.abs(y - ref) <= _tol(case.C) * absum)
+
+
+def test_split_identity_mixing_is_exact(cb, monkeypatch):
+    # with F = I every partial but one is zero, so the cluster's reduction is exact too
+    monkeypatch.setenv("CONV_B200_DWPW_SPLIT", "3")
+    case = workloads.DwPwCase("t", 2, 192, 10, 10, 5, 1, 2, 1, 192, True, seed=12)
+    x, w, bd, _, _ = workloads.dwpw_inputs(case)
+    F = workloads.bf16_bits(np.eye(192, dtype=np.float32))
+    y, _ = _run(cb, case, x, w, bd, F, None, 1)
+    dref = oracle.depthwise(x, w, bd, mult=1, stride=1, pad=2, dil=1, mode=1)
+    assert np.array_equal(y, workloads.bf16_to_f32(workloads.bf16_bits(dref)).astype(np.float64))
