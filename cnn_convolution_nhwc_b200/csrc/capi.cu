@@ -75,6 +75,14 @@ struct DeviceState {
     unsigned int *status = nullptr;   // device address of g_conv_status on this device
     unsigned long long attr_done[2] = {0, 0};   // bit per kernel whose shared-memory limit is raised
     cublasHandle_t blas = nullptr;    // for the explicit-im2col comparison path, made on first use
+    // clusters of a kernel that fit on the device at once, per (kernel bit, cluster size, shared
+    // memory), asked once (outside any stream capture: the first call of a shape runs eagerly)
+    struct ClusterFit {
+        unsigned bit;
+        int S, smem, active;
+    };
+    ClusterFit cluster_fit[64];
+    int n_cluster_fit = 0;
 };
 
 std::mutex g_mu;
@@ -889,8 +897,16 @@ int launch_dw(const float *x, const float *w, const float *bias, float *y, const
 
 // ---- fused depthwise -> pointwise -------------------------------------------------------
 // shared-memory attribute bits 51..56: MODE x (K 3, K 5, other K)
+// Channel split S of the fused kernel: a cluster of S CTAs shares each 128-pixel tile (S = 1:
+// one CTA per tile). S * owned 16-column chunks of 8 KB must fit the 96 KB stage area they reuse,
+// and every rank needs a channel block.
+bool dwpw_split_ok(const DwPwParams &p, int S) {
+    const int nch = p.n_mma / 16;
+    return S >= 1 && S <= 4 && S <= p.num_kblk && S * ((nch + S - 1) / S) * kDwPwChunkBytes <= kDwPwStages;
+}
+
 template <int MODE, int KC>
-int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y, const DwPwParams &p,
+int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y, DwPwParams p, int force_split,
                 cudaStream_t stream, DeviceState *d, unsigned bit) {
     auto kern = dwpw_kernel<MODE, KC>;
     if (int rc = ensure_smem_attr(d, bit, kern, kDwPwMaxSmem)) return rc;
@@ -899,23 +915,60 @@ int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y
     cfg.blockDim = dim3(kDwPwThreads);
     cfg.dynamicSmemBytes = kDwPwFixed + 4 * p.w_floats;
     cfg.stream = stream;
-    int clusters = p.num_tiles < d->num_sms ? p.num_tiles : d->num_sms;
-    if (p.S > 1) {
-        // clusters of S CTAs split a tile's channel blocks; as many clusters as fit at once
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // clusters of S CTAs that can run at once (one CTA per SM)
+    auto active_clusters = [&](int S) {
+        if (S == 1) return d->num_sms;
+        const int smem = static_cast<int>(cfg.dynamicSmemBytes);
+        {
+            std::lock_guard<std::mutex> lock(g_mu);
+            for (int i = 0; i < d->n_cluster_fit; ++i) {
+                const DeviceState::ClusterFit &f = d->cluster_fit[i];
+                if (f.bit == bit && f.S == S && f.smem == smem) return f.active;
+            }
+        }
+        attr[0].val.clusterDim.x = static_cast<unsigned>(S);
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cfg.gridDim = dim3(static_cast<unsigned>(p.S));
+        cfg.gridDim = dim3(static_cast<unsigned>(S));
         int active = 0;
-        if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active < 1) return CONV_ERR_CUDA;
-        if (clusters > active) clusters = active;
-        cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S));
+        if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess) active = 0;
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (d->n_cluster_fit < 64) d->cluster_fit[d->n_cluster_fit++] = DeviceState::ClusterFit{bit, S, smem, active};
+        return active;
+    };
+    // The split that finishes first: rounds of tiles (ceil(tiles / clusters at once)) times the
+    // 1/S share of a tile each CTA computes; a split pays a small reduction cost.
+    int S = 1, clusters = d->num_sms;
+    if (force_split) {
+        if (!dwpw_split_ok(p, force_split)) return CONV_ERR_UNSUPPORTED;
+        S = force_split;
+        clusters = active_clusters(S);
+        if (clusters < 1) return CONV_ERR_CUDA;
     } else {
-        cfg.gridDim = dim3(static_cast<unsigned>(clusters));
+        double best = 1e30;
+        for (int cand = 1; cand <= 4; ++cand) {
+            if (!dwpw_split_ok(p, cand)) continue;
+            const int act = active_clusters(cand);
+            if (act < 1) continue;
+            const double cost = static_cast<double>((p.num_tiles + act - 1) / act) / cand + (cand > 1 ? 0.05 : 0.0);
+            if (cost < best) { best = cost; S = cand; clusters = act; }
+        }
     }
+    p.S = S;
+    p.owned = (p.n_mma / 16 + S - 1) / S;
+    if (clusters > p.num_tiles) clusters = p.num_tiles;
+    if (S > 1) {
+        attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    } else {
+        cfg.attrs = nullptr;
+        cfg.numAttrs = 0;
+    }
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * S));
     return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_kernel");
 }
 
@@ -1329,44 +1382,27 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
     p.b_pw = b_pw;
     p.div_howo = make_fastdiv(static_cast<uint32_t>(p.HoWo));
     p.div_wo = make_fastdiv(static_cast<uint32_t>(p.Wo));
-    // Too few pixel tiles to fill the GPU: a cluster of S CTAs splits each tile's channel blocks
-    // and reduces the partial sums in a fixed rank order through distributed shared memory
-    // (S * owned chunks of 8 KB must fit the 96 KB stage area they reuse).
-    {
-        const int nch = p.n_mma / 16;
-        p.S = 1;
-        p.owned = nch;
-        if (2 * p.num_tiles <= d->num_sms) {
-            int S = d->num_sms / p.num_tiles;
-            if (S > 4) S = 4;
-            if (S > p.num_kblk) S = p.num_kblk;
-            while (S > 1 && S * ((nch + S - 1) / S) * kDwPwChunkBytes > kDwPwStages) --S;
-            if (S > 1) {
-                p.S = S;
-                p.owned = (nch + S - 1) / S;
-            }
-        }
-        const char *force = env("CONV_B200_DWPW_SPLIT");   // tests: force a split (1..4)
-        if (force) {
-            const int S = std::atoi(force);
-            if (S < 1 || S > 4 || S > p.num_kblk || S * ((nch + S - 1) / S) * kDwPwChunkBytes > kDwPwStages)
-                return CONV_ERR_UNSUPPORTED;
-            p.S = S;
-            p.owned = (nch + S - 1) / S;
-        }
+    // CONV_B200_DWPW_SPLIT (tests) forces the channel split S = 1..4; otherwise the launcher
+    // picks the split that fills the GPU best
+    int force_split = 0;
+    if (const char *f = env("CONV_B200_DWPW_SPLIT")) {
+        force_split = std::atoi(f);
+        if (force_split < 1 || force_split > 4) return CONV_ERR_UNSUPPORTED;
     }
+    p.S = 1;
+    p.owned = p.n_mma / 16;
     // K = 3 and K = 5 stage the depthwise weights in shared memory when they fit; other filter
     // sizes (or very many channels) read them from global memory
     const bool staged = (K == 3 || K == 5) && 4LL * C * dwpw_kkp(K) <= kDwPwMaxSmem - kDwPwFixed;
     p.w_floats = staged ? C * dwpw_kkp(K) : 0;
     if (mode == DW_EXACT) {
-        if (staged && K == 3) return launch_dwpw<0, 3>(x, w_dw, tmF, y, p, stream, d, 51);
-        if (staged && K == 5) return launch_dwpw<0, 5>(x, w_dw, tmF, y, p, stream, d, 52);
-        return launch_dwpw<0, 0>(x, w_dw, tmF, y, p, stream, d, 53);
+        if (staged && K == 3) return launch_dwpw<0, 3>(x, w_dw, tmF, y, p, force_split, stream, d, 51);
+        if (staged && K == 5) return launch_dwpw<0, 5>(x, w_dw, tmF, y, p, force_split, stream, d, 52);
+        return launch_dwpw<0, 0>(x, w_dw, tmF, y, p, force_split, stream, d, 53);
     }
-    if (staged && K == 3) return launch_dwpw<1, 3>(x, w_dw, tmF, y, p, stream, d, 54);
-    if (staged && K == 5) return launch_dwpw<1, 5>(x, w_dw, tmF, y, p, stream, d, 55);
-    return launch_dwpw<1, 0>(x, w_dw, tmF, y, p, stream, d, 56);
+    if (staged && K == 3) return launch_dwpw<1, 3>(x, w_dw, tmF, y, p, force_split, stream, d, 54);
+    if (staged && K == 5) return launch_dwpw<1, 5>(x, w_dw, tmF, y, p, force_split, stream, d, 55);
+    return launch_dwpw<1, 0>(x, w_dw, tmF, y, p, force_split, stream, d, 56);
 }
 
 }  // extern "C"
