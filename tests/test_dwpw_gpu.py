@@ -55,6 +55,9 @@ CASES = [
     (1, 8, 9, 7, 1, 3, 1, 256, 0, True),        # 7x7 (runtime filter size), 256 outputs
     (3, 24, 11, 3, 2, 1, 2, 24, 1, True),       # stride 2 with dilation 2, N = 32 MMA
     (2, 40, 12, 3, 1, 0, 1, 8, 0, True),        # no padding, 8 outputs
+    (3, 32, 5, 1, 1, 0, 1, 32, 0, True),        # 1x1 depthwise (a per-channel scale and bias)
+    (5, 24, 1, 3, 1, 1, 1, 16, 0, True),        # 1x1 images: every tap but the centre is padding
+    (1, 200, 3, 3, 2, 1, 1, 200, 1, True),      # 2x2 output, one partial tile, ragged Cout chunk
 ]
 
 
