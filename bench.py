@@ -536,6 +536,11 @@ def run_ours(args, dist):
         if not case.square:
             cfg.update({"KH": case.kh, "KW": case.kw, "stride_w": case.sw, "pad_w": case.pw, "dil_w": case.dw,
                         "groups": case.groups})
+        # the explicit patch matrix the implicit kernels never build (N*Ho*Wo rows by
+        # KH*KW*Cin/groups bf16 columns per group) and its size over the input's
+        patch = 2 * case.N * case.Ho * case.Wo * case.kh * case.kw * case.Cin
+        cfg["patch_matrix_bytes_avoided"] = patch if mode != "im2col" else 0
+        cfg["patch_matrix_expansion"] = round(patch / (2 * case.N * case.H * case.W * case.Cin), 3)
         if mode == "im2col":
             cfg["path"] = "explicit patch matrix in a workspace + one cuBLAS GEMM (comparison path)"
     else:
