@@ -897,23 +897,23 @@ int launch_dw(const float *x, const float *w, const float *bias, float *y, const
 
 // ---- fused depthwise -> pointwise -------------------------------------------------------
 // shared-memory attribute bits 51..56: MODE x (K 3, K 5, other K)
-// Channel split S of the fused kernel: a cluster of S CTAs shares each 128-pixel tile (S = 1:
-// one CTA per tile). S * owned 16-column chunks of 8 KB must fit the 96 KB stage area they reuse,
+// Channel split S of the fused kernels: a cluster of S CTAs shares each tile (S = 1: one CTA per
+// tile). S * owned 16-column chunks of 8 KB must fit the receive area (the stages they reuse),
 // and every rank needs a channel block.
-bool dwpw_split_ok(const DwPwParams &p, int S) {
+bool dwpw_split_ok(const DwPwParams &p, int S, int recv_bytes) {
     const int nch = p.n_mma / 16;
-    return S >= 1 && S <= 4 && S <= p.num_kblk && S * ((nch + S - 1) / S) * kDwPwChunkBytes <= kDwPwStages;
+    return S >= 1 && S <= 4 && S <= p.num_kblk && S * ((nch + S - 1) / S) * kDwPwChunkBytes <= recv_bytes;
 }
 
-template <int MODE, int KC>
-int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y, DwPwParams p, int force_split,
-                cudaStream_t stream, DeviceState *d, unsigned bit) {
-    auto kern = dwpw_kernel<MODE, KC>;
+// Picks the split (or takes the forced one), sets p.S / p.owned and fills the launch geometry
+// of `cfg` (whose cluster attribute lives in `attr`). The caller launches with the updated p.
+template <typename Kern>
+int dwpw_split_config(Kern kern, unsigned bit, int smem, int recv_bytes, DwPwParams &p, int force_split,
+                      cudaStream_t stream, DeviceState *d, cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr) {
     if (int rc = ensure_smem_attr(d, bit, kern, kDwPwMaxSmem)) return rc;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cfg = cudaLaunchConfig_t{};
     cfg.blockDim = dim3(kDwPwThreads);
-    cfg.dynamicSmemBytes = kDwPwFixed + 4 * p.w_floats;
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = stream;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.y = 1;
@@ -921,7 +921,6 @@ int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y
     // clusters of S CTAs that can run at once (one CTA per SM)
     auto active_clusters = [&](int S) {
         if (S == 1) return d->num_sms;
-        const int smem = static_cast<int>(cfg.dynamicSmemBytes);
         {
             std::lock_guard<std::mutex> lock(g_mu);
             for (int i = 0; i < d->n_cluster_fit; ++i) {
@@ -943,14 +942,14 @@ int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y
     // 1/S share of a tile each CTA computes; a split pays a small reduction cost.
     int S = 1, clusters = d->num_sms;
     if (force_split) {
-        if (!dwpw_split_ok(p, force_split)) return CONV_ERR_UNSUPPORTED;
+        if (!dwpw_split_ok(p, force_split, recv_bytes)) return CONV_ERR_UNSUPPORTED;
         S = force_split;
         clusters = active_clusters(S);
         if (clusters < 1) return CONV_ERR_CUDA;
     } else {
         double best = 1e30;
         for (int cand = 1; cand <= 4; ++cand) {
-            if (!dwpw_split_ok(p, cand)) continue;
+            if (!dwpw_split_ok(p, cand, recv_bytes)) continue;
             const int act = active_clusters(cand);
             if (act < 1) continue;
             const double cost = static_cast<double>((p.num_tiles + act - 1) / act) / cand + (cand > 1 ? 0.05 : 0.0);
@@ -969,7 +968,79 @@ int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y
         cfg.numAttrs = 0;
     }
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * S));
+    return CONV_OK;
+}
+
+template <int MODE, int KC>
+int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y, DwPwParams p, int force_split,
+                cudaStream_t stream, DeviceState *d, unsigned bit) {
+    auto kern = dwpw_kernel<MODE, KC>;
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    if (int rc = dwpw_split_config(kern, bit, kDwPwFixed + 4 * p.w_floats, kDwPwStages, p, force_split, stream, d,
+                                   cfg, attr))
+        return rc;
     return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_kernel");
+}
+
+// The staged kernel's tiles for this shape (ok = false: it does not apply).
+struct DwPwStagePlan {
+    bool ok = false;
+    DwPwStage st{};
+    int num_tiles = 0;
+};
+
+DwPwStagePlan plan_dwpw_staged(const DwPwParams &p, int N) {
+    DwPwStagePlan pl;
+    if (p.K != 3 && p.K != 5) return pl;
+    DwPwStage &st = pl.st;
+    st.N = N;
+    // Images of at most 128 outputs would be staged whole, G per tile; that form measured slower
+    // than the flat kernel (7x7, 960 channels: 189 vs 89 us), so it is taken only when forced.
+    const char *kforce = env("CONV_B200_DWPW_KERNEL");
+    const bool force_staged = kforce && std::strcmp(kforce, "staged") == 0;
+    if (p.HoWo <= 128) {   // whole images per tile
+        if (!force_staged) return pl;
+        st.G = 128 / p.HoWo;
+        if (st.G > N) st.G = N;
+        st.RB = p.Ho;
+        st.nbands = 1;
+        pl.num_tiles = (N + st.G - 1) / st.G;
+    } else if (p.Wo <= 128) {   // bands of output rows, as even as possible
+        const int max_rows = 128 / p.Wo;
+        st.nbands = (p.Ho + max_rows - 1) / max_rows;
+        st.RB = (p.Ho + st.nbands - 1) / st.nbands;
+        st.G = 1;
+        pl.num_tiles = N * st.nbands;
+    } else {
+        return pl;
+    }
+    st.R_in = (st.RB - 1) * p.stride + (p.K - 1) * p.dil + 1;
+    st.Wp = (p.Wo - 1) * p.stride + (p.K - 1) * p.dil + 1;
+    st.wcols = p.W < st.Wp - p.pad ? p.W : st.Wp - p.pad;
+    if (st.wcols < 1) return pl;
+    st.div_wcols = make_fastdiv(static_cast<uint32_t>(st.wcols));
+    const long long xf = 64LL * st.G * st.R_in * st.Wp;
+    if (xf > (1 << 20)) return pl;
+    st.x_floats = static_cast<int>((xf + 3) & ~3LL);
+    st.w_floats = 64 * dwpw_kkp(p.K);
+    st.b_bytes = p.n_boxes * kDwPwBox;
+    pl.ok = dwpw_staged_smem(st) <= kDwPwMaxSmem;
+    return pl;
+}
+
+template <int MODE, int KC>
+int launch_dwpw_staged(const float *x, const float *w, const CUtensorMap &tmF, float *y, DwPwParams p,
+                       const DwPwStagePlan &pl, int force_split, cudaStream_t stream, DeviceState *d, unsigned bit) {
+    p.num_tiles = pl.num_tiles;
+    p.w_floats = 0;
+    auto kern = dwpw_staged_kernel<MODE, KC>;
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    if (int rc = dwpw_split_config(kern, bit, dwpw_staged_smem(pl.st), dwpw_staged_body(pl.st), p, force_split,
+                                   stream, d, cfg, attr))
+        return rc;
+    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, pl.st, d->status), "dwpw_staged_kernel");
 }
 
 }  // namespace
@@ -1391,6 +1462,21 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
     }
     p.S = 1;
     p.owned = p.n_mma / 16;
+    // 3x3 and 5x5 on images whose tiles fit: the kernel that stages input windows in shared
+    // memory (CONV_B200_DWPW_KERNEL=flat forces the other one; tests)
+    const char *kforce = env("CONV_B200_DWPW_KERNEL");
+    const bool force_flat = kforce && std::strcmp(kforce, "flat") == 0;
+    if (!force_flat) {
+        const DwPwStagePlan pl = plan_dwpw_staged(p, N);
+        if (pl.ok) {
+            if (mode == DW_EXACT)
+                return K == 3 ? launch_dwpw_staged<0, 3>(x, w_dw, tmF, y, p, pl, force_split, stream, d, 57)
+                              : launch_dwpw_staged<0, 5>(x, w_dw, tmF, y, p, pl, force_split, stream, d, 58);
+            return K == 3 ? launch_dwpw_staged<1, 3>(x, w_dw, tmF, y, p, pl, force_split, stream, d, 59)
+                          : launch_dwpw_staged<1, 5>(x, w_dw, tmF, y, p, pl, force_split, stream, d, 60);
+        }
+        if (kforce && std::strcmp(kforce, "staged") == 0) return CONV_ERR_UNSUPPORTED;
+    }
     // K = 3 and K = 5 stage the depthwise weights in shared memory when they fit; other filter
     // sizes (or very many channels) read them from global memory
     const bool staged = (K == 3 || K == 5) && 4LL * C * dwpw_kkp(K) <= kDwPwMaxSmem - kDwPwFixed;

@@ -426,4 +426,335 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
     if (warp == 0) tmem_dealloc(tmem, p.tmem_cols);
 }
 
+// ---------------------------------------------------------------------------------------
+// Staged variant (3x3 and 5x5). Tiles follow the image grid instead of the flattened pixel
+// order: a band of RB output rows of one image (RB * Wo <= 128, the default for images of more
+// than 128 outputs) or G whole images (G = floor(128 / (Ho*Wo)); measured slower than
+// dwpw_kernel for 7x7 images, so the host takes it only when asked). Per channel block the CTA copies, with
+// cp.async, the zero-padded input window of the tile -- 64 channels x G images x R_in rows x Wp
+// columns, positions outside the image written as +0 by the copy's zero fill -- and the block's
+// weights into shared memory, one block ahead of the compute (two buffers). The depthwise taps
+// are then unpredicated shared-memory loads at offsets fixed per launch; everything else
+// (A tile, TMA filter, MMAs, cluster split, epilogue) is as in dwpw_kernel.
+// ---------------------------------------------------------------------------------------
+struct DwPwStage {
+    int G;        // images per tile (1 in band mode)
+    int RB;       // output rows per tile (Ho in image mode)
+    int nbands;   // bands per image (1 in image mode)
+    int R_in;     // staged input rows per image: (RB - 1) * stride + (K - 1) * dil + 1
+    int Wp;       // staged columns: (Wo - 1) * stride + (K - 1) * dil + 1, from column -pad
+    int N;        // images
+    int x_floats; // one staged input buffer: 64 * G * R_in * Wp, rounded up to 4
+    int w_floats; // one staged weight buffer: 64 * KKP
+    int b_bytes;  // one filter stage: n_boxes * 8 KB
+    int wcols;    // input columns copied per row: min(W, Wp - pad)
+    FastDiv div_wcols;
+};
+
+// bytes before the barriers (A, B, staged input and weights), and the launch's shared memory
+__host__ __device__ inline int dwpw_staged_body(const DwPwStage &st) {
+    return 2 * kDwPwA + 2 * st.b_bytes + 8 * st.x_floats + 8 * st.w_floats;
+}
+__host__ __device__ inline int dwpw_staged_smem(const DwPwStage &st) { return 1024 + dwpw_staged_body(st) + 64; }
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N_>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N_) : "memory"); }
+
+template <int MODE, int KC>
+__global__ void __launch_bounds__(kDwPwThreads, 1)
+dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
+                   float *__restrict__ y, const DwPwParams p, const DwPwStage st, unsigned int *status) {
+    constexpr int KK = KC * KC;
+    constexpr int KKP = (KK + 3) & ~3;
+    constexpr int CG = KC <= 3 ? 4 : 2;   // channels computed together
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw);
+    // [A 2 x 16 KB][B 2 x b_bytes][x 2 x x_floats][w 2 x w_floats][bars 64 B]; everything before
+    // the barriers doubles as the receive area of the cluster reduction
+    const uint32_t sA = base;
+    const uint32_t sB = base + 2 * kDwPwA;
+    float *sx = reinterpret_cast<float *>(smem + 2 * kDwPwA + 2 * st.b_bytes);
+    float *sw = sx + 2 * st.x_floats;
+    const uint32_t bars = smem_u32(sw + 2 * st.w_floats);
+    auto bfull = [&](uint32_t s) { return bars + 8u * s; };
+    auto afree = [&](uint32_t s) { return bars + 16u + 8u * s; };
+    const uint32_t accf = bars + 32u;
+    const uint32_t done = bars + 40u;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + (bars - base) + 48);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + (bars - base) + 52);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int S = p.S;
+    const uint32_t rank = S > 1 ? cluster_rank() : 0u;
+    const int cluster = S > 1 ? static_cast<int>(blockIdx.x) / S : static_cast<int>(blockIdx.x);
+    const int num_clusters = S > 1 ? static_cast<int>(gridDim.x) / S : static_cast<int>(gridDim.x);
+
+    if (tid == 0) {
+        mbar_init(bfull(0), 1);
+        mbar_init(bfull(1), 1);
+        mbar_init(afree(0), 1);
+        mbar_init(afree(1), 1);
+        mbar_init(accf, 1);
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmF);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_holder), p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int r = tid & 127;       // A-tile row (pixel of the tile) of the depthwise stage
+    const int quarter = tid >> 7;  // channels quarter*16 .. +15 of each block
+    const int plane_in = st.R_in * st.Wp;           // staged floats of one image of one channel
+    const int rows_per_ch = st.G * st.R_in;
+    const int tile_px = st.G * st.RB * p.Wo;        // A rows a full tile fills
+    uint32_t it = 0, ntile = 0, stg = 0;
+    bool dead = false;
+    for (int tile = cluster; tile < p.num_tiles; tile += num_clusters, ++ntile) {
+        // tile -> first image n0 and first output row oy0
+        const int n0 = st.nbands > 1 ? tile / st.nbands : tile * st.G;
+        const int oy0 = st.nbands > 1 ? (tile - n0 * st.nbands) * st.RB : 0;
+        const int rows_here = min(st.RB, p.Ho - oy0);
+        const int imgs_here = min(st.G, st.N - n0);
+        const int valid_px = imgs_here * rows_here * p.Wo;   // (image mode: rows_here = Ho)
+        const int iy_start = oy0 * p.stride - p.pad;
+        // this thread's pixel in the staged window (rows past the tile's pixels reuse the last
+        // one: their A rows are computed but never stored)
+        const int rr = min(r, valid_px - 1);
+        const int g = rr / (rows_here * p.Wo);
+        const int rem = rr - g * rows_here * p.Wo;
+        const int oyl = rem / p.Wo, ox = rem - oyl * p.Wo;
+        const int px_off = g * plane_in + oyl * p.stride * st.Wp + ox * p.stride;
+        // Stage channel block kb into buffer b: for each (channel, image) one warp copies the
+        // input rows of the window that lie inside the image -- nr rows of wcols floats -- into
+        // the interior of that channel's padded window; the padding was zeroed at tile start and
+        // is never written. Then the block's weights.
+        const int iy_lo = max(0, iy_start), iy_hi = min(p.H - 1, iy_start + st.R_in - 1);
+        const int nr = iy_hi - iy_lo + 1;
+        const int span = nr * st.wcols;
+        const int row0 = iy_lo - iy_start;
+        auto stage = [&](int kb, uint32_t b) {
+            float *dx = sx + b * st.x_floats;
+            for (int ch = warp; ch < 64; ch += kDwPwThreads / 32) {
+                const int c = kb * 64 + ch;
+                if (c >= p.C) break;   // channels past C are never used
+                for (int gi = 0; gi < imgs_here; ++gi) {
+                    const float *src = x + ((static_cast<long long>(n0 + gi) * p.C + c) * p.H + iy_lo) * p.W;
+                    float *dst = dx + ((ch * st.G + gi) * st.R_in + row0) * st.Wp + p.pad;
+                    for (int k = lane; k < span; k += 32) {
+                        const int rr = fdiv(k, st.div_wcols);
+                        const int cc = k - rr * st.wcols;
+                        cp_async_f32_zfill(smem_u32(dst + rr * st.Wp + cc), src + rr * p.W + cc, true);
+                    }
+                }
+            }
+            float *dw = sw + b * st.w_floats;
+            for (int i = tid; i < 64 * KK; i += kDwPwThreads) {
+                const int ch = i / KK;
+                const int t = i - ch * KK;
+                const int c = kb * 64 + ch;
+                const bool ok = c < p.C;
+                cp_async_f32_zfill(smem_u32(dw + ch * KKP + t), w + (ok ? c * KK + t : 0), ok);
+            }
+        };
+        // both input buffers start the tile as zeros (the padding of every window); the
+        // previous tile's reads, and a cluster reduction's use of this area, are finished
+        {
+            float4 *z = reinterpret_cast<float4 *>(sx);
+            for (int i = tid; i < (2 * st.x_floats) / 4; i += kDwPwThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+        int kcount = 0;
+        int kb = static_cast<int>(rank);
+        if (!dead && kb < p.num_kblk) stage(kb, stg & 1u);
+        cp_async_commit();
+        for (; kb < p.num_kblk && !dead; kb += S, ++it, ++kcount, ++stg) {
+            const uint32_t s = it & 1u, use = it >> 1;
+            const bool w_ok = it < 2 || mbar_wait(afree(s), (use - 1u) & 1u);
+            if (__syncthreads_or(!w_ok || *abort_flag)) { dead = true; break; }
+            if (tid == 0) {
+                mbar_arrive_expect_tx(bfull(s), static_cast<uint32_t>(p.n_boxes * kDwPwBox));
+                for (int h = 0; h < p.n_boxes; ++h)
+                    tma_load_3d(sB + s * st.b_bytes + h * kDwPwBox, &tmF, bfull(s), h * 64, kb * 64, 0);
+            }
+            // the next block's window goes in while this one is computed
+            if (kb + S < p.num_kblk) stage(kb + S, (stg + 1u) & 1u);
+            cp_async_commit();
+            cp_async_wait<1>();
+            __syncthreads();
+            const float *bx = sx + (stg & 1u) * st.x_floats + px_off;
+            const float *bw = sw + (stg & 1u) * st.w_floats;
+            const uint32_t arow = sA + s * kDwPwA + r * 128;
+#pragma unroll 1
+            for (int j = 0; j < 16; j += CG) {
+                float v[CG];
+#pragma unroll
+                for (int u = 0; u < CG; ++u) {
+                    const int ch = quarter * 16 + j + u;
+                    const float *xp = bx + ch * (st.G * plane_in);
+                    const float4 *w4 = reinterpret_cast<const float4 *>(bw + ch * KKP);
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int t4 = 0; t4 < KKP / 4; ++t4) {
+                        const float4 wv = w4[t4];
+                        const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int t = 4 * t4 + e;
+                            if (t < KK) {
+                                const float xv = xp[(t / KC) * p.dil * st.Wp + (t % KC) * p.dil];
+                                acc = dw_tap<MODE>(acc, ws[e], xv);
+                            }
+                        }
+                    }
+                    const int c = kb * 64 + ch;
+                    if (c < p.C)
+                        acc = p.b_dw ? dw_finish<MODE, true>(acc, __ldg(p.b_dw + c)) : dw_finish<MODE, false>(acc, 0.0f);
+                    else
+                        acc = 0.0f;
+                    v[u] = acc;
+                }
+                const int cl = quarter * 16 + j;
+                const uint32_t addr =
+                    arow + ((static_cast<uint32_t>(cl >> 3) ^ static_cast<uint32_t>(r & 7)) << 4) + (cl & 7) * 2;
+                if constexpr (CG == 4)
+                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(pack_bf16x2(v[0], v[1])),
+                                 "r"(pack_bf16x2(v[2], v[3]))
+                                 : "memory");
+                else
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(pack_bf16x2(v[0], v[1])) : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                if (mbar_wait(bfull(s), use & 1u)) {
+                    tc_fence_after();
+                    const uint32_t a0 = sA + s * kDwPwA, b0 = sB + s * st.b_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, kDwPwBox, 1024);
+                        umma_f16_ss(tmem, ad, bd, p.idesc, (kcount | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(afree(s));
+                } else {
+                    atomicOr(status, kStatusTimeout);
+                    *abort_flag = 1;
+                }
+            }
+        }
+        cp_async_wait<0>();   // no copy of this tile outlives it
+        if (!dead) {
+            if (tid == 0) umma_commit(accf);
+            const bool a_ok = mbar_wait(accf, ntile & 1u);
+            if (__syncthreads_or(!a_ok || *abort_flag)) dead = true;
+        }
+        tc_fence_after();
+        const bool have = !dead && kcount > 0;
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int nch = p.n_mma >> 4;
+        // A-tile row -> (image, output pixel); rows past the tile's pixels are not stored
+        auto row_pixel = [&](int rw, int &n_out, int &pix_out) {
+            const int gg = rw / (rows_here * p.Wo);
+            const int rm = rw - gg * rows_here * p.Wo;
+            n_out = n0 + gg;
+            pix_out = oy0 * p.Wo + rm;
+        };
+        if (S == 1) {
+            if (have) {
+                const bool ve = row < valid_px;
+                int ne = 0, pix = 0;
+                if (ve) row_pixel(row, ne, pix);
+                float *yrow = y + static_cast<long long>(ne) * p.Cout * p.HoWo + pix;
+                for (int cb = warp >> 2; cb < nch; cb += kDwPwThreads / 128) {
+                    uint32_t t[16];
+                    tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + cb * 16, t);
+                    tmem_wait_ld();
+                    if (ve) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            const int o = cb * 16 + jj;
+                            if (o < p.Cout) {
+                                float val = __uint_as_float(t[jj]);
+                                if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
+                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                            }
+                        }
+                    }
+                }
+            }
+        } else {
+            // channel-split reduction through distributed shared memory (see dwpw_kernel); the
+            // receive slots reuse the A and filter stages
+            cluster_sync_all();
+            for (int cb = warp >> 2; cb < nch; cb += kDwPwThreads / 128) {
+                uint32_t t[16];
+                if (have) {
+                    tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + cb * 16, t);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) t[jj] = 0u;
+                }
+                const uint32_t owner = static_cast<uint32_t>(cb % S);
+                const uint32_t slot_off = ((rank * p.owned + static_cast<uint32_t>(cb / S)) * 128u + row) * 64u;
+                const uint32_t dst = map_rank(sA + slot_off, owner);
+#pragma unroll
+                for (int jj = 0; jj < 16; jj += 4) st_cluster_v4(dst + jj * 4, t[jj], t[jj + 1], t[jj + 2], t[jj + 3]);
+            }
+            cluster_sync_all();
+            if (!dead) {
+                const int rr2 = tid & 127, cq = tid >> 7;
+                if (rr2 < valid_px) {
+                    int ne, pix;
+                    row_pixel(rr2, ne, pix);
+                    float *yrow = y + static_cast<long long>(ne) * p.Cout * p.HoWo + pix;
+                    for (int lc = 0; lc * S + static_cast<int>(rank) < nch; ++lc) {
+                        const int cb = lc * S + static_cast<int>(rank);
+                        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                        for (int sl = 0; sl < S; ++sl) {
+                            const float4 v = *reinterpret_cast<const float4 *>(
+                                smem + ((sl * p.owned + lc) * 128 + rr2) * 64 + cq * 16);
+                            acc[0] = __fadd_rn(acc[0], v.x);
+                            acc[1] = __fadd_rn(acc[1], v.y);
+                            acc[2] = __fadd_rn(acc[2], v.z);
+                            acc[3] = __fadd_rn(acc[3], v.w);
+                        }
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int o = cb * 16 + cq * 4 + jj;
+                            if (o < p.Cout) {
+                                float val = acc[jj];
+                                if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
+                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                            }
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+    if (tid == 0) {
+        umma_commit(done);
+        if (!mbar_wait(done, 0)) atomicOr(status, kStatusTimeout);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, p.tmem_cols);
+}
+
 }  // namespace convb200

@@ -40,6 +40,9 @@ def _run(cb, case, x, w, bd, F, bp, mode):
     return out, kernel
 
 
+KERNELS = ("dwpw_kernel", "dwpw_staged_kernel")
+
+
 def _tol(C):
     return (C + 2) * 2.0 ** -23
 
@@ -58,6 +61,7 @@ CASES = [
     (3, 32, 5, 1, 1, 0, 1, 32, 0, True),        # 1x1 depthwise (a per-channel scale and bias)
     (5, 24, 1, 3, 1, 1, 1, 16, 0, True),        # 1x1 images: every tap but the centre is padding
     (1, 200, 3, 3, 2, 1, 1, 200, 1, True),      # 2x2 output, one partial tile, ragged Cout chunk
+    (2, 64, 12, 3, 2, 0, 1, 64, 0, True),       # stride 2, no padding: the last input column unused
 ]
 
 
@@ -71,7 +75,7 @@ def test_block_matches_oracle(cb, c):
     case = workloads.DwPwCase("t", N, C, H, H, K, s, p, d, Cout, bias, seed=C + K + Cout)
     x, w, bd, F, bp = workloads.dwpw_inputs(case)
     y, kernel = _run(cb, case, x, w, bd, F, bp, mode)
-    assert kernel == "dwpw_kernel"
+    assert kernel in KERNELS
     ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, s, p, d, mode)
     assert y.shape == ref.shape
     assert np.all(np.isfinite(y))
@@ -104,7 +108,7 @@ def test_full_size_blocks_sampled(cb, case):
     x, w, bd, F, bp = workloads.dwpw_inputs(case)
     for mode in (0, 1):
         y, kernel = _run(cb, case, x, w, bd, F, bp, mode)
-        assert kernel == "dwpw_kernel" and np.all(np.isfinite(y))
+        assert kernel in KERNELS and np.all(np.isfinite(y))
         idx = (workloads.splitmix64(7 + mode, 20000) % np.uint64(y.size)).astype(np.int64)
         ref, absum = oracle.dwpw_points(x, w, bd, workloads.bf16_to_f32(F), bp, idx, case.stride, case.pad, case.dil,
                                         mode)
@@ -120,7 +124,7 @@ def test_channel_split_across_a_cluster(cb, split, monkeypatch):
     x, w, bd, F, bp = workloads.dwpw_inputs(case)
     y, kernel = _run(cb, case, x, w, bd, F, bp, 0)
     y2, _ = _run(cb, case, x, w, bd, F, bp, 0)
-    assert kernel == "dwpw_kernel" and np.array_equal(y, y2)
+    assert kernel in KERNELS and np.array_equal(y, y2)
     ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, 1, 1, 1, 0)
     assert np.all(np.abs(y - ref) <= _tol(case.C) * absum)
 
@@ -134,3 +138,50 @@ def test_split_identity_mixing_is_exact(cb, monkeypatch):
     y, _ = _run(cb, case, x, w, bd, F, None, 1)
     dref = oracle.depthwise(x, w, bd, mult=1, stride=1, pad=2, dil=1, mode=1)
     assert np.array_equal(y, workloads.bf16_to_f32(workloads.bf16_bits(dref)).astype(np.float64))
+
+
+@pytest.mark.parametrize("c", [CASES[0], CASES[2], CASES[3], CASES[4], CASES[10]], ids=_ids)
+def test_staged_and_flat_kernels_agree(cb, c, monkeypatch):
+    # shapes the staged kernel takes by default, run on both kernels: each meets the bar
+    N, C, H, K, s, p, d, Cout, mode, bias = c
+    case = workloads.DwPwCase("t", N, C, H, H, K, s, p, d, Cout, bias, seed=C + 2 * K)
+    x, w, bd, F, bp = workloads.dwpw_inputs(case)
+    ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, s, p, d, mode)
+    for kern, name in (("staged", "dwpw_staged_kernel"), ("flat", "dwpw_kernel")):
+        monkeypatch.setenv("CONV_B200_DWPW_KERNEL", kern)
+        y, kernel = _run(cb, case, x, w, bd, F, bp, mode)
+        assert kernel == name
+        assert np.all(np.abs(y - ref) <= _tol(C) * absum)
+
+
+@pytest.mark.parametrize("kern", ["staged", "flat"])
+@pytest.mark.parametrize("split", ["1", "4"])
+def test_identity_mixing_exact_on_both_kernels(cb, kern, split, monkeypatch):
+    monkeypatch.setenv("CONV_B200_DWPW_KERNEL", kern)
+    monkeypatch.setenv("CONV_B200_DWPW_SPLIT", split)
+    # F = the first 128 columns of I: output o < 128 is depthwise channel o, exactly
+    case = workloads.DwPwCase("t", 6, 256, 7, 7, 5, 1, 2, 1, 128, True, seed=13)
+    x, w, bd, _, _ = workloads.dwpw_inputs(case)
+    F = workloads.bf16_bits(np.eye(256, 128, dtype=np.float32))
+    y, kernel = _run(cb, case, x, w, bd, F, None, 0)
+    assert kernel == ("dwpw_staged_kernel" if kern == "staged" else "dwpw_kernel")
+    dref = oracle.depthwise(x, w, bd, mult=1, stride=1, pad=2, dil=1, mode=0)[:, :128]
+    assert np.array_equal(y, workloads.bf16_to_f32(workloads.bf16_bits(dref)).astype(np.float64))
+
+
+@pytest.mark.parametrize("kern", ["staged", "flat"])
+def test_split_is_live(cb, kern, monkeypatch):
+    # a 4-way split adds four partial sums where one CTA accumulates all blocks in order: over a
+    # million outputs the two orders must differ somewhere (both within the bar), which shows
+    # the split really ran
+    monkeypatch.setenv("CONV_B200_DWPW_KERNEL", kern)
+    case = workloads.DwPwCase("t", 8, 672, 14, 14, 3, 1, 1, 1, 112, True, seed=14)
+    x, w, bd, F, bp = workloads.dwpw_inputs(case)
+    ys = {}
+    for split in ("1", "4"):
+        monkeypatch.setenv("CONV_B200_DWPW_SPLIT", split)
+        ys[split], _ = _run(cb, case, x, w, bd, F, bp, 0)
+    ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, 1, 1, 1, 0)
+    for y in ys.values():
+        assert np.all(np.abs(y - ref) <= _tol(case.C) * absum)
+    assert not np.array_equal(ys["1"], ys["4"])
