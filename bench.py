@@ -88,6 +88,7 @@ KERNEL_SOURCES = {
     "depthwise_reg_kernel": ("depthwise_reg.cuh", "depthwise.cuh"),
     "depthwise_kernel": ("depthwise.cuh",),
     "dwpw_kernel": ("dwpw.cuh", "dense_tc.cuh", "depthwise.cuh", "ptx.cuh"),
+    "dwpw_staged_kernel": ("dwpw.cuh", "dense_tc.cuh", "depthwise.cuh", "ptx.cuh"),
 }
 
 
