@@ -162,9 +162,9 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
         *abort_flag = 1;
     };
     // tile -> (group of this launch, 128-row block, BN-column block)
-    auto split = [&](int tile, int &g, int &mt, int &nt) {
-        g = NG == 1 ? 0 : tile / p.tiles_per_group;
-        const int rem = tile - g * p.tiles_per_group;
+    auto split = [&](int tile, int &grp, int &mt, int &nt) {
+        grp = NG == 1 ? 0 : tile / p.tiles_per_group;
+        const int rem = tile - grp * p.tiles_per_group;
         mt = rem / p.num_ntiles;
         nt = rem - mt * p.num_ntiles;
     };
@@ -174,10 +174,10 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
         // The whole warp walks the loop (it stays converged); lane 0 issues.
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
-            int g, mt, nt;
-            split(tile, g, mt, nt);
-            const CUtensorMap *tmX = &maps.x[g];
-            const CUtensorMap *tmF = &maps.f[g];
+            int grp, mt, nt;
+            split(tile, grp, mt, nt);
+            const CUtensorMap *tmX = &maps.x[grp];
+            const CUtensorMap *tmF = &maps.f[grp];
             const int m0 = mt * Cfg::BM;
             const int n0 = nt * BN;
             const int img = m0 / p.HoWo;
@@ -286,8 +286,8 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
             const bool ok = mbar_wait_warp(accf_bar(b), aph);
             if (!ok) { if (lane == 0) fail(); break; }
             tc_fence_after();
-            int g, mt, nt;
-            split(tile, g, mt, nt);
+            int grp, mt, nt;
+            split(tile, grp, mt, nt);
             const int m0 = mt * Cfg::BM;
             const int n0 = nt * BN;
             // the staging buffer is free once the previous tile's stores have read it
@@ -302,7 +302,7 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                 tmem_wait_ld();
                 if (p.bias) {   // one fp32 addition per output, before the single rounding
                     const int c0 = n0 + h * 64;
-                    const float *bg = p.bias + static_cast<long long>(g) * p.ncols;
+                    const float *bg = p.bias + static_cast<long long>(grp) * p.ncols;
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -338,7 +338,7 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                 if (row0 < p.M) {
 #pragma unroll
                     for (int h = 0; h < BN / 64; ++h)
-                        if (n0 + h * 64 < p.ncols) tma_store_2d(&maps.y[g], stage_s + h * 4096, n0 + h * 64, row0);
+                        if (n0 + h * 64 < p.ncols) tma_store_2d(&maps.y[grp], stage_s + h * 4096, n0 + h * 64, row0);
                     bulk_commit_group();
                 }
             }

@@ -144,7 +144,7 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
         fence_barrier_init();
         prefetch_tensormap(&tmF);
     }
-    if (KC > 0) {   // the depthwise weights, once per CTA, as rows of KKP floats
+    if constexpr (KC > 0) {   // the depthwise weights, once per CTA, as rows of KKP floats
         for (int i = tid; i < p.C * KK; i += kDwPwThreads) {
             const int c = i / KK;
             sW[c * KKP + (i - c * KK)] = __ldg(w + i);
@@ -468,7 +468,6 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
                    float *__restrict__ y, const DwPwParams p, const DwPwStage st, unsigned int *status) {
     constexpr int KK = KC * KC;
     constexpr int KKP = (KK + 3) & ~3;
-    constexpr int CG = KC <= 3 ? 4 : 2;   // channels computed together
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -512,11 +511,7 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    const int r = tid & 127;       // A-tile row (pixel of the tile) of the depthwise stage
-    const int quarter = tid >> 7;  // channels quarter*16 .. +15 of each block
     const int plane_in = st.R_in * st.Wp;           // staged floats of one image of one channel
-    const int rows_per_ch = st.G * st.R_in;
-    const int tile_px = st.G * st.RB * p.Wo;        // A rows a full tile fills
     uint32_t it = 0, ntile = 0, stg = 0;
     bool dead = false;
     for (int tile = cluster; tile < p.num_tiles; tile += num_clusters, ++ntile) {
@@ -527,13 +522,7 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
         const int imgs_here = min(st.G, st.N - n0);
         const int valid_px = imgs_here * rows_here * p.Wo;   // (image mode: rows_here = Ho)
         const int iy_start = oy0 * p.stride - p.pad;
-        // this thread's pixel in the staged window (rows past the tile's pixels reuse the last
-        // one: their A rows are computed but never stored)
-        const int rr = min(r, valid_px - 1);
-        const int g = rr / (rows_here * p.Wo);
-        const int rem = rr - g * rows_here * p.Wo;
-        const int oyl = rem / p.Wo, ox = rem - oyl * p.Wo;
-        const int px_off = g * plane_in + oyl * p.stride * st.Wp + ox * p.stride;
+        const FastDiv div_vpx = make_fastdiv(static_cast<uint32_t>(valid_px));
         // Stage channel block kb into buffer b: for each (channel, image) one warp copies the
         // input rows of the window that lie inside the image -- nr rows of wcols floats -- into
         // the interior of that channel's padded window; the padding was zeroed at tile start and
@@ -591,28 +580,50 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
             cp_async_commit();
             cp_async_wait<1>();
             __syncthreads();
-            const float *bx = sx + (stg & 1u) * st.x_floats + px_off;
+            // Depthwise outputs of the tile's valid pixels only, as (pixel, channel pair) units
+            // spread evenly over the 512 threads (consecutive threads: consecutive pixels of one
+            // channel pair); A rows past the valid pixels are never written (their MMA rows are
+            // never stored).
+            const float *bxs = sx + (stg & 1u) * st.x_floats;
             const float *bw = sw + (stg & 1u) * st.w_floats;
-            const uint32_t arow = sA + s * kDwPwA + r * 128;
+            const uint32_t a_stage = sA + s * kDwPwA;
+            const int nunits = valid_px * 32;
 #pragma unroll 1
-            for (int j = 0; j < 16; j += CG) {
-                float v[CG];
+            for (int unit = tid; unit < nunits; unit += kDwPwThreads) {
+                const int cp2 = fdiv(unit, div_vpx);          // channel pair 0..31
+                const int px = unit - cp2 * valid_px;         // pixel of the tile
+                const int gg = st.G > 1 ? fdiv(px, p.div_howo) : 0;
+                const int remp = px - gg * p.HoWo;
+                const int oyl2 = fdiv(remp, p.div_wo), ox2 = remp - oyl2 * p.Wo;
+                const float *bx = bxs + gg * plane_in + oyl2 * p.stride * st.Wp + ox2 * p.stride;
+                float v[2];
 #pragma unroll
-                for (int u = 0; u < CG; ++u) {
-                    const int ch = quarter * 16 + j + u;
+                for (int u = 0; u < 2; ++u) {
+                    const int ch = 2 * cp2 + u;
                     const float *xp = bx + ch * (st.G * plane_in);
                     const float4 *w4 = reinterpret_cast<const float4 *>(bw + ch * KKP);
                     float acc = 0.0f;
+                    if (p.dil == 1) {   // taps at immediate offsets from each window row
 #pragma unroll
-                    for (int t4 = 0; t4 < KKP / 4; ++t4) {
-                        const float4 wv = w4[t4];
-                        const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
+                        for (int t4 = 0; t4 < KKP / 4; ++t4) {
+                            const float4 wv = w4[t4];
+                            const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int t = 4 * t4 + e;
-                            if (t < KK) {
-                                const float xv = xp[(t / KC) * p.dil * st.Wp + (t % KC) * p.dil];
-                                acc = dw_tap<MODE>(acc, ws[e], xv);
+                            for (int e = 0; e < 4; ++e) {
+                                const int t = 4 * t4 + e;
+                                if (t < KK) acc = dw_tap<MODE>(acc, ws[e], xp[(t / KC) * st.Wp + (t % KC)]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int t4 = 0; t4 < KKP / 4; ++t4) {
+                            const float4 wv = w4[t4];
+                            const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int t = 4 * t4 + e;
+                                if (t < KK)
+                                    acc = dw_tap<MODE>(acc, ws[e], xp[(t / KC) * p.dil * st.Wp + (t % KC) * p.dil]);
                             }
                         }
                     }
@@ -623,15 +634,10 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
                         acc = 0.0f;
                     v[u] = acc;
                 }
-                const int cl = quarter * 16 + j;
-                const uint32_t addr =
-                    arow + ((static_cast<uint32_t>(cl >> 3) ^ static_cast<uint32_t>(r & 7)) << 4) + (cl & 7) * 2;
-                if constexpr (CG == 4)
-                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(pack_bf16x2(v[0], v[1])),
-                                 "r"(pack_bf16x2(v[2], v[3]))
-                                 : "memory");
-                else
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(pack_bf16x2(v[0], v[1])) : "memory");
+                const int cl = 2 * cp2;
+                const uint32_t addr = a_stage + px * 128 +
+                                      ((static_cast<uint32_t>(cl >> 3) ^ static_cast<uint32_t>(px & 7)) << 4) + (cl & 7) * 2;
+                asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(pack_bf16x2(v[0], v[1])) : "memory");
             }
             fence_proxy_async_smem();
             __syncthreads();
