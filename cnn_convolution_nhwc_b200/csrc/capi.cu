@@ -995,12 +995,7 @@ DwPwStagePlan plan_dwpw_staged(const DwPwParams &p, int N) {
     if (p.K != 3 && p.K != 5) return pl;
     DwPwStage &st = pl.st;
     st.N = N;
-    // Images of at most 128 outputs would be staged whole, G per tile; that form measured slower
-    // than the flat kernel (7x7, 960 channels: 189 vs 89 us), so it is taken only when forced.
-    const char *kforce = env("CONV_B200_DWPW_KERNEL");
-    const bool force_staged = kforce && std::strcmp(kforce, "staged") == 0;
     if (p.HoWo <= 128) {   // whole images per tile
-        if (!force_staged) return pl;
         st.G = 128 / p.HoWo;
         if (st.G > N) st.G = N;
         st.RB = p.Ho;

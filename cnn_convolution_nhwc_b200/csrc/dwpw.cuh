@@ -428,9 +428,8 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
 
 // ---------------------------------------------------------------------------------------
 // Staged variant (3x3 and 5x5). Tiles follow the image grid instead of the flattened pixel
-// order: a band of RB output rows of one image (RB * Wo <= 128, the default for images of more
-// than 128 outputs) or G whole images (G = floor(128 / (Ho*Wo)); measured slower than
-// dwpw_kernel for 7x7 images, so the host takes it only when asked). Per channel block the CTA copies, with
+// order: G whole images (G = floor(128 / (Ho*Wo)) when an image has at most 128 outputs) or a
+// band of RB output rows of one image (RB * Wo <= 128). Per channel block the CTA copies, with
 // cp.async, the zero-padded input window of the tile -- 64 channels x G images x R_in rows x Wp
 // columns, positions outside the image written as +0 by the copy's zero fill -- and the block's
 // weights into shared memory, one block ahead of the compute (two buffers). The depthwise taps
