@@ -56,3 +56,18 @@ def test_grouped_and_conv1d_case_shapes():
     assert s1.f_shape == (1, 3, 80, 512) and (s1.Ho, s1.Wo) == (1, 3000)
     assert s2.f_shape == (1, 3, 512, 512) and (s2.Ho, s2.Wo) == (1, 1500)
     assert workloads.DENSE_S2.square and workloads.DENSE_S2.f_shape == (3, 3, 64, 128)
+
+
+def test_depthwise_pointwise_blocks():
+    # algorithmic bytes: x, y (float32), depthwise weights and both biases (float32), pointwise
+    # weights (bf16); the intermediate is not counted
+    c = workloads.DWPW_BLOCKS[0]
+    assert (c.Ho, c.Wo) == (14, 14)
+    assert c.bytes == 4 * (64 * 672 * 196 + 672 * 9 + 64 * 112 * 196) + 2 * 672 * 112 + 4 * (672 + 112)
+    assert c.flops == 2 * 64 * 196 * 672 * 9 + 2 * 64 * 196 * 672 * 112
+    x, w, bd, F, bp = workloads.dwpw_inputs(workloads.DwPwCase("t", 2, 8, 5, 5, 3, 1, 1, 1, 16, True, seed=3))
+    assert x.shape == (2, 8, 5, 5) and w.shape == (8, 3, 3) and F.shape == (8, 16) and F.dtype.name == "uint16"
+    assert bd.shape == (8,) and bp.shape == (16,)
+    assert float(np.abs(x).max()) <= 1.0
+    x2, *_ = workloads.dwpw_inputs(workloads.DwPwCase("t", 2, 8, 5, 5, 3, 1, 1, 1, 16, True, seed=3))
+    assert np.array_equal(x, x2)   # seeded: the same bits every time
