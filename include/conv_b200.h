@@ -39,6 +39,9 @@
  *  - A device-side wait that exceeds its time limit (about one second) makes the kernel
  *    stop, record CONV_ERR_DEVICE_TIMEOUT in a per-process device status word and return;
  *    read it with conv_device_status().
+ *  - The first call of a kernel (and, for dwpw_fwd, of a shape) on a device raises that
+ *    kernel's shared-memory limit and asks the runtime how many thread-block clusters fit;
+ *    make that first call outside CUDA-graph stream capture. Later calls only launch.
  */
 #ifndef CONV_B200_H
 #define CONV_B200_H
