@@ -1472,17 +1472,17 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
         }
         if (kforce && std::strcmp(kforce, "staged") == 0) return CONV_ERR_UNSUPPORTED;
     }
-    // K = 3 and K = 5 stage the depthwise weights in shared memory when they fit; other filter
-    // sizes (or very many channels) read them from global memory
-    const bool staged = (K == 3 || K == 5) && 4LL * C * dwpw_kkp(K) <= kDwPwMaxSmem - kDwPwFixed;
-    p.w_floats = staged ? C * dwpw_kkp(K) : 0;
+    // The flat kernel: for K = 3 and K = 5 it keeps the depthwise weights in shared memory when
+    // they fit; other filter sizes (or very many channels) read them from global memory.
+    const bool w_in_smem = (K == 3 || K == 5) && 4LL * C * dwpw_kkp(K) <= kDwPwMaxSmem - kDwPwFixed;
+    p.w_floats = w_in_smem ? C * dwpw_kkp(K) : 0;
     if (mode == DW_EXACT) {
-        if (staged && K == 3) return launch_dwpw<0, 3>(x, w_dw, tmF, y, p, force_split, stream, d, 51);
-        if (staged && K == 5) return launch_dwpw<0, 5>(x, w_dw, tmF, y, p, force_split, stream, d, 52);
+        if (w_in_smem && K == 3) return launch_dwpw<0, 3>(x, w_dw, tmF, y, p, force_split, stream, d, 51);
+        if (w_in_smem && K == 5) return launch_dwpw<0, 5>(x, w_dw, tmF, y, p, force_split, stream, d, 52);
         return launch_dwpw<0, 0>(x, w_dw, tmF, y, p, force_split, stream, d, 53);
     }
-    if (staged && K == 3) return launch_dwpw<1, 3>(x, w_dw, tmF, y, p, force_split, stream, d, 54);
-    if (staged && K == 5) return launch_dwpw<1, 5>(x, w_dw, tmF, y, p, force_split, stream, d, 55);
+    if (w_in_smem && K == 3) return launch_dwpw<1, 3>(x, w_dw, tmF, y, p, force_split, stream, d, 54);
+    if (w_in_smem && K == 5) return launch_dwpw<1, 5>(x, w_dw, tmF, y, p, force_split, stream, d, 55);
     return launch_dwpw<1, 0>(x, w_dw, tmF, y, p, force_split, stream, d, 56);
 }
 
