@@ -1,25 +1,28 @@
-"""Benchmark: dense NHWC convolution (bf16, N=32, 56x56, 64->64, K=3) on B200, one JSON line.
+"""Benchmark: dense NHWC convolution (bf16, N=64, 112x112, 128->128, K=5) on B200, one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extras]
                     [--workload NAME]
 
-A step is one forward dense convolution over one batch of 32 images (the hot path: tensor
-maps, TMA im2col gather, tcgen05 mainloop, epilogue) with inputs resident in HBM. Inputs and
-outputs rotate over enough buffer sets that their total exceeds twice the L2 size, so every
-step reads cold data. The steps are replayed from CUDA graphs captured around the C-ABI call
-and timed with CUDA events on the launching stream, bracketed by a barrier and a device
-synchronisation; the reported time is the maximum over ranks. Under torchrun every rank
-runs its own batch (weak scaling, no collective on the data path).
+A step is one forward dense convolution over one batch of 64 images (the hot path: tensor
+maps, TMA patch gather, tcgen05 mainloop, epilogue) with inputs resident in HBM; the default
+workload is the largest dense configuration. Inputs and outputs rotate over enough buffer sets
+that their total exceeds twice the L2 size, so every step reads cold data. The W warm-up steps
+and then the K timed steps each run from CUDA graphs captured around the C-ABI call that hold
+the steps back to back (one graph launch per 1000 steps), timed with CUDA events on the
+launching stream, bracketed by a barrier and a device synchronisation; the reported time is
+the maximum over ranks. Under torchrun every rank runs its own batch (weak scaling, no
+collective on the data path).
 
 Also reported: "e2e" -- the same metric through the public Python API with the inputs copied
 from pinned host memory and the output copied back inside the timed region; "roofline" for
-the dense kernel; "cpu_baseline" -- the CPU oracle timed on a bounded sample of the same
-workload (rank 0, N=1); and, unless --no-extras, the other configurations (pointwise, large
-dense, the depthwise sweep in both modes) as secondary measurements.
+the timed kernel; "cpu_baseline" -- the CPU oracle timed on a bounded sample of the same
+workload (rank 0, N=1); and, unless --no-extras, every other configuration (the dense 3x3 and
+pointwise layers, the general-geometry, grouped and Conv1D layers, the depthwise sweep in both
+modes, the fused depthwise-pointwise blocks) as one compact "extras" table at the end of the line.
 
 --impl reference times the CPU oracle itself on the same workload (rank 0 only).
 --workload selects another single configuration (for timing or profiling one kernel alone):
-"pointwise", "dense-large" or "dw-C<C>-K<K>-s<stride>-H<H>-exact|fast" from the depthwise sweep.
+"dense3x3", "pointwise", ... or "dw-C<C>-K<K>-s<stride>-H<H>-exact|fast" from the depthwise sweep.
 """
 from __future__ import annotations
 
@@ -43,11 +46,11 @@ import workloads  # noqa: E402
 
 METRIC = "dense conv TFLOP/s (% bf16 TC peak); depthwise GB/s (% HBM) on 1 B200"
 L2_BYTES = 126 * 1024 * 1024
-CASE = workloads.DENSE_3X3
+DEFAULT_WORKLOAD = "dense-large"
 
 
 def workload_table():
-    """Name -> (kind, case, mode). The default headline is the dense 3x3 configuration; the
+    """Name -> (kind, case, mode). The default headline is the large dense configuration; the
     others exist so any single kernel can be timed or profiled alone."""
     t = {"dense3x3": ("dense", workloads.DENSE_3X3, None),
          "pointwise": ("dense", workloads.DENSE_1X1, None),
@@ -103,18 +106,18 @@ def source_hash(kernel: str) -> str:
 
 
 def traffic_for(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources:
+    (read + write, read, write during the launch, note) or Nones."""
+    none = (None, None, None, None)
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(p):
-        return None
+    if not os.path.exists(p) or kernel not in KERNEL_SOURCES:
+        return none
     with open(p) as f:
         d = json.load(f)
-    if kernel not in KERNEL_SOURCES:
-        return None
     rec = d.get(kernel, {}).get(workload)
     if not rec or rec.get("source_hash") != source_hash(kernel):
-        return None
-    return rec.get("bytes_per_launch")
+        return none
+    return rec.get("bytes_per_launch"), rec.get("read"), rec.get("write"), rec.get("note")
 
 
 # ------------------------------------------------------------------------------------------
@@ -224,43 +227,62 @@ def rotating_sets(set_bytes: int) -> int:
     return max(1, math.ceil(2 * L2_BYTES / max(1, set_bytes)))
 
 
-def capture(fn_list):
-    """One CUDA graph per callable plus one graph running them all in order."""
+CHUNK = 1000   # launches per captured graph (longer runs replay it; one graph launch per CHUNK steps)
+
+
+class StepGraphs:
+    """CUDA graphs that launch exactly `n` C-ABI calls back to back on the current stream,
+    cycling over the rotating buffer sets: one graph of `chunk` calls (a multiple of the number
+    of sets, at most CHUNK) replayed n // chunk times, then one graph of the remaining calls.
+    The calls inside a graph follow each other with no host gap."""
+
+    def __init__(self, fns, n):
+        import torch
+        R = len(fns)
+        chunk = min(n, CHUNK)
+        if chunk >= R:
+            chunk -= chunk % R
+        self.q, r = divmod(n, chunk) if chunk else (0, 0)
+        self.main = self._graph(torch, fns, chunk) if chunk else None
+        self.tail = self._graph(torch, fns, r) if r else None
+
+    @staticmethod
+    def _graph(torch, fns, count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(count):
+                fns[i % len(fns)]()
+        return g
+
+    def replay(self):
+        for _ in range(self.q):
+            self.main.replay()
+        if self.tail is not None:
+            self.tail.replay()
+
+
+def eager_first_calls(fns):
+    """Each call once, eagerly and off any capture: the first call of a kernel sets its
+    shared-memory attribute and may query cluster occupancy, which stream capture forbids."""
     import torch
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        for fn in fn_list:   # eager warm-up off the capture
+        for fn in fns:
             fn()
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
-    singles = []
-    for fn in fn_list:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        singles.append(g)
-    cycle = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(cycle):
-        for fn in fn_list:
-            fn()
-    torch.cuda.synchronize()
-    return singles, cycle
 
 
-def replay(singles, cycle, steps: int):
-    R = len(singles)
-    q, r = divmod(steps, R)
-    for _ in range(q):
-        cycle.replay()
-    for i in range(r):
-        singles[i].replay()
-
-
-def time_graph_steps(singles, cycle, steps: int, warmup: int, dist=None, sampler=None):
-    """Replays `steps` steps; returns elapsed ms on the launching stream (max over ranks)."""
+def time_graph_steps(fns, steps: int, warmup: int, dist=None, sampler=None):
+    """Runs `warmup` untimed steps, then exactly `steps` timed steps from one captured graph
+    (see StepGraphs); returns the elapsed ms on the launching stream (max over ranks)."""
     import torch
-    replay(singles, cycle, warmup)
+    eager_first_calls(fns)
+    warm = StepGraphs(fns, warmup)
+    timed = StepGraphs(fns, steps)
+    torch.cuda.synchronize()
+    warm.replay()
     stream = torch.cuda.current_stream()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -270,7 +292,7 @@ def time_graph_steps(singles, cycle, steps: int, warmup: int, dist=None, sampler
     if sampler is not None:
         sampler.start()
     start.record(stream)
-    replay(singles, cycle, steps)
+    timed.replay()
     end.record(stream)
     torch.cuda.synchronize()
     if sampler is not None:
@@ -278,6 +300,7 @@ def time_graph_steps(singles, cycle, steps: int, warmup: int, dist=None, sampler
     if dist is not None:
         dist.barrier()
     ms = start.elapsed_time(end)
+    del warm, timed
     return dist.max(ms) if dist is not None else ms
 
 
@@ -398,10 +421,9 @@ def steps_fns(cb, torch, kind, case, mode, inputs):
 
 def time_case(cb, torch, kind, case, mode, inputs, steps, warmup, dist=None, sampler=None):
     fns, R, keep = steps_fns(cb, torch, kind, case, mode, inputs)
-    singles, cycle = capture(fns)
+    ms = time_graph_steps(fns, steps, warmup, dist, sampler)
     kernel = cb.conv_last_kernel()      # the dispatcher's choice for this workload
-    ms = time_graph_steps(singles, cycle, steps, warmup, dist, sampler)
-    del singles, cycle, keep
+    del keep
     return ms, R, kernel
 
 
@@ -525,7 +547,7 @@ def run_ours(args, dist):
         achieved = case.flops / (ms_step * 1e-3) / 1e12
         roof = {"kernel": kernel, "bound": "tensor", "achieved": round(achieved, 3), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": traffic_for(kernel, args.workload), "algorithmic_bytes": case.bytes,
+                **traffic_fields(kernel, args.workload), "algorithmic_bytes": case.bytes,
                 "algorithmic_flops": case.flops,
                 "hbm_frac": round(case.bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peaks_src}: bf16 burst (kernel timed alone); HBM copy {peaks['hbm_gbs']} GB/s"}
@@ -549,7 +571,7 @@ def run_ours(args, dist):
         achieved = case.bytes / (ms_step * 1e-3) / 1e9
         roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic_for(kernel, args.workload), "algorithmic_bytes": case.bytes,
+                **traffic_fields(kernel, args.workload), "algorithmic_bytes": case.bytes,
                 "GFLOP/s": round(case.flops / (ms_step * 1e-3) / 1e9, 1),
                 "peak_source": f"{peaks_src}: HBM copy"}
         dtype = "f32"
@@ -566,7 +588,8 @@ def run_ours(args, dist):
                    "mult": case.mult, "H": case.H, "W": case.W, "K": case.KH, "stride": case.stride,
                    "pad": case.pad, "dil": case.dil, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
     cfg.update({"l2": f"inputs larger than L2: {R} rotating buffer sets of {case.bytes / 1e6:.2f} MB",
-                "launch": "CUDA graph replay of the C-ABI call", "parallelism": f"replicas x{dist.world}"})
+                "launch": "CUDA graphs of the C-ABI call, the timed steps back to back (one graph launch per "
+                          f"{CHUNK} steps)", "parallelism": f"replicas x{dist.world}"})
     value = dist.world * work * args.steps / (ms * 1e-3) / scale
     e2e_value = dist.world * work / (e2e_ms * 1e-3) / scale
     line = {
@@ -577,39 +600,49 @@ def run_ours(args, dist):
         "e2e": {"value": round(e2e_value, 4), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4),
                 "path": "python binding -> C ABI, pinned host copies in the timed region"},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps,   # one library kernel per step (the comparison path adds a cuBLAS GEMM)
         "clocks": sampler.summary(),
         "device_status": cb.conv_status_string(status),
     }
-    if dist.world == 1 and not args.no_extras:
-        line["extras"] = extras(cb, torch, peaks, skip=args.workload)
     if dist.rank == 0 and dist.world == 1:
         line["cpu_baseline"] = cpu_baseline(kind, case, mode, host_np)
+    if dist.world == 1 and not args.no_extras:
+        # last, so that the end of the line (what a log tail keeps) holds every row
+        line["extras_format"] = ("workload: [kernel, us per launch, fraction of the bound's measured peak "
+                                 "(dense: bf16 burst TFLOP/s; depthwise and fused blocks: HBM GB/s), "
+                                 "dense only: fraction of HBM]")
+        line["extras"] = extras(cb, torch, peaks, skip=args.workload)
     return line
 
 
+def traffic_fields(kernel, workload):
+    """roofline.traffic (DRAM read + write of one launch, from the committed ncu summary taken on
+    the current sources, else null) and its parts. Output lines still in L2 when the kernel ends
+    are written to DRAM after it, so the write part can be below the output's size."""
+    total, read, write, note = traffic_for(kernel, workload)
+    out = {"traffic": total, "traffic_dram_read": read, "traffic_dram_write_in_launch": write}
+    if note:
+        out["traffic_note"] = note
+    return out
+
+
 def extras(cb, torch, peaks, skip):
-    out = {"dense": [], "depthwise": [], "dwpw": []}
+    """Every other workload, timed like the headline; one short row each (see extras_format)."""
+    out = {}
     for name, (kind, case, mode) in workload_table().items():
         if name == skip:
             continue
+        steps = 200 if case.flops < 1e11 else 40
+        inputs = dense_device_inputs(torch, case, 0) if kind == "dense" else device_inputs(torch, kind, case, 0)
+        ms, R, kernel = time_case(cb, torch, kind, case, mode, inputs, steps, 10)
+        ms /= steps
+        short = kernel.replace("_kernel", "")
+        gbs = case.bytes / (ms * 1e-3) / 1e9
         if kind == "dense":
-            steps = 200 if case.flops < 1e11 else 40
-            ms, R, kernel = time_case(cb, torch, kind, case, mode, dense_device_inputs(torch, case, 0), steps, 5)
-            ms /= steps
             tf = case.flops / (ms * 1e-3) / 1e12
-            out["dense"].append({"workload": name, "kernel": kernel, "ms": round(ms, 5), "TFLOP/s": round(tf, 2),
-                                 "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
-                                 "GB/s": round(case.bytes / (ms * 1e-3) / 1e9, 1),
-                                 "frac_hbm": round(case.bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                                 "rotating_sets": R})
+            out[name] = [short, round(ms * 1e3, 2), round(tf / peaks["bf16_tflops"], 3), round(gbs / peaks["hbm_gbs"], 3)]
         else:
-            ms, R, kernel = time_case(cb, torch, kind, case, mode, device_inputs(torch, kind, case, 0), 200, 20)
-            ms /= 200
-            gbs = case.bytes / (ms * 1e-3) / 1e9
-            out["depthwise" if kind == "depthwise" else "dwpw"].append({"workload": name, "kernel": kernel, "ms": round(ms, 5), "GB/s": round(gbs, 1),
-                                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                                     "GFLOP/s": round(case.flops / (ms * 1e-3) / 1e9, 1), "rotating_sets": R})
+            out[name] = [short, round(ms * 1e3, 2), round(gbs / peaks["hbm_gbs"], 3)]
     return out
 
 
@@ -680,10 +713,10 @@ def run_reference(args, dist):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50000)
-    ap.add_argument("--warmup", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="dense3x3", choices=sorted(workload_table()))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workload_table()))
     ap.add_argument("--no-extras", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -76,11 +76,31 @@ def _check(code: int, what: str) -> None:
         raise ConvError(code, what)
 
 
-def _stream(stream):
+def _stream(stream, device):
+    """The stream handle for a call on `device` (its current stream when None)."""
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream) and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _device(*tensors):
+    """The one CUDA device every given tensor (None skipped) lives on."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"all tensors must be on one CUDA device, got {sorted(map(str, devs))}")
+    return devs.pop()
+
+
+def _call(fn, what, tensors, stream, *args):
+    """Runs one C entry point with the tensors' device current (the library launches on the
+    current device) and its stream as the last argument."""
+    import torch
+    dev = _device(*tensors)
+    with torch.cuda.device(dev):
+        _check(fn(*args, _stream(stream, dev)), what)
 
 
 def _tensor(t, dtype, ndim, name):
@@ -114,7 +134,7 @@ def _dense(X, F, Y, stream, dtype, fn, what):
     elif tuple(Y.shape) != (N, H - K + 1, W - K + 1, Cout):
         raise ValueError("Y has the wrong shape")
     py = _tensor(Y, dtype, 4, "Y")
-    _check(fn(px, pf, py, N, H, W, Cin, Cout, K, _stream(stream)), what)
+    _call(fn, what, (X, F, Y), stream, px, pf, py, N, H, W, Cin, Cout, K)
     return Y
 
 
@@ -154,8 +174,8 @@ def conv2d_nhwc_fwd_ex(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, stream=N
     elif tuple(Y.shape) != (N, Ho, Wo, Cout):
         raise ValueError("Y has the wrong shape")
     py = _tensor(Y, torch.bfloat16, 4, "Y")
-    _check(lib.conv2d_nhwc_fwd_ex(px, pf, pb, py, N, H, W, Cin, Cout, K, stride, pad, dil, _stream(stream)),
-           "conv2d_nhwc_fwd_ex")
+    _call(lib.conv2d_nhwc_fwd_ex, "conv2d_nhwc_fwd_ex", (X, F, bias, Y), stream,
+          px, pf, pb, py, N, H, W, Cin, Cout, K, stride, pad, dil)
     return Y
 
 
@@ -194,8 +214,8 @@ def conv2d_nhwc_fwd_grouped(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, gro
     elif tuple(Y.shape) != (N, Ho, Wo, Cout):
         raise ValueError("Y has the wrong shape")
     py = _tensor(Y, torch.bfloat16, 4, "Y")
-    _check(lib.conv2d_nhwc_fwd_grouped(px, pf, pb, py, N, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups,
-                                       _stream(stream)), "conv2d_nhwc_fwd_grouped")
+    _call(lib.conv2d_nhwc_fwd_grouped, "conv2d_nhwc_fwd_grouped", (X, F, bias, Y), stream,
+          px, pf, pb, py, N, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups)
     return Y
 
 
@@ -219,9 +239,9 @@ def conv2d_nhwc_fwd_im2col(X, F, Y=None, workspace=None, stream=None):
     if Y is None:
         Y = torch.empty((N, H - K + 1, W - K + 1, Cout), dtype=torch.bfloat16, device=X.device)
     py = _tensor(Y, torch.bfloat16, 4, "Y")
-    _check(lib.conv2d_nhwc_fwd_im2col(px, pf, py, ctypes.c_void_p(workspace.data_ptr()),
-                                      workspace.numel() * workspace.element_size(), N, H, W, Cin, Cout, K,
-                                      _stream(stream)), "conv2d_nhwc_fwd_im2col")
+    _call(lib.conv2d_nhwc_fwd_im2col, "conv2d_nhwc_fwd_im2col", (X, F, Y, workspace), stream,
+          px, pf, py, ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
+          N, H, W, Cin, Cout, K)
     return Y
 
 
@@ -249,8 +269,8 @@ def depthwise_fwd(x, w, bias=None, y=None, stride=1, pad=0, dil=1, mode=DW_EXACT
     elif tuple(y.shape) != (N, Cout, Ho, Wo):
         raise ValueError("y has the wrong shape")
     py = _tensor(y, torch.float32, 4, "y")
-    _check(lib.depthwise_fwd(px, pw, pb, py, N, Cin, mult, H, W, KH, KW, stride, pad, dil, int(mode),
-                             _stream(stream)), "depthwise_fwd")
+    _call(lib.depthwise_fwd, "depthwise_fwd", (x, w, bias, y), stream,
+          px, pw, pb, py, N, Cin, mult, H, W, KH, KW, stride, pad, dil, int(mode))
     return y
 
 
@@ -287,8 +307,8 @@ def dwpw_fwd(x, w_dw, b_dw, F, b_pw=None, y=None, stride=1, pad=0, dil=1, mode=D
     elif tuple(y.shape) != (N, Cout, Ho, Wo):
         raise ValueError("y has the wrong shape")
     py = _tensor(y, torch.float32, 4, "y")
-    _check(lib.dwpw_fwd(px, pw, pbd, pf, pbp, py, N, C, H, W, K, stride, pad, dil, Cout, int(mode), _stream(stream)),
-           "dwpw_fwd")
+    _call(lib.dwpw_fwd, "dwpw_fwd", (x, w_dw, b_dw, F, b_pw, y), stream,
+          px, pw, pbd, pf, pbp, py, N, C, H, W, K, stride, pad, dil, Cout, int(mode))
     return y
 
 
@@ -297,11 +317,18 @@ def conv_last_kernel() -> str:
     return lib.conv_last_kernel().decode()
 
 
+def _current():
+    import torch
+    return torch.device("cuda", torch.cuda.current_device())
+
+
 def conv_selftest_wait_timeout(stream=None) -> int:
-    """Runs the bounded-wait diagnostic (about one second); returns the launch status."""
-    return lib.conv_selftest_wait_timeout(_stream(stream))
+    """Runs the bounded-wait diagnostic (about one second) on the current device; returns the
+    launch status."""
+    return lib.conv_selftest_wait_timeout(_stream(stream, _current()))
 
 
 def conv_device_status(stream=None, reset=False) -> int:
-    """Synchronises the stream and returns the device status word as a conv_status code."""
-    return lib.conv_device_status(_stream(stream), 1 if reset else 0)
+    """Synchronises the stream and returns the current device's status word as a conv_status
+    code."""
+    return lib.conv_device_status(_stream(stream, _current()), 1 if reset else 0)

@@ -12,7 +12,9 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstdio>
+#include <atomic>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "../../include/conv_b200.h"
@@ -73,7 +75,7 @@ struct DeviceState {
     bool ready = false;
     int num_sms = 0;
     unsigned int *status = nullptr;   // device address of g_conv_status on this device
-    unsigned long long attr_done[2] = {0, 0};   // bit per kernel whose shared-memory limit is raised
+    std::atomic<unsigned long long> attr_done[2] = {{0}, {0}};   // bit per kernel whose shared-memory limit is raised
     cublasHandle_t blas = nullptr;    // for the explicit-im2col comparison path, made on first use
     // clusters of a kernel that fit on the device at once, per (kernel bit, cluster size, shared
     // memory), asked once (outside any stream capture: the first call of a shape runs eagerly)
@@ -123,11 +125,35 @@ int device_state(DeviceState **out) {
 
 template <typename Kern>
 int ensure_smem_attr(DeviceState *d, unsigned bit, Kern kern, int bytes) {
-    if (d->attr_done[bit >> 6] & (1ull << (bit & 63))) return CONV_OK;
+    const unsigned long long mask = 1ull << (bit & 63);
+    if (d->attr_done[bit >> 6].load(std::memory_order_acquire) & mask) return CONV_OK;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return CONV_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_mu);
-    d->attr_done[bit >> 6] |= 1ull << (bit & 63);
+    d->attr_done[bit >> 6].fetch_or(mask, std::memory_order_release);
+    return CONV_OK;
+}
+
+// Every tensor of a call must be device memory of the current device (or managed memory): the
+// kernels launch on the current device, and a buffer of another GPU, or host memory, would be
+// read through the wrong mapping. Null pointers (absent biases) are skipped. While `stream` is
+// being captured into a CUDA graph the check is skipped (the capture records launches only;
+// the same call made eagerly beforehand is checked).
+int check_device_ptrs(cudaStream_t stream, std::initializer_list<const void *> ptrs) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return CONV_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return CONV_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ERR_CUDA;
+    for (const void *p : ptrs) {
+        if (!p) continue;
+        cudaPointerAttributes a{};
+        if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+            cudaGetLastError();   // clear the (non-sticky) error this query left behind
+            return CONV_ERR_INVALID_ARG;
+        }
+        if (a.type == cudaMemoryTypeManaged) continue;
+        if (a.type != cudaMemoryTypeDevice || a.device != dev) return CONV_ERR_INVALID_ARG;
+    }
     return CONV_OK;
 }
 
@@ -1038,18 +1064,10 @@ int launch_dwpw_staged(const float *x, const float *w, const CUtensorMap &tmF, f
     return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, pl.st, d->status), "dwpw_staged_kernel");
 }
 
-}  // namespace
-}  // namespace convb200
-
-using namespace convb200;
-
-extern "C" {
-
-int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
-                    cudaStream_t stream) {
-    if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 2)) return rc;
-    DeviceState *d = nullptr;
-    if (int rc = device_state(&d)) return rc;
+// Kernel choice and launch of the plain dense convolution (arguments already validated, the
+// device state taken).
+int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
+                cudaStream_t stream, DeviceState *d) {
     const char *force = env("CONV_B200_DENSE");
     // Tensor-core paths need 16-byte rows (Cin, Cout multiples of 8) and 16-byte aligned
     // tensors. The im2col tensor map is used only for inputs of at least 128 KiB.
@@ -1095,11 +1113,28 @@ int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, 
     return launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 2);
 }
 
+}  // namespace
+}  // namespace convb200
+
+using namespace convb200;
+
+extern "C" {
+
+int conv2d_nhwc_fwd(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
+                    cudaStream_t stream) {
+    if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 2)) return rc;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    if (int rc = check_device_ptrs(stream, {X, F, Y})) return rc;
+    return dense_plain(X, F, Y, N, H, W, Cin, Cout, K, stream, d);
+}
+
 int conv2d_nhwc_fwd_f32(const float *X, const float *F, float *Y, int N, int H, int W, int Cin, int Cout,
                         int K, cudaStream_t stream) {
     if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 4)) return rc;
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
+    if (int rc = check_device_ptrs(stream, {X, F, Y})) return rc;
     return launch_dense_direct(X, F, Y, N, H, W, Cin, Cout, DenseGeom::square(K), stream, d);
 }
 
@@ -1124,6 +1159,7 @@ int dense_general(const void *X, const void *F, void *Y, int N, int H, int W, in
         return CONV_ERR_INVALID_ARG;
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
+    if (int rc = check_device_ptrs(stream, {X, F, Y, g.bias})) return rc;
     const char *force = env("CONV_B200_DENSE");
     // Tensor cores through the TMA im2col unit: 16-byte channel rows per group (group bases
     // 16-byte aligned), 16-byte aligned tensors, and window corners and tap offsets inside the
@@ -1219,6 +1255,7 @@ int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspac
         return CONV_ERR_INVALID_ARG;
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
+    if (int rc = check_device_ptrs(stream, {X, F, Y, workspace})) return rc;
     {
         std::lock_guard<std::mutex> lock(g_mu);
         if (!d->blas && cublasCreate(&d->blas) != CUBLAS_STATUS_SUCCESS) return CONV_ERR_CUDA;
@@ -1271,6 +1308,7 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
         return CONV_ERR_INVALID_ARG;
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
+    if (int rc = check_device_ptrs(stream, {x, w, bias, y})) return rc;
 
     // Register-window kernel for the common shapes (CONV_B200_DW_KERNEL=smem forces the
     // shared-memory kernel, =reg requires the register kernel; tests).
@@ -1420,6 +1458,7 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
         return CONV_ERR_INVALID_ARG;
     DeviceState *d = nullptr;
     if (int rc = device_state(&d)) return rc;
+    if (int rc = check_device_ptrs(stream, {x, w_dw, b_dw, F, b_pw, y})) return rc;
     alignas(64) CUtensorMap tmF;
     {   // F: 3-D {Cout, C, 1}; a box is 64 channel rows x 64 outputs (rows past C and columns
         // past Cout read zeros)

@@ -32,6 +32,10 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller (for example allocated by
  *    PyTorch). Tensors are dense and contiguous in the stated layout. The library keeps no
  *    reference to them after the call returns and allocates no device memory per call.
+ *  - Kernels run on the CURRENT device (cudaGetDevice). Every tensor must be memory of that
+ *    device (or managed memory); a tensor of another GPU, or host memory, returns
+ *    CONV_ERR_INVALID_ARG. The check is made on every call except while `stream` is being
+ *    captured into a CUDA graph.
  *  - Calls are asynchronous on `stream` (0 = legacy default stream) and never synchronise.
  *    Outputs are fully overwritten. Inputs are read only. Outputs must not overlap inputs.
  *  - The return value is a conv_status; no exception or abort crosses the ABI. Argument

@@ -199,3 +199,13 @@ def test_im2col_path_rejects(ws, nbytes, code):
 ])
 def test_dwpw_rejects(args, code):
     assert cb.lib.dwpw_fwd(*args, None) == code
+
+
+def test_binding_requires_one_device():
+    # the binding makes the tensors' device current for the call and refuses a mix of devices
+    # (the kernels launch on the current device and would read another GPU's buffer through the
+    # wrong mapping)
+    import torch
+    with pytest.raises(ValueError, match="one CUDA device"):
+        cb._device(torch.empty(1), torch.empty(1, device="meta"))
+    assert cb._device(torch.empty(1), None, torch.empty(2)) == torch.device("cpu")

@@ -311,3 +311,34 @@ def test_plane_kernel(cb, shape):
         _compare(yp, x, w, b, 1, S, case.pad, 1, mode)
         yn = _gpu(cb, x, w, None, S, case.pad, 1, mode)          # no bias
         _compare(yn, x, w, None, 1, S, case.pad, 1, mode)
+
+
+# (N, C, H, K, S, kernel): the production kernels -- planes of 7x7 and 14x14 (a lane per
+# plane), rows that are 16-byte multiples (one TMA box with the padding zeros written by the
+# copy engine) and rows that are not (whole planes by cp.async into pre-zeroed buffers)
+NAN_RULE_SHAPES = [(2, 9, 7, 3, 1, "plane"), (1, 21, 7, 5, 1, "plane"), (2, 6, 14, 3, 2, "plane"),
+                   (1, 5, 14, 5, 1, "plane"), (2, 3, 16, 3, 1, "tma"), (1, 4, 28, 5, 1, "tma"),
+                   (2, 3, 20, 5, 2, "tma"), (1, 3, 14, 3, 1, "tma")]
+
+
+@pytest.mark.parametrize("shape", NAN_RULE_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + "-" + s[5])
+def test_padding_nan_rule_production_kernels(cb, shape):
+    # OneModel "Depthwise convolution", "What each output is": padding is a real zero that is
+    # multiplied, so an infinite weight meeting padding gives NaN, and exact mode rewrites every
+    # NaN result as 0x7FC00000; an input NaN with another payload must come out canonical too
+    N, C, H, K, S, kernel = shape
+    case = workloads.DepthwiseCase("nan", N, C, 1, H, H, K, K, S, (K - 1) // 2, 1, True, 19)
+    x, w, b = workloads.depthwise_inputs(case)
+    w = w.copy()
+    w[0, 0, 0] = np.inf                 # plane 0: top-left tap meets the top row and left column of padding
+    w[C - 1, K - 1, K - 1] = -np.inf    # last plane: bottom-right tap
+    x = x.copy()
+    x.reshape(-1)[H * H + 2 * H + 3] = np.frombuffer(struct.pack("<I", 0xFFC00001), np.float32)[0]   # plane 1
+    for mode in MODES:
+        y = _with_env("CONV_B200_DW_KERNEL", kernel, lambda: _gpu(cb, x, w, b, S, case.pad, 1, mode))
+        assert cb.conv_last_kernel() == f"depthwise_{kernel}_kernel"
+        _compare(y, x, w, b, 1, S, case.pad, 1, mode)
+        ref = oracle.depthwise(x, w, b, mult=1, stride=S, pad=case.pad, dil=1, mode=mode)
+        assert np.isnan(ref).any() and np.isinf(ref).any()    # the planted values reach the outputs
+        if mode == oracle.DW_EXACT:
+            assert set(_bits(y)[np.isnan(y)].tolist()) == {0x7FC00000}
