@@ -76,6 +76,10 @@ def _load():
         lib.oracle_conv2d_grouped.restype = I
         lib.oracle_conv2d_grouped_points.argtypes = [P, P, P, P, L, P, P] + [I] * 13
         lib.oracle_conv2d_grouped_points.restype = I
+        lib.oracle_conv2d_grouped_pads.argtypes = [P, P, P, P, P] + [I] * 16
+        lib.oracle_conv2d_grouped_pads.restype = I
+        lib.oracle_conv2d_grouped_pads_points.argtypes = [P, P, P, P, L, P, P] + [I] * 15
+        lib.oracle_conv2d_grouped_pads_points.restype = I
         lib.oracle_dwpw.argtypes = [P] * 7 + [I] * 10
         lib.oracle_dwpw.restype = I
         lib.oracle_dwpw_points.argtypes = [P] * 6 + [L, P, P] + [I] * 9
@@ -185,28 +189,51 @@ def _pair(v):
     return (v, v) if isinstance(v, int) else (int(v[0]), int(v[1]))
 
 
-def conv2d_grouped(X, F, bias=None, stride=1, pad=0, dil=1, groups=1):
-    """Grouped NHWC convolution with per-axis stride / padding / dilation ((h, w) pairs or one
-    int for both) and a KH x KW kernel, float64. X: [N, H, W, Cin]; F: [KH, KW, Cin/groups, Cout]
-    (output channel o uses input channels of group o // (Cout/groups)); bias: [Cout] or None.
-    Conv1D is H = KH = 1. Returns (Y, abssum), float64 [N, Ho, Wo, Cout]."""
-    X, F = _f32(X), _f32(F)
-    b = None if bias is None else _f32(bias)
+def _pads(pad):
+    """(top, bottom, left, right) from one int, an (h, w) pair, or ((top, bottom), (left, right))."""
+    if isinstance(pad, int):
+        return pad, pad, pad, pad
+    ph, pw = pad
+    (pt, pb) = (ph, ph) if isinstance(ph, int) else (int(ph[0]), int(ph[1]))
+    (pl, pr) = (pw, pw) if isinstance(pw, int) else (int(pw[0]), int(pw[1]))
+    return int(pt), int(pb), int(pl), int(pr)
+
+
+def _grouped_shape(X, F, bias, stride, pad, dil, groups):
     N, H, W, Cin = X.shape
     KH, KW, Cg, Cout = F.shape
-    (sh, sw), (ph, pw), (dh, dw) = _pair(stride), _pair(pad), _pair(dil)
+    (sh, sw), (dh, dw) = _pair(stride), _pair(dil)
+    pt, pb, pl, pr = _pads(pad)
     if groups < 1 or Cin % groups or Cout % groups or Cg * groups != Cin:
         raise ValueError("channels must split into the groups")
-    if b is not None and b.shape != (Cout,):
+    if bias is not None and bias.shape != (Cout,):
         raise ValueError("bias must have Cout entries")
-    Ho = (H + 2 * ph - (dh * (KH - 1) + 1)) // sh + 1
-    Wo = (W + 2 * pw - (dw * (KW - 1) + 1)) // sw + 1
+    Ho = (H + pt + pb - (dh * (KH - 1) + 1)) // sh + 1
+    Wo = (W + pl + pr - (dw * (KW - 1) + 1)) // sw + 1
     if Ho < 1 or Wo < 1:
         raise ValueError("empty output")
+    return (N, H, W, Cin, KH, KW, Cout), (sh, sw, pt, pb, pl, pr, dh, dw), (Ho, Wo)
+
+
+def conv2d_grouped(X, F, bias=None, stride=1, pad=0, dil=1, groups=1):
+    """Grouped NHWC convolution with per-axis stride / padding / dilation and a KH x KW kernel,
+    float64. stride, dil: (h, w) pairs or one int for both; pad: one int, an (h, w) pair, or
+    ((top, bottom), (left, right)) for different padding before and after an axis (a causal
+    Conv1D pads only the left). X: [N, H, W, Cin]; F: [KH, KW, Cin/groups, Cout] (output channel
+    o uses input channels of group o // (Cout/groups)); bias: [Cout] or None. Conv1D is H = KH = 1.
+    Returns (Y, abssum), float64 [N, Ho, Wo, Cout]."""
+    X, F = _f32(X), _f32(F)
+    b = None if bias is None else _f32(bias)
+    (N, H, W, Cin, KH, KW, Cout), (sh, sw, pt, pb, pl, pr, dh, dw), (Ho, Wo) = \
+        _grouped_shape(X, F, b, stride, pad, dil, groups)
     Y = np.empty((N, Ho, Wo, Cout), dtype=np.float64)
     A = np.empty_like(Y)
-    rc = _load().oracle_conv2d_grouped(_ptr(X), _ptr(F), _ptr(b), _ptr(Y), _ptr(A), N, H, W, Cin, Cout, KH, KW,
-                                       sh, sw, ph, pw, dh, dw, groups)
+    if pt == pb and pl == pr:
+        rc = _load().oracle_conv2d_grouped(_ptr(X), _ptr(F), _ptr(b), _ptr(Y), _ptr(A), N, H, W, Cin, Cout, KH, KW,
+                                           sh, sw, pt, pl, dh, dw, groups)
+    else:
+        rc = _load().oracle_conv2d_grouped_pads(_ptr(X), _ptr(F), _ptr(b), _ptr(Y), _ptr(A), N, H, W, Cin, Cout, KH,
+                                                KW, sh, sw, pt, pb, pl, pr, dh, dw, groups)
     if rc != 0:
         raise ValueError("bad shape")
     return Y, A
@@ -216,20 +243,19 @@ def conv2d_grouped_points(X, F, flat_idx, bias=None, stride=1, pad=0, dil=1, gro
     """Selected outputs of conv2d_grouped, by flat index into [N, Ho, Wo, Cout]."""
     X, F = _f32(X), _f32(F)
     b = None if bias is None else _f32(bias)
-    N, H, W, Cin = X.shape
-    KH, KW, Cg, Cout = F.shape
-    (sh, sw), (ph, pw), (dh, dw) = _pair(stride), _pair(pad), _pair(dil)
-    if groups < 1 or Cin % groups or Cout % groups or Cg * groups != Cin:
-        raise ValueError("channels must split into the groups")
-    Ho = (H + 2 * ph - (dh * (KH - 1) + 1)) // sh + 1
-    Wo = (W + 2 * pw - (dw * (KW - 1) + 1)) // sw + 1
+    (N, H, W, Cin, KH, KW, Cout), (sh, sw, pt, pb, pl, pr, dh, dw), (Ho, Wo) = \
+        _grouped_shape(X, F, b, stride, pad, dil, groups)
     idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
-    if Ho < 1 or Wo < 1 or (idx.size and (idx.min() < 0 or idx.max() >= N * Ho * Wo * Cout)):
-        raise ValueError("bad shape or index")
+    if idx.size and (idx.min() < 0 or idx.max() >= N * Ho * Wo * Cout):
+        raise ValueError("bad index")
     y = np.empty(idx.size, dtype=np.float64)
     a = np.empty(idx.size, dtype=np.float64)
-    _load().oracle_conv2d_grouped_points(_ptr(X), _ptr(F), _ptr(b), _ptr(idx), idx.size, _ptr(y), _ptr(a), H, W,
-                                         Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups)
+    if pt == pb and pl == pr:
+        _load().oracle_conv2d_grouped_points(_ptr(X), _ptr(F), _ptr(b), _ptr(idx), idx.size, _ptr(y), _ptr(a), H, W,
+                                             Cin, Cout, KH, KW, sh, sw, pt, pl, dh, dw, groups)
+    else:
+        _load().oracle_conv2d_grouped_pads_points(_ptr(X), _ptr(F), _ptr(b), _ptr(idx), idx.size, _ptr(y), _ptr(a),
+                                                  H, W, Cin, Cout, KH, KW, sh, sw, pt, pb, pl, pr, dh, dw, groups)
     return y, a
 
 

@@ -266,6 +266,64 @@ int oracle_conv2d_grouped_points(const float *X, const float *F, const float *bi
     return 0;
 }
 
+/*
+ * The grouped sum with separate padding before and after each axis: pad_top / pad_left zeros
+ * before the first row / column, pad_bottom / pad_right after the last, so an output's window
+ * starts at (y*sh - pad_top, x*sw - pad_left) and Ho = floor((H + pad_top + pad_bottom -
+ * (dh*(KH-1) + 1)) / sh) + 1 (Wo likewise). The causal Conv1D of the CKE section of "Convolution
+ * Is Wx+b Moving Across a Signal" -- a frame's output reads no later frame -- is H = KH = 1 with
+ * pad_left = dw*(KW-1) and pad_right = 0. Per output the sum is grouped_one's, unchanged.
+ */
+static long out_size_pads(long in, int k, int stride, int pad_begin, int pad_end, int dil)
+{
+    long eff = (long)dil * (k - 1) + 1;
+    return (in + (long)pad_begin + (long)pad_end - eff) / stride + 1;
+}
+
+int oracle_conv2d_grouped_pads(const float *X, const float *F, const float *bias, double *Y, double *abssum,
+                               int N, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int pad_top,
+                               int pad_bottom, int pad_left, int pad_right, int dh, int dw, int groups)
+{
+    if (groups < 1 || Cin % groups || Cout % groups) return -1;
+    const long Ho = out_size_pads(H, KH, sh, pad_top, pad_bottom, dh);
+    const long Wo = out_size_pads(W, KW, sw, pad_left, pad_right, dw);
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (long n = 0; n < N; ++n)
+        for (long y = 0; y < Ho; ++y)
+            for (long x = 0; x < Wo; ++x)
+                for (long o = 0; o < Cout; ++o) {
+                    long t = ((n * Ho + y) * Wo + x) * Cout + o;
+                    double a;
+                    grouped_one(X, F, bias, H, W, Cin, Cout, KH, KW, sh, sw, pad_top, pad_left, dh, dw, groups, n, y,
+                                x, o, &Y[t], &a);
+                    if (abssum) abssum[t] = a;
+                }
+    return 0;
+}
+
+/* Selected outputs of oracle_conv2d_grouped_pads, by flat index into [N][Ho][Wo][Cout]. */
+int oracle_conv2d_grouped_pads_points(const float *X, const float *F, const float *bias, const int64_t *idx,
+                                      int64_t npts, double *y, double *abssum, int H, int W, int Cin, int Cout,
+                                      int KH, int KW, int sh, int sw, int pad_top, int pad_bottom, int pad_left,
+                                      int pad_right, int dh, int dw, int groups)
+{
+    if (groups < 1 || Cin % groups || Cout % groups) return -1;
+    const long Ho = out_size_pads(H, KH, sh, pad_top, pad_bottom, dh);
+    const long Wo = out_size_pads(W, KW, sw, pad_left, pad_right, dw);
+    if (Ho < 1 || Wo < 1) return -1;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t p = 0; p < npts; ++p) {
+        long t = idx[p];
+        long o = t % Cout; t /= Cout;
+        long x = t % Wo; t /= Wo;
+        long yy = t % Ho; t /= Ho;
+        grouped_one(X, F, bias, H, W, Cin, Cout, KH, KW, sh, sw, pad_top, pad_left, dh, dw, groups, t, yy, x, o,
+                    &y[p], &abssum[p]);
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------------------------- */
 /* Depthwise                                                                           */
 /* ---------------------------------------------------------------------------------- */

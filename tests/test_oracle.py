@@ -763,3 +763,78 @@ def test_dwpw_weight_counts_of_the_page():
     # pointwise 4,672, about 7.9x fewer
     dense, factored = 64 * 64 * 3 * 3, 64 * 3 * 3 + 64 * 64
     assert (dense, factored) == (36864, 4672) and round(dense / factored, 1) == 7.9
+
+
+# ------------------------------------------------------------------------------------------
+# Padding that differs before and after an axis; the causal Conv1D ("Convolution Is Wx+b
+# Moving Across a Signal", section "Find the same sum in CKE's C kernels": a frame's output may
+# not read later frames, so the sequence is padded on the left only)
+# ------------------------------------------------------------------------------------------
+
+
+def test_causal_conv1d_is_numpy_correlation_of_the_left_padded_sequence():
+    # every output is numpy's valid 1-D correlation of the sequence with dil*(K-1) zeros in
+    # front, summed over the group's channels (dilation 1 and 2; a bias)
+    for dil in (1, 2):
+        L, Cin, Cout, K, groups = 17, 6, 4, 3, 2
+        Cg, Og = Cin // groups, Cout // groups
+        X = _ints(95 + dil, (2, 1, L, Cin))
+        F = _ints(97 + dil, (1, K, Cg, Cout))
+        b = np.array([1, -2, 3, 0], np.float32)
+        P = dil * (K - 1)
+        Y, _ = oracle.conv2d_grouped(X, F, b, dil=(1, dil), pad=((0, 0), (P, 0)), groups=groups)
+        assert Y.shape == (2, 1, L, Cout)
+        for n in range(2):
+            for o in range(Cout):
+                g = o // Og
+                taps = np.zeros(P + 1)
+                ref = np.full(L, float(b[o]))
+                for c in range(Cg):
+                    taps[::dil] = F[0, :, c, o]
+                    xp = np.concatenate([np.zeros(P), X[n, 0, :, g * Cg + c].astype(np.float64)])
+                    ref = ref + np.correlate(xp, taps, "valid")
+                assert np.array_equal(Y[n, 0, :, o], ref)
+
+
+def test_causal_conv1d_page_example():
+    # the page's x = 1..5 with k = (2, 0, -1) and bias 1: the causal form adds two outputs in
+    # front of the page's three (0, 1, 2), which read the zeros before the sequence
+    e = _golden("wxb_1d_examples.json")["weighted_sum_with_bias"]
+    X = np.array(e["x"], np.float32).reshape(1, 1, -1, 1)
+    F = np.array(e["k"], np.float32).reshape(1, 3, 1, 1)
+    Y, _ = oracle.conv2d_grouped(X, F, np.array([e["bias"]], np.float32), pad=((0, 0), (2, 0)))
+    assert Y.ravel().tolist()[2:] == e["output"]
+    assert Y.ravel().tolist()[:2] == [1 + (-1) * 1, 1 + (-1) * 2]
+
+
+def test_causal_output_ignores_later_frames():
+    # changing frames after t leaves outputs 0..t unchanged
+    X = workloads.normal(99, 1 * 1 * 24 * 8, 1.0).reshape(1, 1, 24, 8)
+    F = workloads.normal(100, 1 * 4 * 8 * 5, 0.3).reshape(1, 4, 8, 5)
+    Y, _ = oracle.conv2d_grouped(X, F, pad=((0, 0), (3, 0)))
+    for t in (0, 7, 22):
+        X2 = X.copy()
+        X2[:, :, t + 1:, :] = workloads.normal(101 + t, X2[:, :, t + 1:, :].size, 5.0).reshape(X2[:, :, t + 1:, :].shape)
+        Y2, _ = oracle.conv2d_grouped(X2, F, pad=((0, 0), (3, 0)))
+        assert np.array_equal(Y2[:, :, :t + 1], Y[:, :, :t + 1])
+        assert not np.array_equal(Y2[:, :, t + 1:], Y[:, :, t + 1:])
+
+
+@pytest.mark.parametrize("pads", [((1, 0), (0, 2)), ((0, 2), (3, 1)), ((2, 1), (0, 0))])
+def test_asymmetric_padding_matches_torch_pad_then_convolve(pads):
+    # explicit zero padding (torch.nn.functional.pad) followed by an unpadded convolution
+    (pt, pb), (pl, pr) = pads
+    X = workloads.normal(102, 2 * 9 * 11 * 6, 1.0).reshape(2, 9, 11, 6)
+    F = workloads.normal(103, 3 * 2 * 3 * 4, 0.3).reshape(3, 2, 3, 4)
+    b = workloads.normal(104, 4, 0.5)
+    Y, A = oracle.conv2d_grouped(X, F, b, stride=(2, 1), pad=pads, dil=(1, 2), groups=2)
+    x = torch.from_numpy(np.asarray(X, dtype=np.float64)).permute(0, 3, 1, 2)
+    x = torch.nn.functional.pad(x, (pl, pr, pt, pb))
+    f = torch.from_numpy(np.asarray(F, dtype=np.float64)).permute(3, 2, 0, 1)
+    ref = torch.nn.functional.conv2d(x, f, torch.from_numpy(np.asarray(b, dtype=np.float64)), stride=(2, 1),
+                                     dilation=(1, 2), groups=2).permute(0, 2, 3, 1).numpy()
+    assert Y.shape == ref.shape
+    assert np.all(np.abs(Y - ref) <= 1e-13 * A)
+    idx = (workloads.splitmix64(105, 200) % np.uint64(Y.size)).astype(np.int64)
+    y, a = oracle.conv2d_grouped_points(X, F, idx, b, stride=(2, 1), pad=pads, dil=(1, 2), groups=2)
+    assert np.array_equal(y, Y.reshape(-1)[idx]) and np.array_equal(a, A.reshape(-1)[idx])
