@@ -59,6 +59,7 @@ def workload_table():
          "grouped": ("dense", workloads.DENSE_GROUPED, None),
          "conv1d-stem1": ("dense", workloads.CONV1D_STEM1, None),
          "conv1d-stem2": ("dense", workloads.CONV1D_STEM2, None),
+         "conv1d-causal": ("dense", workloads.CONV1D_CAUSAL, None),
          # comparison path: explicit patch matrix + one cuBLAS GEMM, packing inside the timing
          "dense3x3-explicit-im2col": ("dense", workloads.DENSE_3X3, "im2col")}
     for c in workloads.DWPW_BLOCKS:
@@ -86,6 +87,7 @@ KERNEL_SOURCES = {
     "dense_fold_kernel": ("dense_fold.cuh", "dense_halo.cuh", "dense_tc.cuh", "depthwise.cuh", "ptx.cuh"),
     "dense_halo_kernel": ("dense_halo.cuh", "ptx.cuh"),
     "dense_tc_kernel": ("dense_tc.cuh", "ptx.cuh"),
+    "dense_stream_kernel": ("dense_stream.cuh", "dense_halo.cuh", "ptx.cuh"),
     "dense_direct_kernel": ("dense_direct.cuh",),
     "depthwise_tma_kernel": ("depthwise_tma.cuh", "depthwise.cuh", "ptx.cuh"),
     "depthwise_reg_kernel": ("depthwise_reg.cuh", "depthwise.cuh"),
@@ -331,7 +333,7 @@ def dense_call(cb, case, X, F, b, Y, mode=None, ws=None):
         return cb.conv2d_nhwc_fwd(X, F, Y)
     if case.square:
         return cb.conv2d_nhwc_fwd_ex(X, F, b, Y, case.stride, case.pad, case.dil)
-    return cb.conv2d_nhwc_fwd_grouped(X, F, b, Y, (case.stride, case.sw), (case.pad, case.pw), (case.dil, case.dw),
+    return cb.conv2d_nhwc_fwd_grouped(X, F, b, Y, (case.stride, case.sw), case.pads, (case.dil, case.dw),
                                       case.groups)
 
 
@@ -341,8 +343,7 @@ def oracle_dense(oracle, case, X, F, b):
         return oracle.conv2d_nhwc(X, F)
     if case.square:
         return oracle.conv2d_nhwc_ex(X, F, b, case.stride, case.pad, case.dil)
-    return oracle.conv2d_grouped(X, F, b, (case.stride, case.sw), (case.pad, case.pw), (case.dil, case.dw),
-                                 case.groups)
+    return oracle.conv2d_grouped(X, F, b, (case.stride, case.sw), case.pads, (case.dil, case.dw), case.groups)
 
 
 def im2col_workspace(cb, torch, case, mode):
@@ -557,7 +558,8 @@ def run_ours(args, dist):
                "Cout": case.Cout, "K": case.K, "stride": case.stride, "pad": case.pad, "dil": case.dil,
                "bias": case.bias, "flop_per_step": case.flops, "bytes_per_step": case.bytes}
         if not case.square:
-            cfg.update({"KH": case.kh, "KW": case.kw, "stride_w": case.sw, "pad_w": case.pw, "dil_w": case.dw,
+            cfg.update({"KH": case.kh, "KW": case.kw, "stride_w": case.sw, "pad_w": case.pw, "pad_w_end": case.pwe,
+                        "dil_w": case.dw,
                         "groups": case.groups})
         # the explicit patch matrix the implicit kernels never build (N*Ho*Wo rows by
         # KH*KW*Cin/groups bf16 columns per group) and its size over the input's
@@ -665,8 +667,8 @@ def run_reference(args, dist):
             elif case.square:
                 oracle.conv2d_nhwc_ex_points(X, F, idx, b, case.stride, case.pad, case.dil)
             else:
-                oracle.conv2d_grouped_points(X, F, idx, b, (case.stride, case.sw), (case.pad, case.pw),
-                                             (case.dil, case.dw), case.groups)
+                oracle.conv2d_grouped_points(X, F, idx, b, (case.stride, case.sw), case.pads, (case.dil, case.dw),
+                                             case.groups)
     elif kind == "dwpw":
         x, w, bd, Fb, bp = workloads.dwpw_inputs(case)
         F = workloads.bf16_to_f32(Fb)

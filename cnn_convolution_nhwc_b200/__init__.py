@@ -39,6 +39,8 @@ lib.conv2d_nhwc_fwd_ex.argtypes = [_P, _P, _P, _P] + [_I] * 9 + [_P]
 lib.conv2d_nhwc_fwd_ex.restype = _I
 lib.conv2d_nhwc_fwd_grouped.argtypes = [_P, _P, _P, _P] + [_I] * 14 + [_P]
 lib.conv2d_nhwc_fwd_grouped.restype = _I
+lib.conv2d_nhwc_fwd_grouped_pads.argtypes = [_P, _P, _P, _P] + [_I] * 16 + [_P]
+lib.conv2d_nhwc_fwd_grouped_pads.restype = _I
 lib.conv2d_nhwc_im2col_workspace.argtypes = [_I] * 5
 lib.conv2d_nhwc_im2col_workspace.restype = ctypes.c_size_t
 lib.conv2d_nhwc_fwd_im2col.argtypes = [_P, _P, _P, _P, ctypes.c_size_t] + [_I] * 6 + [_P]
@@ -57,8 +59,10 @@ lib.conv_selftest_wait_timeout.argtypes = [_P]
 lib.conv_selftest_wait_timeout.restype = _I
 
 EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "conv2d_nhwc_fwd_grouped",
-           "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "dwpw_fwd", "depthwise_fwd", "conv_status_string",
-           "conv_device_status", "conv_last_kernel", "conv_selftest_wait_timeout")
+           "conv2d_nhwc_fwd_grouped_pads",
+           "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "dwpw_fwd",
+           "depthwise_fwd", "conv_status_string", "conv_device_status", "conv_last_kernel",
+           "conv_selftest_wait_timeout")
 
 
 class ConvError(RuntimeError):
@@ -187,9 +191,28 @@ def _pair(v, name):
     return int(v), int(v)
 
 
+def _pads(pad):
+    """(top, bottom, left, right) from one int, an (h, w) pair, or ((top, bottom), (left, right))."""
+    if isinstance(pad, (tuple, list)):
+        if len(pad) != 2:
+            raise ValueError("pad must be an int, an (h, w) pair or ((top, bottom), (left, right))")
+        out = []
+        for v in pad:
+            if isinstance(v, (tuple, list)):
+                if len(v) != 2:
+                    raise ValueError("a per-axis pad must be an int or a (before, after) pair")
+                out += [int(v[0]), int(v[1])]
+            else:
+                out += [int(v), int(v)]
+        return tuple(out)
+    return (int(pad),) * 4
+
+
 def conv2d_nhwc_fwd_grouped(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, groups=1, stream=None):
-    """Grouped dense NHWC convolution, bfloat16, with a KH x KW filter and per-axis stride,
-    zero padding and dilation (ints or (h, w) pairs) and an optional float32 bias [Cout]:
+    """Grouped dense NHWC convolution, bfloat16, with a KH x KW filter, per-axis stride and
+    dilation (ints or (h, w) pairs), zero padding (an int, an (h, w) pair, or ((top, bottom),
+    (left, right)) for different padding before and after an axis -- a causal Conv1D is
+    pad=(0, (KW-1, 0))) and an optional float32 bias [Cout]:
     X [N,H,W,Cin], F [KH,KW,Cin/groups,Cout] -> Y [N,Ho,Wo,Cout]. A Conv1D is H = KH = 1."""
     import torch
     px = _tensor(X, torch.bfloat16, 4, "X")
@@ -199,14 +222,15 @@ def conv2d_nhwc_fwd_grouped(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, gro
     groups = int(groups)
     if groups < 1 or Cin % groups or Cout % groups or Cg != Cin // groups:
         raise ValueError("F must be [KH, KW, Cin/groups, Cout] with groups dividing Cin and Cout")
-    (sh, sw), (ph, pw), (dh, dw) = _pair(stride, "stride"), _pair(pad, "pad"), _pair(dil, "dil")
-    pb = ctypes.c_void_p(None)
+    (sh, sw), (dh, dw) = _pair(stride, "stride"), _pair(dil, "dil")
+    pt, pb, pl, pr = _pads(pad)
+    pbias = ctypes.c_void_p(None)
     if bias is not None:
-        pb = _tensor(bias, torch.float32, 1, "bias")
+        pbias = _tensor(bias, torch.float32, 1, "bias")
         if bias.shape[0] != Cout:
             raise ValueError("bias must have Cout entries")
-    Ho = (H + 2 * ph - (dh * (KH - 1) + 1)) // sh + 1
-    Wo = (W + 2 * pw - (dw * (KW - 1) + 1)) // sw + 1
+    Ho = (H + pt + pb - (dh * (KH - 1) + 1)) // sh + 1
+    Wo = (W + pl + pr - (dw * (KW - 1) + 1)) // sw + 1
     if Ho < 1 or Wo < 1:
         raise ValueError("empty output")
     if Y is None:
@@ -214,8 +238,12 @@ def conv2d_nhwc_fwd_grouped(X, F, bias=None, Y=None, stride=1, pad=0, dil=1, gro
     elif tuple(Y.shape) != (N, Ho, Wo, Cout):
         raise ValueError("Y has the wrong shape")
     py = _tensor(Y, torch.bfloat16, 4, "Y")
-    _call(lib.conv2d_nhwc_fwd_grouped, "conv2d_nhwc_fwd_grouped", (X, F, bias, Y), stream,
-          px, pf, pb, py, N, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, dh, dw, groups)
+    if pt == pb and pl == pr:
+        _call(lib.conv2d_nhwc_fwd_grouped, "conv2d_nhwc_fwd_grouped", (X, F, bias, Y), stream,
+              px, pf, pbias, py, N, H, W, Cin, Cout, KH, KW, sh, sw, pt, pl, dh, dw, groups)
+    else:
+        _call(lib.conv2d_nhwc_fwd_grouped_pads, "conv2d_nhwc_fwd_grouped_pads", (X, F, bias, Y), stream,
+              px, pf, pbias, py, N, H, W, Cin, Cout, KH, KW, sh, sw, pt, pb, pl, pr, dh, dw, groups)
     return Y
 
 

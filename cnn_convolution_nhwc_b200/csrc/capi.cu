@@ -22,6 +22,7 @@
 #include "dense_tc.cuh"
 #include "dense_halo.cuh"
 #include "dense_fold.cuh"
+#include "dense_stream.cuh"
 #include "im2col_gemm.cuh"
 #include "depthwise.cuh"
 #include "depthwise_reg.cuh"
@@ -193,23 +194,24 @@ int check_dense(const void *X, const void *F, const void *Y, int N, int H, int W
 struct DenseGeom {
     int KH = 1, KW = 1;
     int sh = 1, sw = 1, ph = 0, pw = 0, dh = 1, dw = 1;
+    int ph_end = 0, pw_end = 0;   // zeros after the last row / column (ph, pw: before the first)
     int groups = 1;
     const float *bias = nullptr;
     static DenseGeom square(int K, int stride = 1, int pad = 0, int dil = 1, const float *bias = nullptr) {
         DenseGeom g;
         g.KH = g.KW = K;
         g.sh = g.sw = stride;
-        g.ph = g.pw = pad;
+        g.ph = g.pw = g.ph_end = g.pw_end = pad;
         g.dh = g.dw = dil;
         g.bias = bias;
         return g;
     }
     // output extents; the caller has checked that the dilated filter fits the padded input
-    long long ho(int H) const { return (1LL * H + 2LL * ph - (1LL * dh * (KH - 1) + 1)) / sh + 1; }
-    long long wo(int W) const { return (1LL * W + 2LL * pw - (1LL * dw * (KW - 1) + 1)) / sw + 1; }
+    long long ho(int H) const { return (1LL * H + ph + ph_end - (1LL * dh * (KH - 1) + 1)) / sh + 1; }
+    long long wo(int W) const { return (1LL * W + pw + pw_end - (1LL * dw * (KW - 1) + 1)) / sw + 1; }
     bool plain() const {
-        return KH == KW && sh == 1 && sw == 1 && ph == 0 && pw == 0 && dh == 1 && dw == 1 && groups == 1 &&
-               bias == nullptr;
+        return KH == KW && sh == 1 && sw == 1 && ph == 0 && pw == 0 && ph_end == 0 && pw_end == 0 && dh == 1 &&
+               dw == 1 && groups == 1 && bias == nullptr;
     }
 };
 
@@ -267,14 +269,14 @@ int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, 
             // unused slots repeat the first group's maps (never dereferenced)
             const int gg = g0 + (gl < ng ? gl : 0);
             {   // X: 4-D {Cin_g, W, H, N} im2col at channel gg*Cin_g. The bounding box of window
-                // origins runs from -pad to (size - 1) + pad - dil*(taps - 1) on each spatial
-                // axis, walked with that axis's stride as element stride, so its pixels are
-                // exactly the output positions; origins, taps and channels outside read zeros.
+                // origins runs from -pad_before to (size - 1) + pad_after - dil*(taps - 1) on each
+                // spatial axis, walked with that axis's stride as element stride, so its pixels
+                // are exactly the output positions; origins, taps and channels outside read zeros.
                 const cuuint64_t dims[4] = {(cuuint64_t)Cin_g, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)N};
                 const cuuint64_t strides[3] = {(cuuint64_t)Cin * 2, (cuuint64_t)W * Cin * 2,
                                                (cuuint64_t)H * W * Cin * 2};
                 const int lower[2] = {-g.pw, -g.ph};
-                const int upper[2] = {g.pw - g.dw * (g.KW - 1), g.ph - g.dh * (g.KH - 1)};
+                const int upper[2] = {g.pw_end - g.dw * (g.KW - 1), g.ph_end - g.dh * (g.KH - 1)};
                 const cuuint32_t estr[4] = {1, (cuuint32_t)g.sw, (cuuint32_t)g.sh, 1};
                 if (g_encode_im2col(&maps.x[gl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                                     const_cast<__nv_bfloat16 *>(xb + 1LL * gg * Cin_g), dims, strides, lower, upper,
@@ -544,6 +546,101 @@ int dispatch_fold(const void *X, const void *F, void *Y, int Cin, int Cout, int 
     if (K == 2) return launch_dense_fold<2>(X, F, Y, Cin, Cout, pl, stream, d, 29);
     if (K == 3) return launch_dense_fold<3>(X, F, Y, Cin, Cout, pl, stream, d, 30);
     return launch_dense_fold<4>(X, F, Y, Cin, Cout, pl, stream, d, 31);
+}
+
+// ---- streamed-filter kernel (256-row tiles, two accumulators per filter slot) -------------
+struct StreamPlan {
+    bool ok = false;
+    int bn = 0;
+    DenseStreamParams p{};
+    int smem = 0;
+    int grid = 0;
+};
+
+// Halo slots of 32 channels by rows of the 256-row tile plus its (K-1)*W + K-1 reach, three of
+// them when that leaves room for at least 8 filter slots (else two), and as many filter slots as
+// fit (at least 4); !ok when the halo is too tall or the ring too shallow.
+StreamPlan plan_stream(int N, int H, int W, int Cin, int Cout, int K, int num_sms) {
+    StreamPlan pl;
+    const long long rows = 1LL * N * H * W;
+    if (rows + 2048 > kInt32Max) return pl;
+    const long long need = 256 + 1LL * (K - 1) * W + (K - 1);
+    if (need > 1024) return pl;
+    const int n_boxes = static_cast<int>((need + 255) / 256);
+    const int box_rows = ((static_cast<int>((need + n_boxes - 1) / n_boxes)) + 15) & ~15;
+    const int halo_rows = n_boxes * box_rows;
+    const int halo_bytes = halo_rows * 64;
+    const int bn = Cout <= 64 ? 64 : 128;
+    const int b_bytes = 32 * bn * 2;
+    const int fixed = bn == 64 ? DenseStreamCfg<64>::FIXED_BYTES : DenseStreamCfg<128>::FIXED_BYTES;
+    int hs = 3;
+    long long avail = kSmemLimit - fixed - 3LL * halo_bytes;
+    if (avail < 8LL * b_bytes) {
+        hs = 2;
+        avail = kSmemLimit - fixed - 2LL * halo_bytes;
+    }
+    long long bs = avail / b_bytes;
+    if (bs > DenseStreamCfg<64>::MAX_BS) bs = DenseStreamCfg<64>::MAX_BS;
+    if (bs < 4) return pl;
+    DenseStreamParams &p = pl.p;
+    p.rows = static_cast<int>(rows);
+    p.H = H; p.W = W; p.Ho = H - K + 1; p.Wo = W - K + 1;
+    p.K = K; p.KK = K * K; p.Cout = Cout;
+    p.num_cblk = (Cin + 31) / 32;
+    p.halo_rows = halo_rows;
+    p.box_rows = box_rows;
+    p.n_boxes = n_boxes;
+    p.halo_bytes = halo_bytes;
+    p.num_mtiles = static_cast<int>((rows + 255) / 256);
+    p.num_ntiles = (Cout + bn - 1) / bn;
+    if (1LL * p.num_mtiles * p.num_ntiles > kInt32Max) return pl;
+    p.num_tiles = p.num_mtiles * p.num_ntiles;
+    p.HS = hs;
+    p.BS = static_cast<int>(bs);
+    pl.bn = bn;
+    pl.smem = fixed + p.BS * b_bytes + p.HS * halo_bytes;
+    // more than half of the shared memory keeps a second CTA (and its TMEM allocation) off the SM
+    if (pl.smem < 116 * 1024) pl.smem = 116 * 1024;
+    pl.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    pl.ok = pl.smem <= kSmemLimit;
+    return pl;
+}
+
+template <int BN>
+int launch_dense_stream(const void *X, const void *F, void *Y, int Cin, int Cout, int K, const StreamPlan &pl,
+                        cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
+    using Cfg = DenseStreamCfg<BN>;
+    alignas(64) CUtensorMap tmX, tmF;
+    {   // X as a 2-D matrix: rows = flattened (n, y, x), Cin channels per row; a box is 32
+        // channels (64 bytes, 64-byte swizzle) x box_rows rows
+        const cuuint64_t dims[2] = {(cuuint64_t)Cin, (cuuint64_t)pl.p.rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)Cin * 2};
+        const cuuint32_t box[2] = {32, (cuuint32_t)pl.p.box_rows};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode_tiled(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    {   // F: 3-D {Cout, Cin, K*K}; a box is 32 reduction rows (channels) x 64 output channels
+        const cuuint64_t dims[3] = {(cuuint64_t)Cout, (cuuint64_t)Cin, (cuuint64_t)K * K};
+        const cuuint64_t strides[2] = {(cuuint64_t)Cout * 2, (cuuint64_t)Cin * Cout * 2};
+        const cuuint32_t box[3] = {64, 32, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(F), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    auto kern = dense_stream_kernel<Cfg>;
+    if (int rc = ensure_smem_attr(d, attr_bit, kern, kSmemLimit)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
+                    "dense_stream_kernel");
 }
 
 using CfgBN64 = DenseTcCfg<64, 6>;
@@ -1083,6 +1180,7 @@ int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int 
     int force_bn = 0;
     bool force_im2col = false, force_halo = false;
     const bool force_fold = force && std::strcmp(force, "fold") == 0;
+    const bool force_stream = force && std::strcmp(force, "stream") == 0;
     if (force) {
         if (std::strncmp(force, "halo", 4) == 0) { force_halo = true; force_bn = std::atoi(force + 4); }
         if (std::strncmp(force, "bn", 2) == 0) { force_im2col = true; force_bn = std::atoi(force + 2); }
@@ -1090,17 +1188,25 @@ int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int 
     if (force_bn != 0 && force_bn != 64 && force_bn != 128 && force_bn != 256) return CONV_ERR_INVALID_ARG;
     // Narrow layers (Cout <= 64, K = 2..4) with a resident filter: the folded-tap kernel
     // ("fold" forces it).
-    if (force_fold || (!force_im2col && !force_halo)) {
+    if (force_fold || (!force_im2col && !force_halo && !force_stream)) {
         const FoldPlan fp = plan_fold(N, H, W, Cin, Cout, K, d->num_sms);
         if (fp.ok) return dispatch_fold(X, F, Y, Cin, Cout, K, fp, stream, d);
         if (force_fold) return CONV_ERR_UNSUPPORTED;
     }
     if (!force_im2col) {
-        // By default the halo kernel runs when the filter stays resident in shared memory;
-        // with a streamed filter the im2col kernel measured faster (deeper operand ring).
+        // By default the halo kernel runs when the filter stays resident in shared memory; with
+        // a streamed filter the 256-row streamed-filter kernel ("stream" forces it).
         const HaloPlan pl = plan_halo(N, H, W, Cin, Cout, K, d->num_sms, force_bn);
-        if (pl.ok && (pl.bres || force_halo || !im2col_ok)) return dispatch_halo(X, F, Y, Cin, Cout, K, pl, stream, d);
+        if (pl.ok && (pl.bres || force_halo) && !force_stream) return dispatch_halo(X, F, Y, Cin, Cout, K, pl, stream, d);
         if (force_halo) return CONV_ERR_UNSUPPORTED;
+        if (!force_bn) {
+            // shared-memory attribute bits 61..62
+            const StreamPlan sp = plan_stream(N, H, W, Cin, Cout, K, d->num_sms);
+            if (sp.ok) return sp.bn == 64 ? launch_dense_stream<64>(X, F, Y, Cin, Cout, K, sp, stream, d, 61)
+                                          : launch_dense_stream<128>(X, F, Y, Cin, Cout, K, sp, stream, d, 62);
+            if (force_stream) return CONV_ERR_UNSUPPORTED;
+        }
+        if (pl.ok && !im2col_ok) return dispatch_halo(X, F, Y, Cin, Cout, K, pl, stream, d);
     }
     if (!im2col_ok) {
         if (force_im2col) return CONV_ERR_UNSUPPORTED;
@@ -1166,11 +1272,11 @@ int dense_general(const void *X, const void *F, void *Y, int N, int H, int W, in
     // 4-D im2col ranges (|corner| <= 127, offset <= 127).
     const int Cin_g = Cin / g.groups, Cout_g = Cout / g.groups;
     const bool tc_shape = (Cin_g % 8 == 0) && (Cout_g % 8 == 0) && aligned(X, 16) && aligned(F, 16) && aligned(Y, 16);
-    auto axis_ok = [](int pad, int dil, int taps) {
+    auto axis_ok = [](int pad, int pad_end, int dil, int taps) {
         const long long reach = 1LL * dil * (taps - 1);
-        return pad <= 127 && reach <= 127 && pad - reach >= -127 && pad - reach <= 127;
+        return pad <= 127 && reach <= 127 && pad_end - reach >= -127 && pad_end - reach <= 127;
     };
-    const bool im2col_ok = tc_shape && axis_ok(g.ph, g.dh, g.KH) && axis_ok(g.pw, g.dw, g.KW) &&
+    const bool im2col_ok = tc_shape && axis_ok(g.ph, g.ph_end, g.dh, g.KH) && axis_ok(g.pw, g.pw_end, g.dw, g.KW) &&
                            2LL * N * H * W * Cin >= 128 * 1024;
     const bool force_bn = force && std::strncmp(force, "bn", 2) == 0;
     if ((force && std::strcmp(force, "direct") == 0) || !im2col_ok) {
@@ -1228,10 +1334,38 @@ int conv2d_nhwc_fwd_grouped(const void *X, const void *F, const float *bias, voi
     DenseGeom g;
     g.KH = KH; g.KW = KW;
     g.sh = stride_h; g.sw = stride_w; g.ph = pad_h; g.pw = pad_w; g.dh = dil_h; g.dw = dil_w;
+    g.ph_end = pad_h; g.pw_end = pad_w;
     g.groups = groups;
     g.bias = bias;
     if (KH == KW && stride_h == stride_w && pad_h == pad_w && dil_h == dil_w && groups == 1)
         return conv2d_nhwc_fwd_ex(X, F, bias, Y, N, H, W, Cin, Cout, KH, stride_h, pad_h, dil_h, stream);
+    return dense_general(X, F, Y, N, H, W, Cin, Cout, g, stream);
+}
+
+int conv2d_nhwc_fwd_grouped_pads(const void *X, const void *F, const float *bias, void *Y, int N, int H, int W,
+                                 int Cin, int Cout, int KH, int KW, int stride_h, int stride_w, int pad_top,
+                                 int pad_bottom, int pad_left, int pad_right, int dil_h, int dil_w, int groups,
+                                 cudaStream_t stream) {
+    if (pad_top == pad_bottom && pad_left == pad_right)
+        return conv2d_nhwc_fwd_grouped(X, F, bias, Y, N, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_top, pad_left,
+                                       dil_h, dil_w, groups, stream);
+    if (!X || !F || !Y) return CONV_ERR_INVALID_ARG;
+    if (N < 1 || H < 1 || W < 1 || Cin < 1 || Cout < 1 || KH < 1 || KW < 1 || stride_h < 1 || stride_w < 1 ||
+        dil_h < 1 || dil_w < 1 || pad_top < 0 || pad_bottom < 0 || pad_left < 0 || pad_right < 0 || groups < 1 ||
+        Cin % groups != 0 || Cout % groups != 0)
+        return CONV_ERR_INVALID_ARG;
+    if (1LL * H + pad_top + pad_bottom > kInt32Max / 2 || 1LL * W + pad_left + pad_right > kInt32Max / 2 ||
+        1LL * dil_h * (KH - 1) > kInt32Max / 2 || 1LL * dil_w * (KW - 1) > kInt32Max / 2)
+        return CONV_ERR_UNSUPPORTED;
+    if (1LL * H + pad_top + pad_bottom < 1LL * dil_h * (KH - 1) + 1 ||
+        1LL * W + pad_left + pad_right < 1LL * dil_w * (KW - 1) + 1)
+        return CONV_ERR_INVALID_ARG;
+    DenseGeom g;
+    g.KH = KH; g.KW = KW;
+    g.sh = stride_h; g.sw = stride_w; g.dh = dil_h; g.dw = dil_w;
+    g.ph = pad_top; g.ph_end = pad_bottom; g.pw = pad_left; g.pw_end = pad_right;
+    g.groups = groups;
+    g.bias = bias;
     return dense_general(X, F, Y, N, H, W, Cin, Cout, g, stream);
 }
 

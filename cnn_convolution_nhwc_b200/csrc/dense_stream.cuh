@@ -1,0 +1,333 @@
+// Dense NHWC forward convolution for layers whose filter is too large to stay in shared memory:
+// the halo implicit GEMM of dense_halo.cuh with 256-row tiles, two TMEM accumulators that share
+// every streamed filter slot, and 32-channel halo blocks.
+//
+// Same operation and flattened-row addressing as dense_halo.cuh (CMU DLSys Lecture 14 notes,
+// section 1 "Fix the index contract before optimizing it" for the definition, section 2 "Move the
+// channel contraction into matrix multiplication" for the sum of per-tap matrix products): GEMM
+// row P = (n*H + y)*W + x of X viewed as [N*H*W][Cin]; tap (i, j) of row P reads row
+// P + i*W + j, so a tile of rows P0 .. P0+255 needs the contiguous rows P0 .. P0 + 255 + (K-1)*W
+// + K-1 of X, and the A operand of tap (i, j) is that staged halo read from row i*W + j on.
+//
+// What changes against the halo kernel is the operand traffic per tensor-core cycle when the
+// filter has to stream. Each (tap, 32-channel) filter slot -- 32 reduction rows x BN output
+// channels -- feeds four MMAs (two K=16 steps into each of two M=128 accumulators, rows 0..127
+// and 128..255 of the tile) instead of two, halving the filter bytes per MMA, and each halo
+// block serves all K*K taps. The halo is staged 32 channels (64 bytes) per row with the 64-byte
+// swizzle so that three halo slots and a deep filter ring fit in shared memory together.
+//
+// Roles in one persistent CTA of 7 warps (role loops walked by whole converged warps, one lane
+// issuing the asynchronous instructions):
+//   warp 0      TMA: the filter ring, one (tap, channel block) slot at a time;
+//   warp 1      TMEM allocation; tcgen05.mma M=128, N=BN, K=16 into the two accumulators of the
+//               tile's accumulator pair (two pairs: tile t+1's MMAs run while tile t drains);
+//   warps 2..5  epilogue: tcgen05.ld of both accumulators, round to bf16, per-warp swizzled
+//               staging, coalesced 16-byte stores of the valid rows straight to Y;
+//   warp 6      TMA: one halo per (tile, channel block) into a ring of HS slots, running ahead
+//               of the filter ring.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "dense_halo.cuh"
+#include "ptx.cuh"
+
+namespace convb200 {
+
+struct DenseStreamParams {
+    int rows;          // N * H * W: flattened input positions (GEMM rows computed)
+    int H, W, Ho, Wo;
+    int K, KK;         // K and K*K
+    int Cout;
+    int num_cblk;      // ceil(Cin / 32)
+    int halo_rows;     // rows per halo slot (n_boxes * box_rows)
+    int box_rows;      // rows per TMA box (<= 256, a multiple of 16)
+    int n_boxes;
+    int halo_bytes;    // halo_rows * 64
+    int num_mtiles, num_ntiles, num_tiles;
+    int HS;            // halo ring slots
+    int BS;            // filter ring slots
+};
+
+template <int BN_>
+struct DenseStreamCfg {
+    static constexpr int BN = BN_;
+    static constexpr int BM = 256;                     // two M=128 accumulators per tile
+    static constexpr int CB = 32;                      // channels per halo block / filter slot
+    static constexpr int B_BOX_BYTES = CB * 64 * 2;    // 32 reduction rows x 64 channels
+    static constexpr int B_BYTES = CB * BN * 2;        // one (tap, channel block) filter slot
+    static constexpr int EPI_BYTES = 4 * 32 * 128;     // per-warp 32 rows x 64 channels staging
+    static constexpr int MAX_HS = 4;
+    static constexpr int MAX_BS = 16;
+    static constexpr int NUM_BARS = 2 * MAX_HS + 2 * MAX_BS + 4 /*acc pairs*/ + 2;
+    static constexpr int TMEM_COLS = 4 * BN;           // two accumulator pairs
+    static constexpr int THREADS = 224;
+    static constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, /*B MN-major*/ true);
+    // shared-memory bytes besides the filter ring and the halo ring
+    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + NUM_BARS * 8 + 4 * 32 * 8 + 16;
+    static_assert(BN == 64 || BN == 128, "two accumulator pairs of BN columns must fit in TMEM");
+};
+
+// Shared-memory matrix descriptor for a K-major operand with the 64-byte swizzle (layout type 4):
+// rows of 64 bytes, 8-row groups 512 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1u) << 16;                 // leading byte offset (unused when swizzled)
+    d |= static_cast<uint64_t>(512u >> 4) << 32;          // stride byte offset: 8 rows x 64 B
+    d |= 1ull << 46;
+    d |= 4ull << 61;
+    return d;
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
+                    __nv_bfloat16 *__restrict__ Y, const DenseStreamParams p, unsigned int *status) {
+    constexpr int BN = Cfg::BN;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;   // 1024-B alignment for the swizzles
+    uint8_t *smem = smem_raw + (base - raw_base);
+
+    const uint32_t sB = base;                                       // filter ring
+    const uint32_t sH = base + p.BS * Cfg::B_BYTES;                 // halo ring
+    const uint32_t epi_off = p.BS * Cfg::B_BYTES + p.HS * p.halo_bytes;
+    const uint32_t sEpi = base + epi_off;
+    const uint32_t bars = sEpi + Cfg::EPI_BYTES;
+    constexpr int RH = Cfg::MAX_HS, RB = Cfg::MAX_BS;
+    auto hfull = [&](int s) { return bars + 8u * s; };
+    auto hempty = [&](int s) { return bars + 8u * (RH + s); };
+    auto bfull = [&](int s) { return bars + 8u * (2 * RH + s); };
+    auto bempty = [&](int s) { return bars + 8u * (2 * RH + RB + s); };
+    auto accf = [&](int b) { return bars + 8u * (2 * RH + 2 * RB + b); };
+    auto acce = [&](int b) { return bars + 8u * (2 * RH + 2 * RB + 2 + b); };
+    const uint32_t done_bar = bars + 8u * (2 * RH + 2 * RB + 4);
+    long long *rowoff_all = reinterpret_cast<long long *>(smem + epi_off + Cfg::EPI_BYTES + Cfg::NUM_BARS * 8);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rowoff_all + 4 * 32);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RH; ++s) {
+            mbar_init(hfull(s), 1);
+            mbar_init(hempty(s), 1);
+        }
+        for (int s = 0; s < RB; ++s) {
+            mbar_init(bfull(s), 1);
+            mbar_init(bempty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf(b), 1);
+            mbar_init(acce(b), 4);   // one arrival per epilogue warp
+        }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmF);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    auto fail = [&]() {
+        atomicOr(status, kStatusTimeout);
+        *abort_flag = 1;
+    };
+    const int first = static_cast<int>(blockIdx.x);
+    const int step = static_cast<int>(gridDim.x);
+
+    if (warp == 6) {
+        // ------------------------------- halo producer ------------------------------
+        uint32_t hit = 0;
+        bool ok = true;
+        for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step) {
+            const int P0 = (t / p.num_ntiles) * Cfg::BM;
+            for (int cb = 0; cb < p.num_cblk; ++cb, ++hit) {
+                const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
+                if (!mbar_wait_warp_backoff(hempty(hs), hph ^ 1u, 64)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(hfull(hs), p.halo_bytes);
+                    for (int bx = 0; bx < p.n_boxes; ++bx)
+                        tma_load_2d(sH + hs * p.halo_bytes + bx * p.box_rows * 64, &tmX, hfull(hs), cb * Cfg::CB,
+                                    P0 + bx * p.box_rows);
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok && lane == 0) fail();
+        // Drain: every load issued has landed before the CTA may exit.
+        for (uint32_t j = hit > (uint32_t)p.HS ? hit - p.HS : 0u; j < hit; ++j)
+            if (!mbar_wait_warp(hfull(j % p.HS), (j / p.HS) & 1u)) { if (lane == 0) fail(); break; }
+    } else if (warp == 0) {
+        // ------------------------------- filter producer ----------------------------
+        uint32_t bit = 0;
+        bool ok = true;
+        for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step) {
+            const int n0 = (t % p.num_ntiles) * BN;
+            for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
+                for (int tap = 0; tap < p.KK; ++tap, ++bit) {
+                    const uint32_t bs = bit % p.BS, bph = (bit / p.BS) & 1u;
+                    if (!mbar_wait_warp_backoff(bempty(bs), bph ^ 1u, 32)) { ok = false; break; }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bfull(bs), Cfg::B_BYTES);
+#pragma unroll
+                        for (int h = 0; h < BN / 64; ++h)
+                            tma_load_3d(sB + bs * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, &tmF, bfull(bs), n0 + h * 64,
+                                        cb * Cfg::CB, tap);
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        if (!ok && lane == 0) fail();
+        for (uint32_t j = bit > (uint32_t)p.BS ? bit - p.BS : 0u; j < bit; ++j)
+            if (!mbar_wait_warp(bfull(j % p.BS), (j / p.BS) & 1u)) { if (lane == 0) fail(); break; }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer ---------------------------------
+        uint32_t hit = 0, bit = 0, local = 0;
+        bool ok = true;
+        for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step, ++local) {
+            const uint32_t b = local & 1u;
+            // waiting here means the epilogue is the slower role: sleep between polls
+            if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d0 = tmem_base + b * (2 * BN);   // rows 0..127 of the tile
+            const uint32_t d1 = d0 + BN;                    // rows 128..255
+            for (int cb = 0; cb < p.num_cblk && ok; ++cb, ++hit) {
+                const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
+                if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t halo = sH + hs * p.halo_bytes;
+                int ky = 0, kx = 0;
+                for (int tap = 0; tap < p.KK; ++tap, ++bit) {
+                    const uint32_t bs = bit % p.BS, bph = (bit / p.BS) & 1u;
+                    if (!mbar_wait_warp(bfull(bs), bph)) { ok = false; break; }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        // tap (ky, kx): A starts at halo row ky*W + kx (64 B per row); the second
+                        // accumulator's rows start 128 rows further on. A K=16 step is 32 B of
+                        // a row (A) or 16 reduction rows = 2048 B (B).
+                        const uint32_t a_row = halo + static_cast<uint32_t>(ky * p.W + kx) * 64u;
+                        const uint32_t bslot = sB + bs * Cfg::B_BYTES;
+                        const uint32_t first_use = (cb | tap) != 0 ? 1u : 0u;
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk) {
+                            const uint64_t bd = smem_desc_sw128(bslot + kk * 2048, Cfg::B_BOX_BYTES, 1024);
+                            const uint32_t acc = kk != 0 ? 1u : first_use;
+                            umma_f16_ss(d0, smem_desc_sw64(a_row + kk * 32), bd, Cfg::IDESC, acc);
+                            umma_f16_ss(d1, smem_desc_sw64(a_row + 128 * 64 + kk * 32), bd, Cfg::IDESC, acc);
+                        }
+                        umma_commit(bempty(bs));
+                    }
+                    __syncwarp();
+                    if (++kx == p.K) { kx = 0; ++ky; }
+                }
+                if (!ok) break;
+                if (lane == 0) umma_commit(hempty(hs));
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(accf(b));
+            __syncwarp();
+        }
+        if (!ok && lane == 0) fail();
+        // All MMAs issued by this warp complete before TMEM is released.
+        if (lane == 0) {
+            umma_commit(done_bar);
+            if (!mbar_wait(done_bar, 0)) fail();
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------- Epilogue (warps 2..5) -----------------------
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const uint32_t stage = sEpi + q * 4096;
+        long long *rowoff = rowoff_all + q * 32;
+        uint32_t local = 0;
+        for (int t = first; t < p.num_tiles; t += step, ++local) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            const uint32_t b = local & 1u;
+            if (!mbar_wait_warp_backoff(accf(b), (local >> 1) & 1u, 128)) { if (lane == 0) fail(); break; }
+            tc_fence_after();
+            const int mt = t / p.num_ntiles;
+            const int n0 = (t - mt * p.num_ntiles) * BN;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                // this lane's row: flattened input position P -> output row, or -1 if dropped
+                {
+                    const int P = mt * Cfg::BM + half * 128 + q * 32 + lane;
+                    long long off = -1;
+                    if (P < p.rows) {
+                        const int row = P / p.W;
+                        const int x = P - row * p.W;
+                        const int n = row / p.H;
+                        const int y = row - n * p.H;
+                        if (x < p.Wo && y < p.Ho)
+                            off = ((static_cast<long long>(n) * p.Ho + y) * p.Wo + x) * p.Cout;
+                    }
+                    rowoff[lane] = off;
+                }
+                const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * (2 * BN) + half * BN;
+#pragma unroll 1
+                for (int h = 0; h < BN / 64; ++h) {
+                    uint32_t r[4][16];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + h * 64 + g * 16, r[g]);
+                    tmem_wait_ld();
+                    // stage this warp's 32 rows x 64 channels (128-byte swizzled rows)
+                    const uint32_t row_addr = stage + lane * 128;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const uint32_t c = g * 2 + cc;
+                            const uint32_t *v = &r[g][cc * 8];
+                            st_shared_v4(row_addr + ((c ^ (lane & 7)) << 4),
+                                         halo_pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                                         halo_pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                                         halo_pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                                         halo_pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                        }
+                    }
+                    __syncwarp();
+                    // coalesced stores: 8 lanes per row, 4 rows per instruction
+                    const int col = n0 + h * 64 + (lane & 7) * 8;
+                    if (col < p.Cout) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int rr = i * 4 + (lane >> 3);
+                            const long long off = rowoff[rr];
+                            if (off >= 0) {
+                                uint32_t a, bb, c, d;
+                                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                             : "=r"(a), "=r"(bb), "=r"(c), "=r"(d)
+                                             : "r"(stage + rr * 128 + ((((lane & 7) ^ (rr & 7))) << 4)));
+                                uint4 *dst = reinterpret_cast<uint4 *>(Y + off + col);
+                                *dst = make_uint4(a, bb, c, d);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+            // the accumulator pair may now be overwritten by the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce(b));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+}  // namespace convb200

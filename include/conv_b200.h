@@ -146,6 +146,24 @@ int conv2d_nhwc_fwd_grouped(const void *X, const void *F, const float *bias, voi
                             int groups, cudaStream_t stream);
 
 /*
+ * conv2d_nhwc_fwd_grouped with separate zero padding before and after each axis: pad_top rows
+ * above the image and pad_bottom below it, pad_left columns before and pad_right after. An
+ * output's window starts at (y*stride_h - pad_top, x*stride_w - pad_left) and
+ *     Ho = floor((H + pad_top + pad_bottom - (dil_h*(KH-1) + 1)) / stride_h) + 1   (Wo likewise).
+ * The causal Conv1D of "Convolution Is Wx+b Moving Across a Signal", section "Find the same sum
+ * in CKE's C kernels" -- a frame's output reads no later frame -- is H = KH = 1 with
+ * pad_left = dil_w*(KW-1) and pad_right = 0 (Wo = W for stride 1).
+ * Layouts, bias rule and requirements as conv2d_nhwc_fwd_grouped (every pad >= 0); with equal
+ * padding before and after both axes this is exactly conv2d_nhwc_fwd_grouped. The tensor-core
+ * path needs, per axis, pad_before <= 127, dil*(taps-1) <= 127 and |pad_after - dil*(taps-1)|
+ * <= 127 besides its channel and alignment rules; other valid shapes take the CUDA-core path.
+ */
+int conv2d_nhwc_fwd_grouped_pads(const void *X, const void *F, const float *bias, void *Y,
+                                 int N, int H, int W, int Cin, int Cout, int KH, int KW,
+                                 int stride_h, int stride_w, int pad_top, int pad_bottom, int pad_left,
+                                 int pad_right, int dil_h, int dil_w, int groups, cudaStream_t stream);
+
+/*
  * Comparison path: the same operation as conv2d_nhwc_fwd computed the way the CMU DLSys Lecture
  * 14 notes build it in section 5 "Generalize the patch matrix to channels and batches" -- an
  * explicit patch matrix A[(n,y,x), (i,j,c)] = X[n,y+i,x+j,c] of N*Ho*Wo rows by K*K*Cin columns,

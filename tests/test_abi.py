@@ -209,3 +209,18 @@ def test_binding_requires_one_device():
     with pytest.raises(ValueError, match="one CUDA device"):
         cb._device(torch.empty(1), torch.empty(1, device="meta"))
     assert cb._device(torch.empty(1), None, torch.empty(2)) == torch.device("cpu")
+
+
+@pytest.mark.parametrize("args,code", [
+    # X, F, bias, Y, N, H, W, Cin, Cout, KH, KW, sh, sw, pad_top, pad_bottom, pad_left, pad_right, dh, dw, groups
+    ((None, F, B, Y, 1, 1, 20, 8, 8, 1, 3, 1, 1, 0, 0, 2, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),
+    ((X, F, B, Y, 1, 1, 20, 8, 8, 1, 3, 1, 1, 0, 0, -1, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),   # pad_left < 0
+    ((X, F, B, Y, 1, 1, 20, 8, 8, 1, 3, 1, 1, 0, 0, 2, -3, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),   # pad_right < 0
+    ((X, F, B, Y, 1, 1, 20, 8, 8, 1, 3, 1, 1, 0, -1, 2, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),   # pad_bottom < 0
+    ((X, F, B, Y, 1, 1, 2, 8, 8, 1, 5, 1, 1, 0, 0, 1, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),     # window > padded row
+    ((X, F, B, Y, 1, 1, 20, 8, 8, 1, 3, 1, 1, 0, 0, 2, 0, 1, 1, 3), cb.CONV_ERR_INVALID_ARG),    # 3 does not divide 8
+    ((X, F, B, V(1 << 20), 1, 1, 20, 8, 8, 1, 3, 1, 1, 0, 0, 2, 0, 1, 1, 1), cb.CONV_ERR_INVALID_ARG),  # Y aliases X
+])
+def test_dense_grouped_pads_rejects(args, code):
+    # padding that differs before and after an axis (a causal Conv1D pads only the left)
+    assert cb.lib.conv2d_nhwc_fwd_grouped_pads(*args, None) == code

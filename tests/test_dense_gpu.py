@@ -330,3 +330,28 @@ def test_folded_taps_refuses_other_shapes(cb, shape):
     with pytest.raises(cb.ConvError) as e:
         _run_bf16(cb, Xb, Fb, env="fold")
     assert e.value.code == cb.CONV_ERR_UNSUPPORTED
+
+
+# (N, H, W, Cin, Cout, K): the streamed-filter kernel (256-row tiles, 32-channel halo blocks,
+# two accumulators per filter slot): a ragged last tile; several N tiles with a partial last
+# one; a partial 32-channel block and Cout = 64 (64-column accumulators); K = 7 with Cout below
+# the tile width on a wide image (halo of 562 rows in three boxes); K = 1 with an 8-column
+# last N tile; K = H = W (one output per image)
+STREAM_SHAPES = [(3, 21, 19, 64, 128, 5), (2, 30, 26, 192, 320, 5), (4, 16, 16, 40, 64, 3), (2, 12, 50, 96, 96, 7),
+                 (5, 9, 9, 128, 136, 1), (4, 8, 8, 64, 64, 8)]
+
+
+@pytest.mark.parametrize("shape", STREAM_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_streamed_filter_kernel(cb, shape):
+    N, H, W, Cin, Cout, K = shape
+    Xb, Fb = _case_inputs(N, H, W, Cin, Cout, K, seed=sum(shape) + 11)
+    y = _run_bf16(cb, Xb, Fb, env="stream")
+    assert cb.conv_last_kernel() == "dense_stream_kernel"
+    _check_bf16(y, Xb, Fb)
+
+
+def test_streamed_filter_is_the_default_for_large_filters(cb):
+    # 5x5x128x128 bf16 is 800 KiB of filter: it cannot stay in shared memory
+    Xb, Fb = _case_inputs(2, 20, 20, 128, 128, 5, seed=31)
+    _check_bf16(_run_bf16(cb, Xb, Fb), Xb, Fb)
+    assert cb.conv_last_kernel() == "dense_stream_kernel"

@@ -24,13 +24,14 @@ def cb(cuda):
     return cb
 
 
-def _case(N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, seed=0):
+def _case(N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, seed=0, pad_w_end=-1):
     return workloads.DenseCase("t", N, H, W, Cin, Cout, KH, "bf16", "normal", seed, stride=s[0], pad=p[0], dil=d[0],
-                               bias=bias, groups=groups, KW=KW, stride_w=s[1], pad_w=p[1], dil_w=d[1])
+                               bias=bias, groups=groups, KW=KW, stride_w=s[1], pad_w=p[1], dil_w=d[1],
+                               pad_w_end=pad_w_end)
 
 
 def _geom(c):
-    return (c.stride, c.sw), (c.pad, c.pw), (c.dil, c.dw)
+    return (c.stride, c.sw), c.pads, (c.dil, c.dw)
 
 
 def _run(cb, c, Xb, Fb, b, env=None):
@@ -163,18 +164,44 @@ def test_page_two_filters_with_bias_as_conv1d(cb):
     assert np.array_equal(y[0, 0, :, 0], [0, 1, 2]) and np.array_equal(y[0, 0, :, 1], [6, 9, 12])
 
 
-@pytest.mark.parametrize("case", [workloads.DENSE_GROUPED, workloads.CONV1D_STEM1, workloads.CONV1D_STEM2],
-                         ids=["grouped", "conv1d-stem1", "conv1d-stem2"])
-def test_full_size_workloads_sampled(cb, case):
-    # the benchmark's workloads at full size, checked on 20000 sampled outputs
+FULL_SIZE = [workloads.DENSE_GROUPED, workloads.CONV1D_STEM1, workloads.CONV1D_STEM2, workloads.CONV1D_CAUSAL]
+
+
+@pytest.mark.parametrize("case", FULL_SIZE, ids=["grouped", "conv1d-stem1", "conv1d-stem2", "conv1d-causal"])
+def test_full_size_workloads(cb, case):
+    # the benchmark's workloads at full size, every output compared with the oracle
     Xb, Fb = workloads.dense_inputs(case)
     b = workloads.dense_bias(case)
     y, kernel = _run(cb, case, Xb, Fb, b)
     assert kernel == "dense_tc_kernel"
-    idx = (workloads.splitmix64(6, 20000) % np.uint64(y.size)).astype(np.int64)
-    s, p, d = _geom(case)
-    ref, absum = oracle.conv2d_grouped_points(workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb), idx, b, s, p, d,
-                                              case.groups)
-    assert np.all(np.abs(y.reshape(-1)[idx] - ref) <= TOL * absum)
-    assert np.all(np.isfinite(y))
+    _check(case, y, Xb, Fb, b)
 
+
+# Causal Conv1D ("Convolution Is Wx+b Moving Across a Signal", section "Find the same sum in CKE's
+# C kernels": a frame's output reads no later frame): zero padding of dil*(K-1) frames before the
+# sequence and none after it.
+# (N, L, Cin, Cout, K, dil, groups, bias, kernel expected)
+CAUSAL = [(2, 1000, 64, 128, 3, 1, 1, True, "dense_tc_kernel"),
+          (2, 777, 128, 64, 5, 2, 4, True, "dense_tc_kernel"),     # dilated, grouped, ragged length
+          (3, 50, 12, 8, 3, 1, 1, False, "dense_direct_kernel")]   # channel counts for the CUDA cores
+
+
+@pytest.mark.parametrize("case", CAUSAL, ids=lambda c: "N{}L{}C{}-{}k{}d{}g{}".format(*c[:7]))
+def test_causal_conv1d(cb, case):
+    N, L, Cin, Cout, K, d, groups, bias, expected = case
+    c = _case(N, 1, L, Cin, Cout, 1, K, (1, 1), (0, d * (K - 1)), (1, d), groups, bias, seed=L + K, pad_w_end=0)
+    Xb, Fb = workloads.dense_inputs(c)
+    b = workloads.dense_bias(c)
+    y, kernel = _run(cb, c, Xb, Fb, b)
+    assert kernel == expected
+    assert y.shape == (N, 1, L, Cout)
+    _check(c, y, Xb, Fb, b)
+    # the same outputs as the symmetric padding's first L frames, on the CUDA-core kernel too
+    sym = _case(N, 1, L, Cin, Cout, 1, K, (1, 1), (0, d * (K - 1)), (1, d), groups, bias, seed=L + K)
+    y_sym, _ = _run(cb, sym, Xb, Fb, b)
+    ref, absum = oracle.conv2d_grouped(workloads.bf16_to_f32(Xb), workloads.bf16_to_f32(Fb), b, 1, c.pads, (1, d),
+                                       groups)
+    assert np.all(np.abs(y_sym[:, :, :L] - ref) <= TOL * absum)
+    y_cc, k_cc = _run(cb, c, Xb, Fb, b, env="direct")
+    assert k_cc == "dense_direct_kernel"
+    _check(c, y_cc, Xb, Fb, b)

@@ -131,6 +131,7 @@ class DenseCase:
     stride_w: int = 0   # width-axis stride, padding, dilation when they differ (0 / -1: as the
     pad_w: int = -1     # height axis)
     dil_w: int = 0
+    pad_w_end: int = -1 # width-axis padding after the last column when it differs (-1: pad_w)
 
     @property
     def kh(self) -> int:
@@ -149,8 +150,17 @@ class DenseCase:
         return self.pad if self.pad_w < 0 else self.pad_w
 
     @property
+    def pwe(self) -> int:
+        return self.pw if self.pad_w_end < 0 else self.pad_w_end
+
+    @property
     def dw(self) -> int:
         return self.dil_w or self.dil
+
+    @property
+    def pads(self):
+        """((top, bottom), (left, right)) zero padding."""
+        return (self.pad, self.pad), (self.pw, self.pwe)
 
     @property
     def cin_g(self) -> int:
@@ -159,8 +169,8 @@ class DenseCase:
     @property
     def square(self) -> bool:
         """One K, one stride, padding and dilation for both axes, one group."""
-        return self.kw == self.K and self.sw == self.stride and self.pw == self.pad and self.dw == self.dil and \
-            self.groups == 1
+        return self.kw == self.K and self.sw == self.stride and self.pw == self.pad and self.pwe == self.pw and \
+            self.dw == self.dil and self.groups == 1
 
     @property
     def f_shape(self):
@@ -172,7 +182,7 @@ class DenseCase:
 
     @property
     def Wo(self) -> int:
-        return (self.W + 2 * self.pw - (self.dw * (self.kw - 1) + 1)) // self.sw + 1
+        return (self.W + self.pw + self.pwe - (self.dw * (self.kw - 1) + 1)) // self.sw + 1
 
     @property
     def flops(self) -> int:
@@ -291,6 +301,10 @@ CONV1D_STEM1 = DenseCase("conv1d bf16 N16 L3000 Cin80 Cout512 K3 p1 bias", 16, 1
                          0, bias=True, KW=3, pad_w=1)
 CONV1D_STEM2 = DenseCase("conv1d bf16 N16 L3000 Cin512 Cout512 K3 s2 p1 bias", 16, 1, 3000, 512, 512, 1, "bf16",
                          "normal", 0, bias=True, KW=3, stride_w=2, pad_w=1)
+# the causal form of the second layer's channel mixing: 512 -> 512, K 3, stride 1, padded only
+# before the sequence (2 frames), so a frame's output reads no later frame; with a bias
+CONV1D_CAUSAL = DenseCase("conv1d bf16 N16 L3000 Cin512 Cout512 K3 causal bias", 16, 1, 3000, 512, 512, 1, "bf16",
+                          "normal", 0, bias=True, KW=3, pad_w=2, pad_w_end=0)
 # depthwise then pointwise blocks (MobileNetV3-large shapes): 672 channels at 14x14, 3x3, into
 # 112 outputs; 960 channels at 7x7, 5x5, into 160 outputs; batch 64, both biases
 DWPW_BLOCKS = [DwPwCase("dwpw C672 K3 s1 H14 Cout112", 64, 672, 14, 14, 3, 1, 1, 1, 112),
