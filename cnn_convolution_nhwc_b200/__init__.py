@@ -45,6 +45,8 @@ lib.conv2d_nhwc_im2col_workspace.argtypes = [_I] * 5
 lib.conv2d_nhwc_im2col_workspace.restype = ctypes.c_size_t
 lib.conv2d_nhwc_fwd_im2col.argtypes = [_P, _P, _P, _P, ctypes.c_size_t] + [_I] * 6 + [_P]
 lib.conv2d_nhwc_fwd_im2col.restype = _I
+lib.conv2d_nhwc_fwd_im2col_noalloc.argtypes = [_P, _P, _P] + [_I] * 6 + [_P]
+lib.conv2d_nhwc_fwd_im2col_noalloc.restype = _I
 lib.dwpw_fwd.argtypes = [_P] * 6 + [_I] * 10 + [_P]
 lib.dwpw_fwd.restype = _I
 lib.depthwise_fwd.argtypes = [_P, _P, _P, _P] + [_I] * 11 + [_P]
@@ -60,9 +62,10 @@ lib.conv_selftest_wait_timeout.restype = _I
 
 EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "conv2d_nhwc_fwd_grouped",
            "conv2d_nhwc_fwd_grouped_pads",
-           "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "dwpw_fwd",
+           "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "conv2d_nhwc_fwd_im2col_noalloc", "dwpw_fwd",
            "depthwise_fwd", "conv_status_string", "conv_device_status", "conv_last_kernel",
            "conv_selftest_wait_timeout")
+CONV_IM2COL_STATIC_BYTES = 32 * 1024 * 1024   # the scratch of conv2d_nhwc_fwd_im2col_noalloc
 
 
 class ConvError(RuntimeError):
@@ -270,6 +273,27 @@ def conv2d_nhwc_fwd_im2col(X, F, Y=None, workspace=None, stream=None):
     _call(lib.conv2d_nhwc_fwd_im2col, "conv2d_nhwc_fwd_im2col", (X, F, Y, workspace), stream,
           px, pf, py, ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
           N, H, W, Cin, Cout, K)
+    return Y
+
+
+def conv2d_nhwc_fwd_im2col_noalloc(X, F, Y, stream=None):
+    """The explicit-im2col comparison path with its patch matrix in the library's static scratch
+    (CONV_IM2COL_STATIC_BYTES per device) instead of a workspace, for callers that cannot
+    allocate device memory. Y must be passed: this binding allocates nothing either."""
+    import torch
+    px = _tensor(X, torch.bfloat16, 4, "X")
+    pf = _tensor(F, torch.bfloat16, 4, "F")
+    N, H, W, Cin = X.shape
+    K, K2, Cin2, Cout = F.shape
+    if K != K2 or Cin2 != Cin:
+        raise ValueError("F must be [K, K, Cin, Cout] matching X")
+    if K > min(H, W):
+        raise ValueError("K must not exceed min(H, W)")
+    if tuple(Y.shape) != (N, H - K + 1, W - K + 1, Cout):
+        raise ValueError("Y has the wrong shape")
+    py = _tensor(Y, torch.bfloat16, 4, "Y")
+    _call(lib.conv2d_nhwc_fwd_im2col_noalloc, "conv2d_nhwc_fwd_im2col_noalloc", (X, F, Y), stream,
+          px, pf, py, N, H, W, Cin, Cout, K)
     return Y
 
 

@@ -36,6 +36,13 @@ namespace convb200 {
 // One status word per device; kernels set bits in it with atomicOr.
 __device__ unsigned int g_conv_status;
 
+// Scratch of conv2d_nhwc_fwd_im2col_noalloc (its patch matrix), reserved once in every device
+// that loads the library. In host code the name is only a host-side stand-in for the array:
+// the device address comes from cudaGetSymbolAddress, taken once per device with that device
+// current (DeviceState::im2col_scratch). Device code never names it; the kernels get the
+// address as an argument like any caller buffer.
+static __device__ __align__(256) unsigned char g_im2col_scratch[CONV_IM2COL_STATIC_BYTES];
+
 // One CTA waiting on a barrier that nothing completes: exercises the bounded wait.
 __global__ void selftest_wait_kernel(unsigned int *status) {
     __shared__ __align__(8) uint64_t bar;
@@ -78,6 +85,7 @@ struct DeviceState {
     unsigned int *status = nullptr;   // device address of g_conv_status on this device
     std::atomic<unsigned long long> attr_done[2] = {{0}, {0}};   // bit per kernel whose shared-memory limit is raised
     cublasHandle_t blas = nullptr;    // for the explicit-im2col comparison path, made on first use
+    void *im2col_scratch = nullptr;   // device address of g_im2col_scratch on this device
     // clusters of a kernel that fit on the device at once, per (kernel bit, cluster size, shared
     // memory), asked once (outside any stream capture: the first call of a shape runs eagerly)
     struct ClusterFit {
@@ -1419,6 +1427,48 @@ int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspac
         return CONV_ERR_CUDA;
     t_last_kernel = "im2col_pack_kernel+cublas";
     return CONV_OK;
+}
+
+int conv2d_nhwc_fwd_im2col_noalloc(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout,
+                                   int K, cudaStream_t stream) {
+    if (int rc = check_dense(X, F, Y, N, H, W, Cin, Cout, K, 2)) return rc;
+    const size_t need = conv2d_nhwc_im2col_workspace(N, H, W, Cin, K);
+    if (need > CONV_IM2COL_STATIC_BYTES) return CONV_ERR_UNSUPPORTED;
+    const long long Ho = H - K + 1, Wo = W - K + 1, M = 1LL * N * Ho * Wo, kd = 1LL * K * K * Cin;
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    if (int rc = check_device_ptrs(stream, {X, F, Y})) return rc;
+    void *scratch = nullptr;
+    {   // set-up once per device, this device current: the array's device address
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!d->im2col_scratch) {
+            void *addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_im2col_scratch) != cudaSuccess) return CONV_ERR_CUDA;
+            d->im2col_scratch = addr;
+        }
+        scratch = d->im2col_scratch;
+    }
+    // the patch matrix: every one of its M * kd entries is written, so stale contents of an
+    // earlier call never reach the product
+    Im2colParams p;
+    p.H = H; p.W = W; p.Cin = Cin; p.K = K; p.Ho = static_cast<int>(Ho); p.Wo = static_cast<int>(Wo);
+    p.kd = static_cast<int>(kd);
+    p.chunk = (Cin % 8 == 0 && aligned(X, 16)) ? 8 : 1;
+    p.chunks = M * kd / p.chunk;
+    long long blocks = (p.chunks + 255) / 256;
+    if (blocks > 1LL * d->num_sms * 8) blocks = 1LL * d->num_sms * 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    auto *A = static_cast<__nv_bfloat16 *>(scratch);
+    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p),
+                 "im2col_pack_kernel") != CONV_OK)
+        return CONV_ERR_CUDA;
+    // Y = A * F as the 1 x 1 convolution of the patch image [N][Ho][Wo][kd] with F viewed as
+    // [1][1][kd][Cout]
+    return dense_plain(A, F, Y, N, static_cast<int>(Ho), static_cast<int>(Wo), static_cast<int>(kd), Cout, 1, stream,
+                       d);
 }
 
 int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, int N, int Cin, int mult, int H,

@@ -180,6 +180,35 @@ int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspac
                            int N, int H, int W, int Cin, int Cout, int K, cudaStream_t stream);
 
 /*
+ * conv2d_nhwc_fwd_im2col without the caller's workspace and without any device allocation:
+ * the patch matrix goes to scratch memory the library reserves statically. This entry has no
+ * counterpart on the pages; it exists for callers that cannot allocate device memory -- code
+ * running under a framework that owns every byte of the device through its own pool, a plugin
+ * inside a host application that forbids allocation, or a real-time path that must not risk
+ * cudaMalloc's implicit synchronisation or an out-of-memory failure after start-up.
+ *   X, F, Y : as conv2d_nhwc_fwd (bfloat16 NHWC input, KKIO filter, NHWC output), caller-owned
+ * The result is Y = A * F with the patch matrix A of conv2d_nhwc_fwd_im2col (same rows, columns
+ * and (i, j, c) order); the product runs on this library's own tensor-core kernels as the
+ * 1 x 1 convolution of A, viewed as an N x Ho x Wo image of K*K*Cin channels, with F viewed as
+ * [1][1][K*K*Cin][Cout] (float32 accumulation, one rounding to bfloat16), so it matches the
+ * workspace entry within the dense tolerance rather than bit for bit.
+ * Scratch: one array of CONV_IM2COL_STATIC_BYTES in device memory per GPU that loads the library,
+ * held until the process exits. A patch matrix larger than that (N*Ho*Wo*K*K*Cin*2 bytes)
+ * returns CONV_ERR_UNSUPPORTED before any CUDA call. Every call overwrites the whole patch
+ * matrix it reads, so nothing needs clearing between calls, but all calls on a device share
+ * the one array: calls whose kernels overlap in time on the GPU (different streams without an
+ * ordering between them) race on it and give wrong results. Order them on one stream.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current) and raises kernel shared-memory limits; make that first call before
+ * any stream capture. The function calls no cudaMalloc, cudaFree or allocating library routine.
+ * Other requirements and status codes as conv2d_nhwc_fwd; conv_last_kernel() afterwards names
+ * the kernel that ran the product.
+ */
+#define CONV_IM2COL_STATIC_BYTES (32u * 1024u * 1024u)
+int conv2d_nhwc_fwd_im2col_noalloc(const void *X, const void *F, void *Y,
+                                   int N, int H, int W, int Cin, int Cout, int K, cudaStream_t stream);
+
+/*
  * Depthwise forward convolution, float32.
  *   x    : [N][Cin][H][W]
  *   w    : [Cin*mult][KH][KW]   (plane oc belongs to input channel oc / mult)
