@@ -29,6 +29,7 @@
 #include "depthwise_tma.cuh"
 #include "depthwise_plane.cuh"
 #include "dwpw.cuh"
+#include "dwpw_gemm.cuh"
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -176,6 +177,15 @@ bool overlaps(const void *a, long long abytes, const void *b, long long bbytes) 
 const char *env(const char *name) {
     const char *v = std::getenv(name);
     return (v && *v) ? v : nullptr;
+}
+
+// An integer setting from the environment, clamped to [lo, hi]; `def` when unset.
+int env_int(const char *name, int def, int lo, int hi) {
+    const char *v = env(name);
+    int r = v ? std::atoi(v) : def;
+    if (r < lo) r = lo;
+    if (r > hi) r = hi;
+    return r;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -443,7 +453,7 @@ int launch_dense_halo(const void *X, const void *F, void *Y, int Cin, int Cout, 
     if (int rc = ensure_smem_attr(d, attr_bit, kern, kSmemLimit)) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(Cfg::THREADS);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
     return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
@@ -798,7 +808,7 @@ DwRegParams dw_reg_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, 
 }
 
 // ---- TMA-staged kernel ----------------------------------------------------------------------
-constexpr int kDwTmaMaxSmem = 160 * 1024;   // per CTA: 4 warps x 2 buffers
+constexpr int kDwTmaMaxSmem = 220 * 1024;   // per CTA: 4 warps x NB buffers (+ output staging)
 
 struct DwTmaPlan {
     bool ok = false;
@@ -819,10 +829,12 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
     p.num_planes = N * Cin;
     p.Wp = p.lpp * 4 * S + 8;                       // 4 zeros, the lanes' columns, the right reach
     p.use_tma = (W % 4 == 0 && aligned(x, 16)) ? 1 : 0;
-    // staged bytes per job buffer: whole planes when they fit, else bands of rows
-    // (about 9 KB per buffer keeps 12 warps, 3 CTAs, per SM with both buffers resident)
+    // staged bytes per job buffer: whole planes when they fit, else bands of rows of even height;
+    // NB buffers per warp. CONV_B200_DW_RING (buffers), CONV_B200_DW_BUFKB (KiB per buffer) and
+    // CONV_B200_DW_CTAS (CTAs per SM) override the defaults (tuning and tests).
+    p.nbuf = env_int("CONV_B200_DW_RING", 3, 2, kDwTmaMaxBuf);
     const long long row_bytes = 4LL * p.Wp * p.ppw;
-    const long long kBufBytes = 9 * 1024;
+    const long long kBufBytes = 1024LL * env_int("CONV_B200_DW_BUFKB", 9, 2, 48);
     const int whole_rows = (Ho - 1) * S + K;
     if (whole_rows * row_bytes <= kBufBytes || !p.use_tma) {
         p.Rw = Ho;
@@ -830,7 +842,8 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
     } else {
         int Rw = static_cast<int>((kBufBytes / row_bytes - K) / S + 1);
         if (Rw < 4) Rw = 4;
-        p.Rw = Rw;
+        const int nb = (Ho + Rw - 1) / Rw;   // bands of even height: no short last band
+        p.Rw = (Ho + nb - 1) / nb;
     }
     p.rows_in = (p.Rw - 1) * S + K;
     // With several planes per warp, a plane stride rows_in * Wp = 4 * lpp * S (mod 32 floats)
@@ -861,7 +874,7 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
         const double plain = static_cast<double>(p.rows_in) * p.Wp / p.Rw;
         auto ctas = [&](int rows, int wp) {   // CTAs per SM the buffers allow
             const long long buf = ((1LL * p.ppw * rows * wp + 31) & ~31LL) * 4;
-            return (227 * 1024) / (kDwWarpsPerCta * 2 * buf + 128 + 1024);
+            return (227 * 1024) / (kDwWarpsPerCta * p.nbuf * buf + 128 + 1024);
         };
         if (best <= 1.25 * plain && ctas(bRows, bWp) >= ctas(p.rows_in, p.Wp)) {
             p.Rw = bRw; p.rows_in = bRows; p.Wp = bWp;
@@ -884,7 +897,7 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
     p.stage_out = 0;
     p.out_floats = 0;
     p.vec_out_staged = aligned(y, 16) ? 1 : 0;
-    p.warp_floats = 2 * p.buf_floats;
+    p.warp_floats = p.nbuf * p.buf_floats;
     if (p.Rw == Ho && !p.vec_out) {
         const int out_floats = (p.ppw * Ho * Wo + 31) & ~31;
         const int smem_plain = kDwWarpsPerCta * 4 * p.warp_floats + 128;
@@ -900,6 +913,7 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
     if (pl.smem > kDwTmaMaxSmem) return pl;
     int per_sm = (227 * 1024) / (pl.smem + 1024);
     if (per_sm > 16) per_sm = 16;
+    per_sm = env_int("CONV_B200_DW_CTAS", per_sm, 1, per_sm);
     if (per_sm < 1) return pl;
     const long long warps_needed = p.num_jobs;
     long long g = 1LL * num_sms * per_sm;
@@ -971,10 +985,14 @@ DwPlanePlan dw_plane_plan(int N, int Cin, int mult, int H, int W, int K, int S, 
     p.out_floats = (PPJ * HO * HO + 31) & ~31;
     p.vec_y = aligned(y, 16) ? 1 : 0;
     p.div_c = make_fastdiv(static_cast<uint32_t>(Cin));
-    pl.smem = kDwPlaneWarps * (p.in_floats + p.out_floats) * 4;
+    // a ring of input buffers per warp (jobs staged ahead); CONV_B200_DW_RING and
+    // CONV_B200_DW_CTAS (CTAs per SM) override the defaults (tuning and tests)
+    p.nbuf = env_int("CONV_B200_DW_RING", 3, 1, kDwPlaneMaxBuf);
+    pl.smem = kDwPlaneWarps * (p.nbuf * p.in_floats + p.out_floats) * 4;
     if (pl.smem > 200 * 1024) return pl;
     int per_sm = (227 * 1024) / (pl.smem + 1024);
     if (per_sm > 8) per_sm = 8;
+    per_sm = env_int("CONV_B200_DW_CTAS", per_sm, 1, per_sm);
     if (per_sm < 1) return pl;
     const long long g_jobs = (p.num_jobs + kDwPlaneWarps - 1) / kDwPlaneWarps;
     const long long g = 1LL * num_sms * per_sm;
@@ -1225,6 +1243,65 @@ int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int 
     if (bn == 64) return launch_dense_tc<CfgBN64, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 0);
     if (bn == 128) return launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 1);
     return launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 2);
+}
+
+// ---- fused depthwise -> pointwise, transposed GEMM (7x7 and 14x14 images) --------------------
+// shared-memory attribute bits 96..103: MODE x K (3, 5) x image (7, 14)
+bool dwpw_gemm_eligible(int C, int H, int W, int K, int stride, int pad, int dil, int Cout, const float *x,
+                        const float *y) {
+    return H == W && (H == 7 || H == 14) && (K == 3 || K == 5) && stride == 1 && dil == 1 && pad == (K - 1) / 2 &&
+           C % 4 == 0 && Cout <= 256 && aligned(x, 16) && aligned(y, 16);
+}
+
+template <int MODE, int KC, int HW>
+int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, const void *F, const float *b_pw, float *y,
+                         int N, int C, int Cout, cudaStream_t stream, DeviceState *d, unsigned bit) {
+    using G = DwPwGemmGeom<HW>;
+    DwPwGemmParams p;
+    p.C = C;
+    p.Cout = Cout;
+    p.num_tiles = N;
+    p.nblk = (C + G::CB - 1) / G::CB;
+    p.MT = (Cout + 127) / 128;
+    p.fslot = p.MT * 2 * G::BOX;
+    p.idesc = idesc_bf16_f32_amn(128, G::NPAD, /*B MN-major*/ true);
+    p.tmem_cols = 32;
+    while (p.tmem_cols < static_cast<uint32_t>(p.MT * G::NPAD)) p.tmem_cols <<= 1;
+    p.b_dw = b_dw;
+    p.b_pw = b_pw;
+    const int smem = dwpw_gemm_smem<HW>(p.fslot);
+    if (smem > kSmemLimit || p.tmem_cols > 512) return CONV_ERR_UNSUPPORTED;
+    alignas(64) CUtensorMap tmF;
+    {   // F: 2-D {Cout, C}; a box is 64 output columns x CB channel rows (columns past Cout and
+        // rows past C read zeros)
+        const cuuint64_t dims[2] = {(cuuint64_t)Cout, (cuuint64_t)C};
+        const cuuint64_t strides[1] = {(cuuint64_t)Cout * 2};
+        const cuuint32_t box[2] = {64, (cuuint32_t)G::CB};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(F), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    auto kern = dwpw_gemm_kernel<MODE, KC, HW>;
+    if (int rc = ensure_smem_attr(d, bit, kern, kSmemLimit)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(N < d->num_sms ? N : d->num_sms));
+    cfg.blockDim = dim3(G::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_gemm_kernel");
+}
+
+template <int MODE>
+int launch_dwpw_gemm(const float *x, const float *w, const float *b_dw, const void *F, const float *b_pw, float *y,
+                     int N, int C, int H, int K, int Cout, cudaStream_t stream, DeviceState *d) {
+    const unsigned b = 96u + 4u * MODE;
+    if (H == 7)
+        return K == 3 ? launch_dwpw_gemm_one<MODE, 3, 7>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 0)
+                      : launch_dwpw_gemm_one<MODE, 5, 7>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 1);
+    return K == 3 ? launch_dwpw_gemm_one<MODE, 3, 14>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 2)
+                  : launch_dwpw_gemm_one<MODE, 5, 14>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 3);
 }
 
 }  // namespace
@@ -1680,10 +1757,19 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
     }
     p.S = 1;
     p.owned = p.n_mma / 16;
-    // 3x3 and 5x5 on images whose tiles fit: the kernel that stages input windows in shared
-    // memory (CONV_B200_DWPW_KERNEL=flat forces the other one; tests)
+    // 7x7 and 14x14 images with 3x3 or 5x5 "same" filters: the transposed-GEMM kernel; other 3x3
+    // and 5x5 shapes whose tiles fit: the kernel that stages input windows in shared memory
+    // (CONV_B200_DWPW_KERNEL=gemm / staged / flat forces one; tests)
     const char *kforce = env("CONV_B200_DWPW_KERNEL");
     const bool force_flat = kforce && std::strcmp(kforce, "flat") == 0;
+    const bool force_staged = kforce && std::strcmp(kforce, "staged") == 0;
+    const bool force_gemm = kforce && std::strcmp(kforce, "gemm") == 0;
+    if (!force_flat && !force_staged && force_split <= 1) {
+        if (dwpw_gemm_eligible(C, H, W, K, stride, pad, dil, Cout, x, y))
+            return mode == DW_EXACT ? launch_dwpw_gemm<0>(x, w_dw, b_dw, F, b_pw, y, N, C, H, K, Cout, stream, d)
+                                    : launch_dwpw_gemm<1>(x, w_dw, b_dw, F, b_pw, y, N, C, H, K, Cout, stream, d);
+    }
+    if (force_gemm) return CONV_ERR_UNSUPPORTED;
     if (!force_flat) {
         const DwPwStagePlan pl = plan_dwpw_staged(p, N);
         if (pl.ok) {

@@ -19,13 +19,14 @@
 // memory the per-tile operand traffic is the halo alone; the SM's TMA engine is then no
 // longer the bottleneck.
 //
-// Roles in one persistent CTA of 6 warps (role loops walked by whole converged warps, one lane
+// Roles in one persistent CTA of 10 warps (role loops walked by whole converged warps, one lane
 // issuing the asynchronous instructions):
 //   warp 0      TMA: the resident filter once (or a ring of per-tap filter slots), then one
 //               halo per (tile, channel block) into a ring of HS halo slots;
 //   warp 1      TMEM allocation; tcgen05.mma M=128, N=BN, K=16 into one of two accumulators;
-//   warps 2..5  epilogue: tcgen05.ld, round to bf16, per-warp swizzled staging, coalesced
-//               16-byte stores of the valid rows straight to Y.
+//   warps 2..9  epilogue, two warps per TMEM lane quarter taking alternate 64-column chunks:
+//               tcgen05.ld, round to bf16, per-warp swizzled staging, coalesced 16-byte stores
+//               of the valid rows straight to Y.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -58,13 +59,15 @@ struct DenseHaloCfg {
     static constexpr int BM = 128;
     static constexpr int B_BOX_BYTES = 64 * 64 * 2;   // 64 reduction rows x 64 channels
     static constexpr int B_BYTES = 64 * BN * 2;       // one (tap, channel block) filter slot
-    static constexpr int EPI_BYTES = 4 * 32 * 128;    // per-warp 32 rows x 64 channels staging
+    static constexpr int NUM_EPI = 8;                 // epilogue warps: two per TMEM lane quarter
+    static constexpr int THREADS = 64 + 32 * NUM_EPI;
+    static constexpr int EPI_BYTES = NUM_EPI * 32 * 128;   // per-warp 32 rows x 64 channels staging
     static constexpr int MAX_RING = 8;
     static constexpr int NUM_BARS = 2 * MAX_RING /*halo*/ + 2 * MAX_RING /*filter*/ + 4 /*acc*/ + 2;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ true);
     // shared-memory bytes besides the filter region and the halo ring
-    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + NUM_BARS * 8 + 4 * 32 * 8 + 16;
+    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + NUM_BARS * 8 + NUM_EPI * 32 * 8 + 16;
     static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
 };
 
@@ -83,7 +86,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, 
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
 dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
                   __nv_bfloat16 *__restrict__ Y, const DenseHaloParams p, unsigned int *status) {
     constexpr int BN = Cfg::BN;
@@ -107,7 +110,7 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     auto acce = [&](int b) { return bars + 8u * (4 * R + 2 + b); };
     const uint32_t done_bar = bars + 8u * (4 * R + 4);
     long long *rowoff_all = reinterpret_cast<long long *>(smem + epi_off + Cfg::EPI_BYTES + Cfg::NUM_BARS * 8);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rowoff_all + 4 * 32);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rowoff_all + Cfg::NUM_EPI * 32);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -122,7 +125,7 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf(b), 1);
-            mbar_init(acce(b), 4);   // one arrival per epilogue warp
+            mbar_init(acce(b), Cfg::NUM_EPI);   // one arrival per epilogue warp
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -296,9 +299,10 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         __syncwarp();
     } else {
         // ------------------------------- Epilogue -----------------------------------
-        const int q = warp & 3;   // TMEM lane quarter this warp may access
-        const uint32_t stage = sEpi + q * 4096;
-        long long *rowoff = rowoff_all + q * 32;
+        const int q = warp & 3;             // TMEM lane quarter this warp may access
+        const int eg = (warp - 2) >> 2;     // which of the quarter's two warps: chunks eg, eg + 2, ...
+        const uint32_t stage = sEpi + (warp - 2) * 4096;
+        long long *rowoff = rowoff_all + (warp - 2) * 32;
         uint32_t local = 0;
         for (int t = first; t < count; t += step, ++local) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
@@ -324,7 +328,7 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
 #pragma unroll 1
-            for (int h = 0; h < BN / 64; ++h) {
+            for (int h = eg; h < BN / 64; h += 2) {
                 uint32_t r[4][16];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + h * 64 + g * 16, r[g]);

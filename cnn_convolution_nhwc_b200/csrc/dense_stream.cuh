@@ -16,14 +16,17 @@
 // block serves all K*K taps. The halo is staged 32 channels (64 bytes) per row with the 64-byte
 // swizzle so that three halo slots and a deep filter ring fit in shared memory together.
 //
-// Roles in one persistent CTA of 7 warps (role loops walked by whole converged warps, one lane
-// issuing the asynchronous instructions):
+// Roles in one persistent CTA of 11 warps (role loops walked by whole converged warps, one lane
+// issuing the asynchronous instructions; the producers poll their slots without sleeping -- a
+// producer that sleeps between polls refills its slot late and starves the tensor pipe, measured
+// at a third of its active cycles):
 //   warp 0      TMA: the filter ring, one (tap, channel block) slot at a time;
 //   warp 1      TMEM allocation; tcgen05.mma M=128, N=BN, K=16 into the two accumulators of the
 //               tile's accumulator pair (two pairs: tile t+1's MMAs run while tile t drains);
-//   warps 2..5  epilogue: tcgen05.ld of both accumulators, round to bf16, per-warp swizzled
-//               staging, coalesced 16-byte stores of the valid rows straight to Y;
-//   warp 6      TMA: one halo per (tile, channel block) into a ring of HS slots, running ahead
+//   warps 2..9  epilogue, two warps per TMEM lane quarter taking alternate 64-column chunks of
+//               both accumulators: tcgen05.ld, round to bf16, per-warp swizzled staging,
+//               coalesced 16-byte stores of the valid rows straight to Y;
+//   warp 10     TMA: one halo per (tile, channel block) into a ring of HS slots, running ahead
 //               of the filter ring.
 #pragma once
 #include <cuda_bf16.h>
@@ -55,15 +58,17 @@ struct DenseStreamCfg {
     static constexpr int CB = 32;                      // channels per halo block / filter slot
     static constexpr int B_BOX_BYTES = CB * 64 * 2;    // 32 reduction rows x 64 channels
     static constexpr int B_BYTES = CB * BN * 2;        // one (tap, channel block) filter slot
-    static constexpr int EPI_BYTES = 4 * 32 * 128;     // per-warp 32 rows x 64 channels staging
+    static constexpr int NUM_EPI = 8;                  // epilogue warps: two per TMEM lane quarter
+    static constexpr int EPI_BYTES = NUM_EPI * 32 * 128;   // per-warp 32 rows x 64 channels staging
     static constexpr int MAX_HS = 4;
     static constexpr int MAX_BS = 16;
     static constexpr int NUM_BARS = 2 * MAX_HS + 2 * MAX_BS + 4 /*acc pairs*/ + 2;
     static constexpr int TMEM_COLS = 4 * BN;           // two accumulator pairs
-    static constexpr int THREADS = 224;
+    static constexpr int THREADS = 32 * (3 + NUM_EPI);   // TMA x2, MMA, epilogue
+    static constexpr int HALO_WARP = 2 + NUM_EPI;
     static constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, /*B MN-major*/ true);
     // shared-memory bytes besides the filter ring and the halo ring
-    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + NUM_BARS * 8 + 4 * 32 * 8 + 16;
+    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + NUM_BARS * 8 + NUM_EPI * 32 * 8 + 16;
     static_assert(BN == 64 || BN == 128, "two accumulator pairs of BN columns must fit in TMEM");
 };
 
@@ -103,7 +108,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     auto acce = [&](int b) { return bars + 8u * (2 * RH + 2 * RB + 2 + b); };
     const uint32_t done_bar = bars + 8u * (2 * RH + 2 * RB + 4);
     long long *rowoff_all = reinterpret_cast<long long *>(smem + epi_off + Cfg::EPI_BYTES + Cfg::NUM_BARS * 8);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rowoff_all + 4 * 32);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rowoff_all + Cfg::NUM_EPI * 32);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -120,7 +125,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf(b), 1);
-            mbar_init(acce(b), 4);   // one arrival per epilogue warp
+            mbar_init(acce(b), Cfg::NUM_EPI);   // one arrival per epilogue warp
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -144,7 +149,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     const int first = static_cast<int>(blockIdx.x);
     const int step = static_cast<int>(gridDim.x);
 
-    if (warp == 6) {
+    if (warp == Cfg::HALO_WARP) {
         // ------------------------------- halo producer ------------------------------
         uint32_t hit = 0;
         bool ok = true;
@@ -152,7 +157,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             const int P0 = (t / p.num_ntiles) * Cfg::BM;
             for (int cb = 0; cb < p.num_cblk; ++cb, ++hit) {
                 const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
-                if (!mbar_wait_warp_backoff(hempty(hs), hph ^ 1u, 64)) { ok = false; break; }
+                if (!mbar_wait_warp(hempty(hs), hph ^ 1u)) { ok = false; break; }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(hfull(hs), p.halo_bytes);
                     for (int bx = 0; bx < p.n_boxes; ++bx)
@@ -175,7 +180,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
                 for (int tap = 0; tap < p.KK; ++tap, ++bit) {
                     const uint32_t bs = bit % p.BS, bph = (bit / p.BS) & 1u;
-                    if (!mbar_wait_warp_backoff(bempty(bs), bph ^ 1u, 32)) { ok = false; break; }
+                    if (!mbar_wait_warp(bempty(bs), bph ^ 1u)) { ok = false; break; }
                     if (lane == 0) {
                         mbar_arrive_expect_tx(bfull(bs), Cfg::B_BYTES);
 #pragma unroll
@@ -246,10 +251,11 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         }
         __syncwarp();
     } else {
-        // ------------------------------- Epilogue (warps 2..5) -----------------------
-        const int q = warp & 3;   // TMEM lane quarter this warp may access
-        const uint32_t stage = sEpi + q * 4096;
-        long long *rowoff = rowoff_all + q * 32;
+        // ------------------------------- Epilogue (warps 2..9) -----------------------
+        const int q = warp & 3;             // TMEM lane quarter this warp may access
+        const int eg = (warp - 2) >> 2;     // which of the quarter's two warps: chunks eg, eg + 2, ...
+        const uint32_t stage = sEpi + (warp - 2) * 4096;
+        long long *rowoff = rowoff_all + (warp - 2) * 32;
         uint32_t local = 0;
         for (int t = first; t < p.num_tiles; t += step, ++local) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
@@ -276,7 +282,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
                 const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * (2 * BN) + half * BN;
 #pragma unroll 1
-                for (int h = 0; h < BN / 64; ++h) {
+                for (int h = eg; h < BN / 64; h += 2) {
                     uint32_t r[4][16];
 #pragma unroll
                     for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + h * 64 + g * 16, r[g]);

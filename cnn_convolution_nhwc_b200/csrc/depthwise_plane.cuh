@@ -13,8 +13,9 @@
 // (LPP = 2): every output row is WOL independent accumulations (no shuffles, no cross-lane
 // data), the rows are fully unrolled with a ring of K input rows in registers, and a plane
 // stride that is odd (7x7) keeps the lanes' shared loads in different banks. Outputs go to a
-// shared-memory staging area and leave as one contiguous, coalesced range of y. The next job's
-// bulk copy is issued as soon as the compute has read the input buffer.
+// shared-memory staging area and leave as one contiguous, coalesced range of y. Each warp keeps
+// a ring of NB input buffers: its first NB jobs are copied at once, and a buffer is refilled
+// with the job NB ahead as soon as the compute has read it.
 #pragma once
 #include <cstdint>
 
@@ -28,13 +29,15 @@ struct DwPlaneParams {
     int C;               // channels (= planes per image, multiplier 1)
     int num_planes;      // N * C
     int num_jobs;        // ceil(num_planes / planes per job)
-    int in_floats;       // per-warp input buffer (planes per job * HW * HW, rounded to 4)
-    int out_floats;      // per-warp output staging (planes per job * HO * WO, rounded to 4)
+    int in_floats;       // one input buffer (planes per job * HW * HW, rounded to 32 floats)
+    int out_floats;      // per-warp output staging (planes per job * HO * WO, rounded to 32 floats)
+    int nbuf;            // input buffers per warp (1 .. kDwPlaneMaxBuf): jobs staged ahead
     int vec_y;           // 1: y 16-byte aligned
     FastDiv div_c;
 };
 
 constexpr int kDwPlaneWarps = 4;
+constexpr int kDwPlaneMaxBuf = 4;
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -54,46 +57,52 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
     constexpr int WOL = (WO + LPP - 1) / LPP;       // output columns per lane
     constexpr int WINC = (WOL - 1) * S + K;         // input columns a lane reads per row
     extern __shared__ __align__(128) float sraw[];
-    __shared__ __align__(8) uint64_t full_all[kDwPlaneWarps];
+    __shared__ __align__(8) uint64_t full_all[kDwPlaneWarps][kDwPlaneMaxBuf];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float *sin = sraw + static_cast<size_t>(warp) * (p.in_floats + p.out_floats);
-    float *sout = sin + p.in_floats;
-    const uint32_t sin_s = static_cast<uint32_t>(__cvta_generic_to_shared(sin));
-    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&full_all[warp]));
+    const int NB = p.nbuf;
+    float *sin0 = sraw + static_cast<size_t>(warp) * (NB * p.in_floats + p.out_floats);
+    float *sout = sin0 + NB * p.in_floats;
+    const uint32_t sin_s = static_cast<uint32_t>(__cvta_generic_to_shared(sin0));
+    const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(&full_all[warp][0]));
+    auto bar = [&](int b) { return bar0 + 8u * b; };
     const int gw = blockIdx.x * kDwPlaneWarps + warp;
     const int GW = gridDim.x * kDwPlaneWarps;
 
-    // stage job `job`: its planes are one contiguous range of x; the 16-byte multiple goes by
-    // one bulk copy, the last 0..3 floats by lane 0
-    auto issue = [&](int job) {
+    // stage job `job` into buffer b: its planes are one contiguous range of x; the 16-byte
+    // multiple goes by one bulk copy, the last 0..3 floats by lane 0
+    auto issue = [&](int job, int b) {
         const int plane0 = job * PPJ;
         const int nplanes = min(PPJ, p.num_planes - plane0);
         const uint32_t total = static_cast<uint32_t>(nplanes * HW * HW);
         const uint32_t bulk = total & ~3u;
         const float *src = x + static_cast<long long>(plane0) * (HW * HW);
         if (lane == 0) {
-            for (uint32_t e = bulk; e < total; ++e) sin[e] = src[e];
-            mbar_arrive_expect_tx(bar, 4u * bulk);
-            if (bulk) bulk_g2s(sin_s, src, 4u * bulk, bar);
+            float *dst = sin0 + b * p.in_floats;
+            for (uint32_t e = bulk; e < total; ++e) dst[e] = src[e];
+            mbar_arrive_expect_tx(bar(b), 4u * bulk);
+            if (bulk) bulk_g2s(sin_s + 4u * b * p.in_floats, src, 4u * bulk, bar(b));
         }
     };
 
     if (lane == 0) {
-        mbar_init(bar, 1);
+        for (int b = 0; b < NB; ++b) mbar_init(bar(b), 1);
         fence_barrier_init();
     }
     __syncwarp();
-    if (gw < p.num_jobs) issue(gw);
+    // the warp's first NB jobs go in flight at once
+    for (int b = 0; b < NB; ++b)
+        if (gw + b * GW < p.num_jobs) issue(gw + b * GW, b);
 
     const int slot = lane / LPP;          // plane slot of this lane in the job
     const int part = lane - slot * LPP;   // column part
     const int ox0 = part * WOL;
     const int ix0 = ox0 * S - PAD;        // first input column this lane reads
-    const float *pb = sin + slot * (HW * HW);
 
     int k = 0;
     bool ok = true;
     for (int job = gw; job < p.num_jobs; job += GW, ++k) {
+        const int b = k % NB;
+        const float *pb = sin0 + b * p.in_floats + slot * (HW * HW);
         const int plane0 = job * PPJ;
         const int plane = plane0 + slot;
         const bool active = plane < p.num_planes;
@@ -103,7 +112,7 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
 #pragma unroll
         for (int t = 0; t < K * K; ++t) wr[t] = __ldg(w + c * (K * K) + t);
         const float bv = HAS_BIAS ? __ldg(bias + c) : 0.0f;
-        if (!mbar_wait_warp(bar, k & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(bar(b), (k / NB) & 1)) { ok = false; break; }
 
         // input row iy (compile-time) of this lane's columns; zeros outside the plane
         auto load_row = [&](int iy, float (&row)[WINC]) {
@@ -209,9 +218,9 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
                 store_row(oy, acc);
             }
         }
-        // the input buffer is free: stage the next job while this one's outputs leave
+        // input buffer b is free: stage the job NB ahead while this one's outputs leave
         __syncwarp();
-        if (job + GW < p.num_jobs) issue(job + GW);
+        if (job + NB * GW < p.num_jobs) issue(job + NB * GW, b);
         const int nplanes = min(PPJ, p.num_planes - plane0);
         const int total = nplanes * (HO * WO);
         float *gdst = y + static_cast<long long>(plane0) * (HO * WO);
@@ -227,8 +236,9 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
     }
     if (!ok) {
         if (lane == 0) atomicOr(status, kStatusTimeout);
-        // the copy in flight lands before the warp exits (bounded wait)
-        mbar_wait_warp(bar, k & 1);
+        // the copies in flight (jobs k .. k + NB - 1) land before the warp exits (bounded waits)
+        for (int kk = k; kk < k + NB; ++kk)
+            if (gw + kk * GW < p.num_jobs) mbar_wait_warp(bar(kk % NB), (kk / NB) & 1);
     }
 }
 

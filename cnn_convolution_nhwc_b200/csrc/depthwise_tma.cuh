@@ -8,10 +8,10 @@
 // PAD = (K-1)/2, dilation 1, multiplier 1.
 //
 // Work layout. Every warp runs its own pipeline over a list of jobs; a job is ppw planes x Rw
-// output rows. The warp stages a job's input window into one of its two shared-memory buffers
-// while it computes from the other. The buffer holds, per plane and staged input row, 4 zeros,
-// the row, and zeros up to the pitch Wp, so the compute loop has no bounds tests and no
-// shuffles. Rows that are 16-byte multiples arrive as one 3-D TMA box {Wp, rows, planes} whose
+// output rows. The warp stages its next jobs' input windows into a ring of NB shared-memory
+// buffers while it computes from the current one. A buffer holds, per plane and staged input
+// row, 4 zeros, the row, and zeros up to the pitch Wp, so the compute loop has no bounds tests
+// and no shuffles. Rows that are 16-byte multiples arrive as one 3-D TMA box {Wp, rows, planes} whose
 // x starts at -4: the copy engine writes every zero of the padding itself (left, right, above,
 // below). Other widths are staged only as whole planes: 4-byte cp.async copies of the image
 // into buffers whose padding was zeroed once at start (it never changes, since every job
@@ -48,12 +48,14 @@ struct DwTmaParams {
     int stage_out;         // 1: whole-plane jobs collect their outputs in shared memory and write
                            //    the job's contiguous output range with coalesced stores
     int out_floats;        // per-warp output staging (ppw * Ho * Wo rounded up to 128 bytes)
-    int warp_floats;       // per-warp shared memory: 2 * buf_floats + out_floats
+    int warp_floats;       // per-warp shared memory: nbuf * buf_floats + out_floats
+    int nbuf;              // staging buffers per warp (2 .. kDwTmaMaxBuf): jobs staged ahead
     int vec_out_staged;    // 1: y 16-byte aligned (staged copies may use 128-bit stores)
     FastDiv div_nbands, div_lpp, div_c, div_w;
 };
 
 constexpr int kDwWarpsPerCta = 4;
+constexpr int kDwTmaMaxBuf = 4;
 
 // N consecutive floats from shared memory starting at base + A (base 16-byte aligned), with
 // the widest loads the compile-time offset allows
@@ -117,13 +119,14 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
     constexpr int OWN = VX * S;
     constexpr int WIN = (VX - 1) * S + K;
     extern __shared__ __align__(128) float sraw[];
-    __shared__ __align__(8) uint64_t full_all[kDwWarpsPerCta][2];
+    __shared__ __align__(8) uint64_t full_all[kDwWarpsPerCta][kDwTmaMaxBuf];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // the dynamic region is only guaranteed 16-byte alignment: align the buffers to 128 bytes
     const uint32_t raw_s = static_cast<uint32_t>(__cvta_generic_to_shared(sraw));
     float *sbuf = sraw + (((raw_s + 127u) & ~127u) - raw_s) / 4u;
     float *my_buf = sbuf + static_cast<size_t>(warp) * p.warp_floats;
-    float *sout = my_buf + 2 * p.buf_floats;
+    const int NB = p.nbuf;
+    float *sout = my_buf + NB * p.buf_floats;
     const uint32_t buf_s = static_cast<uint32_t>(__cvta_generic_to_shared(my_buf));
     const uint32_t full0 = static_cast<uint32_t>(__cvta_generic_to_shared(&full_all[warp][0]));
     auto full = [&](int b) { return full0 + 8u * b; };
@@ -169,18 +172,18 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
     };
 
     if (lane == 0) {
-        mbar_init(full(0), p.use_tma ? 1 : 32);
-        mbar_init(full(1), p.use_tma ? 1 : 32);
+        for (int b = 0; b < NB; ++b) mbar_init(full(b), p.use_tma ? 1 : 32);
         fence_barrier_init();
         if (p.use_tma) prefetch_tensormap(&tmx);
     }
-    if (!p.use_tma) {   // zero both buffers once: the padding of whole-plane jobs never changes
+    if (!p.use_tma) {   // zero the buffers once: the padding of whole-plane jobs never changes
         float4 *z = reinterpret_cast<float4 *>(my_buf);
-        for (int i = lane; i < p.buf_floats / 2; i += 32) z[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int i = lane; i < NB * p.buf_floats / 4; i += 32) z[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
     __syncwarp();
-    if (gw < p.num_jobs) issue(gw, 0);
-    if (gw + GW < p.num_jobs) issue(gw + GW, 1);
+    // the warp's first NB jobs go in flight at once
+    for (int b = 0; b < NB; ++b)
+        if (gw + b * GW < p.num_jobs) issue(gw + b * GW, b);
 
     // lane geometry (fixed for the kernel's life)
     const int ps = fdiv(lane, p.div_lpp);
@@ -192,8 +195,8 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
     int k = 0;
     bool ok = true;
     for (int job = gw; job < p.num_jobs; job += GW, ++k) {
-        const int b = k & 1;
-        if (!mbar_wait_warp(full(b), (k >> 1) & 1)) { ok = false; break; }
+        const int b = k % NB;
+        if (!mbar_wait_warp(full(b), (k / NB) & 1)) { ok = false; break; }
         const int pg = fdiv(job, p.div_nbands);
         const int band = job - pg * p.nbands;
         const int oy0 = band * p.Rw;
@@ -331,15 +334,15 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
                 for (int e = lane; e < total; e += 32) gdst[e] = sout[e];
             }
         }
-        // every lane is done with buffer b (and the output staging); refill b two jobs ahead
+        // every lane is done with buffer b (and the output staging); refill b NB jobs ahead
         __syncwarp();
-        if (job + 2 * GW < p.num_jobs) issue(job + 2 * GW, b);
+        if (job + NB * GW < p.num_jobs) issue(job + NB * GW, b);
     }
     if (!ok) {
         if (lane == 0) atomicOr(status, kStatusTimeout);
         // drain: copies still in flight land before the warp exits (bounded waits)
-        for (int kk = k; kk < k + 2; ++kk)
-            if (gw + kk * GW < p.num_jobs) mbar_wait_warp(full(kk & 1), (kk >> 1) & 1);
+        for (int kk = k; kk < k + NB; ++kk)
+            if (gw + kk * GW < p.num_jobs) mbar_wait_warp(full(kk % NB), (kk / NB) & 1);
     }
 }
 

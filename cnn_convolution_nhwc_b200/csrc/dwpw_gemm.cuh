@@ -1,0 +1,364 @@
+// Depthwise K x K followed by pointwise 1 x 1, fused, for small square images (7x7, 14x14):
+// the channel-mixing GEMM transposed so that the depthwise stage keeps its row-wise register
+// window.
+//
+// Same block and contract as dwpw.cuh ("Convolution Is Wx+b Moving Across a Signal", section
+// "Why variants matter"; the depthwise stage is the OneModel "Depthwise convolution" contract of
+// section "What each output is", multiplier 1; the intermediate is rounded to bfloat16 once; the
+// pointwise sum is float32 with the pointwise bias added once), for stride 1, "same" padding
+// (K-1)/2 and dilation 1. Per image n the pointwise pass is
+//     Y_n[o, p] = sum_c F[c, o] * bf16(d[n, c, p]),   p = oy*W + ox,
+// a GEMM with M = Cout (A = F read as an MN-major operand straight from its [C][Cout] layout),
+// N = the image's pixels (B = the depthwise outputs, MN-major: pixels contiguous) and K = C.
+// Written this way the depthwise outputs of one channel -- neighbouring pixels of one plane --
+// land next to each other in the B tile, so the depthwise stage is the plane-wise loop of the
+// standalone kernels: a thread owns a strip of two neighbouring output columns over a run of
+// rows, keeps the K input rows it needs as packed pairs in registers (each input value loaded
+// once per run), and applies each tap to both outputs with one f32x2 instruction. TMEM lane o
+// then holds output channel o's row of pixels, which is exactly one contiguous range of the NCHW
+// output plane y[n, o, :, :].
+//
+// Work layout: one CTA of 16 warps per image (tile), the channels in blocks of CB. Per block:
+//   * x: the block's CB planes of the image are one contiguous range of x, staged by one 1-D
+//     bulk copy into a 2-slot ring (issued two blocks ahead);
+//   * F: the block's CB x Cout filter rows, 64-column boxes by TMA into a 3-slot ring (two
+//     blocks ahead); columns past Cout arrive as zeros;
+//   * every thread computes its strip (zeros padding, exact or fast mode, the depthwise bias),
+//     rounds to bf16 and writes the values into the B tile (128-byte swizzled, 64 pixels per
+//     box); channels past C write zeros;
+//   * after the CTA barrier that publishes the B tile, thread 0 issues the block's MMAs
+//     (M = 128 per 128 output channels, N = pixels rounded up to 16, K = 16) into the image's
+//     TMEM accumulators and commits; the B slot is rewritten two blocks later, after that
+//     commit.
+// After the last block all 16 warps read the accumulators (warp w: TMEM lane quarter w % 4, a
+// quarter of the 16-column chunks), add the pointwise bias and store y.
+//
+// Every wait is bounded; a wait that runs out sets the status word, the CTA leaves its loop
+// together (barrier-wide OR), drains the copies it issued and waits for its MMAs before TMEM is
+// freed.
+#pragma once
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "depthwise.cuh"       // dw_finish, dw_tap
+#include "depthwise_tma.cuh"   // packed-pair helpers
+#include "depthwise_plane.cuh" // bulk_g2s
+#include "dense_halo.cuh"      // tma_load_2d
+#include "ptx.cuh"
+
+namespace convb200 {
+
+struct DwPwGemmParams {
+    int C, Cout;
+    int num_tiles;      // images
+    int nblk;           // ceil(C / CB)
+    int MT;             // 128-row M tiles: ceil(Cout / 128)
+    int fslot;          // bytes of one filter slot: MT * 2 boxes of CB x 64 bf16
+    uint32_t idesc;
+    uint32_t tmem_cols;
+    const float *b_dw;  // [C] or null
+    const float *b_pw;  // [Cout] or null
+};
+
+// Compile-time geometry per image size: channels per block, strips of two columns, rows per run.
+template <int HW_>
+struct DwPwGemmGeom {
+    static constexpr int HW = HW_;
+    static constexpr int P = HW * HW;                      // pixels per image
+    static constexpr int NPAD = (P + 15) / 16 * 16;        // MMA N
+    static constexpr int CB = HW <= 8 ? 64 : 32;           // channels per block
+    static constexpr int NSTRIP = (HW + 1) / 2;            // strips of two output columns
+    static constexpr int RR = HW <= 8 ? 4 : 7;             // output rows per run
+    static constexpr int NRUN = (HW + RR - 1) / RR;
+    static constexpr int UPP = NSTRIP * NRUN;              // work units per plane
+    static constexpr int THREADS = 512;
+    static constexpr int BOX = CB * 128;                   // one 64-wide box of CB rows, bf16
+    static constexpr int NBOXB = (NPAD + 63) / 64;
+    static constexpr int BSLOT = NBOXB * BOX;              // B tile: CB rows x NPAD pixels
+    static constexpr int XSLOT = (CB * P * 4 + 127) / 128 * 128;
+    static_assert(CB * UPP <= THREADS, "one work unit per thread");
+    static_assert(CB % 16 == 0, "K = 16 steps");
+};
+
+constexpr int kDwPwGemmFSlots = 3;
+constexpr int kDwPwGemmBars = 2 /*xfull*/ + 3 /*ffull*/ + 2 /*mma_done*/ + 1 /*accf*/ + 1 /*drain*/;
+
+template <int HW>
+__host__ __device__ constexpr int dwpw_gemm_smem(int fslot) {
+    using G = DwPwGemmGeom<HW>;
+    return 1024 + kDwPwGemmFSlots * fslot + 2 * G::BSLOT + 2 * G::XSLOT + kDwPwGemmBars * 8 + 16;
+}
+
+// One bf16 value into the B tile: row k (channel in the block), column n (pixel); 64 pixels per
+// box, 128-byte rows, 16-byte chunks swizzled by k % 8.
+__device__ __forceinline__ void dwpw_store_b(uint8_t *sB, int box_bytes, int k, int n, __nv_bfloat16 v) {
+    const int box = n >> 6, col = n & 63;
+    const int chunk = (col >> 3) ^ (k & 7);
+    *reinterpret_cast<__nv_bfloat16 *>(sB + box * box_bytes + k * 128 + chunk * 16 + (col & 7) * 2) = v;
+}
+
+template <int MODE, int KC, int HW>
+__global__ void __launch_bounds__(512, 1)
+dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
+                 float *__restrict__ y, const DwPwGemmParams p, unsigned int *status) {
+    using G = DwPwGemmGeom<HW>;
+    constexpr int PAD = (KC - 1) / 2;
+    constexpr int WIN = KC + 1;   // input columns of a two-column strip
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw);
+    const uint32_t sF = base;
+    const uint32_t sB = sF + kDwPwGemmFSlots * p.fslot;
+    const uint32_t sX = sB + 2 * G::BSLOT;
+    const uint32_t bars = sX + 2 * G::XSLOT;
+    auto xfull = [&](int s) { return bars + 8u * s; };
+    auto ffull = [&](int s) { return bars + 16u + 8u * s; };
+    auto mma_done = [&](int s) { return bars + 40u + 8u * s; };
+    const uint32_t accf = bars + 56u;
+    const uint32_t drain = bars + 64u;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + (bars - base) + kDwPwGemmBars * 8);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) mbar_init(xfull(s), 1);
+        for (int s = 0; s < 3; ++s) mbar_init(ffull(s), 1);
+        for (int s = 0; s < 2; ++s) mbar_init(mma_done(s), 1);
+        mbar_init(accf, 1);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+        prefetch_tensormap(&tmF);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_holder), p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int my_tiles = p.num_tiles > static_cast<int>(blockIdx.x)
+                             ? (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                                   static_cast<int>(gridDim.x)
+                             : 0;
+    const int total = my_tiles * p.nblk;   // channel blocks this CTA walks, over all its tiles
+    // block g of this CTA -> image and first channel
+    auto block_at = [&](int g, int &n, int &c0) {
+        n = static_cast<int>(blockIdx.x) + (g / p.nblk) * static_cast<int>(gridDim.x);
+        c0 = (g % p.nblk) * G::CB;
+    };
+    int x_issued = 0, f_issued = 0;   // thread 0: blocks whose copies are in flight or landed
+    auto issue_x = [&](int g) {   // thread 0
+        int n, c0;
+        block_at(g, n, c0);
+        x_issued = g + 1;
+        const int planes = min(G::CB, p.C - c0);
+        const uint32_t bytes = static_cast<uint32_t>(planes * G::P * 4);
+        mbar_arrive_expect_tx(xfull(g & 1), bytes);
+        bulk_g2s(sX + (g & 1) * G::XSLOT, x + (static_cast<long long>(n) * p.C + c0) * G::P, bytes, xfull(g & 1));
+    };
+    auto issue_f = [&](int g) {   // thread 0
+        int n, c0;
+        block_at(g, n, c0);
+        f_issued = g + 1;
+        const uint32_t slot = sF + (g % 3) * p.fslot;
+        mbar_arrive_expect_tx(ffull(g % 3), static_cast<uint32_t>(p.fslot));
+        for (int b = 0; b < 2 * p.MT; ++b) tma_load_2d(slot + b * G::BOX, &tmF, ffull(g % 3), b * 64, c0);
+    };
+    if (tid == 0) {
+        for (int g = 0; g < 2 && g < total; ++g) {
+            issue_x(g);
+            issue_f(g);
+        }
+    }
+
+    // this thread's work unit inside a block: plane (channel) cl, strip of columns 2s, 2s+1,
+    // run of output rows r*RR .. r*RR + RR - 1
+    const bool unit_ok = tid < G::CB * G::UPP;
+    const int cl = tid / G::UPP;
+    const int rem = tid - cl * G::UPP;
+    const int s = rem % G::NSTRIP;
+    const int r = rem / G::NSTRIP;
+    const int ox0 = 2 * s;
+    const int ix0 = ox0 - PAD;
+    const int oy_first = r * G::RR;
+    bool colok[WIN];
+#pragma unroll
+    for (int t = 0; t < WIN; ++t) colok[t] = ix0 + t >= 0 && ix0 + t < HW;
+    const bool second = ox0 + 1 < HW;   // the strip's second column exists
+
+    bool ok = true;
+    int stop = 0;   // the block at which a wait ran out
+    int tile_parity = 0;
+    for (int g = 0; g < total; ++g) {
+        int n, c0;
+        block_at(g, n, c0);
+        const int kb = g % p.nblk;
+        // the block's planes staged; the B slot's previous MMAs (block g - 2) done
+        bool good = mbar_wait_warp(xfull(g & 1), (g >> 1) & 1);
+        if (good && g >= 2) good = mbar_wait_warp(mma_done(g & 1), ((g - 2) >> 1) & 1);
+        if (__syncthreads_or(!good)) { ok = false; stop = g; break; }
+
+        uint8_t *bslot = smem + (sB - base) + (g & 1) * G::BSLOT;
+        if (unit_ok) {
+            const int c = c0 + cl;
+            if (c < p.C) {
+                const float *xs = reinterpret_cast<const float *>(smem + (sX - base) + (g & 1) * G::XSLOT) + cl * G::P;
+                float wr[KC * KC];
+#pragma unroll
+                for (int t = 0; t < KC * KC; ++t) wr[t] = __ldg(w + static_cast<long long>(c) * (KC * KC) + t);
+                const float bv = p.b_dw ? __ldg(p.b_dw + c) : 0.0f;
+                uint64_t w2[KC * KC];
+#pragma unroll
+                for (int t = 0; t < KC * KC; ++t) w2[t] = dw_pack(wr[t], wr[t]);
+                // ring of KC input rows, each as KC overlapping pairs (x[t], x[t+1])
+                uint64_t ring[KC][KC];
+                auto load_pairs = [&](int iy, uint64_t (&dst)[KC]) {
+                    float f[WIN];
+                    const bool rowok = iy >= 0 && iy < HW;
+#pragma unroll
+                    for (int t = 0; t < WIN; ++t) f[t] = (rowok && colok[t]) ? xs[iy * HW + ix0 + t] : 0.0f;
+#pragma unroll
+                    for (int t = 0; t < KC; ++t) dst[t] = dw_pack(f[t], f[t + 1]);
+                };
+#pragma unroll
+                for (int q = 0; q < KC - 1; ++q) load_pairs(oy_first - PAD + q, ring[q]);
+#pragma unroll
+                for (int i = 0; i < G::RR; ++i) {
+                    const int oy = oy_first + i;
+                    if (oy < HW) {
+                        load_pairs(oy - PAD + KC - 1, ring[(i + KC - 1) % KC]);
+                        float a0, a1;
+                        if constexpr (MODE == 0) {
+                            a0 = 0.0f;
+                            a1 = 0.0f;
+#pragma unroll
+                            for (int ky = 0; ky < KC; ++ky)
+#pragma unroll
+                                for (int kx = 0; kx < KC; ++kx)
+                                    dw_tap2_exact(a0, a1, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
+                        } else {
+                            uint64_t a2 = dw_pack(0.0f, 0.0f);
+#pragma unroll
+                            for (int ky = 0; ky < KC; ++ky)
+#pragma unroll
+                                for (int kx = 0; kx < KC; ++kx)
+                                    a2 = dw_tap2_fast(a2, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
+                            dw_unpack(a2, a0, a1);
+                        }
+                        if (p.b_dw) {
+                            a0 = dw_finish<MODE, true>(a0, bv);
+                            a1 = dw_finish<MODE, true>(a1, bv);
+                        } else {
+                            a0 = dw_finish<MODE, false>(a0, 0.0f);
+                            a1 = dw_finish<MODE, false>(a1, 0.0f);
+                        }
+                        const int pix = oy * HW + ox0;
+                        dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
+                        if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
+                    }
+                }
+            } else {
+                // channels past C: zero rows, so that the zero filter rows meet finite values
+                const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
+                for (int i = 0; i < G::RR; ++i) {
+                    const int oy = oy_first + i;
+                    if (oy < HW) {
+                        dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0, z);
+                        if (second) dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0 + 1, z);
+                    }
+                }
+            }
+        }
+        fence_proxy_async_smem();   // the B tile's generic writes, visible to the tensor cores
+        __syncthreads();
+
+        int fail = 0;
+        if (tid == 0) {
+            if (!mbar_wait(ffull(g % 3), (g / 3) & 1)) fail = 1;
+            if (!fail) {
+                tc_fence_after();
+                const uint32_t fs = sF + (g % 3) * p.fslot;
+                const uint32_t bs = sB + (g & 1) * G::BSLOT;
+#pragma unroll
+                for (int kk = 0; kk < G::CB / 16; ++kk) {
+                    const uint64_t bd = smem_desc_sw128(bs + kk * 2048, G::BOX, 1024);
+                    for (int mt = 0; mt < p.MT; ++mt) {
+                        const uint64_t ad = smem_desc_sw128(fs + mt * 2 * G::BOX + kk * 2048, G::BOX, 1024);
+                        umma_f16_ss(tmem + mt * G::NPAD, ad, bd, p.idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                }
+                umma_commit(mma_done(g & 1));
+                if (kb == p.nblk - 1) umma_commit(accf);
+                // refill: x two blocks ahead into the slot this block has read; F two blocks
+                // ahead into the slot block g - 1 used, once its MMAs are done
+                if (g + 2 < total) {
+                    issue_x(g + 2);
+                    if (g >= 1 && !mbar_wait(mma_done((g - 1) & 1), ((g - 1) >> 1) & 1)) fail = 1;
+                    if (!fail) issue_f(g + 2);
+                }
+            }
+        }
+        if (__syncthreads_or(fail)) { ok = false; stop = g; break; }
+
+        if (kb == p.nblk - 1) {
+            // ------------------------------- epilogue of image n -------------------------------
+            const bool got = mbar_wait_warp(accf, tile_parity);
+            tile_parity ^= 1;
+            tc_fence_after();
+            if (got) {
+                const int q = warp & 3, cg = warp >> 2;
+                for (int mt = 0; mt < p.MT; ++mt) {
+                    const int o = mt * 128 + q * 32 + lane;
+                    const float bp = (p.b_pw && o < p.Cout) ? __ldg(p.b_pw + o) : 0.0f;
+                    float *yrow = y + (static_cast<long long>(n) * p.Cout + o) * G::P;
+                    for (int j = cg; j < G::NPAD / 16; j += 4) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + mt * G::NPAD + j * 16, v);
+                        tmem_wait_ld();
+                        if (o < p.Cout) {
+                            const int p0 = j * 16;
+                            if constexpr (G::P % 4 == 0) {
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    if (p0 + 4 * u < G::P)
+                                        *reinterpret_cast<float4 *>(yrow + p0 + 4 * u) =
+                                            make_float4(__fadd_rn(__uint_as_float(v[4 * u]), bp),
+                                                        __fadd_rn(__uint_as_float(v[4 * u + 1]), bp),
+                                                        __fadd_rn(__uint_as_float(v[4 * u + 2]), bp),
+                                                        __fadd_rn(__uint_as_float(v[4 * u + 3]), bp));
+                            } else {
+#pragma unroll
+                                for (int u = 0; u < 16; ++u)
+                                    if (p0 + u < G::P) yrow[p0 + u] = __fadd_rn(__uint_as_float(v[u]), bp);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            if (__syncthreads_or(!got)) { ok = false; stop = g; break; }
+            tc_fence_after();
+        }
+    }
+
+    if (!ok) {
+        if (tid == 0) {
+            atomicOr(status, kStatusTimeout);
+            // every copy issued lands, and every MMA issued completes, before the CTA exits
+            // (bounded waits): the copies of blocks stop .. issued - 1 were not waited for yet
+            for (int j = stop; j < x_issued; ++j) mbar_wait(xfull(j & 1), (j >> 1) & 1);
+            for (int j = stop; j < f_issued; ++j) mbar_wait(ffull(j % 3), (j / 3) & 1);
+            umma_commit(drain);
+            mbar_wait(drain, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, p.tmem_cols);
+}
+
+}  // namespace convb200

@@ -244,4 +244,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same with an MN-major A operand as well (bit 15).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N, bool b_mn_major) {
+    return idesc_bf16_f32(M, N, b_mn_major) | (1u << 15);
+}
+
 }  // namespace convb200

@@ -289,15 +289,18 @@ def test_noncontiguous_rejected_and_contiguous_copy_works(cb):
 
 
 def test_dispatcher_choices(cb):
-    # Cout <= 64 with K = 3 -> folded-tap kernel; wider Cout with a resident filter -> halo
-    # kernel; channels not multiples of 8 -> CUDA-core kernel; a forced im2col tile width ->
-    # im2col kernel
+    # Cout <= 64 with K = 3 -> folded-tap kernel; wider Cout with a resident filter (at most
+    # 128 KiB in 64 x 128 slots) -> halo kernel; a larger filter -> streamed-filter kernel; channels not multiples
+    # of 8 -> CUDA-core kernel; a forced im2col tile width -> im2col kernel
     Xb, Fb = _case_inputs(2, 20, 20, 64, 64, 3, seed=21)
     _run_bf16(cb, Xb, Fb)
     assert cb.conv_last_kernel() == "dense_fold_kernel"
-    Xb, Fb = _case_inputs(2, 20, 20, 64, 128, 3, seed=24)
+    Xb, Fb = _case_inputs(2, 20, 20, 64, 128, 2, seed=24)      # 4 taps x 16 KiB of filter
     _run_bf16(cb, Xb, Fb)
     assert cb.conv_last_kernel() == "dense_halo_kernel"
+    Xb, Fb = _case_inputs(2, 20, 20, 64, 128, 3, seed=24)      # 144 KiB of filter
+    _run_bf16(cb, Xb, Fb)
+    assert cb.conv_last_kernel() == "dense_stream_kernel"
     Xb2, Fb2 = _case_inputs(1, 7, 9, 3, 5, 3, seed=22)
     _run_bf16(cb, Xb2, Fb2)
     assert cb.conv_last_kernel() == "dense_direct_kernel"

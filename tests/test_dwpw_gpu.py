@@ -40,7 +40,7 @@ def _run(cb, case, x, w, bd, F, bp, mode):
     return out, kernel
 
 
-KERNELS = ("dwpw_kernel", "dwpw_staged_kernel")
+KERNELS = ("dwpw_kernel", "dwpw_staged_kernel", "dwpw_gemm_kernel")
 
 
 def _tol(C):
@@ -104,15 +104,60 @@ def test_unsupported_output_width_is_refused(cb):
 
 
 @pytest.mark.parametrize("case", workloads.DWPW_BLOCKS, ids=lambda c: c.name.replace(" ", "-"))
-def test_full_size_blocks_sampled(cb, case):
+def test_full_size_blocks(cb, case):
+    # the benchmark's blocks at full size, every output compared with the oracle
     x, w, bd, F, bp = workloads.dwpw_inputs(case)
     for mode in (0, 1):
         y, kernel = _run(cb, case, x, w, bd, F, bp, mode)
-        assert kernel in KERNELS and np.all(np.isfinite(y))
-        idx = (workloads.splitmix64(7 + mode, 20000) % np.uint64(y.size)).astype(np.int64)
-        ref, absum = oracle.dwpw_points(x, w, bd, workloads.bf16_to_f32(F), bp, idx, case.stride, case.pad, case.dil,
-                                        mode)
-        assert np.all(np.abs(y.reshape(-1)[idx] - ref) <= _tol(case.C) * absum)
+        assert kernel == "dwpw_gemm_kernel" and np.all(np.isfinite(y))
+        ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, case.stride, case.pad, case.dil, mode)
+        assert np.all(np.abs(y - ref) <= _tol(case.C) * absum)
+
+
+# (N, C, H, K, Cout, mode, biases): the transposed-GEMM kernel (7x7 and 14x14 images, stride 1,
+# "same" padding): partial last channel block (C = 72 over blocks of 32; C = 100 over 64),
+# 8 outputs, two 128-row M tiles (136, 256 outputs), no biases, more images than CTAs
+GEMM_CASES = [(2, 72, 14, 3, 112, 0, True), (3, 100, 7, 5, 160, 1, True), (2, 64, 14, 5, 8, 0, False),
+              (2, 32, 7, 3, 136, 0, True), (1, 128, 14, 3, 256, 1, True), (160, 8, 14, 3, 16, 0, True),
+              (200, 4, 7, 5, 24, 1, True)]
+
+
+@pytest.mark.parametrize("c", GEMM_CASES, ids=lambda c: "N{}C{}H{}K{}-O{}-{}".format(*c[:5], "exact" if c[5] == 0 else "fast"))
+def test_transposed_gemm_kernel(cb, c, monkeypatch):
+    monkeypatch.setenv("CONV_B200_DWPW_KERNEL", "gemm")
+    N, C, H, K, Cout, mode, bias = c
+    case = workloads.DwPwCase("t", N, C, H, H, K, 1, (K - 1) // 2, 1, Cout, bias, seed=C + K + Cout + N)
+    x, w, bd, F, bp = workloads.dwpw_inputs(case)
+    y, kernel = _run(cb, case, x, w, bd, F, bp, mode)
+    assert kernel == "dwpw_gemm_kernel"
+    ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, 1, (K - 1) // 2, 1, mode)
+    assert np.all(np.isfinite(y))
+    bad = np.abs(y - ref) > _tol(C) * absum
+    assert not bad.any(), f"{bad.sum()} outputs out of tolerance"
+
+
+@pytest.mark.parametrize("hw,K", [(14, 3), (7, 5)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_transposed_gemm_identity_mixing_is_exact(cb, hw, K, mode, monkeypatch):
+    # F = I: every output is one exact product plus zeros, so the block must equal the depthwise
+    # output rounded to bf16, bit for bit (the depthwise stage of this kernel is the page's order)
+    monkeypatch.setenv("CONV_B200_DWPW_KERNEL", "gemm")
+    case = workloads.DwPwCase("t", 3, 96, hw, hw, K, 1, (K - 1) // 2, 1, 96, True, seed=hw + K)
+    x, w, bd, _, _ = workloads.dwpw_inputs(case)
+    F = workloads.bf16_bits(np.eye(96, dtype=np.float32))
+    y, kernel = _run(cb, case, x, w, bd, F, None, mode)
+    assert kernel == "dwpw_gemm_kernel"
+    dref = oracle.depthwise(x, w, bd, mult=1, stride=1, pad=(K - 1) // 2, dil=1, mode=mode)
+    assert np.array_equal(y, workloads.bf16_to_f32(workloads.bf16_bits(dref)).astype(np.float64))
+
+
+def test_transposed_gemm_refuses_other_shapes(cb, monkeypatch):
+    monkeypatch.setenv("CONV_B200_DWPW_KERNEL", "gemm")
+    case = workloads.DwPwCase("t", 1, 8, 12, 12, 3, 1, 1, 1, 16, False)   # 12x12 images
+    x, w, _, F, _ = workloads.dwpw_inputs(case)
+    with pytest.raises(cb.ConvError) as e:
+        _run(cb, case, x, w, None, F, None, 0)
+    assert e.value.code == cb.CONV_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("split", ["1", "2", "3", "4"])
