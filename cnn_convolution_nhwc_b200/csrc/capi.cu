@@ -830,9 +830,9 @@ DwTmaPlan dw_tma_plan(int N, int Cin, int mult, int H, int W, int Ho, int Wo, in
     p.Wp = p.lpp * 4 * S + 8;                       // 4 zeros, the lanes' columns, the right reach
     p.use_tma = (W % 4 == 0 && aligned(x, 16)) ? 1 : 0;
     // staged bytes per job buffer: whole planes when they fit, else bands of rows of even height;
-    // NB buffers per warp. CONV_B200_DW_RING (buffers), CONV_B200_DW_BUFKB (KiB per buffer) and
+    // NB buffers per warp (two measured fastest on the sweep layers). CONV_B200_DW_RING (buffers), CONV_B200_DW_BUFKB (KiB per buffer) and
     // CONV_B200_DW_CTAS (CTAs per SM) override the defaults (tuning and tests).
-    p.nbuf = env_int("CONV_B200_DW_RING", 3, 2, kDwTmaMaxBuf);
+    p.nbuf = env_int("CONV_B200_DW_RING", 2, 2, kDwTmaMaxBuf);
     const long long row_bytes = 4LL * p.Wp * p.ppw;
     const long long kBufBytes = 1024LL * env_int("CONV_B200_DW_BUFKB", 9, 2, 48);
     const int whole_rows = (Ho - 1) * S + K;
@@ -985,9 +985,10 @@ DwPlanePlan dw_plane_plan(int N, int Cin, int mult, int H, int W, int K, int S, 
     p.out_floats = (PPJ * HO * HO + 31) & ~31;
     p.vec_y = aligned(y, 16) ? 1 : 0;
     p.div_c = make_fastdiv(static_cast<uint32_t>(Cin));
-    // a ring of input buffers per warp (jobs staged ahead); CONV_B200_DW_RING and
-    // CONV_B200_DW_CTAS (CTAs per SM) override the defaults (tuning and tests)
-    p.nbuf = env_int("CONV_B200_DW_RING", 3, 1, kDwPlaneMaxBuf);
+    // a ring of input buffers per warp (jobs staged ahead; one buffer measured fastest on the
+    // sweep layers, as it leaves the most CTAs per SM); CONV_B200_DW_RING and CONV_B200_DW_CTAS
+    // (CTAs per SM) override the defaults (tuning and tests)
+    p.nbuf = env_int("CONV_B200_DW_RING", 1, 1, kDwPlaneMaxBuf);
     pl.smem = kDwPlaneWarps * (p.nbuf * p.in_floats + p.out_floats) * 4;
     if (pl.smem > 200 * 1024) return pl;
     int per_sm = (227 * 1024) / (pl.smem + 1024);
@@ -1269,7 +1270,11 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
     while (p.tmem_cols < static_cast<uint32_t>(p.MT * G::NPAD)) p.tmem_cols <<= 1;
     p.b_dw = b_dw;
     p.b_pw = b_pw;
-    const int smem = dwpw_gemm_smem<HW>(p.fslot);
+    // a 2-CTA cluster per image (every other channel block each) when there are two blocks and
+    // its receive area fits; CONV_B200_DWPW_SPLIT=1 keeps one CTA per image (tests)
+    const int want = env_int("CONV_B200_DWPW_SPLIT", 2, 1, 2);
+    p.S = (want == 2 && p.nblk >= 2 && dwpw_gemm_smem<HW>(p.fslot, p.MT, 2) <= kSmemLimit) ? 2 : 1;
+    const int smem = dwpw_gemm_smem<HW>(p.fslot, p.MT, p.S);
     if (smem > kSmemLimit || p.tmem_cols > 512) return CONV_ERR_UNSUPPORTED;
     alignas(64) CUtensorMap tmF;
     {   // F: 2-D {Cout, C}; a box is 64 output columns x CB channel rows (columns past Cout and
@@ -1285,11 +1290,22 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
     }
     auto kern = dwpw_gemm_kernel<MODE, KC, HW>;
     if (int rc = ensure_smem_attr(d, bit, kern, kSmemLimit)) return rc;
+    const int clusters_max = d->num_sms / p.S;
+    const int clusters = N < clusters_max ? N : clusters_max;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(N < d->num_sms ? N : d->num_sms));
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S));
     cfg.blockDim = dim3(G::THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    if (p.S > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
     return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_gemm_kernel");
 }
 
@@ -1764,7 +1780,7 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
     const bool force_flat = kforce && std::strcmp(kforce, "flat") == 0;
     const bool force_staged = kforce && std::strcmp(kforce, "staged") == 0;
     const bool force_gemm = kforce && std::strcmp(kforce, "gemm") == 0;
-    if (!force_flat && !force_staged && force_split <= 1) {
+    if (!force_flat && !force_staged && force_split <= 2) {
         if (dwpw_gemm_eligible(C, H, W, K, stride, pad, dil, Cout, x, y))
             return mode == DW_EXACT ? launch_dwpw_gemm<0>(x, w_dw, b_dw, F, b_pw, y, N, C, H, K, Cout, stream, d)
                                     : launch_dwpw_gemm<1>(x, w_dw, b_dw, F, b_pw, y, N, C, H, K, Cout, stream, d);

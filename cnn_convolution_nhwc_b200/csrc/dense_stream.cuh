@@ -149,14 +149,17 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     const int first = static_cast<int>(blockIdx.x);
     const int step = static_cast<int>(gridDim.x);
 
+    // The role loops keep their ring slots and phases as running counters and advance the MMA
+    // descriptors by adding to their address fields: the MMA warp is one serial instruction
+    // stream, and every instruction of its loop delays the next MMA (a loop with a division per
+    // slot was measured at ~440 cycles per 4-MMA slot against ~260 of tensor work).
     if (warp == Cfg::HALO_WARP) {
         // ------------------------------- halo producer ------------------------------
-        uint32_t hit = 0;
+        uint32_t hit = 0, hs = 0, hph = 0;
         bool ok = true;
         for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step) {
             const int P0 = (t / p.num_ntiles) * Cfg::BM;
             for (int cb = 0; cb < p.num_cblk; ++cb, ++hit) {
-                const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
                 if (!mbar_wait_warp(hempty(hs), hph ^ 1u)) { ok = false; break; }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(hfull(hs), p.halo_bytes);
@@ -165,6 +168,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                                     P0 + bx * p.box_rows);
                 }
                 __syncwarp();
+                if (++hs == static_cast<uint32_t>(p.HS)) { hs = 0; hph ^= 1u; }
             }
         }
         if (!ok && lane == 0) fail();
@@ -173,13 +177,12 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             if (!mbar_wait_warp(hfull(j % p.HS), (j / p.HS) & 1u)) { if (lane == 0) fail(); break; }
     } else if (warp == 0) {
         // ------------------------------- filter producer ----------------------------
-        uint32_t bit = 0;
+        uint32_t bit = 0, bs = 0, bph = 0;
         bool ok = true;
         for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step) {
             const int n0 = (t % p.num_ntiles) * BN;
             for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
                 for (int tap = 0; tap < p.KK; ++tap, ++bit) {
-                    const uint32_t bs = bit % p.BS, bph = (bit / p.BS) & 1u;
                     if (!mbar_wait_warp(bempty(bs), bph ^ 1u)) { ok = false; break; }
                     if (lane == 0) {
                         mbar_arrive_expect_tx(bfull(bs), Cfg::B_BYTES);
@@ -189,6 +192,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                                         cb * Cfg::CB, tap);
                     }
                     __syncwarp();
+                    if (++bs == static_cast<uint32_t>(p.BS)) { bs = 0; bph ^= 1u; }
                 }
             }
         }
@@ -197,8 +201,14 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             if (!mbar_wait_warp(bfull(j % p.BS), (j / p.BS) & 1u)) { if (lane == 0) fail(); break; }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
-        uint32_t hit = 0, bit = 0, local = 0;
+        uint32_t local = 0, hs = 0, hph = 0, bs = 0, bph = 0;
         bool ok = true;
+        // descriptors differ only in the start-address field (16-byte units): A +4 per 64-byte
+        // halo row, +2 per K=16 step, +512 for the second accumulator's rows (128 rows further
+        // on); B +B_BYTES/16 per filter slot, +128 per K=16 step (16 reduction rows = 2048 B)
+        const uint64_t b_desc0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
+        constexpr uint32_t kSlotUnits = Cfg::B_BYTES >> 4;
+        const uint32_t row_skip4 = static_cast<uint32_t>(p.W - p.K) * 4u;
         for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step, ++local) {
             const uint32_t b = local & 1u;
             // waiting here means the epilogue is the slower role: sleep between polls
@@ -206,38 +216,33 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             tc_fence_after();
             const uint32_t d0 = tmem_base + b * (2 * BN);   // rows 0..127 of the tile
             const uint32_t d1 = d0 + BN;                    // rows 128..255
-            for (int cb = 0; cb < p.num_cblk && ok; ++cb, ++hit) {
-                const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
+            for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
                 if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t halo = sH + hs * p.halo_bytes;
-                int ky = 0, kx = 0;
-                for (int tap = 0; tap < p.KK; ++tap, ++bit) {
-                    const uint32_t bs = bit % p.BS, bph = (bit / p.BS) & 1u;
-                    if (!mbar_wait_warp(bfull(bs), bph)) { ok = false; break; }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        // tap (ky, kx): A starts at halo row ky*W + kx (64 B per row); the second
-                        // accumulator's rows start 128 rows further on. A K=16 step is 32 B of
-                        // a row (A) or 16 reduction rows = 2048 B (B).
-                        const uint32_t a_row = halo + static_cast<uint32_t>(ky * p.W + kx) * 64u;
-                        const uint32_t bslot = sB + bs * Cfg::B_BYTES;
-                        const uint32_t first_use = (cb | tap) != 0 ? 1u : 0u;
-#pragma unroll
-                        for (int kk = 0; kk < 2; ++kk) {
-                            const uint64_t bd = smem_desc_sw128(bslot + kk * 2048, Cfg::B_BOX_BYTES, 1024);
-                            const uint32_t acc = kk != 0 ? 1u : first_use;
-                            umma_f16_ss(d0, smem_desc_sw64(a_row + kk * 32), bd, Cfg::IDESC, acc);
-                            umma_f16_ss(d1, smem_desc_sw64(a_row + 128 * 64 + kk * 32), bd, Cfg::IDESC, acc);
+                const uint64_t a_desc0 = smem_desc_sw64(sH + hs * p.halo_bytes);
+                uint32_t row4 = 0;   // (ky*W + kx) * 4: tap (ky, kx) reads the halo from row ky*W + kx on
+                for (int ky = 0; ky < p.K && ok; ++ky, row4 += row_skip4) {
+                    for (int kx = 0; kx < p.K; ++kx, row4 += 4u) {
+                        if (!mbar_wait_warp(bfull(bs), bph)) { ok = false; break; }
+                        tc_fence_after();
+                        if (lane == 0) {
+                            const uint64_t ad = a_desc0 + row4;
+                            const uint64_t bd = b_desc0 + bs * kSlotUnits;
+                            const uint32_t acc = (cb | ky | kx) != 0 ? 1u : 0u;
+                            umma_f16_ss(d0, ad, bd, Cfg::IDESC, acc);
+                            umma_f16_ss(d1, ad + 512, bd, Cfg::IDESC, acc);
+                            umma_f16_ss(d0, ad + 2, bd + 128, Cfg::IDESC, 1u);
+                            umma_f16_ss(d1, ad + 514, bd + 128, Cfg::IDESC, 1u);
+                            umma_commit(bempty(bs));
                         }
-                        umma_commit(bempty(bs));
+                        __syncwarp();
+                        if (++bs == static_cast<uint32_t>(p.BS)) { bs = 0; bph ^= 1u; }
                     }
-                    __syncwarp();
-                    if (++kx == p.K) { kx = 0; ++ky; }
                 }
                 if (!ok) break;
                 if (lane == 0) umma_commit(hempty(hs));
                 __syncwarp();
+                if (++hs == static_cast<uint32_t>(p.HS)) { hs = 0; hph ^= 1u; }
             }
             if (!ok) break;
             if (lane == 0) umma_commit(accf(b));

@@ -25,7 +25,9 @@
 // warps; a single lane issues the asynchronous instructions):
 //   warp 0      TMA loads into a STAGES-deep ring of (A, B) slots;
 //   warp 1      allocates TMEM; issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM
-//               accumulators, and tcgen05.commit to free ring slots;
+//               tile buffers -- for BN <= 128 as two partial accumulators that alternate per
+//               K=16 step and are added once by the epilogue -- and tcgen05.commit to free
+//               ring slots;
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads TMEM lanes
 //               32*(w%4) .. +31), round to bf16, 128-byte-swizzled staging in shared
 //               memory, TMA store to Y. The two accumulators let tile t+1's MMAs run
@@ -85,11 +87,18 @@ struct DenseTcCfg {
     static constexpr int EPI_WARP_BYTES = 32 * BN * 2; // 32 rows x BN channels
     static constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
-    static constexpr int TMEM_COLS = 2 * BN;           // two accumulators
+    // Two partial accumulators per tile when they fit (BN <= 128): consecutive K=16 steps
+    // alternate between them, since back-to-back MMAs into one accumulator wait on each other
+    // (measured 99 against 64 cycles per M=128 x N=128 MMA); the epilogue adds the two partial
+    // sums once in float32. Times two tile buffers.
+    static constexpr int PARTS = BN <= 128 ? 2 : 1;
+    static constexpr int TMEM_COLS = 2 * PARTS * BN;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ true);
     static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
     static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM columns");
+    static constexpr uint32_t A_UNITS = A_BYTES >> 4;   // descriptor address field per A slot
+    static constexpr uint32_t B_UNITS = B_BYTES >> 4;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -172,7 +181,7 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
     if (warp == 0) {
         // ------------------------------- TMA producer -------------------------------
         // The whole warp walks the loop (it stays converged); lane 0 issues.
-        uint32_t it = 0;
+        uint32_t it = 0, s = 0, ph = 0;   // ring slot and phase as running counters
         for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
             int grp, mt, nt;
             split(tile, grp, mt, nt);
@@ -187,8 +196,6 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
             bool ok = true;
             int tap = 0, cb = 0, ky = 0, kx = 0;
             for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
-                const uint32_t s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1u;
                 if (!mbar_wait_warp(empty_bar(s), ph ^ 1u)) {
                     if (lane == 0) fail();
                     ok = false;
@@ -211,6 +218,7 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                     ++tap;
                     if (++kx == p.KW) { kx = 0; ++ky; }
                 }
+                if (++s == static_cast<uint32_t>(STAGES)) { s = 0; ph ^= 1u; }
             }
             if (!ok) break;
         }
@@ -223,8 +231,15 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
             }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
-        // The whole warp walks the loop; lane 0 issues the MMAs and commits.
-        uint32_t it = 0, local = 0;
+        // The whole warp walks the loop; lane 0 issues the MMAs and commits. The loop is one
+        // serial instruction stream, so the ring slot and phase are running counters and the
+        // descriptors advance by adding to their address fields (16-byte units).
+        // A: K-major, +2 per 16 channels (32 B inside the swizzle atom), 8-row groups 1024 B
+        // apart. B: MN-major, +128 per 16 reduction rows (2048 B), 8-row groups 1024 B apart
+        // (SBO), 64-channel boxes B_BOX_BYTES apart (LBO).
+        const uint64_t a_desc0 = smem_desc_sw128(sA, 16, 1024);
+        const uint64_t b_desc0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
+        uint32_t it = 0, local = 0, s = 0, ph = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x, ++local) {
             const uint32_t b = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
@@ -235,11 +250,9 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                 break;
             }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + b * BN;
+            const uint32_t d_tmem = tmem_base + b * (Cfg::PARTS * BN);   // partial p at + p*BN
             bool ok = true;
             for (int kb = 0; kb < p.num_kblk; ++kb, ++it) {
-                const uint32_t s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1u;
                 if (!mbar_wait_warp(full_bar(s), ph)) {
                     if (lane == 0) fail();
                     ok = false;
@@ -247,21 +260,19 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t a0 = sA + s * Cfg::A_BYTES;
-                    const uint32_t b0 = sB + s * Cfg::B_BYTES;
+                    const uint64_t ad = a_desc0 + s * Cfg::A_UNITS;
+                    const uint64_t bd = b_desc0 + s * Cfg::B_UNITS;
 #pragma unroll
                     for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
-                        // A: K-major, advance 16 channels = 32 B inside the swizzle atom;
-                        //    8-row groups are 1024 B apart.
-                        const uint64_t ad = smem_desc_sw128(a0 + kk * 32, 16, 1024);
-                        // B: MN-major, advance 16 reduction rows = 2048 B; 8-row groups
-                        //    1024 B apart (SBO), 64-channel boxes 8 KB apart (LBO).
-                        const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, Cfg::B_BOX_BYTES, 1024);
-                        umma_f16_ss(d_tmem, ad, bd, Cfg::IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        const uint32_t part = Cfg::PARTS == 2 ? (kk & 1) : 0;
+                        // the first MMA into each partial accumulator of the tile overwrites it
+                        const uint32_t acc = (kb != 0 || kk >= Cfg::PARTS) ? 1u : 0u;
+                        umma_f16_ss(d_tmem + part * BN, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC, acc);
                     }
                     umma_commit(empty_bar(s));
                 }
                 __syncwarp();
+                if (++s == static_cast<uint32_t>(STAGES)) { s = 0; ph ^= 1u; }
             }
             if (!ok) break;
             if (lane == 0) umma_commit(accf_bar(b));
@@ -293,13 +304,24 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
             // the staging buffer is free once the previous tile's stores have read it
             if (lane == 0) bulk_wait_group_read0();
             __syncwarp();
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * (Cfg::PARTS * BN);
 #pragma unroll 1
             for (int h = 0; h < BN / 64; ++h) {
                 uint32_t r[4][16];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + h * 64 + g * 16, r[g]);
                 tmem_wait_ld();
+                if (Cfg::PARTS == 2) {   // the two partial sums (even and odd K=16 steps), added once
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        uint32_t r2[16];
+                        tmem_ld_32x32b_x16(t_row + BN + h * 64 + g * 16, r2);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            r[g][c] = __float_as_uint(__fadd_rn(__uint_as_float(r[g][c]), __uint_as_float(r2[c])));
+                    }
+                }
                 if (p.bias) {   // one fp32 addition per output, before the single rounding
                     const int c0 = n0 + h * 64;
                     const float *bg = p.bias + static_cast<long long>(grp) * p.ncols;

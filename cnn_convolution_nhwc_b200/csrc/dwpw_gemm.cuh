@@ -18,7 +18,9 @@
 // then holds output channel o's row of pixels, which is exactly one contiguous range of the NCHW
 // output plane y[n, o, :, :].
 //
-// Work layout: one CTA of 16 warps per image (tile), the channels in blocks of CB. Per block:
+// Work layout: one image per cluster of S CTAs (S = 2 when there are at least two channel
+// blocks: rank k takes blocks k, k + S, ...), 16 warps per CTA, the channels in blocks of CB.
+// Per block:
 //   * x: the block's CB planes of the image are one contiguous range of x, staged by one 1-D
 //     bulk copy into a 2-slot ring (issued two blocks ahead);
 //   * F: the block's CB x Cout filter rows, 64-column boxes by TMA into a 3-slot ring (two
@@ -31,11 +33,15 @@
 //     TMEM accumulators and commits; the B slot is rewritten two blocks later, after that
 //     commit.
 // After the last block all 16 warps read the accumulators (warp w: TMEM lane quarter w % 4, a
-// quarter of the 16-column chunks), add the pointwise bias and store y.
+// quarter of the 16-column chunks). With S = 2, 16-column chunk j belongs to rank j % 2: each
+// rank writes its partial of the chunks it does not own into the owner's receive area through
+// distributed shared memory, and the owner adds the two partials (one IEEE addition, so the
+// result does not depend on which rank adds), the pointwise bias, and stores y.
 //
-// Every wait is bounded; a wait that runs out sets the status word, the CTA leaves its loop
-// together (barrier-wide OR), drains the copies it issued and waits for its MMAs before TMEM is
-// freed.
+// Every wait is bounded; a wait that runs out sets the status word and the CTA stops its work
+// together (barrier-wide OR), but keeps taking every CTA and cluster barrier of its remaining
+// images, so its peer is never left waiting; it drains the copies it issued and waits for its
+// MMAs before TMEM is freed.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -45,6 +51,7 @@
 #include "depthwise_tma.cuh"   // packed-pair helpers
 #include "depthwise_plane.cuh" // bulk_g2s
 #include "dense_halo.cuh"      // tma_load_2d
+#include "dwpw.cuh"            // cluster helpers
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -53,6 +60,7 @@ struct DwPwGemmParams {
     int C, Cout;
     int num_tiles;      // images
     int nblk;           // ceil(C / CB)
+    int S;              // CTAs of a cluster sharing one image (1, or 2 when nblk >= 2)
     int MT;             // 128-row M tiles: ceil(Cout / 128)
     int fslot;          // bytes of one filter slot: MT * 2 boxes of CB x 64 bf16
     uint32_t idesc;
@@ -67,6 +75,7 @@ struct DwPwGemmGeom {
     static constexpr int HW = HW_;
     static constexpr int P = HW * HW;                      // pixels per image
     static constexpr int NPAD = (P + 15) / 16 * 16;        // MMA N
+    static constexpr int NCH = NPAD / 16;                  // 16-column accumulator chunks
     static constexpr int CB = HW <= 8 ? 64 : 32;           // channels per block
     static constexpr int NSTRIP = (HW + 1) / 2;            // strips of two output columns
     static constexpr int RR = HW <= 8 ? 4 : 7;             // output rows per run
@@ -77,6 +86,8 @@ struct DwPwGemmGeom {
     static constexpr int NBOXB = (NPAD + 63) / 64;
     static constexpr int BSLOT = NBOXB * BOX;              // B tile: CB rows x NPAD pixels
     static constexpr int XSLOT = (CB * P * 4 + 127) / 128 * 128;
+    static constexpr int CHUNK = 128 * 16 * 4;             // 128 rows x 16 fp32 columns
+    static constexpr int NOWN = (NCH + 1) / 2;             // chunks a rank of a 2-CTA cluster owns, at most
     static_assert(CB * UPP <= THREADS, "one work unit per thread");
     static_assert(CB % 16 == 0, "K = 16 steps");
 };
@@ -84,10 +95,18 @@ struct DwPwGemmGeom {
 constexpr int kDwPwGemmFSlots = 3;
 constexpr int kDwPwGemmBars = 2 /*xfull*/ + 3 /*ffull*/ + 2 /*mma_done*/ + 1 /*accf*/ + 1 /*drain*/;
 
+// shared memory: filter ring, B ring, x ring, the receive area of the cluster reduction (MT x
+// NOWN chunks), barriers
 template <int HW>
-__host__ __device__ constexpr int dwpw_gemm_smem(int fslot) {
+__host__ __device__ constexpr int dwpw_gemm_recv(int MT, int S) {
+    return S > 1 ? MT * DwPwGemmGeom<HW>::NOWN * DwPwGemmGeom<HW>::CHUNK : 0;
+}
+
+template <int HW>
+__host__ __device__ constexpr int dwpw_gemm_smem(int fslot, int MT, int S) {
     using G = DwPwGemmGeom<HW>;
-    return 1024 + kDwPwGemmFSlots * fslot + 2 * G::BSLOT + 2 * G::XSLOT + kDwPwGemmBars * 8 + 16;
+    return 1024 + kDwPwGemmFSlots * fslot + 2 * G::BSLOT + 2 * G::XSLOT + dwpw_gemm_recv<HW>(MT, S) +
+           kDwPwGemmBars * 8 + 16;
 }
 
 // One bf16 value into the B tile: row k (channel in the block), column n (pixel); 64 pixels per
@@ -112,7 +131,8 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     const uint32_t sF = base;
     const uint32_t sB = sF + kDwPwGemmFSlots * p.fslot;
     const uint32_t sX = sB + 2 * G::BSLOT;
-    const uint32_t bars = sX + 2 * G::XSLOT;
+    const uint32_t sR = sX + 2 * G::XSLOT;   // receive area of the reduction
+    const uint32_t bars = sR + dwpw_gemm_recv<HW>(p.MT, p.S);
     auto xfull = [&](int s) { return bars + 8u * s; };
     auto ffull = [&](int s) { return bars + 16u + 8u * s; };
     auto mma_done = [&](int s) { return bars + 40u + 8u * s; };
@@ -120,6 +140,10 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     const uint32_t drain = bars + 64u;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + (bars - base) + kDwPwGemmBars * 8);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int S = p.S;
+    const int rank = S > 1 ? static_cast<int>(cluster_rank()) : 0;
+    const int cluster = static_cast<int>(blockIdx.x) / S;
+    const int nclusters = static_cast<int>(gridDim.x) / S;
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) mbar_init(xfull(s), 1);
@@ -139,18 +163,16 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    const int my_tiles = p.num_tiles > static_cast<int>(blockIdx.x)
-                             ? (p.num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                                   static_cast<int>(gridDim.x)
-                             : 0;
-    const int total = my_tiles * p.nblk;   // channel blocks this CTA walks, over all its tiles
+    const int my_tiles = p.num_tiles > cluster ? (p.num_tiles - cluster + nclusters - 1) / nclusters : 0;
+    const int nb = (p.nblk - rank + S - 1) / S;   // this rank's blocks per image: rank, rank + S, ...
+    const int total = my_tiles * nb;
     // block g of this CTA -> image and first channel
     auto block_at = [&](int g, int &n, int &c0) {
-        n = static_cast<int>(blockIdx.x) + (g / p.nblk) * static_cast<int>(gridDim.x);
-        c0 = (g % p.nblk) * G::CB;
+        n = cluster + (g / nb) * nclusters;
+        c0 = (rank + (g % nb) * S) * G::CB;
     };
     int x_issued = 0, f_issued = 0;   // thread 0: blocks whose copies are in flight or landed
-    auto issue_x = [&](int g) {   // thread 0
+    auto issue_x = [&](int g) {       // thread 0
         int n, c0;
         block_at(g, n, c0);
         x_issued = g + 1;
@@ -159,7 +181,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
         mbar_arrive_expect_tx(xfull(g & 1), bytes);
         bulk_g2s(sX + (g & 1) * G::XSLOT, x + (static_cast<long long>(n) * p.C + c0) * G::P, bytes, xfull(g & 1));
     };
-    auto issue_f = [&](int g) {   // thread 0
+    auto issue_f = [&](int g) {       // thread 0
         int n, c0;
         block_at(g, n, c0);
         f_issued = g + 1;
@@ -189,171 +211,212 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     for (int t = 0; t < WIN; ++t) colok[t] = ix0 + t >= 0 && ix0 + t < HW;
     const bool second = ox0 + 1 < HW;   // the strip's second column exists
 
-    bool ok = true;
-    int stop = 0;   // the block at which a wait ran out
-    int tile_parity = 0;
-    for (int g = 0; g < total; ++g) {
-        int n, c0;
-        block_at(g, n, c0);
-        const int kb = g % p.nblk;
-        // the block's planes staged; the B slot's previous MMAs (block g - 2) done
-        bool good = mbar_wait_warp(xfull(g & 1), (g >> 1) & 1);
-        if (good && g >= 2) good = mbar_wait_warp(mma_done(g & 1), ((g - 2) >> 1) & 1);
-        if (__syncthreads_or(!good)) { ok = false; stop = g; break; }
-
+    // depthwise outputs of block g (channel c0 + cl of the image) into the B slot, bf16
+    auto depthwise_block = [&](int g, int c0) {
         uint8_t *bslot = smem + (sB - base) + (g & 1) * G::BSLOT;
-        if (unit_ok) {
-            const int c = c0 + cl;
-            if (c < p.C) {
-                const float *xs = reinterpret_cast<const float *>(smem + (sX - base) + (g & 1) * G::XSLOT) + cl * G::P;
-                float wr[KC * KC];
+        const int c = c0 + cl;
+        if (c < p.C) {
+            const float *xs = reinterpret_cast<const float *>(smem + (sX - base) + (g & 1) * G::XSLOT) + cl * G::P;
+            float wr[KC * KC];
 #pragma unroll
-                for (int t = 0; t < KC * KC; ++t) wr[t] = __ldg(w + static_cast<long long>(c) * (KC * KC) + t);
-                const float bv = p.b_dw ? __ldg(p.b_dw + c) : 0.0f;
-                uint64_t w2[KC * KC];
+            for (int t = 0; t < KC * KC; ++t) wr[t] = __ldg(w + static_cast<long long>(c) * (KC * KC) + t);
+            const float bv = p.b_dw ? __ldg(p.b_dw + c) : 0.0f;
+            uint64_t w2[KC * KC];
 #pragma unroll
-                for (int t = 0; t < KC * KC; ++t) w2[t] = dw_pack(wr[t], wr[t]);
-                // ring of KC input rows, each as KC overlapping pairs (x[t], x[t+1])
-                uint64_t ring[KC][KC];
-                auto load_pairs = [&](int iy, uint64_t (&dst)[KC]) {
-                    float f[WIN];
-                    const bool rowok = iy >= 0 && iy < HW;
+            for (int t = 0; t < KC * KC; ++t) w2[t] = dw_pack(wr[t], wr[t]);
+            // ring of KC input rows, each as KC overlapping pairs (x[t], x[t+1])
+            uint64_t ring[KC][KC];
+            auto load_pairs = [&](int iy, uint64_t (&dst)[KC]) {
+                float f[WIN];
+                const bool rowok = iy >= 0 && iy < HW;
 #pragma unroll
-                    for (int t = 0; t < WIN; ++t) f[t] = (rowok && colok[t]) ? xs[iy * HW + ix0 + t] : 0.0f;
+                for (int t = 0; t < WIN; ++t) f[t] = (rowok && colok[t]) ? xs[iy * HW + ix0 + t] : 0.0f;
 #pragma unroll
-                    for (int t = 0; t < KC; ++t) dst[t] = dw_pack(f[t], f[t + 1]);
-                };
+                for (int t = 0; t < KC; ++t) dst[t] = dw_pack(f[t], f[t + 1]);
+            };
 #pragma unroll
-                for (int q = 0; q < KC - 1; ++q) load_pairs(oy_first - PAD + q, ring[q]);
+            for (int q = 0; q < KC - 1; ++q) load_pairs(oy_first - PAD + q, ring[q]);
 #pragma unroll
-                for (int i = 0; i < G::RR; ++i) {
-                    const int oy = oy_first + i;
-                    if (oy < HW) {
-                        load_pairs(oy - PAD + KC - 1, ring[(i + KC - 1) % KC]);
-                        float a0, a1;
-                        if constexpr (MODE == 0) {
-                            a0 = 0.0f;
-                            a1 = 0.0f;
+            for (int i = 0; i < G::RR; ++i) {
+                const int oy = oy_first + i;
+                if (oy < HW) {
+                    load_pairs(oy - PAD + KC - 1, ring[(i + KC - 1) % KC]);
+                    float a0, a1;
+                    if constexpr (MODE == 0) {
+                        a0 = 0.0f;
+                        a1 = 0.0f;
 #pragma unroll
-                            for (int ky = 0; ky < KC; ++ky)
+                        for (int ky = 0; ky < KC; ++ky)
 #pragma unroll
-                                for (int kx = 0; kx < KC; ++kx)
-                                    dw_tap2_exact(a0, a1, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
-                        } else {
-                            uint64_t a2 = dw_pack(0.0f, 0.0f);
+                            for (int kx = 0; kx < KC; ++kx)
+                                dw_tap2_exact(a0, a1, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
+                    } else {
+                        uint64_t a2 = dw_pack(0.0f, 0.0f);
 #pragma unroll
-                            for (int ky = 0; ky < KC; ++ky)
+                        for (int ky = 0; ky < KC; ++ky)
 #pragma unroll
-                                for (int kx = 0; kx < KC; ++kx)
-                                    a2 = dw_tap2_fast(a2, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
-                            dw_unpack(a2, a0, a1);
-                        }
-                        if (p.b_dw) {
-                            a0 = dw_finish<MODE, true>(a0, bv);
-                            a1 = dw_finish<MODE, true>(a1, bv);
-                        } else {
-                            a0 = dw_finish<MODE, false>(a0, 0.0f);
-                            a1 = dw_finish<MODE, false>(a1, 0.0f);
-                        }
-                        const int pix = oy * HW + ox0;
-                        dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
-                        if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
+                            for (int kx = 0; kx < KC; ++kx)
+                                a2 = dw_tap2_fast(a2, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
+                        dw_unpack(a2, a0, a1);
                     }
+                    if (p.b_dw) {
+                        a0 = dw_finish<MODE, true>(a0, bv);
+                        a1 = dw_finish<MODE, true>(a1, bv);
+                    } else {
+                        a0 = dw_finish<MODE, false>(a0, 0.0f);
+                        a1 = dw_finish<MODE, false>(a1, 0.0f);
+                    }
+                    const int pix = oy * HW + ox0;
+                    dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
+                    if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
                 }
-            } else {
-                // channels past C: zero rows, so that the zero filter rows meet finite values
-                const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
-                for (int i = 0; i < G::RR; ++i) {
-                    const int oy = oy_first + i;
-                    if (oy < HW) {
-                        dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0, z);
-                        if (second) dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0 + 1, z);
+            }
+        } else {
+            // channels past C: zero rows, so that the zero filter rows meet finite values
+            const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
+            for (int i = 0; i < G::RR; ++i) {
+                const int oy = oy_first + i;
+                if (oy < HW) {
+                    dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0, z);
+                    if (second) dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0 + 1, z);
+                }
+            }
+        }
+    };
+
+    // 16 consecutive pixels of output channel o: acc (+ the cluster peer's partial) + bias -> y
+    auto store_chunk = [&](float *yrow, int p0, const float (&v)[16], float bp) {
+        if constexpr (G::P % 4 == 0) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (p0 + 4 * u < G::P)
+                    *reinterpret_cast<float4 *>(yrow + p0 + 4 * u) =
+                        make_float4(__fadd_rn(v[4 * u], bp), __fadd_rn(v[4 * u + 1], bp),
+                                    __fadd_rn(v[4 * u + 2], bp), __fadd_rn(v[4 * u + 3], bp));
+        } else {
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                if (p0 + u < G::P) yrow[p0 + u] = __fadd_rn(v[u], bp);
+        }
+    };
+
+    // Every thread walks every tile and every block; after a wait ran out (dead) it skips the
+    // work but still takes each CTA and cluster barrier, so neither this CTA nor its cluster
+    // peer ever waits for it forever.
+    bool dead = false, fail = false;   // fail: thread 0's own waits, or'ed in at the next barrier
+    int stop = 0;                      // the first block whose wait ran out
+    int g = 0;
+    for (int tl = 0; tl < my_tiles; ++tl) {
+        const int n = cluster + tl * nclusters;
+        for (int j = 0; j < nb; ++j, ++g) {
+            int nn, c0;
+            block_at(g, nn, c0);
+            bool good = true;
+            if (!dead) {
+                // the block's planes staged; the B slot's previous MMAs (block g - 2) done
+                good = mbar_wait_warp(xfull(g & 1), (g >> 1) & 1);
+                if (good && g >= 2) good = mbar_wait_warp(mma_done(g & 1), ((g - 2) >> 1) & 1);
+                if (good && unit_ok) depthwise_block(g, c0);
+                fence_proxy_async_smem();   // the B tile's generic writes, visible to the tensor cores
+            }
+            if (__syncthreads_or(!good || fail) && !dead) {
+                dead = true;
+                stop = g;
+            }
+            if (!dead && tid == 0) {
+                if (!mbar_wait(ffull(g % 3), (g / 3) & 1)) {
+                    fail = true;
+                } else {
+                    tc_fence_after();
+                    const uint32_t fs = sF + (g % 3) * p.fslot;
+                    const uint32_t bs = sB + (g & 1) * G::BSLOT;
+#pragma unroll
+                    for (int kk = 0; kk < G::CB / 16; ++kk) {
+                        const uint64_t bd = smem_desc_sw128(bs + kk * 2048, G::BOX, 1024);
+                        for (int mt = 0; mt < p.MT; ++mt) {
+                            const uint64_t ad = smem_desc_sw128(fs + mt * 2 * G::BOX + kk * 2048, G::BOX, 1024);
+                            umma_f16_ss(tmem + mt * G::NPAD, ad, bd, p.idesc, (j | kk) != 0 ? 1u : 0u);
+                        }
+                    }
+                    umma_commit(mma_done(g & 1));
+                    if (j == nb - 1) umma_commit(accf);
+                    // refill: x two blocks ahead into the slot this block has read; F two blocks
+                    // ahead into the slot block g - 1 used, once its MMAs are done
+                    if (g + 2 < total) {
+                        issue_x(g + 2);
+                        if (g >= 1 && !mbar_wait(mma_done((g - 1) & 1), ((g - 1) >> 1) & 1)) fail = true;
+                        else issue_f(g + 2);
                     }
                 }
             }
         }
-        fence_proxy_async_smem();   // the B tile's generic writes, visible to the tensor cores
-        __syncthreads();
 
-        int fail = 0;
-        if (tid == 0) {
-            if (!mbar_wait(ffull(g % 3), (g / 3) & 1)) fail = 1;
-            if (!fail) {
-                tc_fence_after();
-                const uint32_t fs = sF + (g % 3) * p.fslot;
-                const uint32_t bs = sB + (g & 1) * G::BSLOT;
-#pragma unroll
-                for (int kk = 0; kk < G::CB / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(bs + kk * 2048, G::BOX, 1024);
-                    for (int mt = 0; mt < p.MT; ++mt) {
-                        const uint64_t ad = smem_desc_sw128(fs + mt * 2 * G::BOX + kk * 2048, G::BOX, 1024);
-                        umma_f16_ss(tmem + mt * G::NPAD, ad, bd, p.idesc, (kb | kk) != 0 ? 1u : 0u);
-                    }
-                }
-                umma_commit(mma_done(g & 1));
-                if (kb == p.nblk - 1) umma_commit(accf);
-                // refill: x two blocks ahead into the slot this block has read; F two blocks
-                // ahead into the slot block g - 1 used, once its MMAs are done
-                if (g + 2 < total) {
-                    issue_x(g + 2);
-                    if (g >= 1 && !mbar_wait(mma_done((g - 1) & 1), ((g - 1) >> 1) & 1)) fail = 1;
-                    if (!fail) issue_f(g + 2);
-                }
-            }
+        // ------------------------------- epilogue of image n -------------------------------
+        bool got = true;
+        if (!dead) got = mbar_wait_warp(accf, tl & 1);
+        if (__syncthreads_or(!got || fail) && !dead) {
+            dead = true;
+            stop = g;
         }
-        if (__syncthreads_or(fail)) { ok = false; stop = g; break; }
-
-        if (kb == p.nblk - 1) {
-            // ------------------------------- epilogue of image n -------------------------------
-            const bool got = mbar_wait_warp(accf, tile_parity);
-            tile_parity ^= 1;
-            tc_fence_after();
-            if (got) {
-                const int q = warp & 3, cg = warp >> 2;
-                for (int mt = 0; mt < p.MT; ++mt) {
-                    const int o = mt * 128 + q * 32 + lane;
-                    const float bp = (p.b_pw && o < p.Cout) ? __ldg(p.b_pw + o) : 0.0f;
-                    float *yrow = y + (static_cast<long long>(n) * p.Cout + o) * G::P;
-                    for (int j = cg; j < G::NPAD / 16; j += 4) {
+        tc_fence_after();
+        const int q = warp & 3, cg = warp >> 2;   // TMEM lane quarter; a quarter of the chunks
+        if (S > 1) {
+            // the chunks the peer owns: this rank's partial into the peer's receive area
+            if (!dead) {
+                const uint32_t peer_r = map_rank(sR, static_cast<uint32_t>(rank ^ 1));
+                for (int mt = 0; mt < p.MT; ++mt)
+                    for (int jc = cg; jc < G::NCH; jc += 4) {
+                        if ((jc & 1) == rank) continue;
                         uint32_t v[16];
-                        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + mt * G::NPAD + j * 16, v);
+                        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + mt * G::NPAD + jc * 16, v);
                         tmem_wait_ld();
-                        if (o < p.Cout) {
-                            const int p0 = j * 16;
-                            if constexpr (G::P % 4 == 0) {
+                        const uint32_t dst = peer_r + ((mt * G::NOWN + (jc >> 1)) * 128 + q * 32 + lane) * 64;
 #pragma unroll
-                                for (int u = 0; u < 4; ++u)
-                                    if (p0 + 4 * u < G::P)
-                                        *reinterpret_cast<float4 *>(yrow + p0 + 4 * u) =
-                                            make_float4(__fadd_rn(__uint_as_float(v[4 * u]), bp),
-                                                        __fadd_rn(__uint_as_float(v[4 * u + 1]), bp),
-                                                        __fadd_rn(__uint_as_float(v[4 * u + 2]), bp),
-                                                        __fadd_rn(__uint_as_float(v[4 * u + 3]), bp));
-                            } else {
-#pragma unroll
-                                for (int u = 0; u < 16; ++u)
-                                    if (p0 + u < G::P) yrow[p0 + u] = __fadd_rn(__uint_as_float(v[u]), bp);
-                            }
-                        }
+                        for (int u = 0; u < 4; ++u)
+                            st_cluster_v4(dst + 16 * u, v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
                     }
+            }
+            cluster_sync_all();   // the partials have landed in the owners' receive areas
+        }
+        if (!dead) {
+            for (int mt = 0; mt < p.MT; ++mt) {
+                const int o = mt * 128 + q * 32 + lane;
+                const float bp = (p.b_pw && o < p.Cout) ? __ldg(p.b_pw + o) : 0.0f;
+                float *yrow = y + (static_cast<long long>(n) * p.Cout + (o < p.Cout ? o : 0)) * G::P;
+                for (int jc = cg; jc < G::NCH; jc += 4) {
+                    if (S > 1 && (jc & 1) != rank) continue;
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + mt * G::NPAD + jc * 16, v);
+                    tmem_wait_ld();
+                    float sum[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) sum[u] = __uint_as_float(v[u]);
+                    if (S > 1) {
+                        // the two partials added once (an IEEE sum of two terms: the same bits
+                        // whichever rank adds them)
+                        const float *rv = reinterpret_cast<const float *>(
+                            smem + (sR - base) + ((mt * G::NOWN + (jc >> 1)) * 128 + q * 32 + lane) * 64);
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) sum[u] = __fadd_rn(sum[u], rv[u]);
+                    }
+                    if (o < p.Cout) store_chunk(yrow, jc * 16, sum, bp);
                 }
             }
-            tc_fence_before();
-            if (__syncthreads_or(!got)) { ok = false; stop = g; break; }
-            tc_fence_after();
         }
+        if (S > 1) cluster_sync_all();   // the receive area is read before the next image's partials
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
     }
 
-    if (!ok) {
-        if (tid == 0) {
-            atomicOr(status, kStatusTimeout);
-            // every copy issued lands, and every MMA issued completes, before the CTA exits
-            // (bounded waits): the copies of blocks stop .. issued - 1 were not waited for yet
-            for (int j = stop; j < x_issued; ++j) mbar_wait(xfull(j & 1), (j >> 1) & 1);
-            for (int j = stop; j < f_issued; ++j) mbar_wait(ffull(j % 3), (j / 3) & 1);
-            umma_commit(drain);
-            mbar_wait(drain, 0);
-        }
+    if (dead && tid == 0) {
+        atomicOr(status, kStatusTimeout);
+        // every copy issued lands, and every MMA issued completes, before the CTA exits
+        // (bounded waits): the copies of blocks stop .. issued - 1 were not waited for yet
+        for (int jj = stop; jj < x_issued; ++jj) mbar_wait(xfull(jj & 1), (jj >> 1) & 1);
+        for (int jj = stop; jj < f_issued; ++jj) mbar_wait(ffull(jj % 3), (jj / 3) & 1);
+        umma_commit(drain);
+        mbar_wait(drain, 0);
     }
     tc_fence_before();
     __syncthreads();

@@ -122,9 +122,13 @@ GEMM_CASES = [(2, 72, 14, 3, 112, 0, True), (3, 100, 7, 5, 160, 1, True), (2, 64
               (200, 4, 7, 5, 24, 1, True)]
 
 
+@pytest.mark.parametrize("split", ["1", "2"])
 @pytest.mark.parametrize("c", GEMM_CASES, ids=lambda c: "N{}C{}H{}K{}-O{}-{}".format(*c[:5], "exact" if c[5] == 0 else "fast"))
-def test_transposed_gemm_kernel(cb, c, monkeypatch):
+def test_transposed_gemm_kernel(cb, c, split, monkeypatch):
+    # one CTA per image, or a 2-CTA cluster that splits the channel blocks and adds the two
+    # partial sums through distributed shared memory
     monkeypatch.setenv("CONV_B200_DWPW_KERNEL", "gemm")
+    monkeypatch.setenv("CONV_B200_DWPW_SPLIT", split)
     N, C, H, K, Cout, mode, bias = c
     case = workloads.DwPwCase("t", N, C, H, H, K, 1, (K - 1) // 2, 1, Cout, bias, seed=C + K + Cout + N)
     x, w, bd, F, bp = workloads.dwpw_inputs(case)
@@ -134,14 +138,19 @@ def test_transposed_gemm_kernel(cb, c, monkeypatch):
     assert np.all(np.isfinite(y))
     bad = np.abs(y - ref) > _tol(C) * absum
     assert not bad.any(), f"{bad.sum()} outputs out of tolerance"
+    y2, _ = _run(cb, case, x, w, bd, F, bp, mode)
+    assert np.array_equal(y, y2)   # a given split repeats its bits
 
 
+@pytest.mark.parametrize("split", ["1", "2"])
 @pytest.mark.parametrize("hw,K", [(14, 3), (7, 5)])
 @pytest.mark.parametrize("mode", [0, 1])
-def test_transposed_gemm_identity_mixing_is_exact(cb, hw, K, mode, monkeypatch):
-    # F = I: every output is one exact product plus zeros, so the block must equal the depthwise
-    # output rounded to bf16, bit for bit (the depthwise stage of this kernel is the page's order)
+def test_transposed_gemm_identity_mixing_is_exact(cb, hw, K, mode, split, monkeypatch):
+    # F = I: every output is one exact product plus zeros (also each of the two partial sums of
+    # a split), so the block must equal the depthwise output rounded to bf16, bit for bit (the
+    # depthwise stage of this kernel is the page's order)
     monkeypatch.setenv("CONV_B200_DWPW_KERNEL", "gemm")
+    monkeypatch.setenv("CONV_B200_DWPW_SPLIT", split)
     case = workloads.DwPwCase("t", 3, 96, hw, hw, K, 1, (K - 1) // 2, 1, 96, True, seed=hw + K)
     x, w, bd, _, _ = workloads.dwpw_inputs(case)
     F = workloads.bf16_bits(np.eye(96, dtype=np.float32))
