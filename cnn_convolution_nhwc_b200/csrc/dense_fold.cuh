@@ -203,50 +203,52 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (!mbar_wait_warp(hfull(j % p.HS), (j / p.HS) & 1u)) { if (lane == 0) fail(); break; }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
+        // The whole warp walks the loop, converged; the MMAs and commits are predicated on one
+        // elected lane (all of them, so that each commit tracks every MMA of the warp).
+        const uint32_t leader = elect_one_sync();
         uint32_t hit = 0, local = 0;
         bool ok = mbar_wait_warp(bfull(0), 0);
-        for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step, ++local) {
+        for (int t = first; t < p.num_tiles && ok && !__any_sync(0xffffffffu, *abort_flag != 0);
+             t += step, ++local) {
             const uint32_t b = local & 1u;
             // the epilogue is the slower role: sleep between polls instead of taking its issue slots
             if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + b * NF;
-            for (int cb = 0; cb < p.num_cblk; ++cb) {
+            for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
                 const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
                 if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t filter_ok = 1;
-                if (lane == 0) {
-                    // filter row i reads the halo from row i*W on (start field in 16-byte
-                    // units: +8 per 128-byte row, +2 per 16 channels); B spans the K slots
-                    // (i, 0..K-1), 8 KB apart (the leading-byte offset), +128 per 16 channels
-                    const uint64_t a0 = smem_desc_sw128(sH + hs * p.halo_bytes, 16, 1024);
+                // filter row i reads the halo from row i*W on (start field in 16-byte units: +8
+                // per 128-byte row, +2 per 16 channels); B spans the K slots (i, 0..K-1), 8 KB
+                // apart (the leading-byte offset), +128 per 16 channels
+                const uint64_t a0 = smem_desc_sw128(sH + hs * p.halo_bytes, 16, 1024);
 #pragma unroll
-                    for (int i = 0; i < K; ++i) {
-                        if (local == 0 && cb == 0 && i > 0 && !mbar_wait(bfull(i), 0)) { filter_ok = 0; break; }
-                        const uint64_t ad = a0 + static_cast<uint64_t>(i * p.W * 8);
-                        const uint64_t bd = smem_desc_sw128(sB + (cb * p.KK + i * K) * Cfg::SLOT_BYTES,
-                                                            Cfg::SLOT_BYTES, 1024);
-                        umma_f16_ss(d_tmem, ad, bd, Cfg::IDESC, (cb | i) != 0 ? 1u : 0u);
-                        umma_f16_ss(d_tmem, ad + 2, bd + 128, Cfg::IDESC, 1u);
-                        umma_f16_ss(d_tmem, ad + 4, bd + 256, Cfg::IDESC, 1u);
-                        umma_f16_ss(d_tmem, ad + 6, bd + 384, Cfg::IDESC, 1u);
+                for (int i = 0; i < K; ++i) {
+                    // the first tile's filter rows arrive one by one
+                    if (local == 0 && cb == 0 && i > 0) {
+                        if (!mbar_wait_warp(bfull(i), 0)) { ok = false; break; }
+                        tc_fence_after();
                     }
-                    umma_commit(hempty(hs));
+                    const uint64_t ad = a0 + static_cast<uint64_t>(i * p.W * 8);
+                    const uint64_t bd = smem_desc_sw128(sB + (cb * p.KK + i * K) * Cfg::SLOT_BYTES,
+                                                        Cfg::SLOT_BYTES, 1024);
+                    umma_f16_ss_if(d_tmem, ad, bd, Cfg::IDESC, (cb | i) != 0 ? 1u : 0u, leader);
+                    umma_f16_ss_if(d_tmem, ad + 2, bd + 128, Cfg::IDESC, 1u, leader);
+                    umma_f16_ss_if(d_tmem, ad + 4, bd + 256, Cfg::IDESC, 1u, leader);
+                    umma_f16_ss_if(d_tmem, ad + 6, bd + 384, Cfg::IDESC, 1u, leader);
                 }
-                if (!__shfl_sync(0xffffffffu, filter_ok, 0)) { ok = false; break; }
+                if (!ok) break;
+                umma_commit_if(hempty(hs), leader);
                 ++hit;
             }
             if (!ok) break;
-            if (lane == 0) umma_commit(accf(b));
-            __syncwarp();
-        }
-        if (!ok && lane == 0) fail();
-        if (lane == 0) {
-            umma_commit(done_bar);
-            if (!mbar_wait(done_bar, 0)) fail();
+            umma_commit_if(accf(b), leader);
         }
         __syncwarp();
+        if (!ok && lane == 0) fail();
+        umma_commit_if(done_bar, leader);
+        if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
     } else {
         // ------------------------------- Epilogue -----------------------------------
         // warp e = warp - 2: TMEM lane quarter q = warp % 4 (the quarter a warp may access),

@@ -226,10 +226,13 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (!mbar_wait_warp(bfull(j % p.BS), (j / p.BS) & 1u)) { if (lane == 0) fail(); break; }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
+        // The whole warp walks the loop, converged; the MMAs and commits are predicated on one
+        // elected lane (all of them, so that each commit tracks every MMA of the warp).
+        const uint32_t leader = elect_one_sync();
         uint32_t hit = 0, bit = 0, local = 0;
         bool ok = true;
         if (BRES && !mbar_wait_warp(bfull(0), 0)) ok = false;
-        for (int t = first; t < count && ok && !*abort_flag; t += step, ++local) {
+        for (int t = first; t < count && ok && !__any_sync(0xffffffffu, *abort_flag != 0); t += step, ++local) {
             const uint32_t b = local & 1u;
             // waiting here means the epilogue is the slower role: sleep between polls instead
             // of taking its issue slots
@@ -242,61 +245,55 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 tc_fence_after();
                 const uint32_t halo = sH + hs * p.halo_bytes;
                 if (BRES) {
-                    // filter resident: lane 0 issues the whole channel block (all taps x 4
-                    // K-steps) back to back; tap (ky, kx) reads the halo from row ky*W + kx on
-                    if (lane == 0) {
-                        // descriptors differ only in the start-address field (16-byte units):
-                        // +2 per 16 channels of A, +128 per 16 reduction rows of B
-                        const uint64_t a0 = smem_desc_sw128(halo, 16, 1024);
-                        uint64_t bd = smem_desc_sw128(sB + cb * p.KK * Cfg::B_BYTES, Cfg::B_BOX_BYTES, 1024);
-                        const uint32_t accumulate_first = cb != 0 ? 1u : 0u;
-                        uint32_t row = 0;
-                        for (int ky = 0; ky < p.K; ++ky, row += p.W) {
-                            for (int kx = 0; kx < p.K; ++kx, bd += Cfg::B_BYTES >> 4) {
-                                const uint64_t ad = a0 + static_cast<uint64_t>((row + kx) * 8u);
-                                umma_f16_ss(d_tmem, ad, bd, Cfg::IDESC, (ky | kx) != 0 ? 1u : accumulate_first);
-                                umma_f16_ss(d_tmem, ad + 2, bd + 128, Cfg::IDESC, 1u);
-                                umma_f16_ss(d_tmem, ad + 4, bd + 256, Cfg::IDESC, 1u);
-                                umma_f16_ss(d_tmem, ad + 6, bd + 384, Cfg::IDESC, 1u);
-                            }
+                    // filter resident: the whole channel block (all taps x 4 K-steps) back to
+                    // back; tap (ky, kx) reads the halo from row ky*W + kx on. Descriptors
+                    // differ only in the start-address field (16-byte units): +2 per 16
+                    // channels of A, +128 per 16 reduction rows of B
+                    const uint64_t a0 = smem_desc_sw128(halo, 16, 1024);
+                    uint64_t bd = smem_desc_sw128(sB + cb * p.KK * Cfg::B_BYTES, Cfg::B_BOX_BYTES, 1024);
+                    const uint32_t accumulate_first = cb != 0 ? 1u : 0u;
+                    uint32_t row = 0;
+                    for (int ky = 0; ky < p.K; ++ky, row += p.W) {
+                        for (int kx = 0; kx < p.K; ++kx, bd += Cfg::B_BYTES >> 4) {
+                            const uint64_t ad = a0 + static_cast<uint64_t>((row + kx) * 8u);
+                            umma_f16_ss_if(d_tmem, ad, bd, Cfg::IDESC, (ky | kx) != 0 ? 1u : accumulate_first, leader);
+                            umma_f16_ss_if(d_tmem, ad + 2, bd + 128, Cfg::IDESC, 1u, leader);
+                            umma_f16_ss_if(d_tmem, ad + 4, bd + 256, Cfg::IDESC, 1u, leader);
+                            umma_f16_ss_if(d_tmem, ad + 6, bd + 384, Cfg::IDESC, 1u, leader);
                         }
                     }
-                    __syncwarp();
                 } else {
-                    int ky = 0, kx = 0;
+                    uint32_t row8 = 0;   // (ky*W + kx) * 8: A start of tap (ky, kx), 16-byte units
+                    const uint32_t row_skip8 = static_cast<uint32_t>(p.W - p.K) * 8u;
+                    const uint64_t a0 = smem_desc_sw128(halo, 16, 1024);
+                    const uint64_t b0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
+                    int kx = 0;
                     for (int tap = 0; tap < p.KK; ++tap) {
                         const uint32_t bs = bit % p.BS, bph = (bit / p.BS) & 1u;
                         if (!mbar_wait_warp(bfull(bs), bph)) { ok = false; break; }
                         tc_fence_after();
-                        if (lane == 0) {
-                            const uint32_t a_row = halo + static_cast<uint32_t>(ky * p.W + kx) * 128u;
-                            const uint32_t bslot = sB + bs * Cfg::B_BYTES;
+                        const uint64_t ad = a0 + row8;
+                        const uint64_t bd = b0 + bs * (Cfg::B_BYTES >> 4);
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                umma_f16_ss(d_tmem, smem_desc_sw128(a_row + kk * 32, 16, 1024),
-                                            smem_desc_sw128(bslot + kk * 2048, Cfg::B_BOX_BYTES, 1024),
-                                            Cfg::IDESC, (cb | tap | kk) != 0 ? 1u : 0u);
-                            umma_commit(bempty(bs));
-                        }
-                        __syncwarp();
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16_ss_if(d_tmem, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC,
+                                           (cb | tap | kk) != 0 ? 1u : 0u, leader);
+                        umma_commit_if(bempty(bs), leader);
                         ++bit;
-                        if (++kx == p.K) { kx = 0; ++ky; }
+                        row8 += 8u;
+                        if (++kx == p.K) { kx = 0; row8 += row_skip8; }
                     }
                 }
-                if (lane == 0) umma_commit(hempty(hs));
-                __syncwarp();
+                umma_commit_if(hempty(hs), leader);
                 ++hit;
             }
             if (!ok) break;
-            if (lane == 0) umma_commit(accf(b));
-            __syncwarp();
-        }
-        if (!ok && lane == 0) fail();
-        if (lane == 0) {
-            umma_commit(done_bar);
-            if (!mbar_wait(done_bar, 0)) fail();
+            umma_commit_if(accf(b), leader);
         }
         __syncwarp();
+        if (!ok && lane == 0) fail();
+        umma_commit_if(done_bar, leader);
+        if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
     } else {
         // ------------------------------- Epilogue -----------------------------------
         const int q = warp & 3;             // TMEM lane quarter this warp may access

@@ -152,7 +152,10 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     // The role loops keep their ring slots and phases as running counters and advance the MMA
     // descriptors by adding to their address fields: the MMA warp is one serial instruction
     // stream, and every instruction of its loop delays the next MMA (a loop with a division per
-    // slot was measured at ~440 cycles per 4-MMA slot against ~260 of tensor work).
+    // slot was measured at ~440 cycles per 4-MMA slot against ~260 of tensor work). The MMA
+    // warp also stays converged (predicated MMAs, no one-lane branch): measured on B200, a loop
+    // that waits, fences and issues four M=128, N=128 MMAs per slot takes ~310 cycles per slot
+    // that way against ~590 with the MMAs under `if (lane == 0)`.
     if (warp == Cfg::HALO_WARP) {
         // ------------------------------- halo producer ------------------------------
         uint32_t hit = 0, hs = 0, hph = 0;
@@ -201,6 +204,10 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             if (!mbar_wait_warp(bfull(j % p.BS), (j / p.BS) & 1u)) { if (lane == 0) fail(); break; }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
+        // The whole warp runs the loop, converged; the MMAs and commits are predicated on one
+        // elected lane (every commit of this warp comes from that lane, so that each commit
+        // tracks all of the warp's MMAs).
+        const uint32_t leader = elect_one_sync();
         uint32_t local = 0, hs = 0, hph = 0, bs = 0, bph = 0;
         bool ok = true;
         // descriptors differ only in the start-address field (16-byte units): A +4 per 64-byte
@@ -209,7 +216,8 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const uint64_t b_desc0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
         constexpr uint32_t kSlotUnits = Cfg::B_BYTES >> 4;
         const uint32_t row_skip4 = static_cast<uint32_t>(p.W - p.K) * 4u;
-        for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step, ++local) {
+        for (int t = first; t < p.num_tiles && ok && !__any_sync(0xffffffffu, *abort_flag != 0);
+             t += step, ++local) {
             const uint32_t b = local & 1u;
             // waiting here means the epilogue is the slower role: sleep between polls
             if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
@@ -225,36 +233,29 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     for (int kx = 0; kx < p.K; ++kx, row4 += 4u) {
                         if (!mbar_wait_warp(bfull(bs), bph)) { ok = false; break; }
                         tc_fence_after();
-                        if (lane == 0) {
-                            const uint64_t ad = a_desc0 + row4;
-                            const uint64_t bd = b_desc0 + bs * kSlotUnits;
-                            const uint32_t acc = (cb | ky | kx) != 0 ? 1u : 0u;
-                            umma_f16_ss(d0, ad, bd, Cfg::IDESC, acc);
-                            umma_f16_ss(d1, ad + 512, bd, Cfg::IDESC, acc);
-                            umma_f16_ss(d0, ad + 2, bd + 128, Cfg::IDESC, 1u);
-                            umma_f16_ss(d1, ad + 514, bd + 128, Cfg::IDESC, 1u);
-                            umma_commit(bempty(bs));
-                        }
-                        __syncwarp();
+                        const uint64_t ad = a_desc0 + row4;
+                        const uint64_t bd = b_desc0 + bs * kSlotUnits;
+                        const uint32_t acc = (cb | ky | kx) != 0 ? 1u : 0u;
+                        umma_f16_ss_if(d0, ad, bd, Cfg::IDESC, acc, leader);
+                        umma_f16_ss_if(d1, ad + 512, bd, Cfg::IDESC, acc, leader);
+                        umma_f16_ss_if(d0, ad + 2, bd + 128, Cfg::IDESC, 1u, leader);
+                        umma_f16_ss_if(d1, ad + 514, bd + 128, Cfg::IDESC, 1u, leader);
+                        umma_commit_if(bempty(bs), leader);
                         if (++bs == static_cast<uint32_t>(p.BS)) { bs = 0; bph ^= 1u; }
                     }
                 }
                 if (!ok) break;
-                if (lane == 0) umma_commit(hempty(hs));
-                __syncwarp();
+                umma_commit_if(hempty(hs), leader);
                 if (++hs == static_cast<uint32_t>(p.HS)) { hs = 0; hph ^= 1u; }
             }
             if (!ok) break;
-            if (lane == 0) umma_commit(accf(b));
-            __syncwarp();
-        }
-        if (!ok && lane == 0) fail();
-        // All MMAs issued by this warp complete before TMEM is released.
-        if (lane == 0) {
-            umma_commit(done_bar);
-            if (!mbar_wait(done_bar, 0)) fail();
+            umma_commit_if(accf(b), leader);
         }
         __syncwarp();
+        if (!ok && lane == 0) fail();
+        // All MMAs issued by this warp complete before TMEM is released.
+        umma_commit_if(done_bar, leader);
+        if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
     } else {
         // ------------------------------- Epilogue (warps 2..9) -----------------------
         const int q = warp & 3;             // TMEM lane quarter this warp may access

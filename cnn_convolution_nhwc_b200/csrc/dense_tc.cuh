@@ -231,16 +231,19 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
             }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
-        // The whole warp walks the loop; lane 0 issues the MMAs and commits. The loop is one
-        // serial instruction stream, so the ring slot and phase are running counters and the
-        // descriptors advance by adding to their address fields (16-byte units).
+        // The whole warp walks the loop, converged; the MMAs and commits are predicated on one
+        // elected lane (all of them, so that each commit tracks every MMA of the warp). The loop
+        // is one serial instruction stream, so the ring slot and phase are running counters and
+        // the descriptors advance by adding to their address fields (16-byte units).
         // A: K-major, +2 per 16 channels (32 B inside the swizzle atom), 8-row groups 1024 B
         // apart. B: MN-major, +128 per 16 reduction rows (2048 B), 8-row groups 1024 B apart
         // (SBO), 64-channel boxes B_BOX_BYTES apart (LBO).
+        const uint32_t leader = elect_one_sync();
         const uint64_t a_desc0 = smem_desc_sw128(sA, 16, 1024);
         const uint64_t b_desc0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
         uint32_t it = 0, local = 0, s = 0, ph = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x, ++local) {
+        for (int tile = blockIdx.x; tile < p.num_tiles && !__any_sync(0xffffffffu, *abort_flag != 0);
+             tile += gridDim.x, ++local) {
             const uint32_t b = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
             // waiting here means the epilogue is the slower role: sleep between polls instead
@@ -259,31 +262,25 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                     break;
                 }
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t ad = a_desc0 + s * Cfg::A_UNITS;
-                    const uint64_t bd = b_desc0 + s * Cfg::B_UNITS;
+                const uint64_t ad = a_desc0 + s * Cfg::A_UNITS;
+                const uint64_t bd = b_desc0 + s * Cfg::B_UNITS;
 #pragma unroll
-                    for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
-                        const uint32_t part = Cfg::PARTS == 2 ? (kk & 1) : 0;
-                        // the first MMA into each partial accumulator of the tile overwrites it
-                        const uint32_t acc = (kb != 0 || kk >= Cfg::PARTS) ? 1u : 0u;
-                        umma_f16_ss(d_tmem + part * BN, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC, acc);
-                    }
-                    umma_commit(empty_bar(s));
+                for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
+                    const uint32_t part = Cfg::PARTS == 2 ? (kk & 1) : 0;
+                    // the first MMA into each partial accumulator of the tile overwrites it
+                    const uint32_t acc = (kb != 0 || kk >= Cfg::PARTS) ? 1u : 0u;
+                    umma_f16_ss_if(d_tmem + part * BN, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC, acc, leader);
                 }
-                __syncwarp();
+                umma_commit_if(empty_bar(s), leader);
                 if (++s == static_cast<uint32_t>(STAGES)) { s = 0; ph ^= 1u; }
             }
             if (!ok) break;
-            if (lane == 0) umma_commit(accf_bar(b));
-            __syncwarp();
-        }
-        // All MMAs issued by this warp complete before TMEM is released.
-        if (lane == 0) {
-            umma_commit(done_bar);
-            if (!mbar_wait(done_bar, 0)) fail();
+            umma_commit_if(accf_bar(b), leader);
         }
         __syncwarp();
+        // All MMAs issued by this warp complete before TMEM is released.
+        umma_commit_if(done_bar, leader);
+        if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
     } else {
         // ------------------------------- Epilogue -----------------------------------
         const int q = warp & 3;   // TMEM lane quarter this warp may access

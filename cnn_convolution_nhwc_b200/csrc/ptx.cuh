@@ -198,6 +198,40 @@ __device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+// The same MMA issued by a whole converged warp: only the lane whose `leader` is non-zero
+// issues it. An MMA-issuing loop that the whole warp runs, with the MMAs predicated instead of
+// placed under a one-lane branch, keeps the warp converged; measured on B200 that issues a
+// group of four M=128, N=128 MMAs about twice as fast as the one-lane branch does.
+__device__ __forceinline__ void umma_f16_ss_if(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate, uint32_t leader) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :
+        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+        : "memory");
+}
+
+// umma_commit by the lane whose `leader` is non-zero, in a converged warp.
+__device__ __forceinline__ void umma_commit_if(uint32_t bar, uint32_t leader) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+        "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar),
+        "r"(leader)
+        : "memory");
+}
+
+// 1 in exactly one lane of the converged warp, 0 in the others.
+__device__ __forceinline__ uint32_t elect_one_sync() {
+    uint32_t p = 0;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, %1;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+                 : "=r"(p)
+                 : "r"(0xffffffffu));
+    return p;
+}
+
 // Arrives once on the mbarrier when every tcgen05 operation this thread issued before has
 // completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
