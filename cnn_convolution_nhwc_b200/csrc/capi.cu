@@ -143,6 +143,36 @@ int ensure_smem_attr(DeviceState *d, unsigned bit, Kern kern, int bytes) {
     return CONV_OK;
 }
 
+// Clusters of S CTAs (`threads` threads, `smem` dynamic bytes) of kernel `kern` that the device
+// holds at once, asked once per (kernel bit, S, shared memory) and cached: a persistent grid of
+// clusters larger than that would run its last clusters after the others. 0 on failure.
+template <typename Kern>
+int cluster_fit(DeviceState *d, unsigned bit, Kern kern, int S, int smem, int threads) {
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        for (int i = 0; i < d->n_cluster_fit; ++i) {
+            const DeviceState::ClusterFit &f = d->cluster_fit[i];
+            if (f.bit == bit && f.S == S && f.smem == smem) return f.active;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(S));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess) active = 0;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (d->n_cluster_fit < 64) d->cluster_fit[d->n_cluster_fit++] = DeviceState::ClusterFit{bit, S, smem, active};
+    return active;
+}
+
 // Every tensor of a call must be device memory of the current device (or managed memory): the
 // kernels launch on the current device, and a buffer of another GPU, or host memory, would be
 // read through the wrong mapping. Null pointers (absent biases) are skipped. While `stream` is
@@ -569,6 +599,7 @@ int dispatch_fold(const void *X, const void *F, void *Y, int Cin, int Cout, int 
 // ---- streamed-filter kernel (256-row tiles, two accumulators per filter slot) -------------
 struct StreamPlan {
     bool ok = false;
+    bool pair = false;   // 2-CTA clusters sharing each filter slot (cta_group::2 MMAs)
     int bn = 0;
     DenseStreamParams p{};
     int smem = 0;
@@ -589,7 +620,11 @@ StreamPlan plan_stream(int N, int H, int W, int Cin, int Cout, int K, int num_sm
     const int halo_rows = n_boxes * box_rows;
     const int halo_bytes = halo_rows * 64;
     const int bn = Cout <= 64 ? 64 : 128;
-    const int b_bytes = 32 * bn * 2;
+    // BN = 128 runs as CTA pairs: each CTA stages half of every filter slot and the even CTA's
+    // M = 256 MMAs read both halves, halving the filter traffic per tensor-core cycle
+    // (CONV_B200_STREAM_PAIR=0 keeps one CTA per tile)
+    const bool pair = bn == 128 && num_sms >= 2 && env_int("CONV_B200_STREAM_PAIR", 1, 0, 1) == 1;
+    const int b_bytes = 32 * (pair ? 64 : bn) * 2;
     const int fixed = bn == 64 ? DenseStreamCfg<64>::FIXED_BYTES : DenseStreamCfg<128>::FIXED_BYTES;
     int hs = 3;
     long long avail = kSmemLimit - fixed - 3LL * halo_bytes;
@@ -609,22 +644,28 @@ StreamPlan plan_stream(int N, int H, int W, int Cin, int Cout, int K, int num_sm
     p.box_rows = box_rows;
     p.n_boxes = n_boxes;
     p.halo_bytes = halo_bytes;
-    p.num_mtiles = static_cast<int>((rows + 255) / 256);
+    p.num_mtiles = static_cast<int>((rows + (pair ? 511 : 255)) / (pair ? 512 : 256));
     p.num_ntiles = (Cout + bn - 1) / bn;
     if (1LL * p.num_mtiles * p.num_ntiles > kInt32Max) return pl;
     p.num_tiles = p.num_mtiles * p.num_ntiles;
     p.HS = hs;
     p.BS = static_cast<int>(bs);
     pl.bn = bn;
+    pl.pair = pair;
     pl.smem = fixed + p.BS * b_bytes + p.HS * halo_bytes;
     // more than half of the shared memory keeps a second CTA (and its TMEM allocation) off the SM
     if (pl.smem < 116 * 1024) pl.smem = 116 * 1024;
-    pl.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    if (pair) {
+        const int pairs = num_sms / 2;
+        pl.grid = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
+    } else {
+        pl.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    }
     pl.ok = pl.smem <= kSmemLimit;
     return pl;
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 int launch_dense_stream(const void *X, const void *F, void *Y, int Cin, int Cout, int K, const StreamPlan &pl,
                         cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
     using Cfg = DenseStreamCfg<BN>;
@@ -650,13 +691,26 @@ int launch_dense_stream(const void *X, const void *F, void *Y, int Cin, int Cout
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CONV_ERR_CUDA;
     }
-    auto kern = dense_stream_kernel<Cfg>;
+    auto kern = dense_stream_kernel<Cfg, PAIR>;
     if (int rc = ensure_smem_attr(d, attr_bit, kern, kSmemLimit)) return rc;
     cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(Cfg::THREADS);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
+    if (PAIR) {
+        // no more pairs than the device holds at once (the grid is persistent)
+        const int fit = cluster_fit(d, attr_bit, kern, 2, pl.smem, Cfg::THREADS);
+        if (fit < 1) return CONV_ERR_CUDA;
+        if (static_cast<int>(cfg.gridDim.x) > 2 * fit) cfg.gridDim = dim3(static_cast<unsigned>(2 * fit));
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
     return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
                     "dense_stream_kernel");
 }
@@ -1227,10 +1281,13 @@ int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int 
         if (pl.ok && (pl.bres || force_halo) && !force_stream) return dispatch_halo(X, F, Y, Cin, Cout, K, pl, stream, d);
         if (force_halo) return CONV_ERR_UNSUPPORTED;
         if (!force_bn) {
-            // shared-memory attribute bits 61..62
+            // shared-memory attribute bits 61..62, and 104 for the pair form
             const StreamPlan sp = plan_stream(N, H, W, Cin, Cout, K, d->num_sms);
-            if (sp.ok) return sp.bn == 64 ? launch_dense_stream<64>(X, F, Y, Cin, Cout, K, sp, stream, d, 61)
-                                          : launch_dense_stream<128>(X, F, Y, Cin, Cout, K, sp, stream, d, 62);
+            if (sp.ok) {
+                if (sp.pair) return launch_dense_stream<128, true>(X, F, Y, Cin, Cout, K, sp, stream, d, 104);
+                return sp.bn == 64 ? launch_dense_stream<64, false>(X, F, Y, Cin, Cout, K, sp, stream, d, 61)
+                                   : launch_dense_stream<128, false>(X, F, Y, Cin, Cout, K, sp, stream, d, 62);
+            }
             if (force_stream) return CONV_ERR_UNSUPPORTED;
         }
         if (pl.ok && !im2col_ok) return dispatch_halo(X, F, Y, Cin, Cout, K, pl, stream, d);
@@ -1290,7 +1347,9 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
     }
     auto kern = dwpw_gemm_kernel<MODE, KC, HW>;
     if (int rc = ensure_smem_attr(d, bit, kern, kSmemLimit)) return rc;
-    const int clusters_max = d->num_sms / p.S;
+    int clusters_max = d->num_sms / p.S;
+    if (p.S > 1) clusters_max = cluster_fit(d, bit, kern, p.S, smem, G::THREADS);
+    if (clusters_max < 1) return CONV_ERR_CUDA;
     const int clusters = N < clusters_max ? N : clusters_max;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];

@@ -61,12 +61,13 @@ struct DenseStreamCfg {
     static constexpr int NUM_EPI = 8;                  // epilogue warps: two per TMEM lane quarter
     static constexpr int EPI_BYTES = NUM_EPI * 32 * 128;   // per-warp 32 rows x 64 channels staging
     static constexpr int MAX_HS = 4;
-    static constexpr int MAX_BS = 16;
+    static constexpr int MAX_BS = 24;
     static constexpr int NUM_BARS = 2 * MAX_HS + 2 * MAX_BS + 4 /*acc pairs*/ + 2;
     static constexpr int TMEM_COLS = 4 * BN;           // two accumulator pairs
     static constexpr int THREADS = 32 * (3 + NUM_EPI);   // TMA x2, MMA, epilogue
     static constexpr int HALO_WARP = 2 + NUM_EPI;
     static constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, /*B MN-major*/ true);
+    static constexpr uint32_t IDESC_PAIR = idesc_bf16_f32(256, BN, /*B MN-major*/ true);   // cta_group::2
     // shared-memory bytes besides the filter ring and the halo ring
     static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + NUM_BARS * 8 + NUM_EPI * 32 * 8 + 16;
     static_assert(BN == 64 || BN == 128, "two accumulator pairs of BN columns must fit in TMEM");
@@ -84,19 +85,22 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr) {
     return d;
 }
 
-template <class Cfg>
+template <class Cfg, bool PAIR>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
                     __nv_bfloat16 *__restrict__ Y, const DenseStreamParams p, unsigned int *status) {
     constexpr int BN = Cfg::BN;
+    static_assert(!PAIR || BN == 128, "a pair splits the filter slot into two 64-channel boxes");
+    constexpr int B_CTA = PAIR ? Cfg::B_BYTES / 2 : Cfg::B_BYTES;   // filter bytes per slot in this CTA
+    constexpr int TILE_ROWS = PAIR ? 2 * Cfg::BM : Cfg::BM;          // GEMM rows per (pair) tile
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;   // 1024-B alignment for the swizzles
     uint8_t *smem = smem_raw + (base - raw_base);
 
     const uint32_t sB = base;                                       // filter ring
-    const uint32_t sH = base + p.BS * Cfg::B_BYTES;                 // halo ring
-    const uint32_t epi_off = p.BS * Cfg::B_BYTES + p.HS * p.halo_bytes;
+    const uint32_t sH = base + p.BS * B_CTA;                        // halo ring
+    const uint32_t epi_off = p.BS * B_CTA + p.HS * p.halo_bytes;
     const uint32_t sEpi = base + epi_off;
     const uint32_t bars = sEpi + Cfg::EPI_BYTES;
     constexpr int RH = Cfg::MAX_HS, RB = Cfg::MAX_BS;
@@ -113,6 +117,10 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // In a pair the even CTA (rank 0) issues the MMAs for both; its full and accumulator-empty
+    // barriers count both CTAs' copies and epilogues. lead(a): barrier a of the even CTA.
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;
+    auto lead = [&](uint32_t a) { return PAIR ? map_rank(a, 0u) : a; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < RH; ++s) {
@@ -125,7 +133,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf(b), 1);
-            mbar_init(acce(b), Cfg::NUM_EPI);   // one arrival per epilogue warp
+            mbar_init(acce(b), (PAIR ? 2 : 1) * Cfg::NUM_EPI);   // one arrival per epilogue warp
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -134,20 +142,28 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         prefetch_tensormap(&tmF);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_holder), Cfg::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // both CTAs' barriers and TMEM exist before either is used
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
     auto fail = [&]() {
         atomicOr(status, kStatusTimeout);
         *abort_flag = 1;
+        if constexpr (PAIR) st_cluster_u32(map_rank(smem_u32(const_cast<int *>(abort_flag)), rank ^ 1u), 1u);
     };
-    const int first = static_cast<int>(blockIdx.x);
-    const int step = static_cast<int>(gridDim.x);
+    const int first = static_cast<int>(PAIR ? blockIdx.x >> 1 : blockIdx.x);
+    const int step = static_cast<int>(PAIR ? gridDim.x >> 1 : gridDim.x);
+    const int row0 = static_cast<int>(rank) * Cfg::BM;   // this CTA's rows inside the (pair) tile
 
     // The role loops keep their ring slots and phases as running counters and advance the MMA
     // descriptors by adding to their address fields: the MMA warp is one serial instruction
@@ -161,23 +177,31 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         uint32_t hit = 0, hs = 0, hph = 0;
         bool ok = true;
         for (int t = first; t < p.num_tiles && ok && !*abort_flag; t += step) {
-            const int P0 = (t / p.num_ntiles) * Cfg::BM;
+            const int P0 = (t / p.num_ntiles) * TILE_ROWS + row0;
             for (int cb = 0; cb < p.num_cblk; ++cb, ++hit) {
                 if (!mbar_wait_warp(hempty(hs), hph ^ 1u)) { ok = false; break; }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(hfull(hs), p.halo_bytes);
-                    for (int bx = 0; bx < p.n_boxes; ++bx)
-                        tma_load_2d(sH + hs * p.halo_bytes + bx * p.box_rows * 64, &tmX, hfull(hs), cb * Cfg::CB,
-                                    P0 + bx * p.box_rows);
+                    if (rank == 0) mbar_arrive_expect_tx(hfull(hs), (PAIR ? 2 : 1) * p.halo_bytes);
+                    for (int bx = 0; bx < p.n_boxes; ++bx) {
+                        const uint32_t dst = sH + hs * p.halo_bytes + bx * p.box_rows * 64;
+                        if constexpr (PAIR)
+                            tma_load_2d_pair(dst, &tmX, lead(hfull(hs)), cb * Cfg::CB, P0 + bx * p.box_rows);
+                        else
+                            tma_load_2d(dst, &tmX, hfull(hs), cb * Cfg::CB, P0 + bx * p.box_rows);
+                    }
                 }
                 __syncwarp();
                 if (++hs == static_cast<uint32_t>(p.HS)) { hs = 0; hph ^= 1u; }
             }
         }
         if (!ok && lane == 0) fail();
-        // Drain: every load issued has landed before the CTA may exit.
-        for (uint32_t j = hit > (uint32_t)p.HS ? hit - p.HS : 0u; j < hit; ++j)
-            if (!mbar_wait_warp(hfull(j % p.HS), (j / p.HS) & 1u)) { if (lane == 0) fail(); break; }
+        // Drain: every load issued has landed before the CTA may exit (in a pair: has been
+        // consumed by the pair's MMAs, which the even CTA's commits report to both CTAs).
+        for (uint32_t j = hit > (uint32_t)p.HS ? hit - p.HS : 0u; j < hit; ++j) {
+            const bool landed = PAIR ? mbar_wait_warp(hempty(j % p.HS), (j / p.HS) & 1u)
+                                     : mbar_wait_warp(hfull(j % p.HS), (j / p.HS) & 1u);
+            if (!landed) { if (lane == 0) fail(); break; }
+        }
     } else if (warp == 0) {
         // ------------------------------- filter producer ----------------------------
         uint32_t bit = 0, bs = 0, bph = 0;
@@ -188,11 +212,17 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 for (int tap = 0; tap < p.KK; ++tap, ++bit) {
                     if (!mbar_wait_warp(bempty(bs), bph ^ 1u)) { ok = false; break; }
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(bfull(bs), Cfg::B_BYTES);
+                        if (rank == 0) mbar_arrive_expect_tx(bfull(bs), Cfg::B_BYTES);   // both halves
+                        if constexpr (PAIR) {
+                            // this CTA's half of the slot: output channels n0 + 64*rank .. + 63
+                            tma_load_3d_pair(sB + bs * B_CTA, &tmF, lead(bfull(bs)), n0 + 64 * static_cast<int>(rank),
+                                             cb * Cfg::CB, tap);
+                        } else {
 #pragma unroll
-                        for (int h = 0; h < BN / 64; ++h)
-                            tma_load_3d(sB + bs * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, &tmF, bfull(bs), n0 + h * 64,
-                                        cb * Cfg::CB, tap);
+                            for (int h = 0; h < BN / 64; ++h)
+                                tma_load_3d(sB + bs * B_CTA + h * Cfg::B_BOX_BYTES, &tmF, bfull(bs), n0 + h * 64,
+                                            cb * Cfg::CB, tap);
+                        }
                     }
                     __syncwarp();
                     if (++bs == static_cast<uint32_t>(p.BS)) { bs = 0; bph ^= 1u; }
@@ -200,62 +230,78 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             }
         }
         if (!ok && lane == 0) fail();
-        for (uint32_t j = bit > (uint32_t)p.BS ? bit - p.BS : 0u; j < bit; ++j)
-            if (!mbar_wait_warp(bfull(j % p.BS), (j / p.BS) & 1u)) { if (lane == 0) fail(); break; }
+        for (uint32_t j = bit > (uint32_t)p.BS ? bit - p.BS : 0u; j < bit; ++j) {
+            const bool landed = PAIR ? mbar_wait_warp(bempty(j % p.BS), (j / p.BS) & 1u)
+                                     : mbar_wait_warp(bfull(j % p.BS), (j / p.BS) & 1u);
+            if (!landed) { if (lane == 0) fail(); break; }
+        }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
         // The whole warp runs the loop, converged; the MMAs and commits are predicated on one
         // elected lane (every commit of this warp comes from that lane, so that each commit
-        // tracks all of the warp's MMAs).
+        // tracks all of the warp's MMAs). In a pair only the even CTA's warp issues: M = 256
+        // MMAs (128 rows from each CTA) whose commits arrive on the barriers of both CTAs.
         const uint32_t leader = elect_one_sync();
-        uint32_t local = 0, hs = 0, hph = 0, bs = 0, bph = 0;
-        bool ok = true;
-        // descriptors differ only in the start-address field (16-byte units): A +4 per 64-byte
-        // halo row, +2 per K=16 step, +512 for the second accumulator's rows (128 rows further
-        // on); B +B_BYTES/16 per filter slot, +128 per K=16 step (16 reduction rows = 2048 B)
-        const uint64_t b_desc0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
-        constexpr uint32_t kSlotUnits = Cfg::B_BYTES >> 4;
-        const uint32_t row_skip4 = static_cast<uint32_t>(p.W - p.K) * 4u;
-        for (int t = first; t < p.num_tiles && ok && !__any_sync(0xffffffffu, *abort_flag != 0);
-             t += step, ++local) {
-            const uint32_t b = local & 1u;
-            // waiting here means the epilogue is the slower role: sleep between polls
-            if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t d0 = tmem_base + b * (2 * BN);   // rows 0..127 of the tile
-            const uint32_t d1 = d0 + BN;                    // rows 128..255
-            for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
-                if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
+        constexpr uint16_t kBoth = 0x3;
+        auto commit = [&](uint32_t bar) {
+            if constexpr (PAIR) umma_commit_pair_if(bar, kBoth, leader);
+            else umma_commit_if(bar, leader);
+        };
+        auto mma = [&](uint32_t d, uint64_t a, uint64_t bdesc, uint32_t acc) {
+            if constexpr (PAIR) umma_f16_ss_pair_if(d, a, bdesc, Cfg::IDESC_PAIR, acc, leader);
+            else umma_f16_ss_if(d, a, bdesc, Cfg::IDESC, acc, leader);
+        };
+        if (rank == 0) {
+            uint32_t local = 0, hs = 0, hph = 0, bs = 0, bph = 0;
+            bool ok = true;
+            // descriptors differ only in the start-address field (16-byte units): A +4 per 64-byte
+            // halo row, +2 per K=16 step, +512 for the second accumulator's rows (128 rows further
+            // on); B +B_CTA/16 per filter slot, +128 per K=16 step (16 reduction rows = 2048 B)
+            const uint64_t b_desc0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
+            constexpr uint32_t kSlotUnits = B_CTA >> 4;
+            const uint32_t row_skip4 = static_cast<uint32_t>(p.W - p.K) * 4u;
+            for (int t = first; t < p.num_tiles && ok && !__any_sync(0xffffffffu, *abort_flag != 0);
+                 t += step, ++local) {
+                const uint32_t b = local & 1u;
+                // waiting here means the epilogue is the slower role: sleep between polls
+                if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
                 tc_fence_after();
-                const uint64_t a_desc0 = smem_desc_sw64(sH + hs * p.halo_bytes);
-                uint32_t row4 = 0;   // (ky*W + kx) * 4: tap (ky, kx) reads the halo from row ky*W + kx on
-                for (int ky = 0; ky < p.K && ok; ++ky, row4 += row_skip4) {
-                    for (int kx = 0; kx < p.K; ++kx, row4 += 4u) {
-                        if (!mbar_wait_warp(bfull(bs), bph)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint64_t ad = a_desc0 + row4;
-                        const uint64_t bd = b_desc0 + bs * kSlotUnits;
-                        const uint32_t acc = (cb | ky | kx) != 0 ? 1u : 0u;
-                        umma_f16_ss_if(d0, ad, bd, Cfg::IDESC, acc, leader);
-                        umma_f16_ss_if(d1, ad + 512, bd, Cfg::IDESC, acc, leader);
-                        umma_f16_ss_if(d0, ad + 2, bd + 128, Cfg::IDESC, 1u, leader);
-                        umma_f16_ss_if(d1, ad + 514, bd + 128, Cfg::IDESC, 1u, leader);
-                        umma_commit_if(bempty(bs), leader);
-                        if (++bs == static_cast<uint32_t>(p.BS)) { bs = 0; bph ^= 1u; }
+                const uint32_t d0 = tmem_base + b * (2 * BN);   // rows 0..127 of the CTA's tile
+                const uint32_t d1 = d0 + BN;                    // rows 128..255
+                for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
+                    if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t a_desc0 = smem_desc_sw64(sH + hs * p.halo_bytes);
+                    uint32_t row4 = 0;   // (ky*W + kx) * 4: tap (ky, kx) reads the halo from row ky*W + kx on
+                    for (int ky = 0; ky < p.K && ok; ++ky, row4 += row_skip4) {
+                        for (int kx = 0; kx < p.K; ++kx, row4 += 4u) {
+                            if (!mbar_wait_warp(bfull(bs), bph)) { ok = false; break; }
+                            tc_fence_after();
+                            const uint64_t ad = a_desc0 + row4;
+                            const uint64_t bd = b_desc0 + bs * kSlotUnits;
+                            const uint32_t acc = (cb | ky | kx) != 0 ? 1u : 0u;
+                            mma(d0, ad, bd, acc);
+                            mma(d1, ad + 512, bd, acc);
+                            mma(d0, ad + 2, bd + 128, 1u);
+                            mma(d1, ad + 514, bd + 128, 1u);
+                            commit(bempty(bs));
+                            if (++bs == static_cast<uint32_t>(p.BS)) { bs = 0; bph ^= 1u; }
+                        }
                     }
+                    if (!ok) break;
+                    commit(hempty(hs));
+                    if (++hs == static_cast<uint32_t>(p.HS)) { hs = 0; hph ^= 1u; }
                 }
                 if (!ok) break;
-                umma_commit_if(hempty(hs), leader);
-                if (++hs == static_cast<uint32_t>(p.HS)) { hs = 0; hph ^= 1u; }
+                commit(accf(b));
             }
-            if (!ok) break;
-            umma_commit_if(accf(b), leader);
+            __syncwarp();
+            if (!ok && lane == 0) fail();
+            // All MMAs issued by this warp complete before TMEM is released (in a pair: before
+            // the cluster barrier that both CTAs pass ahead of their deallocation).
+            commit(done_bar);
+            if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
         }
-        __syncwarp();
-        if (!ok && lane == 0) fail();
-        // All MMAs issued by this warp complete before TMEM is released.
-        umma_commit_if(done_bar, leader);
-        if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
     } else {
         // ------------------------------- Epilogue (warps 2..9) -----------------------
         const int q = warp & 3;             // TMEM lane quarter this warp may access
@@ -274,7 +320,7 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             for (int half = 0; half < 2; ++half) {
                 // this lane's row: flattened input position P -> output row, or -1 if dropped
                 {
-                    const int P = mt * Cfg::BM + half * 128 + q * 32 + lane;
+                    const int P = mt * TILE_ROWS + row0 + half * 128 + q * 32 + lane;
                     long long off = -1;
                     if (P < p.rows) {
                         const int row = P / p.W;
@@ -329,17 +375,25 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     __syncwarp();
                 }
             }
-            // the accumulator pair may now be overwritten by the MMA warp
+            // the accumulator pair may now be overwritten by the MMA warp (of the even CTA)
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce(b));
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster(lead(acce(b)));
+                else mbar_arrive(acce(b));
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    // neither CTA of a pair leaves while the other may still signal its barriers
+    if constexpr (PAIR) cluster_sync_all();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    if (warp == 1) {
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+        else tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
 }
 
 }  // namespace convb200

@@ -82,28 +82,6 @@ constexpr int kDwPwChunkBytes = 128 * 16 * 4;                     // 128 rows x 
 // taps per channel rounded up to a float4 (the staged weight row)
 __host__ __device__ constexpr int dwpw_kkp(int K) { return (K * K + 3) & ~3; }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// shared::cta address -> the same offset in cluster rank `rank`'s shared memory
-__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
-
 template <int MODE, int KC>
 __global__ void __launch_bounds__(kDwPwThreads, 1)
 dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,

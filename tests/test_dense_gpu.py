@@ -359,6 +359,28 @@ def test_streamed_filter_kernel(cb, shape):
     _check_bf16(y, Xb, Fb)
 
 
+# CTA pairs (BN = 128: each CTA of a 2-CTA cluster stages half of every filter slot, and the even
+# CTA's M = 256 MMAs span both): a pair whose second CTA has no valid rows (ragged end), several
+# N tiles, and more pair tiles than pairs on the device (clusters loop over tiles)
+PAIR_SHAPES = [(3, 21, 19, 64, 128, 5), (2, 30, 26, 192, 320, 5), (16, 50, 50, 32, 128, 3)]
+
+
+@pytest.mark.parametrize("shape", PAIR_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_streamed_filter_pairs_match_single_ctas(cb, shape):
+    # the same MMA sequence per output with or without pairs: identical bits
+    N, H, W, Cin, Cout, K = shape
+    Xb, Fb = _case_inputs(N, H, W, Cin, Cout, K, seed=sum(shape) + 17)
+    os.environ["CONV_B200_STREAM_PAIR"] = "0"
+    try:
+        y_single = _run_bf16(cb, Xb, Fb, env="stream")
+    finally:
+        del os.environ["CONV_B200_STREAM_PAIR"]
+    y_pair = _run_bf16(cb, Xb, Fb, env="stream")
+    assert cb.conv_last_kernel() == "dense_stream_kernel"
+    _check_bf16(y_pair, Xb, Fb)
+    assert np.array_equal(y_pair, y_single)
+
+
 def test_streamed_filter_is_the_default_for_large_filters(cb):
     # 5x5x128x128 bf16 is 800 KiB of filter: it cannot stay in shared memory
     Xb, Fb = _case_inputs(2, 20, 20, 128, 128, 5, seed=31)
