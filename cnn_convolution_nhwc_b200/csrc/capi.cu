@@ -1306,9 +1306,9 @@ int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int 
 // ---- fused depthwise -> pointwise, transposed GEMM (7x7 and 14x14 images) --------------------
 // shared-memory attribute bits 96..103: MODE x K (3, 5) x image (7, 14)
 bool dwpw_gemm_eligible(int C, int H, int W, int K, int stride, int pad, int dil, int Cout, const float *x,
-                        const float *y) {
+                        const float *w, const float *y) {
     return H == W && (H == 7 || H == 14) && (K == 3 || K == 5) && stride == 1 && dil == 1 && pad == (K - 1) / 2 &&
-           C % 4 == 0 && Cout <= 256 && aligned(x, 16) && aligned(y, 16);
+           C % 4 == 0 && Cout <= 256 && aligned(x, 16) && aligned(w, 16) && aligned(y, 16);
 }
 
 template <int MODE, int KC, int HW>
@@ -1330,8 +1330,8 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
     // a 2-CTA cluster per image (every other channel block each) when there are two blocks and
     // its receive area fits; CONV_B200_DWPW_SPLIT=1 keeps one CTA per image (tests)
     const int want = env_int("CONV_B200_DWPW_SPLIT", 2, 1, 2);
-    p.S = (want == 2 && p.nblk >= 2 && dwpw_gemm_smem<HW>(p.fslot, p.MT, 2) <= kSmemLimit) ? 2 : 1;
-    const int smem = dwpw_gemm_smem<HW>(p.fslot, p.MT, p.S);
+    p.S = (want == 2 && p.nblk >= 2 && dwpw_gemm_smem<HW>(p.fslot, p.MT, 2, KC * KC) <= kSmemLimit) ? 2 : 1;
+    const int smem = dwpw_gemm_smem<HW>(p.fslot, p.MT, p.S, KC * KC);
     if (smem > kSmemLimit || p.tmem_cols > 512) return CONV_ERR_UNSUPPORTED;
     alignas(64) CUtensorMap tmF;
     {   // F: 2-D {Cout, C}; a box is 64 output columns x CB channel rows (columns past Cout and
@@ -1342,6 +1342,17 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
         const cuuint32_t estr[2] = {1, 1};
         if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(F), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    alignas(64) CUtensorMap tmX = tmF;   // unused by the 7x7 form (contiguous bulk copies)
+    if (G::PADX) {   // x as [N*C][P] fp32; a box of XP > P columns (the overhang reads zeros) x CB planes
+        const cuuint64_t dims[2] = {(cuuint64_t)G::P, (cuuint64_t)N * C};
+        const cuuint64_t strides[1] = {(cuuint64_t)G::P * 4};
+        const cuuint32_t box[2] = {(cuuint32_t)G::XP, (cuuint32_t)G::CB};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode_tiled(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(x), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CONV_ERR_CUDA;
     }
@@ -1365,7 +1376,7 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_gemm_kernel");
+    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, tmX, y, p, d->status), "dwpw_gemm_kernel");
 }
 
 template <int MODE>
@@ -1840,7 +1851,7 @@ int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F
     const bool force_staged = kforce && std::strcmp(kforce, "staged") == 0;
     const bool force_gemm = kforce && std::strcmp(kforce, "gemm") == 0;
     if (!force_flat && !force_staged && force_split <= 2) {
-        if (dwpw_gemm_eligible(C, H, W, K, stride, pad, dil, Cout, x, y))
+        if (dwpw_gemm_eligible(C, H, W, K, stride, pad, dil, Cout, x, w_dw, y))
             return mode == DW_EXACT ? launch_dwpw_gemm<0>(x, w_dw, b_dw, F, b_pw, y, N, C, H, K, Cout, stream, d)
                                     : launch_dwpw_gemm<1>(x, w_dw, b_dw, F, b_pw, y, N, C, H, K, Cout, stream, d);
     }

@@ -21,14 +21,16 @@
 // Work layout: one image per cluster of S CTAs (S = 2 when there are at least two channel
 // blocks: rank k takes blocks k, k + S, ...), 16 warps per CTA, the channels in blocks of CB.
 // Per block:
-//   * x: the block's CB planes of the image are one contiguous range of x, staged by one 1-D
-//     bulk copy into a 2-slot ring (issued two blocks ahead);
+//   * x: the block's CB planes of the image are one contiguous range of x, staged into a
+//     2-slot ring two blocks ahead: at 14x14 one 1-D bulk copy per plane into a padded pitch
+//     (fewer bank conflicts in the row loads), at 7x7 one copy of the whole range;
 //   * F: the block's CB x Cout filter rows, 64-column boxes by TMA into a 3-slot ring (two
 //     blocks ahead); columns past Cout arrive as zeros;
 //   * every thread computes its strip (zeros padding, exact or fast mode, the depthwise bias),
 //     rounds to bf16 and writes the values into the B tile (128-byte swizzled, 64 pixels per
 //     box); channels past C write zeros;
-//   * after the CTA barrier that publishes the B tile, thread 0 issues the block's MMAs
+//   * after the CTA barrier that publishes the B tile, the issuing warp (at 14x14 the
+//     sixteenth warp, which has no depthwise work; at 7x7 warp 0) issues the block's MMAs
 //     (M = 128 per 128 output channels, N = pixels rounded up to 16, K = 16) into the image's
 //     TMEM accumulators and commits; the B slot is rewritten two blocks later, after that
 //     commit.
@@ -82,31 +84,48 @@ struct DwPwGemmGeom {
     static constexpr int NRUN = (HW + RR - 1) / RR;
     static constexpr int UPP = NSTRIP * NRUN;              // work units per plane
     static constexpr int THREADS = 512;
+    static constexpr int UNITS = CB * UPP;                 // threads with depthwise work
+    // a warp without depthwise work issues the copies and the MMAs; else thread 0 does
+    static constexpr bool SPARE = UNITS <= THREADS - 32;
+    static constexpr int ISSUER_WARP = SPARE ? THREADS / 32 - 1 : 0;
+    // planes whose byte size is a multiple of 16 arrive by one 2-D tensor copy whose box is
+    // wider than a plane (the overhang reads zeros), which lays them out at a padded pitch and
+    // spreads a warp's row loads over more banks (14x14: 196 -> 204 floats); 7x7 planes (196
+    // bytes) arrive as one contiguous range
+    static constexpr bool PADX = (P * 4) % 16 == 0;
+    static constexpr int XP = PADX ? P + 8 : P;            // plane pitch in shared memory, floats
     static constexpr int BOX = CB * 128;                   // one 64-wide box of CB rows, bf16
     static constexpr int NBOXB = (NPAD + 63) / 64;
     static constexpr int BSLOT = NBOXB * BOX;              // B tile: CB rows x NPAD pixels
-    static constexpr int XSLOT = (CB * P * 4 + 127) / 128 * 128;
+    static constexpr int XSLOT = (CB * XP * 4 + 127) / 128 * 128;
     static constexpr int CHUNK = 128 * 16 * 4;             // 128 rows x 16 fp32 columns
     static constexpr int NOWN = (NCH + 1) / 2;             // chunks a rank of a 2-CTA cluster owns, at most
-    static_assert(CB * UPP <= THREADS, "one work unit per thread");
+    static_assert(UNITS <= THREADS, "one work unit per thread");
+    static_assert(!PADX || (XP * 4) % 16 == 0, "a tensor-copy box row is a multiple of 16 bytes");
     static_assert(CB % 16 == 0, "K = 16 steps");
 };
 
 constexpr int kDwPwGemmFSlots = 3;
 constexpr int kDwPwGemmBars = 2 /*xfull*/ + 3 /*ffull*/ + 2 /*mma_done*/ + 1 /*accf*/ + 1 /*drain*/;
 
-// shared memory: filter ring, B ring, x ring, the receive area of the cluster reduction (MT x
-// NOWN chunks), barriers
+// bytes of one block's depthwise taps (CB channels x KK), staged beside its planes
+template <int HW>
+__host__ __device__ constexpr int dwpw_gemm_wslot(int KK) {
+    return (DwPwGemmGeom<HW>::CB * KK * 4 + 127) / 128 * 128;
+}
+
+// shared memory: filter ring, B ring, x ring, taps ring, the receive area of the cluster
+// reduction (MT x NOWN chunks), barriers
 template <int HW>
 __host__ __device__ constexpr int dwpw_gemm_recv(int MT, int S) {
     return S > 1 ? MT * DwPwGemmGeom<HW>::NOWN * DwPwGemmGeom<HW>::CHUNK : 0;
 }
 
 template <int HW>
-__host__ __device__ constexpr int dwpw_gemm_smem(int fslot, int MT, int S) {
+__host__ __device__ constexpr int dwpw_gemm_smem(int fslot, int MT, int S, int KK) {
     using G = DwPwGemmGeom<HW>;
-    return 1024 + kDwPwGemmFSlots * fslot + 2 * G::BSLOT + 2 * G::XSLOT + dwpw_gemm_recv<HW>(MT, S) +
-           kDwPwGemmBars * 8 + 16;
+    return 1024 + kDwPwGemmFSlots * fslot + 2 * G::BSLOT + 2 * G::XSLOT + 2 * dwpw_gemm_wslot<HW>(KK) +
+           dwpw_gemm_recv<HW>(MT, S) + kDwPwGemmBars * 8 + 16;
 }
 
 // One bf16 value into the B tile: row k (channel in the block), column n (pixel); 64 pixels per
@@ -117,10 +136,20 @@ __device__ __forceinline__ void dwpw_store_b(uint8_t *sB, int box_bytes, int k, 
     *reinterpret_cast<__nv_bfloat16 *>(sB + box * box_bytes + k * 128 + chunk * 16 + (col & 7) * 2) = v;
 }
 
+// Two bf16 values for pixels n (even) and n + 1 of row k: one 4-byte store (an even column and
+// its neighbour share a 16-byte chunk of one box).
+__device__ __forceinline__ void dwpw_store_b2(uint8_t *sB, int box_bytes, int k, int n, float v0, float v1) {
+    const int box = n >> 6, col = n & 63;
+    const int chunk = (col >> 3) ^ (k & 7);
+    *reinterpret_cast<__nv_bfloat162 *>(sB + box * box_bytes + k * 128 + chunk * 16 + (col & 7) * 2) =
+        __floats2bfloat162_rn(v0, v1);
+}
+
 template <int MODE, int KC, int HW>
 __global__ void __launch_bounds__(512, 1)
 dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
-                 float *__restrict__ y, const DwPwGemmParams p, unsigned int *status) {
+                 const __grid_constant__ CUtensorMap tmX, float *__restrict__ y, const DwPwGemmParams p,
+                 unsigned int *status) {
     using G = DwPwGemmGeom<HW>;
     constexpr int PAD = (KC - 1) / 2;
     constexpr int WIN = KC + 1;   // input columns of a two-column strip
@@ -131,7 +160,10 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     const uint32_t sF = base;
     const uint32_t sB = sF + kDwPwGemmFSlots * p.fslot;
     const uint32_t sX = sB + 2 * G::BSLOT;
-    const uint32_t sR = sX + 2 * G::XSLOT;   // receive area of the reduction
+    constexpr int KK = KC * KC;
+    constexpr int WSLOT = dwpw_gemm_wslot<HW>(KK);
+    const uint32_t sW = sX + 2 * G::XSLOT;   // the blocks' taps, a 2-slot ring beside x
+    const uint32_t sR = sW + 2 * WSLOT;      // receive area of the reduction
     const uint32_t bars = sR + dwpw_gemm_recv<HW>(p.MT, p.S);
     auto xfull = [&](int s) { return bars + 8u * s; };
     auto ffull = [&](int s) { return bars + 16u + 8u * s; };
@@ -171,25 +203,45 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
         n = cluster + (g / nb) * nclusters;
         c0 = (rank + (g % nb) * S) * G::CB;
     };
-    int x_issued = 0, f_issued = 0;   // thread 0: blocks whose copies are in flight or landed
-    auto issue_x = [&](int g) {       // thread 0
+    // issuing warp: blocks whose copies are in flight or landed
+    int x_issued = 0, f_issued = 0;
+    const bool issuer = warp == G::ISSUER_WARP;
+    const uint32_t leader = issuer ? elect_one_sync() : 0u;
+    auto issue_x = [&](int g) {       // the whole issuing warp
         int n, c0;
         block_at(g, n, c0);
         x_issued = g + 1;
         const int planes = min(G::CB, p.C - c0);
-        const uint32_t bytes = static_cast<uint32_t>(planes * G::P * 4);
-        mbar_arrive_expect_tx(xfull(g & 1), bytes);
-        bulk_g2s(sX + (g & 1) * G::XSLOT, x + (static_cast<long long>(n) * p.C + c0) * G::P, bytes, xfull(g & 1));
+        const float *src = x + (static_cast<long long>(n) * p.C + c0) * G::P;
+        // the planes' taps: planes * KK floats from w[c0], a multiple of 16 bytes (C % 4 == 0)
+        const uint32_t wbytes = static_cast<uint32_t>(planes * KK * 4);
+        if constexpr (G::PADX) {
+            // x viewed as [N*C][P]: a box of XP columns x CB rows (always the full box's bytes;
+            // rows past the image's channels are other planes or zeros, never used)
+            if (lane == 0) {
+                mbar_arrive_expect_tx(xfull(g & 1), static_cast<uint32_t>(G::CB * G::XP * 4) + wbytes);
+                tma_load_2d(sX + (g & 1) * G::XSLOT, &tmX, xfull(g & 1), 0, n * p.C + c0);
+                bulk_g2s(sW + (g & 1) * WSLOT, w + static_cast<long long>(c0) * KK, wbytes, xfull(g & 1));
+            }
+        } else if (lane == 0) {
+            const uint32_t bytes = static_cast<uint32_t>(planes * G::P * 4);
+            mbar_arrive_expect_tx(xfull(g & 1), bytes + wbytes);
+            bulk_g2s(sX + (g & 1) * G::XSLOT, src, bytes, xfull(g & 1));
+            bulk_g2s(sW + (g & 1) * WSLOT, w + static_cast<long long>(c0) * KK, wbytes, xfull(g & 1));
+        }
+        __syncwarp();
     };
-    auto issue_f = [&](int g) {       // thread 0
+    auto issue_f = [&](int g) {       // the whole issuing warp (lane 0 issues)
         int n, c0;
         block_at(g, n, c0);
         f_issued = g + 1;
-        const uint32_t slot = sF + (g % 3) * p.fslot;
-        mbar_arrive_expect_tx(ffull(g % 3), static_cast<uint32_t>(p.fslot));
-        for (int b = 0; b < 2 * p.MT; ++b) tma_load_2d(slot + b * G::BOX, &tmF, ffull(g % 3), b * 64, c0);
+        if (lane == 0) {
+            const uint32_t slot = sF + (g % 3) * p.fslot;
+            mbar_arrive_expect_tx(ffull(g % 3), static_cast<uint32_t>(p.fslot));
+            for (int b = 0; b < 2 * p.MT; ++b) tma_load_2d(slot + b * G::BOX, &tmF, ffull(g % 3), b * 64, c0);
+        }
     };
-    if (tid == 0) {
+    if (issuer) {
         for (int g = 0; g < 2 && g < total; ++g) {
             issue_x(g);
             issue_f(g);
@@ -198,7 +250,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
 
     // this thread's work unit inside a block: plane (channel) cl, strip of columns 2s, 2s+1,
     // run of output rows r*RR .. r*RR + RR - 1
-    const bool unit_ok = tid < G::CB * G::UPP;
+    const bool unit_ok = tid < G::UNITS;
     const int cl = tid / G::UPP;
     const int rem = tid - cl * G::UPP;
     const int s = rem % G::NSTRIP;
@@ -212,15 +264,16 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     const bool second = ox0 + 1 < HW;   // the strip's second column exists
 
     // depthwise outputs of block g (channel c0 + cl of the image) into the B slot, bf16
-    auto depthwise_block = [&](int g, int c0) {
+    // (its taps arrive with its planes; its bias bv was loaded before the waits)
+    auto depthwise_block = [&](int g, int c0, float bv) {
         uint8_t *bslot = smem + (sB - base) + (g & 1) * G::BSLOT;
         const int c = c0 + cl;
         if (c < p.C) {
-            const float *xs = reinterpret_cast<const float *>(smem + (sX - base) + (g & 1) * G::XSLOT) + cl * G::P;
-            float wr[KC * KC];
+            const float *xs = reinterpret_cast<const float *>(smem + (sX - base) + (g & 1) * G::XSLOT) + cl * G::XP;
+            const float *ws = reinterpret_cast<const float *>(smem + (sW - base) + (g & 1) * WSLOT) + cl * KK;
+            float wr[KK];
 #pragma unroll
-            for (int t = 0; t < KC * KC; ++t) wr[t] = __ldg(w + static_cast<long long>(c) * (KC * KC) + t);
-            const float bv = p.b_dw ? __ldg(p.b_dw + c) : 0.0f;
+            for (int t = 0; t < KK; ++t) wr[t] = ws[t];
             uint64_t w2[KC * KC];
 #pragma unroll
             for (int t = 0; t < KC * KC; ++t) w2[t] = dw_pack(wr[t], wr[t]);
@@ -267,8 +320,12 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
                         a1 = dw_finish<MODE, false>(a1, 0.0f);
                     }
                     const int pix = oy * HW + ox0;
-                    dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
-                    if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
+                    if constexpr (HW % 2 == 0) {
+                        dwpw_store_b2(bslot, G::BOX, cl, pix, a0, a1);   // pix even, both columns exist
+                    } else {
+                        dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
+                        if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
+                    }
                 }
             }
         } else {
@@ -277,8 +334,12 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
             for (int i = 0; i < G::RR; ++i) {
                 const int oy = oy_first + i;
                 if (oy < HW) {
-                    dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0, z);
-                    if (second) dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0 + 1, z);
+                    if constexpr (HW % 2 == 0) {
+                        dwpw_store_b2(bslot, G::BOX, cl, oy * HW + ox0, 0.0f, 0.0f);
+                    } else {
+                        dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0, z);
+                        if (second) dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0 + 1, z);
+                    }
                 }
             }
         }
@@ -303,7 +364,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     // Every thread walks every tile and every block; after a wait ran out (dead) it skips the
     // work but still takes each CTA and cluster barrier, so neither this CTA nor its cluster
     // peer ever waits for it forever.
-    bool dead = false, fail = false;   // fail: thread 0's own waits, or'ed in at the next barrier
+    bool dead = false, fail = false;   // fail: the issuing lane's own waits, or'ed in at the next barrier
     int stop = 0;                      // the first block whose wait ran out
     int g = 0;
     for (int tl = 0; tl < my_tiles; ++tl) {
@@ -313,38 +374,44 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
             block_at(g, nn, c0);
             bool good = true;
             if (!dead) {
+                // the channel's bias first, so that its load overlaps the waits
+                float bv = 0.0f;
+                const int c = c0 + cl;
+                if (unit_ok && c < p.C && p.b_dw) bv = __ldg(p.b_dw + c);
                 // the block's planes staged; the B slot's previous MMAs (block g - 2) done
                 good = mbar_wait_warp(xfull(g & 1), (g >> 1) & 1);
                 if (good && g >= 2) good = mbar_wait_warp(mma_done(g & 1), ((g - 2) >> 1) & 1);
-                if (good && unit_ok) depthwise_block(g, c0);
+                if (good && unit_ok) depthwise_block(g, c0, bv);
                 fence_proxy_async_smem();   // the B tile's generic writes, visible to the tensor cores
             }
             if (__syncthreads_or(!good || fail) && !dead) {
                 dead = true;
                 stop = g;
             }
-            if (!dead && tid == 0) {
-                if (!mbar_wait(ffull(g % 3), (g / 3) & 1)) {
+            if (!dead && issuer) {
+                // the whole issuing warp, converged; the MMAs and commits are predicated on the
+                // elected lane (so are the drain's, so that its commit tracks them all)
+                if (!mbar_wait_warp(ffull(g % 3), (g / 3) & 1)) {
                     fail = true;
                 } else {
                     tc_fence_after();
                     const uint32_t fs = sF + (g % 3) * p.fslot;
                     const uint32_t bs = sB + (g & 1) * G::BSLOT;
+                    // descriptors: +128 (2048 B, 16 rows) per K=16 step; A +2*BOX/16 per M tile
+                    const uint64_t bd0 = smem_desc_sw128(bs, G::BOX, 1024);
+                    const uint64_t ad0 = smem_desc_sw128(fs, G::BOX, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < G::CB / 16; ++kk) {
-                        const uint64_t bd = smem_desc_sw128(bs + kk * 2048, G::BOX, 1024);
-                        for (int mt = 0; mt < p.MT; ++mt) {
-                            const uint64_t ad = smem_desc_sw128(fs + mt * 2 * G::BOX + kk * 2048, G::BOX, 1024);
-                            umma_f16_ss(tmem + mt * G::NPAD, ad, bd, p.idesc, (j | kk) != 0 ? 1u : 0u);
-                        }
-                    }
-                    umma_commit(mma_done(g & 1));
-                    if (j == nb - 1) umma_commit(accf);
+                    for (int kk = 0; kk < G::CB / 16; ++kk)
+                        for (int mt = 0; mt < p.MT; ++mt)
+                            umma_f16_ss_if(tmem + mt * G::NPAD, ad0 + kk * 128 + mt * (2 * G::BOX >> 4), bd0 + kk * 128,
+                                           p.idesc, (j | kk) != 0 ? 1u : 0u, leader);
+                    umma_commit_if(mma_done(g & 1), leader);
+                    if (j == nb - 1) umma_commit_if(accf, leader);
                     // refill: x two blocks ahead into the slot this block has read; F two blocks
                     // ahead into the slot block g - 1 used, once its MMAs are done
                     if (g + 2 < total) {
                         issue_x(g + 2);
-                        if (g >= 1 && !mbar_wait(mma_done((g - 1) & 1), ((g - 1) >> 1) & 1)) fail = true;
+                        if (g >= 1 && !mbar_wait_warp(mma_done((g - 1) & 1), ((g - 1) >> 1) & 1)) fail = true;
                         else issue_f(g + 2);
                     }
                 }
@@ -403,20 +470,22 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
                 }
             }
         }
-        if (S > 1) cluster_sync_all();   // the receive area is read before the next image's partials
+        // the receive area is read before the next image's partials land in it (after the last
+        // image no partials follow)
+        if (S > 1 && tl + 1 < my_tiles) cluster_sync_all();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
 
-    if (dead && tid == 0) {
-        atomicOr(status, kStatusTimeout);
+    if (dead && issuer) {
+        if (lane == 0) atomicOr(status, kStatusTimeout);
         // every copy issued lands, and every MMA issued completes, before the CTA exits
         // (bounded waits): the copies of blocks stop .. issued - 1 were not waited for yet
-        for (int jj = stop; jj < x_issued; ++jj) mbar_wait(xfull(jj & 1), (jj >> 1) & 1);
-        for (int jj = stop; jj < f_issued; ++jj) mbar_wait(ffull(jj % 3), (jj / 3) & 1);
-        umma_commit(drain);
-        mbar_wait(drain, 0);
+        for (int jj = stop; jj < x_issued; ++jj) mbar_wait_warp(xfull(jj & 1), (jj >> 1) & 1);
+        for (int jj = stop; jj < f_issued; ++jj) mbar_wait_warp(ffull(jj % 3), (jj / 3) & 1);
+        umma_commit_if(drain, leader);
+        mbar_wait_warp(drain, 0);
     }
     tc_fence_before();
     __syncthreads();
