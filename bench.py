@@ -94,7 +94,8 @@ KERNEL_SOURCES = {
     "depthwise_kernel": ("depthwise.cuh",),
     "dwpw_kernel": ("dwpw.cuh", "dense_tc.cuh", "depthwise.cuh", "ptx.cuh"),
     "dwpw_staged_kernel": ("dwpw.cuh", "dense_tc.cuh", "depthwise.cuh", "ptx.cuh"),
-    "dwpw_gemm_kernel": ("dwpw_gemm.cuh", "depthwise_tma.cuh", "depthwise_plane.cuh", "depthwise.cuh", "ptx.cuh"),
+    "dwpw_gemm_kernel": ("dwpw_gemm.cuh", "depthwise_tma.cuh", "depthwise_plane.cuh", "depthwise.cuh", "dense_halo.cuh",
+                         "ptx.cuh"),
     "depthwise_plane_kernel": ("depthwise_plane.cuh", "depthwise_tma.cuh", "depthwise.cuh", "ptx.cuh"),
 }
 

@@ -14,6 +14,7 @@ importing this package fails if the library cannot be loaded.
 from __future__ import annotations
 
 import ctypes
+import os
 
 from . import build as _build
 
@@ -23,10 +24,14 @@ CONV_ERR_UNSUPPORTED = -2
 CONV_ERR_MISALIGNED = -3
 CONV_ERR_CUDA = -4
 CONV_ERR_DEVICE_TIMEOUT = -5
+CONV_ERR_DEVICE_BOUNDS = -6
 DW_EXACT = 0
 DW_FAST = 1
 
-LIB_PATH = _build.build()
+# CONV_B200_DEBUG_BOUNDS=1 at import loads the bounds-checked build of the same library (every
+# computed global access checked; a failure sets CONV_ERR_DEVICE_BOUNDS and skips the access)
+DEBUG_BOUNDS = os.environ.get("CONV_B200_DEBUG_BOUNDS", "0") == "1"
+LIB_PATH = _build.build(debug_bounds=DEBUG_BOUNDS)
 lib = ctypes.CDLL(LIB_PATH)
 
 _P = ctypes.c_void_p
@@ -59,12 +64,19 @@ lib.conv_last_kernel.argtypes = []
 lib.conv_last_kernel.restype = ctypes.c_char_p
 lib.conv_selftest_wait_timeout.argtypes = [_P]
 lib.conv_selftest_wait_timeout.restype = _I
+lib.conv_debug_bounds_build.argtypes = []
+lib.conv_debug_bounds_build.restype = _I
+lib.conv_debug_bounds_info.argtypes = [ctypes.POINTER(ctypes.c_longlong), _I]
+lib.conv_debug_bounds_info.restype = _I
+lib.conv_selftest_bounds.argtypes = [_P]
+lib.conv_selftest_bounds.restype = _I
 
 EXPORTS = ("conv2d_nhwc_fwd", "conv2d_nhwc_fwd_f32", "conv2d_nhwc_fwd_ex", "conv2d_nhwc_fwd_grouped",
            "conv2d_nhwc_fwd_grouped_pads",
            "conv2d_nhwc_im2col_workspace", "conv2d_nhwc_fwd_im2col", "conv2d_nhwc_fwd_im2col_noalloc", "dwpw_fwd",
            "depthwise_fwd", "conv_status_string", "conv_device_status", "conv_last_kernel",
-           "conv_selftest_wait_timeout")
+           "conv_selftest_wait_timeout", "conv_debug_bounds_build", "conv_debug_bounds_info",
+           "conv_selftest_bounds")
 CONV_IM2COL_STATIC_BYTES = 32 * 1024 * 1024   # the scratch of conv2d_nhwc_fwd_im2col_noalloc
 
 
@@ -378,6 +390,27 @@ def conv_selftest_wait_timeout(stream=None) -> int:
     """Runs the bounded-wait diagnostic (about one second) on the current device; returns the
     launch status."""
     return lib.conv_selftest_wait_timeout(_stream(stream, _current()))
+
+
+def conv_selftest_bounds(stream=None) -> int:
+    """Runs the bounds-check diagnostic (a failing check that touches no memory) on the current
+    device; returns the launch status."""
+    return lib.conv_selftest_bounds(_stream(stream, _current()))
+
+
+def conv_debug_bounds_build() -> bool:
+    """True when the loaded library is the bounds-checked build."""
+    return lib.conv_debug_bounds_build() == 1
+
+
+def conv_debug_bounds_info(reset=False):
+    """First failed bounds check on the current device since the last reset, as (site, index,
+    limit), or None; always None in the normal build."""
+    info = (ctypes.c_longlong * 3)()
+    rc = lib.conv_debug_bounds_info(info, 1 if reset else 0)
+    if rc != CONV_OK:
+        raise ConvError(rc, "conv_debug_bounds_info")
+    return None if info[0] < 0 else (info[0], info[1], info[2])
 
 
 def conv_device_status(stream=None, reset=False) -> int:

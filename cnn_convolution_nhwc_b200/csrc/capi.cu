@@ -56,6 +56,15 @@ __global__ void selftest_wait_kernel(unsigned int *status) {
     if (threadIdx.x == 0 && !mbar_wait(b, 0)) atomicOr(status, kStatusTimeout);
 }
 
+// One thread that checks an element range lying past its (notional) tensor and touches no
+// memory either way: in the bounds-checked build the check fails and is recorded.
+__global__ void selftest_bounds_kernel(unsigned int *status) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        volatile bool ok = in_bounds(1000, 1, 1000, kSiteSelftest, status);
+        (void)ok;
+    }
+}
+
 namespace {
 
 // family name of the kernel the last successful launch on this host thread used
@@ -272,6 +281,7 @@ int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int C
     p.Cin_g = Cin / g.groups; p.Cout_g = Cout / g.groups;
     p.sh = g.sh; p.sw = g.sw; p.ph = g.ph; p.pw = g.pw; p.dh = g.dh; p.dw = g.dw; p.bias = g.bias;
     p.total = 1LL * N * p.Ho * p.Wo * Cout;
+    p.x_elems = 1LL * N * H * W * Cin;
     long long blocks = (p.total + 255) / 256;
     const long long cap = 1LL * d->num_sms * 16;
     if (blocks > cap) blocks = cap;
@@ -279,7 +289,7 @@ int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int C
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, dense_direct_kernel<T>, X, F, Y, p), "dense_direct_kernel");
+    return launched(cudaLaunchKernelEx(&cfg, dense_direct_kernel<T>, X, F, Y, p, d->status), "dense_direct_kernel");
 }
 
 // The im2col tensor-core kernel over groups g0 .. g0 + NG - 1 per launch (one launch when
@@ -804,28 +814,29 @@ int launch_dw_one(const float *x, const float *w, const float *bias, float *y, c
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p), "depthwise_kernel");
+    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p, d->status), "depthwise_kernel");
 }
 
 // ---- register-window kernel ---------------------------------------------------------------
 template <int MODE, bool HB, int K, int S>
 int launch_dw_reg_one(const float *x, const float *w, const float *bias, float *y, const DwRegParams &rp,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, DeviceState *d) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((rp.num_jobs + 7) / 8));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, depthwise_reg_kernel<MODE, HB, K, S, (K - 1) / 2>, x, w, bias, y, rp),
+    return launched(cudaLaunchKernelEx(&cfg, depthwise_reg_kernel<MODE, HB, K, S, (K - 1) / 2>, x, w, bias, y, rp,
+                                       d->status),
                     "depthwise_reg_kernel");
 }
 
 template <int MODE, bool HB>
 int launch_dw_reg(const float *x, const float *w, const float *bias, float *y, const DwRegParams &rp, int K, int S,
-                  cudaStream_t stream) {
-    if (K == 3 && S == 1) return launch_dw_reg_one<MODE, HB, 3, 1>(x, w, bias, y, rp, stream);
-    if (K == 3 && S == 2) return launch_dw_reg_one<MODE, HB, 3, 2>(x, w, bias, y, rp, stream);
-    if (K == 5 && S == 1) return launch_dw_reg_one<MODE, HB, 5, 1>(x, w, bias, y, rp, stream);
-    return launch_dw_reg_one<MODE, HB, 5, 2>(x, w, bias, y, rp, stream);
+                  cudaStream_t stream, DeviceState *d) {
+    if (K == 3 && S == 1) return launch_dw_reg_one<MODE, HB, 3, 1>(x, w, bias, y, rp, stream, d);
+    if (K == 3 && S == 2) return launch_dw_reg_one<MODE, HB, 3, 2>(x, w, bias, y, rp, stream, d);
+    if (K == 5 && S == 1) return launch_dw_reg_one<MODE, HB, 5, 1>(x, w, bias, y, rp, stream, d);
+    return launch_dw_reg_one<MODE, HB, 5, 2>(x, w, bias, y, rp, stream, d);
 }
 
 // The register kernel serves square 3x3 / 5x5 filters, stride 1 or 2, "same" padding
@@ -1242,6 +1253,16 @@ int launch_dwpw_staged(const float *x, const float *w, const CUtensorMap &tmF, f
     return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, pl.st, d->status), "dwpw_staged_kernel");
 }
 
+// Output-channel tile width of the im2col kernel: 64 for narrow groups; 256 for groups of at
+// least 256 output channels while the tiles still cover every SM (measured on B200: the wider
+// tile halves the A-operand traffic per MMA, e.g. a 3-tap 512 -> 512 Conv1D over 48000
+// positions, 94 -> 74 us); else 128.
+int im2col_bn(long long M, int cout_g, int groups, int num_sms) {
+    if (cout_g <= 64) return 64;
+    if (cout_g >= 256 && ((M + 127) / 128) * ((cout_g + 255) / 256) * groups >= num_sms) return 256;
+    return 128;
+}
+
 // Kernel choice and launch of the plain dense convolution (arguments already validated, the
 // device state taken).
 int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout, int K,
@@ -1297,7 +1318,7 @@ int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int 
         return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
                                    static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, sq, stream, d);
     }
-    int bn = force_bn ? force_bn : (Cout <= 64 ? 64 : 128);
+    int bn = force_bn ? force_bn : im2col_bn(1LL * N * sq.ho(H) * sq.wo(W), Cout, 1, d->num_sms);
     if (bn == 64) return launch_dense_tc<CfgBN64, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 0);
     if (bn == 128) return launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 1);
     return launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 2);
@@ -1455,7 +1476,7 @@ int dense_general(const void *X, const void *F, void *Y, int N, int H, int W, in
         return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),
                                    static_cast<__nv_bfloat16 *>(Y), N, H, W, Cin, Cout, g, stream, d);
     }
-    int bn = Cout_g <= 64 ? 64 : 128;
+    int bn = im2col_bn(1LL * N * g.ho(H) * g.wo(W), Cout_g, g.groups, d->num_sms);
     if (force_bn) bn = std::atoi(force + 2);
     if (g.groups == 1) {
         if (bn == 64) return launch_dense_tc<CfgBN64, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 0);
@@ -1577,7 +1598,7 @@ int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspac
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
     auto *A = static_cast<__nv_bfloat16 *>(workspace);
-    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p),
+    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p, d->status),
                  "im2col_pack_kernel") != CONV_OK)
         return CONV_ERR_CUDA;
     // Y (M x Cout, row-major) = A (M x kd) * F (kd x Cout): in cuBLAS's column-major terms
@@ -1625,7 +1646,7 @@ int conv2d_nhwc_fwd_im2col_noalloc(const void *X, const void *F, void *Y, int N,
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
     auto *A = static_cast<__nv_bfloat16 *>(scratch);
-    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p),
+    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p, d->status),
                  "im2col_pack_kernel") != CONV_OK)
         return CONV_ERR_CUDA;
     // Y = A * F as the 1 x 1 convolution of the patch image [N][Ho][Wo][kd] with F viewed as
@@ -1696,10 +1717,10 @@ int depthwise_fwd(const float *x, const float *w, const float *bias, float *y, i
         const DwRegParams rp = dw_reg_plan(N, Cin, mult, H, W, static_cast<int>(Ho), static_cast<int>(Wo), d->num_sms, x, y);
         const bool hb = bias != nullptr;
         if (mode == DW_EXACT)
-            return hb ? launch_dw_reg<0, true>(x, w, bias, y, rp, KH, stride, stream)
-                      : launch_dw_reg<0, false>(x, w, bias, y, rp, KH, stride, stream);
-        return hb ? launch_dw_reg<1, true>(x, w, bias, y, rp, KH, stride, stream)
-                  : launch_dw_reg<1, false>(x, w, bias, y, rp, KH, stride, stream);
+            return hb ? launch_dw_reg<0, true>(x, w, bias, y, rp, KH, stride, stream, d)
+                      : launch_dw_reg<0, false>(x, w, bias, y, rp, KH, stride, stream, d);
+        return hb ? launch_dw_reg<1, true>(x, w, bias, y, rp, KH, stride, stream, d)
+                  : launch_dw_reg<1, false>(x, w, bias, y, rp, KH, stride, stream, d);
     }
 
     DwParams p;
@@ -1750,6 +1771,7 @@ const char *conv_status_string(int status) {
         case CONV_ERR_MISALIGNED: return "misaligned pointer";
         case CONV_ERR_CUDA: return "CUDA call failed";
         case CONV_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case CONV_ERR_DEVICE_BOUNDS: return "device-side bounds check failed (access skipped)";
         default: return "unknown status";
     }
 }
@@ -1776,7 +1798,44 @@ int conv_device_status(cudaStream_t stream, int reset) {
         const unsigned int zero = 0;
         if (cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return CONV_ERR_CUDA;
     }
-    return (v & kStatusTimeout) ? CONV_ERR_DEVICE_TIMEOUT : CONV_OK;
+    if (v & kStatusTimeout) return CONV_ERR_DEVICE_TIMEOUT;
+    return (v & kStatusBounds) ? CONV_ERR_DEVICE_BOUNDS : CONV_OK;
+}
+
+int conv_debug_bounds_build(void) { return kDebugBounds ? 1 : 0; }
+
+int conv_selftest_bounds(cudaStream_t stream) {
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(32);
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, selftest_bounds_kernel, d->status) == cudaSuccess ? CONV_OK : CONV_ERR_CUDA;
+}
+
+int conv_debug_bounds_info(long long *info, int reset) {
+    if (!info) return CONV_ERR_INVALID_ARG;
+    info[0] = info[1] = info[2] = -1;
+#ifdef CONV_DEBUG_BOUNDS
+    DeviceState *d = nullptr;
+    if (int rc = device_state(&d)) return rc;
+    if (cudaDeviceSynchronize() != cudaSuccess) return CONV_ERR_CUDA;
+    long long rec[4] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(rec, g_bounds_first, sizeof rec) != cudaSuccess) return CONV_ERR_CUDA;
+    if (rec[0]) {
+        info[0] = rec[1];
+        info[1] = rec[2];
+        info[2] = rec[3];
+    }
+    if (reset) {
+        const long long zero[4] = {0, 0, 0, 0};
+        if (cudaMemcpyToSymbol(g_bounds_first, zero, sizeof zero) != cudaSuccess) return CONV_ERR_CUDA;
+    }
+#else
+    (void)reset;
+#endif
+    return CONV_OK;
 }
 
 int dwpw_fwd(const float *x, const float *w_dw, const float *b_dw, const void *F, const float *b_pw, float *y, int N,

@@ -16,6 +16,8 @@
 #pragma once
 #include <cuda_bf16.h>
 
+#include "ptx.cuh"   // in_bounds (bounds-checked debug build)
+
 namespace convb200 {
 
 struct DenseDirectParams {
@@ -24,6 +26,7 @@ struct DenseDirectParams {
     int sh, sw, ph, pw, dh, dw;   // "Convolution Is Wx+b Moving Across a Signal" variants
     const float *bias;      // per output channel or null; added in fp32 before the rounding
     long long total;        // N * Ho * Wo * Cout
+    long long x_elems;      // N * H * W * Cin
 };
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
@@ -34,7 +37,7 @@ __device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __fl
 template <typename T>
 __global__ void __launch_bounds__(256)
 dense_direct_kernel(const T *__restrict__ X, const T *__restrict__ F, T *__restrict__ Y,
-                    const DenseDirectParams p) {
+                    const DenseDirectParams p, unsigned int *status) {
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < p.total;
          idx += stride) {
@@ -53,14 +56,16 @@ dense_direct_kernel(const T *__restrict__ X, const T *__restrict__ F, T *__restr
             for (int j = 0; j < p.KW; ++j) {
                 const int q = x * p.sw + j * p.dw - p.pw;
                 if (q < 0 || q >= p.W) continue;
-                const T *xr = X + ((n * p.H + r) * p.W + q) * p.Cin + cin0;
+                const long long xoff = ((n * p.H + r) * p.W + q) * p.Cin + cin0;
+                if (!in_bounds(xoff, p.Cin_g, p.x_elems, kSiteDirectX, status)) continue;
+                const T *xr = X + xoff;
                 const T *fr = F + ((static_cast<long long>(i) * p.KW + j) * p.Cin_g) * p.Cout + o;
                 for (int c = 0; c < p.Cin_g; ++c)
                     acc = __fmaf_rn(to_f32(xr[c]), to_f32(fr[static_cast<long long>(c) * p.Cout]), acc);
             }
         }
         if (p.bias) acc = __fadd_rn(acc, __ldg(p.bias + o));
-        store_out(Y + idx, acc);
+        if (in_bounds(idx, 1, p.total, kSiteDirectY, status)) store_out(Y + idx, acc);
     }
 }
 

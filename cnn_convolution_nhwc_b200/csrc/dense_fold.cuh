@@ -353,12 +353,13 @@ dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const int cc = lane % CPR;
             const int col = h * CW + cc * 8;
             if (col < p.Cout) {
+                const long long y_elems = 1LL * (p.rows / (p.H * p.W)) * p.Ho * p.Wo * p.Cout;   // bounds checks (debug build)
 #pragma unroll
                 for (int i = 0; i < CPR; ++i) {
                     const int rr = i * (32 / CPR) + lane / CPR;
                     long long off;
                     asm volatile("ld.shared.s64 %0, [%1];" : "=l"(off) : "r"(rowoff + 8u * rr));
-                    if (off >= 0) {
+                    if (off >= 0 && in_bounds(off + col, 8, y_elems, kSiteFoldY, status)) {
                         uint32_t a, bb, c, dd;
                         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                      : "=r"(a), "=r"(bb), "=r"(c), "=r"(dd)

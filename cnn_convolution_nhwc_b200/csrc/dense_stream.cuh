@@ -358,11 +358,12 @@ dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     // coalesced stores: 8 lanes per row, 4 rows per instruction
                     const int col = n0 + h * 64 + (lane & 7) * 8;
                     if (col < p.Cout) {
+                        const long long y_elems = 1LL * (p.rows / (p.H * p.W)) * p.Ho * p.Wo * p.Cout;   // bounds checks (debug build)
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const int rr = i * 4 + (lane >> 3);
                             const long long off = rowoff[rr];
-                            if (off >= 0) {
+                            if (off >= 0 && in_bounds(off + col, 8, y_elems, kSiteStreamY, status)) {
                                 uint32_t a, bb, c, d;
                                 asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                              : "=r"(a), "=r"(bb), "=r"(c), "=r"(d)

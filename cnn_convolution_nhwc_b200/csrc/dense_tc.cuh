@@ -327,7 +327,10 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
                             const int col = c0 + u * 16 + c;
-                            const float bv = col < p.ncols ? __ldg(bg + col) : 0.0f;
+                            const bool bok =
+                                col < p.ncols && in_bounds(static_cast<long long>(grp) * p.ncols + col, 1,
+                                                           static_cast<long long>(p.groups) * p.ncols, kSiteTcBias, status);
+                            const float bv = bok ? __ldg(bg + col) : 0.0f;
                             r[u][c] = __float_as_uint(__fadd_rn(__uint_as_float(r[u][c]), bv));
                         }
                 }

@@ -23,6 +23,8 @@
 #pragma once
 #include <cstdint>
 
+#include "ptx.cuh"   // in_bounds (bounds-checked debug build)
+
 namespace convb200 {
 
 // Division by an invariant divisor 1 <= d < 2^31 for dividends 0 <= n < 2^31, by a
@@ -92,7 +94,10 @@ __host__ __device__ inline int dw_smem_head_floats(int P, int w_stride) {
 template <int MODE, bool HAS_BIAS, int KW_T, int S_T, int VX>
 __global__ void __launch_bounds__(256)
 depthwise_kernel(const float *__restrict__ x, const float *__restrict__ w,
-                 const float *__restrict__ bias, float *__restrict__ y, const DwParams p) {
+                 const float *__restrict__ bias, float *__restrict__ y, const DwParams p, unsigned int *status) {
+    // tensor extents for the bounds-checked debug build
+    const long long x_elems = 1LL * (p.num_planes / p.Cout) * p.Cin * p.H * p.W;
+    const long long y_elems = 1LL * p.num_planes * p.Ho * p.Wo;
     extern __shared__ __align__(16) float sm[];
     long long *s_inoff = reinterpret_cast<long long *>(sm);
     float *sb = sm + 2 * ((p.P + 1) & ~1);
@@ -148,7 +153,8 @@ depthwise_kernel(const float *__restrict__ x, const float *__restrict__ w,
             while (pp < nplanes) {
                 if (pp != cur) { xp = x + s_inoff[pp]; cur = pp; }
                 const int gy = iy0 + r;
-                const bool ok = col_ok && gy >= 0 && gy < p.H;
+                const bool ok = col_ok && gy >= 0 && gy < p.H &&
+                                in_bounds(s_inoff[pp] + static_cast<long long>(gy) * p.W + gx, 1, x_elems, kSiteDwX, status);
                 cp_async_f32_zfill(sx_s + 4u * (pp * tile + r * p.pitch + c),
                                    ok ? xp + static_cast<long long>(gy) * p.W + gx : x, ok);
                 r += row_step;
@@ -198,12 +204,14 @@ depthwise_kernel(const float *__restrict__ x, const float *__restrict__ w,
             }
 #pragma unroll
             for (int v = 0; v < VX; ++v) acc[v] = dw_finish<MODE, HAS_BIAS>(acc[v], b);
+            const long long yoff = yrow - y;
             if (VX == 4 && p.vec_store && ox + 4 <= ncols) {
-                *reinterpret_cast<float4 *>(yrow) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                if (in_bounds(yoff, 4, y_elems, kSiteDwY, status))
+                    *reinterpret_cast<float4 *>(yrow) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             } else {
 #pragma unroll
                 for (int v = 0; v < VX; ++v)
-                    if (ox + v < ncols) yrow[v] = acc[v];
+                    if (ox + v < ncols && in_bounds(yoff + v, 1, y_elems, kSiteDwY, status)) yrow[v] = acc[v];
             }
         } else {
             // runtime kernel size, stride and dilation; VX == 1
@@ -213,7 +221,7 @@ depthwise_kernel(const float *__restrict__ x, const float *__restrict__ w,
                 const float *xr = xs + ky * p.dil * p.pitch;
                 for (int kx = 0; kx < p.KW; ++kx) acc = dw_tap<MODE>(acc, ws[ky * p.KW + kx], xr[kx * p.dil]);
             }
-            yrow[0] = dw_finish<MODE, HAS_BIAS>(acc, b);
+            if (in_bounds(yrow - y, 1, y_elems, kSiteDwY, status)) yrow[0] = dw_finish<MODE, HAS_BIAS>(acc, b);
         }
     }
 }

@@ -77,10 +77,18 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
         const uint32_t bulk = total & ~3u;
         const float *src = x + static_cast<long long>(plane0) * (HW * HW);
         if (lane == 0) {
+            // the job's range of x, checked in the bounds-checked debug build (a skipped copy
+            // still completes the barrier's byte count)
+            const bool in = in_bounds(static_cast<long long>(plane0) * (HW * HW), total,
+                                      1LL * p.num_planes * (HW * HW), kSiteDwPlaneX, status);
             float *dst = sin0 + b * p.in_floats;
-            for (uint32_t e = bulk; e < total; ++e) dst[e] = src[e];
+            if (in)
+                for (uint32_t e = bulk; e < total; ++e) dst[e] = src[e];
             mbar_arrive_expect_tx(bar(b), 4u * bulk);
-            if (bulk) bulk_g2s(sin_s + 4u * b * p.in_floats, src, 4u * bulk, bar(b));
+            if (bulk) {
+                if (in) bulk_g2s(sin_s + 4u * b * p.in_floats, src, 4u * bulk, bar(b));
+                else mbar_complete_tx(bar(b), 4u * bulk);
+            }
         }
     };
 
@@ -224,7 +232,10 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
         const int nplanes = min(PPJ, p.num_planes - plane0);
         const int total = nplanes * (HO * WO);
         float *gdst = y + static_cast<long long>(plane0) * (HO * WO);
-        if (p.vec_y && ((plane0 * (HO * WO)) & 3) == 0) {
+        if (!in_bounds(static_cast<long long>(plane0) * (HO * WO), total, 1LL * p.num_planes * (HO * WO), kSiteDwPlaneY,
+                       status)) {
+            // skipped (bounds-checked debug build)
+        } else if (p.vec_y && ((plane0 * (HO * WO)) & 3) == 0) {
             const int n4 = total >> 2;
             for (int e = lane; e < n4; e += 32)
                 reinterpret_cast<float4 *>(gdst)[e] = reinterpret_cast<const float4 *>(sout)[e];

@@ -40,7 +40,8 @@ struct DwRegParams {
 template <int MODE, bool HAS_BIAS, int K, int S, int PAD>
 __global__ void __launch_bounds__(256)
 depthwise_reg_kernel(const float *__restrict__ x, const float *__restrict__ w,
-                     const float *__restrict__ bias, float *__restrict__ y, const DwRegParams p) {
+                     const float *__restrict__ bias, float *__restrict__ y, const DwRegParams p,
+                     unsigned int *status) {
     constexpr int VX = 4;                    // outputs per lane along the row
     constexpr int OWN = VX * S;              // input columns a lane loads per row
     constexpr int WIN = (VX - 1) * S + K;    // input columns one lane's outputs read per row
@@ -71,10 +72,15 @@ depthwise_reg_kernel(const float *__restrict__ x, const float *__restrict__ w,
     const int nrows = min(p.band, p.Ho - oy0);
     const bool lane_has_cols = active && c0 < p.W;
 
+    // tensor extents for the bounds-checked debug build
+    const long long x_elems = 1LL * (p.num_planes / p.Cout) * p.Cin * p.H * p.W;
+    const long long y_elems = 1LL * p.num_planes * p.Ho * p.Wo;
     // loads this lane's OWN columns of input row r (zeros outside the image)
     auto load_own = [&](int r, float (&own)[OWN]) {
-        const bool row_ok = lane_has_cols && r >= 0 && r < p.H;
+        bool row_ok = lane_has_cols && r >= 0 && r < p.H;
         const float *src = xp + static_cast<long long>(row_ok ? r : 0) * p.W + c0;
+        if (row_ok)
+            row_ok = in_bounds(src - x, min(OWN, p.W - c0), x_elems, kSiteDwRegX, status);
         if (p.vec_in && row_ok && c0 + OWN <= p.W) {
 #pragma unroll
             for (int q = 0; q < OWN / 4; ++q) {
@@ -144,7 +150,9 @@ depthwise_reg_kernel(const float *__restrict__ x, const float *__restrict__ w,
         const int ox = cg * VX;
         if (active && ox < p.Wo) {
             float *dst = yp + static_cast<long long>(oy) * p.Wo + ox;
-            if (p.vec_out && ox + VX <= p.Wo) {
+            if (!in_bounds(dst - y, min(VX, p.Wo - ox), y_elems, kSiteDwRegY, status)) {
+                // skipped (bounds-checked debug build)
+            } else if (p.vec_out && ox + VX <= p.Wo) {
                 *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             } else {
 #pragma unroll

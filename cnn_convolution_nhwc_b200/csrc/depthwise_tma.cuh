@@ -162,6 +162,9 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
                 const uint32_t dplane = dst + 4u * (s * p.rows_in + PAD) * p.Wp + 16u;
                 for (int e = lane; e < HW; e += 32) {
                     const int r = fdiv(e, p.div_w);
+                    if (!in_bounds(static_cast<long long>(plane) * HW + e, 1, 1LL * p.num_planes * HW, kSiteDwTmaX,
+                                   status))
+                        continue;
                     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dplane + 4u * (r * p.Wp + e - r * p.W)),
                                  "l"(src + e)
                                  : "memory");
@@ -222,7 +225,9 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
                 }
             } else if (active) {
                 float *dst = yp + static_cast<long long>(i) * p.Wo;
-                if (p.vec_out && ox + VX <= p.Wo) {
+                if (!in_bounds(dst - y, min(VX, p.Wo - ox), 1LL * p.num_planes * p.Ho * p.Wo, kSiteDwTmaY, status)) {
+                    // skipped (bounds-checked debug build)
+                } else if (p.vec_out && ox + VX <= p.Wo) {
                     *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
                 } else {
 #pragma unroll
@@ -325,7 +330,10 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
             const int plane_out = p.Ho * p.Wo;
             const int total = nplanes * plane_out;
             float *gdst = y + static_cast<long long>(plane0) * plane_out;
-            if (p.vec_out_staged && ((plane0 * plane_out) & 3) == 0) {
+            if (!in_bounds(static_cast<long long>(plane0) * plane_out, total, 1LL * p.num_planes * plane_out,
+                           kSiteDwTmaY, status)) {
+                // skipped (bounds-checked debug build)
+            } else if (p.vec_out_staged && ((plane0 * plane_out) & 3) == 0) {
                 const int n4 = total >> 2;
                 for (int e = lane; e < n4; e += 32)
                     reinterpret_cast<float4 *>(gdst)[e] = reinterpret_cast<const float4 *>(sout)[e];

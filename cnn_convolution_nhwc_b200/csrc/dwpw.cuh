@@ -153,7 +153,11 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
             ox = pix - oy * p.Wo;
         }
         const int iy0 = oy * p.stride - p.pad, ix0 = ox * p.stride - p.pad;
-        const float *xn = x + static_cast<long long>(n) * p.C * plane;
+        // the image's planes (bounds-checked debug build: an image past the tensor reads image 0
+        // instead; the tap offsets stay inside a plane by construction)
+        const bool x_in = in_bounds(static_cast<long long>(n) * p.C * plane, p.C * plane,
+                                    1LL * (p.M / p.HoWo) * p.C * plane, kSiteDwPwX, status);
+        const float *xn = x + (x_in ? static_cast<long long>(n) * p.C * plane : 0LL);
         // this pixel's taps, once per tile: which lie inside the image (bit t of inmask, tap
         // t = ky*K + kx) and, for 5x5, an offset inside the plane (a harmless in-plane one for
         // taps outside the image) with a mask that turns those taps into +0
@@ -330,7 +334,9 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
                             if (o < p.Cout) {
                                 float val = __uint_as_float(t[j]);
                                 if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
-                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                                if (in_bounds((yrow - y) + static_cast<long long>(o) * p.HoWo, 1,
+                                              1LL * p.M * p.Cout, kSiteDwPwY, status))
+                                    yrow[static_cast<long long>(o) * p.HoWo] = val;
                             }
                         }
                     }
@@ -382,7 +388,9 @@ dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __gr
                             if (o < p.Cout) {
                                 float val = acc[j];
                                 if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
-                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                                if (in_bounds((yrow - y) + static_cast<long long>(o) * p.HoWo, 1,
+                                              1LL * p.M * p.Cout, kSiteDwPwY, status))
+                                    yrow[static_cast<long long>(o) * p.HoWo] = val;
                             }
                         }
                     }
@@ -516,6 +524,9 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
                 for (int gi = 0; gi < imgs_here; ++gi) {
                     const float *src = x + ((static_cast<long long>(n0 + gi) * p.C + c) * p.H + iy_lo) * p.W;
                     float *dst = dx + ((ch * st.G + gi) * st.R_in + row0) * st.Wp + p.pad;
+                    if (!in_bounds(src - x, static_cast<long long>(nr) * p.W, 1LL * (p.M / p.HoWo) * p.C * p.H * p.W,
+                                   kSiteDwPwX, status))
+                        continue;
                     for (int k = lane; k < span; k += 32) {
                         const int rr = fdiv(k, st.div_wcols);
                         const int cc = k - rr * st.wcols;
@@ -670,7 +681,9 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
                             if (o < p.Cout) {
                                 float val = __uint_as_float(t[jj]);
                                 if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
-                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                                if (in_bounds((yrow - y) + static_cast<long long>(o) * p.HoWo, 1,
+                                              1LL * p.M * p.Cout, kSiteDwPwY, status))
+                                    yrow[static_cast<long long>(o) * p.HoWo] = val;
                             }
                         }
                     }
@@ -719,7 +732,9 @@ dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, con
                             if (o < p.Cout) {
                                 float val = acc[jj];
                                 if (p.b_pw) val = __fadd_rn(val, __ldg(p.b_pw + o));
-                                yrow[static_cast<long long>(o) * p.HoWo] = val;
+                                if (in_bounds((yrow - y) + static_cast<long long>(o) * p.HoWo, 1,
+                                              1LL * p.M * p.Cout, kSiteDwPwY, status))
+                                    yrow[static_cast<long long>(o) * p.HoWo] = val;
                             }
                         }
                     }

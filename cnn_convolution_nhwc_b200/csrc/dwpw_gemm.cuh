@@ -53,7 +53,6 @@
 #include "depthwise_tma.cuh"   // packed-pair helpers
 #include "depthwise_plane.cuh" // bulk_g2s
 #include "dense_halo.cuh"      // tma_load_2d
-#include "dwpw.cuh"            // cluster helpers
 #include "ptx.cuh"
 
 namespace convb200 {
@@ -215,19 +214,32 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
         const float *src = x + (static_cast<long long>(n) * p.C + c0) * G::P;
         // the planes' taps: planes * KK floats from w[c0], a multiple of 16 bytes (C % 4 == 0)
         const uint32_t wbytes = static_cast<uint32_t>(planes * KK * 4);
+        // 1-D bulk copies are not bounded by a tensor map: checked in the bounds-checked debug
+        // build, where a skipped copy still completes the barrier's byte count
+        auto copy_w = [&]() {
+            if (in_bounds(static_cast<long long>(c0) * KK, static_cast<long long>(planes) * KK, 1LL * p.C * KK,
+                          kSiteDwPwGemmW, status))
+                bulk_g2s(sW + (g & 1) * WSLOT, w + static_cast<long long>(c0) * KK, wbytes, xfull(g & 1));
+            else
+                mbar_complete_tx(xfull(g & 1), wbytes);
+        };
         if constexpr (G::PADX) {
             // x viewed as [N*C][P]: a box of XP columns x CB rows (always the full box's bytes;
             // rows past the image's channels are other planes or zeros, never used)
             if (lane == 0) {
                 mbar_arrive_expect_tx(xfull(g & 1), static_cast<uint32_t>(G::CB * G::XP * 4) + wbytes);
                 tma_load_2d(sX + (g & 1) * G::XSLOT, &tmX, xfull(g & 1), 0, n * p.C + c0);
-                bulk_g2s(sW + (g & 1) * WSLOT, w + static_cast<long long>(c0) * KK, wbytes, xfull(g & 1));
+                copy_w();
             }
         } else if (lane == 0) {
             const uint32_t bytes = static_cast<uint32_t>(planes * G::P * 4);
             mbar_arrive_expect_tx(xfull(g & 1), bytes + wbytes);
-            bulk_g2s(sX + (g & 1) * G::XSLOT, src, bytes, xfull(g & 1));
-            bulk_g2s(sW + (g & 1) * WSLOT, w + static_cast<long long>(c0) * KK, wbytes, xfull(g & 1));
+            if (in_bounds((static_cast<long long>(n) * p.C + c0) * G::P, static_cast<long long>(planes) * G::P,
+                          1LL * p.num_tiles * p.C * G::P, kSiteDwPwGemmX, status))
+                bulk_g2s(sX + (g & 1) * G::XSLOT, src, bytes, xfull(g & 1));
+            else
+                mbar_complete_tx(xfull(g & 1), bytes);
+            copy_w();
         }
         __syncwarp();
     };
@@ -347,6 +359,8 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
 
     // 16 consecutive pixels of output channel o: acc (+ the cluster peer's partial) + bias -> y
     auto store_chunk = [&](float *yrow, int p0, const float (&v)[16], float bp) {
+        if (!in_bounds((yrow - y) + p0, min(16, G::P - p0), 1LL * p.num_tiles * p.Cout * G::P, kSiteDwPwGemmY, status))
+            return;   // skipped (bounds-checked debug build)
         if constexpr (G::P % 4 == 0) {
 #pragma unroll
             for (int u = 0; u < 4; ++u)

@@ -14,6 +14,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"   // in_bounds (bounds-checked debug build)
+
 namespace convb200 {
 
 struct Im2colParams {
@@ -24,8 +26,12 @@ struct Im2colParams {
 };
 
 __global__ void __launch_bounds__(256)
-im2col_pack_kernel(const __nv_bfloat16 *__restrict__ X, __nv_bfloat16 *__restrict__ A, const Im2colParams p) {
+im2col_pack_kernel(const __nv_bfloat16 *__restrict__ X, __nv_bfloat16 *__restrict__ A, const Im2colParams p,
+                   unsigned int *status) {
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    // tensor extents for the bounds-checked debug build
+    const long long a_elems = p.chunks * p.chunk;
+    const long long x_elems = (a_elems / p.kd) / (1LL * p.Ho * p.Wo) * p.H * p.W * p.Cin;
     const int per_tap = p.Cin / p.chunk;
     for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < p.chunks; t += stride) {
         long long u = t;
@@ -40,6 +46,9 @@ im2col_pack_kernel(const __nv_bfloat16 *__restrict__ X, __nv_bfloat16 *__restric
         const long long n = r / p.Ho;
         const long long src = ((n * p.H + (y + i)) * p.W + (x + j)) * p.Cin + static_cast<long long>(cc) * p.chunk;
         const long long dst = m * p.kd + static_cast<long long>(tap) * p.Cin + static_cast<long long>(cc) * p.chunk;
+        if (!in_bounds(src, p.chunk, x_elems, kSiteIm2colX, status) ||
+            !in_bounds(dst, p.chunk, a_elems, kSiteIm2colA, status))
+            continue;   // skipped (bounds-checked debug build)
         if (p.chunk == 8)
             *reinterpret_cast<uint4 *>(A + dst) = __ldg(reinterpret_cast<const uint4 *>(X + src));
         else

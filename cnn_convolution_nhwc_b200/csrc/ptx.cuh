@@ -8,7 +8,43 @@
 namespace convb200 {
 
 // Device status word bits (one per failure kind). Written with atomicOr, read by the host.
-enum : unsigned { kStatusTimeout = 1u };
+enum : unsigned { kStatusTimeout = 1u, kStatusBounds = 2u };
+
+// ---- bounds-checked debug build ---------------------------------------------------------
+// Compiled with -DCONV_DEBUG_BOUNDS, every plain global load or store whose address the kernels
+// compute (and every 1-D bulk copy, which no tensor map bounds) is first checked against the
+// extent of its tensor: elements [idx, idx + len) of a tensor of `limit` elements. A failed check
+// sets kStatusBounds in the status word, records the first failure (site, index, limit) and
+// returns false: the caller skips the access -- no assertion, no trap, the context stays usable.
+// Tensor-map (TMA) copies need no check: the hardware bounds them. In the normal build the
+// check is the constant true and costs nothing.
+enum BoundsSite : unsigned {
+    kSiteDirectX = 1, kSiteDirectY, kSiteFoldY, kSiteHaloY, kSiteStreamY, kSiteTcBias, kSiteDwY, kSiteDwRegX,
+    kSiteDwRegY, kSiteDwTmaY, kSiteDwPlaneX, kSiteDwPlaneY, kSiteDwPwX, kSiteDwPwY, kSiteDwPwGemmX,
+    kSiteDwPwGemmW, kSiteDwPwGemmY, kSiteIm2colX, kSiteIm2colA, kSiteDwTmaX, kSiteDwX, kSiteSelftest = 255
+};
+#ifdef CONV_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+// [0] claimed flag, [1] site, [2] index, [3] limit of the first failed check
+__device__ long long g_bounds_first[4];
+__device__ __noinline__ void bounds_record(unsigned site, long long idx, long long limit, unsigned *status) {
+    atomicOr(status, kStatusBounds);
+    if (atomicCAS(reinterpret_cast<unsigned long long *>(&g_bounds_first[0]), 0ull, 1ull) == 0ull) {
+        g_bounds_first[1] = site;
+        g_bounds_first[2] = idx;
+        g_bounds_first[3] = limit;
+    }
+}
+__device__ __forceinline__ bool in_bounds(long long idx, long long len, long long limit, unsigned site,
+                                          unsigned *status) {
+    if (idx >= 0 && len >= 0 && idx + len <= limit) return true;
+    bounds_record(site, idx, limit, status);
+    return false;
+}
+#else
+constexpr bool kDebugBounds = false;
+__device__ __forceinline__ bool in_bounds(long long, long long, long long, unsigned, unsigned *) { return true; }
+#endif
 
 // Every spin on an mbarrier gives up after this many SM clock cycles (about one second at
 // the B200's 1.9-2.0 GHz; longer at lower clocks). The SM-local cycle counter is cheap to read,
@@ -37,6 +73,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Completes `bytes` of the barrier's expected transaction count without a copy (a copy that a
+// bounds check skipped).
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
 // One poll of the phase with the given parity (no suspend-time hint: measured on B200, a

@@ -62,7 +62,9 @@ typedef enum {
     CONV_ERR_UNSUPPORTED = -2,    /* valid arguments outside what this library implements */
     CONV_ERR_MISALIGNED = -3,     /* a pointer not aligned to its element size */
     CONV_ERR_CUDA = -4,           /* a CUDA runtime or driver call failed (launch, tensor map) */
-    CONV_ERR_DEVICE_TIMEOUT = -5  /* a bounded device-side wait ran out (see conv_device_status) */
+    CONV_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait ran out (see conv_device_status) */
+    CONV_ERR_DEVICE_BOUNDS = -6   /* bounds-checked build only: a kernel skipped an access outside
+                                     its tensor (see conv_debug_bounds_info) */
 } conv_status;
 
 typedef enum {
@@ -249,10 +251,42 @@ const char *conv_status_string(int status);
 
 /*
  * Synchronises `stream`, then reads the device status word of the current device:
- * CONV_OK, CONV_ERR_DEVICE_TIMEOUT, or CONV_ERR_CUDA if the synchronisation itself failed.
- * With reset != 0 the word is cleared afterwards.
+ * CONV_OK, CONV_ERR_DEVICE_TIMEOUT, CONV_ERR_DEVICE_BOUNDS (bounds-checked build only; a timeout
+ * takes precedence), or CONV_ERR_CUDA if the synchronisation itself failed. With reset != 0
+ * the word is cleared afterwards.
  */
 int conv_device_status(cudaStream_t stream, int reset);
+
+/*
+ * The bounds-checked build. The library's sources compiled with -DCONV_DEBUG_BOUNDS (the file
+ * libconv_b200_debug.so beside libconv_b200.so; the Python binding loads it when
+ * CONV_B200_DEBUG_BOUNDS=1 at import) check every global-memory element range a kernel computes
+ * before touching it -- plain loads and stores, and 1-D bulk copies, which no tensor map bounds
+ * -- against the extent of the tensor it belongs to. A failed check sets CONV_ERR_DEVICE_BOUNDS
+ * in the device status word, records the first failure, and skips the access (a skipped bulk
+ * copy still completes its barrier's byte count, so no wait is left hanging); no assertion or
+ * trap is raised and the context stays usable. Tensor-map copies are bounded by the hardware
+ * and are not checked. These are a debugging aid of this library; the pages describe no such
+ * mode.
+ *
+ * conv_debug_bounds_build: 1 in the bounds-checked build, 0 in the normal one (no device access).
+ * conv_debug_bounds_info: synchronises the current device and writes to info[0..2] the first
+ * failed check since the last reset -- the site (an internal identifier of the access), the
+ * element index and the tensor's element count -- or -1, -1, -1 if none (always so in the
+ * normal build); reset != 0 clears the record. Returns CONV_OK, CONV_ERR_INVALID_ARG for a null
+ * info, or CONV_ERR_CUDA.
+ */
+int conv_debug_bounds_build(void);
+int conv_debug_bounds_info(long long *info, int reset);
+
+/*
+ * Diagnostic for the bounds checks: one kernel thread checks the element range [1000, 1001) of
+ * a notional 1000-element tensor and touches no memory whatever the outcome. In the
+ * bounds-checked build the check fails: the status word gets CONV_ERR_DEVICE_BOUNDS and
+ * conv_debug_bounds_info reports site 255, index 1000, limit 1000. In the normal build nothing
+ * is recorded. Returns the launch status.
+ */
+int conv_selftest_bounds(cudaStream_t stream);
 
 /*
  * Name of the kernel family the last successful conv2d_nhwc_fwd, conv2d_nhwc_fwd_f32 or

@@ -33,9 +33,27 @@ def test_library_exports_every_declared_symbol():
         assert getattr(cb.lib, name) is not None
 
 
+def test_bounds_checked_build_exports_the_same_symbols():
+    # the -DCONV_DEBUG_BOUNDS variant of the same sources: every declared entry point, and a
+    # build flag that says which variant is loaded (no device access)
+    from cnn_convolution_nhwc_b200 import build as b
+    path = b.build(debug_bounds=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared():
+        assert name in syms, name
+    dbg = ctypes.CDLL(path)
+    assert dbg.conv_debug_bounds_build() == 1
+    assert cb.lib.conv_debug_bounds_build() == (1 if cb.DEBUG_BOUNDS else 0)
+
+
+def test_bounds_info_rejects_null():
+    assert cb.lib.conv_debug_bounds_info(None, 0) == cb.CONV_ERR_INVALID_ARG
+
+
 def test_status_strings():
     for code in (cb.CONV_OK, cb.CONV_ERR_INVALID_ARG, cb.CONV_ERR_UNSUPPORTED, cb.CONV_ERR_MISALIGNED,
-                 cb.CONV_ERR_CUDA, cb.CONV_ERR_DEVICE_TIMEOUT):
+                 cb.CONV_ERR_CUDA, cb.CONV_ERR_DEVICE_TIMEOUT, cb.CONV_ERR_DEVICE_BOUNDS):
         s = cb.conv_status_string(code)
         assert s and s != "unknown status"
     assert cb.conv_status_string(12345) == "unknown status"
