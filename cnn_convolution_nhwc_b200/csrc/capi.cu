@@ -227,6 +227,26 @@ int env_int(const char *name, int def, int lo, int hi) {
     return r;
 }
 
+// Every kernel launch allows programmatic dependent launch: the next kernel on the stream may be
+// scheduled while this one drains, because each kernel waits for its predecessors before its
+// first global-memory access (grid_dependency_wait). CONV_B200_PDL=0 launches without it
+// (measurements).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(cudaLaunchConfig_t cfg, void (*kern)(KArgs...), Args... args) {
+    cudaLaunchAttribute attrs[4];
+    unsigned n = 0;
+    for (unsigned i = 0; i < cfg.numAttrs && n < 3; ++i) attrs[n++] = cfg.attrs[i];
+    if (env_int("CONV_B200_PDL", 1, 0, 1) == 1) {
+        attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+
 // ---------------------------------------------------------------------------------------
 // Dense
 // ---------------------------------------------------------------------------------------
@@ -289,7 +309,7 @@ int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int C
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, dense_direct_kernel<T>, X, F, Y, p, d->status), "dense_direct_kernel");
+    return launched(launch_k(cfg, dense_direct_kernel<T>, X, F, Y, p, d->status), "dense_direct_kernel");
 }
 
 // The im2col tensor-core kernel over groups g0 .. g0 + NG - 1 per launch (one launch when
@@ -374,7 +394,7 @@ int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, 
         cfg.blockDim = dim3(192);
         cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
         cfg.stream = stream;
-        if (int rc = launched(cudaLaunchKernelEx(&cfg, kern, maps, p, d->status), "dense_tc_kernel")) return rc;
+        if (int rc = launched(launch_k(cfg, kern, maps, p, d->status), "dense_tc_kernel")) return rc;
     }
     return CONV_OK;
 }
@@ -460,6 +480,8 @@ HaloPlan plan_halo(int N, int H, int W, int Cin, int Cout, int K, int num_sms, i
         pl.grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
     }
     pl.smem = fixed + p.b_region + p.HS * halo_bytes;
+    // more than half of the shared memory keeps a second CTA (and its TMEM allocation) off the SM
+    if (pl.smem < 116 * 1024) pl.smem = 116 * 1024;
     pl.bn = bn;
     pl.ok = pl.smem <= kSmemLimit && pl.grid >= 1;
     return pl;
@@ -496,7 +518,7 @@ int launch_dense_halo(const void *X, const void *F, void *Y, int Cin, int Cout, 
     cfg.blockDim = dim3(Cfg::THREADS);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
+    return launched(launch_k(cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
                     "dense_halo_kernel");
 }
 
@@ -594,7 +616,7 @@ int launch_dense_fold(const void *X, const void *F, void *Y, int Cin, int Cout, 
     cfg.blockDim = dim3(DenseFoldCfg<KF>::THREADS);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
+    return launched(launch_k(cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
                     "dense_fold_kernel");
 }
 
@@ -721,7 +743,7 @@ int launch_dense_stream(const void *X, const void *F, void *Y, int Cin, int Cout
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return launched(cudaLaunchKernelEx(&cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
+    return launched(launch_k(cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), pl.p, d->status),
                     "dense_stream_kernel");
 }
 
@@ -814,7 +836,7 @@ int launch_dw_one(const float *x, const float *w, const float *bias, float *y, c
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, p, d->status), "depthwise_kernel");
+    return launched(launch_k(cfg, kern, x, w, bias, y, p, d->status), "depthwise_kernel");
 }
 
 // ---- register-window kernel ---------------------------------------------------------------
@@ -825,7 +847,7 @@ int launch_dw_reg_one(const float *x, const float *w, const float *bias, float *
     cfg.gridDim = dim3(static_cast<unsigned>((rp.num_jobs + 7) / 8));
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, depthwise_reg_kernel<MODE, HB, K, S, (K - 1) / 2>, x, w, bias, y, rp,
+    return launched(launch_k(cfg, depthwise_reg_kernel<MODE, HB, K, S, (K - 1) / 2>, x, w, bias, y, rp,
                                        d->status),
                     "depthwise_reg_kernel");
 }
@@ -1013,7 +1035,7 @@ int launch_dw_tma_one(const float *x, const float *w, const float *bias, float *
     cfg.blockDim = dim3(32 * kDwWarpsPerCta);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, kern, tm, x, w, bias, y, p, d->status), "depthwise_tma_kernel");
+    return launched(launch_k(cfg, kern, tm, x, w, bias, y, p, d->status), "depthwise_tma_kernel");
 }
 
 template <int MODE, bool HB>
@@ -1078,7 +1100,7 @@ int launch_dw_plane_one(const float *x, const float *w, const float *bias, float
     cfg.blockDim = dim3(32 * kDwPlaneWarps);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
-    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, bias, y, pl.p, d->status), "depthwise_plane_kernel");
+    return launched(launch_k(cfg, kern, x, w, bias, y, pl.p, d->status), "depthwise_plane_kernel");
 }
 
 template <int MODE, bool HB>
@@ -1195,7 +1217,7 @@ int launch_dwpw(const float *x, const float *w, const CUtensorMap &tmF, float *y
     if (int rc = dwpw_split_config(kern, bit, kDwPwFixed + 4 * p.w_floats, kDwPwStages, p, force_split, stream, d,
                                    cfg, attr))
         return rc;
-    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, d->status), "dwpw_kernel");
+    return launched(launch_k(cfg, kern, x, w, tmF, y, p, d->status), "dwpw_kernel");
 }
 
 // The staged kernel's tiles for this shape (ok = false: it does not apply).
@@ -1250,7 +1272,7 @@ int launch_dwpw_staged(const float *x, const float *w, const CUtensorMap &tmF, f
     if (int rc = dwpw_split_config(kern, bit, dwpw_staged_smem(pl.st), dwpw_staged_body(pl.st), p, force_split,
                                    stream, d, cfg, attr))
         return rc;
-    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, y, p, pl.st, d->status), "dwpw_staged_kernel");
+    return launched(launch_k(cfg, kern, x, w, tmF, y, p, pl.st, d->status), "dwpw_staged_kernel");
 }
 
 // Output-channel tile width of the im2col kernel: 64 for narrow groups; 256 for groups of at
@@ -1397,7 +1419,7 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return launched(cudaLaunchKernelEx(&cfg, kern, x, w, tmF, tmX, y, p, d->status), "dwpw_gemm_kernel");
+    return launched(launch_k(cfg, kern, x, w, tmF, tmX, y, p, d->status), "dwpw_gemm_kernel");
 }
 
 template <int MODE>
@@ -1598,7 +1620,7 @@ int conv2d_nhwc_fwd_im2col(const void *X, const void *F, void *Y, void *workspac
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
     auto *A = static_cast<__nv_bfloat16 *>(workspace);
-    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p, d->status),
+    if (launched(launch_k(cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p, d->status),
                  "im2col_pack_kernel") != CONV_OK)
         return CONV_ERR_CUDA;
     // Y (M x Cout, row-major) = A (M x kd) * F (kd x Cout): in cuBLAS's column-major terms
@@ -1646,7 +1668,7 @@ int conv2d_nhwc_fwd_im2col_noalloc(const void *X, const void *F, void *Y, int N,
     cfg.blockDim = dim3(256);
     cfg.stream = stream;
     auto *A = static_cast<__nv_bfloat16 *>(scratch);
-    if (launched(cudaLaunchKernelEx(&cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p, d->status),
+    if (launched(launch_k(cfg, im2col_pack_kernel, static_cast<const __nv_bfloat16 *>(X), A, p, d->status),
                  "im2col_pack_kernel") != CONV_OK)
         return CONV_ERR_CUDA;
     // Y = A * F as the 1 x 1 convolution of the patch image [N][Ho][Wo][kd] with F viewed as

@@ -38,6 +38,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 dense_direct_kernel(const T *__restrict__ X, const T *__restrict__ F, T *__restrict__ Y,
                     const DenseDirectParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < p.total;
          idx += stride) {

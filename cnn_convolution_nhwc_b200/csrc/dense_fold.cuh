@@ -93,6 +93,8 @@ template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 dense_fold_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
                   __nv_bfloat16 *__restrict__ Y, const DenseFoldParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int K = Cfg::K;
     constexpr int NF = Cfg::NF;
     constexpr int TM = Cfg::TM;

@@ -64,7 +64,11 @@ struct DenseHaloCfg {
     static constexpr int EPI_BYTES = NUM_EPI * 32 * 128;   // per-warp 32 rows x 64 channels staging
     static constexpr int MAX_RING = 8;
     static constexpr int NUM_BARS = 2 * MAX_RING /*halo*/ + 2 * MAX_RING /*filter*/ + 4 /*acc*/ + 2;
-    static constexpr int TMEM_COLS = 2 * BN;
+    // Tiles up to 128 columns wide alternate their MMAs between two partial accumulators (an MMA
+    // into the accumulator the previous one wrote waits for it: measured on B200, 99 against 64
+    // cycles at N = 128), summed once in the epilogue; two tiles in flight either way.
+    static constexpr int PARTS = BN <= 128 ? 2 : 1;
+    static constexpr int TMEM_COLS = 2 * PARTS * BN;
     static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ true);
     // shared-memory bytes besides the filter region and the halo ring
     static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + NUM_BARS * 8 + NUM_EPI * 32 * 8 + 16;
@@ -89,6 +93,8 @@ template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
                   __nv_bfloat16 *__restrict__ Y, const DenseHaloParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int BN = Cfg::BN;
     constexpr bool BRES = Cfg::BRES;
     extern __shared__ uint8_t smem_raw[];
@@ -238,7 +244,7 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             // of taking its issue slots
             if (!mbar_wait_warp_backoff(acce(b), ((local >> 1) & 1u) ^ 1u, 64)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + b * BN;
+            const uint32_t d_tmem = tmem_base + b * (Cfg::PARTS * BN);   // partial k at + k*BN
             for (int cb = 0; cb < p.num_cblk && ok; ++cb) {
                 const uint32_t hs = hit % p.HS, hph = (hit / p.HS) & 1u;
                 if (!mbar_wait_warp(hfull(hs), hph)) { ok = false; break; }
@@ -251,15 +257,19 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     // channels of A, +128 per 16 reduction rows of B
                     const uint64_t a0 = smem_desc_sw128(halo, 16, 1024);
                     uint64_t bd = smem_desc_sw128(sB + cb * p.KK * Cfg::B_BYTES, Cfg::B_BOX_BYTES, 1024);
-                    const uint32_t accumulate_first = cb != 0 ? 1u : 0u;
+                    // the tile's first MMA into each partial accumulator overwrites it
+                    const uint32_t acc_first = cb != 0 ? 1u : 0u;
+                    constexpr uint32_t P1 = Cfg::PARTS == 2 ? BN : 0u;   // the second partial's columns
                     uint32_t row = 0;
                     for (int ky = 0; ky < p.K; ++ky, row += p.W) {
                         for (int kx = 0; kx < p.K; ++kx, bd += Cfg::B_BYTES >> 4) {
                             const uint64_t ad = a0 + static_cast<uint64_t>((row + kx) * 8u);
-                            umma_f16_ss_if(d_tmem, ad, bd, Cfg::IDESC, (ky | kx) != 0 ? 1u : accumulate_first, leader);
-                            umma_f16_ss_if(d_tmem, ad + 2, bd + 128, Cfg::IDESC, 1u, leader);
+                            const uint32_t first = (ky | kx) != 0 ? 1u : acc_first;
+                            umma_f16_ss_if(d_tmem, ad, bd, Cfg::IDESC, first, leader);
+                            umma_f16_ss_if(d_tmem + P1, ad + 2, bd + 128, Cfg::IDESC, Cfg::PARTS == 2 ? first : 1u,
+                                           leader);
                             umma_f16_ss_if(d_tmem, ad + 4, bd + 256, Cfg::IDESC, 1u, leader);
-                            umma_f16_ss_if(d_tmem, ad + 6, bd + 384, Cfg::IDESC, 1u, leader);
+                            umma_f16_ss_if(d_tmem + P1, ad + 6, bd + 384, Cfg::IDESC, 1u, leader);
                         }
                     }
                 } else {
@@ -275,9 +285,11 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         const uint64_t ad = a0 + row8;
                         const uint64_t bd = b0 + bs * (Cfg::B_BYTES >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_f16_ss_if(d_tmem, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC,
-                                           (cb | tap | kk) != 0 ? 1u : 0u, leader);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t part = Cfg::PARTS == 2 ? (kk & 1) : 0;
+                            umma_f16_ss_if(d_tmem + part * BN, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC,
+                                           ((cb | tap) != 0 || kk >= Cfg::PARTS) ? 1u : 0u, leader);
+                        }
                         umma_commit_if(bempty(bs), leader);
                         ++bit;
                         row8 += 8u;
@@ -323,13 +335,26 @@ dense_halo_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 }
                 rowoff[lane] = off;
             }
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * (Cfg::PARTS * BN);
 #pragma unroll 1
             for (int h = eg; h < BN / 64; h += 2) {
                 uint32_t r[4][16];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + h * 64 + g * 16, r[g]);
-                tmem_wait_ld();
+                if constexpr (Cfg::PARTS == 2) {
+                    // the second partial accumulator, added once in fp32
+                    uint32_t r2[4][16];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(t_row + BN + h * 64 + g * 16, r2[g]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            r[g][c] = __float_as_uint(__fadd_rn(__uint_as_float(r[g][c]), __uint_as_float(r2[g][c])));
+                } else {
+                    tmem_wait_ld();
+                }
                 // stage this warp's 32 rows x 64 channels (128-byte swizzled rows)
                 const uint32_t row_addr = stage + lane * 128;
 #pragma unroll

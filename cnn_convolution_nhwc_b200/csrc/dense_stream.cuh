@@ -89,6 +89,8 @@ template <class Cfg, bool PAIR>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 dense_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmF,
                     __nv_bfloat16 *__restrict__ Y, const DenseStreamParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int BN = Cfg::BN;
     static_assert(!PAIR || BN == 128, "a pair splits the filter slot into two 64-channel boxes");
     constexpr int B_CTA = PAIR ? Cfg::B_BYTES / 2 : Cfg::B_BYTES;   // filter bytes per slot in this CTA

@@ -116,6 +116,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 template <class Cfg, int NG>
 __global__ void __launch_bounds__(192, 1)
 dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int BN = Cfg::BN;
     constexpr int STAGES = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];

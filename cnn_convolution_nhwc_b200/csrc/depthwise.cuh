@@ -95,6 +95,8 @@ template <int MODE, bool HAS_BIAS, int KW_T, int S_T, int VX>
 __global__ void __launch_bounds__(256)
 depthwise_kernel(const float *__restrict__ x, const float *__restrict__ w,
                  const float *__restrict__ bias, float *__restrict__ y, const DwParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     // tensor extents for the bounds-checked debug build
     const long long x_elems = 1LL * (p.num_planes / p.Cout) * p.Cin * p.H * p.W;
     const long long y_elems = 1LL * p.num_planes * p.Ho * p.Wo;

@@ -49,6 +49,8 @@ template <int MODE, bool HAS_BIAS, int K, int S, int HW>
 __global__ void __launch_bounds__(32 * kDwPlaneWarps)
 depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
                        float *__restrict__ y, const DwPlaneParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int PAD = (K - 1) / 2;
     constexpr int HO = (HW + 2 * PAD - K) / S + 1;
     constexpr int WO = HO;

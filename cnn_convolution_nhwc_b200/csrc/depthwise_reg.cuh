@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(256)
 depthwise_reg_kernel(const float *__restrict__ x, const float *__restrict__ w,
                      const float *__restrict__ bias, float *__restrict__ y, const DwRegParams p,
                      unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int VX = 4;                    // outputs per lane along the row
     constexpr int OWN = VX * S;              // input columns a lane loads per row
     constexpr int WIN = (VX - 1) * S + K;    // input columns one lane's outputs read per row

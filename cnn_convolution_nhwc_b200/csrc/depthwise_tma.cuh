@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(32 * kDwWarpsPerCta)
 depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__restrict__ x,
                      const float *__restrict__ w, const float *__restrict__ bias, float *__restrict__ y,
                      const DwTmaParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int PAD = (K - 1) / 2;
     constexpr int VX = 4;
     constexpr int OWN = VX * S;

@@ -86,6 +86,8 @@ template <int MODE, int KC>
 __global__ void __launch_bounds__(kDwPwThreads, 1)
 dwpw_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
             float *__restrict__ y, const DwPwParams p, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     const int K = KC ? KC : p.K;
     constexpr int KK = KC * KC;
     constexpr int KKP = (KK + 3) & ~3;
@@ -451,6 +453,8 @@ template <int MODE, int KC>
 __global__ void __launch_bounds__(kDwPwThreads, 1)
 dwpw_staged_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
                    float *__restrict__ y, const DwPwParams p, const DwPwStage st, unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     constexpr int KK = KC * KC;
     constexpr int KKP = (KK + 3) & ~3;
     extern __shared__ uint8_t smem_raw[];

@@ -149,6 +149,8 @@ __global__ void __launch_bounds__(512, 1)
 dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
                  const __grid_constant__ CUtensorMap tmX, float *__restrict__ y, const DwPwGemmParams p,
                  unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     using G = DwPwGemmGeom<HW>;
     constexpr int PAD = (KC - 1) / 2;
     constexpr int WIN = KC + 1;   // input columns of a two-column strip

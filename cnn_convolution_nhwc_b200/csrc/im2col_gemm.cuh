@@ -28,6 +28,8 @@ struct Im2colParams {
 __global__ void __launch_bounds__(256)
 im2col_pack_kernel(const __nv_bfloat16 *__restrict__ X, __nv_bfloat16 *__restrict__ A, const Im2colParams p,
                    unsigned int *status) {
+    grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
+    grid_dependency_wait();
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     // tensor extents for the bounds-checked debug build
     const long long a_elems = p.chunks * p.chunk;

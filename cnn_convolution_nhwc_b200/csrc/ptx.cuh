@@ -56,6 +56,25 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 }
 
 // ---------------------------------------------------------------------------------------
+// Programmatic dependent launch
+// ---------------------------------------------------------------------------------------
+// Every kernel of the library is launched with programmatic stream serialisation allowed: the
+// next kernel on the stream may be scheduled while this one finishes. A kernel lets its
+// dependents launch as soon as it starts (grid_dependents_launch) and, before its first
+// global-memory access, waits until every kernel it depends on has completed and its memory
+// operations are visible (grid_dependency_wait) -- so a chain of dependent convolutions keeps
+// stream order, and only launch latency and the on-chip prologue (barrier set-up, TMEM
+// allocation, tensor-map prefetch) overlap the previous kernel's tail. Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

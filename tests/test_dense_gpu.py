@@ -240,19 +240,18 @@ def test_unaligned_channels_direct_path(cb, shape):
 
 
 def test_kernel_and_tile_width_choices_agree(cb):
-    # Cin = 64 is one channel block, so the halo kernel at every tile width and the im2col
-    # kernel at width 256 issue the same MMA sequence per output (taps in (i, j) order, 16
-    # channels per step): identical bits. The im2col kernel at widths 64 and 128 sums the
-    # 16-channel steps into two alternating accumulators and adds them in the epilogue, a
-    # different rounding order: those agree with the oracle's bound instead.
+    # Cin = 64 is one channel block, so every kernel and tile width walks the same MMA sequence
+    # per output (taps in (i, j) order, 16 channels per step). At widths 64 and 128 the halo and
+    # im2col kernels alternate those steps between two partial accumulators and add the two in
+    # the epilogue; at width 256 one accumulator takes them all. Within each of the two orders:
+    # identical bits; across them: the oracle's bound.
     Xb, Fb = _case_inputs(4, 24, 24, 64, 256, 3, seed=5)
     ys = {v: _run_bf16(cb, Xb, Fb, env=v) for v in ("halo64", "halo128", "halo256", "bn64", "bn128", "bn256")}
-    _check_bf16(ys["halo64"], Xb, Fb)
     for v, y in ys.items():
-        if v in ("bn64", "bn128"):
-            _check_bf16(y, Xb, Fb)
-        else:
-            assert np.array_equal(y, ys["halo64"]), v
+        _check_bf16(y, Xb, Fb)
+    for v in ("halo128", "bn64", "bn128"):
+        assert np.array_equal(ys[v], ys["halo64"]), v
+    assert np.array_equal(ys["bn256"], ys["halo256"])
     yd = _run_bf16(cb, Xb, Fb, env="direct")
     _check_bf16(yd, Xb, Fb)
 
