@@ -88,6 +88,7 @@ KERNEL_SOURCES = {
     "dense_halo_kernel": ("dense_halo.cuh", "ptx.cuh"),
     "dense_tc_kernel": ("dense_tc.cuh", "ptx.cuh"),
     "dense_stream_kernel": ("dense_stream.cuh", "dense_halo.cuh", "ptx.cuh"),
+    "dense_halo_pad_kernel": ("dense_halo_pad.cuh", "dense_halo.cuh", "ptx.cuh"),
     "dense_direct_kernel": ("dense_direct.cuh",),
     "depthwise_tma_kernel": ("depthwise_tma.cuh", "depthwise.cuh", "ptx.cuh"),
     "depthwise_reg_kernel": ("depthwise_reg.cuh", "depthwise.cuh"),

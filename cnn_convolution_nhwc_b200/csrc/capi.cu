@@ -23,6 +23,7 @@
 #include "dense_halo.cuh"
 #include "dense_fold.cuh"
 #include "dense_stream.cuh"
+#include "dense_halo_pad.cuh"
 #include "im2col_gemm.cuh"
 #include "depthwise.cuh"
 #include "depthwise_reg.cuh"
@@ -1465,6 +1466,115 @@ namespace {
 
 // Validation, dispatch and launch of the general dense convolution (every geometry field of g
 // set; g.plain() operations already routed to the plain entry by the callers).
+// ---- padded halo kernel (stride 1, zero padding, dilation, groups; resident filter) ---------
+struct HaloPadPlan {
+    bool ok = false;
+    int bn = 0;
+    DenseHaloPadParams p{};
+    int smem = 0;
+    int grid = 0;
+};
+
+// Tiles of Rout output rows x Wt columns whose padded input window (Rin x Wbox pixels) is one
+// tensor copy; the window's flattened rows hold the tile's GEMM rows (at most 128 of them) and
+// every tap's reach. Eligible: stride 1, whole 64-channel blocks per group (Cin_g % 64 == 0),
+// Cout_g % 8 == 0, the group's filter slice and two window slots fit in shared memory.
+HaloPadPlan plan_halo_pad(int N, int H, int W, int Cin, int Cout, const DenseGeom &g, int num_sms) {
+    HaloPadPlan pl;
+    const int Cin_g = Cin / g.groups, Cout_g = Cout / g.groups;
+    if (g.sh != 1 || g.sw != 1 || Cin_g % 64 != 0 || Cout_g % 8 != 0) return pl;
+    const long long Ho = g.ho(H), Wo = g.wo(W);
+    if (Ho < 1 || Wo < 1) return pl;
+    const int reach_w = g.dw * (g.KW - 1), reach_h = g.dh * (g.KH - 1);
+    if (reach_w > 96 || reach_h > 127) return pl;
+    const int Wt = static_cast<int>(Wo < 128 - reach_w ? Wo : 128 - reach_w);
+    const int Wbox = Wt + reach_w;
+    int Rout = 128 / Wbox;
+    if (Rout > Ho) Rout = static_cast<int>(Ho);
+    if (Rout < 1) Rout = 1;
+    const int Rin = Rout + reach_h;
+    if (Wbox > 256 || Rin > 256) return pl;
+    const int bn = Cout_g <= 64 ? 64 : 128;
+    const long long reach_rows = 1LL * reach_h * Wbox + reach_w + 128;
+    long long slot_rows = 1LL * Rin * Wbox > reach_rows ? 1LL * Rin * Wbox : reach_rows;
+    slot_rows = (slot_rows + 7) & ~7LL;
+    const long long halo_bytes = slot_rows * 128;
+    const int num_cblk = Cin_g / 64;
+    const int KK = g.KH * g.KW;
+    const long long b_res = 1LL * KK * num_cblk * 64 * bn * 2;
+    const int fixed = bn == 64 ? DenseHaloPadCfg<64>::FIXED_BYTES : DenseHaloPadCfg<128>::FIXED_BYTES;
+    const long long avail = kSmemLimit - fixed - b_res;
+    if (avail < 2 * halo_bytes) return pl;
+    int HS = static_cast<int>(avail / halo_bytes);
+    if (HS > DenseHaloPadCfg<64>::MAX_RING) HS = DenseHaloPadCfg<64>::MAX_RING;
+    const long long n_rb = (Ho + Rout - 1) / Rout, n_cb = (Wo + Wt - 1) / Wt;
+    const long long num_spatial = 1LL * N * n_rb * n_cb;
+    if (num_spatial > kInt32Max) return pl;
+    DenseHaloPadParams &p = pl.p;
+    p.H = H; p.W = W; p.Ho = static_cast<int>(Ho); p.Wo = static_cast<int>(Wo);
+    p.Cout = Cout; p.Cin_g = Cin_g; p.Cout_g = Cout_g;
+    p.KH = g.KH; p.KW = g.KW; p.dh = g.dh; p.dw = g.dw; p.ph = g.ph; p.pw = g.pw;
+    p.Rout = Rout; p.Wt = Wt; p.Wbox = Wbox; p.Rin = Rin;
+    p.n_rb = static_cast<int>(n_rb); p.n_cb = static_cast<int>(n_cb);
+    p.num_spatial = static_cast<int>(num_spatial);
+    p.num_cblk = num_cblk; p.KK = KK; p.num_kblk = KK * num_cblk;
+    p.num_nt = (Cout_g + bn - 1) / bn;
+    p.num_gn = g.groups * p.num_nt;
+    p.box_bytes = Rin * Wbox * 128;
+    p.halo_bytes = static_cast<int>(halo_bytes);
+    p.HS = HS;
+    p.b_region = static_cast<int>(b_res);
+    p.bias = g.bias;
+    p.y_elems = 1LL * N * Ho * Wo * Cout;
+    int per = num_sms / p.num_gn;
+    if (per < 1) per = 1;
+    if (per > p.num_spatial) per = p.num_spatial;
+    pl.grid = per * p.num_gn;
+    pl.smem = fixed + static_cast<int>(b_res) + HS * p.halo_bytes;
+    // more than half of the shared memory keeps a second CTA (and its TMEM allocation) off the SM
+    if (pl.smem < 116 * 1024) pl.smem = 116 * 1024;
+    pl.bn = bn;
+    pl.ok = pl.smem <= kSmemLimit;
+    return pl;
+}
+
+template <class Cfg>
+int launch_dense_halo_pad(const void *X, const void *F, void *Y, int N, int Cin, const HaloPadPlan &pl,
+                          cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
+    const DenseHaloPadParams &p = pl.p;
+    alignas(64) CUtensorMap tmX, tmF;
+    {   // X 4-D {Cin, W, H, N}; a box is 64 channels (128 bytes, 128-byte swizzle) x Wbox columns
+        // x Rin rows of one image; parts outside the image read zeros (the padding)
+        const cuuint64_t dims[4] = {(cuuint64_t)Cin, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)N};
+        const cuuint64_t strides[3] = {(cuuint64_t)Cin * 2, (cuuint64_t)p.W * Cin * 2, (cuuint64_t)p.H * p.W * Cin * 2};
+        const cuuint32_t box[4] = {64, (cuuint32_t)p.Wbox, (cuuint32_t)p.Rin, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (g_encode_tiled(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(X), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    {   // F 3-D {Cout, Cin_g, KH*KW}; a box is 64 reduction rows x 64 output channels
+        const cuuint64_t dims[3] = {(cuuint64_t)p.Cout, (cuuint64_t)p.Cin_g, (cuuint64_t)p.KK};
+        const cuuint64_t strides[2] = {(cuuint64_t)p.Cout * 2, (cuuint64_t)p.Cin_g * p.Cout * 2};
+        const cuuint32_t box[3] = {64, 64, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode_tiled(&tmF, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(F), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONV_ERR_CUDA;
+    }
+    auto kern = dense_halo_pad_kernel<Cfg>;
+    if (int rc = ensure_smem_attr(d, attr_bit, kern, kSmemLimit)) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    return launched(launch_k(cfg, kern, tmX, tmF, static_cast<__nv_bfloat16 *>(Y), p, d->status),
+                    "dense_halo_pad_kernel");
+}
+
 int dense_general(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout,
                   const DenseGeom &g, cudaStream_t stream) {
     const long long Ho = g.ho(H), Wo = g.wo(W);
@@ -1493,6 +1603,17 @@ int dense_general(const void *X, const void *F, void *Y, int N, int H, int W, in
     const bool im2col_ok = tc_shape && axis_ok(g.ph, g.ph_end, g.dh, g.KH) && axis_ok(g.pw, g.pw_end, g.dw, g.KW) &&
                            2LL * N * H * W * Cin >= 128 * 1024;
     const bool force_bn = force && std::strncmp(force, "bn", 2) == 0;
+    // Stride 1 with whole 64-channel blocks per group: the padded halo kernel (each input pixel
+    // of a tile staged once; shared-memory attribute bits 105..106). CONV_B200_DENSE=halo
+    // requires it, bnXX or direct skip it.
+    const bool force_halo = force && std::strcmp(force, "halo") == 0;
+    if (tc_shape && (!g.bias || aligned(g.bias, 16)) && (!force || force_halo)) {
+        const HaloPadPlan hp = plan_halo_pad(N, H, W, Cin, Cout, g, d->num_sms);
+        if (hp.ok)
+            return hp.bn == 64 ? launch_dense_halo_pad<DenseHaloPadCfg<64>>(X, F, Y, N, Cin, hp, stream, d, 105)
+                               : launch_dense_halo_pad<DenseHaloPadCfg<128>>(X, F, Y, N, Cin, hp, stream, d, 106);
+    }
+    if (force_halo) return CONV_ERR_UNSUPPORTED;
     if ((force && std::strcmp(force, "direct") == 0) || !im2col_ok) {
         if (force_bn) return CONV_ERR_UNSUPPORTED;
         return launch_dense_direct(static_cast<const __nv_bfloat16 *>(X), static_cast<const __nv_bfloat16 *>(F),

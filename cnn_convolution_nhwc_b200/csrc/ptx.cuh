@@ -21,7 +21,8 @@ enum : unsigned { kStatusTimeout = 1u, kStatusBounds = 2u };
 enum BoundsSite : unsigned {
     kSiteDirectX = 1, kSiteDirectY, kSiteFoldY, kSiteHaloY, kSiteStreamY, kSiteTcBias, kSiteDwY, kSiteDwRegX,
     kSiteDwRegY, kSiteDwTmaY, kSiteDwPlaneX, kSiteDwPlaneY, kSiteDwPwX, kSiteDwPwY, kSiteDwPwGemmX,
-    kSiteDwPwGemmW, kSiteDwPwGemmY, kSiteIm2colX, kSiteIm2colA, kSiteDwTmaX, kSiteDwX, kSiteSelftest = 255
+    kSiteDwPwGemmW, kSiteDwPwGemmY, kSiteIm2colX, kSiteIm2colA, kSiteDwTmaX, kSiteDwX, kSiteHaloPadBias, kSiteHaloPadY,
+    kSiteSelftest = 255
 };
 #ifdef CONV_DEBUG_BOUNDS
 constexpr bool kDebugBounds = true;

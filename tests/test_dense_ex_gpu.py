@@ -61,7 +61,7 @@ def _check(y, Xb, Fb, b, stride, pad, dil):
 # (N, H, W, Cin, Cout, K, stride, pad, dil, bias, kernel expected by default)
 CASES = [
     (4, 56, 56, 64, 128, 3, 2, 1, 1, True, "dense_tc_kernel"),     # stage transition 56 -> 28
-    (2, 30, 30, 64, 64, 3, 1, 1, 1, True, "dense_tc_kernel"),      # "same" padding with a bias
+    (2, 30, 30, 64, 64, 3, 1, 1, 1, True, "dense_halo_pad_kernel"),   # "same" padding with a bias
     (2, 40, 36, 32, 64, 3, 1, 2, 2, False, "dense_tc_kernel"),     # dilation 2
     (4, 32, 32, 64, 64, 1, 2, 0, 1, True, "dense_tc_kernel"),      # 1x1 stride-2 projection
     (2, 64, 64, 8, 64, 4, 4, 0, 1, True, "dense_tc_kernel"),       # patch projection, K = stride

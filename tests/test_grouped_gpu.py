@@ -67,13 +67,13 @@ def _check(c, y, Xb, Fb, b):
 
 # (N, H, W, Cin, Cout, KH, KW, stride, pad, dil, groups, bias, kernel expected by default)
 CASES = [
-    (4, 28, 28, 128, 128, 3, 3, (1, 1), (1, 1), (1, 1), 2, True, "dense_tc_kernel"),       # two 64-wide groups
+    (4, 28, 28, 128, 128, 3, 3, (1, 1), (1, 1), (1, 1), 2, True, "dense_halo_pad_kernel"),  # two 64-wide groups
     (2, 28, 28, 256, 256, 3, 3, (2, 2), (1, 1), (1, 1), 4, True, "dense_tc_kernel"),       # RegNet-style, stride 2
     (2, 16, 16, 256, 256, 3, 3, (1, 1), (1, 1), (1, 1), 16, False, "dense_tc_kernel"),     # 16 groups: two launches
     (1, 20, 20, 256, 256, 3, 3, (1, 1), (1, 1), (1, 1), 32, True, "dense_tc_kernel"),      # 8-channel groups
     (2, 24, 20, 96, 192, 3, 3, (1, 1), (2, 2), (2, 1), 3, True, "dense_tc_kernel"),        # dilation per axis, ragged N tile
-    (4, 17, 17, 64, 64, 1, 7, (1, 1), (0, 3), (1, 1), 1, True, "dense_tc_kernel"),         # 1x7, one group
-    (4, 17, 17, 64, 96, 7, 1, (1, 1), (3, 0), (1, 1), 1, False, "dense_tc_kernel"),        # 7x1
+    (4, 17, 17, 64, 64, 1, 7, (1, 1), (0, 3), (1, 1), 1, True, "dense_halo_pad_kernel"),   # 1x7, one group
+    (4, 17, 17, 64, 96, 7, 1, (1, 1), (3, 0), (1, 1), 1, False, "dense_halo_pad_kernel"),  # 7x1
     (4, 30, 30, 64, 64, 3, 1, (2, 1), (1, 0), (1, 1), 1, True, "dense_tc_kernel"),         # stride per axis
     (2, 1, 3000, 80, 512, 1, 3, (1, 1), (0, 1), (1, 1), 1, True, "dense_tc_kernel"),      # Conv1D, 80 channels
     (2, 1, 3000, 256, 256, 1, 3, (1, 2), (0, 1), (1, 1), 1, True, "dense_tc_kernel"),     # Conv1D, stride 2
@@ -112,6 +112,47 @@ def test_tensor_core_and_direct_paths_agree(cb, case):
     _check(c, y_cc, Xb, Fb, b)
 
 
+# Stride 1 with whole 64-channel blocks per group: the padded halo kernel by default (one 4-D
+# tensor copy of a zero-padded window per tile), the im2col kernel when forced; both against the
+# oracle. Two 64-wide groups with a bias; one group with "same" padding; dilation 2; an image
+# wider than one window (three column bands); 40-wide groups (a partial bias chunk, a partial
+# column tile); 128-wide groups (two 64-column boxes per filter slot); a 1 x 5 Conv1D
+PAD_HALO = [   # inputs of at least 128 KiB, so that the im2col kernel can be forced for comparison
+    (2, 20, 20, 128, 128, 3, 3, (1, 1), (1, 1), (1, 1), 2, True),
+    (2, 30, 30, 64, 64, 3, 3, (1, 1), (1, 1), (1, 1), 1, True),
+    (3, 24, 20, 64, 64, 3, 3, (1, 1), (2, 2), (2, 2), 1, False),
+    (1, 4, 300, 64, 64, 3, 3, (1, 1), (1, 1), (1, 1), 1, True),
+    (4, 14, 14, 128, 80, 3, 3, (1, 1), (1, 1), (1, 1), 2, True),
+    (4, 12, 12, 128, 256, 3, 3, (1, 1), (1, 1), (1, 1), 2, True),
+    (2, 1, 700, 64, 64, 1, 5, (1, 1), (0, 2), (1, 1), 1, True),
+]
+
+
+@pytest.mark.parametrize("case", PAD_HALO, ids=_ids)
+def test_padded_halo_kernel(cb, case):
+    N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias = case
+    c = _case(N, H, W, Cin, Cout, KH, KW, s, p, d, groups, bias, seed=sum(case[:7]) + 13)
+    Xb, Fb = workloads.dense_inputs(c)
+    b = workloads.dense_bias(c)
+    y, kernel = _run(cb, c, Xb, Fb, b)
+    assert kernel == "dense_halo_pad_kernel"
+    _check(c, y, Xb, Fb, b)
+    y2, kernel2 = _run(cb, c, Xb, Fb, b, env="bn128")
+    assert kernel2 == "dense_tc_kernel"
+    _check(c, y2, Xb, Fb, b)
+    y3, kernel3 = _run(cb, c, Xb, Fb, b, env="halo")
+    assert kernel3 == "dense_halo_pad_kernel" and np.array_equal(y3, y)
+
+
+def test_padded_halo_refuses_what_it_cannot_do(cb):
+    # forced onto a shape it does not take (32-channel groups): CONV_ERR_UNSUPPORTED
+    c = _case(2, 16, 16, 64, 64, 3, 3, (1, 1), (1, 1), (1, 1), 2, False, seed=1)
+    Xb, Fb = workloads.dense_inputs(c)
+    with pytest.raises(cb.ConvError) as e:
+        _run(cb, c, Xb, Fb, None, env="halo")
+    assert e.value.code == cb.CONV_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("bn", ["bn64", "bn128", "bn256"])
 def test_grouped_tile_widths(cb, bn):
     c = _case(2, 20, 20, 384, 384, 3, 3, (1, 1), (1, 1), (1, 1), 2, True, seed=8)   # 192-wide groups
@@ -140,12 +181,14 @@ def test_groups_do_not_mix(cb):
     Xb, Fb = workloads.dense_inputs(c)
     Xb = Xb.copy()
     Xb[..., 64:] = np.uint16(0x7FC0)   # bf16 quiet NaN
-    y, kernel = _run(cb, c, Xb, Fb, None)
-    assert kernel == "dense_tc_kernel"
-    assert np.all(np.isnan(y[..., 64:]))
     ref, absum = oracle.conv2d_grouped(workloads.bf16_to_f32(Xb[..., :64]), workloads.bf16_to_f32(Fb[..., :64]), None,
                                        1, 1, 1, 1)
-    assert np.all(np.abs(y[..., :64] - ref) <= TOL * absum)
+    # the padded halo kernel (default here) and the im2col kernel (forced)
+    for env, name in ((None, "dense_halo_pad_kernel"), ("bn64", "dense_tc_kernel")):
+        y, kernel = _run(cb, c, Xb, Fb, None, env=env)
+        assert kernel == name
+        assert np.all(np.isnan(y[..., 64:]))
+        assert np.all(np.abs(y[..., :64] - ref) <= TOL * absum)
 
 
 def test_page_two_filters_with_bias_as_conv1d(cb):
@@ -164,24 +207,29 @@ def test_page_two_filters_with_bias_as_conv1d(cb):
     assert np.array_equal(y[0, 0, :, 0], [0, 1, 2]) and np.array_equal(y[0, 0, :, 1], [6, 9, 12])
 
 
-FULL_SIZE = [workloads.DENSE_GROUPED, workloads.CONV1D_STEM1, workloads.CONV1D_STEM2, workloads.CONV1D_CAUSAL]
+# the benchmark's workloads and the kernel the dispatcher gives each (the grouped 3x3 runs the
+# padded halo kernel; the Conv1D layers have 80 channels, a stride or a filter too large to stay
+# resident, and run the im2col kernel)
+FULL_SIZE = [(workloads.DENSE_GROUPED, "dense_halo_pad_kernel"), (workloads.CONV1D_STEM1, "dense_tc_kernel"),
+             (workloads.CONV1D_STEM2, "dense_tc_kernel"), (workloads.CONV1D_CAUSAL, "dense_tc_kernel")]
 
 
 @pytest.mark.parametrize("case", FULL_SIZE, ids=["grouped", "conv1d-stem1", "conv1d-stem2", "conv1d-causal"])
 def test_full_size_workloads(cb, case):
     # the benchmark's workloads at full size, every output compared with the oracle
+    case, expected = case
     Xb, Fb = workloads.dense_inputs(case)
     b = workloads.dense_bias(case)
     y, kernel = _run(cb, case, Xb, Fb, b)
-    assert kernel == "dense_tc_kernel"
     _check(case, y, Xb, Fb, b)
+    assert kernel == expected
 
 
 # Causal Conv1D ("Convolution Is Wx+b Moving Across a Signal", section "Find the same sum in CKE's
 # C kernels": a frame's output reads no later frame): zero padding of dil*(K-1) frames before the
 # sequence and none after it.
 # (N, L, Cin, Cout, K, dil, groups, bias, kernel expected)
-CAUSAL = [(2, 1000, 64, 128, 3, 1, 1, True, "dense_tc_kernel"),
+CAUSAL = [(2, 1000, 64, 128, 3, 1, 1, True, "dense_halo_pad_kernel"),
           (2, 777, 128, 64, 5, 2, 4, True, "dense_tc_kernel"),     # dilated, grouped, ragged length
           (3, 50, 12, 8, 3, 1, 1, False, "dense_direct_kernel")]   # channel counts for the CUDA cores
 
