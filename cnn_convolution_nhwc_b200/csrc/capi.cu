@@ -317,7 +317,7 @@ int launch_dense_direct(const T *X, const T *F, T *Y, int N, int H, int W, int C
 // there is one group). Per group: X channels g*Cin_g .. +Cin_g, filter and Y columns
 // g*Cout_g .. +Cout_g; the caller guarantees Cin_g and Cout_g multiples of 8 (16-byte map
 // bases) and window corners and tap reaches inside the 4-D im2col ranges.
-template <class Cfg, int NG>
+template <class Cfg, int NG, bool PAIR = false>
 int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, int Cin, int Cout,
                     const DenseGeom &g, cudaStream_t stream, DeviceState *d, unsigned attr_bit) {
     const int Ho = static_cast<int>(g.ho(H)), Wo = static_cast<int>(g.wo(W));
@@ -333,11 +333,13 @@ int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, 
     p.num_kblk = g.KH * g.KW * p.num_cblk;
     p.num_ntiles = (Cout_g + Cfg::BN - 1) / Cfg::BN;
     p.sh = g.sh; p.sw = g.sw; p.ph = g.ph; p.pw = g.pw; p.dh = g.dh; p.dw = g.dw;
-    const long long per_group = ((M + Cfg::BM - 1) / Cfg::BM) * p.num_ntiles;
+    constexpr int TILE_ROWS = PAIR ? 2 * Cfg::BM : Cfg::BM;   // a CTA pair computes 256 rows per tile
+    constexpr int SMEM = PAIR ? Cfg::SMEM_BYTES_PAIR : Cfg::SMEM_BYTES;
+    const long long per_group = ((M + TILE_ROWS - 1) / TILE_ROWS) * p.num_ntiles;
     if (per_group * NG > kInt32Max) return CONV_ERR_UNSUPPORTED;
     p.tiles_per_group = static_cast<int>(per_group);
-    auto kern = dense_tc_kernel<Cfg, NG>;
-    if (int rc = ensure_smem_attr(d, attr_bit, kern, Cfg::SMEM_BYTES)) return rc;
+    auto kern = dense_tc_kernel<Cfg, NG, PAIR>;
+    if (int rc = ensure_smem_attr(d, attr_bit, kern, SMEM)) return rc;
     const auto *xb = static_cast<const __nv_bfloat16 *>(X);
     const auto *fb = static_cast<const __nv_bfloat16 *>(F);
     auto *yb = static_cast<__nv_bfloat16 *>(Y);
@@ -393,8 +395,22 @@ int launch_dense_tc(const void *X, const void *F, void *Y, int N, int H, int W, 
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(p.num_tiles < d->num_sms ? p.num_tiles : d->num_sms));
         cfg.blockDim = dim3(192);
-        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cfg.dynamicSmemBytes = SMEM;
         cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        if (PAIR) {
+            // 2-CTA clusters, no more than the device holds at once (the grid is persistent)
+            const int fit = cluster_fit(d, attr_bit, kern, 2, SMEM, 192);
+            if (fit < 1) return CONV_ERR_CUDA;
+            const int pairs = p.num_tiles < fit ? p.num_tiles : fit;
+            cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+        }
         if (int rc = launched(launch_k(cfg, kern, maps, p, d->status), "dense_tc_kernel")) return rc;
     }
     return CONV_OK;
@@ -1276,6 +1292,16 @@ int launch_dwpw_staged(const float *x, const float *w, const CUtensorMap &tmF, f
     return launched(launch_k(cfg, kern, x, w, tmF, y, p, pl.st, d->status), "dwpw_staged_kernel");
 }
 
+// Whether the im2col kernel runs as CTA pairs: by default for 256-column tiles whose reduction
+// is at least 16 blocks of 64 channels; CONV_B200_TC_PAIR=1 / 0 forces it on / off (tile
+// widths of 128 and 256).
+bool tc_pair_choice(int bn, int num_kblk, int num_sms) {
+    if (bn < 128 || num_sms < 2) return false;
+    const int forced = env_int("CONV_B200_TC_PAIR", -1, -1, 1);
+    if (forced >= 0) return forced == 1;
+    return bn == 256 && num_kblk >= 16;
+}
+
 // Output-channel tile width of the im2col kernel: 64 for narrow groups; 256 for groups of at
 // least 256 output channels while the tiles still cover every SM (measured on B200: the wider
 // tile halves the A-operand traffic per MMA, e.g. a 3-tap 512 -> 512 Conv1D over 48000
@@ -1343,8 +1369,16 @@ int dense_plain(const void *X, const void *F, void *Y, int N, int H, int W, int 
     }
     int bn = force_bn ? force_bn : im2col_bn(1LL * N * sq.ho(H) * sq.wo(W), Cout, 1, d->num_sms);
     if (bn == 64) return launch_dense_tc<CfgBN64, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 0);
-    if (bn == 128) return launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 1);
-    return launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 2);
+    // 256-wide tiles with long reductions run as CTA pairs (each CTA stages half of every B slot:
+    // measured on B200, a 3-tap 512-channel causal Conv1D 76 -> 70 us; with a 6-block reduction
+    // the pair's hand-offs cost more than they save). CONV_B200_TC_PAIR=1 / 0 forces pairs on /
+    // off for tiles of at least 128 columns. Shared-memory attribute bits 107..108.
+    const bool tc_pair = tc_pair_choice(bn, K * K * ((Cin + 63) / 64), d->num_sms);
+    if (bn == 128)
+        return tc_pair ? launch_dense_tc<CfgBN128, 1, true>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 107)
+                       : launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 1);
+    return tc_pair ? launch_dense_tc<CfgBN256, 1, true>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 108)
+                   : launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, sq, stream, d, 2);
 }
 
 // ---- fused depthwise -> pointwise, transposed GEMM (7x7 and 14x14 images) --------------------
@@ -1623,8 +1657,13 @@ int dense_general(const void *X, const void *F, void *Y, int N, int H, int W, in
     if (force_bn) bn = std::atoi(force + 2);
     if (g.groups == 1) {
         if (bn == 64) return launch_dense_tc<CfgBN64, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 0);
-        if (bn == 128) return launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 1);
-        if (bn == 256) return launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 2);
+        const bool tc_pair = tc_pair_choice(bn, g.KH * g.KW * ((Cin_g + 63) / 64), d->num_sms);
+        if (bn == 128)
+            return tc_pair ? launch_dense_tc<CfgBN128, 1, true>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 107)
+                           : launch_dense_tc<CfgBN128, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 1);
+        if (bn == 256)
+            return tc_pair ? launch_dense_tc<CfgBN256, 1, true>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 108)
+                           : launch_dense_tc<CfgBN256, 1>(X, F, Y, N, H, W, Cin, Cout, g, stream, d, 2);
         return CONV_ERR_INVALID_ARG;
     }
     // several groups: up to kTcGroups per launch (shared-memory attribute bits 48..50)

@@ -95,6 +95,9 @@ struct DenseTcCfg {
     static constexpr int TMEM_COLS = 2 * PARTS * BN;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ true);
+    static constexpr uint32_t IDESC_PAIR = idesc_bf16_f32(2 * BM, BN, /*B MN-major*/ true);   // cta_group::2
+    // shared memory of the CTA-pair form: each CTA stages its A tile and half of every B slot
+    static constexpr int SMEM_BYTES_PAIR = 1024 + STAGES * (A_BYTES + B_BYTES / 2) + EPI_BYTES + NUM_BARS * 8 + 16;
     static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
     static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM columns");
     static constexpr uint32_t A_UNITS = A_BYTES >> 4;   // descriptor address field per A slot
@@ -113,13 +116,22 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-template <class Cfg, int NG>
+// PAIR (one group, BN >= 128): 2-CTA clusters; each CTA stages the A tile of its own 128 rows
+// and half of every B slot (its BN/2 output channels); the even CTA issues M = 256 MMAs
+// (cta_group::2) that read both CTAs' operands and commit to both CTAs' barriers -- the B bytes
+// each SM stages per MMA halve. Its full barriers count both CTAs' bytes; its
+// accumulator-empty barriers both CTAs' epilogue warps.
+template <class Cfg, int NG, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
 dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParams p, unsigned int *status) {
     grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
     grid_dependency_wait();
     constexpr int BN = Cfg::BN;
     constexpr int STAGES = Cfg::STAGES;
+    static_assert(!PAIR || (NG == 1 && BN >= 128), "pairs: one group, at least two 64-channel boxes");
+    constexpr int B_CTA = PAIR ? Cfg::B_BYTES / 2 : Cfg::B_BYTES;   // B bytes per slot in this CTA
+    constexpr int STAGE_CTA = Cfg::A_BYTES + B_CTA;
+    constexpr int TILE_ROWS = PAIR ? 2 * Cfg::BM : Cfg::BM;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;   // 1024-B alignment for the swizzle
@@ -127,19 +139,21 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
 
     const uint32_t sA = base;
     const uint32_t sB = base + STAGES * Cfg::A_BYTES;
-    uint8_t *sEpi = smem + STAGES * Cfg::STAGE_BYTES;
-    const uint32_t bars = base + STAGES * Cfg::STAGE_BYTES + Cfg::EPI_BYTES;
+    uint8_t *sEpi = smem + STAGES * STAGE_CTA;
+    const uint32_t bars = base + STAGES * STAGE_CTA + Cfg::EPI_BYTES;
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
     auto accf_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
     auto acce_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
     const uint32_t done_bar = bars + 8u * (2 * STAGES + 4);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + STAGES * Cfg::STAGE_BYTES +
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + STAGES * STAGE_CTA +
                                                          Cfg::EPI_BYTES + Cfg::NUM_BARS * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;
+    auto lead = [&](uint32_t a) { return PAIR ? map_rank(a, 0u) : a; };   // the even CTA's barrier
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -148,7 +162,7 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf_bar(b), 1);
-            mbar_init(acce_bar(b), 4);   // one arrival per epilogue warp
+            mbar_init(acce_bar(b), PAIR ? 8 : 4);   // one arrival per epilogue warp (of both CTAs)
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -160,18 +174,27 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
         }
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_holder), Cfg::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_holder), Cfg::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // both CTAs' barriers and TMEM exist before either is used
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
     auto fail = [&]() {
         atomicOr(status, kStatusTimeout);
         *abort_flag = 1;
+        if constexpr (PAIR) st_cluster_u32(map_rank(smem_u32(const_cast<int *>(abort_flag)), rank ^ 1u), 1u);
     };
+    const int first = static_cast<int>(PAIR ? blockIdx.x >> 1 : blockIdx.x);
+    const int step = static_cast<int>(PAIR ? gridDim.x >> 1 : gridDim.x);
     // tile -> (group of this launch, 128-row block, BN-column block)
     auto split = [&](int tile, int &grp, int &mt, int &nt) {
         grp = NG == 1 ? 0 : tile / p.tiles_per_group;
@@ -184,12 +207,12 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
         // ------------------------------- TMA producer -------------------------------
         // The whole warp walks the loop (it stays converged); lane 0 issues.
         uint32_t it = 0, s = 0, ph = 0;   // ring slot and phase as running counters
-        for (int tile = blockIdx.x; tile < p.num_tiles && !*abort_flag; tile += gridDim.x) {
+        for (int tile = first; tile < p.num_tiles && !*abort_flag; tile += step) {
             int grp, mt, nt;
             split(tile, grp, mt, nt);
             const CUtensorMap *tmX = &maps.x[grp];
             const CUtensorMap *tmF = &maps.f[grp];
-            const int m0 = mt * Cfg::BM;
+            const int m0 = mt * TILE_ROWS + static_cast<int>(rank) * Cfg::BM;   // this CTA's rows
             const int n0 = nt * BN;
             const int img = m0 / p.HoWo;
             const int rem = m0 - img * p.HoWo;
@@ -204,14 +227,26 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                     break;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(full_bar(s), Cfg::STAGE_BYTES);
-                    tma_load_im2col_4d(sA + s * Cfg::A_BYTES, tmX, full_bar(s), cb * 64, ox * p.sw - p.pw,
-                                       oy * p.sh - p.ph, img, static_cast<uint16_t>(kx * p.dw),
-                                       static_cast<uint16_t>(ky * p.dh));
+                    if constexpr (PAIR) {
+                        // both CTAs' A tiles and B halves complete on the even CTA's barrier
+                        if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * Cfg::A_BYTES + Cfg::B_BYTES);
+                        tma_load_im2col_4d_pair(sA + s * Cfg::A_BYTES, tmX, lead(full_bar(s)), cb * 64,
+                                                ox * p.sw - p.pw, oy * p.sh - p.ph, img,
+                                                static_cast<uint16_t>(kx * p.dw), static_cast<uint16_t>(ky * p.dh));
 #pragma unroll
-                    for (int h = 0; h < BN / 64; ++h)
-                        tma_load_3d(sB + s * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, tmF, full_bar(s),
-                                    n0 + h * 64, cb * 64, tap);
+                        for (int h = 0; h < BN / 128; ++h)
+                            tma_load_3d_pair(sB + s * B_CTA + h * Cfg::B_BOX_BYTES, tmF, lead(full_bar(s)),
+                                             n0 + static_cast<int>(rank) * (BN / 2) + h * 64, cb * 64, tap);
+                    } else {
+                        mbar_arrive_expect_tx(full_bar(s), Cfg::STAGE_BYTES);
+                        tma_load_im2col_4d(sA + s * Cfg::A_BYTES, tmX, full_bar(s), cb * 64, ox * p.sw - p.pw,
+                                           oy * p.sh - p.ph, img, static_cast<uint16_t>(kx * p.dw),
+                                           static_cast<uint16_t>(ky * p.dh));
+#pragma unroll
+                        for (int h = 0; h < BN / 64; ++h)
+                            tma_load_3d(sB + s * Cfg::B_BYTES + h * Cfg::B_BOX_BYTES, tmF, full_bar(s),
+                                        n0 + h * 64, cb * 64, tap);
+                    }
                 }
                 __syncwarp();
                 // next (tap, channel block) in (i, j, c) order
@@ -224,13 +259,17 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
             }
             if (!ok) break;
         }
-        // Drain: every load issued has landed before the CTA may exit.
-        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
-        for (uint32_t j = first; j < it; ++j)
-            if (!mbar_wait_warp(full_bar(j % STAGES), (j / STAGES) & 1u)) {
+        // Drain: every load issued has landed before the CTA may exit (in a pair: has been
+        // consumed by the pair's MMAs, which the even CTA's commits report to both CTAs).
+        const uint32_t j0 = it > (uint32_t)STAGES ? it - STAGES : 0u;
+        for (uint32_t j = j0; j < it; ++j) {
+            const bool landed = PAIR ? mbar_wait_warp(empty_bar(j % STAGES), (j / STAGES) & 1u)
+                                     : mbar_wait_warp(full_bar(j % STAGES), (j / STAGES) & 1u);
+            if (!landed) {
                 if (lane == 0) fail();
                 break;
             }
+        }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
         // The whole warp walks the loop, converged; the MMAs and commits are predicated on one
@@ -241,11 +280,18 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
         // apart. B: MN-major, +128 per 16 reduction rows (2048 B), 8-row groups 1024 B apart
         // (SBO), 64-channel boxes B_BOX_BYTES apart (LBO).
         const uint32_t leader = elect_one_sync();
+        constexpr uint16_t kBoth = 0x3;
+        auto commit = [&](uint32_t bar) {
+            if constexpr (PAIR) umma_commit_pair_if(bar, kBoth, leader);
+            else umma_commit_if(bar, leader);
+        };
         const uint64_t a_desc0 = smem_desc_sw128(sA, 16, 1024);
         const uint64_t b_desc0 = smem_desc_sw128(sB, Cfg::B_BOX_BYTES, 1024);
+        constexpr uint32_t kBUnits = B_CTA >> 4;
         uint32_t it = 0, local = 0, s = 0, ph = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles && !__any_sync(0xffffffffu, *abort_flag != 0);
-             tile += gridDim.x, ++local) {
+        // in a pair only the even CTA's MMA warp walks the tiles
+        for (int tile = first; rank == 0 && tile < p.num_tiles && !__any_sync(0xffffffffu, *abort_flag != 0);
+             tile += step, ++local) {
             const uint32_t b = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
             // waiting here means the epilogue is the slower role: sleep between polls instead
@@ -265,31 +311,38 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                 }
                 tc_fence_after();
                 const uint64_t ad = a_desc0 + s * Cfg::A_UNITS;
-                const uint64_t bd = b_desc0 + s * Cfg::B_UNITS;
+                const uint64_t bd = b_desc0 + s * kBUnits;
 #pragma unroll
                 for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
                     const uint32_t part = Cfg::PARTS == 2 ? (kk & 1) : 0;
                     // the first MMA into each partial accumulator of the tile overwrites it
                     const uint32_t acc = (kb != 0 || kk >= Cfg::PARTS) ? 1u : 0u;
-                    umma_f16_ss_if(d_tmem + part * BN, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC, acc, leader);
+                    if constexpr (PAIR)
+                        umma_f16_ss_pair_if(d_tmem + part * BN, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC_PAIR, acc,
+                                            leader);
+                    else
+                        umma_f16_ss_if(d_tmem + part * BN, ad + 2 * kk, bd + 128 * kk, Cfg::IDESC, acc, leader);
                 }
-                umma_commit_if(empty_bar(s), leader);
+                commit(empty_bar(s));
                 if (++s == static_cast<uint32_t>(STAGES)) { s = 0; ph ^= 1u; }
             }
             if (!ok) break;
-            umma_commit_if(accf_bar(b), leader);
+            commit(accf_bar(b));
         }
         __syncwarp();
-        // All MMAs issued by this warp complete before TMEM is released.
-        umma_commit_if(done_bar, leader);
-        if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
+        // All MMAs issued by this warp complete before TMEM is released (in a pair: before the
+        // cluster barrier both CTAs pass ahead of their deallocation).
+        if (rank == 0) {
+            commit(done_bar);
+            if (!mbar_wait_warp(done_bar, 0) && lane == 0) fail();
+        }
     } else {
         // ------------------------------- Epilogue -----------------------------------
         const int q = warp & 3;   // TMEM lane quarter this warp may access
         uint8_t *stage = sEpi + q * Cfg::EPI_WARP_BYTES;
         const uint32_t stage_s = smem_u32(stage);
         uint32_t local = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+        for (int tile = first; tile < p.num_tiles; tile += step, ++local) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const uint32_t b = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
@@ -298,7 +351,7 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
             tc_fence_after();
             int grp, mt, nt;
             split(tile, grp, mt, nt);
-            const int m0 = mt * Cfg::BM;
+            const int m0 = mt * TILE_ROWS + static_cast<int>(rank) * Cfg::BM;
             const int n0 = nt * BN;
             // the staging buffer is free once the previous tile's stores have read it
             if (lane == 0) bulk_wait_group_read0();
@@ -351,10 +404,13 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
                     }
                 }
             }
-            // accumulator b may now be overwritten by the MMA warp
+            // accumulator b may now be overwritten by the MMA warp (of the even CTA)
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce_bar(b));
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster(lead(acce_bar(b)));
+                else mbar_arrive(acce_bar(b));
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -373,8 +429,13 @@ dense_tc_kernel(const __grid_constant__ DenseTcMaps<NG> maps, const DenseTcParam
 
     tc_fence_before();
     __syncthreads();
+    // neither CTA of a pair leaves while the other may still signal its barriers
+    if constexpr (PAIR) cluster_sync_all();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    if (warp == 1) {
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+        else tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
 }
 
 }  // namespace convb200

@@ -144,6 +144,35 @@ def test_padded_halo_kernel(cb, case):
     assert kernel3 == "dense_halo_pad_kernel" and np.array_equal(y3, y)
 
 
+# The im2col kernel at tile widths 128 and 256 can run as CTA pairs (each CTA stages half of
+# every filter slot; M = 256 MMAs across both; forced here): the same MMA sequence per output as
+# one CTA per tile, so identical bits. Stride 2 with 128-wide tiles; a causal Conv1D with 256-wide tiles and a
+# ragged last pair (the odd CTA's rows past the end); a dilated 5x5
+TC_PAIR = [
+    ((2, 28, 28, 64, 128, 3, 3, (2, 2), (1, 1), (1, 1), 1, True), "bn128"),
+    ((2, 1, 999, 256, 512, 1, 3, (1, 1), (0, 2), (1, 1), 1, True), "bn256"),
+    ((2, 24, 24, 96, 256, 5, 5, (1, 1), (4, 4), (2, 2), 1, False), "bn256"),
+]
+
+
+@pytest.mark.parametrize("case", TC_PAIR, ids=lambda c: _ids(c[0]) + c[1])
+def test_im2col_pairs_match_single_ctas(cb, case, monkeypatch):
+    geom, bn = case
+    N, H, W, Cin, Cout, KH, KW, s_, p_, d_, groups, bias = geom
+    # the Conv1D case (KH = 1) is causal: padding before the sequence only
+    c = _case(N, H, W, Cin, Cout, KH, KW, s_, p_, d_, groups, bias, seed=sum(geom[:7]) + 29,
+              **({} if KH > 1 else {"pad_w_end": 0}))
+    Xb, Fb = workloads.dense_inputs(c)
+    b = workloads.dense_bias(c)
+    monkeypatch.setenv("CONV_B200_TC_PAIR", "1")
+    y_pair, k1 = _run(cb, c, Xb, Fb, b, env=bn)
+    monkeypatch.setenv("CONV_B200_TC_PAIR", "0")
+    y_one, k2 = _run(cb, c, Xb, Fb, b, env=bn)
+    assert k1 == k2 == "dense_tc_kernel"
+    _check(c, y_pair, Xb, Fb, b)
+    assert np.array_equal(y_pair, y_one)
+
+
 def test_padded_halo_refuses_what_it_cannot_do(cb):
     # forced onto a shape it does not take (32-channel groups): CONV_ERR_UNSUPPORTED
     c = _case(2, 16, 16, 64, 64, 3, 3, (1, 1), (1, 1), (1, 1), 2, False, seed=1)
