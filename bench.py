@@ -610,7 +610,7 @@ def run_ours(args, dist):
         "clocks": sampler.summary(),
         "device_status": cb.conv_status_string(status),
     }
-    if dist.rank == 0 and dist.world == 1:
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(kind, case, mode, host_np)
     if dist.world == 1 and not args.no_extras:
         # last, so that the end of the line (what a log tail keeps) holds every row
@@ -724,6 +724,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workload_table()))
     ap.add_argument("--no-extras", action="store_true")
+    # profiling runs (ncu captures of one workload) skip the seconds-long CPU oracle sample
+    ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
