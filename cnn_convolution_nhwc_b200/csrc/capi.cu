@@ -1389,10 +1389,9 @@ bool dwpw_gemm_eligible(int C, int H, int W, int K, int stride, int pad, int dil
            C % 4 == 0 && Cout <= 256 && aligned(x, 16) && aligned(w, 16) && aligned(y, 16);
 }
 
-template <int MODE, int KC, int HW>
+template <int MODE, int KC, class G>
 int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, const void *F, const float *b_pw, float *y,
                          int N, int C, int Cout, cudaStream_t stream, DeviceState *d, unsigned bit) {
-    using G = DwPwGemmGeom<HW>;
     DwPwGemmParams p;
     p.C = C;
     p.Cout = Cout;
@@ -1407,9 +1406,10 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
     p.b_pw = b_pw;
     // a 2-CTA cluster per image (every other channel block each) when there are two blocks and
     // its receive area fits; CONV_B200_DWPW_SPLIT=1 keeps one CTA per image (tests)
-    const int want = env_int("CONV_B200_DWPW_SPLIT", 2, 1, 2);
-    p.S = (want == 2 && p.nblk >= 2 && dwpw_gemm_smem<HW>(p.fslot, p.MT, 2, KC * KC) <= kSmemLimit) ? 2 : 1;
-    const int smem = dwpw_gemm_smem<HW>(p.fslot, p.MT, p.S, KC * KC);
+    // (the pixel-split form: two CTAs per image without a cluster, S = 1)
+    const int want = G::HALF ? 1 : env_int("CONV_B200_DWPW_SPLIT", 2, 1, 2);
+    p.S = (want == 2 && p.nblk >= 2 && dwpw_gemm_smem<G>(p.fslot, p.MT, 2, KC * KC) <= kSmemLimit) ? 2 : 1;
+    const int smem = dwpw_gemm_smem<G>(p.fslot, p.MT, p.S, KC * KC);
     if (smem > kSmemLimit || p.tmem_cols > 512) return CONV_ERR_UNSUPPORTED;
     alignas(64) CUtensorMap tmF;
     {   // F: 2-D {Cout, C}; a box is 64 output columns x CB channel rows (columns past Cout and
@@ -1424,7 +1424,7 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
             return CONV_ERR_CUDA;
     }
     alignas(64) CUtensorMap tmX = tmF;   // unused by the 7x7 form (contiguous bulk copies)
-    if (G::PADX) {   // x as [N*C][P] fp32; a box of XP > P columns (the overhang reads zeros) x CB planes
+    if (G::PADX) {   // x as [N*C][P] fp32; a box of XP columns (past P it reads zeros) x CB planes
         const cuuint64_t dims[2] = {(cuuint64_t)G::P, (cuuint64_t)N * C};
         const cuuint64_t strides[1] = {(cuuint64_t)G::P * 4};
         const cuuint32_t box[2] = {(cuuint32_t)G::XP, (cuuint32_t)G::CB};
@@ -1434,15 +1434,16 @@ int launch_dwpw_gemm_one(const float *x, const float *w, const float *b_dw, cons
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CONV_ERR_CUDA;
     }
-    auto kern = dwpw_gemm_kernel<MODE, KC, HW>;
+    auto kern = dwpw_gemm_kernel<MODE, KC, G>;
     if (int rc = ensure_smem_attr(d, bit, kern, kSmemLimit)) return rc;
-    int clusters_max = d->num_sms / p.S;
+    const int per = G::HALF ? 2 : p.S;   // CTAs per image
+    int clusters_max = d->num_sms / per;
     if (p.S > 1) clusters_max = cluster_fit(d, bit, kern, p.S, smem, G::THREADS);
     if (clusters_max < 1) return CONV_ERR_CUDA;
     const int clusters = N < clusters_max ? N : clusters_max;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S));
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * per));
     cfg.blockDim = dim3(G::THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -1461,11 +1462,24 @@ template <int MODE>
 int launch_dwpw_gemm(const float *x, const float *w, const float *b_dw, const void *F, const float *b_pw, float *y,
                      int N, int C, int H, int K, int Cout, cudaStream_t stream, DeviceState *d) {
     const unsigned b = 96u + 4u * MODE;
+    using G7 = DwPwGemmGeom<7>;
+    using G14 = DwPwGemmGeom<14>;
+    using G14H3 = DwPwGemmGeom<14, true, 3>;
+    using G14H5 = DwPwGemmGeom<14, true, 5>;
     if (H == 7)
-        return K == 3 ? launch_dwpw_gemm_one<MODE, 3, 7>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 0)
-                      : launch_dwpw_gemm_one<MODE, 5, 7>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 1);
-    return K == 3 ? launch_dwpw_gemm_one<MODE, 3, 14>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 2)
-                  : launch_dwpw_gemm_one<MODE, 5, 14>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 3);
+        return K == 3 ? launch_dwpw_gemm_one<MODE, 3, G7>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 0)
+                      : launch_dwpw_gemm_one<MODE, 5, G7>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 1);
+    // 14x14: the row split (each CTA half of the rows, all channels; shared-memory attribute
+    // bits 109..112) unless CONV_B200_DWPW_HALF=0 asks for the channel-split cluster, or its
+    // rings do not fit (5x5 taps with more than 128 outputs)
+    if (env_int("CONV_B200_DWPW_HALF", 1, 0, 1) == 1) {
+        const unsigned bh = 109u + 2u * MODE;
+        const int rc = K == 3 ? launch_dwpw_gemm_one<MODE, 3, G14H3>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, bh + 0)
+                              : launch_dwpw_gemm_one<MODE, 5, G14H5>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, bh + 1);
+        if (rc != CONV_ERR_UNSUPPORTED) return rc;
+    }
+    return K == 3 ? launch_dwpw_gemm_one<MODE, 3, G14>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 2)
+                  : launch_dwpw_gemm_one<MODE, 5, G14>(x, w, b_dw, F, b_pw, y, N, C, Cout, stream, d, b + 3);
 }
 
 }  // namespace

@@ -18,12 +18,19 @@
 // then holds output channel o's row of pixels, which is exactly one contiguous range of the NCHW
 // output plane y[n, o, :, :].
 //
-// Work layout: one image per cluster of S CTAs (S = 2 when there are at least two channel
-// blocks: rank k takes blocks k, k + S, ...), 16 warps per CTA, the channels in blocks of CB.
-// Per block:
+// Work layout, two forms. Channel split: one image per cluster of S CTAs (S = 2 when there are
+// at least two channel blocks: rank k takes blocks k, k + S, ...). Row split (14x14, the
+// default there): two CTAs per image, no cluster; CTA 2k + h computes output rows 7h .. 7h + 6
+// for every channel, so each output's whole channel sum stays in one CTA's accumulator and in
+// the channel order of the one-CTA form (the same bits), while the image's MMA N halves
+// (208 -> 112 columns) and twice as many CTAs share the images. 16 warps per CTA, the
+// channels in blocks of CB. Per block:
 //   * x: the block's CB planes of the image are one contiguous range of x, staged into a
-//     2-slot ring two blocks ahead: at 14x14 one 1-D bulk copy per plane into a padded pitch
-//     (fewer bank conflicts in the row loads), at 7x7 one copy of the whole range;
+//     2-slot ring two blocks ahead: at 14x14 one 2-D tensor copy viewing x as [N*C][P] whose
+//     box is wider than a plane (a padded pitch: fewer bank conflicts in the row loads; the
+//     row-split form copies a 136-float window holding the input rows its half reads), at
+//     7x7 one bulk copy of the whole range; the block's taps arrive by a bulk copy on the same
+//     barrier;
 //   * F: the block's CB x Cout filter rows, 64-column boxes by TMA into a 3-slot ring (two
 //     blocks ahead); columns past Cout arrive as zeros;
 //   * every thread computes its strip (zeros padding, exact or fast mode, the depthwise bias),
@@ -35,7 +42,7 @@
 //     TMEM accumulators and commits; the B slot is rewritten two blocks later, after that
 //     commit.
 // After the last block all 16 warps read the accumulators (warp w: TMEM lane quarter w % 4, a
-// quarter of the 16-column chunks). With S = 2, 16-column chunk j belongs to rank j % 2: each
+// quarter of the 16-column chunks; the row split stores its 98 pixels of each plane). With S = 2, 16-column chunk j belongs to rank j % 2: each
 // rank writes its partial of the chunks it does not own into the owner's receive area through
 // distributed shared memory, and the owner adds the two partials (one IEEE addition, so the
 // result does not depend on which rank adds), the pointwise bias, and stores y.
@@ -71,16 +78,23 @@ struct DwPwGemmParams {
 };
 
 // Compile-time geometry per image size: channels per block, strips of two columns, rows per run.
-template <int HW_>
+// HALF (14x14): the two CTAs of an image each take half of its output rows and all of its
+// channels (64 per block), so that neither holds a partial sum of the other's outputs; its
+// plane window depends on the filter size KC_.
+template <int HW_, bool HALF_ = false, int KC_ = 3>
 struct DwPwGemmGeom {
     static constexpr int HW = HW_;
+    static constexpr bool HALF = HALF_;
+    static constexpr int KC = KC_;
     static constexpr int P = HW * HW;                      // pixels per image
-    static constexpr int NPAD = (P + 15) / 16 * 16;        // MMA N
+    static constexpr int ROWS = HALF ? HW / 2 : HW;        // output rows a CTA computes
+    static constexpr int PC = ROWS * HW;                   // output pixels a CTA computes
+    static constexpr int NPAD = (PC + 15) / 16 * 16;       // MMA N
     static constexpr int NCH = NPAD / 16;                  // 16-column accumulator chunks
-    static constexpr int CB = HW <= 8 ? 64 : 32;           // channels per block
+    static constexpr int CB = HALF ? 64 : (HW <= 8 ? 64 : 32);   // channels per block
     static constexpr int NSTRIP = (HW + 1) / 2;            // strips of two output columns
-    static constexpr int RR = HW <= 8 ? 4 : 7;             // output rows per run
-    static constexpr int NRUN = (HW + RR - 1) / RR;
+    static constexpr int RR = HALF ? ROWS : (HW <= 8 ? 4 : 7);   // output rows per run
+    static constexpr int NRUN = (ROWS + RR - 1) / RR;
     static constexpr int UPP = NSTRIP * NRUN;              // work units per plane
     static constexpr int THREADS = 512;
     static constexpr int UNITS = CB * UPP;                 // threads with depthwise work
@@ -92,7 +106,20 @@ struct DwPwGemmGeom {
     // spreads a warp's row loads over more banks (14x14: 196 -> 204 floats); 7x7 planes (196
     // bytes) arrive as one contiguous range
     static constexpr bool PADX = (P * 4) % 16 == 0;
-    static constexpr int XP = PADX ? P + 8 : P;            // plane pitch in shared memory, floats
+    // HALF: each CTA copies a window of the flat plane, first float XTOP (top half, negative:
+    // the rows above the image) or XBOT (bottom half), both multiples of 4 floats (16 bytes),
+    // wide enough that every input row and column its strips read -- the padding rows and
+    // columns included -- falls inside; rows outside the image lie outside the tensor and arrive
+    // as the copy's zero fill, so only the padding columns need a select
+    static constexpr int PADH = (KC - 1) / 2;
+    static constexpr int XTOP = HALF ? -((PADH * (HW + 1) + 3) / 4 * 4) : 0;
+    static constexpr int XBOT = HALF ? ((ROWS - PADH) * HW - PADH) / 4 * 4 : 0;
+    static constexpr int XLAST_TOP = (ROWS + PADH - 1) * HW + HW - 1 + PADH - XTOP;       // last float read
+    static constexpr int XLAST_BOT = (2 * ROWS + PADH - 1) * HW + HW - 1 + PADH - XBOT;
+    static constexpr int XNEED = ((XLAST_TOP > XLAST_BOT ? XLAST_TOP : XLAST_BOT) + 1 + 3) / 4 * 4;
+    // plane pitch in shared memory, floats; 8 mod 32, which spreads the planes of a warp's row
+    // loads over more banks (14x14 whole planes: 196 -> 204; HALF windows: 136 (3x3), 168 (5x5))
+    static constexpr int XP = HALF ? XNEED + (8 - XNEED % 32 + 32) % 32 : (PADX ? P + 8 : P);
     static constexpr int BOX = CB * 128;                   // one 64-wide box of CB rows, bf16
     static constexpr int NBOXB = (NPAD + 63) / 64;
     static constexpr int BSLOT = NBOXB * BOX;              // B tile: CB rows x NPAD pixels
@@ -100,6 +127,8 @@ struct DwPwGemmGeom {
     static constexpr int CHUNK = 128 * 16 * 4;             // 128 rows x 16 fp32 columns
     static constexpr int NOWN = (NCH + 1) / 2;             // chunks a rank of a 2-CTA cluster owns, at most
     static_assert(UNITS <= THREADS, "one work unit per thread");
+    static_assert(!HALF || (HW % 2 == 0 && PADX && SPARE), "halves of an even, 16-byte-row image");
+    static_assert(!HALF || ((ROWS - PADH) * HW - PADH >= XBOT && -PADH * (HW + 1) >= XTOP), "windows start early enough");
     static_assert(!PADX || (XP * 4) % 16 == 0, "a tensor-copy box row is a multiple of 16 bytes");
     static_assert(CB % 16 == 0, "K = 16 steps");
 };
@@ -108,23 +137,22 @@ constexpr int kDwPwGemmFSlots = 3;
 constexpr int kDwPwGemmBars = 2 /*xfull*/ + 3 /*ffull*/ + 2 /*mma_done*/ + 1 /*accf*/ + 1 /*drain*/;
 
 // bytes of one block's depthwise taps (CB channels x KK), staged beside its planes
-template <int HW>
+template <class G>
 __host__ __device__ constexpr int dwpw_gemm_wslot(int KK) {
-    return (DwPwGemmGeom<HW>::CB * KK * 4 + 127) / 128 * 128;
+    return (G::CB * KK * 4 + 127) / 128 * 128;
 }
 
 // shared memory: filter ring, B ring, x ring, taps ring, the receive area of the cluster
 // reduction (MT x NOWN chunks), barriers
-template <int HW>
+template <class G>
 __host__ __device__ constexpr int dwpw_gemm_recv(int MT, int S) {
-    return S > 1 ? MT * DwPwGemmGeom<HW>::NOWN * DwPwGemmGeom<HW>::CHUNK : 0;
+    return S > 1 ? MT * G::NOWN * G::CHUNK : 0;
 }
 
-template <int HW>
+template <class G>
 __host__ __device__ constexpr int dwpw_gemm_smem(int fslot, int MT, int S, int KK) {
-    using G = DwPwGemmGeom<HW>;
-    return 1024 + kDwPwGemmFSlots * fslot + 2 * G::BSLOT + 2 * G::XSLOT + 2 * dwpw_gemm_wslot<HW>(KK) +
-           dwpw_gemm_recv<HW>(MT, S) + kDwPwGemmBars * 8 + 16;
+    return 1024 + kDwPwGemmFSlots * fslot + 2 * G::BSLOT + 2 * G::XSLOT + 2 * dwpw_gemm_wslot<G>(KK) +
+           dwpw_gemm_recv<G>(MT, S) + kDwPwGemmBars * 8 + 16;
 }
 
 // One bf16 value into the B tile: row k (channel in the block), column n (pixel); 64 pixels per
@@ -144,16 +172,17 @@ __device__ __forceinline__ void dwpw_store_b2(uint8_t *sB, int box_bytes, int k,
         __floats2bfloat162_rn(v0, v1);
 }
 
-template <int MODE, int KC, int HW>
+template <int MODE, int KC, class G>
 __global__ void __launch_bounds__(512, 1)
 dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const __grid_constant__ CUtensorMap tmF,
                  const __grid_constant__ CUtensorMap tmX, float *__restrict__ y, const DwPwGemmParams p,
                  unsigned int *status) {
     grid_dependents_launch();   // programmatic dependent launch (see ptx.cuh)
     grid_dependency_wait();
-    using G = DwPwGemmGeom<HW>;
+    constexpr int HW = G::HW;
     constexpr int PAD = (KC - 1) / 2;
     constexpr int WIN = KC + 1;   // input columns of a two-column strip
+    static_assert(!G::HALF || G::KC == KC, "the row split's plane window is laid out for this filter size");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -162,10 +191,10 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     const uint32_t sB = sF + kDwPwGemmFSlots * p.fslot;
     const uint32_t sX = sB + 2 * G::BSLOT;
     constexpr int KK = KC * KC;
-    constexpr int WSLOT = dwpw_gemm_wslot<HW>(KK);
+    constexpr int WSLOT = dwpw_gemm_wslot<G>(KK);
     const uint32_t sW = sX + 2 * G::XSLOT;   // the blocks' taps, a 2-slot ring beside x
     const uint32_t sR = sW + 2 * WSLOT;      // receive area of the reduction
-    const uint32_t bars = sR + dwpw_gemm_recv<HW>(p.MT, p.S);
+    const uint32_t bars = sR + dwpw_gemm_recv<G>(p.MT, p.S);
     auto xfull = [&](int s) { return bars + 8u * s; };
     auto ffull = [&](int s) { return bars + 16u + 8u * s; };
     auto mma_done = [&](int s) { return bars + 40u + 8u * s; };
@@ -175,8 +204,14 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int S = p.S;
     const int rank = S > 1 ? static_cast<int>(cluster_rank()) : 0;
-    const int cluster = static_cast<int>(blockIdx.x) / S;
-    const int nclusters = static_cast<int>(gridDim.x) / S;
+    // HALF: CTA pairs 2k, 2k + 1 take the top and bottom halves of the same images (no cluster)
+    const int per = G::HALF ? 2 : S;
+    const int half = G::HALF ? static_cast<int>(blockIdx.x & 1u) : 0;
+    const int cluster = static_cast<int>(blockIdx.x) / per;
+    const int nclusters = static_cast<int>(gridDim.x) / per;
+    // HALF: the first output row of this CTA, and the first float of its plane window
+    const int row0 = half * G::ROWS;
+    const int xbase = G::HALF ? (half ? G::XBOT : G::XTOP) : 0;
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) mbar_init(xfull(s), 1);
@@ -230,7 +265,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
             // rows past the image's channels are other planes or zeros, never used)
             if (lane == 0) {
                 mbar_arrive_expect_tx(xfull(g & 1), static_cast<uint32_t>(G::CB * G::XP * 4) + wbytes);
-                tma_load_2d(sX + (g & 1) * G::XSLOT, &tmX, xfull(g & 1), 0, n * p.C + c0);
+                tma_load_2d(sX + (g & 1) * G::XSLOT, &tmX, xfull(g & 1), xbase, n * p.C + c0);
                 copy_w();
             }
         } else if (lane == 0) {
@@ -271,14 +306,38 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     const int r = rem / G::NSTRIP;
     const int ox0 = 2 * s;
     const int ix0 = ox0 - PAD;
-    const int oy_first = r * G::RR;
+    const int oy_first = row0 + r * G::RR;   // absolute output row (HALF: inside this CTA's half)
+    constexpr int ROWS = G::ROWS;
     bool colok[WIN];
 #pragma unroll
     for (int t = 0; t < WIN; ++t) colok[t] = ix0 + t >= 0 && ix0 + t < HW;
     const bool second = ox0 + 1 < HW;   // the strip's second column exists
 
     // depthwise outputs of block g (channel c0 + cl of the image) into the B slot, bf16
-    // (its taps arrive with its planes; its bias bv was loaded before the waits)
+    // (its taps arrive with its planes; its bias bv was loaded before the waits). The rows of
+    // a run are one branch-free stretch of code, so that their tap chains -- each output's taps
+    // in the page's order -- can interleave; only the B-tile store of a row past the image is
+    // skipped.
+    constexpr bool ALLROWS = G::RR * G::NRUN == ROWS;   // every run's rows exist
+    const bool hb = p.b_dw != nullptr;
+    // the finished output: NaN made canonical (exact mode), the bias added once when given
+    auto finish = [&](float a, float bv) {
+        const float a0 = dw_finish<MODE, false>(a, 0.0f);
+        const float a1 = dw_finish<MODE, true>(a, bv);
+        return hb ? a1 : a0;
+    };
+    auto store_pair = [&](uint8_t *bslot, int i, float a0, float a1) {
+        const int oy = oy_first + i;
+        if (ALLROWS || oy < row0 + ROWS) {
+            const int pix = (oy - row0) * HW + ox0;   // pixel within this CTA's rows
+            if constexpr (HW % 2 == 0) {
+                dwpw_store_b2(bslot, G::BOX, cl, pix, a0, a1);   // pix even, both columns exist
+            } else {
+                dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
+                if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
+            }
+        }
+    };
     auto depthwise_block = [&](int g, int c0, float bv) {
         uint8_t *bslot = smem + (sB - base) + (g & 1) * G::BSLOT;
         const int c = c0 + cl;
@@ -291,23 +350,70 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
             uint64_t w2[KC * KC];
 #pragma unroll
             for (int t = 0; t < KC * KC; ++t) w2[t] = dw_pack(wr[t], wr[t]);
-            // ring of KC input rows, each as KC overlapping pairs (x[t], x[t+1])
-            uint64_t ring[KC][KC];
+            // input row iy as KC overlapping pairs (x[t], x[t+1]); rows and columns outside the
+            // image read as zeros
             auto load_pairs = [&](int iy, uint64_t (&dst)[KC]) {
                 float f[WIN];
-                const bool rowok = iy >= 0 && iy < HW;
+                if constexpr (G::HALF) {
+                    // the window holds zeros for the rows outside the image; the middle columns
+                    // of a strip are always inside it
 #pragma unroll
-                for (int t = 0; t < WIN; ++t) f[t] = (rowok && colok[t]) ? xs[iy * HW + ix0 + t] : 0.0f;
+                    for (int t = 0; t < WIN; ++t) {
+                        const float v = xs[iy * HW + ix0 + t - xbase];
+                        f[t] = (t >= PAD && t <= PAD + 1) || colok[t] ? v : 0.0f;
+                    }
+                } else {
+                    const bool rowok = iy >= 0 && iy < HW;
+#pragma unroll
+                    for (int t = 0; t < WIN; ++t) f[t] = (rowok && colok[t]) ? xs[iy * HW + ix0 + t - xbase] : 0.0f;
+                }
 #pragma unroll
                 for (int t = 0; t < KC; ++t) dst[t] = dw_pack(f[t], f[t + 1]);
             };
+            if constexpr (KC == 3) {
+                // every input row of the run held at once (RR + 2 rows of 3 pairs), then tap by
+                // tap over the RR rows: RR independent chains per output column
+                constexpr int NR = G::RR + KC - 1;
+                uint64_t rows[NR][KC];
 #pragma unroll
-            for (int q = 0; q < KC - 1; ++q) load_pairs(oy_first - PAD + q, ring[q]);
+                for (int q = 0; q < NR; ++q) load_pairs(oy_first - PAD + q, rows[q]);
+                if constexpr (MODE == 0) {
+                    float a0[G::RR], a1[G::RR];
 #pragma unroll
-            for (int i = 0; i < G::RR; ++i) {
-                const int oy = oy_first + i;
-                if (oy < HW) {
-                    load_pairs(oy - PAD + KC - 1, ring[(i + KC - 1) % KC]);
+                    for (int i = 0; i < G::RR; ++i) a0[i] = a1[i] = 0.0f;
+#pragma unroll
+                    for (int ky = 0; ky < KC; ++ky)
+#pragma unroll
+                        for (int kx = 0; kx < KC; ++kx)
+#pragma unroll
+                            for (int i = 0; i < G::RR; ++i) dw_tap2_exact(a0[i], a1[i], w2[ky * KC + kx], rows[i + ky][kx]);
+#pragma unroll
+                    for (int i = 0; i < G::RR; ++i) store_pair(bslot, i, finish(a0[i], bv), finish(a1[i], bv));
+                } else {
+                    uint64_t a2[G::RR];
+#pragma unroll
+                    for (int i = 0; i < G::RR; ++i) a2[i] = dw_pack(0.0f, 0.0f);
+#pragma unroll
+                    for (int ky = 0; ky < KC; ++ky)
+#pragma unroll
+                        for (int kx = 0; kx < KC; ++kx)
+#pragma unroll
+                            for (int i = 0; i < G::RR; ++i) a2[i] = dw_tap2_fast(a2[i], w2[ky * KC + kx], rows[i + ky][kx]);
+#pragma unroll
+                    for (int i = 0; i < G::RR; ++i) {
+                        float a0, a1;
+                        dw_unpack(a2[i], a0, a1);
+                        store_pair(bslot, i, finish(a0, bv), finish(a1, bv));
+                    }
+                }
+            } else {
+                // larger filters: a ring of KC input rows, one output row after another
+                uint64_t ring[KC][KC];
+#pragma unroll
+                for (int q = 0; q < KC - 1; ++q) load_pairs(oy_first - PAD + q, ring[q]);
+#pragma unroll
+                for (int i = 0; i < G::RR; ++i) {
+                    load_pairs(oy_first + i - PAD + KC - 1, ring[(i + KC - 1) % KC]);
                     float a0, a1;
                     if constexpr (MODE == 0) {
                         a0 = 0.0f;
@@ -326,40 +432,18 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
                                 a2 = dw_tap2_fast(a2, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
                         dw_unpack(a2, a0, a1);
                     }
-                    if (p.b_dw) {
-                        a0 = dw_finish<MODE, true>(a0, bv);
-                        a1 = dw_finish<MODE, true>(a1, bv);
-                    } else {
-                        a0 = dw_finish<MODE, false>(a0, 0.0f);
-                        a1 = dw_finish<MODE, false>(a1, 0.0f);
-                    }
-                    const int pix = oy * HW + ox0;
-                    if constexpr (HW % 2 == 0) {
-                        dwpw_store_b2(bslot, G::BOX, cl, pix, a0, a1);   // pix even, both columns exist
-                    } else {
-                        dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
-                        if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
-                    }
+                    store_pair(bslot, i, finish(a0, bv), finish(a1, bv));
                 }
             }
         } else {
             // channels past C: zero rows, so that the zero filter rows meet finite values
-            const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
-            for (int i = 0; i < G::RR; ++i) {
-                const int oy = oy_first + i;
-                if (oy < HW) {
-                    if constexpr (HW % 2 == 0) {
-                        dwpw_store_b2(bslot, G::BOX, cl, oy * HW + ox0, 0.0f, 0.0f);
-                    } else {
-                        dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0, z);
-                        if (second) dwpw_store_b(bslot, G::BOX, cl, oy * HW + ox0 + 1, z);
-                    }
-                }
-            }
+#pragma unroll
+            for (int i = 0; i < G::RR; ++i) store_pair(bslot, i, 0.0f, 0.0f);
         }
     };
 
     // 16 consecutive pixels of output channel o: acc (+ the cluster peer's partial) + bias -> y
+    // (the channel split; the row split stages its tile through shared memory)
     auto store_chunk = [&](float *yrow, int p0, const float (&v)[16], float bp) {
         if (!in_bounds((yrow - y) + p0, min(16, G::P - p0), 1LL * p.num_tiles * p.Cout * G::P, kSiteDwPwGemmY, status))
             return;   // skipped (bounds-checked debug build)
@@ -406,7 +490,10 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
             }
             if (!dead && issuer) {
                 // the whole issuing warp, converged; the MMAs and commits are predicated on the
-                // elected lane (so are the drain's, so that its commit tracks them all)
+                // elected lane (so are the drain's, so that its commit tracks them all). First the
+                // refill of x two blocks ahead, into the slot this block's depthwise stage has just
+                // finished reading (the barrier above), so that its copy overlaps the MMAs too
+                if (g + 2 < total) issue_x(g + 2);
                 if (!mbar_wait_warp(ffull(g % 3), (g / 3) & 1)) {
                     fail = true;
                 } else {
@@ -423,10 +510,8 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
                                            p.idesc, (j | kk) != 0 ? 1u : 0u, leader);
                     umma_commit_if(mma_done(g & 1), leader);
                     if (j == nb - 1) umma_commit_if(accf, leader);
-                    // refill: x two blocks ahead into the slot this block has read; F two blocks
-                    // ahead into the slot block g - 1 used, once its MMAs are done
+                    // F two blocks ahead into the slot block g - 1 used, once its MMAs are done
                     if (g + 2 < total) {
-                        issue_x(g + 2);
                         if (g >= 1 && !mbar_wait_warp(mma_done((g - 1) & 1), ((g - 1) >> 1) & 1)) fail = true;
                         else issue_f(g + 2);
                     }
@@ -461,7 +546,56 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
             }
             cluster_sync_all();   // the partials have landed in the owners' receive areas
         }
-        if (!dead) {
+        if constexpr (G::HALF) {
+            // Row split: staged through the B ring (its last MMAs are complete and the next
+            // image's depthwise writes come after this epilogue), one tile of 128 output
+            // channels x 64 pixels at a time, so that y is written in contiguous runs of a
+            // channel's pixels rather than one 8-byte piece per channel. The 16-byte chunks of a
+            // staged row are XOR-swizzled by the row: conflict-free column writes and row reads.
+            float *stage = reinterpret_cast<float *>(smem + (sB - base));
+            static_assert(2 * G::BSLOT >= 128 * 64 * 4, "the staging tile fits the B ring");
+            constexpr int NPASS = (G::PC + 63) / 64;
+            for (int mt = 0; mt < p.MT; ++mt) {
+                const int o = mt * 128 + q * 32 + lane;
+                const float bp = (p.b_pw && o < p.Cout) ? __ldg(p.b_pw + o) : 0.0f;
+                for (int pass = 0; pass < NPASS; ++pass) {
+                    const int jc = pass * 4 + cg;   // this warp's 16-column chunk
+                    if (!dead && jc < G::NCH) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + mt * G::NPAD + jc * 16, v);
+                        tmem_wait_ld();
+                        const int r = q * 32 + lane;
+                        float *srow = stage + r * 64;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int chunk = (cg * 4 + u) ^ (r & 15);
+                            *reinterpret_cast<float4 *>(srow + chunk * 4) =
+                                make_float4(__fadd_rn(__uint_as_float(v[4 * u]), bp),
+                                            __fadd_rn(__uint_as_float(v[4 * u + 1]), bp),
+                                            __fadd_rn(__uint_as_float(v[4 * u + 2]), bp),
+                                            __fadd_rn(__uint_as_float(v[4 * u + 3]), bp));
+                        }
+                    }
+                    __syncthreads();
+                    // 128 staged rows, 16 warps: a warp writes a row's pixels as 8-byte pieces (a
+                    // half plane starts 8-byte aligned)
+                    const int ncols = min(64, G::PC - pass * 64);
+                    if (!dead && 2 * lane < ncols) {
+                        for (int rr = warp; rr < 128; rr += 16) {
+                            const int oo = mt * 128 + rr;
+                            if (oo >= p.Cout) break;
+                            const int col = 2 * lane;
+                            const float2 val = *reinterpret_cast<const float2 *>(
+                                stage + rr * 64 + (((col >> 2) ^ (rr & 15)) << 2) + (col & 3));
+                            float *dst = y + (static_cast<long long>(n) * p.Cout + oo) * G::P + row0 * HW + pass * 64 + col;
+                            if (in_bounds(dst - y, 2, 1LL * p.num_tiles * p.Cout * G::P, kSiteDwPwGemmY, status))
+                                *reinterpret_cast<float2 *>(dst) = val;
+                        }
+                    }
+                    __syncthreads();
+                }
+            }
+        } else if (!dead) {
             for (int mt = 0; mt < p.MT; ++mt) {
                 const int o = mt * 128 + q * 32 + lane;
                 const float bp = (p.b_pw && o < p.Cout) ? __ldg(p.b_pw + o) : 0.0f;

@@ -39,6 +39,9 @@ CASES = [
     ("dw-tma", {"CONV_B200_DW_KERNEL": "tma"}, ("dw", (2, 8, 112, 112, 3, 2, 1, 1))),
     ("dw-plane", {}, ("dw", (4, 64, 14, 14, 3, 1, 1, 1))),
     ("dwpw-gemm", {}, ("dwpw", (4, 64, 14, 14, 3, 32))),
+    ("dwpw-gemm-half-k5", {}, ("dwpw", (3, 136, 14, 14, 5, 48))),
+    ("dwpw-gemm-cluster", {"CONV_B200_DWPW_HALF": "0"}, ("dwpw", (4, 128, 14, 14, 3, 32))),
+    ("dwpw-gemm-7", {}, ("dwpw", (4, 96, 7, 7, 5, 160))),
     ("dwpw-staged", {"CONV_B200_DWPW_KERNEL": "staged"}, ("dwpw", (2, 64, 28, 28, 3, 32))),
     ("dwpw-flat", {"CONV_B200_DWPW_KERNEL": "flat"}, ("dwpw", (2, 64, 28, 28, 3, 32))),
     ("im2col-explicit", {}, ("im2col", (2, 12, 12, 16, 24, 3))),

@@ -119,16 +119,30 @@ def test_full_size_blocks(cb, case):
 # 8 outputs, two 128-row M tiles (136, 256 outputs), no biases, more images than CTAs
 GEMM_CASES = [(2, 72, 14, 3, 112, 0, True), (3, 100, 7, 5, 160, 1, True), (2, 64, 14, 5, 8, 0, False),
               (2, 32, 7, 3, 136, 0, True), (1, 128, 14, 3, 256, 1, True), (160, 8, 14, 3, 16, 0, True),
-              (200, 4, 7, 5, 24, 1, True)]
+              (200, 4, 7, 5, 24, 1, True),
+              (2, 48, 14, 5, 144, 1, True)]   # 5x5 with more than 128 outputs: the row split's rings do not fit
 
 
-@pytest.mark.parametrize("split", ["1", "2"])
-@pytest.mark.parametrize("c", GEMM_CASES, ids=lambda c: "N{}C{}H{}K{}-O{}-{}".format(*c[:5], "exact" if c[5] == 0 else "fast"))
-def test_transposed_gemm_kernel(cb, c, split, monkeypatch):
-    # one CTA per image, or a 2-CTA cluster that splits the channel blocks and adds the two
-    # partial sums through distributed shared memory
+# the forms of the transposed-GEMM kernel: one CTA per image; a 2-CTA cluster that splits the
+# channel blocks and adds the two partial sums through distributed shared memory; and (14x14
+# images) two CTAs per image that each take half of the output rows and every channel
+GEMM_FORMS = {"one-cta": {"CONV_B200_DWPW_SPLIT": "1", "CONV_B200_DWPW_HALF": "0"},
+              "cluster": {"CONV_B200_DWPW_SPLIT": "2", "CONV_B200_DWPW_HALF": "0"},
+              "half-rows": {"CONV_B200_DWPW_HALF": "1"}}
+
+
+def _form(monkeypatch, form):
     monkeypatch.setenv("CONV_B200_DWPW_KERNEL", "gemm")
-    monkeypatch.setenv("CONV_B200_DWPW_SPLIT", split)
+    for k in ("CONV_B200_DWPW_SPLIT", "CONV_B200_DWPW_HALF"):
+        monkeypatch.delenv(k, raising=False)
+    for k, v in GEMM_FORMS[form].items():
+        monkeypatch.setenv(k, v)
+
+
+@pytest.mark.parametrize("form", list(GEMM_FORMS))
+@pytest.mark.parametrize("c", GEMM_CASES, ids=lambda c: "N{}C{}H{}K{}-O{}-{}".format(*c[:5], "exact" if c[5] == 0 else "fast"))
+def test_transposed_gemm_kernel(cb, c, form, monkeypatch):
+    _form(monkeypatch, form)
     N, C, H, K, Cout, mode, bias = c
     case = workloads.DwPwCase("t", N, C, H, H, K, 1, (K - 1) // 2, 1, Cout, bias, seed=C + K + Cout + N)
     x, w, bd, F, bp = workloads.dwpw_inputs(case)
@@ -142,15 +156,34 @@ def test_transposed_gemm_kernel(cb, c, split, monkeypatch):
     assert np.array_equal(y, y2)   # a given split repeats its bits
 
 
-@pytest.mark.parametrize("split", ["1", "2"])
-@pytest.mark.parametrize("hw,K", [(14, 3), (7, 5)])
+@pytest.mark.parametrize("K,mode", [(3, 0), (3, 1), (5, 0)])
+def test_half_rows_form_is_live(cb, K, mode, monkeypatch):
+    # the row halves accumulate every channel of an output in one chain, in channel order, as
+    # one CTA per image does: the same bits. The channel-split cluster adds two partial sums:
+    # over 700k outputs its bits differ somewhere, so equality with the one-CTA form shows that
+    # the half-rows form really ran (all three within the bar)
+    case = workloads.DwPwCase("t", 8, 672, 14, 14, K, 1, (K - 1) // 2, 1, 112, True, seed=15 + K)
+    x, w, bd, F, bp = workloads.dwpw_inputs(case)
+    ys = {}
+    for form in GEMM_FORMS:
+        _form(monkeypatch, form)
+        ys[form], kernel = _run(cb, case, x, w, bd, F, bp, mode)
+        assert kernel == "dwpw_gemm_kernel"
+    ref, absum = oracle.dwpw(x, w, bd, workloads.bf16_to_f32(F), bp, 1, (K - 1) // 2, 1, mode)
+    for y in ys.values():
+        assert np.all(np.abs(y - ref) <= _tol(case.C) * absum)
+    assert np.array_equal(ys["half-rows"], ys["one-cta"])
+    assert not np.array_equal(ys["cluster"], ys["one-cta"])
+
+
+@pytest.mark.parametrize("form", list(GEMM_FORMS))
+@pytest.mark.parametrize("hw,K", [(14, 3), (14, 5), (7, 5)])
 @pytest.mark.parametrize("mode", [0, 1])
-def test_transposed_gemm_identity_mixing_is_exact(cb, hw, K, mode, split, monkeypatch):
+def test_transposed_gemm_identity_mixing_is_exact(cb, hw, K, mode, form, monkeypatch):
     # F = I: every output is one exact product plus zeros (also each of the two partial sums of
     # a split), so the block must equal the depthwise output rounded to bf16, bit for bit (the
     # depthwise stage of this kernel is the page's order)
-    monkeypatch.setenv("CONV_B200_DWPW_KERNEL", "gemm")
-    monkeypatch.setenv("CONV_B200_DWPW_SPLIT", split)
+    _form(monkeypatch, form)
     case = workloads.DwPwCase("t", 3, 96, hw, hw, K, 1, (K - 1) // 2, 1, 96, True, seed=hw + K)
     x, w, bd, _, _ = workloads.dwpw_inputs(case)
     F = workloads.bf16_bits(np.eye(96, dtype=np.float32))
