@@ -55,6 +55,7 @@
 #include <cuda_bf16.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "depthwise.cuh"       // dw_finish, dw_tap
 #include "depthwise_tma.cuh"   // packed-pair helpers
@@ -155,21 +156,11 @@ __host__ __device__ constexpr int dwpw_gemm_smem(int fslot, int MT, int S, int K
            dwpw_gemm_recv<G>(MT, S) + kDwPwGemmBars * 8 + 16;
 }
 
-// One bf16 value into the B tile: row k (channel in the block), column n (pixel); 64 pixels per
-// box, 128-byte rows, 16-byte chunks swizzled by k % 8.
-__device__ __forceinline__ void dwpw_store_b(uint8_t *sB, int box_bytes, int k, int n, __nv_bfloat16 v) {
+// Byte offset of one bf16 value of the B tile: row k (channel in the block), column n (pixel);
+// 64 pixels per box, 128-byte rows, 16-byte chunks swizzled by k % 8.
+__device__ __forceinline__ uint32_t dwpw_b_offset(int box_bytes, int k, int n) {
     const int box = n >> 6, col = n & 63;
-    const int chunk = (col >> 3) ^ (k & 7);
-    *reinterpret_cast<__nv_bfloat16 *>(sB + box * box_bytes + k * 128 + chunk * 16 + (col & 7) * 2) = v;
-}
-
-// Two bf16 values for pixels n (even) and n + 1 of row k: one 4-byte store (an even column and
-// its neighbour share a 16-byte chunk of one box).
-__device__ __forceinline__ void dwpw_store_b2(uint8_t *sB, int box_bytes, int k, int n, float v0, float v1) {
-    const int box = n >> 6, col = n & 63;
-    const int chunk = (col >> 3) ^ (k & 7);
-    *reinterpret_cast<__nv_bfloat162 *>(sB + box * box_bytes + k * 128 + chunk * 16 + (col & 7) * 2) =
-        __floats2bfloat162_rn(v0, v1);
+    return static_cast<uint32_t>(box * box_bytes + k * 128 + (((col >> 3) ^ (k & 7)) << 4) + (col & 7) * 2);
 }
 
 template <int MODE, int KC, class G>
@@ -319,26 +310,34 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     // in the page's order -- can interleave; only the B-tile store of a row past the image is
     // skipped.
     constexpr bool ALLROWS = G::RR * G::NRUN == ROWS;   // every run's rows exist
-    const bool hb = p.b_dw != nullptr;
-    // the finished output: NaN made canonical (exact mode), the bias added once when given
-    auto finish = [&](float a, float bv) {
-        const float a0 = dw_finish<MODE, false>(a, 0.0f);
-        const float a1 = dw_finish<MODE, true>(a, bv);
-        return hb ? a1 : a0;
-    };
+    // The B-tile byte offsets of this unit's outputs are the same in every block: row i of the
+    // run at pixel pix = (oy - row0) * HW + ox0 of this CTA's rows (and pix + 1 for odd images,
+    // whose pair may straddle a 16-byte chunk)
+    auto b_off = [&](int n) { return dwpw_b_offset(G::BOX, cl, n); };
+    uint32_t boff[G::RR], boff1[G::RR];
+#pragma unroll
+    for (int i = 0; i < G::RR; ++i) {
+        const int pix = (oy_first + i - row0) * HW + ox0;
+        boff[i] = b_off(pix);
+        boff1[i] = HW % 2 == 0 ? 0u : b_off(pix + 1);
+    }
     auto store_pair = [&](uint8_t *bslot, int i, float a0, float a1) {
-        const int oy = oy_first + i;
-        if (ALLROWS || oy < row0 + ROWS) {
-            const int pix = (oy - row0) * HW + ox0;   // pixel within this CTA's rows
+        if (ALLROWS || oy_first + i < row0 + ROWS) {
             if constexpr (HW % 2 == 0) {
-                dwpw_store_b2(bslot, G::BOX, cl, pix, a0, a1);   // pix even, both columns exist
+                // pix even: both columns exist and share a 16-byte chunk
+                *reinterpret_cast<__nv_bfloat162 *>(bslot + boff[i]) = __floats2bfloat162_rn(a0, a1);
             } else {
-                dwpw_store_b(bslot, G::BOX, cl, pix, __float2bfloat16_rn(a0));
-                if (second) dwpw_store_b(bslot, G::BOX, cl, pix + 1, __float2bfloat16_rn(a1));
+                *reinterpret_cast<__nv_bfloat16 *>(bslot + boff[i]) = __float2bfloat16_rn(a0);
+                if (second) *reinterpret_cast<__nv_bfloat16 *>(bslot + boff1[i]) = __float2bfloat16_rn(a1);
             }
         }
     };
-    auto depthwise_block = [&](int g, int c0, float bv) {
+    // hb_tag: std::true_type when the depthwise bias is given (a compile-time choice per call,
+    // so that the finished rows carry no select)
+    auto depthwise_block = [&](int g, int c0, float bv, auto hb_tag) {
+        constexpr bool HB = decltype(hb_tag)::value;
+        // the finished output: NaN made canonical (exact mode), the bias added once when given
+        auto finish = [&](float a, float b) { return dw_finish<MODE, HB>(a, b); };
         uint8_t *bslot = smem + (sB - base) + (g & 1) * G::BSLOT;
         const int c = c0 + cl;
         if (c < p.C) {
@@ -470,8 +469,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     for (int tl = 0; tl < my_tiles; ++tl) {
         const int n = cluster + tl * nclusters;
         for (int j = 0; j < nb; ++j, ++g) {
-            int nn, c0;
-            block_at(g, nn, c0);
+            const int c0 = (rank + j * S) * G::CB;   // block g = tl * nb + j (block_at without the division)
             bool good = true;
             if (!dead) {
                 // the channel's bias first, so that its load overlaps the waits
@@ -481,7 +479,12 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
                 // the block's planes staged; the B slot's previous MMAs (block g - 2) done
                 good = mbar_wait_warp(xfull(g & 1), (g >> 1) & 1);
                 if (good && g >= 2) good = mbar_wait_warp(mma_done(g & 1), ((g - 2) >> 1) & 1);
-                if (good && unit_ok) depthwise_block(g, c0, bv);
+                if (good && unit_ok) {
+                    if (p.b_dw)
+                        depthwise_block(g, c0, bv, std::true_type{});
+                    else
+                        depthwise_block(g, c0, bv, std::false_type{});
+                }
                 fence_proxy_async_smem();   // the B tile's generic writes, visible to the tensor cores
             }
             if (__syncthreads_or(!good || fail) && !dead) {
