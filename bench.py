@@ -434,37 +434,69 @@ def time_case(cb, torch, kind, case, mode, inputs, steps, warmup, dist=None, sam
     return ms, R, kernel
 
 
+E2E_SETS = 2   # device buffer sets of the end-to-end pipeline
+
+
 def e2e_bench(cb, torch, kind, case, mode, host, steps, warmup):
-    """Public API end to end: pinned host inputs -> device, convolution, output -> pinned host."""
-    dev = [torch.empty(h.shape, dtype=h.dtype, device="cuda") if h is not None else None for h in host]
-    if kind == "dense":
-        out = torch.empty(out_shape(kind, case), dtype=host[0].dtype, device="cuda")
-    else:
-        out = torch.empty(out_shape(kind, case), device="cuda")
-    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    ws = im2col_workspace(cb, torch, case, mode) if kind == "dense" else None
-
-    def step():
-        for d, h in zip(dev, host):
-            if h is not None:
-                d.copy_(h, non_blocking=True)
+    """Public API end to end: every step copies its inputs from pinned host memory to the
+    device, runs the convolution and copies its output back to pinned host memory. The copies
+    in and out and the convolution run on three streams over E2E_SETS device buffer sets,
+    ordered by events (a set's inputs are rewritten only after the convolution that read them,
+    its output only after the copy that read it), so step i+1's upload overlaps step i's
+    download as in a serving loop; the timed region spans the first upload to the last
+    download."""
+    def dev_set():
+        d = [torch.empty(h.shape, dtype=h.dtype, device="cuda") if h is not None else None for h in host]
         if kind == "dense":
-            dense_call(cb, case, dev[0], dev[1], dev[2], out, mode, ws)
-        elif kind == "dwpw":
-            dwpw_call(cb, case, dev[0], dev[1], dev[2], dev[3], dev[4], out, mode)
+            o = torch.empty(out_shape(kind, case), dtype=host[0].dtype, device="cuda")
         else:
-            cb.depthwise_fwd(dev[0], dev[1], dev[2], out, case.stride, case.pad, case.dil, mode)
-        out_h.copy_(out, non_blocking=True)
+            o = torch.empty(out_shape(kind, case), device="cuda")
+        w = im2col_workspace(cb, torch, case, mode) if kind == "dense" else None
+        return d, o, w
 
-    for _ in range(warmup):
-        step()
-    stream = torch.cuda.current_stream()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sets = [dev_set() for _ in range(E2E_SETS)]
+    out_h = torch.empty(sets[0][1].shape, dtype=sets[0][1].dtype, pin_memory=True)
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: [torch.cuda.Event() for _ in range(E2E_SETS)]   # noqa: E731
+    ev_in, ev_cmp, ev_out = ev(), ev(), ev()
+
+    def step(i):
+        k = i % E2E_SETS
+        dev, out, ws = sets[k]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[k])          # the convolution that read this set is done
+            for d, h in zip(dev, host):
+                if h is not None:
+                    d.copy_(h, non_blocking=True)
+            ev_in[k].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[k])
+            s_cmp.wait_event(ev_out[k])         # this set's previous output has been copied out
+            if kind == "dense":
+                dense_call(cb, case, dev[0], dev[1], dev[2], out, mode, ws)
+            elif kind == "dwpw":
+                dwpw_call(cb, case, dev[0], dev[1], dev[2], dev[3], dev[4], out, mode)
+            else:
+                cb.depthwise_fwd(dev[0], dev[1], dev[2], out, case.stride, case.pad, case.dil, mode)
+            ev_cmp[k].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[k])
+            out_h.copy_(out, non_blocking=True)
+            ev_out[k].record(s_out)
+
+    main = torch.cuda.current_stream()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
-    start.record(stream)
-    for _ in range(steps):
-        step()
-    end.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(main)
+    for st in (s_in, s_cmp, s_out):
+        st.wait_stream(main)
+    for i in range(steps):
+        step(i)
+    for st in (s_in, s_cmp, s_out):
+        main.wait_stream(st)
+    end.record(main)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end) / steps
     h2d = sum(h.numel() * h.element_size() for h in host if h is not None)
@@ -612,7 +644,9 @@ def run_ours(args, dist):
         "config": cfg, "roofline": roof,
         "e2e": {"value": round(e2e_value, 4), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4),
-                "path": "python binding -> C ABI, pinned host copies in the timed region"},
+                "path": "python binding -> C ABI, pinned host copies in the timed region; uploads, "
+                        f"convolutions and downloads on three streams over {E2E_SETS} device buffer sets "
+                        "(step i+1's upload overlaps step i's download)"},
         "gpu_launches": args.steps,   # one library kernel per step (the comparison path adds a cuBLAS GEMM)
         "clocks": sampler.summary(),
         "device_status": cb.conv_status_string(status),

@@ -92,7 +92,7 @@ struct DwPwGemmGeom {
     static constexpr int PC = ROWS * HW;                   // output pixels a CTA computes
     static constexpr int NPAD = (PC + 15) / 16 * 16;       // MMA N
     static constexpr int NCH = NPAD / 16;                  // 16-column accumulator chunks
-    static constexpr int CB = HALF ? 64 : (HW <= 8 ? 64 : 32);   // channels per block
+    static constexpr int CB = HALF ? 64 : (HW <= 8 ? 48 : 32);   // channels per block
     static constexpr int NSTRIP = (HW + 1) / 2;            // strips of two output columns
     static constexpr int RR = HALF ? ROWS : (HW <= 8 ? 4 : 7);   // output rows per run
     static constexpr int NRUN = (ROWS + RR - 1) / RR;
