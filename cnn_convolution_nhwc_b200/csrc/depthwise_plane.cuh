@@ -165,21 +165,7 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
                 load_pairs(oy - PAD + K - 1, ring[(oy + K - 1) % K]);
                 float acc[WOL];
                 constexpr int NP = WOL / 2;
-                if constexpr (MODE == 0) {
-#pragma unroll
-                    for (int v = 0; v < WOL; ++v) acc[v] = 0.0f;
-#pragma unroll
-                    for (int ky = 0; ky < K; ++ky)
-#pragma unroll
-                        for (int kx = 0; kx < K; ++kx) {
-#pragma unroll
-                            for (int q = 0; q < NP; ++q)
-                                dw_tap2_exact(acc[2 * q], acc[2 * q + 1], w2[ky * K + kx], ring[(oy + ky) % K][2 * q + kx]);
-                            if constexpr (WOL % 2 == 1)
-                                acc[WOL - 1] = dw_tap<MODE>(acc[WOL - 1], wr[ky * K + kx],
-                                                            pair_elem(ring[(oy + ky) % K], WOL - 1 + kx));
-                        }
-                } else {
+                {
                     uint64_t a2[NP > 0 ? NP : 1];
 #pragma unroll
                     for (int q = 0; q < NP; ++q) a2[q] = dw_pack(0.0f, 0.0f);
@@ -190,7 +176,7 @@ depthwise_plane_kernel(const float *__restrict__ x, const float *__restrict__ w,
                         for (int kx = 0; kx < K; ++kx) {
 #pragma unroll
                             for (int q = 0; q < NP; ++q)
-                                a2[q] = dw_tap2_fast(a2[q], w2[ky * K + kx], ring[(oy + ky) % K][2 * q + kx]);
+                                a2[q] = dw_tap2<MODE>(a2[q], w2[ky * K + kx], ring[(oy + ky) % K][2 * q + kx]);
                             if constexpr (WOL % 2 == 1)
                                 last = dw_tap<MODE>(last, wr[ky * K + kx], pair_elem(ring[(oy + ky) % K], WOL - 1 + kx));
                         }

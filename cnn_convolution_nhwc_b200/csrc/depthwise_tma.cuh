@@ -90,10 +90,31 @@ __device__ __forceinline__ void dw_unpack(uint64_t v, float &lo, float &hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 
-// Exact-mode tap for two outputs (lo, hi): one packed multiply and two scalar rounded additions
-// -- a packed multiply whose only use is a packed addition was measured to come out fused (one
-// rounding), so the additions stay scalar.
-__device__ __forceinline__ void dw_tap2_exact(float &lo, float &hi, uint64_t w2, uint64_t x2) {
+// Exact-mode tap for two outputs (lo, hi): each product rounded once, then each sum rounded
+// once, as the page's rounded multiply then rounded add. The product is formed as fma(w, x, +0),
+// which equals the rounded product except that an exact zero product comes out +0 where the
+// multiply gives -0. A running sum that starts at +0 is never -0 (a rounded sum is -0 only when
+// both terms are), and adding +0 or -0 to it gives the same value, so every sum is bit-identical
+// to the page's. One packed fma and one packed add per tap pair, and no multiply: a packed
+// multiply whose only use is a packed add was measured to come out fused (one rounding).
+__device__ __forceinline__ uint64_t dw_tap2_exact(uint64_t acc, uint64_t w2, uint64_t x2) {
+    uint64_t prod, r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(prod) : "l"(w2), "l"(x2), "l"(0ull));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(acc), "l"(prod));
+    return r;
+}
+
+// Fast-mode tap for two outputs: one packed fused multiply-add.
+__device__ __forceinline__ uint64_t dw_tap2_fast(uint64_t acc, uint64_t w2, uint64_t x2) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(w2), "l"(x2), "l"(acc));
+    return r;
+}
+
+// The same exact-mode tap with the two sums kept as scalars: one packed multiply and two scalar
+// rounded additions (bit-identical to dw_tap2_exact; the fused depthwise-pointwise kernel,
+// bound by its shared-memory loads, measured faster with this form).
+__device__ __forceinline__ void dw_tap2_exact_split(float &lo, float &hi, uint64_t w2, uint64_t x2) {
     uint64_t prod;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(prod) : "l"(w2), "l"(x2));
     float p0, p1;
@@ -102,11 +123,13 @@ __device__ __forceinline__ void dw_tap2_exact(float &lo, float &hi, uint64_t w2,
     hi = __fadd_rn(hi, p1);
 }
 
-// Fast-mode tap for two outputs: one packed fused multiply-add.
-__device__ __forceinline__ uint64_t dw_tap2_fast(uint64_t acc, uint64_t w2, uint64_t x2) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(w2), "l"(x2), "l"(acc));
-    return r;
+// A tap for two outputs held as one packed pair, in either mode.
+template <int MODE>
+__device__ __forceinline__ uint64_t dw_tap2(uint64_t acc, uint64_t w2, uint64_t x2) {
+    if constexpr (MODE == 0)
+        return dw_tap2_exact(acc, w2, x2);
+    else
+        return dw_tap2_fast(acc, w2, x2);
 }
 
 template <int MODE, bool HAS_BIAS, int K, int S>
@@ -263,18 +286,7 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
                         // of staged row r: (u + r - i) % K, base being a multiple of K)
                         load_pairs(i + K - 1, ring[(u + K - 1) % K]);
                         float acc[VX];
-                        if constexpr (MODE == 0) {
-#pragma unroll
-                            for (int v = 0; v < VX; ++v) acc[v] = 0.0f;
-#pragma unroll
-                            for (int ky = 0; ky < K; ++ky)
-#pragma unroll
-                                for (int kx = 0; kx < K; ++kx)
-#pragma unroll
-                                    for (int q = 0; q < VX / 2; ++q)
-                                        dw_tap2_exact(acc[2 * q], acc[2 * q + 1], w2[ky * K + kx],
-                                                      ring[(u + ky) % K][2 * q + kx]);
-                        } else {
+                        {
                             uint64_t a2[VX / 2];
 #pragma unroll
                             for (int q = 0; q < VX / 2; ++q) a2[q] = dw_pack(0.0f, 0.0f);
@@ -284,7 +296,7 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
                                 for (int kx = 0; kx < K; ++kx)
 #pragma unroll
                                     for (int q = 0; q < VX / 2; ++q)
-                                        a2[q] = dw_tap2_fast(a2[q], w2[ky * K + kx], ring[(u + ky) % K][2 * q + kx]);
+                                        a2[q] = dw_tap2<MODE>(a2[q], w2[ky * K + kx], ring[(u + ky) % K][2 * q + kx]);
 #pragma unroll
                             for (int q = 0; q < VX / 2; ++q) dw_unpack(a2[q], acc[2 * q], acc[2 * q + 1]);
                         }

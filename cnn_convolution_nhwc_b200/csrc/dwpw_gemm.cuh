@@ -385,7 +385,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
 #pragma unroll
                         for (int kx = 0; kx < KC; ++kx)
 #pragma unroll
-                            for (int i = 0; i < G::RR; ++i) dw_tap2_exact(a0[i], a1[i], w2[ky * KC + kx], rows[i + ky][kx]);
+                            for (int i = 0; i < G::RR; ++i) dw_tap2_exact_split(a0[i], a1[i], w2[ky * KC + kx], rows[i + ky][kx]);
 #pragma unroll
                     for (int i = 0; i < G::RR; ++i) store_pair(bslot, i, finish(a0[i], bv), finish(a1[i], bv));
                 } else {
@@ -421,7 +421,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
                         for (int ky = 0; ky < KC; ++ky)
 #pragma unroll
                             for (int kx = 0; kx < KC; ++kx)
-                                dw_tap2_exact(a0, a1, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
+                                dw_tap2_exact_split(a0, a1, w2[ky * KC + kx], ring[(i + ky) % KC][kx]);
                     } else {
                         uint64_t a2 = dw_pack(0.0f, 0.0f);
 #pragma unroll

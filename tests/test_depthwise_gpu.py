@@ -343,3 +343,44 @@ def test_padding_nan_rule_production_kernels(cb, shape):
         assert np.isnan(ref).any() and np.isinf(ref).any()    # the planted values reach the outputs
         if mode == oracle.DW_EXACT:
             assert set(_bits(y)[np.isnan(y)].tolist()) == {0x7FC00000}
+
+
+# (N, C, H, K, S, kernel): the packed-pair production kernels
+ROUNDING_SHAPES = [(1, 8, 7, 3, 1, "plane"), (1, 8, 14, 3, 1, "plane"), (1, 8, 7, 5, 1, "plane"),
+                   (1, 8, 16, 3, 1, "tma"), (1, 8, 28, 5, 1, "tma")]
+
+
+def rounding_case(C, H, K):
+    """Channel 3, output (3, 3): two products, -(1 + 2^-11) and a^2 with a = 1 + 2^-12. Rounded
+    separately they cancel to +0; fused (one rounding) they leave 2^-24. Channel 0: zero input
+    and negative taps, every product -0, every output +0. Returns x, w, the output position."""
+    pad = (K - 1) // 2
+    a = np.float32(1 + 2.0 ** -12)
+    x = np.zeros((1, C, H, H), np.float32)
+    w = workloads.normal(31, C * K * K, 0.5).reshape(C, K, K).astype(np.float32)
+    w[0] = -1.0
+    w[3] = 0.0
+    w[3, 0, 0], w[3, 0, 1] = -1.0, a
+    oy = ox = 3
+    x[0, 3, oy - pad, ox - pad] = np.float32(1 + 2.0 ** -11)
+    x[0, 3, oy - pad, ox - pad + 1] = a
+    return x, w, (oy, ox)
+
+
+@pytest.mark.parametrize("shape", ROUNDING_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + "-" + s[5])
+def test_exact_mode_rounds_each_product_production_kernels(cb, shape):
+    # OneModel "Depthwise convolution", "What each output is": exact mode rounds every product
+    # and every sum; the accumulator starts at +0. Pinned on the kernels that compute two
+    # outputs per packed instruction, where a fused product would go unnoticed on random data
+    N, C, H, K, S, kernel = shape
+    x, w, (oy, ox) = rounding_case(C, H, K)
+    pad = (K - 1) // 2
+    for mode in MODES:
+        y = _with_env("CONV_B200_DW_KERNEL", kernel, lambda: _gpu(cb, x, w, None, S, pad, 1, mode))
+        assert cb.conv_last_kernel() == f"depthwise_{kernel}_kernel"
+        _compare(y, x, w, None, 1, S, pad, 1, mode)
+        assert np.all(_bits(y[0, 0]) == 0)          # all products -0: +0
+        if mode == oracle.DW_EXACT:
+            assert _bits(y[0, 3, oy, ox]) == 0      # rounded separately: exact cancellation
+        else:
+            assert y[0, 3, oy, ox] == np.float32(2.0 ** -24)   # one rounding

@@ -272,3 +272,25 @@ def test_split_is_live(cb, kern, monkeypatch):
     for y in ys.values():
         assert np.all(np.abs(y - ref) <= _tol(case.C) * absum)
     assert not np.array_equal(ys["1"], ys["4"])
+
+
+@pytest.mark.parametrize("form", list(GEMM_FORMS))
+@pytest.mark.parametrize("hw,K", [(14, 3), (7, 5)])
+def test_transposed_gemm_exact_mode_rounds_each_product(cb, hw, K, form, monkeypatch):
+    # the depthwise stage's exact mode rounds every product and every sum (OneModel "Depthwise
+    # convolution", "What each output is"): with F = I the block returns the bf16 depthwise
+    # output, and two products that cancel only when rounded separately must give +0 (fast
+    # mode: 2^-24, a bf16 value); zero inputs under negative taps give zeros
+    from tests.test_depthwise_gpu import rounding_case
+    _form(monkeypatch, form)
+    C = 16
+    x, w, (oy, ox) = rounding_case(C, hw, K)
+    F = workloads.bf16_bits(np.eye(C, dtype=np.float32))
+    case = workloads.DwPwCase("t", 1, C, hw, hw, K, 1, (K - 1) // 2, 1, C, False, seed=5)
+    for mode in (0, 1):
+        y, kernel = _run(cb, case, x, w, None, F, None, mode)
+        assert kernel == "dwpw_gemm_kernel"
+        dref = oracle.depthwise(x, w, None, mult=1, stride=1, pad=(K - 1) // 2, dil=1, mode=mode)
+        assert np.array_equal(y, workloads.bf16_to_f32(workloads.bf16_bits(dref)).astype(np.float64))
+        assert np.all(y[0, 0] == 0)
+        assert y[0, 3, oy, ox] == (0.0 if mode == 0 else 2.0 ** -24)   # (the mixing sum's zero signs are the tensor cores')
