@@ -281,10 +281,21 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
             for (int b = 0; b < 2 * p.MT; ++b) tma_load_2d(slot + b * G::BOX, &tmF, ffull(g % 3), b * 64, c0);
         }
     };
-    if (issuer) {
-        for (int g = 0; g < 2 && g < total; ++g) {
-            issue_x(g);
-            issue_f(g);
+    // fail: the issuing warp's own waits, or'ed into the CTA at the next block barrier
+    bool fail = false;
+    if (issuer && total > 0) {
+        // the first block's copies alone, and the second block's once its planes have landed:
+        // every CTA starts at once, and the first block's bytes need not share HBM with the
+        // second's (which then arrive while the first block is computed)
+        issue_x(0);
+        issue_f(0);
+        if (total > 1) {
+            if (mbar_wait_warp(xfull(0), 0)) {
+                issue_x(1);
+                issue_f(1);
+            } else {
+                fail = true;
+            }
         }
     }
 
@@ -463,7 +474,7 @@ dwpw_gemm_kernel(const float *__restrict__ x, const float *__restrict__ w, const
     // Every thread walks every tile and every block; after a wait ran out (dead) it skips the
     // work but still takes each CTA and cluster barrier, so neither this CTA nor its cluster
     // peer ever waits for it forever.
-    bool dead = false, fail = false;   // fail: the issuing lane's own waits, or'ed in at the next barrier
+    bool dead = false;
     int stop = 0;                      // the first block whose wait ran out
     int g = 0;
     for (int tl = 0; tl < my_tiles; ++tl) {
