@@ -51,6 +51,8 @@ struct DwTmaParams {
     int warp_floats;       // per-warp shared memory: nbuf * buf_floats + out_floats
     int nbuf;              // staging buffers per warp (2 .. kDwTmaMaxBuf): jobs staged ahead
     int vec_out_staged;    // 1: y 16-byte aligned (staged copies may use 128-bit stores)
+    int stagger;           // 1: a warp's first job is copied alone, the rest of its first NB after it
+                           //    (the first jobs' bytes need not share HBM at start)
     FastDiv div_nbands, div_lpp, div_c, div_w;
 };
 
@@ -209,8 +211,11 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
         for (int i = lane; i < NB * p.buf_floats / 4; i += 32) z[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
     __syncwarp();
-    // the warp's first NB jobs go in flight at once
-    for (int b = 0; b < NB; ++b)
+    // the warp's first NB jobs go in flight at once, or with p.stagger the first job alone and
+    // the rest once it has landed (in the loop): every warp starts at once, and the first jobs'
+    // bytes need not share HBM with the next ones' (which then arrive while the first is
+    // computed)
+    for (int b = 0; b < (p.stagger ? 1 : NB); ++b)
         if (gw + b * GW < p.num_jobs) issue(gw + b * GW, b);
 
     // lane geometry (fixed for the kernel's life)
@@ -225,6 +230,9 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
     for (int job = gw; job < p.num_jobs; job += GW, ++k) {
         const int b = k % NB;
         if (!mbar_wait_warp(full(b), (k / NB) & 1)) { ok = false; break; }
+        if (k == 0 && p.stagger)
+            for (int bb = 1; bb < NB; ++bb)
+                if (gw + bb * GW < p.num_jobs) issue(gw + bb * GW, bb);
         const int pg = fdiv(job, p.div_nbands);
         const int band = job - pg * p.nbands;
         const int oy0 = band * p.Rw;
@@ -362,8 +370,9 @@ depthwise_tma_kernel(const __grid_constant__ CUtensorMap tmx, const float *__res
     }
     if (!ok) {
         if (lane == 0) atomicOr(status, kStatusTimeout);
-        // drain: copies still in flight land before the warp exits (bounded waits)
-        for (int kk = k; kk < k + NB; ++kk)
+        // drain: copies still in flight land before the warp exits (bounded waits); with
+        // p.stagger a wait that ran out on the first job leaves only that job issued
+        for (int kk = k; kk < (k == 0 && p.stagger ? 1 : k + NB); ++kk)
             if (gw + kk * GW < p.num_jobs) mbar_wait_warp(full(kk % NB), (kk / NB) & 1);
     }
 }

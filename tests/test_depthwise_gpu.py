@@ -384,3 +384,32 @@ def test_exact_mode_rounds_each_product_production_kernels(cb, shape):
             assert _bits(y[0, 3, oy, ox]) == 0      # rounded separately: exact cancellation
         else:
             assert y[0, 3, oy, ox] == np.float32(2.0 ** -24)   # one rounding
+
+
+@pytest.mark.parametrize("ring", ["2", "3"])
+@pytest.mark.parametrize("shape", [(2, 16, 56, 3, 2), (1, 8, 28, 5, 1), (2, 4, 112, 3, 1)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_tma_staggered_first_copies(cb, shape, ring):
+    # the TMA kernel's first copies with and without the stagger (a warp's first job alone,
+    # the rest of its ring after it), over rings of 2 and 3 buffers: the same bits, the oracle's
+    N, C, H, K, S = shape
+    case = workloads.DepthwiseCase("stagger", N, C, 1, H, H, K, K, S, (K - 1) // 2, 1, True, 23)
+    x, w, b = workloads.depthwise_inputs(case)
+    old = {k: os.environ.get(k) for k in ("CONV_B200_DW_KERNEL", "CONV_B200_DW_RING", "CONV_B200_DW_STAGGER")}
+    try:
+        os.environ["CONV_B200_DW_KERNEL"] = "tma"
+        os.environ["CONV_B200_DW_RING"] = ring
+        for mode in MODES:
+            ys = []
+            for st in ("0", "1"):
+                os.environ["CONV_B200_DW_STAGGER"] = st
+                ys.append(_gpu(cb, x, w, b, S, case.pad, 1, mode))
+                assert cb.conv_last_kernel() == "depthwise_tma_kernel"
+            assert np.array_equal(_bits(ys[0]), _bits(ys[1]))
+            _compare(ys[1], x, w, b, 1, S, case.pad, 1, mode)
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
